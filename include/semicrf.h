@@ -1,0 +1,181 @@
+/*
+ * semicrf.h -- C ABI of the B200 (sm_100a) streaming semi-CRF library.
+ *
+ * The library computes, on one GPU, the hot path of the semi-Markov CRF
+ * described by "Streaming Structured Inference with Flash-SemiCRF"
+ * (abstract; explainer sections 1-2):
+ *
+ *   1. prefix sums of zero-centred emissions        semicrf_prefix_center
+ *   2. a streaming log-semiring forward pass with a
+ *      K-slot ring, normalised and checkpointed      semicrf_forward
+ *   3. a checkpointed backward pass giving exact
+ *      marginals and gradients                       semicrf_backward
+ *   4. max-semiring (Viterbi) decoding               semicrf_viterbi
+ *
+ * Model.  A sequence b has length L_b (0 <= L_b <= T).  A segmentation
+ * splits its positions 0..L_b-1 into consecutive segments [s, t) of duration
+ * k = t - s in 1..K, each with a label c in 0..C-1.  Its score is the sum over
+ * segments of  content(s,t,c) + dur[k-1, c]  plus  trans[c', c]  between
+ * consecutive segments (labels c' then c); the first segment has no
+ * transition term and there is no end term.  content(s,t,c) is the sum of the
+ * centred emissions e~[u, c] = em[b, u, c] - nu[b, c] over u = s..t-1, with
+ * nu[b, c] the mean of em[b, :L_b, c] (explainer section 2, "Emission
+ * Baseline Centering"; centering can be switched off).  log Z_b is the
+ * log-sum-exp of the scores of all segmentations.
+ *
+ * Conventions shared by every entry point.
+ *  - All array arguments are DEVICE pointers to contiguous row-major memory
+ *    owned by the caller.  The library never allocates, frees or keeps a
+ *    pointer after the call returns.
+ *  - em       [B, T, C] float32 raw emissions; rows u >= L_b are never read.
+ *  - lengths  [B] int32, device memory.  A length outside [0, T] is reported
+ *             through the workspace status word (SEMICRF_ERR_BAD_LENGTH); that
+ *             sequence's outputs are zeroed and its log Z is NaN.
+ *  - trans    [C, C] float32, trans[c', c] scores the transition c' -> c.
+ *  - dur      [K, C] float32, dur[k-1, c] scores a label-c segment of length k.
+ *  - stream   a cudaStream_t (NULL = legacy default stream).  All work is
+ *             asynchronous on that stream; a return value of SEMICRF_OK means
+ *             the launches were enqueued.
+ *  - Every call returns a status code.  Argument errors are detected on the
+ *    host before anything is launched.  Device-side conditions (bad lengths,
+ *    a bounded wait that gave up) are recorded in the workspace status word,
+ *    read with semicrf_get_status.
+ *  - Limits of this build: 1 <= C <= 128, T <= 2^26, B <= 2^20, and
+ *    K <= 512 (C <= 16), K <= 256 (C <= 32), K <= 128 (C <= 64),
+ *    K <= 64 (C <= 128).  Larger values return SEMICRF_ERR_UNSUPPORTED.
+ *  - Numbers are computed in float32 in base-2 log units with exactly
+ *    representable integer frames and float64 normalisers; results are
+ *    deterministic (no floating-point atomics).
+ */
+#ifndef SEMICRF_H
+#define SEMICRF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SEMICRF_API __attribute__((visibility("default")))
+#else
+#define SEMICRF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *semicrf_stream_t;
+
+enum semicrf_status {
+    SEMICRF_OK = 0,
+    SEMICRF_ERR_INVALID_ARG = 1,         /* null pointer, negative size, unknown flag */
+    SEMICRF_ERR_UNSUPPORTED = 2,         /* C, K, K*C, T or B above the limits above */
+    SEMICRF_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < semicrf_workspace_bytes(...) */
+    SEMICRF_ERR_CUDA = 4,                /* a CUDA launch or copy failed */
+    SEMICRF_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device wait gave up */
+    SEMICRF_ERR_BAD_LENGTH = 6           /* some lengths[b] outside [0, T] */
+};
+
+/* flags */
+#define SEMICRF_FLAG_NO_CENTER 0x1u    /* use raw emissions (nu = 0) */
+#define SEMICRF_FLAG_FORWARD_ONLY 0x2u /* forward skips the backward ring (inference);
+                                          a backward given the same flag runs it itself */
+
+/*
+ * Bytes of device workspace needed by forward/backward/viterbi for these
+ * sizes and flags.  The workspace holds the status word, the prefix-sum array
+ * (stored as an exact integer part plus a float32 fraction, 8 bytes per
+ * entry), the ring checkpoints taken every Delta = ceil(sqrt(T*K)) positions
+ * (explainer section 2, "Streaming Forward-Backward with Ring Buffers",
+ * checkpointing), the per-segment recompute buffers and the partial sums of
+ * the backward pass.  Host-only; launches nothing.
+ */
+SEMICRF_API int semicrf_workspace_bytes(int B, int T, int C, int K, unsigned flags, size_t *bytes);
+
+/*
+ * Step 1 (explainer section 2, "On-the-Fly Edge Computation via Prefix Sums"
+ * and "Emission Baseline Centering"): nu[b, c] = mean of em[b, :L_b, c]
+ * (0 with SEMICRF_FLAG_NO_CENTER) and the float64 prefix sums
+ * S[b, t, c] = sum_{u < t} (em[b, u, c] - nu[b, c]) for t = 0..L_b; rows
+ * t > L_b are zero.  S is [B, T+1, C] float64, nu is [B, C] float32.
+ * ws must hold semicrf_workspace_bytes(B, T, C, 1, flags) bytes (per-chunk
+ * partial sums and the status word live there).
+ */
+SEMICRF_API int semicrf_prefix_center(const float *em, const int32_t *lengths, int B, int T, int C,
+                          unsigned flags, void *ws, size_t ws_bytes, double *S, float *nu,
+                          semicrf_stream_t stream);
+
+/*
+ * Steps 1-2 (explainer section 2, "Streaming Forward-Backward with Ring
+ * Buffers"; abstract): writes logZ[b] (float64) for every sequence.  The
+ * forward recursion
+ *   alpha[t, c] = LSE_{k <= min(K,t)} LSE_{c'} alpha[t-k, c'] + trans[c', c]
+ *                 + S[t, c] - S[t-k, c] + dur[k-1, c]
+ * (no c' term when t-k = 0) keeps a K-slot ring per sequence in shared memory,
+ * never materialises an edge, and saves the ring plus its normaliser every
+ * Delta positions into the workspace.  Unless SEMICRF_FLAG_FORWARD_ONLY is
+ * given, the backward ring runs in the same launch on other SMs and is
+ * checkpointed the same way, so a following semicrf_backward needs only the
+ * workspace.  The workspace must be 256-byte aligned (cudaMalloc is).
+ */
+SEMICRF_API int semicrf_forward(const float *em, const int32_t *lengths, const float *trans, const float *dur,
+                    int B, int T, int C, int K, unsigned flags, void *ws, size_t ws_bytes,
+                    double *logZ, semicrf_stream_t stream);
+
+/*
+ * Step 3 (explainer section 2, checkpointing; section 4 "Correctness"):
+ * consumes the workspace of the immediately preceding semicrf_forward with
+ * the same arguments (the workspace must not be reused in between).  Each
+ * checkpoint segment restores its ring checkpoints, recomputes alpha and beta
+ * locally and accumulates the exact posteriors.  Outputs:
+ *   grad_em    [B, T, C]  g_b * d logZ_b / d em[b, u, c]  (through centering)
+ *   grad_trans [C, C]     sum_b g_b * E[#transitions c' -> c]
+ *   grad_dur   [K, C]     sum_b g_b * E[#label-c segments of length k]
+ *   pos_marg   [B, T, C]  P(position u lies in a label-c segment)   (nullable)
+ *   start_marg [B, T+1, C] P(a label-c segment starts at boundary s) (nullable)
+ *   end_marg   [B, T+1, C] P(a label-c segment ends at boundary t)   (nullable)
+ * g_b = grad_logZ[b] (device float64 [B]; NULL means all ones).  Marginals
+ * are not scaled by g_b.  Entries past L_b are zero.
+ */
+SEMICRF_API int semicrf_backward(const int32_t *lengths, const float *trans, const float *dur,
+                     int B, int T, int C, int K, unsigned flags, void *ws, size_t ws_bytes,
+                     const double *grad_logZ, float *grad_em, float *grad_trans, float *grad_dur,
+                     float *pos_marg, float *start_marg, float *end_marg,
+                     semicrf_stream_t stream);
+
+/*
+ * Step 4: max-semiring decoding with the same recursion (max in place of
+ * log-sum-exp).  Ties go to the smallest duration k, then the smallest
+ * previous label c', and at the end to the smallest final label.  Writes
+ * score[b] (float64), labels[b, u] (int32, -1 for u >= L_b) and
+ * seg_start[b, u] (1 where a segment starts, else 0).  Uses the workspace for
+ * the prefix sums and the backpointers.
+ */
+SEMICRF_API int semicrf_viterbi(const float *em, const int32_t *lengths, const float *trans, const float *dur,
+                    int B, int T, int C, int K, unsigned flags, void *ws, size_t ws_bytes,
+                    double *score, int32_t *labels, uint8_t *seg_start, semicrf_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word of workspace
+ * `ws` into *status (a semicrf_status value; the first device error wins).
+ * Forward and viterbi reset the word when they start.
+ */
+SEMICRF_API int semicrf_get_status(const void *ws, semicrf_stream_t stream, int *status);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SEMICRF_API const char *semicrf_strerror(int code);
+
+/*
+ * Diagnostic: runs the library's bounded shared-memory-barrier wait on a
+ * barrier nothing will ever complete, with a limit of `spins` polls, and
+ * records the outcome in the workspace status word (SEMICRF_ERR_DEVICE_TIMEOUT
+ * when the limit is hit).  Lets a test check that a wait that never
+ * completes ends with an error status instead of hanging.  No counterpart on
+ * the pages.
+ */
+SEMICRF_API int semicrf_selftest_bounded_wait(void *ws, size_t ws_bytes, int spins, semicrf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SEMICRF_H */

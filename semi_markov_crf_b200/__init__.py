@@ -13,6 +13,7 @@ from __future__ import annotations
 _BINDING_NAMES = {
     "workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
     "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
+    "FLAG_FORWARD_ONLY", "selftest_bounded_wait",
 }
 
 

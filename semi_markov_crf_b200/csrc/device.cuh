@@ -1,0 +1,118 @@
+// device.cuh -- sm_100a device helpers shared by the semi-CRF kernels.
+//
+// Everything here is plain CUDA C++ or inline PTX written for this library:
+// base-2 transcendental instructions, group reductions over aligned lane
+// groups, shared-memory float max through an order-preserving integer map,
+// and TMA bulk copies (cp.async.bulk, no multicast) completed on an mbarrier
+// whose wait is bounded.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace semicrf {
+
+constexpr unsigned FULL_MASK = 0xffffffffu;
+constexpr double LOG2E_D = 1.4426950408889634073599246810019;
+constexpr double LN2_D = 0.69314718055994530941723212145818;
+constexpr float NEG_INF = -__builtin_huge_valf();
+
+// Status codes written to the workspace status word (mirror semicrf.h).
+constexpr int ST_DEVICE_TIMEOUT = 5;
+constexpr int ST_BAD_LENGTH = 6;
+
+// Polls of an mbarrier before a wait gives up (each try_wait may itself
+// suspend for a bounded, hardware-defined time).
+constexpr int WAIT_SPIN_LIMIT = 1 << 22;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// All-reduce over aligned groups of G lanes (G a power of two <= 32).  Every
+// lane of the warp must execute the call.
+__device__ __forceinline__ float group_max(float v, int G) {
+  for (int o = G >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL_MASK, v, o));
+  return v;
+}
+__device__ __forceinline__ float group_sum(float v, int G) {
+  for (int o = G >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+  return v;
+}
+
+// Order-preserving float <-> int map, so shared-memory atomicMax on int gives
+// a float max.
+__device__ __forceinline__ int f2ord(float f) {
+  int i = __float_as_int(f);
+  return i >= 0 ? i : (i ^ 0x7fffffff);
+}
+__device__ __forceinline__ float ord2f(int i) {
+  return __int_as_float(i >= 0 ? i : (i ^ 0x7fffffff));
+}
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One-dimensional TMA bulk copy global -> shared, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bounded wait for phase `parity` of `bar`.  Returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int spins) {
+  const uint32_t a = smem_addr(bar);
+  for (int i = 0; i < spins; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+}  // namespace semicrf

@@ -1,0 +1,104 @@
+// finalize.cu -- step 3 epilogue: position marginals, the emission gradient
+// through centering, and the fixed-order reduction of per-segment partials.
+//
+// The checkpoint segments leave, for every position u of segment j, the
+// suffix sum v[u, c] = sum_{u < s < t1_j} (start_marg[s,c] - end_marg[s,c]) in
+// the grad_em buffer, plus per segment the total T_j[c] of (start - end) and
+// V_j[c] = sum_u v[u, c].  Then
+//   pos_marg[u, c] = sum_{s <= u} (start_marg[s,c] - end_marg[s,c])
+//                  = sum_{j' <= j} T_j'[c] - v[u, c]
+// (a position lies in a label-c segment iff one started at or before it and
+// none of those ended at or before it), and with centering the emission
+// gradient is g_b * (pos_marg[u,c] - mean_v pos_marg[v,c]) (the Jacobian of
+// subtracting the per-label mean; "Emission Baseline Centering", explainer
+// section 2).
+#include "kernels.cuh"
+
+namespace semicrf {
+
+constexpr int FIN_ROWS = 32;
+
+__global__ void __launch_bounds__(256)
+    finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                              const double* __restrict__ grad_logZ, unsigned center,
+                              float* __restrict__ grad_em, float* __restrict__ pos_marg,
+                              float* __restrict__ start_marg, float* __restrict__ end_marg) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* mean = reinterpret_cast<double*>(smem_raw);  // [C]
+  double* pinc = mean + d.C;                            // [nj][C]
+  const int C = d.C, T = d.T;
+  const int b = blockIdx.y;
+  const int u0 = blockIdx.x * FIN_ROWS;
+  const int u1 = min(u0 + FIN_ROWS, T);
+  int L = lengths[b];
+  const bool bad = (L < 0 || L > T);
+  if (bad) L = 0;
+  const double gb = grad_logZ ? grad_logZ[b] : 1.0;
+  const int delta = d.delta;
+  const int j_lo = u0 / delta;
+  const int j_hi = (max(u0, min(u1, L) - 1)) / delta;
+  if (threadIdx.x < C && L > 0) {
+    const int c = threadIdx.x;
+    const int nseg = (L + delta - 1) / delta;
+    double run = 0.0, msum = 0.0;
+    for (int j = 0; j < nseg; ++j) {
+      const size_t o = ((size_t)b * d.nck + j) * C + c;
+      run += ws.segT[o];
+      const int len = min((j + 1) * delta, L) - j * delta;
+      msum += (double)len * run - ws.segV[o];
+      if (j >= j_lo && j <= j_hi) pinc[(j - j_lo) * C + c] = run;
+    }
+    mean[c] = center ? msum / (double)L : 0.0;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < (u1 - u0) * C; idx += blockDim.x) {
+    const int u = u0 + idx / C, c = idx % C;
+    const size_t o = ((size_t)b * T + u) * C + c;
+    if (u < L) {
+      const int j = u / delta;
+      const double mu = pinc[(j - j_lo) * C + c] - (double)grad_em[o];
+      grad_em[o] = (float)(gb * (mu - mean[c]));
+      if (pos_marg) pos_marg[o] = (float)mu;
+    } else {
+      grad_em[o] = 0.f;
+      if (pos_marg) pos_marg[o] = 0.f;
+    }
+  }
+  // boundary rows t in [u0, u1) (and t = T for the last block) past the length
+  const int tb1 = (u1 == T) ? T + 1 : u1;
+  for (int idx = threadIdx.x; idx < (tb1 - u0) * C; idx += blockDim.x) {
+    const int t = u0 + idx / C, c = idx % C;
+    if (t > L || L == 0) {
+      const size_t o = ((size_t)b * (T + 1) + t) * C + c;
+      if (start_marg) start_marg[o] = 0.f;
+      if (end_marg) end_marg[o] = 0.f;
+    }
+  }
+}
+
+// grad_trans (entries 0..C*C-1) and grad_dur (entries C*C..C*C+K*C-1):
+// float64 sums of the per-segment partials in (sequence, segment) order.
+__global__ void __launch_bounds__(256)
+    reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                           float* __restrict__ grad_trans, float* __restrict__ grad_dur) {
+  const int C = d.C, K = d.K;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nt = C * C;
+  if (e >= nt + K * C) return;
+  double acc = 0.0;
+  for (int b = 0; b < d.B; ++b) {
+    const int L = lengths[b];
+    if (L <= 0 || L > d.T) continue;
+    const int nseg = (L + d.delta - 1) / d.delta;
+    for (int j = 0; j < nseg; ++j) {
+      const size_t seg = (size_t)b * d.nck + j;
+      acc += (e < nt) ? ws.pgt[seg * nt + e] : ws.pgd[seg * K * C + (e - nt)];
+    }
+  }
+  if (e < nt)
+    grad_trans[e] = (float)acc;
+  else
+    grad_dur[e - nt] = (float)acc;
+}
+
+}  // namespace semicrf

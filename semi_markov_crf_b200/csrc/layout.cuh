@@ -1,0 +1,55 @@
+// layout.cuh -- sizes, launch geometry and workspace layout shared by the
+// host layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector_types.h>
+
+namespace semicrf {
+
+constexpr int C_MAX = 128;
+constexpr int K_MAX = 512;
+constexpr int KC_MAX = 16384;
+constexpr int KB_MAX = 16;   // duration terms per lane in the k fan-in
+constexpr int CA_MAX = 32;   // label terms per lane in the label fan-in
+constexpr int NT_MAX = 512;  // threads per CTA
+constexpr int TS = 32;       // prefix-sum rows per TMA tile
+constexpr int FLUSH_EVERY = 64;  // positions between fp32 -> fp64 partial flushes
+
+// Problem sizes and the lane mapping chosen for them.
+struct Dims {
+  int B, T, C, K;
+  int delta;     // checkpoint spacing ceil(sqrt(T*K))
+  int nck;       // checkpoint segments per sequence, ceil(T / delta)
+  int Tstride;   // rows per sequence in the prefix-sum arrays (>= T+1, multiple of TS)
+  int GB, KB;    // k fan-in: lanes per label, duration terms per lane
+  int GA, CA;    // label fan-in: lanes per output label, label terms per lane
+  int NT;        // threads per CTA of the recursion kernels
+  int prefR;     // rows per prefix-sum chunk
+  int nchunk;    // prefix-sum chunks per sequence
+  int store_w;   // floats per position in the segment recompute store (2C + 2)
+  int store_smem;  // 1: the recompute store lives in shared memory
+};
+
+// Device pointers into the caller's workspace.
+struct WsPtrs {
+  int* status;
+  int32_t* sint;   // [B][Tstride][C] integer part of the base-2 prefix sums
+  float* sfrac;    // [B][Tstride][C] fractional part
+  double* chunk;   // [B][nchunk][C] per-chunk emission sums
+  double* logz2;   // [B] log2 Z from the forward ring
+  double* logz2b;  // [B] log2 Z from the backward ring
+  float2* ack;     // [B][nck][K][C] forward ring checkpoints
+  double* acf;     // [B][nck] their frame bases
+  float2* bck;     // [B][nck][K][C] backward ring checkpoints
+  double* bcf;     // [B][nck]
+  float* store;    // [B][nck][delta][store_w] recompute store (when not in smem)
+  double* pgt;     // [B][nck][C][C] transition-count partials
+  double* pgd;     // [B][nck][K][C] duration-count partials
+  double* segT;    // [B][nck][C] per-segment sum of (start - end) marginals
+  double* segV;    // [B][nck][C] per-segment sum of the within-segment suffix sums
+  int32_t* bp;     // [B][T+1][C] Viterbi backpointers
+};
+
+}  // namespace semicrf

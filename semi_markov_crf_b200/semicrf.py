@@ -1,0 +1,217 @@
+"""Thin Python binding of the C ABI in ``include/semicrf.h``.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libsemicrf_b200.so``.  PyTorch supplies device memory (tensors,
+the workspace) and the current CUDA stream.  There is no CPU fallback: if the
+library is missing or no CUDA device is present, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
+           "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
+           "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "lib"]
+
+FLAG_NO_CENTER = 0x1
+FLAG_FORWARD_ONLY = 0x2
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsemicrf_b200.so")
+if not os.path.exists(library_path):
+    raise ImportError(f"{library_path} is missing: build it with `python -m semi_markov_crf_b200.build`")
+
+lib = ctypes.CDLL(library_path)
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_u = ctypes.c_uint
+_sz = ctypes.c_size_t
+
+lib.semicrf_workspace_bytes.argtypes = [_i, _i, _i, _i, _u, ctypes.POINTER(_sz)]
+lib.semicrf_prefix_center.argtypes = [_vp, _vp, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp]
+lib.semicrf_forward.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.semicrf_backward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _vp, _vp]
+lib.semicrf_viterbi.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp,
+                                _vp]
+lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
+lib.semicrf_strerror.argtypes = [_i]
+lib.semicrf_strerror.restype = ctypes.c_char_p
+lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
+for _f in ("semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+           "semicrf_backward", "semicrf_viterbi", "semicrf_get_status",
+           "semicrf_selftest_bounded_wait"):
+    getattr(lib, _f).restype = _i
+
+
+class SemiCRFError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (status {code})")
+
+
+def strerror(code: int) -> str:
+    return lib.semicrf_strerror(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        if rc == 4:  # surface the CUDA runtime's own message
+            try:
+                torch.cuda.synchronize()
+            except RuntimeError as e:
+                raise SemiCRFError(rc, where) from e
+        raise SemiCRFError(rc, where)
+
+
+def workspace_bytes(B: int, T: int, C: int, K: int, flags: int = 0) -> int:
+    n = _sz(0)
+    _check(lib.semicrf_workspace_bytes(B, T, C, K, flags, ctypes.byref(n)), "semicrf_workspace_bytes")
+    return int(n.value)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, name, device):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if t.device != device:
+        raise TypeError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+class Workspace:
+    """Device workspace of the right size for (B, T, C, K, flags), allocated by torch."""
+
+    def __init__(self, B: int, T: int, C: int, K: int, flags: int = 0, device=None):
+        self.dims = (B, T, C, K)
+        self.flags = flags
+        self.nbytes = workspace_bytes(B, T, C, K, flags)
+        self.buf = torch.empty(max(self.nbytes, 256), dtype=torch.uint8, device=device or "cuda")
+
+    def matches(self, B, T, C, K, flags) -> bool:
+        return self.dims == (B, T, C, K) and self.flags == flags
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+
+def _flags(center: bool, forward_only: bool = False) -> int:
+    return (0 if center else FLAG_NO_CENTER) | (FLAG_FORWARD_ONLY if forward_only else 0)
+
+
+def prefix_center(em, lengths, center: bool = True, ws: Workspace | None = None):
+    """Step 1: float64 prefix sums S [B, T+1, C] and nu [B, C] (float32)."""
+    dev = em.device
+    _need(em, torch.float32, "em", dev)
+    _need(lengths, torch.int32, "lengths", dev)
+    B, T, C = em.shape
+    flags = _flags(center)
+    if ws is None or not ws.matches(B, T, C, 1, flags):
+        ws = Workspace(B, T, C, 1, flags, dev)
+    S = torch.empty((B, T + 1, C), dtype=torch.float64, device=dev)
+    nu = torch.empty((B, C), dtype=torch.float32, device=dev)
+    _check(lib.semicrf_prefix_center(_ptr(em), _ptr(lengths), B, T, C, flags, ws.ptr, ws.nbytes,
+                                     _ptr(S), _ptr(nu), _stream(dev)), "semicrf_prefix_center")
+    return S, nu
+
+
+def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = False,
+            ws: Workspace | None = None, logZ=None):
+    """Steps 1-2: log Z [B] (float64).  Returns (logZ, workspace); pass the
+    workspace to :func:`backward`."""
+    dev = em.device
+    _need(em, torch.float32, "em", dev)
+    _need(lengths, torch.int32, "lengths", dev)
+    _need(trans, torch.float32, "trans", dev)
+    _need(dur, torch.float32, "dur", dev)
+    B, T, C = em.shape
+    K = dur.shape[0]
+    flags = _flags(center, forward_only)
+    if ws is None or not ws.matches(B, T, C, K, flags):
+        ws = Workspace(B, T, C, K, flags, dev)
+    if logZ is None:
+        logZ = torch.empty(B, dtype=torch.float64, device=dev)
+    _check(lib.semicrf_forward(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, flags,
+                               ws.ptr, ws.nbytes, _ptr(logZ), _stream(dev)), "semicrf_forward")
+    return logZ, ws
+
+
+def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool = False,
+             out: dict | None = None):
+    """Step 3 on the workspace of the preceding :func:`forward`.
+
+    Returns a dict with grad_em [B,T,C], grad_trans [C,C], grad_dur [K,C]
+    (float32) and, when ``marginals``, pos_marg [B,T,C], start_marg and
+    end_marg [B,T+1,C].  ``out`` may supply preallocated tensors."""
+    B, T, C, K = ws.dims
+    dev = ws.buf.device
+    _need(lengths, torch.int32, "lengths", dev)
+    _need(trans, torch.float32, "trans", dev)
+    _need(dur, torch.float32, "dur", dev)
+    if grad_logZ is not None:
+        _need(grad_logZ, torch.float64, "grad_logZ", dev)
+    o = {} if out is None else out
+    if "grad_em" not in o:
+        o["grad_em"] = torch.empty((B, T, C), dtype=torch.float32, device=dev)
+        o["grad_trans"] = torch.empty((C, C), dtype=torch.float32, device=dev)
+        o["grad_dur"] = torch.empty((K, C), dtype=torch.float32, device=dev)
+    if marginals and "pos_marg" not in o:
+        o["pos_marg"] = torch.empty((B, T, C), dtype=torch.float32, device=dev)
+        o["start_marg"] = torch.empty((B, T + 1, C), dtype=torch.float32, device=dev)
+        o["end_marg"] = torch.empty((B, T + 1, C), dtype=torch.float32, device=dev)
+    _check(lib.semicrf_backward(_ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, ws.flags, ws.ptr,
+                                ws.nbytes, _ptr(grad_logZ), _ptr(o["grad_em"]), _ptr(o["grad_trans"]),
+                                _ptr(o["grad_dur"]), _ptr(o.get("pos_marg") if marginals else None),
+                                _ptr(o.get("start_marg") if marginals else None),
+                                _ptr(o.get("end_marg") if marginals else None), _stream(dev)),
+           "semicrf_backward")
+    return o
+
+
+def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None = None):
+    """Step 4: (score [B] float64, labels [B,T] int32, seg_start [B,T] uint8)."""
+    dev = em.device
+    _need(em, torch.float32, "em", dev)
+    _need(lengths, torch.int32, "lengths", dev)
+    _need(trans, torch.float32, "trans", dev)
+    _need(dur, torch.float32, "dur", dev)
+    B, T, C = em.shape
+    K = dur.shape[0]
+    flags = _flags(center)
+    if ws is None or not ws.matches(B, T, C, K, flags):
+        ws = Workspace(B, T, C, K, flags, dev)
+    score = torch.empty(B, dtype=torch.float64, device=dev)
+    labels = torch.empty((B, T), dtype=torch.int32, device=dev)
+    seg = torch.empty((B, T), dtype=torch.uint8, device=dev)
+    _check(lib.semicrf_viterbi(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, flags,
+                               ws.ptr, ws.nbytes, _ptr(score), _ptr(labels), _ptr(seg), _stream(dev)),
+           "semicrf_viterbi")
+    return score, labels, seg
+
+
+def get_status(ws: Workspace) -> int:
+    """Synchronises the current stream and returns the workspace status word."""
+    st = _i(0)
+    _check(lib.semicrf_get_status(ws.ptr, _stream(ws.buf.device), ctypes.byref(st)),
+           "semicrf_get_status")
+    return int(st.value)
+
+
+def selftest_bounded_wait(ws: Workspace, spins: int) -> int:
+    """Runs the never-completing bounded wait with `spins` polls; returns the
+    resulting status word (SEMICRF_ERR_DEVICE_TIMEOUT = 5 expected)."""
+    _check(lib.semicrf_selftest_bounded_wait(ws.ptr, ws.nbytes, int(spins), _stream(ws.buf.device)),
+           "semicrf_selftest_bounded_wait")
+    return get_status(ws)

@@ -1,0 +1,88 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every entry point
+that include/semicrf.h declares, and rejects bad arguments on the host before
+launching anything (no GPU needed for any of this)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "semicrf.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from semi_markov_crf_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*SEMICRF_API\s+(?:const\s+)?\w+\s*\*?\s*(semicrf_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_four_steps():
+    names = declared_functions()
+    for n in ("semicrf_prefix_center", "semicrf_forward", "semicrf_backward", "semicrf_viterbi",
+              "semicrf_workspace_bytes", "semicrf_get_status", "semicrf_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def _ws_bytes(lib, B, T, C, K, flags=0):
+    n = ctypes.c_size_t(0)
+    rc = lib.semicrf_workspace_bytes(B, T, C, K, ctypes.c_uint(flags), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_bytes_and_limits(lib):
+    rc, n = _ws_bytes(lib, 32, 800, 39, 30)
+    assert rc == 0 and n > 32 * 801 * 39 * 8  # at least the split prefix sums
+    rc2, n2 = _ws_bytes(lib, 1, 1_000_000, 6, 200)
+    assert rc2 == 0
+    # checkpoint memory grows like sqrt(T): 4x T -> about 2x checkpoint bytes
+    _, a = _ws_bytes(lib, 1, 100_000, 6, 200)
+    assert n2 < 12 * a
+    assert _ws_bytes(lib, 1, 10, 129, 4)[0] == 2          # C above the limit
+    assert _ws_bytes(lib, 1, 10, 128, 65)[0] == 2         # K above the limit for C=128
+    assert _ws_bytes(lib, 1, 10, 16, 512)[0] == 0
+    assert _ws_bytes(lib, 1, 10, 16, 513)[0] == 2
+    assert _ws_bytes(lib, -1, 10, 4, 4)[0] == 1
+    assert _ws_bytes(lib, 1, 10, 0, 4)[0] == 1
+    assert _ws_bytes(lib, 1, 10, 4, 4, flags=0x80)[0] == 1
+    assert lib.semicrf_workspace_bytes(1, 10, 4, 4, ctypes.c_uint(0), None) == 1
+
+
+def test_host_side_argument_errors_launch_nothing(lib):
+    vp = ctypes.c_void_p
+    fake = vp(256 * 1024)  # never dereferenced: every call below fails validation first
+    # null pointers
+    assert lib.semicrf_forward(None, fake, fake, fake, 1, 8, 2, 2, ctypes.c_uint(0), fake,
+                               ctypes.c_size_t(1 << 30), fake, None) == 1
+    # workspace too small
+    assert lib.semicrf_forward(fake, fake, fake, fake, 1, 8, 2, 2, ctypes.c_uint(0), fake,
+                               ctypes.c_size_t(16), fake, None) == 3
+    # unsupported size
+    assert lib.semicrf_viterbi(fake, fake, fake, fake, 1, 8, 200, 2, ctypes.c_uint(0), fake,
+                               ctypes.c_size_t(1 << 30), fake, fake, fake, None) == 2
+    # unknown flag
+    assert lib.semicrf_backward(fake, fake, fake, 1, 8, 2, 2, ctypes.c_uint(0x40), fake,
+                                ctypes.c_size_t(1 << 30), None, fake, fake, fake, None, None, None,
+                                None) == 1
+    # misaligned workspace
+    assert lib.semicrf_forward(fake, fake, fake, fake, 1, 8, 2, 2, ctypes.c_uint(0), vp(256 * 1024 + 8),
+                               ctypes.c_size_t(1 << 30), fake, None) == 1
+
+
+def test_strerror_names_every_status(lib):
+    lib.semicrf_strerror.restype = ctypes.c_char_p
+    seen = {lib.semicrf_strerror(i).decode() for i in range(7)}
+    assert len(seen) == 7 and "unknown status" not in seen
+    assert lib.semicrf_strerror(99).decode() == "unknown status"

@@ -175,6 +175,18 @@ SEMICRF_API const char *semicrf_strerror(int code);
  */
 SEMICRF_API int semicrf_selftest_bounded_wait(void *ws, size_t ws_bytes, int spins, semicrf_stream_t stream);
 
+/*
+ * Diagnostic timing (no counterpart on the pages).  semicrf_profile_enable(1)
+ * clears the record and starts bracketing every kernel this library launches
+ * with two CUDA events on the launch stream; semicrf_profile_enable(0) stops.
+ * semicrf_profile_read(name, &ms, &n) waits for the recorded events of kernel
+ * `name` (e.g. "chain_kernel", "segment_kernel", "viterbi_kernel") and returns
+ * their summed device time in milliseconds and the number of launches.
+ * Host-side bookkeeping only; not thread-safe across concurrent enables.
+ */
+SEMICRF_API int semicrf_profile_enable(int on);
+SEMICRF_API int semicrf_profile_read(const char *kernel, double *total_ms, int *launches);
+
 #ifdef __cplusplus
 }
 #endif

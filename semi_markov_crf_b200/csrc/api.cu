@@ -1,8 +1,11 @@
 // api.cu -- the C ABI declared in include/semicrf.h: argument validation,
 // launch geometry, workspace layout and kernel launches.  Host code only.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "semicrf.h"
 #include "kernels.cuh"
@@ -16,6 +19,12 @@ constexpr int FIN_ROWS_HOST = 32;  // must match FIN_ROWS in finalize.cu
 int pow2floor(int x) {
   int p = 1;
   while (p * 2 <= x) p *= 2;
+  return p;
+}
+
+int pow2ceil(int x) {
+  int p = 1;
+  while (p < x) p *= 2;
   return p;
 }
 
@@ -57,14 +66,33 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
-  d.GB = std::min(32, pow2floor(NT_MAX / C));
-  d.KB = (K + d.GB - 1) / d.GB;
-  d.GA = std::min(std::min(32, pow2floor(NT_MAX / C)), pow2floor(C));
-  d.CA = (C + d.GA - 1) / d.GA;
-  if (d.KB > KB_MAX || d.CA > CA_MAX) return SEMICRF_ERR_UNSUPPORTED;
-  int nt = std::max(C * d.GB, C * d.GA);
-  nt = ((nt + 31) / 32) * 32;
-  d.NT = std::max(nt, 32);
+  // lanes per label are a power of two <= 32 with at most NT_MAX threads in all
+  const int gmax = std::min(32, pow2floor(NT_MAX / C));
+  // fewest durations per lane that fit: KBT in {2, 4, 8, 16}
+  d.KBT = 0;
+  for (int kb : {2, 4, 8, 16}) {
+    if ((K + kb - 1) / kb <= gmax) {
+      d.KBT = kb;
+      break;
+    }
+  }
+  if (d.KBT == 0) return SEMICRF_ERR_UNSUPPORTED;
+  // lanes per group: enough for the durations, and for the labels (<= 32 per lane)
+  d.GB = std::max(pow2ceil((K + d.KBT - 1) / d.KBT), pow2ceil((C + 31) / 32));
+  // the label fan-in uses the same groups: CAT >= ceil(C / GB) in {1, 2, 4, 8, 32}
+  d.CAT = 0;
+  for (int ca : {1, 2, 4, 8, 32}) {
+    if (ca * d.GB >= C) {
+      d.CAT = ca;
+      break;
+    }
+  }
+  if (d.CAT == 0 || !shape_supported(d.KBT, d.CAT)) return SEMICRF_ERR_UNSUPPORTED;
+  d.GA = d.GB;
+  d.RL = K + d.KBT;
+  d.PC = ((std::max(C, d.GB * d.CAT) + 3) / 4) * 4;
+  d.NT = std::max(32, ((C * d.GB + 31) / 32) * 32);
+  if (d.NT > NT_MAX) return SEMICRF_ERR_UNSUPPORTED;
   d.prefR = std::max(16, pow2floor(8192 / C));
   d.nchunk = T > 0 ? (T + d.prefR - 1) / d.prefR : 1;
   d.store_w = 2 * C + 2;
@@ -151,17 +179,57 @@ int launched() {
   return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Optional per-kernel device timing: when enabled, every kernel launch is
+// bracketed by two CUDA events recorded on its own stream; reading the
+// profile synchronises on them and sums the elapsed times per kernel name.
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::mutex prof_mu;
+bool prof_on = false;
+std::vector<ProfRec> prof_recs;
+
+struct ProfScope {
+  cudaStream_t st;
+  ProfRec rec{nullptr, nullptr, nullptr};
+  ProfScope(const char* name, cudaStream_t s) : st(s) {
+    std::lock_guard<std::mutex> g(prof_mu);
+    if (!prof_on) return;
+    rec.name = name;
+    if (cudaEventCreate(&rec.a) != cudaSuccess || cudaEventCreate(&rec.b) != cudaSuccess) {
+      cudaGetLastError();
+      rec.name = nullptr;
+      return;
+    }
+    cudaEventRecord(rec.a, st);
+  }
+  ~ProfScope() {
+    if (!rec.name) return;
+    cudaEventRecord(rec.b, st);
+    std::lock_guard<std::mutex> g(prof_mu);
+    prof_recs.push_back(rec);
+  }
+};
+
 int run_prefix(const float* em, const int32_t* lengths, const Dims& d, const WsPtrs& p,
                unsigned flags, int mode, double* S64, float* nu, cudaStream_t st) {
   if (d.B == 0 || d.T == 0) return SEMICRF_OK;
   const dim3 grid(d.nchunk, d.B);
-  prefix_reduce_kernel<<<grid, 256, 0, st>>>(em, lengths, d, p);
+  {
+    ProfScope ps("prefix_reduce_kernel", st);
+    prefix_reduce_kernel<<<grid, 256, 0, st>>>(em, lengths, d, p);
+  }
   const size_t sm = prefix_scan_smem_bytes(d);
   int rc = set_smem((const void*)prefix_scan_kernel, sm);
   if (rc) return rc;
-  prefix_scan_kernel<<<grid, 256, sm, st>>>(em, lengths, d, p,
-                                            (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, mode, S64,
-                                            nu);
+  {
+    ProfScope ps("prefix_scan_kernel", st);
+    prefix_scan_kernel<<<grid, 256, sm, st>>>(em, lengths, d, p,
+                                              (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, mode,
+                                              S64, nu);
+  }
   return launched();
 }
 
@@ -212,12 +280,13 @@ extern "C" int semicrf_forward(const float* em, const int32_t* lengths, const fl
   if (B == 0) return SEMICRF_OK;
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
   if (rc) return rc;
-  const size_t sm = recursion_smem_bytes(d, false);
-  rc = set_smem((const void*)chain_kernel, sm);
-  if (rc) return rc;
-  const int nb = (flags & SEMICRF_FLAG_FORWARD_ONLY) ? B : 2 * B;
-  chain_kernel<<<nb, d.NT, sm, st>>>(d, p, lengths, trans, dur, logZ, B);
-  return launched();
+  const int nbeta = (flags & SEMICRF_FLAG_FORWARD_ONLY) ? 0 : B;
+  cudaError_t e;
+  {
+    ProfScope ps("chain_kernel", st);
+    e = launch_chain(d, p, lengths, trans, dur, logZ, B, nbeta, st);
+  }
+  return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }
 
 extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, const float* dur,
@@ -239,26 +308,31 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     return SEMICRF_OK;
   }
   if (flags & SEMICRF_FLAG_FORWARD_ONLY) {
-    const size_t sm = recursion_smem_bytes(d, false);
-    rc = set_smem((const void*)chain_kernel, sm);
-    if (rc) return rc;
-    chain_kernel<<<B, d.NT, sm, st>>>(d, p, lengths, trans, dur, nullptr, 0);
-    if ((rc = launched())) return rc;
+    cudaError_t e;
+    {
+      ProfScope ps("chain_kernel", st);
+      e = launch_chain(d, p, lengths, trans, dur, nullptr, 0, B, st);
+    }
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
   }
   if (T > 0) {
-    const size_t sm = recursion_smem_bytes(d, d.store_smem != 0);
-    rc = set_smem((const void*)segment_kernel, sm);
-    if (rc) return rc;
-    segment_kernel<<<dim3(d.nck, B), d.NT, sm, st>>>(d, p, lengths, trans, dur, grad_logZ, grad_em,
-                                                     start_marg, end_marg);
-    if ((rc = launched())) return rc;
+    cudaError_t e;
+    {
+      ProfScope ps("segment_kernel", st);
+      e = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
+    }
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
     const int nj = FIN_ROWS_HOST / d.delta + 2;
     const size_t fsm = ((size_t)C + (size_t)nj * C) * sizeof(double);
     rc = set_smem((const void*)finalize_positions_kernel, fsm);
     if (rc) return rc;
-    finalize_positions_kernel<<<dim3((T + FIN_ROWS_HOST - 1) / FIN_ROWS_HOST, B), 256, fsm, st>>>(
-        d, p, lengths, grad_logZ, (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, grad_em, pos_marg,
-        start_marg, end_marg);
+    {
+      ProfScope ps("finalize_positions_kernel", st);
+      finalize_positions_kernel<<<dim3((T + FIN_ROWS_HOST - 1) / FIN_ROWS_HOST, B), 256, fsm,
+                                  st>>>(d, p, lengths, grad_logZ,
+                                        (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, grad_em,
+                                        pos_marg, start_marg, end_marg);
+    }
     if ((rc = launched())) return rc;
   } else {
     // T == 0: only boundary row 0 exists, and nothing starts or ends there
@@ -268,7 +342,10 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
       return SEMICRF_ERR_CUDA;
   }
   const int ne = C * C + K * C;
-  reduce_partials_kernel<<<(ne + 255) / 256, 256, 0, st>>>(d, p, lengths, grad_trans, grad_dur);
+  {
+    ProfScope ps("reduce_partials_kernel", st);
+    reduce_partials_kernel<<<(ne + 255) / 256, 256, 0, st>>>(d, p, lengths, grad_trans, grad_dur);
+  }
   return launched();
 }
 
@@ -287,11 +364,12 @@ extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const fl
   if (B == 0) return SEMICRF_OK;
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
   if (rc) return rc;
-  const size_t sm = recursion_smem_bytes(d, false);
-  rc = set_smem((const void*)viterbi_kernel, sm);
-  if (rc) return rc;
-  viterbi_kernel<<<B, d.NT, sm, st>>>(d, p, lengths, trans, dur, score, labels, seg_start);
-  return launched();
+  cudaError_t e;
+  {
+    ProfScope ps("viterbi_kernel", st);
+    e = launch_viterbi(d, p, lengths, trans, dur, score, labels, seg_start, st);
+  }
+  return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }
 
 extern "C" int semicrf_get_status(const void* ws, semicrf_stream_t stream, int* status) {
@@ -326,4 +404,35 @@ extern "C" int semicrf_selftest_bounded_wait(void* ws, size_t ws_bytes, int spin
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
   selftest_wait_kernel<<<1, 32, 0, st>>>(status, spins);
   return launched();
+}
+
+extern "C" int semicrf_profile_enable(int on) {
+  std::lock_guard<std::mutex> g(prof_mu);
+  prof_on = on != 0;
+  if (on) {
+    for (auto& r : prof_recs) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+    prof_recs.clear();
+  }
+  return SEMICRF_OK;
+}
+
+extern "C" int semicrf_profile_read(const char* kernel, double* total_ms, int* launches) {
+  if (!kernel || !total_ms || !launches) return SEMICRF_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(prof_mu);
+  double tot = 0.0;
+  int n = 0;
+  for (auto& r : prof_recs) {
+    if (std::strcmp(r.name, kernel) != 0) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return SEMICRF_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return SEMICRF_ERR_CUDA;
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
+  return SEMICRF_OK;
 }

@@ -58,6 +58,17 @@ __device__ __forceinline__ float ord2f(int i) {
   return __int_as_float(i >= 0 ? i : (i ^ 0x7fffffff));
 }
 
+__device__ __forceinline__ uint32_t smem_addr(const void* p);
+
+// Contributes `key` (an f2ord value; pass INT_MIN for "no value") to the
+// shared-memory max at `slot`: a warp-level max first, then one native
+// shared-memory reduction per warp.  Every lane of the warp must call it.
+__device__ __forceinline__ void warp_max_to_shared(int* slot, int key) {
+  const int m = __reduce_max_sync(FULL_MASK, key);
+  if ((threadIdx.x & 31) == 0)
+    asm volatile("red.shared.max.s32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(m) : "memory");
+}
+
 __device__ __forceinline__ void set_status(int* status, int code) {
   atomicCAS(status, 0, code);
 }

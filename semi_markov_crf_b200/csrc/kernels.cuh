@@ -1,6 +1,6 @@
-// kernels.cuh -- declarations of the semi-CRF kernels and their shared-memory
-// budgets.  Definitions live in prefix.cu, recursion.cu, finalize.cu and
-// viterbi.cu; the host layer in api.cu launches them.
+// kernels.cuh -- declarations of the semi-CRF kernels, their shared-memory
+// budgets and the host-side launchers that pick a compile-time lane shape.
+// Definitions live in prefix.cu, recursion.cu, finalize.cu and viterbi.cu.
 #pragma once
 
 #include "device.cuh"
@@ -8,14 +8,14 @@
 
 namespace semicrf {
 
-// Shared-memory bytes of the recursion kernels (carve order in recursion.cu).
+// Shared-memory bytes of the recursion kernels (carve order in ring.cuh).
 __host__ __device__ inline size_t recursion_smem_bytes(const Dims& d, bool with_store) {
   size_t b = 64;                                  // mbarriers + max slots + flags
   b += 2ull * TS * d.C * sizeof(int32_t);         // prefix-sum integer tiles
   b += 2ull * TS * d.C * sizeof(float);           // prefix-sum fraction tiles
-  b += (size_t)d.K * d.C * sizeof(float2);        // ring
-  b += 8ull * d.C * sizeof(float);                // Acur, pcur, stS[2], stE[2], tmp, Sbase
-  b += 16;
+  b += (size_t)d.RL * d.C * sizeof(float2);       // mirrored ring
+  b += (2ull * d.PC + 4ull * d.C) * sizeof(float);  // pcur[2], Acur[2], tmp, Sbase
+  b += 32;
   if (with_store) b += (size_t)d.delta * d.store_w * sizeof(float);
   return b;
 }
@@ -31,19 +31,6 @@ __global__ void prefix_scan_kernel(const float* __restrict__ em, const int32_t* 
                                    Dims d, WsPtrs ws, unsigned center, int mode,
                                    double* __restrict__ S64, float* __restrict__ nu_out);
 
-// grid.x = n_alpha + n_beta CTAs: the first n_alpha run the forward ring of
-// sequence blockIdx.x, the rest the backward ring of sequence
-// blockIdx.x - n_alpha (n_alpha is 0 or B; so is n_beta).
-__global__ void chain_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                             const float* __restrict__ trans, const float* __restrict__ dur,
-                             double* __restrict__ logZ_out, int n_alpha);
-
-// grid = (nck, B): one CTA per checkpoint segment.
-__global__ void segment_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                               const float* __restrict__ trans, const float* __restrict__ dur,
-                               const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
-                               float* __restrict__ start_marg, float* __restrict__ end_marg);
-
 __global__ void finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                           const double* __restrict__ grad_logZ, unsigned center,
                                           float* __restrict__ grad_em, float* __restrict__ pos_marg,
@@ -53,11 +40,28 @@ __global__ void finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __re
 __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                        float* __restrict__ grad_trans, float* __restrict__ grad_dur);
 
-__global__ void viterbi_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                               const float* __restrict__ trans, const float* __restrict__ dur,
-                               double* __restrict__ score, int32_t* __restrict__ labels,
-                               uint8_t* __restrict__ seg_start);
-
 __global__ void selftest_wait_kernel(int* status, int spins);
+
+// Lane shapes with a compiled instantiation (KBT durations, CAT labels per lane).
+bool shape_supported(int KBT, int CAT);
+
+// Host launchers for the shape in `d` (return the cudaError_t of the launch).
+// Forward ring of sequences [0, n_alpha) and backward ring of the rest:
+// grid = n_alpha + n_beta CTAs.
+cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths, const float* trans,
+                         const float* dur, double* logZ_out, int n_alpha, int n_beta,
+                         cudaStream_t st);
+// One CTA per (checkpoint segment, sequence).
+cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                           const float* trans, const float* dur, const double* grad_logZ,
+                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st);
+cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                           const float* trans, const float* dur, double* score, int32_t* labels,
+                           uint8_t* seg_start, cudaStream_t st);
+
+// Every lane shape the library instantiates.
+#define SEMICRF_FOR_EACH_SHAPE(X)                                                      \
+  X(2, 1) X(2, 2) X(2, 4) X(2, 8) X(2, 32) X(4, 1) X(4, 2) X(4, 4) X(4, 8) X(4, 32)    \
+  X(8, 1) X(8, 2) X(8, 4) X(8, 8) X(8, 32) X(16, 1) X(16, 2) X(16, 4) X(16, 8) X(16, 32)
 
 }  // namespace semicrf

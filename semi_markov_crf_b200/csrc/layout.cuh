@@ -11,20 +11,25 @@ namespace semicrf {
 constexpr int C_MAX = 128;
 constexpr int K_MAX = 512;
 constexpr int KC_MAX = 16384;
-constexpr int KB_MAX = 16;   // duration terms per lane in the k fan-in
-constexpr int CA_MAX = 32;   // label terms per lane in the label fan-in
 constexpr int NT_MAX = 512;  // threads per CTA
 constexpr int TS = 32;       // prefix-sum rows per TMA tile
 constexpr int FLUSH_EVERY = 64;  // positions between fp32 -> fp64 partial flushes
 
 // Problem sizes and the lane mapping chosen for them.
+//
+// Lane groups of GB lanes (a power of two <= 32) own one label each, for both
+// fan-ins: in the k fan-in lane j owns KBT consecutive durations, in the label
+// fan-in CAT consecutive labels of the other side.  KBT and CAT are
+// compile-time shapes of the kernel instantiation; GA == GB.
 struct Dims {
   int B, T, C, K;
   int delta;     // checkpoint spacing ceil(sqrt(T*K))
   int nck;       // checkpoint segments per sequence, ceil(T / delta)
   int Tstride;   // rows per sequence in the prefix-sum arrays (>= T+1, multiple of TS)
-  int GB, KB;    // k fan-in: lanes per label, duration terms per lane
-  int GA, CA;    // label fan-in: lanes per output label, label terms per lane
+  int KBT, GB;   // durations per lane, lanes per label (k fan-in)
+  int CAT, GA;   // labels per lane, lanes per output label (label fan-in)
+  int RL;        // ring entries per label: K + KBT (the first KBT slots are mirrored)
+  int PC;        // padded length of the exp-domain label vector (>= GA * CAT)
   int NT;        // threads per CTA of the recursion kernels
   int prefR;     // rows per prefix-sum chunk
   int nchunk;    // prefix-sum chunks per sequence
@@ -40,7 +45,7 @@ struct WsPtrs {
   double* chunk;   // [B][nchunk][C] per-chunk emission sums
   double* logz2;   // [B] log2 Z from the forward ring
   double* logz2b;  // [B] log2 Z from the backward ring
-  float2* ack;     // [B][nck][K][C] forward ring checkpoints
+  float2* ack;     // [B][nck][K][C] forward ring checkpoints (boundary order)
   double* acf;     // [B][nck] their frame bases
   float2* bck;     // [B][nck][K][C] backward ring checkpoints
   double* bcf;     // [B][nck]

@@ -24,279 +24,81 @@
 // the exponential domain (sum_c' 2^alpha[c'] * 2^trans[c',c], one ex2 per
 // label) and falls back to the log domain for any label whose sum underflows.
 //
-// Lane mapping (per CTA = one sequence or one checkpoint segment):
-//   k fan-in:     GB lanes per label, lane j handles k = 1 + j + i*GB (i < KB)
-//   label fan-in: GA lanes per label, lane j handles c' = j + i*GA (i < CA)
-// Group reductions are xor-shuffles inside aligned lane groups.
-#include "kernels.cuh"
+// Schedule.  One lane group owns one label for both fan-ins, so the k fan-in
+// of label c only reads label c's own ring, written by the same warp: a step
+// needs a single CTA barrier (between the k fan-in, which produces alpha[t, :],
+// and the label fan-in, which reads all of it).
+//
+// Ring entries are float2 (value v, exact integer part P); a term of the k
+// fan-in is ((P + Q) + v) + dur2 with Q the per-step integer offset.
+#include "ring.cuh"
 
 namespace semicrf {
 
+using namespace ring;
+
 namespace {
 
-struct Smem {
-  uint64_t* mbar;   // [2] tile barriers
-  int* maxslot;     // [2] per-step max (order-preserving ints)
-  int* flag;        // [4]
-  int32_t* tint;    // [2][TS][C]
-  float* tfrac;     // [2][TS][C]
-  float2* ring;     // [K][C] (value, exact integer part)
-  float* Acur;      // [C]
-  float* pcur;      // [C]
-  float* stS;       // [2][C]
-  float* stE;       // [2][C]
-  float* tmp;       // [C]
-  int* Sbase;       // [C]
-  float* store;     // [delta][store_w] (segment kernel, when in shared memory)
-};
-
-__device__ Smem carve(unsigned char* raw, const Dims& d, bool with_store) {
-  Smem s;
-  const int C = d.C;
-  unsigned char* p = raw;
-  s.mbar = reinterpret_cast<uint64_t*>(p);
-  s.maxslot = reinterpret_cast<int*>(p + 16);
-  s.flag = reinterpret_cast<int*>(p + 32);
-  p += 64;
-  s.tint = reinterpret_cast<int32_t*>(p);
-  p += 2ull * TS * C * sizeof(int32_t);
-  s.tfrac = reinterpret_cast<float*>(p);
-  p += 2ull * TS * C * sizeof(float);
-  s.ring = reinterpret_cast<float2*>(p);
-  p += (size_t)d.K * C * sizeof(float2);
-  float* f = reinterpret_cast<float*>(p);
-  s.Acur = f;
-  s.pcur = f + C;
-  s.stS = f + 2 * C;
-  s.stE = f + 4 * C;
-  s.tmp = f + 6 * C;
-  s.Sbase = reinterpret_cast<int*>(f + 7 * C);
-  p += 8ull * C * sizeof(float);
-  p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
-  s.store = with_store ? reinterpret_cast<float*>(p) : nullptr;
-  return s;
-}
-
-// Double-buffered TMA stream of prefix-sum tiles (TS rows each) for one
-// sequence, moving up (dir = +1) or down (dir = -1).
-struct TileStream {
-  int cur, lo, hi, dir;
-  uint32_t ph[2];
-};
-
-__device__ __forceinline__ void tile_issue(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
-                                           const TileStream& ts, int i) {
-  if (i < ts.lo || i > ts.hi) return;
-  if (threadIdx.x == 0) {
-    const int buf = i & 1;
-    const uint32_t bytes = (uint32_t)(TS * d.C * 4);
-    const size_t row0 = (size_t)b * d.Tstride + (size_t)i * TS;
-    fence_proxy_async();
-    mbar_expect_tx(&sm.mbar[buf], 2 * bytes);
-    bulk_g2s(sm.tint + (size_t)buf * TS * d.C, ws.sint + row0 * d.C, bytes, &sm.mbar[buf]);
-    bulk_g2s(sm.tfrac + (size_t)buf * TS * d.C, ws.sfrac + row0 * d.C, bytes, &sm.mbar[buf]);
+// Forward k fan-in at boundary t: A = alpha[t,c] - F_{t-1}; the leader writes
+// Acur/pcur (buffer `par`) and every warp adds to the step max (slot q).
+template <int KBT>
+__device__ __forceinline__ float fwd_kphase(const Smem& sm, const Dims& d, const KLane<KBT>& kl,
+                                            int base, const int32_t* ri, const float* rf,
+                                            float Frel, int par, int q, float (&e)[KBT]) {
+  const int c = kl.act ? kl.c : 0;
+  const float Q = (float)(ri[c] - sm.Sbase[c]) - Frel;
+  const KFan kf = k_fanin<KBT>(sm, d, kl, base, Q, e);
+  const float A = (kf.lse == NEG_INF) ? NEG_INF : rf[c] + kf.lse;
+  int key = INT_MIN;
+  if (kl.act && kl.j == 0) {
+    sm.Acur[par * d.C + c] = A;
+    sm.pcur[par * d.PC + c] = ex2(A);
+    key = f2ord(A);
   }
+  warp_max_to_shared(&sm.maxslot[q], key);
+  return A;
 }
 
-// Makes row r readable; returns false (uniformly) if a tile wait gave up.
-__device__ __forceinline__ bool tile_row(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
-                                         TileStream& ts, int r, const int32_t*& ri,
-                                         const float*& rf) {
-  const int i = r / TS;
-  bool ok = true;
-  if (i != ts.cur) {
-    const int buf = i & 1;
-    ok = mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
-    ts.ph[buf] ^= 1u;
-    ts.cur = i;
-    tile_issue(sm, d, ws, b, ts, i + ts.dir);
-    ok = !__syncthreads_or(!ok);
+// Label fan-in for output label al.c; returns the log2 sum minus the shift
+// (gamma - F_t for the forward side, beta - G_s for the backward side) in
+// the leader lane, with the log-domain fallback when the sum underflows.
+template <int CAT>
+__device__ __forceinline__ float aphase(const Smem& sm, const Dims& d, const ALane<CAT>& al, int par,
+                                        float n, float shift, const float* trans, bool rows,
+                                        float& acc, float (&prod)[CAT]) {
+  acc = label_fanin<CAT>(sm.pcur + par * d.PC, d, al, prod);
+  float g = 0.f;
+  if (al.act && al.j == 0) {
+    if (acc >= UNDERFLOW && acc <= 3.0e38f)
+      g = lg2(acc) + al.tmax - shift;
+    else
+      g = label_lse_slow(d, sm.Acur + par * d.C, n, trans, al.c, rows);
   }
-  const int buf = i & 1;
-  const size_t o = ((size_t)buf * TS + (r - i * TS)) * d.C;
-  ri = sm.tint + o;
-  rf = sm.tfrac + o;
-  return ok;
+  return g;
 }
 
-__device__ __forceinline__ void tile_start(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
-                                           TileStream& ts, int first_row, int lo_row, int hi_row,
-                                           int dir) {
-  ts.lo = lo_row / TS;
-  ts.hi = hi_row / TS;
-  ts.dir = dir;
-  ts.cur = -1;
-  // only the first tile here: entering a tile (tile_row) issues the next one
-  tile_issue(sm, d, ws, b, ts, first_row / TS);
+// Uniform slow path: the step's frame jump is too large for 2^A in float32.
+__device__ __forceinline__ void refresh_p(const Smem& sm, const Dims& d, int par, float n) {
+  for (int c = threadIdx.x; c < d.C; c += blockDim.x)
+    sm.pcur[par * d.PC + c] = ex2(sm.Acur[par * d.C + c] - n);
+  __syncthreads();
 }
 
-// Gives up on outstanding tiles after a timeout (bounded), so the CTA can
-// exit without copies in flight.
-__device__ void tile_drain(const Smem& sm, TileStream& ts) {
-  if (threadIdx.x == 0) {
-    for (int buf = 0; buf < 2; ++buf) mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
-  }
-}
-
-// Per-thread constant operands of the two fan-ins.
-struct Roles {
-  int cB, jB, cA, jA;
-  bool warpB, warpA;  // warp has at least one active lane in the phase
-};
-
-__device__ __forceinline__ Roles make_roles(const Dims& d) {
-  Roles r;
-  const int tid = threadIdx.x;
-  r.cB = tid / d.GB;
-  r.jB = tid % d.GB;
-  r.cA = tid / d.GA;
-  r.jA = tid % d.GA;
-  const int w0 = tid & ~31;
-  r.warpB = (w0 / d.GB) < d.C;
-  r.warpA = (w0 / d.GA) < d.C;
-  return r;
-}
-
-__device__ __forceinline__ float LOG2E() { return (float)LOG2E_D; }
-
-// dur2 values for this lane's durations.
-__device__ __forceinline__ void load_dur(const Dims& d, const Roles& r, const float* dur,
-                                         float (&dreg)[KB_MAX]) {
-  const int c = r.cB < d.C ? r.cB : 0;
-#pragma unroll
-  for (int i = 0; i < KB_MAX; ++i) {
-    const int k = 1 + r.jB + i * d.GB;
-    dreg[i] = (i < d.KB && k <= d.K) ? __ldg(dur + (size_t)(k - 1) * d.C + c) * LOG2E() : NEG_INF;
-  }
-}
-
-// Column-normalised 2^(trans2[c', c] - max_c' trans2[c', c]) for output c = cA
-// (forward label fan-in), or row-normalised for output row c' = cA (backward).
-__device__ __forceinline__ float load_trans_exp(const Dims& d, const Roles& r, const float* trans,
-                                                bool rows, float (&ereg)[CA_MAX]) {
-  const int C = d.C;
-  const int o = r.cA < C ? r.cA : 0;
-  float mx = NEG_INF;
-  for (int x = 0; x < C; ++x) {
-    const float v = __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * LOG2E();
-    mx = fmaxf(mx, v);
-  }
-  if (mx == NEG_INF) mx = 0.f;
-#pragma unroll
-  for (int i = 0; i < CA_MAX; ++i) {
-    const int x = r.jA + i * d.GA;
-    float e = 0.f;
-    if (i < d.CA && x < C) {
-      const float v = __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * LOG2E();
-      e = ex2(v - mx);
-    }
-    ereg[i] = e;
-  }
-  return mx;
-}
-
-// Log-domain label fan-in for one output (rare fallback when the
-// exponential-domain sum underflows): LSE_x (vals[x] - shift + trans2).
-__device__ float label_lse_slow(const Dims& d, const float* vals, float shift, const float* trans,
-                                int o, bool rows) {
-  const int C = d.C;
-  float mx = NEG_INF;
-  for (int x = 0; x < C; ++x) {
-    const float t2 = __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * LOG2E();
-    mx = fmaxf(mx, vals[x] - shift + t2);
-  }
-  if (mx == NEG_INF) return NEG_INF;
-  float s = 0.f;
-  for (int x = 0; x < C; ++x) {
-    const float t2 = __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * LOG2E();
-    s += ex2(vals[x] - shift + t2 - mx);
-  }
-  return mx + lg2(s);
-}
-
-// ---------------------------------------------------------------------------
-// k fan-in.  Forward (up = true): terms at boundary t from ring slots t-k,
-//   y_k = (P[t-k] + Q) + v[t-k] + dur2[k-1],  Q = (Sint[t]-Sbase) - Frel.
-// Backward (up = false): terms at boundary s from ring slots s+k,
-//   y_k = (P[s+k] + Q) + v[s+k] + dur2[k-1],  Q = -(Sint[s]-Sbase) - Grel.
-// Returns the group LSE (valid in every lane of the group) and leaves the
-// per-term exponentials e[i] = 2^(y_i - m) and their sum for posterior use.
-struct KFan {
-  float lse;  // m + lg2(sum), NEG_INF if no valid term
-  float m, sum;
-};
-
-__device__ __forceinline__ KFan k_fanin(const Smem& sm, const Dims& d, const Roles& r, int tb,
-                                        int kmax, float Q, bool up, const float (&dreg)[KB_MAX],
-                                        float (&e)[KB_MAX]) {
-  const int C = d.C, K = d.K;
-  const bool act = r.cB < C;
-  const int c = act ? r.cB : 0;
-  float y[KB_MAX];
+__device__ __forceinline__ void final_lse(const float* A, int C, double base, double* out2,
+                                          double* out_nat) {
+  if (threadIdx.x >= 32) return;
   float m = NEG_INF;
-#pragma unroll
-  for (int i = 0; i < KB_MAX; ++i) {
-    y[i] = NEG_INF;
-    const int k = 1 + r.jB + i * d.GB;
-    if (i < d.KB && act && k <= kmax) {
-      int slot = up ? tb - k : tb + k;
-      if (up) {
-        if (slot < 0) slot += K;
-      } else {
-        if (slot >= K) slot -= K;
-      }
-      const float2 v = sm.ring[slot * C + c];
-      y[i] = ((v.y + Q) + v.x) + dreg[i];
-      m = fmaxf(m, y[i]);
-    }
-  }
-  m = group_max(m, d.GB);
+  for (int c = threadIdx.x; c < C; c += 32) m = fmaxf(m, A[c]);
+  m = group_max(m, 32);
   float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < KB_MAX; ++i) {
-    e[i] = 0.f;
-    if (i < d.KB && m != NEG_INF) {
-      e[i] = ex2(y[i] - m);
-      s += e[i];
-    }
+  if (m != NEG_INF)
+    for (int c = threadIdx.x; c < C; c += 32) s += ex2(A[c] - m);
+  s = group_sum(s, 32);
+  if (threadIdx.x == 0) {
+    const double lz = (m == NEG_INF) ? -INFINITY : base + (double)(m + lg2(s));
+    *out2 = lz;
+    if (out_nat) *out_nat = lz * LN2_D;
   }
-  s = group_sum(s, d.GB);
-  KFan out;
-  out.m = m;
-  out.sum = s;
-  out.lse = (m == NEG_INF) ? NEG_INF : m + lg2(s);
-  return out;
-}
-
-// Label fan-in in the exponential domain: sum_x p[x] * ereg[x] over this
-// lane's labels, group-reduced.  prod[i] keeps the per-term products.
-__device__ __forceinline__ float label_fanin(const Smem& sm, const Dims& d, const Roles& r,
-                                             const float (&ereg)[CA_MAX], float (&prod)[CA_MAX]) {
-  const bool act = r.cA < d.C;
-  float acc = 0.f;
-#pragma unroll
-  for (int i = 0; i < CA_MAX; ++i) {
-    prod[i] = 0.f;
-    const int x = r.jA + i * d.GA;
-    if (i < d.CA && act && x < d.C) {
-      prod[i] = sm.pcur[x] * ereg[i];
-      acc += prod[i];
-    }
-  }
-  return group_sum(acc, d.GA);
-}
-
-constexpr float EXP_SAFE = 100.f;      // |frame jump| beyond which p is recomputed
-constexpr float UNDERFLOW = 0x1p-100f;  // label sums below this use the log domain
-
-// Reads the step max, resets the other slot, and returns the integer frame
-// step n.  `slow` is set when 2^(value) may overflow/underflow.
-__device__ __forceinline__ float step_frame(const Smem& sm, int parity, bool& slow) {
-  const float M = ord2f(sm.maxslot[parity]);
-  __syncwarp();
-  const bool fin = isfinite(M);
-  slow = fin && (M > EXP_SAFE || M < -EXP_SAFE);
-  return fin ? rintf(M) : 0.f;
 }
 
 }  // namespace
@@ -304,6 +106,7 @@ __device__ __forceinline__ float step_frame(const Smem& sm, int parity, bool& sl
 // ===========================================================================
 // Forward and backward rings over whole sequences.
 // ===========================================================================
+template <int KBT, int CAT>
 __global__ void __launch_bounds__(NT_MAX, 1)
     chain_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                  const float* __restrict__ trans, const float* __restrict__ dur,
@@ -314,141 +117,104 @@ __global__ void __launch_bounds__(NT_MAX, 1)
   const bool is_alpha = (int)blockIdx.x < n_alpha;
   const int b = is_alpha ? blockIdx.x : blockIdx.x - n_alpha;
   const int L = lengths[b];
-  if (L < 0 || L > d.T) {
+  if (L < 0 || L > d.T || L == 0) {
     if (tid == 0) {
-      set_status(ws.status, ST_BAD_LENGTH);
+      const double v = (L == 0) ? 0.0 : __longlong_as_double(0x7ff8000000000000ll);
+      if (L != 0) set_status(ws.status, ST_BAD_LENGTH);
       if (is_alpha) {
-        logZ_out[b] = __longlong_as_double(0x7ff8000000000000ll);
-        ws.logz2[b] = __longlong_as_double(0x7ff8000000000000ll);
+        logZ_out[b] = v;
+        ws.logz2[b] = v;
       } else {
-        ws.logz2b[b] = __longlong_as_double(0x7ff8000000000000ll);
+        ws.logz2b[b] = v;
       }
     }
     return;
   }
-  if (L == 0) {
-    if (tid == 0) {
-      if (is_alpha) {
-        logZ_out[b] = 0.0;
-        ws.logz2[b] = 0.0;
-      } else {
-        ws.logz2b[b] = 0.0;
-      }
-    }
-    return;
-  }
-  const Roles r = make_roles(d);
-  float dreg[KB_MAX], ereg[CA_MAX], e[KB_MAX], prod[CA_MAX];
-  load_dur(d, r, dur, dreg);
-  const float tmax2 = load_trans_exp(d, r, trans, !is_alpha, ereg);
-
-  if (tid == 0) {
-    mbar_init(&sm.mbar[0], 1);
-    mbar_init(&sm.mbar[1], 1);
-    fence_mbar_init();
-    sm.maxslot[0] = f2ord(NEG_INF);
-    sm.maxslot[1] = f2ord(NEG_INF);
-  }
+  const bool warp_on = ((tid & ~31) / d.GB) < C;
+  KLane<KBT> kl;
+  kl.init(d, dur, is_alpha);
+  ALane<CAT> al;
+  al.init(d, trans, !is_alpha);
+  float e[KBT], prod[CAT], acc;
+  init_smem(sm, d);
   __syncthreads();
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
-  const int* Sb = sm.Sbase;
   const int32_t* ri;
   const float* rf;
+  int par = 0, q = 0;
 
   if (is_alpha) {
     // ---------------------------------------------------------------- forward
     for (int c = tid; c < C; c += blockDim.x) {
-      sm.ring[c] = make_float2(0.f, 0.f);  // boundary 0: gamma = 0, frame 0, S = 0
+      ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));  // boundary 0: gamma 0, frame 0, S 0
       sm.Sbase[c] = 0;
     }
-    tile_start(sm, d, ws, b, ts, 0, 0, L, +1);
+    tile_start(sm, d, ws, b, ts, 1, 0, L, +1);
     double F0 = 0.0;
     float Frel = 0.f;
-    int tb = 0;
+    int slot = 0;                 // t mod K
+    int base = kl.base_up(1, K);  // window base at t = 1
+    int to_ck = d.delta;          // steps to the next checkpoint boundary
     __syncthreads();
     for (int t = 1; t <= L; ++t) {
-      tb = (tb + 1 == K) ? 0 : tb + 1;
+      if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
+      slot = (slot + 1 == K) ? 0 : slot + 1;
+      par = t & 1;
+      q = mod3_next(q);
       if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
         if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
         tile_drain(sm, ts);
         return;
       }
-      if (t % d.delta == 0 && t < L) {
-        // checkpoint j: rebase frames to (F0 + Frel, S_int[t]) and save the ring
-        const int j = t / d.delta;
-        const float dF = Frel;
-        for (int idx = tid; idx < K * C; idx += blockDim.x) {
-          const int i = idx / C, c = idx % C;
-          if (t - K + i < 0) continue;
-          int slot = tb + i;
-          if (slot >= K) slot -= K;
-          float2 v = sm.ring[slot * C + c];
-          v.y = (v.y - dF) + (float)(ri[c] - Sb[c]);
-          sm.ring[slot * C + c] = v;
-          ws.ack[(((size_t)b * d.nck + j) * K + i) * C + c] = v;
-        }
-        __syncthreads();
-        for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
-        F0 += (double)dF;
-        Frel = 0.f;
-        if (tid == 0) ws.acf[(size_t)b * d.nck + j] = F0;
-        __syncthreads();
-      }
-      const int par = t & 1;
-      if (r.warpB) {
-        const bool act = r.cB < C;
-        const int c = act ? r.cB : 0;
-        const float Q = (float)(ri[c] - Sb[c]) - Frel;
-        const KFan kf = k_fanin(sm, d, r, tb, min(K, t), Q, true, dreg, e);
-        if (act && r.jB == 0) {
-          const float A = (kf.lse == NEG_INF) ? NEG_INF : rf[c] + kf.lse;
-          sm.Acur[c] = A;
-          sm.pcur[c] = ex2(A);
-          atomicMax(&sm.maxslot[par], f2ord(A));
+      if (--to_ck == 0) {
+        to_ck = d.delta;
+        if (t < L) {
+          // checkpoint j: rebase to (F0 + Frel, S_int[t]), save the ring in boundary order
+          __syncthreads();
+          const int j = t / d.delta;
+          const float dF = Frel;
+          for (int idx = tid; idx < C * d.RL; idx += blockDim.x) {
+            const int c = idx / d.RL;
+            float2 v = sm.ring[idx];
+            v.y = (v.y - dF) + (float)(ri[c] - sm.Sbase[c]);
+            sm.ring[idx] = v;
+          }
+          __syncthreads();
+          for (int idx = tid; idx < K * C; idx += blockDim.x) {
+            const int i = idx / C, c = idx % C;
+            if (t - K + i >= 0)
+              ws.ack[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t - K + i);
+          }
+          for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
+          F0 += (double)dF;
+          Frel = 0.f;
+          if (tid == 0) ws.acf[(size_t)b * d.nck + j] = F0;
+          __syncthreads();
         }
       }
+      if (warp_on) fwd_kphase<KBT>(sm, d, kl, base, ri, rf, Frel, par, q, e);
       __syncthreads();
       bool slow;
-      const float n = step_frame(sm, par, slow);
-      if (tid == 0) sm.maxslot[par ^ 1] = f2ord(NEG_INF);
+      const float n = step_frame(sm, q, slow);
       if (t == L) break;
       float shift = n;
       if (slow) {
-        for (int c = tid; c < C; c += blockDim.x) sm.pcur[c] = ex2(sm.Acur[c] - n);
-        __syncthreads();
+        refresh_p(sm, d, par, n);
         shift = 0.f;
       }
-      if (r.warpA) {
-        const float acc = label_fanin(sm, d, r, ereg, prod);
-        if (r.cA < C && r.jA == 0) {
-          const int c = r.cA;
-          float g;
-          if (acc >= UNDERFLOW && acc <= 3.0e38f)
-            g = lg2(acc) + tmax2 - shift;
-          else
-            g = label_lse_slow(d, sm.Acur, n, trans, c, false);
-          sm.ring[tb * C + c] = make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - Sb[c]));
+      if (warp_on) {
+        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, false, acc, prod);
+        if (al.act && al.j == 0) {
+          const int c = al.c;
+          ring_put<KBT>(sm, d, c, slot,
+                        make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
         }
+        __syncwarp();
       }
       Frel += n;
-      __syncthreads();
     }
-    // log Z = F_{L-1} + LSE_c A_L[c]
-    if (tid < 32) {
-      float m = NEG_INF;
-      for (int c = tid; c < C; c += 32) m = fmaxf(m, sm.Acur[c]);
-      m = group_max(m, 32);
-      float s = 0.f;
-      if (m != NEG_INF)
-        for (int c = tid; c < C; c += 32) s += ex2(sm.Acur[c] - m);
-      s = group_sum(s, 32);
-      if (tid == 0) {
-        const double lz = (m == NEG_INF) ? -INFINITY : F0 + (double)Frel + (double)(m + lg2(s));
-        ws.logz2[b] = lz;
-        logZ_out[b] = lz * LN2_D;
-      }
-    }
+    final_lse(sm.Acur + par * C, C, F0 + (double)Frel, &ws.logz2[b], &logZ_out[b]);
   } else {
     // --------------------------------------------------------------- backward
     tile_start(sm, d, ws, b, ts, L, 0, L, -1);
@@ -457,40 +223,40 @@ __global__ void __launch_bounds__(NT_MAX, 1)
       tile_drain(sm, ts);
       return;
     }
-    int sb = L % K;
+    int slot = L % K;
     for (int c = tid; c < C; c += blockDim.x) {
-      sm.ring[sb * C + c] = make_float2(rf[c], 0.f);  // beta[L] = 0, frame 0, base S_int[L]
+      ring_put<KBT>(sm, d, c, slot, make_float2(rf[c], 0.f));  // beta[L] = 0, frame 0, base S_int[L]
       sm.Sbase[c] = ri[c];
     }
     double G0 = 0.0;
     float Grel = 0.f;
+    int base = kl.base_down(L - 1, K);
+    int to_ck = L % d.delta;  // (s + 1) mod delta
     __syncthreads();
     for (int s = L - 1; s >= 0; --s) {
-      sb = (sb == 0) ? K - 1 : sb - 1;
+      if (s < L - 1) base = (base == 0) ? K - 1 : base - 1;
+      slot = (slot == 0) ? K - 1 : slot - 1;
+      par = s & 1;
+      q = mod3_next(q);
       if (!tile_row(sm, d, ws, b, ts, s, ri, rf)) {
         if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
         tile_drain(sm, ts);
         return;
       }
-      const int t1 = s + 1;
-      if (t1 % d.delta == 0 && t1 < L) {
+      if (to_ck == 0 && s + 1 < L) {
         // checkpoint j: the ring holds boundaries t1..t1+K-1; rebase to (G0 + Grel, S_int[t1])
+        __syncthreads();
+        const int t1 = s + 1;
         const int j = t1 / d.delta - 1;
-        int s1 = sb + 1;
-        if (s1 >= K) s1 -= K;
-        for (int c = tid; c < C; c += blockDim.x) sm.tmp[c] = sm.ring[s1 * C + c].y;
+        for (int c = tid; c < C; c += blockDim.x) sm.tmp[c] = ring_at(sm, d, c, t1).y;
+        __syncthreads();
+        for (int idx = tid; idx < C * d.RL; idx += blockDim.x) sm.ring[idx].y -= sm.tmp[idx / d.RL];
         __syncthreads();
         for (int idx = tid; idx < K * C; idx += blockDim.x) {
           const int i = idx / C, c = idx % C;
-          if (t1 + i > L) continue;
-          int slot = s1 + i;
-          if (slot >= K) slot -= K;
-          float2 v = sm.ring[slot * C + c];
-          v.y = v.y - sm.tmp[c];
-          sm.ring[slot * C + c] = v;
-          ws.bck[(((size_t)b * d.nck + j) * K + i) * C + c] = v;
+          if (t1 + i <= L)
+            ws.bck[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t1 + i);
         }
-        __syncthreads();
         for (int c = tid; c < C; c += blockDim.x)
           sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
         G0 += (double)Grel;
@@ -498,62 +264,56 @@ __global__ void __launch_bounds__(NT_MAX, 1)
         if (tid == 0) ws.bcf[(size_t)b * d.nck + j] = G0;
         __syncthreads();
       }
-      const int par = s & 1;
-      if (r.warpB) {
-        const bool act = r.cB < C;
-        const int c = act ? r.cB : 0;
-        const float Q = -(float)(ri[c] - Sb[c]) - Grel;
-        const KFan kf = k_fanin(sm, d, r, sb, min(K, L - s), Q, false, dreg, e);
-        if (act && r.jB == 0) {
-          const float Bt = (kf.lse == NEG_INF) ? NEG_INF : kf.lse - rf[c];
-          sm.Acur[c] = Bt;
-          sm.pcur[c] = ex2(Bt);
-          atomicMax(&sm.maxslot[par], f2ord(Bt));
+      to_ck = (to_ck == 0) ? d.delta - 1 : to_ck - 1;
+      if (warp_on) {
+        const int c = kl.act ? kl.c : 0;
+        const float Q = -(float)(ri[c] - sm.Sbase[c]) - Grel;
+        const KFan kf = k_fanin<KBT>(sm, d, kl, base, Q, e);
+        const float Bt = (kf.lse == NEG_INF) ? NEG_INF : kf.lse - rf[c];
+        int key = INT_MIN;
+        if (kl.act && kl.j == 0) {
+          sm.Acur[par * C + c] = Bt;
+          sm.pcur[par * d.PC + c] = ex2(Bt);
+          key = f2ord(Bt);
         }
+        warp_max_to_shared(&sm.maxslot[q], key);
       }
       __syncthreads();
       bool slow;
-      const float n = step_frame(sm, par, slow);
-      if (tid == 0) sm.maxslot[par ^ 1] = f2ord(NEG_INF);
+      const float n = step_frame(sm, q, slow);
       if (s == 0) break;
       float shift = n;
       if (slow) {
-        for (int c = tid; c < C; c += blockDim.x) sm.pcur[c] = ex2(sm.Acur[c] - n);
-        __syncthreads();
+        refresh_p(sm, d, par, n);
         shift = 0.f;
       }
-      if (r.warpA) {
-        const float acc = label_fanin(sm, d, r, ereg, prod);
-        if (r.cA < C && r.jA == 0) {
-          const int c = r.cA;
-          float g;
-          if (acc >= UNDERFLOW && acc <= 3.0e38f)
-            g = lg2(acc) + tmax2 - shift;
-          else
-            g = label_lse_slow(d, sm.Acur, n, trans, c, true);
-          sm.ring[sb * C + c] = make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - Sb[c]));
+      if (warp_on) {
+        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, true, acc, prod);
+        if (al.act && al.j == 0) {
+          const int c = al.c;
+          ring_put<KBT>(sm, d, c, slot,
+                        make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - sm.Sbase[c])));
         }
+        __syncwarp();
       }
       Grel += n;
-      __syncthreads();
     }
-    if (tid < 32) {
-      float m = NEG_INF;
-      for (int c = tid; c < C; c += 32) m = fmaxf(m, sm.Acur[c]);
-      m = group_max(m, 32);
-      float s = 0.f;
-      if (m != NEG_INF)
-        for (int c = tid; c < C; c += 32) s += ex2(sm.Acur[c] - m);
-      s = group_sum(s, 32);
-      if (tid == 0)
-        ws.logz2b[b] = (m == NEG_INF) ? -INFINITY : G0 + (double)Grel + (double)(m + lg2(s));
-    }
+    final_lse(sm.Acur + par * C, C, G0 + (double)Grel, &ws.logz2b[b], nullptr);
   }
 }
 
 // ===========================================================================
 // Checkpoint-parallel posteriors: one CTA per (segment j, sequence b).
+// Restores the forward ring at t0 = j*Delta and recomputes alpha over
+// [t0, t1) into a per-position store, then restores the backward ring at t1
+// and walks down to t0 accumulating the exact posteriors:
+//   start_marg[s,c] = 2^(gamma[s,c] + btil[s,c] - log2 Z)
+//   end_marg[s,c]   = 2^(alpha[s,c] + beta[s,c] - log2 Z)
+//   P(segment [s, s+k), c) = start_marg[s,c] * (normalised k term of btil)
+//   P(c' -> c at s)        = end_marg[s,c'] * (normalised c term of beta)
+// The leader lane of label c's group keeps c's running sums.
 // ===========================================================================
+template <int KBT, int CAT>
 __global__ void __launch_bounds__(NT_MAX, 1)
     segment_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                    const float* __restrict__ trans, const float* __restrict__ dur,
@@ -569,293 +329,257 @@ __global__ void __launch_bounds__(NT_MAX, 1)
   if (t0 >= L) return;
   const int t1 = min(t0 + d.delta, L);
   const bool last = (t1 == L);
-  const double gb = grad_logZ ? grad_logZ[b] : 1.0;
-  const float gbf = (float)gb;
+  const float gbf = (float)(grad_logZ ? grad_logZ[b] : 1.0);
   const double logz2 = ws.logz2[b];
   const int SW = d.store_w;
   float* store = sm.store ? sm.store : ws.store + ((size_t)b * d.nck + j) * d.delta * SW;
   const size_t seg = (size_t)b * d.nck + j;
-
-  const Roles r = make_roles(d);
-  float dreg[KB_MAX], ereg[CA_MAX], e[KB_MAX], prod[CA_MAX];
-  float accd[KB_MAX], acct[CA_MAX];
-  load_dur(d, r, dur, dreg);
-#pragma unroll
-  for (int i = 0; i < KB_MAX; ++i) accd[i] = 0.f;
-#pragma unroll
-  for (int i = 0; i < CA_MAX; ++i) acct[i] = 0.f;
-  // zero this CTA's float64 partials (each thread its own entries)
-  if (r.cB < C) {
-    for (int i = 0; i < d.KB; ++i) {
-      const int k = 1 + r.jB + i * d.GB;
-      if (k <= K) ws.pgd[(seg * K + (k - 1)) * C + r.cB] = 0.0;
-    }
-  }
-  if (r.cA < C) {
-    for (int i = 0; i < d.CA; ++i) {
-      const int x = r.jA + i * d.GA;
-      if (x < C) ws.pgt[(seg * C + r.cA) * C + x] = 0.0;
-    }
-  }
-  if (tid == 0) {
-    mbar_init(&sm.mbar[0], 1);
-    mbar_init(&sm.mbar[1], 1);
-    fence_mbar_init();
-    sm.maxslot[0] = f2ord(NEG_INF);
-    sm.maxslot[1] = f2ord(NEG_INF);
-  }
+  const bool warp_on = ((tid & ~31) / d.GB) < C;
+  float e[KBT], prod[CAT], acc;
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
-  const int* Sb = sm.Sbase;
   const int32_t* ri;
   const float* rf;
-
-  // ------------------------------------------------------ alpha recompute
-  float tmax2 = load_trans_exp(d, r, trans, false, ereg);
   double F0 = 0.0;
   float Frel = 0.f;
-  int t_start;
-  if (j == 0) {
-    for (int c = tid; c < C; c += blockDim.x) {
-      sm.ring[c] = make_float2(0.f, 0.f);
-      sm.Sbase[c] = 0;
-      store[c] = NEG_INF;   // no alpha at boundary 0
-      store[C + c] = 0.f;   // gamma[0] = 0 in frame 0
+  int par = 0, q = 0;
+
+  // ------------------------------------------------------ alpha recompute
+  {
+    KLane<KBT> kl;
+    kl.init(d, dur, true);
+    ALane<CAT> al;
+    al.init(d, trans, false);
+    init_smem(sm, d);
+    __syncthreads();
+    int t_start;
+    if (j == 0) {
+      for (int c = tid; c < C; c += blockDim.x) {
+        ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));
+        sm.Sbase[c] = 0;
+        store[c] = NEG_INF;  // no alpha at boundary 0
+        store[C + c] = 0.f;  // gamma[0] = 0 in frame 0
+      }
+      if (tid == 0) {
+        store[2 * C] = 0.f;
+        store[2 * C + 1] = 0.f;
+      }
+      t_start = 1;
+    } else {
+      const float2* ck = ws.ack + seg * K * C;
+      for (int idx = tid; idx < K * C; idx += blockDim.x) {
+        const int i = idx / C, c = idx % C;
+        const int bnd = t0 - K + i;
+        if (bnd >= 0) ring_put<KBT>(sm, d, c, bnd % K, ck[idx]);
+      }
+      for (int c = tid; c < C; c += blockDim.x)
+        sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t0) * C + c];
+      F0 = ws.acf[seg];
+      t_start = t0;
     }
-    if (tid == 0) {
-      store[2 * C] = 0.f;
-      store[2 * C + 1] = 0.f;
-    }
-    t_start = 1;
-  } else {
-    const float2* ck = ws.ack + seg * K * C;
-    for (int idx = tid; idx < K * C; idx += blockDim.x) {
-      const int i = idx / C, c = idx % C;
-      const int bnd = t0 - K + i;
-      if (bnd < 0) continue;
-      sm.ring[(bnd % K) * C + c] = ck[idx];
-    }
-    for (int c = tid; c < C; c += blockDim.x)
-      sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t0) * C + c];
-    F0 = ws.acf[seg];
-    t_start = t0;
-  }
-  const int t_end = last ? L : t1 - 1;
-  __syncthreads();
-  if (t_start <= t_end) {
+    const int t_end = last ? L : t1 - 1;
+    __syncthreads();
     tile_start(sm, d, ws, b, ts, t_start, t_start, t_end, +1);
-    int tb = t_start % K;
+    int slot = t_start % K;
+    int base = kl.base_up(t_start, K);
     for (int t = t_start; t <= t_end; ++t) {
-      if (t > t_start) tb = (tb + 1 == K) ? 0 : tb + 1;
+      if (t > t_start) {
+        base = (base + 1 == K) ? 0 : base + 1;
+        slot = (slot + 1 == K) ? 0 : slot + 1;
+      }
+      par = t & 1;
+      q = mod3_next(q);
       if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
         if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
         tile_drain(sm, ts);
         return;
       }
-      const int par = t & 1;
-      if (r.warpB) {
-        const bool act = r.cB < C;
-        const int c = act ? r.cB : 0;
-        const float Q = (float)(ri[c] - Sb[c]) - Frel;
-        const KFan kf = k_fanin(sm, d, r, tb, min(K, t), Q, true, dreg, e);
-        if (act && r.jB == 0) {
-          const float A = (kf.lse == NEG_INF) ? NEG_INF : rf[c] + kf.lse;
-          sm.Acur[c] = A;
-          sm.pcur[c] = ex2(A);
-          atomicMax(&sm.maxslot[par], f2ord(A));
-        }
-      }
+      float A = 0.f;
+      if (warp_on) A = fwd_kphase<KBT>(sm, d, kl, base, ri, rf, Frel, par, q, e);
       __syncthreads();
       bool slow;
-      const float n = step_frame(sm, par, slow);
-      if (tid == 0) sm.maxslot[par ^ 1] = f2ord(NEG_INF);
+      const float n = step_frame(sm, q, slow);
       if (t == L) break;
       float shift = n;
       if (slow) {
-        for (int c = tid; c < C; c += blockDim.x) sm.pcur[c] = ex2(sm.Acur[c] - n);
-        __syncthreads();
+        refresh_p(sm, d, par, n);
         shift = 0.f;
       }
       float* row = store + (size_t)(t - t0) * SW;
-      if (r.warpA) {
-        const float acc = label_fanin(sm, d, r, ereg, prod);
-        if (r.cA < C && r.jA == 0) {
-          const int c = r.cA;
-          float g;
-          if (acc >= UNDERFLOW && acc <= 3.0e38f)
-            g = lg2(acc) + tmax2 - shift;
-          else
-            g = label_lse_slow(d, sm.Acur, n, trans, c, false);
-          sm.ring[tb * C + c] = make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - Sb[c]));
-          row[c] = sm.Acur[c];
+      if (warp_on) {
+        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, false, acc, prod);
+        if (al.act && al.j == 0) {
+          const int c = al.c;
+          ring_put<KBT>(sm, d, c, slot,
+                        make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
+          row[c] = A;
           row[C + c] = g;
         }
+        __syncwarp();
       }
       if (tid == 0) {
         row[2 * C] = Frel;
         row[2 * C + 1] = Frel + n;
       }
       Frel += n;
-      __syncthreads();
     }
   }
+  __syncthreads();
   if (last) {
     // end marginal at boundary L (beta[L] = 0); nothing starts at L
     const float XL = (float)(F0 + (double)Frel - logz2);
     for (int c = tid; c < C; c += blockDim.x) {
       const size_t o = ((size_t)b * (d.T + 1) + L) * C + c;
-      if (end_marg) end_marg[o] = ex2(sm.Acur[c] + XL);
+      if (end_marg) end_marg[o] = ex2(sm.Acur[par * C + c] + XL);
       if (start_marg) start_marg[o] = 0.f;
     }
   }
-  __syncthreads();
 
   // ------------------------------------------------------ beta recompute + posteriors
-  tmax2 = load_trans_exp(d, r, trans, true, ereg);  // row-normalised now
+  KLane<KBT> kb;
+  kb.init(d, dur, false);
+  ALane<CAT> ab;
+  ab.init(d, trans, true);
+  __syncthreads();
+  for (int i = tid; i < d.RL * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  __syncthreads();
   double G0 = 0.0;
   float Grel = 0.f;
-  int sb = t1 % K;
   if (last) {
     for (int c = tid; c < C; c += blockDim.x) {
       const size_t o = ((size_t)b * d.Tstride + L) * C + c;
-      sm.ring[sb * C + c] = make_float2(ws.sfrac[o], 0.f);
+      ring_put<KBT>(sm, d, c, L % K, make_float2(ws.sfrac[o], 0.f));
       sm.Sbase[c] = ws.sint[o];
     }
   } else {
     const float2* ck = ws.bck + seg * K * C;
     for (int idx = tid; idx < K * C; idx += blockDim.x) {
       const int i = idx / C, c = idx % C;
-      if (t1 + i > L) continue;
-      sm.ring[((t1 + i) % K) * C + c] = ck[idx];
+      if (t1 + i <= L) ring_put<KBT>(sm, d, c, (t1 + i) % K, ck[idx]);
     }
     for (int c = tid; c < C; c += blockDim.x)
       sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
     G0 = ws.bcf[seg];
   }
+  // this CTA's float64 partials start at zero (each thread its own entries)
+  float accd[KBT];
+  float acct[CAT];
+#pragma unroll
+  for (int i = 0; i < KBT; ++i) {
+    accd[i] = 0.f;
+    const int k = kb.k_of(i, false);
+    if (kb.act && k <= K) ws.pgd[(seg * K + (k - 1)) * C + kb.c] = 0.0;
+  }
+#pragma unroll
+  for (int i = 0; i < CAT; ++i) {
+    acct[i] = 0.f;
+    const int x = ab.j * CAT + i;
+    if (ab.act && x < C) ws.pgt[(seg * C + ab.c) * C + x] = 0.0;
+  }
   const double Xc = F0 + G0 - logz2;
-  double accmu = 0.0, vsum = 0.0;  // thread c < C: suffix sum of (start - end) marginals
+  double accmu = 0.0, vsum = 0.0;  // leader of label c: suffix sum of (start - end) marginals
+  const bool leader = kb.act && kb.j == 0;
   __syncthreads();
   tile_start(sm, d, ws, b, ts, t1 - 1, t0, t1 - 1, -1);
   int nflush = 0;
+  int slot = t1 % K;
+  int base = kb.base_down(t1 - 1, K);
   for (int s = t1 - 1; s >= t0; --s) {
-    sb = (sb == 0) ? K - 1 : sb - 1;
+    if (s < t1 - 1) base = (base == 0) ? K - 1 : base - 1;
+    slot = (slot == 0) ? K - 1 : slot - 1;
+    par = s & 1;
+    q = mod3_next(q);
     if (!tile_row(sm, d, ws, b, ts, s, ri, rf)) {
       if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
       tile_drain(sm, ts);
       return;
     }
-    const int par = s & 1;
-    if (s < t1 - 1 && tid < C) {
-      // position s+1: v = sum of (start - end) marginals strictly after it
-      const int u = s + 1;
-      const float v = (float)accmu;
-      grad_em[((size_t)b * d.T + u) * C + tid] = v;
-      vsum += (double)v;
-      accmu += (double)sm.stS[(par ^ 1) * C + tid] - (double)sm.stE[(par ^ 1) * C + tid];
-    }
     const float* row = store + (size_t)(s - t0) * SW;
-    if (r.warpB) {
-      const bool act = r.cB < C;
-      const int c = act ? r.cB : 0;
-      const float Q = -(float)(ri[c] - Sb[c]) - Grel;
-      const KFan kf = k_fanin(sm, d, r, sb, min(K, L - s), Q, false, dreg, e);
+    float St = 0.f;
+    if (warp_on) {
+      const int c = kb.act ? kb.c : 0;
+      const float Q = -(float)(ri[c] - sm.Sbase[c]) - Grel;
+      const KFan kf = k_fanin<KBT>(sm, d, kb, base, Q, e);
       const float Bt = (kf.lse == NEG_INF) ? NEG_INF : kf.lse - rf[c];
-      // start marginal St[s, c] = 2^(gamma[s,c] + btil[s,c] - log2 Z)
-      float St = 0.f;
-      if (act && r.jB == 0) {
+      int key = INT_MIN;
+      if (leader) {
         const float Xs = (float)(Xc + (double)row[2 * C + 1] + (double)Grel);
         St = (Bt == NEG_INF) ? 0.f : ex2(row[C + c] + Bt + Xs);
-        sm.Acur[c] = Bt;
-        sm.pcur[c] = ex2(Bt);
-        atomicMax(&sm.maxslot[par], f2ord(Bt));
-        sm.stS[par * C + c] = St;
+        sm.Acur[par * C + c] = Bt;
+        sm.pcur[par * d.PC + c] = ex2(Bt);
+        key = f2ord(Bt);
         if (start_marg) start_marg[((size_t)b * (d.T + 1) + s) * C + c] = St;
       }
-      St = __shfl_sync(FULL_MASK, St, (threadIdx.x & 31) & ~(d.GB - 1));
-      if (act && kf.sum > 0.f) {
-        const float coef = gbf * St / kf.sum;
+      warp_max_to_shared(&sm.maxslot[q], key);
+      const float Stg = __shfl_sync(FULL_MASK, St, (tid & 31) & ~(d.GB - 1));
+      if (kb.act && kf.sum > 0.f) {
+        const float coef = gbf * Stg / kf.sum;
 #pragma unroll
-        for (int i = 0; i < KB_MAX; ++i)
-          if (i < d.KB) accd[i] += coef * e[i];
+        for (int i = 0; i < KBT; ++i) accd[i] += coef * e[i];
       }
     }
     __syncthreads();
     bool slow;
-    const float n = step_frame(sm, par, slow);
-    if (tid == 0) sm.maxslot[par ^ 1] = f2ord(NEG_INF);
+    const float n = step_frame(sm, q, slow);
+    float E = 0.f;
     if (s >= 1) {
       float shift = n;
       if (slow) {
-        for (int c = tid; c < C; c += blockDim.x) sm.pcur[c] = ex2(sm.Acur[c] - n);
-        __syncthreads();
+        refresh_p(sm, d, par, n);
         shift = 0.f;
       }
-      if (r.warpA) {
-        const bool act = r.cA < C;
-        const int c = act ? r.cA : 0;
-        const float acc = label_fanin(sm, d, r, ereg, prod);
-        float E = 0.f;
-        if (act && r.jA == 0) {
-          float g;
-          if (acc >= UNDERFLOW && acc <= 3.0e38f)
-            g = lg2(acc) + tmax2 - shift;
-          else
-            g = label_lse_slow(d, sm.Acur, n, trans, c, true);
-          sm.ring[sb * C + c] = make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - Sb[c]));
-          // end marginal E[s, c] = 2^(alpha[s,c] + beta[s,c] - log2 Z)
+      if (warp_on) {
+        const float g = aphase<CAT>(sm, d, ab, par, n, shift, trans, true, acc, prod);
+        if (leader) {
+          const int c = ab.c;
+          ring_put<KBT>(sm, d, c, slot,
+                        make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - sm.Sbase[c])));
           const float Ys = (float)(Xc + (double)row[2 * C] + (double)(Grel + n));
           E = (g == NEG_INF || row[c] == NEG_INF) ? 0.f : ex2(row[c] + g + Ys);
-          sm.stE[par * C + c] = E;
           if (end_marg) end_marg[((size_t)b * (d.T + 1) + s) * C + c] = E;
         }
-        E = __shfl_sync(FULL_MASK, E, (threadIdx.x & 31) & ~(d.GA - 1));
-        if (act && acc > 0.f) {
-          const float coef = gbf * E / acc;
+        const float Eg = __shfl_sync(FULL_MASK, E, (tid & 31) & ~(d.GB - 1));
+        if (ab.act && acc > 0.f) {
+          const float coef = gbf * Eg / acc;
 #pragma unroll
-          for (int i = 0; i < CA_MAX; ++i)
-            if (i < d.CA) acct[i] += coef * prod[i];
+          for (int i = 0; i < CAT; ++i) acct[i] += coef * prod[i];
         }
+        __syncwarp();
       }
-    } else {
-      for (int c = tid; c < C; c += blockDim.x) {
-        sm.stE[par * C + c] = 0.f;
-        if (end_marg) end_marg[((size_t)b * (d.T + 1)) * C + c] = 0.f;
-      }
+    } else if (leader && end_marg) {
+      end_marg[((size_t)b * (d.T + 1)) * C + kb.c] = 0.f;
+    }
+    if (leader) {
+      // position s: v = sum of (start - end) marginals strictly after it in the segment
+      const float v = (float)accmu;
+      grad_em[((size_t)b * d.T + s) * C + kb.c] = v;
+      vsum += (double)v;
+      accmu += (double)St - (double)E;
     }
     Grel += n;
     if (++nflush == FLUSH_EVERY || s == t0) {
       nflush = 0;
-      if (r.cB < C) {
+      if (kb.act) {
 #pragma unroll
-        for (int i = 0; i < KB_MAX; ++i) {
-          const int k = 1 + r.jB + i * d.GB;
-          if (i < d.KB && k <= K) {
-            ws.pgd[(seg * K + (k - 1)) * C + r.cB] += (double)accd[i];
-            accd[i] = 0.f;
-          }
+        for (int i = 0; i < KBT; ++i) {
+          const int k = kb.k_of(i, false);
+          if (k <= K) ws.pgd[(seg * K + (k - 1)) * C + kb.c] += (double)accd[i];
+          accd[i] = 0.f;
         }
       }
-      if (r.cA < C) {
+      if (ab.act) {
 #pragma unroll
-        for (int i = 0; i < CA_MAX; ++i) {
-          const int x = r.jA + i * d.GA;
-          if (i < d.CA && x < C) {
-            ws.pgt[(seg * C + r.cA) * C + x] += (double)acct[i];
-            acct[i] = 0.f;
-          }
+        for (int i = 0; i < CAT; ++i) {
+          const int x = ab.j * CAT + i;
+          if (x < C) ws.pgt[(seg * C + ab.c) * C + x] += (double)acct[i];
+          acct[i] = 0.f;
         }
       }
     }
-    __syncthreads();
   }
-  if (tid < C) {
-    const int par = t0 & 1;
-    const float v = (float)accmu;
-    grad_em[((size_t)b * d.T + t0) * C + tid] = v;
-    vsum += (double)v;
-    accmu += (double)sm.stS[par * C + tid] - (double)sm.stE[par * C + tid];
-    ws.segT[seg * C + tid] = accmu;
-    ws.segV[seg * C + tid] = vsum;
+  if (leader) {
+    ws.segT[seg * C + kb.c] = accmu;
+    ws.segV[seg * C + kb.c] = vsum;
   }
 }
 
@@ -870,6 +594,58 @@ __global__ void selftest_wait_kernel(int* status, int spins) {
   const bool ok = mbar_wait(&bar, 0, spins);
   if (!__syncthreads_or(!ok)) return;
   if (threadIdx.x == 0) set_status(status, ST_DEVICE_TIMEOUT);
+}
+
+// ----------------------------------------------------------------------------- launchers
+bool shape_supported(int KBT, int CAT) {
+#define SEMICRF_SHAPE_OK(a, b) \
+  if (KBT == a && CAT == b) return true;
+  SEMICRF_FOR_EACH_SHAPE(SEMICRF_SHAPE_OK)
+#undef SEMICRF_SHAPE_OK
+  return false;
+}
+
+namespace {
+template <typename F>
+cudaError_t allow_smem(F fn, size_t sm) {
+  if (sm <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+}
+}  // namespace
+
+cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths, const float* trans,
+                         const float* dur, double* logZ_out, int n_alpha, int n_beta,
+                         cudaStream_t st) {
+  const size_t sm = recursion_smem_bytes(d, false);
+#define SEMICRF_LAUNCH_CHAIN(a, b)                                                          \
+  if (d.KBT == a && d.CAT == b) {                                                           \
+    const cudaError_t e = allow_smem(chain_kernel<a, b>, sm);                               \
+    if (e != cudaSuccess) return e;                                                         \
+    chain_kernel<a, b><<<n_alpha + n_beta, d.NT, sm, st>>>(d, ws, lengths, trans, dur, logZ_out, \
+                                                           n_alpha);                        \
+    return cudaGetLastError();                                                              \
+  }
+  SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_CHAIN)
+#undef SEMICRF_LAUNCH_CHAIN
+  return cudaErrorInvalidConfiguration;
+}
+
+cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                           const float* trans, const float* dur, const double* grad_logZ,
+                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st) {
+  const size_t sm = recursion_smem_bytes(d, d.store_smem != 0);
+#define SEMICRF_LAUNCH_SEG(a, b)                                                         \
+  if (d.KBT == a && d.CAT == b) {                                                        \
+    const cudaError_t e = allow_smem(segment_kernel<a, b>, sm);                          \
+    if (e != cudaSuccess) return e;                                                      \
+    segment_kernel<a, b><<<dim3(d.nck, d.B), d.NT, sm, st>>>(d, ws, lengths, trans, dur,   \
+                                                             grad_logZ, grad_em, start_marg, \
+                                                             end_marg);                    \
+    return cudaGetLastError();                                                           \
+  }
+  SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_SEG)
+#undef SEMICRF_LAUNCH_SEG
+  return cudaErrorInvalidConfiguration;
 }
 
 }  // namespace semicrf

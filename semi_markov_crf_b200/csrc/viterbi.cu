@@ -3,48 +3,20 @@
 // The forward recursion of recursion.cu with max in place of log-sum-exp:
 //   G[s, c] = max_{c'} V[s, c'] + trans[c', c]             (G[0, c] = 0)
 //   V[t, c] = max_{k <= min(K,t)} G[t-k, c] + S[t,c] - S[t-k,c] + dur[k-1,c]
-// with the same exact integer frames, base-2 units and K-slot ring.  Ties go
-// to the smallest k and then the smallest c' (first maximum in ascending
-// order within a lane, then the smaller index across lanes), and at the end to
-// the smallest final label.  Backpointers are packed per (boundary, label):
-// bits 0-15 the best duration of a segment ending there, bits 16-31 the best
-// previous label of a segment starting there.  One warp then walks them back
-// from the best final label.
-#include "kernels.cuh"
+// on the same mirrored K-slot ring, exact integer frames, base-2 units and
+// one-barrier-per-step schedule.  Ties go to the smallest k and then the
+// smallest c' (first maximum in ascending order within a lane, then the
+// smaller index across lanes), and at the end to the smallest final label.
+// Backpointers are packed per (boundary, label): bits 0-15 the best duration
+// of a segment ending there, bits 16-31 the best previous label of a segment
+// starting there.  One warp then walks them back from the best final label.
+#include "ring.cuh"
 
 namespace semicrf {
 
+using namespace ring;
+
 namespace {
-
-struct VSmem {
-  uint64_t* mbar;
-  int* maxslot;
-  int32_t* tint;
-  float* tfrac;
-  float2* ring;
-  float* Vcur;
-  int* kbest;
-  int* Sbase;
-};
-
-__device__ VSmem vcarve(unsigned char* raw, const Dims& d) {
-  VSmem s;
-  const int C = d.C;
-  unsigned char* p = raw;
-  s.mbar = reinterpret_cast<uint64_t*>(p);
-  s.maxslot = reinterpret_cast<int*>(p + 16);
-  p += 64;
-  s.tint = reinterpret_cast<int32_t*>(p);
-  p += 2ull * TS * C * sizeof(int32_t);
-  s.tfrac = reinterpret_cast<float*>(p);
-  p += 2ull * TS * C * sizeof(float);
-  s.ring = reinterpret_cast<float2*>(p);
-  p += (size_t)d.K * C * sizeof(float2);
-  s.Vcur = reinterpret_cast<float*>(p);
-  s.kbest = reinterpret_cast<int*>(s.Vcur + C);
-  s.Sbase = s.kbest + C;
-  return s;
-}
 
 // (value, index) max with ties to the smaller index, over aligned groups.
 __device__ __forceinline__ void group_argmax(float& v, int& i, int G) {
@@ -60,114 +32,79 @@ __device__ __forceinline__ void group_argmax(float& v, int& i, int G) {
 
 }  // namespace
 
+template <int KBT, int CAT>
 __global__ void __launch_bounds__(NT_MAX, 1)
     viterbi_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                    const float* __restrict__ trans, const float* __restrict__ dur,
                    double* __restrict__ score, int32_t* __restrict__ labels,
                    uint8_t* __restrict__ seg_start) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const VSmem sm = vcarve(smem_raw, d);
+  const Smem sm = carve(smem_raw, d, false);
   const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x;
   const int b = blockIdx.x;
-  int L = lengths[b];
+  const int L = lengths[b];
   const bool bad = (L < 0 || L > T);
   // positions past the length (all of them for a bad length)
   for (int u = (bad ? 0 : L) + tid; u < T; u += blockDim.x) {
     labels[(size_t)b * T + u] = -1;
     seg_start[(size_t)b * T + u] = 0;
   }
-  if (bad) {
+  if (bad || L == 0) {
     if (tid == 0) {
-      set_status(ws.status, ST_BAD_LENGTH);
-      score[b] = __longlong_as_double(0x7ff8000000000000ll);
+      if (bad) set_status(ws.status, ST_BAD_LENGTH);
+      score[b] = bad ? __longlong_as_double(0x7ff8000000000000ll) : 0.0;
     }
     return;
   }
-  if (L == 0) {
-    if (tid == 0) score[b] = 0.0;
-    return;
-  }
-  const int GB = d.GB, GA = d.GA;
-  const int cB = tid / GB, jB = tid % GB, cA = tid / GA, jA = tid % GA;
-  const bool warpB = ((tid & ~31) / GB) < C, warpA = ((tid & ~31) / GA) < C;
-  const float l2e = (float)LOG2E_D;
-  float dreg[KB_MAX], treg[CA_MAX];
-  {
-    const int c = cB < C ? cB : 0;
+  const bool warp_on = ((tid & ~31) / d.GB) < C;
+  KLane<KBT> kl;
+  kl.init(d, dur, true);
+  // raw trans2 column values for this lane's previous labels (no exponentials)
+  float tr[CAT];
 #pragma unroll
-    for (int i = 0; i < KB_MAX; ++i) {
-      const int k = 1 + jB + i * GB;
-      dreg[i] = (i < d.KB && k <= K) ? __ldg(dur + (size_t)(k - 1) * C + c) * l2e : NEG_INF;
-    }
-    const int o = cA < C ? cA : 0;
-#pragma unroll
-    for (int i = 0; i < CA_MAX; ++i) {
-      const int x = jA + i * GA;
-      treg[i] = (i < d.CA && x < C) ? __ldg(trans + (size_t)x * C + o) * l2e : NEG_INF;
-    }
+  for (int i = 0; i < CAT; ++i) {
+    const int x = kl.j * CAT + i;
+    tr[i] = (kl.act && x < C) ? __ldg(trans + (size_t)x * C + kl.c) * l2e() : NEG_INF;
   }
-  if (tid == 0) {
-    mbar_init(&sm.mbar[0], 1);
-    mbar_init(&sm.mbar[1], 1);
-    fence_mbar_init();
-    sm.maxslot[0] = f2ord(NEG_INF);
-    sm.maxslot[1] = f2ord(NEG_INF);
-  }
+  init_smem(sm, d);
+  __syncthreads();
   for (int c = tid; c < C; c += blockDim.x) {
-    sm.ring[c] = make_float2(0.f, 0.f);
+    ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));
     sm.Sbase[c] = 0;
   }
   __syncthreads();
   int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
-  // tile stream (same protocol as the recursion kernels)
-  const int lo = 0, hi = L / TS;
-  uint32_t ph[2] = {0u, 0u};
-  int cur = -1;
-  auto issue = [&](int i) {
-    if (i < lo || i > hi || tid != 0) return;
-    const int buf = i & 1;
-    const uint32_t bytes = (uint32_t)(TS * C * 4);
-    const size_t row0 = (size_t)b * d.Tstride + (size_t)i * TS;
-    fence_proxy_async();
-    mbar_expect_tx(&sm.mbar[buf], 2 * bytes);
-    bulk_g2s(sm.tint + (size_t)buf * TS * C, ws.sint + row0 * C, bytes, &sm.mbar[buf]);
-    bulk_g2s(sm.tfrac + (size_t)buf * TS * C, ws.sfrac + row0 * C, bytes, &sm.mbar[buf]);
-  };
-  issue(0);  // entering a tile issues the next one
+  TileStream ts;
+  ts.ph[0] = ts.ph[1] = 0;
+  const int32_t* ri;
+  const float* rf;
+  tile_start(sm, d, ws, b, ts, 1, 0, L, +1);
   double F0 = 0.0;
   float Frel = 0.f;
-  int tb = 0;
+  int slot = 0, par = 0, q = 0;
+  int base = kl.base_up(1, K);
+  int to_ck = d.delta;
+  int bk = 0;
   for (int t = 1; t <= L; ++t) {
-    tb = (tb + 1 == K) ? 0 : tb + 1;
-    const int ti = t / TS;
-    if (ti != cur) {
-      const int buf = ti & 1;
-      bool ok = mbar_wait(&sm.mbar[buf], ph[buf], WAIT_SPIN_LIMIT);
-      ph[buf] ^= 1u;
-      cur = ti;
-      issue(ti + 1);
-      if (__syncthreads_or(!ok)) {
-        if (tid == 0) {
-          set_status(ws.status, ST_DEVICE_TIMEOUT);
-          for (int q = 0; q < 2; ++q) mbar_wait(&sm.mbar[q], ph[q], WAIT_SPIN_LIMIT);
-        }
-        return;
-      }
+    if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
+    slot = (slot + 1 == K) ? 0 : slot + 1;
+    par = t & 1;
+    q = mod3_next(q);
+    if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
+      if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+      tile_drain(sm, ts);
+      return;
     }
-    const size_t ro = ((size_t)(ti & 1) * TS + (t - ti * TS)) * C;
-    const int32_t* ri = sm.tint + ro;
-    const float* rf = sm.tfrac + ro;
-    if (t % d.delta == 0) {
+    if (--to_ck == 0) {
       // rebase the integer frames (keeps every stored integer small)
+      to_ck = d.delta;
+      __syncthreads();
       const float dF = Frel;
-      for (int idx = tid; idx < K * C; idx += blockDim.x) {
-        const int i = idx / C, c = idx % C;
-        if (t - K + i < 0) continue;
-        int slot = tb + i;
-        if (slot >= K) slot -= K;
-        float2 v = sm.ring[slot * C + c];
+      for (int idx = tid; idx < C * d.RL; idx += blockDim.x) {
+        const int c = idx / d.RL;
+        float2 v = sm.ring[idx];
         v.y = (v.y - dF) + (float)(ri[c] - sm.Sbase[c]);
-        sm.ring[slot * C + c] = v;
+        sm.ring[idx] = v;
       }
       __syncthreads();
       for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
@@ -175,73 +112,69 @@ __global__ void __launch_bounds__(NT_MAX, 1)
       Frel = 0.f;
       __syncthreads();
     }
-    const int par = t & 1;
-    if (warpB) {
-      const bool act = cB < C;
-      const int c = act ? cB : 0;
+    if (warp_on) {
+      const int c = kl.act ? kl.c : 0;
       const float Q = (float)(ri[c] - sm.Sbase[c]) - Frel;
-      const int kmax = min(K, t);
+      const float2* r = sm.ring + (size_t)c * d.RL + base;
+      // lane term i has k = (j+1)*KBT - i: walk i downwards for ascending k
       float best = NEG_INF;
-      int bk = 0x7fffffff;
+      bk = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < KB_MAX; ++i) {
-        const int k = 1 + jB + i * GB;
-        if (i < d.KB && act && k <= kmax) {
-          int slot = tb - k;
-          if (slot < 0) slot += K;
-          const float2 v = sm.ring[slot * C + c];
-          const float y = ((v.y + Q) + v.x) + dreg[i];
-          if (y > best || bk == 0x7fffffff) {
-            best = y;
-            bk = k;
-          }
+      for (int i = KBT - 1; i >= 0; --i) {
+        const float2 v = r[i];
+        const float y = ((v.y + Q) + v.x) + kl.d[i];
+        if (y > best || bk == 0x7fffffff) {
+          best = y;
+          bk = kl.k_of(i, true);
         }
       }
-      group_argmax(best, bk, GB);
-      if (act && jB == 0) {
+      group_argmax(best, bk, d.GB);
+      int key = INT_MIN;
+      if (kl.act && kl.j == 0) {
         const float V = rf[c] + best;
-        sm.Vcur[c] = V;
-        sm.kbest[c] = bk;
-        atomicMax(&sm.maxslot[par], f2ord(V));
+        sm.Acur[par * C + c] = V;
+        key = f2ord(V);
       }
+      warp_max_to_shared(&sm.maxslot[q], key);
     }
     __syncthreads();
-    const float M = ord2f(sm.maxslot[par]);
-    const float n = isfinite(M) ? rintf(M) : 0.f;
-    if (tid == 0) sm.maxslot[par ^ 1] = f2ord(NEG_INF);
+    bool slow;
+    const float n = step_frame(sm, q, slow);
     if (t == L) break;
-    if (warpA) {
-      const bool act = cA < C;
+    if (warp_on) {
+      const float* V = sm.Acur + par * C;
       float best = NEG_INF;
       int bc = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < CA_MAX; ++i) {
-        const int x = jA + i * GA;
-        if (i < d.CA && act && x < C) {
-          const float v = sm.Vcur[x] + treg[i];
-          if (v > best || bc == 0x7fffffff) {
-            best = v;
-            bc = x;
-          }
+      for (int i = 0; i < CAT; ++i) {
+        const int x = kl.j * CAT + i;
+        const float vx = (x < C) ? V[x] + tr[i] : NEG_INF;
+        if (vx > best || bc == 0x7fffffff) {
+          best = vx;
+          bc = x;
         }
       }
-      group_argmax(best, bc, GA);
-      if (act && jA == 0) {
-        const int c = cA;
+      group_argmax(best, bc, d.GB);
+      if (kl.act && kl.j == 0) {
+        const int c = kl.c;
         const float g = best - n;
-        sm.ring[tb * C + c] = make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c]));
-        bp[(size_t)t * C + c] = (sm.kbest[c] & 0xffff) | (bc << 16);
+        ring_put<KBT>(sm, d, c, slot,
+                      make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
+        bp[(size_t)t * C + c] = (bk & 0xffff) | (bc << 16);
       }
+      __syncwarp();
     }
     Frel += n;
-    __syncthreads();
   }
-  // best final label (smallest on ties), score, then the traceback
+  // the last step's best durations, then the best final label (smallest on ties)
+  if (kl.act && kl.j == 0) bp[(size_t)L * C + kl.c] = bk & 0xffff;
+  __syncthreads();
   if (tid < 32) {
+    const float* V = sm.Acur + par * C;
     float best = NEG_INF;
     int bc = 0x7fffffff;
     for (int c = tid; c < C; c += 32) {
-      const float v = sm.Vcur[c];
+      const float v = V[c];
       if (v > best || bc == 0x7fffffff) {
         best = v;
         bc = c;
@@ -250,9 +183,8 @@ __global__ void __launch_bounds__(NT_MAX, 1)
     group_argmax(best, bc, 32);
     if (tid == 0) score[b] = (F0 + (double)Frel + (double)best) * LN2_D;
     int t = L, c = bc;
-    int kL = sm.kbest[bc];
     while (t > 0) {
-      const int k = (t == L) ? kL : (bp[(size_t)t * C + c] & 0xffff);
+      const int k = bp[(size_t)t * C + c] & 0xffff;
       const int s = t - k;
       for (int u = s + tid; u < t; u += 32) {
         labels[(size_t)b * T + u] = c;
@@ -262,6 +194,27 @@ __global__ void __launch_bounds__(NT_MAX, 1)
       t = s;
     }
   }
+}
+
+cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                           const float* trans, const float* dur, double* score, int32_t* labels,
+                           uint8_t* seg_start, cudaStream_t st) {
+  const size_t sm = recursion_smem_bytes(d, false);
+#define SEMICRF_LAUNCH_VIT(a, b)                                                               \
+  if (d.KBT == a && d.CAT == b) {                                                              \
+    if (sm > 48 * 1024) {                                                                      \
+      const cudaError_t e = cudaFuncSetAttribute(viterbi_kernel<a, b>,                         \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                                 (int)sm);                                     \
+      if (e != cudaSuccess) return e;                                                          \
+    }                                                                                          \
+    viterbi_kernel<a, b><<<d.B, d.NT, sm, st>>>(d, ws, lengths, trans, dur, score, labels,     \
+                                                seg_start);                                    \
+    return cudaGetLastError();                                                                 \
+  }
+  SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_VIT)
+#undef SEMICRF_LAUNCH_VIT
+  return cudaErrorInvalidConfiguration;
 }
 
 }  // namespace semicrf

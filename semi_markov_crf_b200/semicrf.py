@@ -15,7 +15,12 @@ import torch
 
 __all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
-           "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "lib"]
+           "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "profile_enable", "profile_read",
+           "KERNELS", "lib"]
+
+# every kernel the library launches (names used by the profiler)
+KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_kernel", "segment_kernel",
+           "finalize_positions_kernel", "reduce_partials_kernel", "viterbi_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2
@@ -42,7 +47,9 @@ lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
 lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
-for _f in ("semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+lib.semicrf_profile_enable.argtypes = [_i]
+lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
+for _f in ("semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_get_status",
            "semicrf_selftest_bounded_wait"):
     getattr(lib, _f).restype = _i
@@ -215,3 +222,17 @@ def selftest_bounded_wait(ws: Workspace, spins: int) -> int:
     _check(lib.semicrf_selftest_bounded_wait(ws.ptr, ws.nbytes, int(spins), _stream(ws.buf.device)),
            "semicrf_selftest_bounded_wait")
     return get_status(ws)
+
+
+def profile_enable(on: bool = True):
+    """Start (clearing) or stop per-kernel CUDA-event timing inside the library."""
+    _check(lib.semicrf_profile_enable(1 if on else 0), "semicrf_profile_enable")
+
+
+def profile_read(kernel: str):
+    """(total device ms, launches) recorded for `kernel` since profile_enable(True)."""
+    ms = ctypes.c_double(0.0)
+    n = _i(0)
+    _check(lib.semicrf_profile_read(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)),
+           "semicrf_profile_read")
+    return float(ms.value), int(n.value)

@@ -2,6 +2,7 @@
 // launch geometry, workspace layout and kernel launches.  Host code only.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -22,11 +23,6 @@ int pow2floor(int x) {
   return p;
 }
 
-int pow2ceil(int x) {
-  int p = 1;
-  while (p < x) p *= 2;
-  return p;
-}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -66,33 +62,45 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
-  // lanes per label are a power of two <= 32 with at most NT_MAX threads in all
-  const int gmax = std::min(32, pow2floor(NT_MAX / C));
-  // fewest durations per lane that fit: KBT in {2, 4, 8, 16}
+  // Kernel shape: G lanes per label (a power of two), each with KBT durations
+  // and CAT labels, picked from the instantiated menu by a latency model.
+  // Per step about one warp runs per scheduler and the step is latency
+  // bound: the model charges the warps sharing a scheduler, the sequential
+  // k fan-in terms of a lane, its shuffle levels and its label terms (weights
+  // fitted to measured step times on B200).
+  // SEMICRF_LANES=G restricts the choice to that G (tuning; ignored if no
+  // shape with that G fits).
+  int forced = 0;
+  if (const char* env = std::getenv("SEMICRF_LANES")) forced = std::atoi(env);
   d.KBT = 0;
-  for (int kb : {2, 4, 8, 16}) {
-    if ((K + kb - 1) / kb <= gmax) {
-      d.KBT = kb;
-      break;
-    }
+  double best = 1e30;
+  for (int pass = 0; pass < 2 && d.KBT == 0; ++pass) {
+#define SEMICRF_CONSIDER(a, b, g, lb)                                                   \
+  {                                                                                     \
+    const int nt = std::max(32, ((C * g + 31) / 32) * 32);                              \
+    const bool fits = (K <= a * g) && (C <= b * g) && (nt <= lb) && (lb == 512 || nt <= 256); \
+    if (fits && (pass == 1 || forced <= 0 || forced == g)) {                            \
+      int lg = 0;                                                                       \
+      while ((1 << lg) < g) ++lg;                                                       \
+      const int warps = nt / 32;                                                        \
+      const double cost = ((warps + 3) / 4) * 60.0 + 12.0 * a + 6.0 * lg + 1.25 * b;   \
+      if (cost < best) {                                                                \
+        best = cost;                                                                    \
+        d.KBT = a;                                                                      \
+        d.CAT = b;                                                                      \
+        d.GB = g;                                                                       \
+        d.LB = lb;                                                                      \
+        d.NT = nt;                                                                      \
+      }                                                                                 \
+    }                                                                                   \
+  }
+    SEMICRF_FOR_EACH_SHAPE(SEMICRF_CONSIDER)
+#undef SEMICRF_CONSIDER
   }
   if (d.KBT == 0) return SEMICRF_ERR_UNSUPPORTED;
-  // lanes per group: enough for the durations, and for the labels (<= 32 per lane)
-  d.GB = std::max(pow2ceil((K + d.KBT - 1) / d.KBT), pow2ceil((C + 31) / 32));
-  // the label fan-in uses the same groups: CAT >= ceil(C / GB) in {1, 2, 4, 8, 32}
-  d.CAT = 0;
-  for (int ca : {1, 2, 4, 8, 32}) {
-    if (ca * d.GB >= C) {
-      d.CAT = ca;
-      break;
-    }
-  }
-  if (d.CAT == 0 || !shape_supported(d.KBT, d.CAT)) return SEMICRF_ERR_UNSUPPORTED;
   d.GA = d.GB;
   d.RL = K + d.KBT;
   d.PC = ((std::max(C, d.GB * d.CAT) + 3) / 4) * 4;
-  d.NT = std::max(32, ((C * d.GB + 31) / 32) * 32);
-  if (d.NT > NT_MAX) return SEMICRF_ERR_UNSUPPORTED;
   d.prefR = std::max(16, pow2floor(8192 / C));
   d.nchunk = T > 0 ? (T + d.prefR - 1) / d.prefR : 1;
   d.store_w = 2 * C + 2;

@@ -43,7 +43,7 @@ __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restr
 __global__ void selftest_wait_kernel(int* status, int spins);
 
 // Lane shapes with a compiled instantiation (KBT durations, CAT labels per lane).
-bool shape_supported(int KBT, int CAT);
+bool shape_supported(int KBT, int CAT, int G, int LB);
 
 // Host launchers for the shape in `d` (return the cudaError_t of the launch).
 // Forward ring of sequences [0, n_alpha) and backward ring of the rest:
@@ -59,9 +59,15 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
                            const float* trans, const float* dur, double* score, int32_t* labels,
                            uint8_t* seg_start, cudaStream_t st);
 
-// Every lane shape the library instantiates.
-#define SEMICRF_FOR_EACH_SHAPE(X)                                                      \
-  X(2, 1) X(2, 2) X(2, 4) X(2, 8) X(2, 32) X(4, 1) X(4, 2) X(4, 4) X(4, 8) X(4, 32)    \
-  X(8, 1) X(8, 2) X(8, 4) X(8, 8) X(8, 32) X(16, 1) X(16, 2) X(16, 4) X(16, 8) X(16, 32)
+// Every kernel shape the library instantiates: (durations per lane KBT,
+// labels per lane CAT, lanes per label G, launch bound LB).  The (16, 32, G,
+// 512) family alone covers every supported size; the others are tuned for
+// smaller problems (fewer wasted terms, fewer registers).
+#define SEMICRF_FOR_EACH_SHAPE(X)                                                        \
+  X(4, 4, 1, 256) X(8, 4, 1, 256) X(4, 8, 1, 256) X(8, 8, 1, 256) X(16, 8, 1, 256)       \
+  X(16, 32, 1, 256) X(4, 4, 2, 256) X(8, 8, 2, 256) X(16, 32, 2, 256) X(4, 8, 4, 256)    \
+  X(8, 16, 4, 256) X(16, 32, 4, 512) X(4, 8, 8, 512) X(8, 4, 8, 256) X(8, 8, 8, 512)     \
+  X(16, 8, 8, 512) X(16, 32, 8, 512) X(8, 1, 16, 256) X(16, 1, 16, 256) X(16, 4, 16, 512) \
+  X(16, 32, 16, 512) X(8, 1, 32, 256) X(16, 1, 32, 512) X(16, 32, 32, 512)
 
 }  // namespace semicrf

@@ -31,6 +31,7 @@ struct Dims {
   int RL;        // ring entries per label: K + KBT (the first KBT slots are mirrored)
   int PC;        // padded length of the exp-domain label vector (>= GA * CAT)
   int NT;        // threads per CTA of the recursion kernels
+  int LB;        // launch bound of the instantiation (256 or 512 threads)
   int prefR;     // rows per prefix-sum chunk
   int nchunk;    // prefix-sum chunks per sequence
   int store_w;   // floats per position in the segment recompute store (2C + 2)

@@ -39,51 +39,6 @@ using namespace ring;
 
 namespace {
 
-// Forward k fan-in at boundary t: A = alpha[t,c] - F_{t-1}; the leader writes
-// Acur/pcur (buffer `par`) and every warp adds to the step max (slot q).
-template <int KBT>
-__device__ __forceinline__ float fwd_kphase(const Smem& sm, const Dims& d, const KLane<KBT>& kl,
-                                            int base, const int32_t* ri, const float* rf,
-                                            float Frel, int par, int q, float (&e)[KBT]) {
-  const int c = kl.act ? kl.c : 0;
-  const float Q = (float)(ri[c] - sm.Sbase[c]) - Frel;
-  const KFan kf = k_fanin<KBT>(sm, d, kl, base, Q, e);
-  const float A = (kf.lse == NEG_INF) ? NEG_INF : rf[c] + kf.lse;
-  int key = INT_MIN;
-  if (kl.act && kl.j == 0) {
-    sm.Acur[par * d.C + c] = A;
-    sm.pcur[par * d.PC + c] = ex2(A);
-    key = f2ord(A);
-  }
-  warp_max_to_shared(&sm.maxslot[q], key);
-  return A;
-}
-
-// Label fan-in for output label al.c; returns the log2 sum minus the shift
-// (gamma - F_t for the forward side, beta - G_s for the backward side) in
-// the leader lane, with the log-domain fallback when the sum underflows.
-template <int CAT>
-__device__ __forceinline__ float aphase(const Smem& sm, const Dims& d, const ALane<CAT>& al, int par,
-                                        float n, float shift, const float* trans, bool rows,
-                                        float& acc, float (&prod)[CAT]) {
-  acc = label_fanin<CAT>(sm.pcur + par * d.PC, d, al, prod);
-  float g = 0.f;
-  if (al.act && al.j == 0) {
-    if (acc >= UNDERFLOW && acc <= 3.0e38f)
-      g = lg2(acc) + al.tmax - shift;
-    else
-      g = label_lse_slow(d, sm.Acur + par * d.C, n, trans, al.c, rows);
-  }
-  return g;
-}
-
-// Uniform slow path: the step's frame jump is too large for 2^A in float32.
-__device__ __forceinline__ void refresh_p(const Smem& sm, const Dims& d, int par, float n) {
-  for (int c = threadIdx.x; c < d.C; c += blockDim.x)
-    sm.pcur[par * d.PC + c] = ex2(sm.Acur[par * d.C + c] - n);
-  __syncthreads();
-}
-
 __device__ __forceinline__ void final_lse(const float* A, int C, double base, double* out2,
                                           double* out_nat) {
   if (threadIdx.x >= 32) return;
@@ -101,19 +56,62 @@ __device__ __forceinline__ void final_lse(const float* A, int C, double base, do
   }
 }
 
+// Forward checkpoint at boundary t (start of step t): rebase every ring entry
+// to the frame (F0 + Frel, S_int[t]) and save the K boundaries before t.
+__device__ __forceinline__ void fwd_checkpoint(const Smem& sm, const Dims& d, const WsPtrs& ws,
+                                               int b, int t, const int32_t* ri, float Frel) {
+  const int C = d.C, K = d.K;
+  const int j = t / d.delta;
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < C * d.RL; idx += blockDim.x) {
+    const int c = idx / d.RL;
+    float2 v = sm.ring[idx];
+    v.y = (v.y - Frel) + (float)(ri[c] - sm.Sbase[c]);
+    sm.ring[idx] = v;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < K * C; idx += blockDim.x) {
+    const int i = idx / C, c = idx % C;
+    if (t - K + i >= 0)
+      ws.ack[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t - K + i);
+  }
+  for (int c = threadIdx.x; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
+  __syncthreads();
+}
+
+// Backward checkpoint at boundary t1 (start of step t1 - 1): rebase to
+// (G0 + Grel, S_int[t1]) and save boundaries t1..t1+K-1.
+__device__ __forceinline__ void bwd_checkpoint(const Smem& sm, const Dims& d, const WsPtrs& ws,
+                                               int b, int t1, int L) {
+  const int C = d.C, K = d.K;
+  const int j = t1 / d.delta - 1;
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) sm.tmp[c] = ring_at(sm, d, c, t1).y;
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < C * d.RL; idx += blockDim.x) sm.ring[idx].y -= sm.tmp[idx / d.RL];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < K * C; idx += blockDim.x) {
+    const int i = idx / C, c = idx % C;
+    if (t1 + i <= L) ws.bck[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t1 + i);
+  }
+  for (int c = threadIdx.x; c < C; c += blockDim.x)
+    sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
+  __syncthreads();
+}
+
 }  // namespace
 
 // ===========================================================================
 // Forward and backward rings over whole sequences.
 // ===========================================================================
-template <int KBT, int CAT>
-__global__ void __launch_bounds__(NT_MAX, 1)
+template <int KBT, int CAT, int G, int LB>
+__global__ void __launch_bounds__(LB, 1)
     chain_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                  const float* __restrict__ trans, const float* __restrict__ dur,
                  double* __restrict__ logZ_out, int n_alpha) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const Smem sm = carve(smem_raw, d, false);
-  const int C = d.C, K = d.K, tid = threadIdx.x;
+  const int C = d.C, K = d.K, PC = d.PC, tid = threadIdx.x;
   const bool is_alpha = (int)blockIdx.x < n_alpha;
   const int b = is_alpha ? blockIdx.x : blockIdx.x - n_alpha;
   const int L = lengths[b];
@@ -130,173 +128,185 @@ __global__ void __launch_bounds__(NT_MAX, 1)
     }
     return;
   }
-  const bool warp_on = ((tid & ~31) / d.GB) < C;
-  KLane<KBT> kl;
-  kl.init(d, dur, is_alpha);
-  ALane<CAT> al;
-  al.init(d, trans, !is_alpha);
-  float e[KBT], prod[CAT], acc;
+  Lane<KBT, CAT, G> ln;
+  ln.init_ids(d);
+  ln.init_dur(d, dur, is_alpha);
+  ln.init_trans(d, trans, !is_alpha);
+  float2* const rl = sm.ring + (size_t)ln.cc * d.RL;  // this lane's label ring
+  float e[KBT], p[CAT];
   init_smem(sm, d);
   __syncthreads();
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
-  const int32_t* ri;
-  const float* rf;
   int par = 0, q = 0;
+  float mk = 0.f;  // shift of the k fan-in (predicted LSE)
 
   if (is_alpha) {
     // ---------------------------------------------------------------- forward
     for (int c = tid; c < C; c += blockDim.x) {
-      ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));  // boundary 0: gamma 0, frame 0, S 0
+      ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));  // boundary 0
       sm.Sbase[c] = 0;
     }
-    tile_start(sm, d, ws, b, ts, 1, 0, L, +1);
+    tile_start(sm, d, ws, b, ts, 1, 1, L, +1);
     double F0 = 0.0;
     float Frel = 0.f;
-    int slot = 0;                 // t mod K
-    int base = kl.base_up(1, K);  // window base at t = 1
+    int Sb = 0;                   // Sbase of this lane's label
+    int wslot = 0;                // t mod K
+    int base = ln.base_up(1, K);  // window base at t = 1
     int to_ck = d.delta;          // steps to the next checkpoint boundary
+    int cur = -1, t = 1;
     __syncthreads();
-    for (int t = 1; t <= L; ++t) {
-      if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
-      slot = (slot + 1 == K) ? 0 : slot + 1;
-      par = t & 1;
-      q = mod3_next(q);
-      if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
-        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-        tile_drain(sm, ts);
-        return;
-      }
-      if (--to_ck == 0) {
-        to_ck = d.delta;
-        if (t < L) {
-          // checkpoint j: rebase to (F0 + Frel, S_int[t]), save the ring in boundary order
-          __syncthreads();
-          const int j = t / d.delta;
-          const float dF = Frel;
-          for (int idx = tid; idx < C * d.RL; idx += blockDim.x) {
-            const int c = idx / d.RL;
-            float2 v = sm.ring[idx];
-            v.y = (v.y - dF) + (float)(ri[c] - sm.Sbase[c]);
-            sm.ring[idx] = v;
-          }
-          __syncthreads();
-          for (int idx = tid; idx < K * C; idx += blockDim.x) {
-            const int i = idx / C, c = idx % C;
-            if (t - K + i >= 0)
-              ws.ack[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t - K + i);
-          }
-          for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
-          F0 += (double)dF;
-          Frel = 0.f;
-          if (tid == 0) ws.acf[(size_t)b * d.nck + j] = F0;
-          __syncthreads();
+    for (;;) {
+      const int ti = t / TS;
+      if (ti != cur) {
+        if (!tile_enter(sm, d, ws, b, ts, ti)) {
+          if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+          tile_drain(sm, ts);
+          return;
         }
+        cur = ti;
       }
-      if (warp_on) fwd_kphase<KBT>(sm, d, kl, base, ri, rf, Frel, par, q, e);
-      __syncthreads();
-      bool slow;
-      const float n = step_frame(sm, q, slow);
-      if (t == L) break;
-      float shift = n;
-      if (slow) {
-        refresh_p(sm, d, par, n);
-        shift = 0.f;
-      }
-      if (warp_on) {
-        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, false, acc, prod);
-        if (al.act && al.j == 0) {
-          const int c = al.c;
-          ring_put<KBT>(sm, d, c, slot,
-                        make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
+      const int t_stop = min(L, ti * TS + TS - 1);
+      const size_t off = tile_row_off(t, C);
+      const int32_t* ri = sm.tint + off;
+      const float* rf = sm.tfrac + off;
+      bool done = false;
+      for (; t <= t_stop; ++t, ri += C, rf += C) {
+        if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
+        wslot = (wslot + 1 == K) ? 0 : wslot + 1;
+        par = t & 1;
+        q = mod3_next(q);
+        if (--to_ck == 0) {
+          to_ck = d.delta;
+          if (t < L) {
+            fwd_checkpoint(sm, d, ws, b, t, ri, Frel);
+            F0 += (double)Frel;
+            Frel = 0.f;
+            if (tid == 0) ws.acf[(size_t)b * d.nck + t / d.delta] = F0;
+            Sb = ri[ln.cc];
+          }
+        }
+        const int si = ri[ln.cc];
+        const float sf = rf[ln.cc];
+        float s;
+        const float lse =
+            k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e);
+        const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
+        if (ln.leader) {
+          sm.Acur[par * C + ln.c] = A;
+          sm.pcur[par * PC + ln.c] = ex2(A);
+        }
+        warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(A) : INT_MIN);
+        __syncthreads();
+        bool slow;
+        const float n = step_frame(sm, q, slow);
+        if (t == L) {
+          done = true;
+          break;
+        }
+        mk = next_shift(lse, n, mk);
+        float shift = n;
+        if (slow) {
+          refresh_p(sm, d, par, n);
+          shift = 0.f;
+        }
+        const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
+        if (ln.leader) {
+          const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
+          ring_put<KBT>(rl, d, wslot, make_float2(g - sf, (Frel + n) - (float)(si - Sb)));
         }
         __syncwarp();
+        Frel += n;
       }
-      Frel += n;
+      if (done) break;
     }
     final_lse(sm.Acur + par * C, C, F0 + (double)Frel, &ws.logz2[b], &logZ_out[b]);
   } else {
     // --------------------------------------------------------------- backward
     tile_start(sm, d, ws, b, ts, L, 0, L, -1);
-    if (!tile_row(sm, d, ws, b, ts, L, ri, rf)) {
+    int cur = L / TS;
+    if (!tile_enter(sm, d, ws, b, ts, cur)) {
       if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
       tile_drain(sm, ts);
       return;
     }
-    int slot = L % K;
-    for (int c = tid; c < C; c += blockDim.x) {
-      ring_put<KBT>(sm, d, c, slot, make_float2(rf[c], 0.f));  // beta[L] = 0, frame 0, base S_int[L]
-      sm.Sbase[c] = ri[c];
+    {
+      const size_t off = tile_row_off(L, C);
+      for (int c = tid; c < C; c += blockDim.x) {
+        // beta[L] = 0 in frame 0 with base S_int[L]
+        ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, L % K, make_float2(sm.tfrac[off + c], 0.f));
+        sm.Sbase[c] = sm.tint[off + c];
+      }
     }
+    __syncthreads();
+    int Sb = sm.Sbase[ln.cc];
     double G0 = 0.0;
     float Grel = 0.f;
-    int base = kl.base_down(L - 1, K);
+    int wslot = L % K;
+    int base = ln.base_down(L - 1, K);
     int to_ck = L % d.delta;  // (s + 1) mod delta
-    __syncthreads();
-    for (int s = L - 1; s >= 0; --s) {
-      if (s < L - 1) base = (base == 0) ? K - 1 : base - 1;
-      slot = (slot == 0) ? K - 1 : slot - 1;
-      par = s & 1;
-      q = mod3_next(q);
-      if (!tile_row(sm, d, ws, b, ts, s, ri, rf)) {
-        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-        tile_drain(sm, ts);
-        return;
-      }
-      if (to_ck == 0 && s + 1 < L) {
-        // checkpoint j: the ring holds boundaries t1..t1+K-1; rebase to (G0 + Grel, S_int[t1])
-        __syncthreads();
-        const int t1 = s + 1;
-        const int j = t1 / d.delta - 1;
-        for (int c = tid; c < C; c += blockDim.x) sm.tmp[c] = ring_at(sm, d, c, t1).y;
-        __syncthreads();
-        for (int idx = tid; idx < C * d.RL; idx += blockDim.x) sm.ring[idx].y -= sm.tmp[idx / d.RL];
-        __syncthreads();
-        for (int idx = tid; idx < K * C; idx += blockDim.x) {
-          const int i = idx / C, c = idx % C;
-          if (t1 + i <= L)
-            ws.bck[(((size_t)b * d.nck + j) * K + i) * C + c] = ring_at(sm, d, c, t1 + i);
+    int s = L - 1;
+    for (;;) {
+      const int ti = s / TS;
+      if (ti != cur) {
+        if (!tile_enter(sm, d, ws, b, ts, ti)) {
+          if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+          tile_drain(sm, ts);
+          return;
         }
-        for (int c = tid; c < C; c += blockDim.x)
-          sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
-        G0 += (double)Grel;
-        Grel = 0.f;
-        if (tid == 0) ws.bcf[(size_t)b * d.nck + j] = G0;
-        __syncthreads();
+        cur = ti;
       }
-      to_ck = (to_ck == 0) ? d.delta - 1 : to_ck - 1;
-      if (warp_on) {
-        const int c = kl.act ? kl.c : 0;
-        const float Q = -(float)(ri[c] - sm.Sbase[c]) - Grel;
-        const KFan kf = k_fanin<KBT>(sm, d, kl, base, Q, e);
-        const float Bt = (kf.lse == NEG_INF) ? NEG_INF : kf.lse - rf[c];
-        int key = INT_MIN;
-        if (kl.act && kl.j == 0) {
-          sm.Acur[par * C + c] = Bt;
-          sm.pcur[par * d.PC + c] = ex2(Bt);
-          key = f2ord(Bt);
+      const int s_stop = ti * TS;
+      const size_t off = tile_row_off(s, C);
+      const int32_t* ri = sm.tint + off;
+      const float* rf = sm.tfrac + off;
+      bool done = false;
+      for (; s >= s_stop; --s, ri -= C, rf -= C) {
+        if (s < L - 1) base = (base == 0) ? K - 1 : base - 1;
+        wslot = (wslot == 0) ? K - 1 : wslot - 1;
+        par = s & 1;
+        q = mod3_next(q);
+        if (to_ck == 0 && s + 1 < L) {
+          bwd_checkpoint(sm, d, ws, b, s + 1, L);
+          G0 += (double)Grel;
+          Grel = 0.f;
+          if (tid == 0) ws.bcf[(size_t)b * d.nck + (s + 1) / d.delta - 1] = G0;
+          Sb = sm.Sbase[ln.cc];
         }
-        warp_max_to_shared(&sm.maxslot[q], key);
-      }
-      __syncthreads();
-      bool slow;
-      const float n = step_frame(sm, q, slow);
-      if (s == 0) break;
-      float shift = n;
-      if (slow) {
-        refresh_p(sm, d, par, n);
-        shift = 0.f;
-      }
-      if (warp_on) {
-        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, true, acc, prod);
-        if (al.act && al.j == 0) {
-          const int c = al.c;
-          ring_put<KBT>(sm, d, c, slot,
-                        make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - sm.Sbase[c])));
+        to_ck = (to_ck == 0) ? d.delta - 1 : to_ck - 1;
+        const int si = ri[ln.cc];
+        const float sf = rf[ln.cc];
+        float ssum;
+        const float lse =
+            k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e);
+        const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
+        if (ln.leader) {
+          sm.Acur[par * C + ln.c] = Bt;
+          sm.pcur[par * PC + ln.c] = ex2(Bt);
+        }
+        warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(Bt) : INT_MIN);
+        __syncthreads();
+        bool slow;
+        const float n = step_frame(sm, q, slow);
+        if (s == 0) {
+          done = true;
+          break;
+        }
+        mk = next_shift(lse, n, mk);
+        float shift = n;
+        if (slow) {
+          refresh_p(sm, d, par, n);
+          shift = 0.f;
+        }
+        const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
+        if (ln.leader) {
+          const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, true);
+          ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
         }
         __syncwarp();
+        Grel += n;
       }
-      Grel += n;
+      if (done) break;
     }
     final_lse(sm.Acur + par * C, C, G0 + (double)Grel, &ws.logz2b[b], nullptr);
   }
@@ -313,15 +323,15 @@ __global__ void __launch_bounds__(NT_MAX, 1)
 //   P(c' -> c at s)        = end_marg[s,c'] * (normalised c term of beta)
 // The leader lane of label c's group keeps c's running sums.
 // ===========================================================================
-template <int KBT, int CAT>
-__global__ void __launch_bounds__(NT_MAX, 1)
+template <int KBT, int CAT, int G, int LB>
+__global__ void __launch_bounds__(LB, 1)
     segment_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                    const float* __restrict__ trans, const float* __restrict__ dur,
                    const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
                    float* __restrict__ start_marg, float* __restrict__ end_marg) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const Smem sm = carve(smem_raw, d, d.store_smem != 0);
-  const int C = d.C, K = d.K, tid = threadIdx.x;
+  const int C = d.C, K = d.K, PC = d.PC, tid = threadIdx.x;
   const int j = blockIdx.x, b = blockIdx.y;
   const int L = lengths[b];
   if (L < 0 || L > d.T) return;  // reported by the forward pass
@@ -334,29 +344,26 @@ __global__ void __launch_bounds__(NT_MAX, 1)
   const int SW = d.store_w;
   float* store = sm.store ? sm.store : ws.store + ((size_t)b * d.nck + j) * d.delta * SW;
   const size_t seg = (size_t)b * d.nck + j;
-  const bool warp_on = ((tid & ~31) / d.GB) < C;
-  float e[KBT], prod[CAT], acc;
+  Lane<KBT, CAT, G> ln;
+  ln.init_ids(d);
+  float2* const rl = sm.ring + (size_t)ln.cc * d.RL;
+  float e[KBT], p[CAT];
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
-  const int32_t* ri;
-  const float* rf;
   double F0 = 0.0;
   float Frel = 0.f;
   int par = 0, q = 0;
 
   // ------------------------------------------------------ alpha recompute
   {
-    KLane<KBT> kl;
-    kl.init(d, dur, true);
-    ALane<CAT> al;
-    al.init(d, trans, false);
+    ln.init_dur(d, dur, true);
+    ln.init_trans(d, trans, false);
     init_smem(sm, d);
     __syncthreads();
-    int t_start;
+    int t_start, Sb;
     if (j == 0) {
       for (int c = tid; c < C; c += blockDim.x) {
-        ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));
-        sm.Sbase[c] = 0;
+        ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));
         store[c] = NEG_INF;  // no alpha at boundary 0
         store[C + c] = 0.f;  // gamma[0] = 0 in frame 0
       }
@@ -364,64 +371,87 @@ __global__ void __launch_bounds__(NT_MAX, 1)
         store[2 * C] = 0.f;
         store[2 * C + 1] = 0.f;
       }
+      Sb = 0;
       t_start = 1;
     } else {
       const float2* ck = ws.ack + seg * K * C;
       for (int idx = tid; idx < K * C; idx += blockDim.x) {
         const int i = idx / C, c = idx % C;
         const int bnd = t0 - K + i;
-        if (bnd >= 0) ring_put<KBT>(sm, d, c, bnd % K, ck[idx]);
+        if (bnd >= 0) ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, bnd % K, ck[idx]);
       }
-      for (int c = tid; c < C; c += blockDim.x)
-        sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t0) * C + c];
+      Sb = ws.sint[((size_t)b * d.Tstride + t0) * C + ln.cc];
       F0 = ws.acf[seg];
       t_start = t0;
     }
     const int t_end = last ? L : t1 - 1;
     __syncthreads();
     tile_start(sm, d, ws, b, ts, t_start, t_start, t_end, +1);
-    int slot = t_start % K;
-    int base = kl.base_up(t_start, K);
-    for (int t = t_start; t <= t_end; ++t) {
-      if (t > t_start) {
-        base = (base + 1 == K) ? 0 : base + 1;
-        slot = (slot + 1 == K) ? 0 : slot + 1;
+    int wslot = t_start % K;
+    int base = ln.base_up(t_start, K);
+    float mk = 0.f;
+    int cur = -1, t = t_start;
+    bool done = false;
+    while (!done) {
+      const int ti = t / TS;
+      if (ti != cur) {
+        if (!tile_enter(sm, d, ws, b, ts, ti)) {
+          if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+          tile_drain(sm, ts);
+          return;
+        }
+        cur = ti;
       }
-      par = t & 1;
-      q = mod3_next(q);
-      if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
-        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-        tile_drain(sm, ts);
-        return;
-      }
-      float A = 0.f;
-      if (warp_on) A = fwd_kphase<KBT>(sm, d, kl, base, ri, rf, Frel, par, q, e);
-      __syncthreads();
-      bool slow;
-      const float n = step_frame(sm, q, slow);
-      if (t == L) break;
-      float shift = n;
-      if (slow) {
-        refresh_p(sm, d, par, n);
-        shift = 0.f;
-      }
-      float* row = store + (size_t)(t - t0) * SW;
-      if (warp_on) {
-        const float g = aphase<CAT>(sm, d, al, par, n, shift, trans, false, acc, prod);
-        if (al.act && al.j == 0) {
-          const int c = al.c;
-          ring_put<KBT>(sm, d, c, slot,
-                        make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
-          row[c] = A;
-          row[C + c] = g;
+      const int t_stop = min(t_end, ti * TS + TS - 1);
+      const size_t off = tile_row_off(t, C);
+      const int32_t* ri = sm.tint + off;
+      const float* rf = sm.tfrac + off;
+      for (; t <= t_stop; ++t, ri += C, rf += C) {
+        if (t > t_start) {
+          base = (base + 1 == K) ? 0 : base + 1;
+          wslot = (wslot + 1 == K) ? 0 : wslot + 1;
+        }
+        par = t & 1;
+        q = mod3_next(q);
+        const int si = ri[ln.cc];
+        const float sf = rf[ln.cc];
+        float s;
+        const float lse = k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e);
+        const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
+        if (ln.leader) {
+          sm.Acur[par * C + ln.c] = A;
+          sm.pcur[par * PC + ln.c] = ex2(A);
+        }
+        warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(A) : INT_MIN);
+        __syncthreads();
+        bool slow;
+        const float n = step_frame(sm, q, slow);
+        if (t == L) {
+          done = true;
+          break;
+        }
+        mk = next_shift(lse, n, mk);
+        float shift = n;
+        if (slow) {
+          refresh_p(sm, d, par, n);
+          shift = 0.f;
+        }
+        const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
+        float* row = store + (size_t)(t - t0) * SW;
+        if (ln.leader) {
+          const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
+          ring_put<KBT>(rl, d, wslot, make_float2(g - sf, (Frel + n) - (float)(si - Sb)));
+          row[ln.c] = A;
+          row[C + ln.c] = g;
+        }
+        if (tid == 0) {
+          row[2 * C] = Frel;
+          row[2 * C + 1] = Frel + n;
         }
         __syncwarp();
+        Frel += n;
       }
-      if (tid == 0) {
-        row[2 * C] = Frel;
-        row[2 * C + 1] = Frel + n;
-      }
-      Frel += n;
+      if (t > t_end) done = true;
     }
   }
   __syncthreads();
@@ -436,29 +466,27 @@ __global__ void __launch_bounds__(NT_MAX, 1)
   }
 
   // ------------------------------------------------------ beta recompute + posteriors
-  KLane<KBT> kb;
-  kb.init(d, dur, false);
-  ALane<CAT> ab;
-  ab.init(d, trans, true);
+  ln.init_dur(d, dur, false);
+  ln.init_trans(d, trans, true);
   __syncthreads();
   for (int i = tid; i < d.RL * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   __syncthreads();
   double G0 = 0.0;
   float Grel = 0.f;
+  int Sb;
   if (last) {
     for (int c = tid; c < C; c += blockDim.x) {
       const size_t o = ((size_t)b * d.Tstride + L) * C + c;
-      ring_put<KBT>(sm, d, c, L % K, make_float2(ws.sfrac[o], 0.f));
-      sm.Sbase[c] = ws.sint[o];
+      ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, L % K, make_float2(ws.sfrac[o], 0.f));
     }
+    Sb = ws.sint[((size_t)b * d.Tstride + L) * C + ln.cc];
   } else {
     const float2* ck = ws.bck + seg * K * C;
     for (int idx = tid; idx < K * C; idx += blockDim.x) {
       const int i = idx / C, c = idx % C;
-      if (t1 + i <= L) ring_put<KBT>(sm, d, c, (t1 + i) % K, ck[idx]);
+      if (t1 + i <= L) ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, (t1 + i) % K, ck[idx]);
     }
-    for (int c = tid; c < C; c += blockDim.x)
-      sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
+    Sb = ws.sint[((size_t)b * d.Tstride + t1) * C + ln.cc];
     G0 = ws.bcf[seg];
   }
   // this CTA's float64 partials start at zero (each thread its own entries)
@@ -467,119 +495,122 @@ __global__ void __launch_bounds__(NT_MAX, 1)
 #pragma unroll
   for (int i = 0; i < KBT; ++i) {
     accd[i] = 0.f;
-    const int k = kb.k_of(i, false);
-    if (kb.act && k <= K) ws.pgd[(seg * K + (k - 1)) * C + kb.c] = 0.0;
+    const int k = ln.k_of(i, false);
+    if (ln.act && k <= K) ws.pgd[(seg * K + (k - 1)) * C + ln.c] = 0.0;
   }
 #pragma unroll
   for (int i = 0; i < CAT; ++i) {
     acct[i] = 0.f;
-    const int x = ab.j * CAT + i;
-    if (ab.act && x < C) ws.pgt[(seg * C + ab.c) * C + x] = 0.0;
+    const int x = ln.j * CAT + i;
+    if (ln.act && x < C) ws.pgt[(seg * C + ln.c) * C + x] = 0.0;
   }
   const double Xc = F0 + G0 - logz2;
   double accmu = 0.0, vsum = 0.0;  // leader of label c: suffix sum of (start - end) marginals
-  const bool leader = kb.act && kb.j == 0;
   __syncthreads();
   tile_start(sm, d, ws, b, ts, t1 - 1, t0, t1 - 1, -1);
   int nflush = 0;
-  int slot = t1 % K;
-  int base = kb.base_down(t1 - 1, K);
-  for (int s = t1 - 1; s >= t0; --s) {
-    if (s < t1 - 1) base = (base == 0) ? K - 1 : base - 1;
-    slot = (slot == 0) ? K - 1 : slot - 1;
-    par = s & 1;
-    q = mod3_next(q);
-    if (!tile_row(sm, d, ws, b, ts, s, ri, rf)) {
-      if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-      tile_drain(sm, ts);
-      return;
+  int wslot = t1 % K;
+  int base = ln.base_down(t1 - 1, K);
+  float mk = 0.f;
+  int cur = -1, s = t1 - 1;
+  while (s >= t0) {
+    const int ti = s / TS;
+    if (ti != cur) {
+      if (!tile_enter(sm, d, ws, b, ts, ti)) {
+        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+        tile_drain(sm, ts);
+        return;
+      }
+      cur = ti;
     }
-    const float* row = store + (size_t)(s - t0) * SW;
-    float St = 0.f;
-    if (warp_on) {
-      const int c = kb.act ? kb.c : 0;
-      const float Q = -(float)(ri[c] - sm.Sbase[c]) - Grel;
-      const KFan kf = k_fanin<KBT>(sm, d, kb, base, Q, e);
-      const float Bt = (kf.lse == NEG_INF) ? NEG_INF : kf.lse - rf[c];
-      int key = INT_MIN;
-      if (leader) {
+    const int s_stop = max(t0, ti * TS);
+    const size_t off = tile_row_off(s, C);
+    const int32_t* ri = sm.tint + off;
+    const float* rf = sm.tfrac + off;
+    for (; s >= s_stop; --s, ri -= C, rf -= C) {
+      if (s < t1 - 1) base = (base == 0) ? K - 1 : base - 1;
+      wslot = (wslot == 0) ? K - 1 : wslot - 1;
+      par = s & 1;
+      q = mod3_next(q);
+      const float* row = store + (size_t)(s - t0) * SW;
+      const int si = ri[ln.cc];
+      const float sf = rf[ln.cc];
+      float ksum;
+      const float lse = k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e);
+      const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
+      float St = 0.f;
+      if (ln.leader) {
         const float Xs = (float)(Xc + (double)row[2 * C + 1] + (double)Grel);
-        St = (Bt == NEG_INF) ? 0.f : ex2(row[C + c] + Bt + Xs);
-        sm.Acur[par * C + c] = Bt;
-        sm.pcur[par * d.PC + c] = ex2(Bt);
-        key = f2ord(Bt);
-        if (start_marg) start_marg[((size_t)b * (d.T + 1) + s) * C + c] = St;
+        St = (Bt == NEG_INF) ? 0.f : ex2(row[C + ln.c] + Bt + Xs);
+        sm.Acur[par * C + ln.c] = Bt;
+        sm.pcur[par * PC + ln.c] = ex2(Bt);
+        if (start_marg) start_marg[((size_t)b * (d.T + 1) + s) * C + ln.c] = St;
       }
-      warp_max_to_shared(&sm.maxslot[q], key);
-      const float Stg = __shfl_sync(FULL_MASK, St, (tid & 31) & ~(d.GB - 1));
-      if (kb.act && kf.sum > 0.f) {
-        const float coef = gbf * Stg / kf.sum;
+      warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(Bt) : INT_MIN);
+      {
+        const float Stg = __shfl_sync(FULL_MASK, St, (tid & 31) & ~(G - 1));
+        const float coef = (ksum > 0.f) ? gbf * Stg / ksum : 0.f;
 #pragma unroll
-        for (int i = 0; i < KBT; ++i) accd[i] += coef * e[i];
+        for (int i = 0; i < KBT; ++i) accd[i] = fmaf(coef, e[i], accd[i]);
       }
-    }
-    __syncthreads();
-    bool slow;
-    const float n = step_frame(sm, q, slow);
-    float E = 0.f;
-    if (s >= 1) {
-      float shift = n;
-      if (slow) {
-        refresh_p(sm, d, par, n);
-        shift = 0.f;
-      }
-      if (warp_on) {
-        const float g = aphase<CAT>(sm, d, ab, par, n, shift, trans, true, acc, prod);
-        if (leader) {
-          const int c = ab.c;
-          ring_put<KBT>(sm, d, c, slot,
-                        make_float2(g + rf[c], (Grel + n) + (float)(ri[c] - sm.Sbase[c])));
+      __syncthreads();
+      bool slow;
+      const float n = step_frame(sm, q, slow);
+      mk = next_shift(lse, n, mk);
+      float E = 0.f;
+      if (s >= 1) {
+        float shift = n;
+        if (slow) {
+          refresh_p(sm, d, par, n);
+          shift = 0.f;
+        }
+        const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
+        if (ln.leader) {
+          const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, true);
+          ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
           const float Ys = (float)(Xc + (double)row[2 * C] + (double)(Grel + n));
-          E = (g == NEG_INF || row[c] == NEG_INF) ? 0.f : ex2(row[c] + g + Ys);
-          if (end_marg) end_marg[((size_t)b * (d.T + 1) + s) * C + c] = E;
+          E = (g == NEG_INF || row[ln.c] == NEG_INF) ? 0.f : ex2(row[ln.c] + g + Ys);
+          if (end_marg) end_marg[((size_t)b * (d.T + 1) + s) * C + ln.c] = E;
         }
-        const float Eg = __shfl_sync(FULL_MASK, E, (tid & 31) & ~(d.GB - 1));
-        if (ab.act && acc > 0.f) {
-          const float coef = gbf * Eg / acc;
+        // transition posterior = coef * p * e; the constant e is applied at flush
+        const float Eg = __shfl_sync(FULL_MASK, E, (tid & 31) & ~(G - 1));
+        const float coef = (acc > 0.f) ? gbf * Eg / acc : 0.f;
 #pragma unroll
-          for (int i = 0; i < CAT; ++i) acct[i] += coef * prod[i];
-        }
+        for (int i = 0; i < CAT; ++i) acct[i] = fmaf(coef, p[i], acct[i]);
         __syncwarp();
+      } else if (ln.leader && end_marg) {
+        end_marg[((size_t)b * (d.T + 1)) * C + ln.c] = 0.f;
       }
-    } else if (leader && end_marg) {
-      end_marg[((size_t)b * (d.T + 1)) * C + kb.c] = 0.f;
-    }
-    if (leader) {
-      // position s: v = sum of (start - end) marginals strictly after it in the segment
-      const float v = (float)accmu;
-      grad_em[((size_t)b * d.T + s) * C + kb.c] = v;
-      vsum += (double)v;
-      accmu += (double)St - (double)E;
-    }
-    Grel += n;
-    if (++nflush == FLUSH_EVERY || s == t0) {
-      nflush = 0;
-      if (kb.act) {
-#pragma unroll
-        for (int i = 0; i < KBT; ++i) {
-          const int k = kb.k_of(i, false);
-          if (k <= K) ws.pgd[(seg * K + (k - 1)) * C + kb.c] += (double)accd[i];
-          accd[i] = 0.f;
-        }
+      if (ln.leader) {
+        // position s: v = sum of (start - end) marginals strictly after it in the segment
+        const float v = (float)accmu;
+        grad_em[((size_t)b * d.T + s) * C + ln.c] = v;
+        vsum += (double)v;
+        accmu += (double)St - (double)E;
       }
-      if (ab.act) {
+      Grel += n;
+      if (++nflush == FLUSH_EVERY || s == t0) {
+        nflush = 0;
+        if (ln.act) {
 #pragma unroll
-        for (int i = 0; i < CAT; ++i) {
-          const int x = ab.j * CAT + i;
-          if (x < C) ws.pgt[(seg * C + ab.c) * C + x] += (double)acct[i];
-          acct[i] = 0.f;
+          for (int i = 0; i < KBT; ++i) {
+            const int k = ln.k_of(i, false);
+            if (k <= K) ws.pgd[(seg * K + (k - 1)) * C + ln.c] += (double)accd[i];
+            accd[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < CAT; ++i) {
+            const int x = ln.j * CAT + i;
+            if (x < C) ws.pgt[(seg * C + ln.c) * C + x] += (double)(acct[i] * ln.e[i]);
+            acct[i] = 0.f;
+          }
         }
       }
     }
   }
-  if (leader) {
-    ws.segT[seg * C + kb.c] = accmu;
-    ws.segV[seg * C + kb.c] = vsum;
+  if (ln.leader) {
+    ws.segT[seg * C + ln.c] = accmu;
+    ws.segV[seg * C + ln.c] = vsum;
   }
 }
 
@@ -597,9 +628,9 @@ __global__ void selftest_wait_kernel(int* status, int spins) {
 }
 
 // ----------------------------------------------------------------------------- launchers
-bool shape_supported(int KBT, int CAT) {
-#define SEMICRF_SHAPE_OK(a, b) \
-  if (KBT == a && CAT == b) return true;
+bool shape_supported(int KBT, int CAT, int G, int LB) {
+#define SEMICRF_SHAPE_OK(a, b, g, lb) \
+  if (KBT == a && CAT == b && G == g && LB == lb) return true;
   SEMICRF_FOR_EACH_SHAPE(SEMICRF_SHAPE_OK)
 #undef SEMICRF_SHAPE_OK
   return false;
@@ -617,13 +648,13 @@ cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths
                          const float* dur, double* logZ_out, int n_alpha, int n_beta,
                          cudaStream_t st) {
   const size_t sm = recursion_smem_bytes(d, false);
-#define SEMICRF_LAUNCH_CHAIN(a, b)                                                          \
-  if (d.KBT == a && d.CAT == b) {                                                           \
-    const cudaError_t e = allow_smem(chain_kernel<a, b>, sm);                               \
-    if (e != cudaSuccess) return e;                                                         \
-    chain_kernel<a, b><<<n_alpha + n_beta, d.NT, sm, st>>>(d, ws, lengths, trans, dur, logZ_out, \
-                                                           n_alpha);                        \
-    return cudaGetLastError();                                                              \
+#define SEMICRF_LAUNCH_CHAIN(a, b, g, lb)                                                    \
+  if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \
+    const cudaError_t e = allow_smem(chain_kernel<a, b, g, lb>, sm);                         \
+    if (e != cudaSuccess) return e;                                                          \
+    chain_kernel<a, b, g, lb><<<n_alpha + n_beta, d.NT, sm, st>>>(d, ws, lengths, trans, dur, \
+                                                                  logZ_out, n_alpha);        \
+    return cudaGetLastError();                                                               \
   }
   SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_CHAIN)
 #undef SEMICRF_LAUNCH_CHAIN
@@ -634,14 +665,13 @@ cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengt
                            const float* trans, const float* dur, const double* grad_logZ,
                            float* grad_em, float* start_marg, float* end_marg, cudaStream_t st) {
   const size_t sm = recursion_smem_bytes(d, d.store_smem != 0);
-#define SEMICRF_LAUNCH_SEG(a, b)                                                         \
-  if (d.KBT == a && d.CAT == b) {                                                        \
-    const cudaError_t e = allow_smem(segment_kernel<a, b>, sm);                          \
-    if (e != cudaSuccess) return e;                                                      \
-    segment_kernel<a, b><<<dim3(d.nck, d.B), d.NT, sm, st>>>(d, ws, lengths, trans, dur,   \
-                                                             grad_logZ, grad_em, start_marg, \
-                                                             end_marg);                    \
-    return cudaGetLastError();                                                           \
+#define SEMICRF_LAUNCH_SEG(a, b, g, lb)                                                      \
+  if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \
+    const cudaError_t e = allow_smem(segment_kernel<a, b, g, lb>, sm);                       \
+    if (e != cudaSuccess) return e;                                                          \
+    segment_kernel<a, b, g, lb><<<dim3(d.nck, d.B), d.NT, sm, st>>>(                         \
+        d, ws, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg);               \
+    return cudaGetLastError();                                                               \
   }
   SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_SEG)
 #undef SEMICRF_LAUNCH_SEG

@@ -4,11 +4,18 @@
 //
 // Ring layout.  Each label owns RL = K + KBT float2 entries (value, exact
 // integer part); boundary x lives in slot x mod K, and slots below KBT are
-// mirrored at slot + K.  A lane owns KBT consecutive durations, so at every
-// step it reads KBT consecutive entries starting at a base index that moves by
-// one per step: no per-term index arithmetic, no wrap test.  Entries of
-// boundaries that do not exist (before 0, after L) hold -inf, and durations
-// above K carry dur2 = -inf, so no per-term validity test is needed either.
+// mirrored at slot + K (and further multiples of K when K < KBT).  A lane
+// owns KBT consecutive durations, so at every step it reads KBT consecutive
+// entries starting at a base index that moves by one per step: no per-term
+// index arithmetic, no wrap test.  Entries of boundaries that do not exist
+// (before 0, after L) hold -inf, and durations above K carry dur2 = -inf, so
+// no per-term validity test is needed either.
+//
+// Lane groups.  A group of G consecutive lanes (G a power of two, a
+// compile-time shape parameter) owns one label for both fan-ins; per-step
+// work is latency bound (about one warp per scheduler), so the step code keeps
+// everything a lane needs in registers and avoids index arithmetic and
+// branches on the critical path.
 #pragma once
 
 #include <climits>
@@ -60,8 +67,8 @@ __device__ __forceinline__ Smem carve(unsigned char* raw, const Dims& d, bool wi
   return s;
 }
 
-// Fills the ring with (-inf, 0), zeroes the padded label vector and resets
-// the barriers' and the max slots' state.  Call before the first __syncthreads.
+// Fills the ring with (-inf, 0), zeroes the padded label vectors and resets
+// the barriers and the max slots.  A __syncthreads must follow.
 __device__ __forceinline__ void init_smem(const Smem& sm, const Dims& d) {
   for (int i = threadIdx.x; i < d.RL * d.C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = threadIdx.x; i < 2 * d.PC; i += blockDim.x) sm.pcur[i] = 0.f;
@@ -73,12 +80,13 @@ __device__ __forceinline__ void init_smem(const Smem& sm, const Dims& d) {
   }
 }
 
-// Writes ring slot `slot` of label c (and its mirror).
+// Writes ring slot `slot` of one label (rl = its first entry) and its mirrors
+// (every index slot + mK below RL = K + KBT).
 template <int KBT>
-__device__ __forceinline__ void ring_put(const Smem& sm, const Dims& d, int c, int slot, float2 v) {
-  float2* r = sm.ring + (size_t)c * d.RL;
-  r[slot] = v;
-  if (slot < KBT) r[slot + d.K] = v;
+__device__ __forceinline__ void ring_put(float2* rl, const Dims& d, int slot, float2 v) {
+  rl[slot] = v;
+  if (slot < KBT)
+    for (int x = slot + d.K; x < d.RL; x += d.K) rl[x] = v;
 }
 
 // Ring entry of boundary `bnd` (0 <= bnd) for label c.
@@ -90,7 +98,7 @@ __device__ __forceinline__ float2& ring_at(const Smem& sm, const Dims& d, int c,
 // Double-buffered TMA stream of prefix-sum tiles (TS rows) for one sequence,
 // moving up (dir = +1) or down (dir = -1).  Entering a tile issues the next.
 struct TileStream {
-  int cur, lo, hi, dir;
+  int lo, hi, dir;
   uint32_t ph[2];
 };
 
@@ -106,34 +114,26 @@ __device__ __forceinline__ void tile_issue(const Smem& sm, const Dims& d, const 
   bulk_g2s(sm.tfrac + (size_t)buf * TS * d.C, ws.sfrac + row0 * d.C, bytes, &sm.mbar[buf]);
 }
 
+// Rows lo_row..hi_row will be visited starting at first_row.
 __device__ __forceinline__ void tile_start(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
                                            TileStream& ts, int first_row, int lo_row, int hi_row,
                                            int dir) {
   ts.lo = lo_row / TS;
   ts.hi = hi_row / TS;
   ts.dir = dir;
-  ts.cur = -1;
   tile_issue(sm, d, ws, b, ts, first_row / TS);
 }
 
-// Makes row r readable (ri, rf); returns false (uniformly) if a wait gave up.
-__device__ __forceinline__ bool tile_row(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
-                                         TileStream& ts, int r, const int32_t*& ri,
-                                         const float*& rf) {
-  const int i = r / TS;
-  bool ok = true;
-  if (i != ts.cur) {
-    const int buf = i & 1;
-    ok = mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
-    ts.ph[buf] ^= 1u;
-    ts.cur = i;
-    // every thread is done with the previous tile before its buffer is refilled
-    ok = !__syncthreads_or(!ok);
-    tile_issue(sm, d, ws, b, ts, i + ts.dir);
-  }
-  const size_t o = ((size_t)(i & 1) * TS + (r - i * TS)) * d.C;
-  ri = sm.tint + o;
-  rf = sm.tfrac + o;
+// Waits for tile i, then (after every thread is done with the previous tile)
+// issues the next one into the other buffer.  Returns false, uniformly, if
+// the bounded wait gave up.
+__device__ __forceinline__ bool tile_enter(const Smem& sm, const Dims& d, const WsPtrs& ws, int b,
+                                           TileStream& ts, int i) {
+  const int buf = i & 1;
+  bool ok = mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
+  ts.ph[buf] ^= 1u;
+  ok = !__syncthreads_or(!ok);
+  tile_issue(sm, d, ws, b, ts, i + ts.dir);
   return ok;
 }
 
@@ -143,29 +143,90 @@ __device__ __forceinline__ void tile_drain(const Smem& sm, TileStream& ts) {
     for (int buf = 0; buf < 2; ++buf) mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
 }
 
+// Offset of row r in the tile buffers (its tile must be the current one).
+__device__ __forceinline__ size_t tile_row_off(int r, int C) {
+  const int i = r / TS;
+  return ((size_t)(i & 1) * TS + (r - i * TS)) * C;
+}
+
+// ----------------------------------------------------------------------------- reductions
+template <int G>
+__device__ __forceinline__ float gsum(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+  return v;
+}
+
+template <int G>
+__device__ __forceinline__ unsigned gmask() {
+  if constexpr (G >= 32) {
+    return FULL_MASK;
+  } else {
+    const int lane = threadIdx.x & 31;
+    return ((1u << G) - 1u) << (lane & ~(G - 1));
+  }
+}
+
+// (value, index) max with ties to the smaller index, over the lane group.
+template <int G>
+__device__ __forceinline__ void gargmax(float& v, int& i) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(FULL_MASK, v, o);
+    const int i2 = __shfl_xor_sync(FULL_MASK, i, o);
+    if (v2 > v || (v2 == v && i2 < i)) {
+      v = v2;
+      i = i2;
+    }
+  }
+}
+
 // ----------------------------------------------------------------------------- lanes
 __device__ __forceinline__ float l2e() { return (float)LOG2E_D; }
 
-// k fan-in role: label cB, lane jB of GB; durations of lane term i:
-//   up   (forward, terms at t - k):  k_i = (jB + 1) * KBT - i
-//   down (backward, terms at s + k): k_i = jB * KBT + 1 + i
-template <int KBT>
-struct KLane {
-  int c, j;
-  bool act;
+// One lane of a label group: label c, lane j of G.  Durations of lane term i:
+//   up   (forward, terms at t - k):  k_i = (j + 1) * KBT - i
+//   down (backward, terms at s + k): k_i = j * KBT + 1 + i
+// Label-fan-in operands e[i] = 2^(trans2 - max) for the other side's labels
+// j*CAT + i: column-normalised for the forward side (sum over c' into c),
+// row-normalised for the backward side (sum over c out of c').
+template <int KBT, int CAT, int G>
+struct Lane {
+  int c, cc, j;
+  bool act, leader;
+  float tmax;
   float d[KBT];
+  float e[CAT];
   __device__ __forceinline__ int k_of(int i, bool up) const {
     return up ? (j + 1) * KBT - i : j * KBT + 1 + i;
   }
-  __device__ __forceinline__ void init(const Dims& dm, const float* dur, bool up) {
-    c = threadIdx.x / dm.GB;
-    j = threadIdx.x % dm.GB;
+  __device__ __forceinline__ void init_ids(const Dims& dm) {
+    c = threadIdx.x / G;
+    j = threadIdx.x % G;
     act = c < dm.C;
-    const int cc = act ? c : 0;
+    cc = act ? c : 0;
+    leader = act && j == 0;
+  }
+  __device__ __forceinline__ void init_dur(const Dims& dm, const float* dur, bool up) {
 #pragma unroll
     for (int i = 0; i < KBT; ++i) {
       const int k = k_of(i, up);
       d[i] = (act && k <= dm.K) ? __ldg(dur + (size_t)(k - 1) * dm.C + cc) * l2e() : NEG_INF;
+    }
+  }
+  __device__ __forceinline__ void init_trans(const Dims& dm, const float* trans, bool rows) {
+    const int C = dm.C;
+    float mx = NEG_INF;
+    for (int x = 0; x < C; ++x)
+      mx = fmaxf(mx, __ldg(trans + (rows ? (size_t)cc * C + x : (size_t)x * C + cc)) * l2e());
+    if (mx == NEG_INF) mx = 0.f;
+    tmax = mx;
+#pragma unroll
+    for (int i = 0; i < CAT; ++i) {
+      const int x = j * CAT + i;
+      e[i] = (act && x < C)
+                 ? ex2(__ldg(trans + (rows ? (size_t)cc * C + x : (size_t)x * C + cc)) * l2e() - mx)
+                 : 0.f;
     }
   }
   // first ring index of this lane's window
@@ -176,37 +237,7 @@ struct KLane {
   __device__ __forceinline__ int base_down(int s, int K) const { return (s + j * KBT + 1) % K; }
 };
 
-// label fan-in role: output label c of GA lanes; lane j owns labels
-// j*CAT .. j*CAT+CAT-1 of the other side.  e[i] = 2^(trans2 - max) with the
-// forward (column, rows=false) or backward (row, rows=true) normalisation.
-template <int CAT>
-struct ALane {
-  int c, j;
-  bool act;
-  float tmax;
-  float e[CAT];
-  __device__ __forceinline__ void init(const Dims& dm, const float* trans, bool rows) {
-    c = threadIdx.x / dm.GB;  // same lane groups as the k fan-in
-    j = threadIdx.x % dm.GB;
-    act = c < dm.C;
-    const int C = dm.C;
-    const int o = act ? c : 0;
-    float mx = NEG_INF;
-    for (int x = 0; x < C; ++x)
-      mx = fmaxf(mx, __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * l2e());
-    if (mx == NEG_INF) mx = 0.f;
-    tmax = mx;
-#pragma unroll
-    for (int i = 0; i < CAT; ++i) {
-      const int x = j * CAT + i;
-      e[i] = (act && x < C)
-                 ? ex2(__ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * l2e() - mx)
-                 : 0.f;
-    }
-  }
-};
-
-// Loads v[0..CAT) = p[j*CAT ..] with the widest aligned vector loads.
+// Loads v[0..CAT) = p[0..CAT) with the widest aligned vector loads.
 template <int CAT>
 __device__ __forceinline__ void load_block(const float* p, float (&v)[CAT]) {
   if constexpr (CAT % 4 == 0) {
@@ -231,54 +262,69 @@ __device__ __forceinline__ void load_block(const float* p, float (&v)[CAT]) {
   }
 }
 
-// k fan-in over this lane's window: y_i = (P + Q) + v + dur2[k_i - 1];
-// group LSE (lse, m, sum valid in every lane of the group); e[i] = 2^(y_i - m).
-struct KFan {
-  float lse, m, sum;
-};
-
-template <int KBT>
-__device__ __forceinline__ KFan k_fanin(const Smem& sm, const Dims& d, const KLane<KBT>& L, int base,
-                                        float Q, float (&e)[KBT]) {
-  const float2* r = sm.ring + (size_t)(L.act ? L.c : 0) * d.RL + base;
-  float y[KBT];
-  float m = NEG_INF;
+// ----------------------------------------------------------------------------- fan-ins
+// k fan-in over a lane's window r[0..KBT), y_i = ((P + Q) + v) + dur2.
+// The exponentials are taken against an exact-integer shift m (a prediction
+// of the group LSE: no max pass, no max reduction): e[i] = 2^(y_i - m) and
+// s = group sum.  If s leaves [2^-64, 2^64] the group redoes the fan-in
+// against ceil(exact max).  Returns the LSE (NEG_INF if nothing is finite);
+// on return m and s describe e[] (e[i] / s are the normalised weights).
+template <int KBT, int G>
+__device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (&d)[KBT], float& m,
+                                         float& s, float (&e)[KBT]) {
+  {
+    const float Qm = Q - m;  // exact: both integers
+    float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < KBT; ++i) {
-    const float2 v = r[i];
-    y[i] = ((v.y + Q) + v.x) + L.d[i];
-    m = fmaxf(m, y[i]);
+    for (int i = 0; i < KBT; ++i) {
+      const float2 v = r[i];
+      e[i] = ex2(((v.y + Qm) + v.x) + d[i]);
+      sp[i & 3] += e[i];
+    }
+    s = gsum<G>((sp[0] + sp[1]) + (sp[2] + sp[3]));
   }
-  m = group_max(m, d.GB);
-  float s = 0.f;
-  const float mm = (m == NEG_INF) ? 0.f : m;
+  if (!(s >= 0x1p-64f && s <= 0x1p64f)) {
+    // rare: the prediction was far off (or nothing is finite)
+    const unsigned gm = gmask<G>();
+    float mx = NEG_INF;
 #pragma unroll
-  for (int i = 0; i < KBT; ++i) {
-    e[i] = ex2(y[i] - mm);
-    s += e[i];
+    for (int i = 0; i < KBT; ++i) {
+      const float2 v = r[i];
+      mx = fmaxf(mx, ((v.y + Q) + v.x) + d[i]);
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gm, mx, o));
+    m = (mx == NEG_INF) ? 0.f : ceilf(mx);
+    const float Qm = Q - m;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < KBT; ++i) {
+      const float2 v = r[i];
+      e[i] = ex2(((v.y + Qm) + v.x) + d[i]);
+      ss += e[i];
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gm, ss, o);
+    s = ss;
   }
-  s = group_sum(s, d.GB);
-  KFan out;
-  out.m = m;
-  out.sum = s;
-  out.lse = (m == NEG_INF) ? NEG_INF : m + lg2(s);
-  return out;
+  return (s > 0.f) ? m + lg2(s) : NEG_INF;
 }
 
-// Label fan-in in the exponential domain: sum_x pcur[x] * e[x], group-summed.
-// prod[i] keeps the per-term products.
-template <int CAT>
-__device__ __forceinline__ float label_fanin(const float* pcur, const Dims& d, const ALane<CAT>& A,
-                                             float (&prod)[CAT]) {
-  float p[CAT];
-  load_block<CAT>(pcur + A.j * CAT, p);
-  float acc = 0.f;
+// Next step's shift: this step's LSE moved into the next frame (step n).
+__device__ __forceinline__ float next_shift(float lse, float n, float m) {
+  return isfinite(lse) ? rintf(lse) - n : m;
+}
+
+// Label fan-in in the exponential domain: sum_x pcur[x] * e[x] over the group;
+// p[i] keeps this lane's loaded pcur values.
+template <int CAT, int G>
+__device__ __forceinline__ float label_fanin(const float* pj, const float (&e)[CAT],
+                                             float (&p)[CAT]) {
+  load_block<CAT>(pj, p);
+  float ap[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < CAT; ++i) {
-    prod[i] = p[i] * A.e[i];
-    acc += prod[i];
-  }
-  return group_sum(acc, d.GB);
+  for (int i = 0; i < CAT; ++i) ap[i & 3] = fmaf(p[i], e[i], ap[i & 3]);
+  return gsum<G>((ap[0] + ap[1]) + (ap[2] + ap[3]));
 }
 
 constexpr float EXP_SAFE = 100.f;       // |frame step| beyond which p is recomputed
@@ -286,9 +332,8 @@ constexpr float UNDERFLOW = 0x1p-100f;  // label sums below this use the log dom
 
 // Log-domain label fan-in for one output (rare fallback when the
 // exponential-domain sum underflows): LSE_x (vals[x] - shift + trans2).
-__device__ __forceinline__ float label_lse_slow(const Dims& d, const float* vals, float shift,
-                                                const float* trans, int o, bool rows) {
-  const int C = d.C;
+static __device__ __noinline__ float label_lse_slow(int C, const float* vals, float shift,
+                                             const float* trans, int o, bool rows) {
   float mx = NEG_INF;
   for (int x = 0; x < C; ++x) {
     const float t2 = __ldg(trans + (rows ? (size_t)o * C + x : (size_t)x * C + o)) * l2e();
@@ -303,9 +348,17 @@ __device__ __forceinline__ float label_lse_slow(const Dims& d, const float* vals
   return mx + lg2(s);
 }
 
-// Reads the max of step `q` (mod 3), resets slot q+2 for the step after next,
-// and returns the integer frame step n; `slow` is set when 2^(value) could
-// overflow or underflow in the exponential-domain fan-in.
+// log2 of a label sum minus the frame shift, with the log-domain fallback.
+__device__ __forceinline__ float label_log(float acc, float tmax, float shift, int C,
+                                           const float* vals, float n, const float* trans, int o,
+                                           bool rows) {
+  if (acc >= UNDERFLOW && acc <= 3.0e38f) return lg2(acc) + tmax - shift;
+  return label_lse_slow(C, vals, n, trans, o, rows);
+}
+
+// Reads the max of step slot q (mod 3), resets slot q+2 for the step after
+// next, and returns the integer frame step n; `slow` is set when 2^(value)
+// could overflow or underflow in the exponential-domain fan-in.
 __device__ __forceinline__ float step_frame(const Smem& sm, int q, bool& slow) {
   const float M = ord2f(sm.maxslot[q]);
   if (threadIdx.x == 0) sm.maxslot[q == 0 ? 2 : q - 1] = f2ord(NEG_INF);
@@ -315,6 +368,13 @@ __device__ __forceinline__ float step_frame(const Smem& sm, int q, bool& slow) {
 }
 
 __device__ __forceinline__ int mod3_next(int q) { return q == 2 ? 0 : q + 1; }
+
+// Uniform slow path: the step's frame jump is too large for 2^A in float32.
+__device__ __forceinline__ void refresh_p(const Smem& sm, const Dims& d, int par, float n) {
+  for (int c = threadIdx.x; c < d.C; c += blockDim.x)
+    sm.pcur[par * d.PC + c] = ex2(sm.Acur[par * d.C + c] - n);
+  __syncthreads();
+}
 
 }  // namespace ring
 }  // namespace semicrf

@@ -16,24 +16,8 @@ namespace semicrf {
 
 using namespace ring;
 
-namespace {
-
-// (value, index) max with ties to the smaller index, over aligned groups.
-__device__ __forceinline__ void group_argmax(float& v, int& i, int G) {
-  for (int o = G >> 1; o > 0; o >>= 1) {
-    const float v2 = __shfl_xor_sync(FULL_MASK, v, o);
-    const int i2 = __shfl_xor_sync(FULL_MASK, i, o);
-    if (v2 > v || (v2 == v && i2 < i)) {
-      v = v2;
-      i = i2;
-    }
-  }
-}
-
-}  // namespace
-
-template <int KBT, int CAT>
-__global__ void __launch_bounds__(NT_MAX, 1)
+template <int KBT, int CAT, int G, int LB>
+__global__ void __launch_bounds__(LB, 1)
     viterbi_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                    const float* __restrict__ trans, const float* __restrict__ dur,
                    double* __restrict__ score, int32_t* __restrict__ labels,
@@ -56,118 +40,127 @@ __global__ void __launch_bounds__(NT_MAX, 1)
     }
     return;
   }
-  const bool warp_on = ((tid & ~31) / d.GB) < C;
-  KLane<KBT> kl;
-  kl.init(d, dur, true);
+  Lane<KBT, CAT, G> ln;
+  ln.init_ids(d);
+  ln.init_dur(d, dur, true);
   // raw trans2 column values for this lane's previous labels (no exponentials)
   float tr[CAT];
 #pragma unroll
   for (int i = 0; i < CAT; ++i) {
-    const int x = kl.j * CAT + i;
-    tr[i] = (kl.act && x < C) ? __ldg(trans + (size_t)x * C + kl.c) * l2e() : NEG_INF;
+    const int x = ln.j * CAT + i;
+    tr[i] = (ln.act && x < C) ? __ldg(trans + (size_t)x * C + ln.cc) * l2e() : NEG_INF;
   }
+  float2* const rl = sm.ring + (size_t)ln.cc * d.RL;
   init_smem(sm, d);
   __syncthreads();
   for (int c = tid; c < C; c += blockDim.x) {
-    ring_put<KBT>(sm, d, c, 0, make_float2(0.f, 0.f));
+    ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));
     sm.Sbase[c] = 0;
   }
   __syncthreads();
   int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
-  const int32_t* ri;
-  const float* rf;
-  tile_start(sm, d, ws, b, ts, 1, 0, L, +1);
+  tile_start(sm, d, ws, b, ts, 1, 1, L, +1);
   double F0 = 0.0;
   float Frel = 0.f;
-  int slot = 0, par = 0, q = 0;
-  int base = kl.base_up(1, K);
+  int Sb = 0;
+  int wslot = 0, par = 0, q = 0;
+  int base = ln.base_up(1, K);
   int to_ck = d.delta;
   int bk = 0;
-  for (int t = 1; t <= L; ++t) {
-    if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
-    slot = (slot + 1 == K) ? 0 : slot + 1;
-    par = t & 1;
-    q = mod3_next(q);
-    if (!tile_row(sm, d, ws, b, ts, t, ri, rf)) {
-      if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-      tile_drain(sm, ts);
-      return;
-    }
-    if (--to_ck == 0) {
-      // rebase the integer frames (keeps every stored integer small)
-      to_ck = d.delta;
-      __syncthreads();
-      const float dF = Frel;
-      for (int idx = tid; idx < C * d.RL; idx += blockDim.x) {
-        const int c = idx / d.RL;
-        float2 v = sm.ring[idx];
-        v.y = (v.y - dF) + (float)(ri[c] - sm.Sbase[c]);
-        sm.ring[idx] = v;
+  int cur = -1, t = 1;
+  bool done = false;
+  while (!done) {
+    const int ti = t / TS;
+    if (ti != cur) {
+      if (!tile_enter(sm, d, ws, b, ts, ti)) {
+        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+        tile_drain(sm, ts);
+        return;
       }
-      __syncthreads();
-      for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
-      F0 += (double)dF;
-      Frel = 0.f;
-      __syncthreads();
+      cur = ti;
     }
-    if (warp_on) {
-      const int c = kl.act ? kl.c : 0;
-      const float Q = (float)(ri[c] - sm.Sbase[c]) - Frel;
-      const float2* r = sm.ring + (size_t)c * d.RL + base;
-      // lane term i has k = (j+1)*KBT - i: walk i downwards for ascending k
-      float best = NEG_INF;
-      bk = 0x7fffffff;
-#pragma unroll
-      for (int i = KBT - 1; i >= 0; --i) {
-        const float2 v = r[i];
-        const float y = ((v.y + Q) + v.x) + kl.d[i];
-        if (y > best || bk == 0x7fffffff) {
-          best = y;
-          bk = kl.k_of(i, true);
+    const int t_stop = min(L, ti * TS + TS - 1);
+    const size_t off = tile_row_off(t, C);
+    const int32_t* ri = sm.tint + off;
+    const float* rf = sm.tfrac + off;
+    for (; t <= t_stop; ++t, ri += C, rf += C) {
+      if (t > 1) base = (base + 1 == K) ? 0 : base + 1;
+      wslot = (wslot + 1 == K) ? 0 : wslot + 1;
+      par = t & 1;
+      q = mod3_next(q);
+      if (--to_ck == 0) {
+        // rebase the integer frames (keeps every stored integer small)
+        to_ck = d.delta;
+        __syncthreads();
+        for (int idx = tid; idx < C * d.RL; idx += blockDim.x) {
+          const int c = idx / d.RL;
+          float2 v = sm.ring[idx];
+          v.y = (v.y - Frel) + (float)(ri[c] - sm.Sbase[c]);
+          sm.ring[idx] = v;
         }
+        __syncthreads();
+        for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ri[c];
+        F0 += (double)Frel;
+        Frel = 0.f;
+        Sb = ri[ln.cc];
+        __syncthreads();
       }
-      group_argmax(best, bk, d.GB);
-      int key = INT_MIN;
-      if (kl.act && kl.j == 0) {
-        const float V = rf[c] + best;
-        sm.Acur[par * C + c] = V;
-        key = f2ord(V);
-      }
-      warp_max_to_shared(&sm.maxslot[q], key);
-    }
-    __syncthreads();
-    bool slow;
-    const float n = step_frame(sm, q, slow);
-    if (t == L) break;
-    if (warp_on) {
-      const float* V = sm.Acur + par * C;
-      float best = NEG_INF;
-      int bc = 0x7fffffff;
+      const int si = ri[ln.cc];
+      const float sf = rf[ln.cc];
+      {
+        const float Q = (float)(si - Sb) - Frel;
+        const float2* r = rl + base;
+        // lane term i has k = (j+1)*KBT - i: walk i downwards for ascending k
+        float best = NEG_INF;
+        bk = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < CAT; ++i) {
-        const int x = kl.j * CAT + i;
-        const float vx = (x < C) ? V[x] + tr[i] : NEG_INF;
-        if (vx > best || bc == 0x7fffffff) {
-          best = vx;
-          bc = x;
+        for (int i = KBT - 1; i >= 0; --i) {
+          const float2 v = r[i];
+          const float y = ((v.y + Q) + v.x) + ln.d[i];
+          if (y > best || bk == 0x7fffffff) {
+            best = y;
+            bk = ln.k_of(i, true);
+          }
         }
+        gargmax<G>(best, bk);
+        const float V = sf + best;
+        if (ln.leader) sm.Acur[par * C + ln.c] = V;
+        warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(V) : INT_MIN);
       }
-      group_argmax(best, bc, d.GB);
-      if (kl.act && kl.j == 0) {
-        const int c = kl.c;
-        const float g = best - n;
-        ring_put<KBT>(sm, d, c, slot,
-                      make_float2(g - rf[c], (Frel + n) - (float)(ri[c] - sm.Sbase[c])));
-        bp[(size_t)t * C + c] = (bk & 0xffff) | (bc << 16);
+      __syncthreads();
+      bool slow;
+      const float n = step_frame(sm, q, slow);
+      if (t == L) {
+        done = true;
+        break;
+      }
+      {
+        const float* V = sm.Acur + par * C;
+        float best = NEG_INF;
+        int bc = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < CAT; ++i) {
+          const int x = ln.j * CAT + i;
+          const float vx = (x < C) ? V[x] + tr[i] : NEG_INF;
+          if (vx > best || bc == 0x7fffffff) {
+            best = vx;
+            bc = x;
+          }
+        }
+        gargmax<G>(best, bc);
+        if (ln.leader) {
+          ring_put<KBT>(rl, d, wslot, make_float2((best - n) - sf, (Frel + n) - (float)(si - Sb)));
+          bp[(size_t)t * C + ln.c] = (bk & 0xffff) | (bc << 16);
+        }
       }
       __syncwarp();
+      Frel += n;
     }
-    Frel += n;
   }
   // the last step's best durations, then the best final label (smallest on ties)
-  if (kl.act && kl.j == 0) bp[(size_t)L * C + kl.c] = bk & 0xffff;
+  if (ln.leader) bp[(size_t)L * C + ln.c] = bk & 0xffff;
   __syncthreads();
   if (tid < 32) {
     const float* V = sm.Acur + par * C;
@@ -180,18 +173,18 @@ __global__ void __launch_bounds__(NT_MAX, 1)
         bc = c;
       }
     }
-    group_argmax(best, bc, 32);
+    gargmax<32>(best, bc);
     if (tid == 0) score[b] = (F0 + (double)Frel + (double)best) * LN2_D;
-    int t = L, c = bc;
-    while (t > 0) {
-      const int k = bp[(size_t)t * C + c] & 0xffff;
-      const int s = t - k;
-      for (int u = s + tid; u < t; u += 32) {
+    int tt = L, c = bc;
+    while (tt > 0) {
+      const int k = bp[(size_t)tt * C + c] & 0xffff;
+      const int s = tt - k;
+      for (int u = s + tid; u < tt; u += 32) {
         labels[(size_t)b * T + u] = c;
         seg_start[(size_t)b * T + u] = (u == s) ? 1 : 0;
       }
       if (s > 0) c = (bp[(size_t)s * C + c] >> 16) & 0xffff;
-      t = s;
+      tt = s;
     }
   }
 }
@@ -200,17 +193,17 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
                            const float* trans, const float* dur, double* score, int32_t* labels,
                            uint8_t* seg_start, cudaStream_t st) {
   const size_t sm = recursion_smem_bytes(d, false);
-#define SEMICRF_LAUNCH_VIT(a, b)                                                               \
-  if (d.KBT == a && d.CAT == b) {                                                              \
-    if (sm > 48 * 1024) {                                                                      \
-      const cudaError_t e = cudaFuncSetAttribute(viterbi_kernel<a, b>,                         \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                                 (int)sm);                                     \
-      if (e != cudaSuccess) return e;                                                          \
-    }                                                                                          \
-    viterbi_kernel<a, b><<<d.B, d.NT, sm, st>>>(d, ws, lengths, trans, dur, score, labels,     \
-                                                seg_start);                                    \
-    return cudaGetLastError();                                                                 \
+#define SEMICRF_LAUNCH_VIT(a, b, g, lb)                                                      \
+  if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \
+    if (sm > 48 * 1024) {                                                                    \
+      const cudaError_t e = cudaFuncSetAttribute(viterbi_kernel<a, b, g, lb>,                \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                                 (int)sm);                                   \
+      if (e != cudaSuccess) return e;                                                        \
+    }                                                                                        \
+    viterbi_kernel<a, b, g, lb><<<d.B, d.NT, sm, st>>>(d, ws, lengths, trans, dur, score,    \
+                                                       labels, seg_start);                   \
+    return cudaGetLastError();                                                               \
   }
   SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_VIT)
 #undef SEMICRF_LAUNCH_VIT

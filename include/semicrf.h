@@ -187,6 +187,32 @@ SEMICRF_API int semicrf_selftest_bounded_wait(void *ws, size_t ws_bytes, int spi
 SEMICRF_API int semicrf_profile_enable(int on);
 SEMICRF_API int semicrf_profile_read(const char *kernel, double *total_ms, int *launches);
 
+/*
+ * log Z without a workspace and without allocating (no counterpart on the
+ * pages).  For callers that cannot allocate device memory when they run --
+ * a plugin whose execution hook may not allocate because its memory was
+ * planned ahead, or code where a cudaMalloc would stall the device -- this
+ * runs the same prefix-sum and forward-ring kernels as semicrf_forward with
+ * SEMICRF_FLAG_FORWARD_ONLY, keeping their scratch in one fixed array inside
+ * the library's device image (SEMICRF_NOALLOC_SCRATCH_BYTES; every GPU that
+ * loads the library holds it until the process exits).  The caller still
+ * passes the inputs and logZ [B] (float64), all device memory.
+ *  - Sizes whose forward working set exceeds the array (prefix sums, chunk
+ *    sums and ring checkpoints: about 8*B*(T+1)*C bytes plus the
+ *    checkpoints) return SEMICRF_ERR_UNSUPPORTED before anything runs.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - No cudaMalloc, cudaFree or allocating library call is made.
+ *  - Every call on a device shares the array and leaves its contents behind;
+ *    only the status word is cleared per call.  Calls that overlap on the GPU
+ *    (two streams or two host threads at once) race on it: serialise them.
+ *  - A length outside [0, T] gives logZ[b] = NaN (no status word to read).
+ */
+#define SEMICRF_NOALLOC_SCRATCH_BYTES (32u << 20)
+SEMICRF_API int semicrf_forward_noalloc(const float *em, const int32_t *lengths, const float *trans,
+                                        const float *dur, int B, int T, int C, int K,
+                                        unsigned flags, double *logZ, semicrf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

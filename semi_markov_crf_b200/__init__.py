@@ -13,7 +13,8 @@ from __future__ import annotations
 _BINDING_NAMES = {
     "workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
     "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
-    "FLAG_FORWARD_ONLY", "selftest_bounded_wait",
+    "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "forward_noalloc", "profile_enable",
+    "profile_read",
 }
 
 

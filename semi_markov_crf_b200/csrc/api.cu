@@ -49,6 +49,8 @@ int max_smem_optin() {
   return cached;
 }
 
+}  // namespace
+
 // Sizes, lane mapping and limits.  Returns a semicrf_status.
 int make_dims(int B, int T, int C, int K, Dims& d) {
   if (B < 0 || T < 0 || C < 1 || K < 1) return SEMICRF_ERR_INVALID_ARG;
@@ -109,6 +111,8 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (recursion_smem_bytes(d, false) > budget) return SEMICRF_ERR_UNSUPPORTED;
   return SEMICRF_OK;
 }
+
+namespace {
 
 // Workspace layout; fills `p` when base != nullptr.  Returns total bytes.
 size_t layout(const Dims& d, void* base, WsPtrs* p) {

@@ -42,6 +42,9 @@ __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restr
 
 __global__ void selftest_wait_kernel(int* status, int spins);
 
+// Sizes, launch geometry and limits for (B, T, C, K); returns a semicrf_status.
+int make_dims(int B, int T, int C, int K, Dims& d);
+
 // Lane shapes with a compiled instantiation (KBT durations, CAT labels per lane).
 bool shape_supported(int KBT, int CAT, int G, int LB);
 

@@ -16,6 +16,7 @@ import torch
 __all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
            "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "profile_enable", "profile_read",
+           "forward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "KERNELS", "lib"]
 
 # every kernel the library launches (names used by the profiler)
@@ -24,6 +25,7 @@ KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_kernel", "segmen
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2
+NOALLOC_SCRATCH_BYTES = 32 << 20  # SEMICRF_NOALLOC_SCRATCH_BYTES
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsemicrf_b200.so")
 if not os.path.exists(library_path):
@@ -47,9 +49,10 @@ lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
 lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
+lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _vp]
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
-for _f in ("semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+for _f in ("semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_get_status",
            "semicrf_selftest_bounded_wait"):
     getattr(lib, _f).restype = _i
@@ -236,3 +239,23 @@ def profile_read(kernel: str):
     _check(lib.semicrf_profile_read(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)),
            "semicrf_profile_read")
     return float(ms.value), int(n.value)
+
+
+def forward_noalloc(em, lengths, trans, dur, center: bool = True, logZ=None):
+    """log Z [B] (float64) through semicrf_forward_noalloc: no workspace, no
+    allocation inside the library (the output tensor is allocated here unless
+    passed).  Raises SemiCRFError(SEMICRF_ERR_UNSUPPORTED) when the problem
+    does not fit the library's fixed scratch array."""
+    dev = em.device
+    _need(em, torch.float32, "em", dev)
+    _need(lengths, torch.int32, "lengths", dev)
+    _need(trans, torch.float32, "trans", dev)
+    _need(dur, torch.float32, "dur", dev)
+    B, T, C = em.shape
+    K = dur.shape[0]
+    if logZ is None:
+        logZ = torch.empty(B, dtype=torch.float64, device=dev)
+    _check(lib.semicrf_forward_noalloc(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K,
+                                       _flags(center, True), _ptr(logZ), _stream(dev)),
+           "semicrf_forward_noalloc")
+    return logZ

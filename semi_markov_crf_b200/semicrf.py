@@ -190,8 +190,10 @@ def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool
     return o
 
 
-def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None = None):
-    """Step 4: (score [B] float64, labels [B,T] int32, seg_start [B,T] uint8)."""
+def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None = None,
+            out=None):
+    """Step 4: (score [B] float64, labels [B,T] int32, seg_start [B,T] uint8).
+    ``out`` may supply that triple preallocated."""
     dev = em.device
     _need(em, torch.float32, "em", dev)
     _need(lengths, torch.int32, "lengths", dev)
@@ -202,9 +204,15 @@ def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None =
     flags = _flags(center)
     if ws is None or not ws.matches(B, T, C, K, flags):
         ws = Workspace(B, T, C, K, flags, dev)
-    score = torch.empty(B, dtype=torch.float64, device=dev)
-    labels = torch.empty((B, T), dtype=torch.int32, device=dev)
-    seg = torch.empty((B, T), dtype=torch.uint8, device=dev)
+    if out is None:
+        score = torch.empty(B, dtype=torch.float64, device=dev)
+        labels = torch.empty((B, T), dtype=torch.int32, device=dev)
+        seg = torch.empty((B, T), dtype=torch.uint8, device=dev)
+    else:
+        score, labels, seg = out
+        _need(score, torch.float64, "score", dev)
+        _need(labels, torch.int32, "labels", dev)
+        _need(seg, torch.uint8, "seg_start", dev)
     _check(lib.semicrf_viterbi(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, flags,
                                ws.ptr, ws.nbytes, _ptr(score), _ptr(labels), _ptr(seg), _stream(dev)),
            "semicrf_viterbi")

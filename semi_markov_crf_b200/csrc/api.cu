@@ -106,7 +106,8 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   d.prefR = std::max(16, pow2floor(8192 / C));
   d.nchunk = T > 0 ? (T + d.prefR - 1) / d.prefR : 1;
   d.store_w = 2 * C + 2;
-  const size_t budget = (size_t)max_smem_optin();
+  // the per-block limit covers static shared memory too (a few bytes here)
+  const size_t budget = (size_t)max_smem_optin() - 256;
   d.store_smem = recursion_smem_bytes(d, true) <= budget ? 1 : 0;
   if (recursion_smem_bytes(d, false) > budget) return SEMICRF_ERR_UNSUPPORTED;
   return SEMICRF_OK;

@@ -3,12 +3,15 @@
 //
 // The checkpoint segments leave, for every position u of segment j, the
 // suffix sum v[u, c] = sum_{u < s < t1_j} (start_marg[s,c] - end_marg[s,c]) in
-// the grad_em buffer, plus per segment the total T_j[c] of (start - end) and
-// V_j[c] = sum_u v[u, c].  Then
+// the grad_em buffer, plus per segment P_j[c] = mu[t0_j - 1, c] + the total
+// of (start - end) over the segment (mu[t0_j - 1] from the segment's cut
+// normaliser, 0 for j = 0) and V_j[c] = sum_u v[u, c].  Then
 //   pos_marg[u, c] = sum_{s <= u} (start_marg[s,c] - end_marg[s,c])
-//                  = sum_{j' <= j} T_j'[c] - v[u, c]
+//                  = P_j[c] - v[u, c]
 // (a position lies in a label-c segment iff one started at or before it and
-// none of those ended at or before it), and with centering the emission
+// none of those ended at or before it); taking the carry from the cut rather
+// than summing earlier segments' totals keeps every segment independent of
+// the others' rounding.  With centering the emission
 // gradient is g_b * (pos_marg[u,c] - mean_v pos_marg[v,c]) (the Jacobian of
 // subtracting the per-label mean; "Emission Baseline Centering", explainer
 // section 2).
@@ -43,7 +46,7 @@ __global__ void __launch_bounds__(256)
     double run = 0.0, msum = 0.0;
     for (int j = 0; j < nseg; ++j) {
       const size_t o = ((size_t)b * d.nck + j) * C + c;
-      run += ws.segT[o];
+      run = ws.segT[o];
       const int len = min((j + 1) * delta, L) - j * delta;
       msum += (double)len * run - ws.segV[o];
       if (j >= j_lo && j <= j_hi) pinc[(j - j_lo) * C + c] = run;

@@ -99,6 +99,87 @@ __device__ __forceinline__ void bwd_checkpoint(const Smem& sm, const Dims& d, co
   __syncthreads();
 }
 
+// Local normaliser of checkpoint segment j >= 1, from the cut at position
+// u = t0 - 1 (t0 = j Delta): every segmentation has exactly one segment
+// [s, t) with s <= u < t, so
+//   Z = sum_{c, s < t0 <= t, t - s <= K} 2^(gamma[s,c] - S[s,c]) 2^(dur2[t-s-1,c]) 2^(S[t,c] + beta[t,c])
+// and the share of label c in that sum is mu[u, c].  Both factors come from
+// the rings the two chains saved at boundary t0: the forward ring (boundaries
+// t0-K..t0-1, an entry (x, y) encoding gamma - S = x + y + F0 - S_int[t0]) and
+// the backward ring (boundaries t0..t0+K-1, beta + S = x + y + G0 + S_int[t0]);
+// the S_int[t0] cancel.  Normalising the segment's posteriors by this Z, which
+// is built from the very forward and backward values the segment restarts
+// from, keeps them exact however far rounding has carried the chains (and
+// their log Z) over the positions before t0 and after t1.
+// Returns log2 Z (float64) to every thread and leaves mu[u, c] in sm.tmp[c].
+// Uses the ring area as scratch; starts and ends with a barrier.
+__device__ double segment_cut(const Smem& sm, const Dims& d, const WsPtrs& ws, int b, int j, int L,
+                              const float* __restrict__ dur, double* lz_out) {
+  const int C = d.C, K = d.K, t0 = j * d.delta;
+  const size_t seg = (size_t)b * d.nck + j;
+  const float2* fa = ws.ack + seg * K * C;        // boundary t0 - K + i
+  const float2* fb = ws.bck + (seg - 1) * K * C;  // boundary t0 + i
+  float2* bs = sm.ring;                           // staged [c][K] backward entries
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < K * C; idx += blockDim.x) {
+    const int i = idx / C, c = idx % C;
+    bs[(size_t)c * K + i] = (t0 + i <= L) ? fb[idx] : make_float2(NEG_INF, 0.f);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int kb_max = min(K - 1, L - t0);  // t - t0 <= K - 1 and t <= L
+  for (int c = threadIdx.x >> 5; c < C; c += nw) {
+    const float2* bc = bs + (size_t)c * K;
+    float zmax = NEG_INF;
+    for (int ia = lane; ia < K; ia += 32) {
+      if (t0 - K + ia < 0) continue;
+      const float2 a = fa[(size_t)ia * C + c];
+      const int kbe = min(ia, kb_max);  // t = t0 + kb <= s + K = t0 + ia
+      for (int kb = 0; kb <= kbe; ++kb) {
+        const float2 v = bc[kb];
+        const float dk = __ldg(dur + (size_t)(kb + K - ia - 1) * C + c) * l2e();
+        zmax = fmaxf(zmax, ((a.y + v.y) + (a.x + v.x)) + dk);
+      }
+    }
+    zmax = group_max(zmax, 32);
+    const float M = (zmax == NEG_INF) ? 0.f : ceilf(zmax);
+    float sum = 0.f;
+    for (int ia = lane; ia < K; ia += 32) {
+      if (t0 - K + ia < 0) continue;
+      const float2 a = fa[(size_t)ia * C + c];
+      const int kbe = min(ia, kb_max);
+      for (int kb = 0; kb <= kbe; ++kb) {
+        const float2 v = bc[kb];
+        const float dk = __ldg(dur + (size_t)(kb + K - ia - 1) * C + c) * l2e();
+        sum += ex2((((a.y + v.y) - M) + (a.x + v.x)) + dk);
+      }
+    }
+    sum = group_sum(sum, 32);
+    if (lane == 0) {
+      sm.Acur[c] = M;                                  // exact integer shift
+      sm.tmp[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;   // log2 of the label's share
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float Mz = NEG_INF;
+    for (int c = lane; c < C; c += 32)
+      if (sm.tmp[c] != NEG_INF) Mz = fmaxf(Mz, sm.Acur[c]);
+    Mz = group_max(Mz, 32);
+    if (Mz == NEG_INF) Mz = 0.f;
+    float tot = 0.f;
+    for (int c = lane; c < C; c += 32) tot += ex2((sm.Acur[c] - Mz) + sm.tmp[c]);
+    tot = group_sum(tot, 32);
+    const float lt = (tot > 0.f) ? lg2(tot) : NEG_INF;
+    __syncwarp();
+    for (int c = lane; c < C; c += 32) sm.tmp[c] = ex2(((sm.Acur[c] - Mz) + sm.tmp[c]) - lt);
+    if (lane == 0)
+      *lz_out = (ws.acf[seg] + ws.bcf[seg - 1]) + ((double)Mz + (double)lt);
+  }
+  __syncthreads();
+  return *lz_out;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -131,11 +212,11 @@ __global__ void __launch_bounds__(LB, 1)
   Lane<KBT, CAT, G> ln;
   ln.init_ids(d);
   ln.init_dur(d, dur, is_alpha);
-  ln.init_trans(d, trans, !is_alpha);
   float2* const rl = sm.ring + (size_t)ln.cc * d.RL;  // this lane's label ring
   float e[KBT], p[CAT];
   init_smem(sm, d);
   __syncthreads();
+  ln.init_trans(d, trans, !is_alpha, block_trans_max(sm, d, trans));
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
   int par = 0, q = 0;
@@ -317,10 +398,13 @@ __global__ void __launch_bounds__(LB, 1)
 // Restores the forward ring at t0 = j*Delta and recomputes alpha over
 // [t0, t1) into a per-position store, then restores the backward ring at t1
 // and walks down to t0 accumulating the exact posteriors:
-//   start_marg[s,c] = 2^(gamma[s,c] + btil[s,c] - log2 Z)
-//   end_marg[s,c]   = 2^(alpha[s,c] + beta[s,c] - log2 Z)
+//   start_marg[s,c] = 2^(gamma[s,c] + btil[s,c] - log2 Z_j)
+//   end_marg[s,c]   = 2^(alpha[s,c] + beta[s,c] - log2 Z_j)
 //   P(segment [s, s+k), c) = start_marg[s,c] * (normalised k term of btil)
 //   P(c' -> c at s)        = end_marg[s,c'] * (normalised c term of beta)
+// Z_j is the segment's own cut normaliser (segment_cut; the backward chain's
+// log Z for j = 0): equal to Z in exact arithmetic, and made of the same
+// restored forward and backward values as the segment's posteriors.
 // The leader lane of label c's group keeps c's running sums.
 // ===========================================================================
 template <int KBT, int CAT, int G, int LB>
@@ -340,7 +424,6 @@ __global__ void __launch_bounds__(LB, 1)
   const int t1 = min(t0 + d.delta, L);
   const bool last = (t1 == L);
   const float gbf = (float)(grad_logZ ? grad_logZ[b] : 1.0);
-  const double logz2 = ws.logz2[b];
   const int SW = d.store_w;
   float* store = sm.store ? sm.store : ws.store + ((size_t)b * d.nck + j) * d.delta * SW;
   const size_t seg = (size_t)b * d.nck + j;
@@ -352,14 +435,27 @@ __global__ void __launch_bounds__(LB, 1)
   ts.ph[0] = ts.ph[1] = 0;
   double F0 = 0.0;
   float Frel = 0.f;
+  float tmax2 = 0.f;
   int par = 0, q = 0;
+
+  // Local normaliser and mu[t0 - 1, c] (left in sm.tmp).  Segment 0 starts
+  // at boundary 0, where the backward chain's own log Z is the cut.
+  __shared__ double s_lz;
+  double logz2;
+  if (j == 0) {
+    for (int c = tid; c < C; c += blockDim.x) sm.tmp[c] = 0.f;
+    logz2 = ws.logz2b[b];
+  } else {
+    logz2 = segment_cut(sm, d, ws, b, j, L, dur, &s_lz);
+  }
 
   // ------------------------------------------------------ alpha recompute
   {
     ln.init_dur(d, dur, true);
-    ln.init_trans(d, trans, false);
     init_smem(sm, d);
     __syncthreads();
+    tmax2 = block_trans_max(sm, d, trans);
+    ln.init_trans(d, trans, false, tmax2);
     int t_start, Sb;
     if (j == 0) {
       for (int c = tid; c < C; c += blockDim.x) {
@@ -467,7 +563,7 @@ __global__ void __launch_bounds__(LB, 1)
 
   // ------------------------------------------------------ beta recompute + posteriors
   ln.init_dur(d, dur, false);
-  ln.init_trans(d, trans, true);
+  ln.init_trans(d, trans, true, tmax2);
   __syncthreads();
   for (int i = tid; i < d.RL * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   __syncthreads();
@@ -609,7 +705,7 @@ __global__ void __launch_bounds__(LB, 1)
     }
   }
   if (ln.leader) {
-    ws.segT[seg * C + ln.c] = accmu;
+    ws.segT[seg * C + ln.c] = (double)sm.tmp[ln.c] + accmu;  // mu[t0 - 1] + segment total
     ws.segV[seg * C + ln.c] = vsum;
   }
 }

@@ -31,6 +31,7 @@ namespace ring {
 struct Smem {
   uint64_t* mbar;   // [2] tile barriers
   int* maxslot;     // [3] per-step max (order-preserving ints)
+  int* aux;         // [1] block-wide max of the transition scores
   int32_t* tint;    // [2][TS][C]
   float* tfrac;     // [2][TS][C]
   float2* ring;     // [C][RL]
@@ -41,12 +42,15 @@ struct Smem {
   float* store;     // [delta][store_w] (posterior kernel, when in shared memory)
 };
 
+__device__ __forceinline__ float l2e() { return (float)LOG2E_D; }
+
 __device__ __forceinline__ Smem carve(unsigned char* raw, const Dims& d, bool with_store) {
   Smem s;
   const int C = d.C;
   unsigned char* p = raw;
   s.mbar = reinterpret_cast<uint64_t*>(p);
   s.maxslot = reinterpret_cast<int*>(p + 16);
+  s.aux = reinterpret_cast<int*>(p + 32);
   p += 64;
   s.tint = reinterpret_cast<int32_t*>(p);
   p += 2ull * TS * C * sizeof(int32_t);
@@ -77,7 +81,24 @@ __device__ __forceinline__ void init_smem(const Smem& sm, const Dims& d) {
     mbar_init(&sm.mbar[1], 1);
     fence_mbar_init();
     for (int i = 0; i < 3; ++i) sm.maxslot[i] = f2ord(NEG_INF);
+    sm.aux[0] = f2ord(NEG_INF);
   }
+}
+
+// Largest transition score (base 2) over the whole C x C matrix, by every
+// thread of the block (called after init_smem's barrier; holds one barrier).
+// Both directions and every kernel scale the exp-domain transition weights
+// 2^(trans2 - M) by this same M, so the forward and backward label fan-ins
+// use bitwise the same weights: their rounding is one model, not two, and
+// the posteriors (ratios of forward, backward and log Z) see no drift
+// between the chains.  0 if nothing is finite.
+__device__ __forceinline__ float block_trans_max(const Smem& sm, const Dims& d, const float* trans) {
+  float mx = NEG_INF;
+  for (int i = threadIdx.x; i < d.C * d.C; i += blockDim.x) mx = fmaxf(mx, __ldg(trans + i) * l2e());
+  warp_max_to_shared(sm.aux, f2ord(mx));
+  __syncthreads();
+  const float m = ord2f(sm.aux[0]);
+  return isfinite(m) ? m : 0.f;
 }
 
 // Writes ring slot `slot` of one label (rl = its first entry) and its mirrors
@@ -182,7 +203,6 @@ __device__ __forceinline__ void gargmax(float& v, int& i) {
 }
 
 // ----------------------------------------------------------------------------- lanes
-__device__ __forceinline__ float l2e() { return (float)LOG2E_D; }
 
 // One lane of a label group: label c, lane j of G.  Durations of lane term i:
 //   up   (forward, terms at t - k):  k_i = (j + 1) * KBT - i
@@ -214,12 +234,11 @@ struct Lane {
       d[i] = (act && k <= dm.K) ? __ldg(dur + (size_t)(k - 1) * dm.C + cc) * l2e() : NEG_INF;
     }
   }
-  __device__ __forceinline__ void init_trans(const Dims& dm, const float* trans, bool rows) {
+  // e[i] = 2^(trans2 - mx) for this lane's CAT sources (rows: trans[c][x],
+  // else trans[x][c]); mx is block_trans_max, the same in every kernel.
+  __device__ __forceinline__ void init_trans(const Dims& dm, const float* trans, bool rows,
+                                             float mx) {
     const int C = dm.C;
-    float mx = NEG_INF;
-    for (int x = 0; x < C; ++x)
-      mx = fmaxf(mx, __ldg(trans + (rows ? (size_t)cc * C + x : (size_t)x * C + cc)) * l2e());
-    if (mx == NEG_INF) mx = 0.f;
     tmax = mx;
 #pragma unroll
     for (int i = 0; i < CAT; ++i) {

@@ -43,7 +43,10 @@ WORKLOAD = "speech"
 METRIC = "semi-CRF fwd+bwd edge evals/s (B·T·K·C²), positions/s, peak HBM, % roofline"
 UNIT = "edge evals/s"
 MUFU_PER_SM_PER_CLK = 16          # ex2/lg2 results per SM per clock (SFU)
+FP32_PER_SM_PER_CLK = 128         # fp32 lanes per SM per clock (4 partitions x 32)
 L2_BYTES = 126 * 1024 * 1024
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "semi_markov_crf_b200", "csrc")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -91,6 +94,63 @@ def mufu_ops_per_position(kernel: str, K: int, C: int) -> int:
     if kernel == "segment_kernel":
         return 2 * one_ring + 2 * C
     return 0
+
+
+def alu_ops_per_position(kernel: str, K: int, C: int) -> int:
+    """Algorithmic fp32 operations per position of the max-semiring kernel:
+    one add and one max per (duration, label) term of the k fan-in and per
+    (label, label) term of the label fan-in."""
+    if kernel == "viterbi_kernel":
+        return 2 * (K * C + C * C)
+    return 0
+
+
+def csrc_digest() -> str:
+    """sha256 over the kernel sources, to tie a stored ncu traffic figure to
+    the build it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summary, or None when it was taken on other kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("csrc_sha256") != csrc_digest() or t.get("workload") != WORKLOAD:
+        return None
+    return t.get("kernels", {}).get(kernel)
+
+
+def kernel_roofline(name: str, info: dict, K: int, C: int, positions: int, steps: int,
+                    sm_count: int, sm_max_mhz: float) -> dict | None:
+    """Roofline entry of one kernel: algorithmic ops per launch over its mean
+    launch time, against the unit that bounds it (MUFU for the log-semiring
+    kernels, fp32 lanes for Viterbi).  None for the O(T C) HBM kernels."""
+    mufu = mufu_ops_per_position(name, K, C)
+    alu = alu_ops_per_position(name, K, C)
+    if mufu:
+        per_clk, ops_pos, what = MUFU_PER_SM_PER_CLK, mufu, "MUFU ops/clk"
+    elif alu:
+        per_clk, ops_pos, what = FP32_PER_SM_PER_CLK, alu, "fp32 lanes/clk"
+    else:
+        return None
+    peak = sm_count * per_clk * sm_max_mhz * 1e6
+    per_launch = ops_pos * positions / (info["launches"] / steps)
+    achieved = per_launch / (info["ms_per_launch"] * 1e-3)
+    return {"bound": "alu", "kernel": name, "achieved": achieved / 1e9, "peak": peak / 1e9,
+            "unit": "Gop/s", "frac": achieved / peak, "traffic": stored_traffic(name),
+            "peak_source": f"derived: {sm_count} SMs x {per_clk} {what} x {sm_max_mhz:.0f} MHz "
+                           f"(sm_max_mhz of MEASURED_PEAKS.json)",
+            "ops_per_launch": per_launch}
 
 
 class ClockSampler:
@@ -350,18 +410,12 @@ def run_ours(args):
         sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
         sm_max = float(peaks.get("sm_max_mhz", 1965.0))
         mufu_peak = sm_count * MUFU_PER_SM_PER_CLK * sm_max * 1e6      # ops/s
+        roofs = {k: kernel_roofline(k, v, K, C, positions, args.steps, sm_count, sm_max)
+                 for k, v in kern.items()}
+        roofs = {k: v for k, v in roofs.items() if v}
+        # the dominant kernel: the largest share of device time
         dom = max(kern, key=lambda k: kern[k]["ms_total"]) if kern else None
-        roof = None
-        if dom:
-            ops = mufu_ops_per_position(dom, K, C) * positions
-            per_launch = ops / (kern[dom]["launches"] / args.steps)
-            achieved = per_launch / (kern[dom]["ms_per_launch"] * 1e-3)
-            roof = {"bound": "alu", "kernel": dom, "achieved": achieved / 1e9,
-                    "peak": mufu_peak / 1e9, "unit": "Gop/s", "frac": achieved / mufu_peak,
-                    "traffic": None,
-                    "peak_source": f"derived: {sm_count} SMs x {MUFU_PER_SM_PER_CLK} MUFU ops/clk x "
-                                   f"{sm_max:.0f} MHz (sm_max_mhz of MEASURED_PEAKS.json)",
-                    "ops_per_launch": per_launch}
+        roof = roofs.get(dom)
         step_ops = (mufu_ops_per_position("chain_kernel", K, C) +
                     mufu_ops_per_position("segment_kernel", K, C)) * positions
         value = edges * world / (ms_step * 1e-3)
@@ -383,6 +437,8 @@ def run_ours(args):
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "step_mufu_frac": step_ops / (ms_step * 1e-3) / mufu_peak,
             "roofline": roof,
+            "roofline_all": {k: {"frac": v["frac"], "achieved": v["achieved"], "peak": v["peak"]}
+                             for k, v in roofs.items()},
             "e2e": {"value": edges * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "results_checked": bool(ok)},

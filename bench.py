@@ -89,7 +89,7 @@ def mufu_ops_per_position(kernel: str, K: int, C: int) -> int:
     recomputes both over its segment and adds 2C exponentials for the start
     and end marginals.  Viterbi uses no MUFU."""
     one_ring = K * C + 3 * C
-    if kernel == "chain_kernel":
+    if kernel in ("chain_kernel", "chain_exp_kernel"):
         return 2 * one_ring
     if kernel == "segment_kernel":
         return 2 * one_ring + 2 * C
@@ -137,6 +137,8 @@ def kernel_roofline(name: str, info: dict, K: int, C: int, positions: int, steps
     kernels, fp32 lanes for Viterbi).  None for the O(T C) HBM kernels."""
     mufu = mufu_ops_per_position(name, K, C)
     alu = alu_ops_per_position(name, K, C)
+    if positions <= 0:
+        return None
     if mufu:
         per_clk, ops_pos, what = MUFU_PER_SM_PER_CLK, mufu, "MUFU ops/clk"
     elif alu:
@@ -329,6 +331,12 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if semicrf.get_status(ws) != 0:
         raise RuntimeError(f"device status {semicrf.get_status(ws)}")
+    # which kernel ran each ring (both ring kernels launch every step; each
+    # takes its own sequences): positions per ring kernel, both directions
+    dom = semicrf.ring_domains(ws)
+    lens = [int(x) for x in w["lengths"]]
+    ring_pos = {"chain_exp_kernel": sum(lens[i % B] for i, m in enumerate(dom) if m == 1) / 2,
+                "chain_kernel": sum(lens[i % B] for i, m in enumerate(dom) if m == 2) / 2}
 
     stream = torch.cuda.current_stream(dev)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -410,7 +418,8 @@ def run_ours(args):
         sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
         sm_max = float(peaks.get("sm_max_mhz", 1965.0))
         mufu_peak = sm_count * MUFU_PER_SM_PER_CLK * sm_max * 1e6      # ops/s
-        roofs = {k: kernel_roofline(k, v, K, C, positions, args.steps, sm_count, sm_max)
+        roofs = {k: kernel_roofline(k, v, K, C, ring_pos.get(k, positions), args.steps,
+                                    sm_count, sm_max)
                  for k, v in kern.items()}
         roofs = {k: v for k, v in roofs.items() if v}
         # the dominant kernel: the largest share of device time

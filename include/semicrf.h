@@ -80,6 +80,11 @@ enum semicrf_status {
 #define SEMICRF_FLAG_NO_CENTER 0x1u    /* use raw emissions (nu = 0) */
 #define SEMICRF_FLAG_FORWARD_ONLY 0x2u /* forward skips the backward ring (inference);
                                           a backward given the same flag runs it itself */
+#define SEMICRF_FLAG_LOG_DOMAIN 0x4u   /* run the rings in the log domain for every
+                                          sequence (by default a sequence whose scores
+                                          keep every step within float32's exponent
+                                          range runs in the faster exponential domain;
+                                          results agree to rounding) */
 
 /*
  * Bytes of device workspace needed by forward/backward/viterbi for these
@@ -161,6 +166,16 @@ SEMICRF_API int semicrf_viterbi(const float *em, const int32_t *lengths, const f
  * Forward and viterbi reset the word when they start.
  */
 SEMICRF_API int semicrf_get_status(const void *ws, semicrf_stream_t stream, int *status);
+
+/*
+ * Which arithmetic ran each ring of the last forward (or forward-only
+ * backward) on this workspace: synchronises `stream` and copies 2*B host ints
+ * into `domains` -- [0, B) the forward rings, [B, 2B) the backward rings --
+ * each 1 (exponential domain), 2 (log domain) or 0 (not run).  (B, T, C, K,
+ * flags) must be those of that call.  Diagnostic; nothing else depends on it.
+ */
+SEMICRF_API int semicrf_ring_domains(const void *ws, size_t ws_bytes, int B, int T, int C, int K,
+                                     unsigned flags, semicrf_stream_t stream, int32_t *domains);
 
 /* Human-readable name of a status code (static string, never NULL). */
 SEMICRF_API const char *semicrf_strerror(int code);

@@ -51,6 +51,51 @@ int max_smem_optin() {
 
 }  // namespace
 
+// Shape of the pipelined exponential-domain rings (xG = 0: none fits, every
+// sequence takes the log-domain kernel).  The step's latency is the longer of
+// the combine path (CAT multiply-adds, log2 G shuffle levels) and the helper
+// path (KBH exponentials, log2 H shuffle levels), plus issue time for the
+// warps that share a scheduler.  SEMICRF_XSHAPE=i forces the i-th fitting
+// shape of the menu (tuning).
+void choose_xshape(Dims& d, size_t budget) {
+  const int C = d.C, K = d.K;
+  int forced = -1;
+  if (const char* env = std::getenv("SEMICRF_XSHAPE")) forced = std::atoi(env);
+  d.xG = 0;
+  double best = 1e30;
+  int idx = 0;
+  auto lg = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+#define SEMICRF_XCONSIDER(g, cat, h, kbh, lb)                                             \
+  {                                                                                       \
+    const int nwc = (C + 32 / g - 1) / (32 / g), nwh = (C + 32 / h - 1) / (32 / h);       \
+    const int nt = 32 * (nwc + nwh);                                                      \
+    if (C <= g * cat && K <= h * kbh + 2 && nt <= lb) {                                   \
+      const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +        \
+                          10.0 * ((nwc + nwh + 3) / 4);                                   \
+      if ((forced < 0 && cost < best) || forced == idx) {                                 \
+        best = cost;                                                                      \
+        d.xG = g;                                                                         \
+        d.xCAT = cat;                                                                     \
+        d.xH = h;                                                                         \
+        d.xKBH = kbh;                                                                     \
+        d.xLB = lb;                                                                       \
+        d.xNT = nt;                                                                       \
+      }                                                                                   \
+      ++idx;                                                                              \
+    }                                                                                     \
+  }
+  SEMICRF_FOR_EACH_XSHAPE(SEMICRF_XCONSIDER)
+#undef SEMICRF_XCONSIDER
+  if (d.xG == 0) return;
+  d.xRL = K + d.xKBH;
+  d.xPC = d.xG * d.xCAT;
+  if (chain_exp_smem_bytes(d) > budget) d.xG = 0;
+}
+
 // Sizes, lane mapping and limits.  Returns a semicrf_status.
 int make_dims(int B, int T, int C, int K, Dims& d) {
   if (B < 0 || T < 0 || C < 1 || K < 1) return SEMICRF_ERR_INVALID_ARG;
@@ -110,6 +155,7 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   const size_t budget = (size_t)max_smem_optin() - 256;
   d.store_smem = recursion_smem_bytes(d, true) <= budget ? 1 : 0;
   if (recursion_smem_bytes(d, false) > budget) return SEMICRF_ERR_UNSUPPORTED;
+  choose_xshape(d, budget);
   return SEMICRF_OK;
 }
 
@@ -140,6 +186,8 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_segT = take(B * nck * C * 8);
   const size_t o_segV = take(B * nck * C * 8);
   const size_t o_bp = take(B * (size_t)(d.T + 1) * C * 4);
+  const size_t o_emax = take(B * 4);
+  const size_t o_mode = take(2 * B * 4);
   if (base && p) {
     char* c = static_cast<char*>(base);
     p->status = reinterpret_cast<int*>(c + o_status);
@@ -158,11 +206,14 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segT = reinterpret_cast<double*>(c + o_segT);
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
+    p->emax = reinterpret_cast<float*>(c + o_emax);
+    p->mode = reinterpret_cast<int*>(c + o_mode);
   }
   return off;
 }
 
-constexpr unsigned KNOWN_FLAGS = SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY;
+constexpr unsigned KNOWN_FLAGS =
+    SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY | SEMICRF_FLAG_LOG_DOMAIN;
 
 int prepare(int B, int T, int C, int K, unsigned flags, void* ws, size_t ws_bytes, Dims& d,
             WsPtrs& p) {
@@ -225,6 +276,27 @@ struct ProfScope {
     prof_recs.push_back(rec);
   }
 };
+
+// Both rings (forward of n_alpha sequences, backward of n_beta): the
+// exponential-domain kernel takes every sequence whose scores fit it and
+// marks the rest, which the log-domain kernel then runs.
+int run_chains(const Dims& d, WsPtrs p, const int32_t* lengths, const float* trans,
+               const float* dur, double* logZ, int n_alpha, int n_beta, unsigned flags,
+               cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  if (d.xG && !(flags & SEMICRF_FLAG_LOG_DOMAIN)) {
+    ProfScope ps("chain_exp_kernel", st);
+    e = launch_chain_exp(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st);
+  } else {
+    p.mode = nullptr;  // the log-domain kernel runs every sequence
+  }
+  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+  {
+    ProfScope ps("chain_kernel", st);
+    e = launch_chain(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st);
+  }
+  return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
+}
 
 int run_prefix(const float* em, const int32_t* lengths, const Dims& d, const WsPtrs& p,
                unsigned flags, int mode, double* S64, float* nu, cudaStream_t st) {
@@ -294,12 +366,7 @@ extern "C" int semicrf_forward(const float* em, const int32_t* lengths, const fl
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
   if (rc) return rc;
   const int nbeta = (flags & SEMICRF_FLAG_FORWARD_ONLY) ? 0 : B;
-  cudaError_t e;
-  {
-    ProfScope ps("chain_kernel", st);
-    e = launch_chain(d, p, lengths, trans, dur, logZ, B, nbeta, st);
-  }
-  return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
+  return run_chains(d, p, lengths, trans, dur, logZ, B, nbeta, flags, st);
 }
 
 extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, const float* dur,
@@ -321,12 +388,8 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     return SEMICRF_OK;
   }
   if (flags & SEMICRF_FLAG_FORWARD_ONLY) {
-    cudaError_t e;
-    {
-      ProfScope ps("chain_kernel", st);
-      e = launch_chain(d, p, lengths, trans, dur, nullptr, 0, B, st);
-    }
-    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    rc = run_chains(d, p, lengths, trans, dur, nullptr, 0, B, flags, st);
+    if (rc) return rc;
   }
   if (T > 0) {
     cudaError_t e;
@@ -393,6 +456,26 @@ extern "C" int semicrf_get_status(const void* ws, semicrf_stream_t stream, int* 
       cudaStreamSynchronize(st) != cudaSuccess)
     return SEMICRF_ERR_CUDA;
   *status = v;
+  return SEMICRF_OK;
+}
+
+extern "C" int semicrf_ring_domains(const void* ws, size_t ws_bytes, int B, int T, int C, int K,
+                                    unsigned flags, semicrf_stream_t stream, int32_t* domains) {
+  if (!domains) return SEMICRF_ERR_INVALID_ARG;
+  Dims d;
+  WsPtrs p;
+  const int rc = prepare(B, T, C, K, flags, const_cast<void*>(ws), ws_bytes, d, p);
+  if (rc) return rc;
+  if (B == 0) return SEMICRF_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(domains, p.mode, 2ull * B * sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SEMICRF_ERR_CUDA;
+  // a run without the exponential-domain kernel leaves the array untouched:
+  // report those rings as log domain
+  if (!d.xG || (flags & SEMICRF_FLAG_LOG_DOMAIN))
+    for (int i = 0; i < 2 * B; ++i) domains[i] = 2;
   return SEMICRF_OK;
 }
 

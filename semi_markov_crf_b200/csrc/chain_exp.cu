@@ -1,0 +1,491 @@
+// chain_exp.cu -- steps 2 and 3: the forward and backward rings with the
+// label fan-in in the exponential domain on the critical path and the long
+// part of the duration fan-in computed one step ahead.
+//
+// "Streaming Structured Inference with Flash-SemiCRF", explainer section 2,
+// "Streaming Forward-Backward with Ring Buffers".  The recursion is the one of
+// chain_kernel (recursion.cu), in base-2 log units:
+//   gamma[s, c] = LSE_{c'} alpha[s, c'] + trans[c', c]             (gamma[0] = 0)
+//   alpha[t, c] = S[t,c] + LSE_{k <= min(K,t)} gamma[t-k, c] - S[t-k, c] + dur[k-1, c]
+// with the backward mirror (btil after the k fan-in, beta after the label
+// fan-in).  What one step really waits for is small: only the k = 1 term of
+// alpha[t] needs gamma[t-1], which needs the whole vector alpha[t-1, :].
+// The kernel is organised around that dependency.
+//
+// Representation.  Step t keeps the label vector in the exponential domain,
+//   p_t[c] = 2^(alpha[t, c] - Phi_t),   Phi_t = Phi_{t-1} + n_t  (integers),
+// with n_t the binary exponent of max_c p_{t-1}[c]: Phi_t follows max alpha[t-1]
+// one step late, so no reduction sits on the critical path.  With
+//   acc_s[c] = sum_{c'} p_s[c'] * 2^(trans2[c', c] - M)          (M = max trans2)
+// we have gamma[s, c] = Phi_s + M + log2 acc_s[c] (acc_0 = 2^-M, Phi_0 = 0), and
+//   p_t = 2^-n_t * ( acc_{t-1} A1 + acc_{t-2} A2 2^-n_{t-1} + O_t 2^(Z_t + sf_t - n_{t-1}) )
+//   A1 = 2^(M + dur2[0] + S[t] - S[t-1]),  A2 = 2^(M + dur2[1] + S[t] - S[t-2]),
+// where O_t 2^(Z_t + sf_t) is the k >= 3 part of the duration sum relative to
+// Phi_{t-2}.  Everything but acc_{t-1} and n_t is known when step t begins, so
+// the critical path of a step is: read p_{t-1} -> dot product with the
+// transition weights -> one multiply-add -> store p_t -> barrier.
+//
+// Roles.  Combine warps (xG lanes per label, xCAT weights per lane) run that
+// path, keep acc_{t-2} and the rolling prefix-sum rows in registers, publish
+// n_t, and write gamma[t-1] into the label's ring in the log domain (off the
+// critical path; exactly the entry format of chain_kernel, so checkpoints and
+// the posterior kernel are shared).  Helper warps (xH lanes per label, xKBH
+// durations each) compute O_{t+1} for every label during step t from ring
+// entries of boundaries <= t-2 -- the same predicted-shift k fan-in as
+// chain_kernel -- and publish it before the step's barrier.  One CTA barrier
+// per step orders everything.
+//
+// Exactness.  The exponential domain is exact up to float32 rounding while
+// every label's alpha stays within fp32's exponent range of the frame.  Per
+// step, alpha[t, c] - max alpha[t-1] lies in
+//   [tmin + dmin - e, log2(K C) + max(tmax + dmax, dmax - dmin) + e]
+// (tmin/tmax, dmin/dmax: ranges of the finite transition and duration scores,
+// e: the largest |centred emission|), so the kernel takes a sequence only when
+// all scores are finite and that span is below FAST_BOUND; otherwise it
+// records mode 2 and chain_kernel (log domain, any input) runs the sequence.
+#include "ring.cuh"
+
+namespace semicrf {
+
+using namespace ring;
+
+namespace {
+
+constexpr float FAST_BOUND = 100.f;  // log2 units of exponent head-room (fp32 has 126)
+
+struct XSmem {
+  Smem s;      // mbar, tint, tfrac, ring (tile stream and ring helpers)
+  float* P;    // [2][xPC] exp-domain label vector, by step parity
+  float* Oh;   // [2][C]   helper sums for the step of that parity
+  float* Zh;   // [2][C]   their integer shifts
+  float* nsl;  // [2]      frame step n published by the combine warps
+  int* aux;    // [4]      block reductions
+  int* Sb;     // [C]      label integer bases of the prefix sums
+};
+
+__device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
+  XSmem x;
+  const int C = d.C;
+  unsigned char* p = raw;
+  x.s.mbar = reinterpret_cast<uint64_t*>(p);
+  x.s.maxslot = reinterpret_cast<int*>(p + 16);
+  x.aux = reinterpret_cast<int*>(p + 32);
+  x.s.aux = x.aux;
+  x.nsl = reinterpret_cast<float*>(p + 48);
+  p += 64;
+  x.s.tint = reinterpret_cast<int32_t*>(p);
+  p += 2ull * TS * C * sizeof(int32_t);
+  x.s.tfrac = reinterpret_cast<float*>(p);
+  p += 2ull * TS * C * sizeof(float);
+  x.s.ring = reinterpret_cast<float2*>(p);
+  p += (size_t)d.xRL * C * sizeof(float2);
+  p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
+  float* f = reinterpret_cast<float*>(p);
+  x.P = f;
+  f += 2 * d.xPC;
+  x.Oh = f;
+  f += 2 * C;
+  x.Zh = f;
+  f += 2 * C;
+  x.Sb = reinterpret_cast<int*>(f);
+  x.s.pcur = nullptr;
+  x.s.Acur = nullptr;
+  x.s.tmp = nullptr;
+  x.s.Sbase = x.Sb;
+  x.s.store = nullptr;
+  return x;
+}
+
+// Block-wide max of f(i) over i < n (all threads; one barrier; aux slot must
+// hold f2ord(-inf) beforehand and is left holding the result).
+template <typename F>
+__device__ __forceinline__ float block_max(int* slot, int n, F f) {
+  float m = NEG_INF;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, f(i));
+  warp_max_to_shared(slot, f2ord(m));
+  __syncthreads();
+  return ord2f(*slot);
+}
+
+// 2^-n for an integer-valued n in [-126, 127] (exact, no rounding).
+__device__ __forceinline__ float pow2_neg(float n) {
+  return __int_as_float((127 - (int)n) << 23);
+}
+
+// Binary exponent of a positive normal float (0 for 0).
+__device__ __forceinline__ float exponent_of(float x) {
+  return x > 0.f ? (float)(((__float_as_int(x) >> 23) & 0xff) - 127) : 0.f;
+}
+
+// Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
+__device__ __forceinline__ bool xtile_wait(const Smem& sm, TileStream& ts, int ti) {
+  const int buf = ti & 1;
+  bool ok = mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
+  ts.ph[buf] ^= 1u;
+  return !__syncthreads_or(!ok);
+}
+
+// Row r is the first one a walk in direction `up` meets in its tile.
+__device__ __forceinline__ bool first_in_tile(int r, bool up) {
+  return up ? (r % TS) == 0 : (r % TS) == TS - 1;
+}
+
+// ===========================================================================
+// One CTA per (direction, sequence): blockIdx.x < n_alpha runs the forward
+// ring of sequence blockIdx.x, the others the backward ring of sequence
+// blockIdx.x - n_alpha.  Writes mode[direction][b]; returns at once (mode 2)
+// when the sequence needs the log-domain kernel.
+// ===========================================================================
+template <int G, int CAT, int H, int KBH, int LB>
+__global__ void __launch_bounds__(LB, 1)
+    chain_exp_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                     const float* __restrict__ trans, const float* __restrict__ dur,
+                     double* __restrict__ logZ_out, int n_alpha) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const XSmem xs = xcarve(smem_raw, d);
+  const Smem& sm = xs.s;
+  const int C = d.C, K = d.K, tid = threadIdx.x;
+  const bool up = (int)blockIdx.x < n_alpha;
+  const int b = up ? blockIdx.x : blockIdx.x - n_alpha;
+  const int L = lengths[b];
+  int* const mode = ws.mode + (up ? 0 : d.B) + b;
+  if (L < 0 || L > d.T || L == 0) {
+    if (tid == 0) {
+      const double v = (L == 0) ? 0.0 : __longlong_as_double(0x7ff8000000000000ll);
+      if (L != 0) set_status(ws.status, ST_BAD_LENGTH);
+      if (up) {
+        logZ_out[b] = v;
+        ws.logz2[b] = v;
+      } else {
+        ws.logz2b[b] = v;
+      }
+      *mode = 1;
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- the fast-path test
+  if (tid < 4) xs.aux[tid] = f2ord(NEG_INF);
+  bool bad = false;
+  for (int i = tid; i < C * C; i += blockDim.x) bad |= !isfinite(__ldg(trans + i));
+  for (int i = tid; i < K * C; i += blockDim.x) bad |= !isfinite(__ldg(dur + i));
+  bad = __syncthreads_or(bad);  // also orders the aux reset
+  const float M = block_max(&xs.aux[0], C * C, [&](int i) { return __ldg(trans + i) * l2e(); });
+  const float tmin = -block_max(&xs.aux[1], C * C, [&](int i) { return -__ldg(trans + i) * l2e(); });
+  const float dmax = block_max(&xs.aux[2], K * C, [&](int i) { return __ldg(dur + i) * l2e(); });
+  const float dmin = -block_max(&xs.aux[3], K * C, [&](int i) { return -__ldg(dur + i) * l2e(); });
+  const float span = fabsf(M) + (M - tmin) + fabsf(dmax) + fabsf(dmin) + 2.f * ws.emax[b] +
+                     lg2((float)(K * C));
+  if (bad || !(span < FAST_BOUND)) {
+    if (tid == 0) *mode = 2;
+    return;
+  }
+  if (tid == 0) *mode = 1;
+
+  // ---------------------------------------------------------------- roles
+  constexpr int LPWC = 32 / G, LPWH = 32 / H;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nwc = (C + LPWC - 1) / LPWC;
+  const bool comb = warp < nwc;
+  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
+  const int jl = comb ? lane % G : lane % H;
+  const bool act = c < C;
+  const int cc = act ? c : 0;
+  const bool leader = act && jl == 0;
+  const float sg = up ? 1.f : -1.f;
+  const int RL = d.xRL;
+  float2* const rl = sm.ring + (size_t)cc * RL;
+  // writes ring slot `slot` of this label and its mirrors (slot + mK < RL)
+  auto put = [&](int slot, float2 v) {
+    rl[slot] = v;
+    if (slot < KBH)
+      for (int x = slot + K; x < RL; x += K) rl[x] = v;
+  };
+
+  // One register array serves both roles: combine lanes keep the transition
+  // weights 2^(trans2 - M) of their CAT source labels (up: trans[x][c], down:
+  // trans[c][x]); helper lanes the durations of their window, k = 3 + jl*KBH
+  // + q (down) or k = 2 + (jl+1)*KBH - q (up), -inf beyond K.
+  constexpr int NR = CAT > KBH ? CAT : KBH;
+  float w[NR];
+  float d1 = NEG_INF, d2 = NEG_INF;
+  if (comb) {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int x = jl * CAT + q;
+      w[q] = (q < CAT && act && x < C)
+                 ? ex2(__ldg(trans + (up ? (size_t)x * C + cc : (size_t)cc * C + x)) * l2e() - M)
+                 : 0.f;
+    }
+    d1 = __ldg(dur + cc) * l2e();
+    if (K >= 2) d2 = __ldg(dur + C + cc) * l2e();
+  } else {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int k = up ? 2 + (jl + 1) * KBH - q : 3 + jl * KBH + q;
+      w[q] = (q < KBH && act && k <= K) ? __ldg(dur + (size_t)(k - 1) * C + cc) * l2e() : NEG_INF;
+    }
+  }
+
+  // ---------------------------------------------------------------- shared state
+  for (int i = tid; i < d.xRL * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  for (int i = tid; i < 2 * d.xPC; i += blockDim.x) xs.P[i] = 0.f;
+  for (int i = tid; i < 2 * C; i += blockDim.x) {
+    xs.Oh[i] = 0.f;
+    xs.Zh[i] = 0.f;
+  }
+  if (tid == 0) {
+    xs.nsl[0] = xs.nsl[1] = 0.f;
+    mbar_init(&sm.mbar[0], 1);
+    mbar_init(&sm.mbar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int r0 = up ? 0 : L;  // the walk's start boundary
+  TileStream ts;
+  ts.ph[0] = ts.ph[1] = 0;
+  ts.lo = 0;
+  ts.hi = L / TS;
+  ts.dir = up ? 1 : -1;
+  tile_issue(sm, d, ws, b, ts, r0 / TS);
+  tile_issue(sm, d, ws, b, ts, r0 / TS + ts.dir);
+  bool ok = xtile_wait(sm, ts, r0 / TS);
+  const int r1 = up ? 1 : L - 1;
+  if (ok && r1 / TS != r0 / TS) ok = xtile_wait(sm, ts, r1 / TS);
+  if (!ok) {
+    if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+    tile_drain(sm, ts);
+    return;
+  }
+  {
+    const size_t o0 = tile_row_off(r0, C);
+    for (int x = tid; x < C; x += blockDim.x) {
+      // gamma[0] = 0 at S = 0 (forward); beta[L] = 0 at S[L] (backward)
+      const float2 v = make_float2(up ? 0.f : sm.tfrac[o0 + x], 0.f);
+      float2* r = sm.ring + (size_t)x * RL;
+      r[r0 % K] = v;
+      if (r0 % K < KBH)
+        for (int y = r0 % K + K; y < RL; y += K) r[y] = v;
+      xs.Sb[x] = up ? 0 : sm.tint[o0 + x];
+    }
+  }
+  // combine state: rows r-1, r-2 (walk order) of S, acc of the last step,
+  // n of the last step, the frame of p_{i-1} relative to F0
+  int si_p = 0, si_pp = 0;
+  float sf_p = 0.f, sf_pp = 0.f;
+  {
+    const size_t o0 = tile_row_off(r0, C);
+    if (!up) {
+      si_p = si_pp = sm.tint[o0 + cc];
+      sf_p = sf_pp = sm.tfrac[o0 + cc];
+    }
+  }
+  float acc2 = 0.f, nprev = 0.f, snprev = 1.f, Fp = 0.f;
+  int wslot = r0 % K;  // ring slot of the previous row's boundary
+  // helper state: frame Phi_{i-1} relative to F0, label base, predicted shift
+  float Fph = 0.f, rel = 0.f;
+  int hbase = 0;
+  double F0 = 0.0;
+  __syncthreads();
+  int Sbc = xs.Sb[cc];
+  if (!comb) {
+    const int first = up ? 1 - 1 - (jl + 1) * KBH : L - 1 + 2 + jl * KBH;  // step 1's window
+    hbase = ((first % K) + K) % K;
+  }
+  // checkpoint steps: forward boundary t = i - 1 at step i; backward
+  // boundary t1 = r + 2 at step i
+  const int delta = d.delta;
+  int next_ck;
+  if (up) {
+    next_ck = delta + 1;
+  } else {
+    const int t1 = ((L - 1) / delta) * delta;
+    next_ck = (t1 >= delta && t1 >= 2) ? L + 2 - t1 : INT_MAX;
+  }
+
+  for (int i = 1; i <= L; ++i) {
+    const int r = up ? i : L - i;
+    // ---- frame of p_{i-1} for the helpers (published by the combine warps)
+    if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
+    // ---- prefix-sum tiles: wait for the next row's tile when the walk
+    // first needs it; refill the buffer the walk has left behind
+    if (i < L && first_in_tile(r + ts.dir, up)) {
+      if (!xtile_wait(sm, ts, (r + ts.dir) / TS)) {
+        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+        tile_drain(sm, ts);
+        return;
+      }
+    }
+    if (first_in_tile(r, up)) tile_issue(sm, d, ws, b, ts, r / TS + ts.dir);
+    // ---- checkpoint: rebase the ring to (F0 + D, S_int at the boundary) and save it
+    if (i == next_ck) {
+      const int bnd = up ? i - 1 : r + 2;
+      const int j = up ? bnd / delta : bnd / delta - 1;
+      const float D = comb ? Fp : Fph;  // both are Phi_{i-1} - F0
+      if (comb) {
+        // the G lanes of a label rebase its ring, then save it (every lane
+        // of the warp passes the __syncwarp, labels >= C included)
+        const int sit = up ? si_p : si_pp;
+        if (act) {
+          const float adj = sg * (float)(sit - Sbc) - D;
+          for (int x = jl; x < RL; x += G) rl[x].y += adj;
+        }
+        __syncwarp();
+        if (act) {
+          float2* dst = (up ? ws.ack : ws.bck) + (((size_t)b * d.nck + j) * K) * C + c;
+          for (int q = jl; q < K; q += G) {
+            const int bb = up ? bnd - K + q : bnd + q;
+            if (up ? bb >= 0 : bb <= L) dst[(size_t)q * C] = rl[bb % K];
+          }
+          if (leader) xs.Sb[c] = sit;
+        }
+        Sbc = sit;
+      }
+      if (tid == 0) (up ? ws.acf : ws.bcf)[(size_t)b * d.nck + j] = F0 + (double)D;
+      __syncthreads();
+      F0 += (double)D;
+      if (comb) {
+        Fp -= D;
+      } else {
+        Fph -= D;
+        Sbc = xs.Sb[cc];
+      }
+      next_ck += delta;
+      if (!up) {
+        if (L + 2 - next_ck < delta) next_ck = INT_MAX;  // t1 below delta: no more
+      } else if (next_ck - 1 >= L) {
+        next_ck = INT_MAX;
+      }
+    }
+    if (comb) {
+      // ---------------------------------------------------------- combine
+      float acc, mx;
+      if (i == 1) {
+        acc = ex2(-M);  // the start boundary: gamma = 0 in frame 0
+        mx = 0.f;
+      } else {
+        const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < CAT; q += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(pv + q);
+          a0 = fmaf(v.x, w[q], a0);
+          a1 = fmaf(v.y, w[q + 1], a1);
+          a2 = fmaf(v.z, w[q + 2], a2);
+          a3 = fmaf(v.w, w[q + 3], a3);
+          m0 = fmaxf(m0, fmaxf(v.x, v.y));
+          m1 = fmaxf(m1, fmaxf(v.z, v.w));
+        }
+        acc = gsum<G>((a0 + a1) + (a2 + a3));
+        mx = fmaxf(m0, m1);
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
+      }
+      const float n = exponent_of(mx);
+      const float sn = pow2_neg(n);
+      const size_t off = tile_row_off(r, C);
+      const int si = sm.tint[off + cc];
+      const float sf = sm.tfrac[off + cc];
+      const float A1 = ex2(((M + d1) + sg * (float)(si - si_p)) + sg * (sf - sf_p));
+      float R = 0.f;
+      if (i >= 2) {
+        const float A2 = ex2(((M + d2) + sg * (float)(si - si_pp)) + sg * (sf - sf_pp));
+        const float oh = xs.Oh[(i & 1) * C + cc];
+        const float fo = (oh > 0.f) ? ex2((xs.Zh[(i & 1) * C + cc] + sg * sf) - nprev) : 0.f;
+        R = fmaf(acc2 * A2, snprev, oh * fo);
+      }
+      const float pn = fmaf(acc * sn, A1, R * sn);
+      if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
+      if (tid == 0) xs.nsl[i & 1] = n;
+      if (i >= 2 && leader) {
+        // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
+        const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
+        put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
+      }
+      wslot = up ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
+      acc2 = acc;
+      nprev = n;
+      snprev = sn;
+      si_pp = si_p;
+      sf_pp = sf_p;
+      si_p = si;
+      sf_p = sf;
+      Fp += n;
+    } else if (i < L) {
+      // ---------------------------------------------------------- helpers
+      const size_t offn = tile_row_off(r + ts.dir, C);
+      const float Qh = sg * (float)(sm.tint[offn + cc] - Sbc) - Fph;
+      float m = Qh + rel;
+      float s;
+      float e[KBH], dh[KBH];
+#pragma unroll
+      for (int q = 0; q < KBH; ++q) dh[q] = w[q];
+      const float lse = k_fanin<KBH, H>(rl + hbase, Qh, dh, m, s, e);
+      if (leader) {
+        xs.Oh[((i + 1) & 1) * C + c] = s;
+        xs.Zh[((i + 1) & 1) * C + c] = m;
+      }
+      if (isfinite(lse)) rel = rintf(lse - Qh);
+      hbase = up ? (hbase + 1 == K ? 0 : hbase + 1) : (hbase == 0 ? K - 1 : hbase - 1);
+    }
+    __syncthreads();
+  }
+
+  // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
+  if (warp == 0) {
+    float s = 0.f;
+    for (int x = lane; x < C; x += 32) s += xs.P[(L & 1) * d.xPC + x];
+    s = group_sum(s, 32);
+    if (lane == 0) {
+      const double lz = (s > 0.f) ? F0 + (double)Fp + (double)lg2(s) : -INFINITY;
+      if (up) {
+        ws.logz2[b] = lz;
+        logZ_out[b] = lz * LN2_D;
+      } else {
+        ws.logz2b[b] = lz;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t chain_exp_smem_bytes(const Dims& d) {
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRL * d.C * 8 + 16 +
+         (2ull * d.xPC + 5ull * d.C) * 4;
+}
+
+}  // namespace semicrf
+
+namespace semicrf {
+
+bool xshape_supported(int G, int CAT, int H, int KBH, int LB) {
+#define SEMICRF_XSHAPE_OK(g, cat, h, kbh, lb) \
+  if (G == g && CAT == cat && H == h && KBH == kbh && LB == lb) return true;
+  SEMICRF_FOR_EACH_XSHAPE(SEMICRF_XSHAPE_OK)
+#undef SEMICRF_XSHAPE_OK
+  return false;
+}
+
+cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const float* trans, const float* dur, double* logZ_out, int n_alpha,
+                             int n_beta, cudaStream_t st) {
+  const size_t sm = chain_exp_smem_bytes(d);
+#define SEMICRF_LAUNCH_XCHAIN(g, cat, h, kbh, lb)                                              \
+  if (d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb) {               \
+    if (sm > 48 * 1024) {                                                                      \
+      const cudaError_t e = cudaFuncSetAttribute(chain_exp_kernel<g, cat, h, kbh, lb>,         \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                                 (int)sm);                                     \
+      if (e != cudaSuccess) return e;                                                          \
+    }                                                                                          \
+    chain_exp_kernel<g, cat, h, kbh, lb><<<n_alpha + n_beta, d.xNT, sm, st>>>(                 \
+        d, ws, lengths, trans, dur, logZ_out, n_alpha);                                        \
+    return cudaGetLastError();                                                                 \
+  }
+  SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_XCHAIN)
+#undef SEMICRF_LAUNCH_XCHAIN
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace semicrf

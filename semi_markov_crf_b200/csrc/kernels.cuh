@@ -73,4 +73,25 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(16, 8, 8, 512) X(16, 32, 8, 512) X(8, 1, 16, 256) X(16, 1, 16, 256) X(16, 4, 16, 512) \
   X(16, 32, 16, 512) X(8, 1, 32, 256) X(16, 1, 32, 512) X(16, 32, 32, 512)
 
+// Pipelined exponential-domain rings (chain_exp.cu): shapes (combine lanes
+// per label G, weights per combine lane CAT, helper lanes per label H,
+// durations per helper lane KBH, launch bound LB).  A shape serves C <= G*CAT
+// and K <= H*KBH + 2 with 32*(ceil(C*G/32) + ceil(C*H/32)) <= LB threads
+// (labels never straddle a warp).
+#define SEMICRF_FOR_EACH_XSHAPE(X)                                                     \
+  X(1, 8, 1, 8, 64) X(1, 8, 4, 8, 64) X(1, 8, 8, 16, 96) X(1, 8, 16, 16, 160)          \
+  X(1, 8, 32, 16, 288) X(1, 16, 1, 8, 64) X(1, 16, 4, 8, 96) X(1, 16, 8, 16, 160)      \
+  X(1, 16, 16, 16, 288) X(1, 16, 32, 16, 544) X(1, 32, 4, 8, 160) X(1, 32, 8, 16, 288) \
+  X(1, 32, 16, 16, 544) X(2, 24, 4, 8, 288) X(2, 24, 4, 16, 288) X(2, 24, 8, 16, 480) \
+  X(2, 32, 4, 8, 384) X(2, 32, 4, 16, 384) X(2, 32, 8, 16, 640) X(4, 24, 4, 8, 768)   \
+  X(4, 24, 2, 32, 576) X(4, 32, 4, 8, 1024) X(4, 32, 2, 32, 768)
+
+size_t chain_exp_smem_bytes(const Dims& d);
+bool xshape_supported(int G, int CAT, int H, int KBH, int LB);
+// Same grid and outputs as launch_chain for the sequences whose scores fit
+// the exponential domain; writes ws.mode for every (direction, sequence).
+cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const float* trans, const float* dur, double* logZ_out, int n_alpha,
+                             int n_beta, cudaStream_t st);
+
 }  // namespace semicrf

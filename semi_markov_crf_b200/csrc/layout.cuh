@@ -36,6 +36,11 @@ struct Dims {
   int nchunk;    // prefix-sum chunks per sequence
   int store_w;   // floats per position in the segment recompute store (2C + 2)
   int store_smem;  // 1: the recompute store lives in shared memory
+  // Pipelined exponential-domain rings (chain_exp.cu): xG combine lanes per
+  // label with xCAT weights each, xH helper lanes per label with xKBH
+  // durations each (k = 3..K), xNT threads (launch bound xLB), ring of
+  // xRL = K + xKBH entries per label, label vector padded to xPC = xG * xCAT.
+  int xG, xCAT, xH, xKBH, xNT, xLB, xRL, xPC;
 };
 
 // Device pointers into the caller's workspace.
@@ -56,6 +61,8 @@ struct WsPtrs {
   double* segT;    // [B][nck][C] per-segment sum of (start - end) marginals
   double* segV;    // [B][nck][C] per-segment sum of the within-segment suffix sums
   int32_t* bp;     // [B][T+1][C] Viterbi backpointers
+  float* emax;     // [B] largest |centred emission| * log2(e) over the valid positions
+  int* mode;       // [2][B] ring path per (direction, sequence): 1 exponential, 2 log domain
 };
 
 }  // namespace semicrf

@@ -68,6 +68,8 @@ size_t forward_layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_lz = take(B * 8);
   const size_t o_ack = take(B * nck * K * C * 8);
   const size_t o_acf = take(B * nck * 8);
+  const size_t o_emax = take(B * 4);
+  const size_t o_mode = take(2 * B * 4);
   if (base && p) {
     char* c = static_cast<char*>(base);
     *p = WsPtrs{};
@@ -78,6 +80,8 @@ size_t forward_layout(const Dims& d, void* base, WsPtrs* p) {
     p->logz2 = reinterpret_cast<double*>(c + o_lz);
     p->ack = reinterpret_cast<float2*>(c + o_ack);
     p->acf = reinterpret_cast<double*>(c + o_acf);
+    p->emax = reinterpret_cast<float*>(c + o_emax);
+    p->mode = reinterpret_cast<int*>(c + o_mode);
   }
   return off;
 }
@@ -91,7 +95,8 @@ extern "C" int semicrf_forward_noalloc(const float* em, const int32_t* lengths, 
                                        const float* dur, int B, int T, int C, int K,
                                        unsigned flags, double* logZ, semicrf_stream_t stream) {
   if (!lengths || !trans || !dur || !logZ || (B > 0 && T > 0 && !em)) return SEMICRF_ERR_INVALID_ARG;
-  if (flags & ~(SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY)) return SEMICRF_ERR_INVALID_ARG;
+  if (flags & ~(SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY | SEMICRF_FLAG_LOG_DOMAIN))
+    return SEMICRF_ERR_INVALID_ARG;
   Dims d;
   int rc = make_dims(B, T, C, K, d);
   if (rc != SEMICRF_OK) return rc;
@@ -116,6 +121,13 @@ extern "C" int semicrf_forward_noalloc(const float* em, const int32_t* lengths, 
                                               (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, 1,
                                               nullptr, nullptr);
     if (cudaGetLastError() != cudaSuccess) return SEMICRF_ERR_CUDA;
+  }
+  // exponential-domain ring where the scores allow it, log domain for the rest
+  if (d.xG && !(flags & SEMICRF_FLAG_LOG_DOMAIN)) {
+    if (launch_chain_exp(d, p, lengths, trans, dur, logZ, B, 0, st) != cudaSuccess)
+      return SEMICRF_ERR_CUDA;
+  } else {
+    p.mode = nullptr;
   }
   return launch_chain(d, p, lengths, trans, dur, logZ, B, 0, st) == cudaSuccess ? SEMICRF_OK
                                                                                 : SEMICRF_ERR_CUDA;

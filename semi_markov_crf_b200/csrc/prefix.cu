@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(256) prefix_reduce_kernel(const float* __restr
   if (L < 0 || L > d.T) L = 0;  // reported by the scan pass
   const int r0 = j * R;
   const int r1 = min(r0 + R, L);
+  if (j == 0 && threadIdx.x == 0 && ws.emax) ws.emax[b] = 0.f;  // maxed by the scan pass
   __shared__ double part[256];
   const int G = 256 / C;  // row groups
   const int g = threadIdx.x / C, c = threadIdx.x % C;
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
     grp[g * C + c] = local;
   }
   __syncthreads();
+  float emx = 0.f;  // largest |centred emission| of this thread's rows
   if (g < G) {
     const double nuc = nu[c];
     double run = off[c];
@@ -119,8 +121,10 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
       if (t > T) break;
       double val = 0.0;
       if (r < nrows) {
-        run += (double)tile[r * C + c] - nuc;
+        const double x = (double)tile[r * C + c] - nuc;
+        run += x;
         val = run;
+        emx = fmaxf(emx, (float)fabs(x));
       }
       const bool valid = (t <= L);
       if (mode == 0) {
@@ -142,6 +146,14 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
         ws.sfrac[o] = 0.f;
       }
     }
+  }
+  // per-sequence bound for the choice of the ring arithmetic (non-negative
+  // floats order like their bit patterns); NaN never compares larger
+  if (mode == 1 && ws.emax) {
+    float m = emx * (float)LOG2E_D;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0.f)
+      atomicMax(reinterpret_cast<int*>(ws.emax + b), __float_as_int(m));
   }
 }
 

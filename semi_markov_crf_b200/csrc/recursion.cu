@@ -99,46 +99,42 @@ __device__ __forceinline__ void bwd_checkpoint(const Smem& sm, const Dims& d, co
   __syncthreads();
 }
 
-// Local normaliser of checkpoint segment j >= 1, from the cut at position
+// Normaliser of checkpoint segment j >= 1, from the cut at position
 // u = t0 - 1 (t0 = j Delta): every segmentation has exactly one segment
 // [s, t) with s <= u < t, so
 //   Z = sum_{c, s < t0 <= t, t - s <= K} 2^(gamma[s,c] - S[s,c]) 2^(dur2[t-s-1,c]) 2^(S[t,c] + beta[t,c])
-// and the share of label c in that sum is mu[u, c].  Both factors come from
-// the rings the two chains saved at boundary t0: the forward ring (boundaries
-// t0-K..t0-1, an entry (x, y) encoding gamma - S = x + y + F0 - S_int[t0]) and
-// the backward ring (boundaries t0..t0+K-1, beta + S = x + y + G0 + S_int[t0]);
-// the S_int[t0] cancel.  Normalising the segment's posteriors by this Z, which
-// is built from the very forward and backward values the segment restarts
-// from, keeps them exact however far rounding has carried the chains (and
-// their log Z) over the positions before t0 and after t1.
+// and the share of label c in that sum is mu[u, c].  The forward factors come
+// from the ring the forward chain saved at t0 (boundaries t0-K..t0-1, entry
+// (x, y) encoding gamma - S = x + y + F0 - S_int[t0]), which is also where
+// the segment's alpha recompute starts; the backward factors from the
+// segment's own backward ring once its walk has reached t0 (boundaries
+// t0..t0+K-1, beta + S = x + y + G0 + Sbase[c]).  Dividing the segment's
+// posteriors by this Z makes them ratios of the very values they were built
+// from, whatever rounding separates those from the chains' values over the
+// positions before t0 and after t1 -- and whatever arithmetic the chains used.
 // Returns log2 Z (float64) to every thread and leaves mu[u, c] in sm.tmp[c].
-// Uses the ring area as scratch; starts and ends with a barrier.
+// Uses sm.Acur as scratch; starts and ends with a barrier.
 __device__ double segment_cut(const Smem& sm, const Dims& d, const WsPtrs& ws, int b, int j, int L,
-                              const float* __restrict__ dur, double* lz_out) {
+                              double G0, const float* __restrict__ dur, double* lz_out) {
   const int C = d.C, K = d.K, t0 = j * d.delta;
   const size_t seg = (size_t)b * d.nck + j;
-  const float2* fa = ws.ack + seg * K * C;        // boundary t0 - K + i
-  const float2* fb = ws.bck + (seg - 1) * K * C;  // boundary t0 + i
-  float2* bs = sm.ring;                           // staged [c][K] backward entries
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < K * C; idx += blockDim.x) {
-    const int i = idx / C, c = idx % C;
-    bs[(size_t)c * K + i] = (t0 + i <= L) ? fb[idx] : make_float2(NEG_INF, 0.f);
-  }
+  const float2* fa = ws.ack + seg * K * C;  // boundary t0 - K + i
+  const int32_t* s0 = ws.sint + ((size_t)b * d.Tstride + t0) * C;
   __syncthreads();
   const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int kb_max = min(K - 1, L - t0);  // t - t0 <= K - 1 and t <= L
   for (int c = threadIdx.x >> 5; c < C; c += nw) {
-    const float2* bc = bs + (size_t)c * K;
+    const float2* bc = sm.ring + (size_t)c * d.RL;
+    const float sh = (float)(sm.Sbase[c] - __ldg(s0 + c));  // exact integer
     float zmax = NEG_INF;
     for (int ia = lane; ia < K; ia += 32) {
       if (t0 - K + ia < 0) continue;
       const float2 a = fa[(size_t)ia * C + c];
       const int kbe = min(ia, kb_max);  // t = t0 + kb <= s + K = t0 + ia
       for (int kb = 0; kb <= kbe; ++kb) {
-        const float2 v = bc[kb];
+        const float2 v = bc[(t0 + kb) % K];
         const float dk = __ldg(dur + (size_t)(kb + K - ia - 1) * C + c) * l2e();
-        zmax = fmaxf(zmax, ((a.y + v.y) + (a.x + v.x)) + dk);
+        zmax = fmaxf(zmax, (((a.y + v.y) + sh) + (a.x + v.x)) + dk);
       }
     }
     zmax = group_max(zmax, 32);
@@ -149,15 +145,15 @@ __device__ double segment_cut(const Smem& sm, const Dims& d, const WsPtrs& ws, i
       const float2 a = fa[(size_t)ia * C + c];
       const int kbe = min(ia, kb_max);
       for (int kb = 0; kb <= kbe; ++kb) {
-        const float2 v = bc[kb];
+        const float2 v = bc[(t0 + kb) % K];
         const float dk = __ldg(dur + (size_t)(kb + K - ia - 1) * C + c) * l2e();
-        sum += ex2((((a.y + v.y) - M) + (a.x + v.x)) + dk);
+        sum += ex2(((((a.y + v.y) + sh) - M) + (a.x + v.x)) + dk);
       }
     }
     sum = group_sum(sum, 32);
     if (lane == 0) {
-      sm.Acur[c] = M;                                  // exact integer shift
-      sm.tmp[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;   // log2 of the label's share
+      sm.Acur[c] = M;                                 // exact integer shift
+      sm.tmp[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;  // log2 of the label's share
     }
   }
   __syncthreads();
@@ -173,8 +169,7 @@ __device__ double segment_cut(const Smem& sm, const Dims& d, const WsPtrs& ws, i
     const float lt = (tot > 0.f) ? lg2(tot) : NEG_INF;
     __syncwarp();
     for (int c = lane; c < C; c += 32) sm.tmp[c] = ex2(((sm.Acur[c] - Mz) + sm.tmp[c]) - lt);
-    if (lane == 0)
-      *lz_out = (ws.acf[seg] + ws.bcf[seg - 1]) + ((double)Mz + (double)lt);
+    if (lane == 0) *lz_out = (ws.acf[seg] + G0) + ((double)Mz + (double)lt);
   }
   __syncthreads();
   return *lz_out;
@@ -195,6 +190,8 @@ __global__ void __launch_bounds__(LB, 1)
   const int C = d.C, K = d.K, PC = d.PC, tid = threadIdx.x;
   const bool is_alpha = (int)blockIdx.x < n_alpha;
   const int b = is_alpha ? blockIdx.x : blockIdx.x - n_alpha;
+  // already run by the exponential-domain kernel (chain_exp.cu)
+  if (ws.mode && ws.mode[(is_alpha ? 0 : d.B) + b] == 1) return;
   const int L = lengths[b];
   if (L < 0 || L > d.T || L == 0) {
     if (tid == 0) {
@@ -402,9 +399,10 @@ __global__ void __launch_bounds__(LB, 1)
 //   end_marg[s,c]   = 2^(alpha[s,c] + beta[s,c] - log2 Z_j)
 //   P(segment [s, s+k), c) = start_marg[s,c] * (normalised k term of btil)
 //   P(c' -> c at s)        = end_marg[s,c'] * (normalised c term of beta)
-// Z_j is the segment's own cut normaliser (segment_cut; the backward chain's
-// log Z for j = 0): equal to Z in exact arithmetic, and made of the same
-// restored forward and backward values as the segment's posteriors.
+// Z_j is the segment's own cut normaliser (segment_cut; sum_c start_marg[0, c]
+// for j = 0), found when the walk reaches t0 -- equal to Z in exact
+// arithmetic and made of the same forward and backward values as the
+// segment's posteriors -- which rescales the walk's provisional results.
 // The leader lane of label c's group keeps c's running sums.
 // ===========================================================================
 template <int KBT, int CAT, int G, int LB>
@@ -438,16 +436,13 @@ __global__ void __launch_bounds__(LB, 1)
   float tmax2 = 0.f;
   int par = 0, q = 0;
 
-  // Local normaliser and mu[t0 - 1, c] (left in sm.tmp).  Segment 0 starts
-  // at boundary 0, where the backward chain's own log Z is the cut.
+  // Provisional normaliser for the walk (the forward chain's log Z: close
+  // enough to keep every posterior O(1)); the segment's own normaliser is
+  // computed once its backward walk has reached t0, and the outputs are
+  // rescaled by the ratio.
   __shared__ double s_lz;
-  double logz2;
-  if (j == 0) {
-    for (int c = tid; c < C; c += blockDim.x) sm.tmp[c] = 0.f;
-    logz2 = ws.logz2b[b];
-  } else {
-    logz2 = segment_cut(sm, d, ws, b, j, L, dur, &s_lz);
-  }
+  __shared__ float s_r;
+  const double logz2 = ws.logz2[b];
 
   // ------------------------------------------------------ alpha recompute
   {
@@ -576,6 +571,7 @@ __global__ void __launch_bounds__(LB, 1)
       ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, L % K, make_float2(ws.sfrac[o], 0.f));
     }
     Sb = ws.sint[((size_t)b * d.Tstride + L) * C + ln.cc];
+    for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + L) * C + c];
   } else {
     const float2* ck = ws.bck + seg * K * C;
     for (int idx = tid; idx < K * C; idx += blockDim.x) {
@@ -583,6 +579,7 @@ __global__ void __launch_bounds__(LB, 1)
       if (t1 + i <= L) ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, (t1 + i) % K, ck[idx]);
     }
     Sb = ws.sint[((size_t)b * d.Tstride + t1) * C + ln.cc];
+    for (int c = tid; c < C; c += blockDim.x) sm.Sbase[c] = ws.sint[((size_t)b * d.Tstride + t1) * C + c];
     G0 = ws.bcf[seg];
   }
   // this CTA's float64 partials start at zero (each thread its own entries)
@@ -641,6 +638,7 @@ __global__ void __launch_bounds__(LB, 1)
         sm.Acur[par * C + ln.c] = Bt;
         sm.pcur[par * PC + ln.c] = ex2(Bt);
         if (start_marg) start_marg[((size_t)b * (d.T + 1) + s) * C + ln.c] = St;
+        if (s == 0) sm.tmp[ln.c] = St;  // segment 0's normaliser: sum_c St[0, c]
       }
       warp_max_to_shared(&sm.maxslot[q], ln.leader ? f2ord(Bt) : INT_MIN);
       {
@@ -704,9 +702,40 @@ __global__ void __launch_bounds__(LB, 1)
       }
     }
   }
+  // ---- the segment's own normaliser: r = Z_provisional / Z_j
+  __syncthreads();
+  if (j == 0) {
+    // position 0 is covered by the segments starting at 0: Z_0 / Z_prov = sum_c St[0, c]
+    if (tid < 32) {
+      float tot = 0.f;
+      for (int c = tid; c < C; c += 32) tot += sm.tmp[c];
+      tot = group_sum(tot, 32);
+      __syncwarp();
+      for (int c = tid; c < C; c += 32) sm.tmp[c] = 0.f;  // nothing before position 0
+      if (tid == 0) s_r = (tot > 0.f) ? 1.f / tot : 1.f;
+    }
+  } else {
+    const double lzj = segment_cut(sm, d, ws, b, j, L, G0, dur, &s_lz);
+    if (tid == 0) s_r = ex2((float)(logz2 - lzj));
+  }
+  __syncthreads();
+  const float rs = s_r;
+  // rescale what the walk wrote: boundary rows [t0, t1) (and the end
+  // marginal at L), the suffix sums v, the count partials
+  for (int idx = tid; idx < (t1 - t0) * C; idx += blockDim.x) {
+    const int u = t0 + idx / C, c = idx % C;
+    const size_t ob = ((size_t)b * (d.T + 1) + u) * C + c;
+    if (start_marg) start_marg[ob] *= rs;
+    if (end_marg) end_marg[ob] *= rs;
+    grad_em[((size_t)b * d.T + u) * C + c] *= rs;
+  }
+  if (last && end_marg)
+    for (int c = tid; c < C; c += blockDim.x) end_marg[((size_t)b * (d.T + 1) + L) * C + c] *= rs;
+  for (int idx = tid; idx < K * C; idx += blockDim.x) ws.pgd[seg * K * C + idx] *= (double)rs;
+  for (int idx = tid; idx < C * C; idx += blockDim.x) ws.pgt[seg * C * C + idx] *= (double)rs;
   if (ln.leader) {
-    ws.segT[seg * C + ln.c] = (double)sm.tmp[ln.c] + accmu;  // mu[t0 - 1] + segment total
-    ws.segV[seg * C + ln.c] = vsum;
+    ws.segT[seg * C + ln.c] = (double)sm.tmp[ln.c] + (double)rs * accmu;  // mu[t0 - 1] + total
+    ws.segV[seg * C + ln.c] = (double)rs * vsum;
   }
 }
 

@@ -15,16 +15,18 @@ import torch
 
 __all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
-           "FLAG_FORWARD_ONLY", "selftest_bounded_wait", "profile_enable", "profile_read",
+           "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "ring_domains", "profile_enable", "profile_read",
            "forward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "KERNELS", "lib"]
 
 # every kernel the library launches (names used by the profiler)
-KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_kernel", "segment_kernel",
-           "finalize_positions_kernel", "reduce_partials_kernel", "viterbi_kernel")
+KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "chain_kernel",
+           "segment_kernel", "finalize_positions_kernel", "reduce_partials_kernel",
+           "viterbi_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2
+FLAG_LOG_DOMAIN = 0x4
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SEMICRF_NOALLOC_SCRATCH_BYTES
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsemicrf_b200.so")
@@ -50,11 +52,12 @@ lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
 lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
 lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _vp]
+lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.POINTER(ctypes.c_int32)]
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
 for _f in ("semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_get_status",
-           "semicrf_selftest_bounded_wait"):
+           "semicrf_selftest_bounded_wait", "semicrf_ring_domains"):
     getattr(lib, _f).restype = _i
 
 
@@ -117,8 +120,9 @@ class Workspace:
         return self.buf.data_ptr()
 
 
-def _flags(center: bool, forward_only: bool = False) -> int:
-    return (0 if center else FLAG_NO_CENTER) | (FLAG_FORWARD_ONLY if forward_only else 0)
+def _flags(center: bool, forward_only: bool = False, log_domain: bool = False) -> int:
+    return ((0 if center else FLAG_NO_CENTER) | (FLAG_FORWARD_ONLY if forward_only else 0) |
+            (FLAG_LOG_DOMAIN if log_domain else 0))
 
 
 def prefix_center(em, lengths, center: bool = True, ws: Workspace | None = None):
@@ -138,9 +142,10 @@ def prefix_center(em, lengths, center: bool = True, ws: Workspace | None = None)
 
 
 def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = False,
-            ws: Workspace | None = None, logZ=None):
+            ws: Workspace | None = None, logZ=None, log_domain: bool = False):
     """Steps 1-2: log Z [B] (float64).  Returns (logZ, workspace); pass the
-    workspace to :func:`backward`."""
+    workspace to :func:`backward`.  log_domain=True runs every sequence's
+    rings in the log domain (SEMICRF_FLAG_LOG_DOMAIN)."""
     dev = em.device
     _need(em, torch.float32, "em", dev)
     _need(lengths, torch.int32, "lengths", dev)
@@ -148,7 +153,7 @@ def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = F
     _need(dur, torch.float32, "dur", dev)
     B, T, C = em.shape
     K = dur.shape[0]
-    flags = _flags(center, forward_only)
+    flags = _flags(center, forward_only, log_domain)
     if ws is None or not ws.matches(B, T, C, K, flags):
         ws = Workspace(B, T, C, K, flags, dev)
     if logZ is None:
@@ -227,6 +232,17 @@ def get_status(ws: Workspace) -> int:
     return int(st.value)
 
 
+def ring_domains(ws: Workspace):
+    """Arithmetic of each ring in the last forward on `ws`: a list of 2B ints,
+    forward rings then backward rings, 1 = exponential domain, 2 = log
+    domain, 0 = not run (synchronises)."""
+    B, T, C, K = ws.dims
+    out = (ctypes.c_int32 * max(1, 2 * B))()
+    _check(lib.semicrf_ring_domains(ws.ptr, ws.nbytes, B, T, C, K, ws.flags,
+                                    _stream(ws.buf.device), out), "semicrf_ring_domains")
+    return list(out)[:2 * B]
+
+
 def selftest_bounded_wait(ws: Workspace, spins: int) -> int:
     """Runs the never-completing bounded wait with `spins` polls; returns the
     resulting status word (SEMICRF_ERR_DEVICE_TIMEOUT = 5 expected)."""
@@ -249,7 +265,8 @@ def profile_read(kernel: str):
     return float(ms.value), int(n.value)
 
 
-def forward_noalloc(em, lengths, trans, dur, center: bool = True, logZ=None):
+def forward_noalloc(em, lengths, trans, dur, center: bool = True, logZ=None,
+                    log_domain: bool = False):
     """log Z [B] (float64) through semicrf_forward_noalloc: no workspace, no
     allocation inside the library (the output tensor is allocated here unless
     passed).  Raises SemiCRFError(SEMICRF_ERR_UNSUPPORTED) when the problem
@@ -264,6 +281,7 @@ def forward_noalloc(em, lengths, trans, dur, center: bool = True, logZ=None):
     if logZ is None:
         logZ = torch.empty(B, dtype=torch.float64, device=dev)
     _check(lib.semicrf_forward_noalloc(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K,
-                                       _flags(center, True), _ptr(logZ), _stream(dev)),
+                                       _flags(center, True, log_domain), _ptr(logZ),
+                                       _stream(dev)),
            "semicrf_forward_noalloc")
     return logZ

@@ -24,11 +24,12 @@ def to_dev(case, dev="cuda"):
             torch.from_numpy(np.ascontiguousarray(case["dur"])).to(dev))
 
 
-def gpu_fb(case, center=True, grad_logZ=None, forward_only=False):
+def gpu_fb(case, center=True, grad_logZ=None, forward_only=False, log_domain=False):
     from semi_markov_crf_b200 import semicrf
     em, lengths, trans, dur = to_dev(case)
     g = None if grad_logZ is None else torch.as_tensor(grad_logZ, dtype=torch.float64, device="cuda")
-    logZ, ws = semicrf.forward(em, lengths, trans, dur, center=center, forward_only=forward_only)
+    logZ, ws = semicrf.forward(em, lengths, trans, dur, center=center, forward_only=forward_only,
+                               log_domain=log_domain)
     out = semicrf.backward(ws, lengths, trans, dur, grad_logZ=g, marginals=True)
     status = semicrf.get_status(ws)
     res = {k: v.cpu().numpy() for k, v in out.items()}

@@ -50,6 +50,77 @@ def test_forward_backward_matches_oracle(fb_case):
     assert_fb_close(got, ref, case["lengths"], name)
 
 
+def test_log_domain_rings_match_oracle(fb_case):
+    """The same cases with every ring forced into the log-domain kernel."""
+    name, case, ref = fb_case
+    got = gpu_fb(case, log_domain=True)
+    assert got["status"] == 0
+    print(name, errors(got, ref))
+    assert_fb_close(got, ref, case["lengths"], name)
+
+
+def _wide_range_cases():
+    """Inputs outside the exponential-domain kernel's exponent head-room:
+    forbidden (-inf) transitions and durations, and emissions of about a
+    hundred nats per position; the library runs them in the log domain.
+    (Float32 log-domain values carry ulp(|one step's score|): at scores of
+    several hundred log2 units per position -- emissions x25 here -- that
+    alone reaches 1e-4 on marginals.)"""
+    forbidden = synth.make("speech", B=3, T=120, seed=21)
+    forbidden["trans"][0, 1] = -np.inf
+    forbidden["trans"][2, :5] = -np.inf
+    forbidden["dur"][3, 7] = -np.inf
+    loud = synth.make("speech", B=3, T=120, seed=22)
+    loud["em"] *= np.float32(10.0)
+    long_loud = synth.make("genomic", B=1, T=2500, seed=23)
+    long_loud["em"] *= np.float32(10.0)
+    return {"forbidden": forbidden, "loud": loud, "long_loud": long_loud}
+
+
+def test_ring_domain_choice():
+    """Workload-like inputs run in the exponential domain, the wide-range ones
+    and log_domain=True in the log domain; both give the oracle's results."""
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make("speech", B=4, T=200, seed=24)
+    em, lengths, trans, dur = to_dev(case)
+    _, ws = semicrf.forward(em, lengths, trans, dur)
+    assert semicrf.ring_domains(ws) == [1] * 8
+    _, ws = semicrf.forward(em, lengths, trans, dur, log_domain=True)
+    assert semicrf.ring_domains(ws) == [2] * 8
+    for name, c in _wide_range_cases().items():
+        em, lengths, trans, dur = to_dev(c)
+        _, ws = semicrf.forward(em, lengths, trans, dur)
+        B = len(c["lengths"])
+        assert semicrf.ring_domains(ws) == [2] * (2 * B), name
+
+
+def test_moderately_loud_inputs_stay_exact_in_the_exponential_domain():
+    """Emissions x3 (per-step exponent span about 60 of fp32's 126): still the
+    exponential domain, still within tolerance."""
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make("genomic", B=2, T=2000, seed=25)
+    case["em"] *= np.float32(3.0)
+    em, lengths, trans, dur = to_dev(case)
+    _, ws = semicrf.forward(em, lengths, trans, dur)
+    assert semicrf.ring_domains(ws) == [1] * 4
+    ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"],
+                                  case["dur"].shape[0])
+    got = gpu_fb(case)
+    print(errors(got, ref))
+    assert_fb_close(got, ref, case["lengths"], "loud x3")
+
+
+@pytest.mark.parametrize("name", ["forbidden", "loud", "long_loud"])
+def test_wide_range_inputs_match_oracle(name):
+    case = _wide_range_cases()[name]
+    ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"],
+                                  case["dur"].shape[0])
+    got = gpu_fb(case)
+    assert got["status"] == 0
+    print(name, errors(got, ref))
+    assert_fb_close(got, ref, case["lengths"], name)
+
+
 def test_viterbi_matches_oracle(fb_case):
     name, case, _ = fb_case
     ref = oracle.viterbi(case["em"], case["lengths"], case["trans"], case["dur"], case["dur"].shape[0])

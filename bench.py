@@ -100,7 +100,7 @@ def alu_ops_per_position(kernel: str, K: int, C: int) -> int:
     """Algorithmic fp32 operations per position of the max-semiring kernel:
     one add and one max per (duration, label) term of the k fan-in and per
     (label, label) term of the label fan-in."""
-    if kernel == "viterbi_kernel":
+    if kernel in ("viterbi_kernel", "viterbi_pipe_kernel"):
         return 2 * (K * C + C * C)
     return 0
 

@@ -93,7 +93,9 @@ void choose_xshape(Dims& d, size_t budget) {
   if (d.xG == 0) return;
   d.xRL = K + d.xKBH;
   d.xPC = d.xG * d.xCAT;
-  if (chain_exp_smem_bytes(d) > budget) d.xG = 0;
+  d.xRLP = K + d.xH * d.xKBH;
+  if (d.xH < 16) d.xRLP += (((d.xH - d.xRLP) % 16) + 16) % 16;
+  if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget) d.xG = 0;
 }
 
 // Sizes, lane mapping and limits.  Returns a semicrf_status.
@@ -441,7 +443,10 @@ extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const fl
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
   if (rc) return rc;
   cudaError_t e;
-  {
+  if (d.xG) {
+    ProfScope ps("viterbi_pipe_kernel", st);
+    e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st);
+  } else {
     ProfScope ps("viterbi_kernel", st);
     e = launch_viterbi(d, p, lengths, trans, dur, score, labels, seg_start, st);
   }

@@ -87,6 +87,11 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(4, 24, 2, 32, 576) X(4, 32, 4, 8, 1024) X(4, 32, 2, 32, 768)
 
 size_t chain_exp_smem_bytes(const Dims& d);
+size_t viterbi_pipe_smem_bytes(const Dims& d);
+// Viterbi with the pipelined schedule (shapes of SEMICRF_FOR_EACH_XSHAPE).
+cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                const float* trans, const float* dur, double* score,
+                                int32_t* labels, uint8_t* seg_start, cudaStream_t st);
 bool xshape_supported(int G, int CAT, int H, int KBH, int LB);
 // Same grid and outputs as launch_chain for the sequences whose scores fit
 // the exponential domain; writes ws.mode for every (direction, sequence).

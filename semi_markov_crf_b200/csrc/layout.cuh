@@ -41,6 +41,11 @@ struct Dims {
   // durations each (k = 3..K), xNT threads (launch bound xLB), ring of
   // xRL = K + xKBH entries per label, label vector padded to xPC = xG * xCAT.
   int xG, xCAT, xH, xKBH, xNT, xLB, xRL, xPC;
+  // Pipelined Viterbi (viterbi_pipe.cu): helper lanes stride over a window
+  // of xH * xKBH ring entries; the label rows of its ring are xRLP >= K +
+  // xH * xKBH entries apart, padded so that a half warp's 64-bit reads of
+  // consecutive entries of different labels fall in distinct banks.
+  int xRLP;
 };
 
 // Device pointers into the caller's workspace.

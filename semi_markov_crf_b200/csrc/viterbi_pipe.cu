@@ -1,0 +1,445 @@
+// viterbi_pipe.cu -- step 4: max-semiring decoding, pipelined.
+//
+// The recursion of viterbi.cu (base-2 units, exact integer frames):
+//   G[s, c] = max_{c'} V[s, c'] + trans2[c', c]                 (G[0, c] = 0)
+//   V[t, c] = S[t,c] + max_{k <= min(K,t)} G[t-k, c] - S[t-k, c] + dur2[k-1, c]
+// organised around its real dependency: only the k = 1 term of V[t] needs
+// G[t-1], which needs all of V[t-1, :]; the k = 2 term needs G[t-2] (known a
+// step earlier) and the k >= 3 terms only ring entries written two or more
+// steps before.
+//
+// Roles (one CTA per sequence).  Combine warps (G lanes per label, CAT
+// source labels per lane) run the critical path of step t: read V[t-1, :],
+// take max_{c'} V + trans2 for their label, combine it with the step's
+// precomputed candidates, store V[t] and arrive at the barrier.  The argmax
+// label and the ring write of G[t-1] follow the store, off the path.  Helper
+// warps (H lanes per label, KBH durations per lane, strided over the window
+// so that a label's lanes read consecutive ring entries) compute during step
+// t everything step t+1 needs besides G[t]: the best k >= 3 term and its k,
+// and the additive constants of the k = 1 and k = 2 terms.  One barrier per
+// step.
+//
+// Frames: V[t, :] is stored relative to Phi_t = Phi_{t-1} + n_t, where n_t =
+// rint(max_c V[t-1, c]) relative to Phi_{t-1} -- taken from the vector every
+// combine lane has just read, so no reduction sits before the barrier.
+//
+// Ties: k = 1 before k = 2 before the helpers' best k (itself the smallest
+// k among equal terms), the smallest c' among equal label terms, and the
+// smallest final label; a re-scan finds each argmax once the maximum is
+// known (equal floating-point sums compare bit-exactly).
+//
+// Backpointers: bits 0-15 of bp[t, c] hold the best duration of a segment of
+// label c ending at t (written in step t), bits 16-31 the best previous label
+// of a segment of label c starting at t (written in step t+1).
+#include "ring.cuh"
+
+namespace semicrf {
+
+using namespace ring;
+
+namespace {
+
+constexpr int VREBASE = 4096;  // steps between integer rebases (keeps y exact)
+
+struct VSmem {
+  Smem s;      // mbar, tint, tfrac, ring
+  float* V;    // [2][xPC]  V of the step of that parity (-inf padded)
+  float* Om;   // [2][C]    helpers' best k >= 3 candidate, frame Phi_{t-2}
+  int* Ok;     // [2][C]    its duration
+  float* A1;   // [2][C]    dur2[0] + S[t] - S[t-1]
+  float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
+  float* nsl;  // [2]       frame step published by the combine warps
+  int* Sb;     // [C]       label integer bases
+};
+
+__device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
+  VSmem x;
+  const int C = d.C;
+  unsigned char* p = raw;
+  x.s.mbar = reinterpret_cast<uint64_t*>(p);
+  x.s.maxslot = reinterpret_cast<int*>(p + 16);
+  x.s.aux = reinterpret_cast<int*>(p + 32);
+  x.nsl = reinterpret_cast<float*>(p + 48);
+  p += 64;
+  x.s.tint = reinterpret_cast<int32_t*>(p);
+  p += 2ull * TS * C * sizeof(int32_t);
+  x.s.tfrac = reinterpret_cast<float*>(p);
+  p += 2ull * TS * C * sizeof(float);
+  x.s.ring = reinterpret_cast<float2*>(p);
+  p += (size_t)d.xRLP * C * sizeof(float2);
+  p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
+  float* f = reinterpret_cast<float*>(p);
+  x.V = f;
+  f += 2 * d.xPC;
+  x.Om = f;
+  f += 2 * C;
+  x.Ok = reinterpret_cast<int*>(f);
+  f += 2 * C;
+  x.A1 = f;
+  f += 2 * C;
+  x.A2 = f;
+  f += 2 * C;
+  x.Sb = reinterpret_cast<int*>(f);
+  x.s.pcur = nullptr;
+  x.s.Acur = nullptr;
+  x.s.tmp = nullptr;
+  x.s.Sbase = x.Sb;
+  x.s.store = nullptr;
+  return x;
+}
+
+// Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
+__device__ __forceinline__ bool vtile_wait(const Smem& sm, TileStream& ts, int ti) {
+  const int buf = ti & 1;
+  bool ok = mbar_wait(&sm.mbar[buf], ts.ph[buf], WAIT_SPIN_LIMIT);
+  ts.ph[buf] ^= 1u;
+  return !__syncthreads_or(!ok);
+}
+
+// Smallest i' > i with i' % TS == rem.
+__device__ __forceinline__ int next_with_rem(int i, int rem) {
+  int x = (i / TS) * TS + rem;
+  return x > i ? x : x + TS;
+}
+
+template <int G, int CAT, int H, int KBH, int LB>
+__global__ void __launch_bounds__(LB, 1)
+    viterbi_pipe_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                        const float* __restrict__ trans, const float* __restrict__ dur,
+                        double* __restrict__ score, int32_t* __restrict__ labels,
+                        uint8_t* __restrict__ seg_start) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const VSmem vs = vcarve(smem_raw, d);
+  const Smem& sm = vs.s;
+  const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x;
+  const int b = blockIdx.x;
+  const int L = lengths[b];
+  const bool bad = (L < 0 || L > T);
+  // positions past the length (all of them for a bad length)
+  for (int u = (bad ? 0 : L) + tid; u < T; u += blockDim.x) {
+    labels[(size_t)b * T + u] = -1;
+    seg_start[(size_t)b * T + u] = 0;
+  }
+  if (bad || L == 0) {
+    if (tid == 0) {
+      if (bad) set_status(ws.status, ST_BAD_LENGTH);
+      score[b] = bad ? __longlong_as_double(0x7ff8000000000000ll) : 0.0;
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- roles
+  constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
+  constexpr int NR = CAT > KBH ? CAT : KBH;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nwc = (C + LPWC - 1) / LPWC;
+  const bool comb = warp < nwc;
+  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
+  const int jl = comb ? lane % G : lane % H;
+  const bool act = c < C;
+  const int cc = act ? c : 0;
+  const bool leader = act && jl == 0;
+  const int RL = K + WL, RLP = d.xRLP;
+  float2* const rl = sm.ring + (size_t)cc * RLP;
+
+  // combine lanes: trans2[x][c] of their sources x = jl*CAT + q (-inf past C);
+  // helper lanes: dur2 of window index q*H + jl, k = 2 + WL - (q*H + jl)
+  float w[NR];
+  float d1 = NEG_INF, d2 = NEG_INF;
+  if (comb) {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int x = jl * CAT + q;
+      w[q] = (q < CAT && act && x < C) ? __ldg(trans + (size_t)x * C + cc) * l2e() : NEG_INF;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int k = 2 + WL - (q * H + jl);
+      w[q] = (q < KBH && act && k >= 3 && k <= K) ? __ldg(dur + (size_t)(k - 1) * C + cc) * l2e()
+                                                 : NEG_INF;
+    }
+    d1 = __ldg(dur + cc) * l2e();
+    if (K >= 2) d2 = __ldg(dur + C + cc) * l2e();
+  }
+
+  // ---------------------------------------------------------------- shared state
+  for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  for (int i = tid; i < 2 * d.xPC; i += blockDim.x) vs.V[i] = NEG_INF;
+  for (int i = tid; i < 2 * C; i += blockDim.x) {
+    vs.Om[i] = NEG_INF;
+    vs.Ok[i] = 3;
+    vs.A1[i] = NEG_INF;
+    vs.A2[i] = NEG_INF;
+  }
+  if (tid == 0) {
+    vs.nsl[0] = vs.nsl[1] = 0.f;
+    mbar_init(&sm.mbar[0], 1);
+    mbar_init(&sm.mbar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  TileStream ts;
+  ts.ph[0] = ts.ph[1] = 0;
+  ts.lo = 0;
+  ts.hi = L / TS;
+  ts.dir = 1;
+  tile_issue(sm, d, ws, b, ts, 0);
+  tile_issue(sm, d, ws, b, ts, 1);
+  if (!vtile_wait(sm, ts, 0)) {
+    if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+    tile_drain(sm, ts);
+    return;
+  }
+  // boundary 0: G = 0 at S = 0, base 0; helpers set step 1's k = 1 constant
+  for (int x = tid; x < C; x += blockDim.x) {
+    float2* r = sm.ring + (size_t)x * RLP;
+    for (int y = 0; y < RL; y += K) r[y] = make_float2(0.f, 0.f);
+    vs.Sb[x] = 0;
+  }
+  // helper state: rows i (cur) and i-1 (prev) of S, frame Phi_{i-1} - F0
+  int hs_c = 0, hs_p = 0;
+  float hf_c = 0.f, hf_p = 0.f, Fph = 0.f;
+  const int32_t* hrow_i = sm.tint;  // row i+1 of the current step (set below)
+  const float* hrow_f = sm.tfrac;
+  if (!comb) {
+    hs_c = sm.tint[C + cc];  // row 1
+    hf_c = sm.tfrac[C + cc];
+    if (leader) vs.A1[1 * C + c] = d1 + ((float)hs_c + hf_c);  // S[1] - S[0]
+    hrow_i = sm.tint + 2 * C;  // row 2 for step 1
+    hrow_f = sm.tfrac + 2 * C;
+  }
+  int hbase = (((-WL) % K) + K) % K;  // window start b_lo = i - 1 - WL, at i = 1
+  // combine state
+  float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
+  int si_p = 0;
+  float sf_p = 0.f;
+  const int32_t* crow_i = sm.tint + C;  // row i of the current step
+  const float* crow_f = sm.tfrac + C;
+  int wslot = 0;
+  double F0 = 0.0;
+  int16_t* bp16 = reinterpret_cast<int16_t*>(ws.bp + (size_t)b * (T + 1) * C);
+  __syncthreads();
+  int Sbc = 0;
+  int next_rb = VREBASE + 1;
+  // next step with an event: a tile to wait for (row i+1 opens a tile), a
+  // tile to issue (row i opens a tile), a rebase, or the last step
+  auto next_event = [&](int i) {
+    int e = min(next_with_rem(i, TS - 1), next_with_rem(i, 0));
+    e = min(e, next_rb);
+    return min(e, L);
+  };
+  int next_ev = next_event(0);
+
+  for (int i = 1; i <= L; ++i) {
+    if (!comb && i >= 2) Fph += vs.nsl[(i - 1) & 1];
+    if (i == next_ev) {
+      if (i < L && (i + 1) % TS == 0) {
+        if (!vtile_wait(sm, ts, (i + 1) / TS)) {
+          if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+          tile_drain(sm, ts);
+          return;
+        }
+        const size_t o = tile_row_off(i + 1, C);
+        hrow_i = sm.tint + o;
+        hrow_f = sm.tfrac + o;
+      }
+      if (i % TS == 0) {
+        tile_issue(sm, d, ws, b, ts, i / TS + 1);
+        const size_t o = tile_row_off(i, C);
+        crow_i = sm.tint + o;
+        crow_f = sm.tfrac + o;
+      }
+      if (i == next_rb) {
+        // rebase the integer frames to (F0 + Phi_{i-1}, S_int[i-1])
+        const float D = comb ? Fp : Fph;
+        if (comb && act) {
+          const float adj = (float)(si_p - Sbc) - D;
+          for (int x = jl; x < RL; x += G) rl[x].y += adj;
+          if (leader) vs.Sb[c] = si_p;
+        }
+        __syncthreads();
+        F0 += (double)D;
+        if (comb) {
+          Fp -= D;
+        } else {
+          Fph -= D;
+        }
+        Sbc = vs.Sb[cc];
+        next_rb += VREBASE;
+      }
+      next_ev = next_event(i);
+    }
+    if (comb) {
+      // ---------------------------------------------------------- combine
+      float gv, mx = NEG_INF;
+      float vv[CAT];
+      if (i == 1) {
+        gv = 0.f;  // G[0] = 0 in frame 0
+#pragma unroll
+        for (int q = 0; q < CAT; ++q) vv[q] = NEG_INF;
+      } else {
+        const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
+        float b0 = NEG_INF, b1 = NEG_INF, m0 = NEG_INF, m1 = NEG_INF;
+#pragma unroll
+        for (int q = 0; q < CAT; q += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(pv + q);
+          vv[q] = v.x;
+          vv[q + 1] = v.y;
+          vv[q + 2] = v.z;
+          vv[q + 3] = v.w;
+          b0 = fmaxf(b0, fmaxf(v.x + w[q], v.y + w[q + 1]));
+          b1 = fmaxf(b1, fmaxf(v.z + w[q + 2], v.w + w[q + 3]));
+          m0 = fmaxf(m0, fmaxf(v.x, v.y));
+          m1 = fmaxf(m1, fmaxf(v.z, v.w));
+        }
+        gv = fmaxf(b0, b1);
+        mx = fmaxf(m0, m1);
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) {
+          gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
+        }
+      }
+      const float n = (mx == NEG_INF) ? 0.f : rintf(mx);
+      const float a1 = vs.A1[(i & 1) * C + cc];
+      const float a2 = vs.A2[(i & 1) * C + cc];
+      const float om = vs.Om[(i & 1) * C + cc];
+      // candidates relative to Phi_{i-1}; ties to the smaller k
+      const float c1 = gv + a1;
+      const float c2 = (g2 + a2) - nprev;
+      const float c3 = om - nprev;
+      const float v = fmaxf(c1, fmaxf(c2, c3));
+      if (leader) {
+        vs.V[(i & 1) * d.xPC + c] = v - n;
+        const int k = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : vs.Ok[(i & 1) * C + cc]);
+        bp16[((size_t)i * C + c) * 2] = (int16_t)k;
+      }
+      if (tid == 0) vs.nsl[i & 1] = n;
+      if (i >= 2) {
+        // off the path: the best previous label (smallest on ties) and the
+        // ring entry of G[i-1] (frame Phi_{i-1})
+        int bc = 0x7fffffff;
+#pragma unroll
+        for (int q = CAT - 1; q >= 0; --q)
+          if (vv[q] + w[q] == gv) bc = jl * CAT + q;
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
+        bc = min(bc, C - 1);  // every term -inf: an unreachable state, any label
+        if (leader) {
+          bp16[((size_t)(i - 1) * C + c) * 2 + 1] = (int16_t)bc;
+          const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
+          rl[wslot] = e;
+          for (int x = wslot + K; x < RL; x += K) rl[x] = e;
+        }
+      }
+      wslot = (wslot + 1 == K) ? 0 : wslot + 1;
+      g2 = gv;
+      nprev = n;
+      Fp += n;
+      si_p = crow_i[cc];
+      sf_p = crow_f[cc];
+      crow_i += C;
+      crow_f += C;
+    } else if (i < L) {
+      // ---------------------------------------------------------- helpers
+      const int sn = hrow_i[cc];
+      const float fn = hrow_f[cc];
+      const float Qh = (float)(sn - Sbc) - Fph;
+      float best = NEG_INF;
+      float tv[KBH];
+#pragma unroll
+      for (int q = 0; q < KBH; ++q) {
+        const float2 e = rl[hbase + q * H + jl];
+        tv[q] = ((e.y + Qh) + e.x) + w[q];
+        best = fmaxf(best, tv[q]);
+      }
+#pragma unroll
+      for (int o = H / 2; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
+      // smallest k among equal terms: k falls as the window index grows
+      int kb = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < KBH; ++q)
+        if (tv[q] == best) kb = 2 + WL - (q * H + jl);
+#pragma unroll
+      for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
+      if (leader) {
+        const int o2 = ((i + 1) & 1) * C + c;
+        vs.Om[o2] = best + fn;
+        vs.Ok[o2] = kb;
+        vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
+        vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
+      }
+      hs_p = hs_c;
+      hf_p = hf_c;
+      hs_c = sn;
+      hf_c = fn;
+      hrow_i += C;
+      hrow_f += C;
+      hbase = (hbase + 1 == K) ? 0 : hbase + 1;
+    }
+    __syncthreads();
+  }
+
+  // best final label (smallest on ties), then the traceback
+  if (tid < 32) {
+    const float* V = vs.V + (L & 1) * d.xPC;
+    float best = NEG_INF;
+    int bc = 0x7fffffff;
+    for (int x = tid; x < C; x += 32) {
+      const float v = V[x];
+      if (v > best || bc == 0x7fffffff) {
+        best = v;
+        bc = x;
+      }
+    }
+    gargmax<32>(best, bc);
+    if (tid == 0) score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
+    const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
+    int tt = L, cl = bc;
+    while (tt > 0) {
+      const int k = bp[(size_t)tt * C + cl] & 0xffff;
+      const int s = tt - k;
+      for (int u = s + tid; u < tt; u += 32) {
+        labels[(size_t)b * T + u] = cl;
+        seg_start[(size_t)b * T + u] = (u == s) ? 1 : 0;
+      }
+      if (s > 0) cl = (bp[(size_t)s * C + cl] >> 16) & 0xffff;
+      tt = s;
+    }
+  }
+}
+
+}  // namespace
+
+size_t viterbi_pipe_smem_bytes(const Dims& d) {
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
+         (2ull * d.xPC + 9ull * d.C) * 4;
+}
+
+}  // namespace semicrf
+
+namespace semicrf {
+
+cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                const float* trans, const float* dur, double* score,
+                                int32_t* labels, uint8_t* seg_start, cudaStream_t st) {
+  const size_t sm = viterbi_pipe_smem_bytes(d);
+#define SEMICRF_LAUNCH_VPIPE(g, cat, h, kbh, lb)                                               \
+  if (d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb) {               \
+    if (sm > 48 * 1024) {                                                                      \
+      const cudaError_t e = cudaFuncSetAttribute(viterbi_pipe_kernel<g, cat, h, kbh, lb>,      \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                                 (int)sm);                                     \
+      if (e != cudaSuccess) return e;                                                          \
+    }                                                                                          \
+    viterbi_pipe_kernel<g, cat, h, kbh, lb><<<d.B, d.xNT, sm, st>>>(d, ws, lengths, trans, dur,  \
+                                                                    score, labels, seg_start); \
+    return cudaGetLastError();                                                                 \
+  }
+  SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_VPIPE)
+#undef SEMICRF_LAUNCH_VPIPE
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace semicrf

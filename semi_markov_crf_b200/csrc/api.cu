@@ -75,7 +75,7 @@ void choose_xshape(Dims& d, size_t budget) {
     const int nt = 32 * (nwc + nwh);                                                      \
     if (C <= g * cat && K <= h * kbh + 2 && nt <= lb) {                                   \
       const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +        \
-                          10.0 * ((nwc + nwh + 3) / 4);                                   \
+                          10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0);       \
       if ((forced < 0 && cost < best) || forced == idx) {                                 \
         best = cost;                                                                      \
         d.xG = g;                                                                         \

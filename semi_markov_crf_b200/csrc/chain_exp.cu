@@ -1,6 +1,6 @@
 // chain_exp.cu -- steps 2 and 3: the forward and backward rings with the
-// label fan-in in the exponential domain on the critical path and the long
-// part of the duration fan-in computed one step ahead.
+// label fan-in in the exponential domain on the critical path and the rest of
+// each step computed one step ahead.
 //
 // "Streaming Structured Inference with Flash-SemiCRF", explainer section 2,
 // "Streaming Forward-Backward with Ring Buffers".  The recursion is the one of
@@ -18,31 +18,34 @@
 // one step late, so no reduction sits on the critical path.  With
 //   acc_s[c] = sum_{c'} p_s[c'] * 2^(trans2[c', c] - M)          (M = max trans2)
 // we have gamma[s, c] = Phi_s + M + log2 acc_s[c] (acc_0 = 2^-M, Phi_0 = 0), and
-//   p_t = 2^-n_t * ( acc_{t-1} A1 + acc_{t-2} A2 2^-n_{t-1} + O_t 2^(Z_t + sf_t - n_{t-1}) )
-//   A1 = 2^(M + dur2[0] + S[t] - S[t-1]),  A2 = 2^(M + dur2[1] + S[t] - S[t-2]),
-// where O_t 2^(Z_t + sf_t) is the k >= 3 part of the duration sum relative to
-// Phi_{t-2}.  Everything but acc_{t-1} and n_t is known when step t begins, so
-// the critical path of a step is: read p_{t-1} -> dot product with the
-// transition weights -> one multiply-add -> store p_t -> barrier.
+//   p_t = 2^-n_t * ( acc_{t-1} A1_t + 2^-n_{t-1} (acc_{t-2} A2_t + O_t) )
+//   A1_t = 2^(M + dur2[0] + S[t] - S[t-1]),  A2_t = 2^(M + dur2[1] + S[t] - S[t-2]),
+// where O_t is the k >= 3 part of the duration sum relative to Phi_{t-2}.
+// Everything but acc_{t-1} and n_t is known when step t begins, so the
+// critical path of a step is: read p_{t-1} -> dot product with the transition
+// weights -> two multiplies and a multiply-add -> store p_t -> barrier.
 //
 // Roles.  Combine warps (xG lanes per label, xCAT weights per lane) run that
-// path, keep acc_{t-2} and the rolling prefix-sum rows in registers, publish
+// path, keep acc_{t-2} and the previous prefix-sum row in registers, publish
 // n_t, and write gamma[t-1] into the label's ring in the log domain (off the
 // critical path; exactly the entry format of chain_kernel, so checkpoints and
 // the posterior kernel are shared).  Helper warps (xH lanes per label, xKBH
-// durations each) compute O_{t+1} for every label during step t from ring
-// entries of boundaries <= t-2 -- the same predicted-shift k fan-in as
-// chain_kernel -- and publish it before the step's barrier.  One CTA barrier
-// per step orders everything.
+// durations each, interleaved over the window so that a label's lanes read
+// consecutive ring entries) compute during step t everything step t+1 needs
+// besides acc_t: O_{t+1} -- the same predicted-shift k fan-in as chain_kernel,
+// from ring entries of boundaries <= t-2 -- and A1_{t+1}, A2_{t+1}.  One CTA
+// barrier per step orders everything.  The two directions are separate
+// instantiations (no per-step direction tests).
 //
 // Exactness.  The exponential domain is exact up to float32 rounding while
 // every label's alpha stays within fp32's exponent range of the frame.  Per
 // step, alpha[t, c] - max alpha[t-1] lies in
 //   [tmin + dmin - e, log2(K C) + max(tmax + dmax, dmax - dmin) + e]
 // (tmin/tmax, dmin/dmax: ranges of the finite transition and duration scores,
-// e: the largest |centred emission|), so the kernel takes a sequence only when
-// all scores are finite and that span is below FAST_BOUND; otherwise it
-// records mode 2 and chain_kernel (log domain, any input) runs the sequence.
+// e: the largest |centred emission|), and O_t spans two steps, so the kernel
+// takes a sequence only when all scores are finite and that span is below
+// FAST_BOUND (half the exponent range); otherwise it records mode 2 and
+// chain_kernel (log domain, any input) runs the sequence.
 #include "ring.cuh"
 
 namespace semicrf {
@@ -51,13 +54,14 @@ using namespace ring;
 
 namespace {
 
-constexpr float FAST_BOUND = 100.f;  // log2 units of exponent head-room (fp32 has 126)
+constexpr float FAST_BOUND = 60.f;  // log2 units; two steps stay inside fp32's 126
 
 struct XSmem {
   Smem s;      // mbar, tint, tfrac, ring (tile stream and ring helpers)
   float* P;    // [2][xPC] exp-domain label vector, by step parity
-  float* Oh;   // [2][C]   helper sums for the step of that parity
-  float* Zh;   // [2][C]   their integer shifts
+  float* Oh;   // [2][C]   k >= 3 sums for the step of that parity (frame Phi_{t-2})
+  float* A1;   // [2][C]   k = 1 factors
+  float* A2;   // [2][C]   k = 2 factors
   float* nsl;  // [2]      frame step n published by the combine warps
   int* aux;    // [4]      block reductions
   int* Sb;     // [C]      label integer bases of the prefix sums
@@ -78,14 +82,16 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   x.s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
   x.s.ring = reinterpret_cast<float2*>(p);
-  p += (size_t)d.xRL * C * sizeof(float2);
+  p += (size_t)d.xRLP * C * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
   float* f = reinterpret_cast<float*>(p);
   x.P = f;
   f += 2 * d.xPC;
   x.Oh = f;
   f += 2 * C;
-  x.Zh = f;
+  x.A1 = f;
+  f += 2 * C;
+  x.A2 = f;
   f += 2 * C;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
@@ -125,10 +131,311 @@ __device__ __forceinline__ bool xtile_wait(const Smem& sm, TileStream& ts, int t
   return !__syncthreads_or(!ok);
 }
 
-// Row r is the first one a walk in direction `up` meets in its tile.
-__device__ __forceinline__ bool first_in_tile(int r, bool up) {
-  return up ? (r % TS) == 0 : (r % TS) == TS - 1;
+// Smallest i' > i with i' = rem (mod TS), rem in [0, TS).
+__device__ __forceinline__ int next_mod(int i, int rem) {
+  const int x = (i / TS) * TS + rem;
+  return x > i ? x : x + TS;
 }
+
+// One ring (direction UP: forward over rows 1..L; else backward over rows
+// L-1..0) of sequence b, after the fast-path test has passed.
+template <bool UP, int G, int CAT, int H, int KBH>
+__device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPtrs& ws, int b,
+                                      int L, const float* __restrict__ trans,
+                                      const float* __restrict__ dur, float M,
+                                      double* __restrict__ logZ_out) {
+  const Smem& sm = xs.s;
+  const int C = d.C, K = d.K, tid = threadIdx.x;
+  constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
+  constexpr int NR = CAT > KBH ? CAT : KBH;
+  constexpr int SG = UP ? 1 : -1;  // walk direction over rows
+  const float sg = UP ? 1.f : -1.f;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nwc = (C + LPWC - 1) / LPWC;
+  const bool comb = warp < nwc;
+  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
+  const int jl = comb ? lane % G : lane % H;
+  const bool act = c < C;
+  const int cc = act ? c : 0;
+  const bool leader = act && jl == 0;
+  const int RL = K + WL, RLP = d.xRLP;
+  float2* const rl = sm.ring + (size_t)cc * RLP;
+  auto put = [&](int slot, float2 v) {  // slot and its mirrors slot + mK < RL
+    for (int x = slot; x < RL; x += K) rl[x] = v;
+  };
+
+  // One register array serves both roles: combine lanes keep the transition
+  // weights 2^(trans2 - M) of their CAT source labels (forward trans[x][c],
+  // backward trans[c][x]); helper lanes the durations of window index
+  // q*H + jl: k = 2 + WL - (q*H + jl) forward, 3 + q*H + jl backward.
+  float w[NR];
+  float d1 = NEG_INF, d2 = NEG_INF;
+  if (comb) {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int x = jl * CAT + q;
+      w[q] = (q < CAT && act && x < C)
+                 ? ex2(__ldg(trans + (UP ? (size_t)x * C + cc : (size_t)cc * C + x)) * l2e() - M)
+                 : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < NR; ++q) {
+      const int k = UP ? 2 + WL - (q * H + jl) : 3 + q * H + jl;
+      w[q] = (q < KBH && act && k <= K) ? __ldg(dur + (size_t)(k - 1) * C + cc) * l2e() : NEG_INF;
+    }
+    d1 = __ldg(dur + cc) * l2e();
+    if (K >= 2) d2 = __ldg(dur + C + cc) * l2e();
+  }
+
+  // ---------------------------------------------------------------- shared state
+  for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  for (int i = tid; i < 2 * d.xPC; i += blockDim.x) xs.P[i] = 0.f;
+  for (int i = tid; i < 2 * C; i += blockDim.x) {
+    xs.Oh[i] = 0.f;
+    xs.A1[i] = 0.f;
+    xs.A2[i] = 0.f;
+  }
+  if (tid == 0) {
+    xs.nsl[0] = xs.nsl[1] = 0.f;
+    mbar_init(&sm.mbar[0], 1);
+    mbar_init(&sm.mbar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int r0 = UP ? 0 : L;  // the walk's start boundary
+  const int r1 = r0 + SG;
+  TileStream ts;
+  ts.ph[0] = ts.ph[1] = 0;
+  ts.lo = 0;
+  ts.hi = L / TS;
+  ts.dir = SG;
+  tile_issue(sm, d, ws, b, ts, r0 / TS);
+  tile_issue(sm, d, ws, b, ts, r0 / TS + SG);
+  bool ok = xtile_wait(sm, ts, r0 / TS);
+  if (ok && r1 / TS != r0 / TS) ok = xtile_wait(sm, ts, r1 / TS);
+  if (!ok) {
+    if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+    tile_drain(sm, ts);
+    return;
+  }
+  const size_t o0 = tile_row_off(r0, C), o1 = tile_row_off(r1, C);
+  for (int x = tid; x < C; x += blockDim.x) {
+    // gamma[0] = 0 at S = 0 (forward); beta[L] = 0 at S[L] (backward)
+    const float2 v = make_float2(UP ? 0.f : sm.tfrac[o0 + x], 0.f);
+    float2* r = sm.ring + (size_t)x * RLP;
+    for (int y = r0 % K; y < RL; y += K) r[y] = v;
+    xs.Sb[x] = UP ? 0 : sm.tint[o0 + x];
+  }
+  // combine state: rows r-1 and r-2 (walk order) of S_int, row r-1 of S_frac,
+  // acc and n of the last step, the frame of p_{i-1} relative to F0
+  int si_p = UP ? 0 : sm.tint[o0 + cc], si_pp = si_p;
+  float sf_p = UP ? 0.f : sm.tfrac[o0 + cc];
+  float acc2 = 0.f, snprev = 1.f, Fp = 0.f;
+  int wslot = r0 % K;
+  const int32_t* crow_i = sm.tint + o1;
+  const float* crow_f = sm.tfrac + o1;
+  // helper state: rows r (cur) and r-1 (prev) of S, frame Phi_{i-1} - F0,
+  // predicted shift relative to Q, window base
+  int hs_c = sm.tint[o1 + cc], hs_p = si_p;
+  float hf_c = sm.tfrac[o1 + cc], hf_p = sf_p;
+  float Fph = 0.f, rel = 0.f;
+  const int32_t* hrow_i = sm.tint + o1 + SG * C;  // row r + SG of step 1
+  const float* hrow_f = sm.tfrac + o1 + SG * C;
+  int hbase = UP ? -WL : L + 1;  // window start boundary at step 1
+  hbase = ((hbase % K) + K) % K;
+  if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
+    xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
+  double F0 = 0.0;
+  __syncthreads();
+  int Sbc = xs.Sb[cc];
+  // checkpoint steps: forward boundary t = i - 1 at step i; backward
+  // boundary t1 = r + 2 at step i
+  const int delta = d.delta;
+  int next_ck;
+  if (UP) {
+    next_ck = delta + 1;
+  } else {
+    const int t1 = ((L - 1) / delta) * delta;
+    next_ck = (t1 >= delta && t1 >= 2) ? L + 2 - t1 : INT_MAX;
+  }
+  // events: a tile to wait for (the helpers' row opens a tile), a tile to
+  // issue (the combine's row opens a tile), a checkpoint, the last step
+  const int rem_w = UP ? TS - 1 : L % TS, rem_i = UP ? 0 : (L + 1) % TS;
+  auto next_event = [&](int i) {
+    return min(min(next_mod(i, rem_w), next_mod(i, rem_i)), min(next_ck, L));
+  };
+  int next_ev = next_event(0);
+
+  for (int i = 1; i <= L; ++i) {
+    const int r = UP ? i : L - i;
+    if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
+    if (i == next_ev) {
+      if (i < L && i % TS == rem_w) {
+        if (!xtile_wait(sm, ts, (r + SG) / TS)) {
+          if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
+          tile_drain(sm, ts);
+          return;
+        }
+        const size_t o = tile_row_off(r + SG, C);
+        hrow_i = sm.tint + o;
+        hrow_f = sm.tfrac + o;
+      }
+      if (i % TS == rem_i) {
+        tile_issue(sm, d, ws, b, ts, r / TS + SG);
+        const size_t o = tile_row_off(r, C);
+        crow_i = sm.tint + o;
+        crow_f = sm.tfrac + o;
+      }
+      if (i == next_ck) {
+        // rebase the ring to (F0 + D, S_int at the boundary) and save it
+        const int bnd = UP ? i - 1 : r + 2;
+        const int j = UP ? bnd / delta : bnd / delta - 1;
+        const float D = comb ? Fp : Fph;  // both are Phi_{i-1} - F0
+        if (comb) {
+          const int sit = UP ? si_p : si_pp;
+          if (act) {
+            const float adj = sg * (float)(sit - Sbc) - D;
+            for (int x = jl; x < RL; x += G) rl[x].y += adj;
+          }
+          __syncwarp();  // every lane of the warp, labels >= C included
+          if (act) {
+            float2* dst = (UP ? ws.ack : ws.bck) + (((size_t)b * d.nck + j) * K) * C + c;
+            for (int q = jl; q < K; q += G) {
+              const int bb = UP ? bnd - K + q : bnd + q;
+              if (UP ? bb >= 0 : bb <= L) dst[(size_t)q * C] = rl[bb % K];
+            }
+            if (leader) xs.Sb[c] = sit;
+          }
+        }
+        if (tid == 0) (UP ? ws.acf : ws.bcf)[(size_t)b * d.nck + j] = F0 + (double)D;
+        __syncthreads();
+        F0 += (double)D;
+        if (comb) {
+          Fp -= D;
+        } else {
+          Fph -= D;
+        }
+        Sbc = xs.Sb[cc];
+        next_ck += delta;
+        if (UP ? next_ck - 1 >= L : L + 2 - next_ck < delta) next_ck = INT_MAX;
+      }
+      next_ev = next_event(i);
+    }
+    if (comb) {
+      // ---------------------------------------------------------- combine
+      float acc, mx;
+      if (i == 1) {
+        acc = ex2(-M);  // the start boundary: gamma = 0 in frame 0
+        mx = 0.f;
+      } else {
+        const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+#pragma unroll
+        for (int q = 0; q < CAT; q += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(pv + q);
+          a0 = fmaf(v.x, w[q], a0);
+          a1 = fmaf(v.y, w[q + 1], a1);
+          a2 = fmaf(v.z, w[q + 2], a2);
+          a3 = fmaf(v.w, w[q + 3], a3);
+          m0 = fmaxf(m0, v.x);
+          m1 = fmaxf(m1, v.y);
+          m2 = fmaxf(m2, v.z);
+          m3 = fmaxf(m3, v.w);
+        }
+        acc = gsum<G>((a0 + a1) + (a2 + a3));
+        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
+      }
+      const float n = exponent_of(mx);
+      const float sn = pow2_neg(n);
+      const int po = (i & 1) * C + cc;
+      const float R = fmaf(acc2, xs.A2[po], xs.Oh[po]) * snprev;  // frame Phi_{i-1}
+      const float pn = fmaf(acc * sn, xs.A1[po], R * sn);
+      if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
+      if (tid == 0) xs.nsl[i & 1] = n;
+      if (i >= 2 && leader) {
+        // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
+        const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
+        put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
+      }
+      wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
+      acc2 = acc;
+      snprev = sn;
+      Fp += n;
+      si_pp = si_p;
+      si_p = crow_i[cc];
+      sf_p = crow_f[cc];
+      crow_i += SG * C;
+      crow_f += SG * C;
+    } else if (i < L) {
+      // ---------------------------------------------------------- helpers
+      const int sn = hrow_i[cc];
+      const float fn = hrow_f[cc];
+      const float Qh = sg * (float)(sn - Sbc) - Fph;
+      float m = Qh + rel;
+      float s;
+      const float lse = k_fanin_strided<KBH, H>(rl + hbase + jl, Qh, w, m, s, act);
+      if (isfinite(lse)) rel = rintf(lse - Qh);
+      // the three values step i+1 reads: lanes 0, 1, 2 of the group take one
+      // exponential each (no divergent branches); narrower groups take all
+      const float aO = m + sg * fn;
+      const float aA1 = (M + d1) + sg * ((float)(sn - hs_c) + (fn - hf_c));
+      const float aA2 = (M + d2) + sg * ((float)(sn - hs_p) + (fn - hf_p));
+      const int o2 = ((i + 1) & 1) * C + c;
+      if constexpr (H >= 3) {
+        const float e = ex2(jl == 0 ? aO : (jl == 1 ? aA1 : aA2));
+        if (act && jl == 0) xs.Oh[o2] = (s > 0.f) ? s * e : 0.f;
+        if (act && jl == 1) xs.A1[o2] = e;
+        if (act && jl == 2) xs.A2[o2] = e;
+      } else {
+        const float eO = ex2(aO), e1 = ex2(aA1), e2 = ex2(aA2);
+        if (leader) {
+          xs.Oh[o2] = (s > 0.f) ? s * eO : 0.f;
+          xs.A1[o2] = e1;
+          xs.A2[o2] = e2;
+        }
+      }
+      hs_p = hs_c;
+      hf_p = hf_c;
+      hs_c = sn;
+      hf_c = fn;
+      hrow_i += SG * C;
+      hrow_f += SG * C;
+      hbase = UP ? (hbase + 1 == K ? 0 : hbase + 1) : (hbase == 0 ? K - 1 : hbase - 1);
+    }
+    __syncthreads();
+  }
+
+  // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
+  if (warp == 0) {
+    float s = 0.f;
+    for (int x = lane; x < C; x += 32) s += xs.P[(L & 1) * d.xPC + x];
+    s = group_sum(s, 32);
+    if (lane == 0) {
+      const double lz = (s > 0.f) ? F0 + (double)Fp + (double)lg2(s) : -INFINITY;
+      if (UP) {
+        ws.logz2[b] = lz;
+        logZ_out[b] = lz * LN2_D;
+      } else {
+        ws.logz2b[b] = lz;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t chain_exp_smem_bytes(const Dims& d) {
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
+         (2ull * d.xPC + 7ull * d.C) * 4;
+}
+
+}  // namespace semicrf
+
+namespace semicrf {
+namespace {
 
 // ===========================================================================
 // One CTA per (direction, sequence): blockIdx.x < n_alpha runs the forward
@@ -143,7 +450,6 @@ __global__ void __launch_bounds__(LB, 1)
                      double* __restrict__ logZ_out, int n_alpha) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const XSmem xs = xcarve(smem_raw, d);
-  const Smem& sm = xs.s;
   const int C = d.C, K = d.K, tid = threadIdx.x;
   const bool up = (int)blockIdx.x < n_alpha;
   const int b = up ? blockIdx.x : blockIdx.x - n_alpha;
@@ -163,8 +469,7 @@ __global__ void __launch_bounds__(LB, 1)
     }
     return;
   }
-
-  // ---------------------------------------------------------------- the fast-path test
+  // ---- the fast-path test (identical in every CTA of the sequence)
   if (tid < 4) xs.aux[tid] = f2ord(NEG_INF);
   bool bad = false;
   for (int i = tid; i < C * C; i += blockDim.x) bad |= !isfinite(__ldg(trans + i));
@@ -181,283 +486,13 @@ __global__ void __launch_bounds__(LB, 1)
     return;
   }
   if (tid == 0) *mode = 1;
-
-  // ---------------------------------------------------------------- roles
-  constexpr int LPWC = 32 / G, LPWH = 32 / H;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int nwc = (C + LPWC - 1) / LPWC;
-  const bool comb = warp < nwc;
-  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
-  const int jl = comb ? lane % G : lane % H;
-  const bool act = c < C;
-  const int cc = act ? c : 0;
-  const bool leader = act && jl == 0;
-  const float sg = up ? 1.f : -1.f;
-  const int RL = d.xRL;
-  float2* const rl = sm.ring + (size_t)cc * RL;
-  // writes ring slot `slot` of this label and its mirrors (slot + mK < RL)
-  auto put = [&](int slot, float2 v) {
-    rl[slot] = v;
-    if (slot < KBH)
-      for (int x = slot + K; x < RL; x += K) rl[x] = v;
-  };
-
-  // One register array serves both roles: combine lanes keep the transition
-  // weights 2^(trans2 - M) of their CAT source labels (up: trans[x][c], down:
-  // trans[c][x]); helper lanes the durations of their window, k = 3 + jl*KBH
-  // + q (down) or k = 2 + (jl+1)*KBH - q (up), -inf beyond K.
-  constexpr int NR = CAT > KBH ? CAT : KBH;
-  float w[NR];
-  float d1 = NEG_INF, d2 = NEG_INF;
-  if (comb) {
-#pragma unroll
-    for (int q = 0; q < NR; ++q) {
-      const int x = jl * CAT + q;
-      w[q] = (q < CAT && act && x < C)
-                 ? ex2(__ldg(trans + (up ? (size_t)x * C + cc : (size_t)cc * C + x)) * l2e() - M)
-                 : 0.f;
-    }
-    d1 = __ldg(dur + cc) * l2e();
-    if (K >= 2) d2 = __ldg(dur + C + cc) * l2e();
-  } else {
-#pragma unroll
-    for (int q = 0; q < NR; ++q) {
-      const int k = up ? 2 + (jl + 1) * KBH - q : 3 + jl * KBH + q;
-      w[q] = (q < KBH && act && k <= K) ? __ldg(dur + (size_t)(k - 1) * C + cc) * l2e() : NEG_INF;
-    }
-  }
-
-  // ---------------------------------------------------------------- shared state
-  for (int i = tid; i < d.xRL * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
-  for (int i = tid; i < 2 * d.xPC; i += blockDim.x) xs.P[i] = 0.f;
-  for (int i = tid; i < 2 * C; i += blockDim.x) {
-    xs.Oh[i] = 0.f;
-    xs.Zh[i] = 0.f;
-  }
-  if (tid == 0) {
-    xs.nsl[0] = xs.nsl[1] = 0.f;
-    mbar_init(&sm.mbar[0], 1);
-    mbar_init(&sm.mbar[1], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const int r0 = up ? 0 : L;  // the walk's start boundary
-  TileStream ts;
-  ts.ph[0] = ts.ph[1] = 0;
-  ts.lo = 0;
-  ts.hi = L / TS;
-  ts.dir = up ? 1 : -1;
-  tile_issue(sm, d, ws, b, ts, r0 / TS);
-  tile_issue(sm, d, ws, b, ts, r0 / TS + ts.dir);
-  bool ok = xtile_wait(sm, ts, r0 / TS);
-  const int r1 = up ? 1 : L - 1;
-  if (ok && r1 / TS != r0 / TS) ok = xtile_wait(sm, ts, r1 / TS);
-  if (!ok) {
-    if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-    tile_drain(sm, ts);
-    return;
-  }
-  {
-    const size_t o0 = tile_row_off(r0, C);
-    for (int x = tid; x < C; x += blockDim.x) {
-      // gamma[0] = 0 at S = 0 (forward); beta[L] = 0 at S[L] (backward)
-      const float2 v = make_float2(up ? 0.f : sm.tfrac[o0 + x], 0.f);
-      float2* r = sm.ring + (size_t)x * RL;
-      r[r0 % K] = v;
-      if (r0 % K < KBH)
-        for (int y = r0 % K + K; y < RL; y += K) r[y] = v;
-      xs.Sb[x] = up ? 0 : sm.tint[o0 + x];
-    }
-  }
-  // combine state: rows r-1, r-2 (walk order) of S, acc of the last step,
-  // n of the last step, the frame of p_{i-1} relative to F0
-  int si_p = 0, si_pp = 0;
-  float sf_p = 0.f, sf_pp = 0.f;
-  {
-    const size_t o0 = tile_row_off(r0, C);
-    if (!up) {
-      si_p = si_pp = sm.tint[o0 + cc];
-      sf_p = sf_pp = sm.tfrac[o0 + cc];
-    }
-  }
-  float acc2 = 0.f, nprev = 0.f, snprev = 1.f, Fp = 0.f;
-  int wslot = r0 % K;  // ring slot of the previous row's boundary
-  // helper state: frame Phi_{i-1} relative to F0, label base, predicted shift
-  float Fph = 0.f, rel = 0.f;
-  int hbase = 0;
-  double F0 = 0.0;
-  __syncthreads();
-  int Sbc = xs.Sb[cc];
-  if (!comb) {
-    const int first = up ? 1 - 1 - (jl + 1) * KBH : L - 1 + 2 + jl * KBH;  // step 1's window
-    hbase = ((first % K) + K) % K;
-  }
-  // checkpoint steps: forward boundary t = i - 1 at step i; backward
-  // boundary t1 = r + 2 at step i
-  const int delta = d.delta;
-  int next_ck;
-  if (up) {
-    next_ck = delta + 1;
-  } else {
-    const int t1 = ((L - 1) / delta) * delta;
-    next_ck = (t1 >= delta && t1 >= 2) ? L + 2 - t1 : INT_MAX;
-  }
-
-  for (int i = 1; i <= L; ++i) {
-    const int r = up ? i : L - i;
-    // ---- frame of p_{i-1} for the helpers (published by the combine warps)
-    if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
-    // ---- prefix-sum tiles: wait for the next row's tile when the walk
-    // first needs it; refill the buffer the walk has left behind
-    if (i < L && first_in_tile(r + ts.dir, up)) {
-      if (!xtile_wait(sm, ts, (r + ts.dir) / TS)) {
-        if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
-        tile_drain(sm, ts);
-        return;
-      }
-    }
-    if (first_in_tile(r, up)) tile_issue(sm, d, ws, b, ts, r / TS + ts.dir);
-    // ---- checkpoint: rebase the ring to (F0 + D, S_int at the boundary) and save it
-    if (i == next_ck) {
-      const int bnd = up ? i - 1 : r + 2;
-      const int j = up ? bnd / delta : bnd / delta - 1;
-      const float D = comb ? Fp : Fph;  // both are Phi_{i-1} - F0
-      if (comb) {
-        // the G lanes of a label rebase its ring, then save it (every lane
-        // of the warp passes the __syncwarp, labels >= C included)
-        const int sit = up ? si_p : si_pp;
-        if (act) {
-          const float adj = sg * (float)(sit - Sbc) - D;
-          for (int x = jl; x < RL; x += G) rl[x].y += adj;
-        }
-        __syncwarp();
-        if (act) {
-          float2* dst = (up ? ws.ack : ws.bck) + (((size_t)b * d.nck + j) * K) * C + c;
-          for (int q = jl; q < K; q += G) {
-            const int bb = up ? bnd - K + q : bnd + q;
-            if (up ? bb >= 0 : bb <= L) dst[(size_t)q * C] = rl[bb % K];
-          }
-          if (leader) xs.Sb[c] = sit;
-        }
-        Sbc = sit;
-      }
-      if (tid == 0) (up ? ws.acf : ws.bcf)[(size_t)b * d.nck + j] = F0 + (double)D;
-      __syncthreads();
-      F0 += (double)D;
-      if (comb) {
-        Fp -= D;
-      } else {
-        Fph -= D;
-        Sbc = xs.Sb[cc];
-      }
-      next_ck += delta;
-      if (!up) {
-        if (L + 2 - next_ck < delta) next_ck = INT_MAX;  // t1 below delta: no more
-      } else if (next_ck - 1 >= L) {
-        next_ck = INT_MAX;
-      }
-    }
-    if (comb) {
-      // ---------------------------------------------------------- combine
-      float acc, mx;
-      if (i == 1) {
-        acc = ex2(-M);  // the start boundary: gamma = 0 in frame 0
-        mx = 0.f;
-      } else {
-        const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f;
-#pragma unroll
-        for (int q = 0; q < CAT; q += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(pv + q);
-          a0 = fmaf(v.x, w[q], a0);
-          a1 = fmaf(v.y, w[q + 1], a1);
-          a2 = fmaf(v.z, w[q + 2], a2);
-          a3 = fmaf(v.w, w[q + 3], a3);
-          m0 = fmaxf(m0, fmaxf(v.x, v.y));
-          m1 = fmaxf(m1, fmaxf(v.z, v.w));
-        }
-        acc = gsum<G>((a0 + a1) + (a2 + a3));
-        mx = fmaxf(m0, m1);
-#pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
-      }
-      const float n = exponent_of(mx);
-      const float sn = pow2_neg(n);
-      const size_t off = tile_row_off(r, C);
-      const int si = sm.tint[off + cc];
-      const float sf = sm.tfrac[off + cc];
-      const float A1 = ex2(((M + d1) + sg * (float)(si - si_p)) + sg * (sf - sf_p));
-      float R = 0.f;
-      if (i >= 2) {
-        const float A2 = ex2(((M + d2) + sg * (float)(si - si_pp)) + sg * (sf - sf_pp));
-        const float oh = xs.Oh[(i & 1) * C + cc];
-        const float fo = (oh > 0.f) ? ex2((xs.Zh[(i & 1) * C + cc] + sg * sf) - nprev) : 0.f;
-        R = fmaf(acc2 * A2, snprev, oh * fo);
-      }
-      const float pn = fmaf(acc * sn, A1, R * sn);
-      if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
-      if (tid == 0) xs.nsl[i & 1] = n;
-      if (i >= 2 && leader) {
-        // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
-        const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
-        put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
-      }
-      wslot = up ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
-      acc2 = acc;
-      nprev = n;
-      snprev = sn;
-      si_pp = si_p;
-      sf_pp = sf_p;
-      si_p = si;
-      sf_p = sf;
-      Fp += n;
-    } else if (i < L) {
-      // ---------------------------------------------------------- helpers
-      const size_t offn = tile_row_off(r + ts.dir, C);
-      const float Qh = sg * (float)(sm.tint[offn + cc] - Sbc) - Fph;
-      float m = Qh + rel;
-      float s;
-      float e[KBH], dh[KBH];
-#pragma unroll
-      for (int q = 0; q < KBH; ++q) dh[q] = w[q];
-      const float lse = k_fanin<KBH, H>(rl + hbase, Qh, dh, m, s, e);
-      if (leader) {
-        xs.Oh[((i + 1) & 1) * C + c] = s;
-        xs.Zh[((i + 1) & 1) * C + c] = m;
-      }
-      if (isfinite(lse)) rel = rintf(lse - Qh);
-      hbase = up ? (hbase + 1 == K ? 0 : hbase + 1) : (hbase == 0 ? K - 1 : hbase - 1);
-    }
-    __syncthreads();
-  }
-
-  // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
-  if (warp == 0) {
-    float s = 0.f;
-    for (int x = lane; x < C; x += 32) s += xs.P[(L & 1) * d.xPC + x];
-    s = group_sum(s, 32);
-    if (lane == 0) {
-      const double lz = (s > 0.f) ? F0 + (double)Fp + (double)lg2(s) : -INFINITY;
-      if (up) {
-        ws.logz2[b] = lz;
-        logZ_out[b] = lz * LN2_D;
-      } else {
-        ws.logz2b[b] = lz;
-      }
-    }
-  }
+  if (up)
+    xring<true, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out);
+  else
+    xring<false, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out);
 }
 
 }  // namespace
-
-size_t chain_exp_smem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRL * d.C * 8 + 16 +
-         (2ull * d.xPC + 5ull * d.C) * 4;
-}
-
-}  // namespace semicrf
-
-namespace semicrf {
 
 bool xshape_supported(int G, int CAT, int H, int KBH, int LB) {
 #define SEMICRF_XSHAPE_OK(g, cat, h, kbh, lb) \

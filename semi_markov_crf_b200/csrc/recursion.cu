@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float s;
         const float lse =
-            k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e);
+            k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float ssum;
         const float lse =
-            k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e);
+            k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
         const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = Bt;
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(LB, 1)
         const int si = ri[ln.cc];
         const float sf = rf[ln.cc];
         float s;
-        const float lse = k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e);
+        const float lse = k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(LB, 1)
       const int si = ri[ln.cc];
       const float sf = rf[ln.cc];
       float ksum;
-      const float lse = k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e);
+      const float lse = k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
       const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
       float St = 0.f;
       if (ln.leader) {

@@ -288,9 +288,12 @@ __device__ __forceinline__ void load_block(const float* p, float (&v)[CAT]) {
 // s = group sum.  If s leaves [2^-64, 2^64] the group redoes the fan-in
 // against ceil(exact max).  Returns the LSE (NEG_INF if nothing is finite);
 // on return m and s describe e[] (e[i] / s are the normalised weights).
+// `live` is false (uniformly over the group) for the padding groups of labels
+// >= C: their sum is 0 by construction and must not take the fallback, which
+// would hold up the rest of their warp every step.
 template <int KBT, int G>
 __device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (&d)[KBT], float& m,
-                                         float& s, float (&e)[KBT]) {
+                                         float& s, float (&e)[KBT], bool live = true) {
   {
     const float Qm = Q - m;  // exact: both integers
     float sp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -302,7 +305,7 @@ __device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (
     }
     s = gsum<G>((sp[0] + sp[1]) + (sp[2] + sp[3]));
   }
-  if (!(s >= 0x1p-64f && s <= 0x1p64f)) {
+  if (live && !(s >= 0x1p-64f && s <= 0x1p64f)) {
     // rare: the prediction was far off (or nothing is finite)
     const unsigned gm = gmask<G>();
     float mx = NEG_INF;
@@ -324,6 +327,49 @@ __device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (
     }
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gm, ss, o);
+    s = ss;
+  }
+  return (s > 0.f) ? m + lg2(s) : NEG_INF;
+}
+
+// k fan-in over a strided window: lane term q reads r[q * H] (the lanes of a
+// group interleave over consecutive ring entries, so a group's reads of one q
+// are contiguous), y_q = ((P + Q) + v) + dur2.  Same predicted-shift scheme
+// and fallback as k_fanin; returns the group LSE, m and s describe the sum.
+template <int KBH, int H, int N>
+__device__ __forceinline__ float k_fanin_strided(const float2* r, float Q, const float (&d)[N],
+                                                 float& m, float& s, bool live) {
+  static_assert(N >= KBH, "duration array shorter than the lane's terms");
+  {
+    const float Qm = Q - m;  // exact: both integers
+    float sp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < KBH; ++q) {
+      const float2 v = r[q * H];
+      sp[q & 3] += ex2(((v.y + Qm) + v.x) + d[q]);
+    }
+    s = gsum<H>((sp[0] + sp[1]) + (sp[2] + sp[3]));
+  }
+  if (live && !(s >= 0x1p-64f && s <= 0x1p64f)) {
+    const unsigned gm = gmask<H>();
+    float mx = NEG_INF;
+#pragma unroll
+    for (int q = 0; q < KBH; ++q) {
+      const float2 v = r[q * H];
+      mx = fmaxf(mx, ((v.y + Q) + v.x) + d[q]);
+    }
+#pragma unroll
+    for (int o = H / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gm, mx, o));
+    m = (mx == NEG_INF) ? 0.f : ceilf(mx);
+    const float Qm = Q - m;
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < KBH; ++q) {
+      const float2 v = r[q * H];
+      ss += ex2(((v.y + Qm) + v.x) + d[q]);
+    }
+#pragma unroll
+    for (int o = H / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gm, ss, o);
     s = ss;
   }
   return (s > 0.f) ? m + lg2(s) : NEG_INF;

@@ -178,6 +178,10 @@ __global__ void __launch_bounds__(LB, 1)
     int tt = L, c = bc;
     while (tt > 0) {
       const int k = bp[(size_t)tt * C + c] & 0xffff;
+      if (k < 1 || k > tt) {  // impossible for backpointers this kernel wrote
+        for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
+        break;
+      }
       const int s = tt - k;
       for (int u = s + tid; u < tt; u += 32) {
         labels[(size_t)b * T + u] = c;

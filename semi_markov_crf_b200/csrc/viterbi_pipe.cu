@@ -273,28 +273,33 @@ __global__ void __launch_bounds__(LB, 1)
     if (comb) {
       // ---------------------------------------------------------- combine
       float gv, mx = NEG_INF;
-      float vv[CAT];
+      float sv[CAT];  // this lane's label terms V[x] + trans2[x][c]
       if (i == 1) {
         gv = 0.f;  // G[0] = 0 in frame 0
 #pragma unroll
-        for (int q = 0; q < CAT; ++q) vv[q] = NEG_INF;
+        for (int q = 0; q < CAT; ++q) sv[q] = NEG_INF;
       } else {
         const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
-        float b0 = NEG_INF, b1 = NEG_INF, m0 = NEG_INF, m1 = NEG_INF;
+        float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
+        float m0 = NEG_INF, m1 = NEG_INF, m2 = NEG_INF, m3 = NEG_INF;
 #pragma unroll
         for (int q = 0; q < CAT; q += 4) {
           const float4 v = *reinterpret_cast<const float4*>(pv + q);
-          vv[q] = v.x;
-          vv[q + 1] = v.y;
-          vv[q + 2] = v.z;
-          vv[q + 3] = v.w;
-          b0 = fmaxf(b0, fmaxf(v.x + w[q], v.y + w[q + 1]));
-          b1 = fmaxf(b1, fmaxf(v.z + w[q + 2], v.w + w[q + 3]));
-          m0 = fmaxf(m0, fmaxf(v.x, v.y));
-          m1 = fmaxf(m1, fmaxf(v.z, v.w));
+          sv[q] = v.x + w[q];
+          sv[q + 1] = v.y + w[q + 1];
+          sv[q + 2] = v.z + w[q + 2];
+          sv[q + 3] = v.w + w[q + 3];
+          b0 = fmaxf(b0, sv[q]);
+          b1 = fmaxf(b1, sv[q + 1]);
+          b2 = fmaxf(b2, sv[q + 2]);
+          b3 = fmaxf(b3, sv[q + 3]);
+          m0 = fmaxf(m0, v.x);
+          m1 = fmaxf(m1, v.y);
+          m2 = fmaxf(m2, v.z);
+          m3 = fmaxf(m3, v.w);
         }
-        gv = fmaxf(b0, b1);
-        mx = fmaxf(m0, m1);
+        gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
+        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 #pragma unroll
         for (int o = G / 2; o > 0; o >>= 1) {
           gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
@@ -319,10 +324,14 @@ __global__ void __launch_bounds__(LB, 1)
       if (i >= 2) {
         // off the path: the best previous label (smallest on ties) and the
         // ring entry of G[i-1] (frame Phi_{i-1})
-        int bc = 0x7fffffff;
+        // bit q of the mask: term q attains the maximum (four independent
+        // chains, then the lowest set bit)
+        static_assert(CAT <= 64, "argmax mask is 64 bits");
+        unsigned long long mk[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int q = CAT - 1; q >= 0; --q)
-          if (vv[q] + w[q] == gv) bc = jl * CAT + q;
+        for (int q = 0; q < CAT; ++q) mk[q & 3] |= (sv[q] == gv ? 1ull : 0ull) << q;
+        const unsigned long long msk = (mk[0] | mk[1]) | (mk[2] | mk[3]);
+        int bc = msk ? jl * CAT + (__ffsll((long long)msk) - 1) : 0x7fffffff;
 #pragma unroll
         for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
         bc = min(bc, C - 1);  // every term -inf: an unreachable state, any label
@@ -395,16 +404,40 @@ __global__ void __launch_bounds__(LB, 1)
     }
     gargmax<32>(best, bc);
     if (tid == 0) score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
+    // Traceback.  Every issued tile has been waited for, so the two tile
+    // buffers are free: they hold WR = 4 TS rows of C backpointers, staged
+    // by the whole warp (coalesced) ahead of the serial walk, which then
+    // reads shared memory only.  A duration outside [1, t] (impossible for
+    // backpointers this kernel wrote) ends the walk with the positions not
+    // reached labelled -1.
     const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
+    int32_t* buf = sm.tint;
+    const int WR = 4 * TS;
+    int lo = L + 1;  // staged rows [lo, lo + WR)
+    auto stage = [&](int top) {
+      lo = max(0, top - WR + 1);
+      __syncwarp();
+      const int n = (top - lo + 1) * C;
+      for (int idx = tid; idx < n; idx += 32) buf[idx] = bp[(size_t)lo * C + idx];
+      __syncwarp();
+    };
     int tt = L, cl = bc;
     while (tt > 0) {
-      const int k = bp[(size_t)tt * C + cl] & 0xffff;
+      if (tt < lo) stage(tt);
+      const int k = buf[(tt - lo) * C + cl] & 0xffff;
+      if (k < 1 || k > tt) {
+        for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
+        break;
+      }
       const int s = tt - k;
       for (int u = s + tid; u < tt; u += 32) {
         labels[(size_t)b * T + u] = cl;
         seg_start[(size_t)b * T + u] = (u == s) ? 1 : 0;
       }
-      if (s > 0) cl = (bp[(size_t)s * C + cl] >> 16) & 0xffff;
+      if (s > 0) {
+        if (s < lo) stage(s);
+        cl = (buf[(s - lo) * C + cl] >> 16) & 0xffff;
+      }
       tt = s;
     }
   }

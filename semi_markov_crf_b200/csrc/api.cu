@@ -107,7 +107,18 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   d.T = T;
   d.C = C;
   d.K = K;
+  // Checkpoint spacing: ceil(sqrt(T K)) balances checkpoint memory against
+  // recompute, but memory is not what binds here -- the posterior pass runs
+  // one CTA per (segment, sequence) and each CTA walks 2 Delta serial steps.
+  // So Delta is also capped at what gives the batch about SEGMENTS_WANTED
+  // segments (two CTAs per SM), though never below 2K.  Any spacing gives the
+  // same results in exact arithmetic.
+  constexpr long long SEGMENTS_WANTED = 320;
   d.delta = T > 0 ? isqrt_ceil((long long)T * K) : 1;
+  if (T > 0) {
+    const long long par = ((long long)B * T + SEGMENTS_WANTED - 1) / SEGMENTS_WANTED;
+    d.delta = (int)std::min<long long>(d.delta, std::max<long long>(2LL * K, par));
+  }
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;

@@ -187,7 +187,14 @@ __global__ void __launch_bounds__(LB, 1)
         labels[(size_t)b * T + u] = c;
         seg_start[(size_t)b * T + u] = (u == s) ? 1 : 0;
       }
-      if (s > 0) c = (bp[(size_t)s * C + c] >> 16) & 0xffff;
+      if (s > 0) {
+        const int nc = (bp[(size_t)s * C + c] >> 16) & 0xffff;
+        if (nc >= C) {  // impossible for backpointers this kernel wrote
+          for (int u = tid; u < s; u += 32) labels[(size_t)b * T + u] = -1;
+          break;
+        }
+        c = nc;
+      }
       tt = s;
     }
   }

@@ -88,6 +88,12 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   return x;
 }
 
+// Dynamic shared memory of the kernel (carve order of vcarve).
+__host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
+         (2ull * d.xPC + 9ull * d.C) * 4;
+}
+
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
 __device__ __forceinline__ bool vtile_wait(const Smem& sm, TileStream& ts, int ti) {
   const int buf = ti & 1;
@@ -391,6 +397,7 @@ __global__ void __launch_bounds__(LB, 1)
   }
 
   // best final label (smallest on ties), then the traceback
+  __shared__ int s_tb[3];  // walk state shared by the block: row, label, pending
   if (tid < 32) {
     const float* V = vs.V + (L & 1) * d.xPC;
     float best = NEG_INF;
@@ -403,52 +410,73 @@ __global__ void __launch_bounds__(LB, 1)
       }
     }
     gargmax<32>(best, bc);
-    if (tid == 0) score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
-    // Traceback.  Every issued tile has been waited for, so the two tile
-    // buffers are free: they hold WR = 4 TS rows of C backpointers, staged
-    // by the whole warp (coalesced) ahead of the serial walk, which then
-    // reads shared memory only.  A duration outside [1, t] (impossible for
-    // backpointers this kernel wrote) ends the walk with the positions not
-    // reached labelled -1.
-    const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
-    int32_t* buf = sm.tint;
-    const int WR = 4 * TS;
-    int lo = L + 1;  // staged rows [lo, lo + WR)
-    auto stage = [&](int top) {
-      lo = max(0, top - WR + 1);
-      __syncwarp();
-      const int n = (top - lo + 1) * C;
-      for (int idx = tid; idx < n; idx += 32) buf[idx] = bp[(size_t)lo * C + idx];
-      __syncwarp();
-    };
-    int tt = L, cl = bc;
-    while (tt > 0) {
-      if (tt < lo) stage(tt);
-      const int k = buf[(tt - lo) * C + cl] & 0xffff;
-      if (k < 1 || k > tt) {
-        for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
-        break;
-      }
-      const int s = tt - k;
-      for (int u = s + tid; u < tt; u += 32) {
-        labels[(size_t)b * T + u] = cl;
-        seg_start[(size_t)b * T + u] = (u == s) ? 1 : 0;
-      }
-      if (s > 0) {
-        if (s < lo) stage(s);
-        cl = (buf[(s - lo) * C + cl] >> 16) & 0xffff;
-      }
-      tt = s;
+    if (tid == 0) {
+      score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
+      s_tb[0] = L;
+      s_tb[1] = bc;
+      s_tb[2] = 0;
     }
+  }
+  __syncthreads();
+  // Traceback.  The whole dynamic shared memory is free now: the block
+  // stages as many backpointer rows as fit (coalesced, every thread), warp 0
+  // walks them, and the block stages the next rows where the walk left off.
+  // A walk state (row tt, label cl) may carry a pending previous-label
+  // lookup at row tt when that row was not yet staged.  A duration outside
+  // [1, t] or a previous label >= C (impossible for backpointers this kernel
+  // wrote) ends the walk with the positions not reached labelled -1.
+  const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
+  int32_t* buf = reinterpret_cast<int32_t*>(smem_raw + 64);
+  const int WR = (int)((vsmem_bytes(d) - 64) / ((size_t)C * 4));
+  for (;;) {
+    const int tt0 = s_tb[0];
+    if (tt0 <= 0) break;
+    const int lo = max(0, tt0 - WR + 1);
+    for (int idx = tid; idx < (tt0 - lo + 1) * C; idx += blockDim.x) buf[idx] = bp[(size_t)lo * C + idx];
+    __syncthreads();
+    if (tid < 32) {
+      int tt = tt0, cl = s_tb[1];
+      bool pend = s_tb[2] != 0, stop = false;
+      while (tt > 0) {
+        if (pend) {  // previous label of a segment starting at tt
+          const int nc = (buf[(tt - lo) * C + cl] >> 16) & 0xffff;
+          if (nc >= C) {
+            for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
+            stop = true;
+            break;
+          }
+          cl = nc;
+          pend = false;
+        }
+        const int k = buf[(tt - lo) * C + cl] & 0xffff;
+        if (k < 1 || k > tt) {
+          for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
+          stop = true;
+          break;
+        }
+        const int sb = tt - k;
+        for (int u = sb + tid; u < tt; u += 32) {
+          labels[(size_t)b * T + u] = cl;
+          seg_start[(size_t)b * T + u] = (u == sb) ? 1 : 0;
+        }
+        tt = sb;
+        pend = true;
+        if (tt < lo) break;  // next rows not staged yet
+      }
+      __syncwarp();
+      if (tid == 0) {
+        s_tb[0] = stop ? 0 : tt;
+        s_tb[1] = cl;
+        s_tb[2] = pend ? 1 : 0;
+      }
+    }
+    __syncthreads();
   }
 }
 
 }  // namespace
 
-size_t viterbi_pipe_smem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 9ull * d.C) * 4;
-}
+size_t viterbi_pipe_smem_bytes(const Dims& d) { return vsmem_bytes(d); }
 
 }  // namespace semicrf
 

@@ -219,6 +219,8 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segT = reinterpret_cast<double*>(c + o_segT);
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
+    p->fst = nullptr;  // per-boundary forward values: not kept (no consumer)
+    p->fsf = nullptr;
     p->emax = reinterpret_cast<float*>(c + o_emax);
     p->mode = reinterpret_cast<int*>(c + o_mode);
   }
@@ -301,6 +303,10 @@ int run_chains(const Dims& d, WsPtrs p, const int32_t* lengths, const float* tra
     ProfScope ps("chain_exp_kernel", st);
     e = launch_chain_exp(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st);
   } else {
+    // no ring kept anything: the posterior pass must not trust a record left
+    // in the workspace by an earlier call
+    if (cudaMemsetAsync(p.mode, 0, 2ull * d.B * sizeof(int), st) != cudaSuccess)
+      return SEMICRF_ERR_CUDA;
     p.mode = nullptr;  // the log-domain kernel runs every sequence
   }
   if (e != cudaSuccess) return SEMICRF_ERR_CUDA;

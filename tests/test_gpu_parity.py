@@ -94,6 +94,27 @@ def test_ring_domain_choice():
         assert semicrf.ring_domains(ws) == [2] * (2 * B), name
 
 
+def test_log_domain_ignores_a_stale_workspace():
+    """A workspace whose bytes say that every ring ran in the exponential
+    domain and kept its values (int32 ones everywhere) must not mislead a
+    log-domain forward-backward on it."""
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make("genomic", B=2, T=3000, seed=26)
+    em, lengths, trans, dur = to_dev(case)
+    B, T, C = case["em"].shape
+    K = case["dur"].shape[0]
+    ws = semicrf.Workspace(B, T, C, K, semicrf.FLAG_LOG_DOMAIN, em.device)
+    ws.buf.view(torch.int32).fill_(1)
+    logZ, ws = semicrf.forward(em, lengths, trans, dur, ws=ws, log_domain=True)
+    out = semicrf.backward(ws, lengths, trans, dur, marginals=True)
+    assert semicrf.get_status(ws) == 0
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    got["logZ"] = logZ.cpu().numpy()
+    ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"], K)
+    print(errors(got, ref))
+    assert_fb_close(got, ref, case["lengths"], "stale workspace")
+
+
 def test_moderately_loud_inputs_stay_exact_in_the_exponential_domain():
     """Emissions x3 (per-step exponent span about 60 of fp32's 126): still the
     exponential domain, still within tolerance."""

@@ -219,8 +219,6 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segT = reinterpret_cast<double*>(c + o_segT);
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
-    p->fst = nullptr;  // per-boundary forward values: not kept (no consumer)
-    p->fsf = nullptr;
     p->emax = reinterpret_cast<float*>(c + o_emax);
     p->mode = reinterpret_cast<int*>(c + o_mode);
   }

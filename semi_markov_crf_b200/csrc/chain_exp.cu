@@ -247,14 +247,6 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
     xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
-  // forward: keep log alpha / log gamma per boundary (alpha[0] = -inf, frame 0)
-  const bool keep = UP && ws.fst != nullptr;
-  float* const fst = keep ? ws.fst + (size_t)b * (d.T + 1) * 2 * C : nullptr;
-  double* const fsf = keep ? ws.fsf + (size_t)b * (d.T + 1) : nullptr;
-  if (keep) {
-    for (int x = tid; x < C; x += blockDim.x) fst[x] = NEG_INF;
-    if (tid == 0) fsf[0] = 0.0;
-  }
   __syncthreads();
   int Sbc = xs.Sb[cc];
   // checkpoint steps: forward boundary t = i - 1 at step i; backward
@@ -363,18 +355,11 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float pn = fmaf(acc * sn, xs.A1[po], R * sn);
       if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
       if (tid == 0) xs.nsl[i & 1] = n;
-      if (leader && (i >= 2 || (UP && keep))) {
+      if (i >= 2 && leader) {
         // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
         const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
-        if (i >= 2) put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
-        if (UP && keep) {
-          // the forward ring keeps log alpha[i] and log gamma[i-1] for the
-          // posterior pass, each relative to its boundary's frame
-          fst[(size_t)i * 2 * C + c] = (pn > 0.f) ? lg2(pn) : NEG_INF;
-          fst[(size_t)(i - 1) * 2 * C + C + c] = g;
-        }
+        put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
       }
-      if (UP && keep && tid == 0) fsf[i] = F0 + (double)(Fp + n);
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;

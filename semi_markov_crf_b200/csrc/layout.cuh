@@ -66,9 +66,6 @@ struct WsPtrs {
   double* segT;    // [B][nck][C] per-segment sum of (start - end) marginals
   double* segV;    // [B][nck][C] per-segment sum of the within-segment suffix sums
   int32_t* bp;     // [B][T+1][C] Viterbi backpointers
-  float* fst;      // [B][T+1][2C] forward ring's log alpha and log gamma per boundary,
-                   //   each relative to the boundary's frame (null: not kept)
-  double* fsf;     // [B][T+1] that frame (absolute, log2 units)
   float* emax;     // [B] largest |centred emission| * log2(e) over the valid positions
   int* mode;       // [2][B] ring path per (direction, sequence): 1 exponential, 2 log domain
 };

@@ -28,9 +28,11 @@
 // smallest final label; a re-scan finds each argmax once the maximum is
 // known (equal floating-point sums compare bit-exactly).
 //
-// Backpointers: bits 0-15 of bp[t, c] hold the best duration of a segment of
-// label c ending at t (written in step t), bits 16-31 the best previous label
-// of a segment of label c starting at t (written in step t+1).
+// Backpointers: bp[t, c] holds, for the best segment of label c ending at
+// t, its duration k (bits 0-15) and the best label before it (bits 16-31,
+// the argmax of G[t-k, c]).  The argmax labels of recent boundaries live in
+// a K-slot ring per label in shared memory, so the word is complete when step
+// t writes it and the traceback reads one word per decoded segment.
 #include "ring.cuh"
 
 namespace semicrf {
@@ -50,6 +52,7 @@ struct VSmem {
   float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
   float* nsl;  // [2]       frame step published by the combine warps
   int* Sb;     // [C]       label integer bases
+  int16_t* lab;  // [C][K]  argmax label of G[b, c] for the last K boundaries b
 };
 
 __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
@@ -80,6 +83,8 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   x.A2 = f;
   f += 2 * C;
   x.Sb = reinterpret_cast<int*>(f);
+  f += C;
+  x.lab = reinterpret_cast<int16_t*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
   x.s.tmp = nullptr;
@@ -91,7 +96,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 9ull * d.C) * 4;
+         (2ull * d.xPC + 9ull * d.C) * 4 + (size_t)d.C * d.K * 2 + 16;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -172,6 +177,7 @@ __global__ void __launch_bounds__(LB, 1)
   // ---------------------------------------------------------------- shared state
   for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) vs.V[i] = NEG_INF;
+  for (int i = tid; i < C * K; i += blockDim.x) vs.lab[i] = 0;
   for (int i = tid; i < 2 * C; i += blockDim.x) {
     vs.Om[i] = NEG_INF;
     vs.Ok[i] = 3;
@@ -224,7 +230,7 @@ __global__ void __launch_bounds__(LB, 1)
   const float* crow_f = sm.tfrac + C;
   int wslot = 0;
   double F0 = 0.0;
-  int16_t* bp16 = reinterpret_cast<int16_t*>(ws.bp + (size_t)b * (T + 1) * C);
+  int32_t* bpw = ws.bp + (size_t)b * (T + 1) * C;
   __syncthreads();
   int Sbc = 0;
   int next_rb = VREBASE + 1;
@@ -321,10 +327,11 @@ __global__ void __launch_bounds__(LB, 1)
       const float c2 = (g2 + a2) - nprev;
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
+      int kdec = 1;
       if (leader) {
         vs.V[(i & 1) * d.xPC + c] = v - n;
         const int k = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : vs.Ok[(i & 1) * C + cc]);
-        bp16[((size_t)i * C + c) * 2] = (int16_t)k;
+        kdec = k;
       }
       if (tid == 0) vs.nsl[i & 1] = n;
       if (i >= 2) {
@@ -342,11 +349,19 @@ __global__ void __launch_bounds__(LB, 1)
         for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
         bc = min(bc, C - 1);  // every term -inf: an unreachable state, any label
         if (leader) {
-          bp16[((size_t)(i - 1) * C + c) * 2 + 1] = (int16_t)bc;
+          // the previous label of the best segment ending at i: this step's
+          // argmax for k = 1, the ring's entry of boundary i - k otherwise
+          vs.lab[(size_t)c * K + wslot] = (int16_t)bc;  // boundary i - 1
+          int ps = wslot - kdec + 1;
+          if (ps < 0) ps += K;
+          const int pred = (kdec == 1) ? bc : vs.lab[(size_t)c * K + ps];
+          bpw[(size_t)i * C + c] = kdec | (pred << 16);
           const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
           rl[wslot] = e;
           for (int x = wslot + K; x < RL; x += K) rl[x] = e;
         }
+      } else if (leader) {
+        bpw[(size_t)C + c] = kdec;  // segment [0, 1): nothing before it
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
       g2 = gv;
@@ -397,7 +412,7 @@ __global__ void __launch_bounds__(LB, 1)
   }
 
   // best final label (smallest on ties), then the traceback
-  __shared__ int s_tb[3];  // walk state shared by the block: row, label, pending
+  __shared__ int s_tb[2];  // walk state shared by the block: row, label
   if (tid < 32) {
     const float* V = vs.V + (L & 1) * d.xPC;
     float best = NEG_INF;
@@ -414,17 +429,15 @@ __global__ void __launch_bounds__(LB, 1)
       score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
       s_tb[0] = L;
       s_tb[1] = bc;
-      s_tb[2] = 0;
     }
   }
   __syncthreads();
   // Traceback.  The whole dynamic shared memory is free now: the block
   // stages as many backpointer rows as fit (coalesced, every thread), warp 0
-  // walks them, and the block stages the next rows where the walk left off.
-  // A walk state (row tt, label cl) may carry a pending previous-label
-  // lookup at row tt when that row was not yet staged.  A duration outside
-  // [1, t] or a previous label >= C (impossible for backpointers this kernel
-  // wrote) ends the walk with the positions not reached labelled -1.
+  // walks them -- one word per decoded segment -- and the block stages the
+  // next rows where the walk left off.  A duration outside [1, t] or a
+  // previous label >= C (impossible for backpointers this kernel wrote) ends
+  // the walk with the positions not reached labelled -1.
   const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
   int32_t* buf = reinterpret_cast<int32_t*>(smem_raw + 64);
   const int WR = (int)((vsmem_bytes(d) - 64) / ((size_t)C * 4));
@@ -436,22 +449,12 @@ __global__ void __launch_bounds__(LB, 1)
     __syncthreads();
     if (tid < 32) {
       int tt = tt0, cl = s_tb[1];
-      bool pend = s_tb[2] != 0, stop = false;
-      while (tt > 0) {
-        if (pend) {  // previous label of a segment starting at tt
-          const int nc = (buf[(tt - lo) * C + cl] >> 16) & 0xffff;
-          if (nc >= C) {
-            for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
-            stop = true;
-            break;
-          }
-          cl = nc;
-          pend = false;
-        }
-        const int k = buf[(tt - lo) * C + cl] & 0xffff;
-        if (k < 1 || k > tt) {
+      while (tt >= lo && tt > 0) {
+        const int w = buf[(tt - lo) * C + cl];
+        const int k = w & 0xffff, pred = (w >> 16) & 0xffff;
+        if (k < 1 || k > tt || (tt - k > 0 && pred >= C)) {
           for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
-          stop = true;
+          tt = 0;
           break;
         }
         const int sb = tt - k;
@@ -460,14 +463,12 @@ __global__ void __launch_bounds__(LB, 1)
           seg_start[(size_t)b * T + u] = (u == sb) ? 1 : 0;
         }
         tt = sb;
-        pend = true;
-        if (tt < lo) break;  // next rows not staged yet
+        cl = pred;
       }
       __syncwarp();
       if (tid == 0) {
-        s_tb[0] = stop ? 0 : tt;
+        s_tb[0] = tt;
         s_tb[1] = cl;
-        s_tb[2] = pend ? 1 : 0;
       }
     }
     __syncthreads();

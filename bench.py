@@ -93,6 +93,9 @@ def mufu_ops_per_position(kernel: str, K: int, C: int) -> int:
         return 2 * one_ring
     if kernel == "segment_kernel":
         return 2 * one_ring + 2 * C
+    if kernel == "posterior_kernel":
+        # one exponential per (start, duration, label) term and per boundary
+        return K * C + 1
     return 0
 
 

@@ -122,6 +122,8 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
+  d.GS = 128;
+  d.ngrid = T > 0 ? (T - 1) / d.GS + 2 : 1;  // positions 0, GS, 2GS, ... and L - 1
   // Kernel shape: G lanes per label (a power of two), each with KBT durations
   // and CAT labels, picked from the instantiated menu by a latency model.
   // Per step about one warp runs per scheduler and the step is latency
@@ -199,6 +201,9 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_segT = take(B * nck * C * 8);
   const size_t o_segV = take(B * nck * C * 8);
   const size_t o_bp = take(B * (size_t)(d.T + 1) * C * 4);
+  const size_t o_kv = take(B * 2ull * (d.T + 1) * 2 * C * 4);
+  const size_t o_kf = take(B * 2ull * (d.T + 1) * 8);
+  const size_t o_ncut = take(B * (size_t)d.ngrid * 8);
   const size_t o_emax = take(B * 4);
   const size_t o_mode = take(2 * B * 4);
   if (base && p) {
@@ -219,6 +224,9 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segT = reinterpret_cast<double*>(c + o_segT);
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
+    p->kv = reinterpret_cast<float*>(c + o_kv);
+    p->kf = reinterpret_cast<double*>(c + o_kf);
+    p->ncut = reinterpret_cast<double*>(c + o_ncut);
     p->emax = reinterpret_cast<float*>(c + o_emax);
     p->mode = reinterpret_cast<int*>(c + o_mode);
   }
@@ -409,6 +417,22 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     if (rc) return rc;
   }
   if (T > 0) {
+    // sequences whose rings both ran in the exponential domain: posteriors
+    // from the kept values (cut normalisers, then one parallel pass); the
+    // others: the checkpoint walk.  Each kernel skips the other's sequences.
+    {
+      ProfScope ps("cut_grid_kernel", st);
+      cut_grid_kernel<<<dim3(d.ngrid, B), 256, 0, st>>>(d, p, lengths, trans, dur);
+    }
+    if ((rc = launched())) return rc;
+    const size_t psm = posterior_smem_bytes(d);
+    if ((rc = set_smem((const void*)posterior_kernel, psm))) return rc;
+    {
+      ProfScope ps("posterior_kernel", st);
+      posterior_kernel<<<dim3(d.nck, B), 512, psm, st>>>(d, p, lengths, trans, dur, grad_logZ,
+                                                         grad_em, start_marg, end_marg);
+    }
+    if ((rc = launched())) return rc;
     cudaError_t e;
     {
       ProfScope ps("segment_kernel", st);

@@ -247,6 +247,19 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
     xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
+  // kept values for the posterior pass: per boundary (row) the vector p and
+  // the label fan-in acc, both relative to the boundary's frame kf
+  const int dir = UP ? 0 : 1;
+  float* const kv = ws.kv ? ws.kv + (((size_t)b * 2 + dir) * (d.T + 1)) * 2 * C : nullptr;
+  double* const kf = ws.kf ? ws.kf + ((size_t)b * 2 + dir) * (d.T + 1) : nullptr;
+  if (kv) {
+    const int rL = UP ? L : 0;  // the walk's last row: no label fan-in there
+    for (int x = tid; x < C; x += blockDim.x) {
+      kv[(size_t)r0 * 2 * C + x] = 0.f;  // no forward vector at 0, no btil at L
+      kv[(size_t)rL * 2 * C + C + x] = 0.f;
+    }
+    if (tid == 0) kf[r0] = 0.0;
+  }
   __syncthreads();
   int Sbc = xs.Sb[cc];
   // checkpoint steps: forward boundary t = i - 1 at step i; backward
@@ -355,6 +368,13 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float pn = fmaf(acc * sn, xs.A1[po], R * sn);
       if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
       if (tid == 0) xs.nsl[i & 1] = n;
+      if (kv) {
+        if (leader) {
+          kv[(size_t)r * 2 * C + c] = pn;                       // frame Phi_i
+          kv[(size_t)(r - SG) * 2 * C + C + c] = acc;           // frame Phi_{i-1}
+        }
+        if (tid == 0) kf[r] = F0 + (double)(Fp + n);
+      }
       if (i >= 2 && leader) {
         // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
         const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;

@@ -43,10 +43,13 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x < C && L > 0) {
     const int c = threadIdx.x;
     const int nseg = (L + delta - 1) / delta;
+    // segT: mu[t0 - 1] + segment total (segment_kernel, its own carry from
+    // the cut) or the plain segment total (posterior_kernel: running sum)
+    const bool cum = posterior_from_kept(ws, d, b);
     double run = 0.0, msum = 0.0;
     for (int j = 0; j < nseg; ++j) {
       const size_t o = ((size_t)b * d.nck + j) * C + c;
-      run = ws.segT[o];
+      run = cum ? run + ws.segT[o] : ws.segT[o];
       const int len = min((j + 1) * delta, L) - j * delta;
       msum += (double)len * run - ws.segV[o];
       if (j >= j_lo && j <= j_hi) pinc[(j - j_lo) * C + c] = run;

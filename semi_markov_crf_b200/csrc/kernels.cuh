@@ -42,6 +42,22 @@ __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restr
 
 __global__ void selftest_wait_kernel(int* status, int spins);
 
+// Posteriors of sequence b come from the values both exponential-domain
+// rings kept (posterior.cu) rather than from the checkpoint walk
+// (segment_kernel).  The same test in every kernel that depends on it.
+__device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims& d, int b) {
+  return ws.kv != nullptr && ws.mode != nullptr && ws.mode[b] == 1 && ws.mode[d.B + b] == 1;
+}
+
+__global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                                const float* __restrict__ trans, const float* __restrict__ dur);
+__global__ void posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                                 const float* __restrict__ trans, const float* __restrict__ dur,
+                                 const double* __restrict__ grad_logZ,
+                                 float* __restrict__ grad_em, float* __restrict__ start_marg,
+                                 float* __restrict__ end_marg);
+size_t posterior_smem_bytes(const Dims& d);
+
 // Sizes, launch geometry and limits for (B, T, C, K); returns a semicrf_status.
 int make_dims(int B, int T, int C, int K, Dims& d);
 

@@ -46,6 +46,9 @@ struct Dims {
   // xH * xKBH entries apart, padded so that a half warp's 64-bit reads of
   // consecutive entries of different labels fall in distinct banks.
   int xRLP;
+  // Posteriors from kept ring values (posterior.cu): cut normaliser every
+  // GS positions, ngrid grid points per sequence.
+  int GS, ngrid;
 };
 
 // Device pointers into the caller's workspace.
@@ -66,6 +69,10 @@ struct WsPtrs {
   double* segT;    // [B][nck][C] per-segment sum of (start - end) marginals
   double* segV;    // [B][nck][C] per-segment sum of the within-segment suffix sums
   int32_t* bp;     // [B][T+1][C] Viterbi backpointers
+  float* kv;       // [B][2][T+1][2][C] exponential-domain ring values per boundary:
+                   //   direction (forward, backward) x (p, acc), relative to the frame
+  double* kf;      // [B][2][T+1] that frame (absolute, log2 units)
+  double* ncut;    // [B][ngrid] log2 of the cut normaliser at the grid positions
   float* emax;     // [B] largest |centred emission| * log2(e) over the valid positions
   int* mode;       // [2][B] ring path per (direction, sequence): 1 exponential, 2 log domain
 };

@@ -417,6 +417,7 @@ __global__ void __launch_bounds__(LB, 1)
   const int j = blockIdx.x, b = blockIdx.y;
   const int L = lengths[b];
   if (L < 0 || L > d.T) return;  // reported by the forward pass
+  if (posterior_from_kept(ws, d, b)) return;  // posterior_kernel runs it
   const int t0 = j * d.delta;
   if (t0 >= L) return;
   const int t1 = min(t0 + d.delta, L);

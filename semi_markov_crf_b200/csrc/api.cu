@@ -62,6 +62,7 @@ void choose_xshape(Dims& d, size_t budget) {
   int forced = -1;
   if (const char* env = std::getenv("SEMICRF_XSHAPE")) forced = std::atoi(env);
   d.xG = 0;
+  d.pRT = 0;
   double best = 1e30;
   int idx = 0;
   auto lg = [](int v) {
@@ -92,10 +93,16 @@ void choose_xshape(Dims& d, size_t budget) {
 #undef SEMICRF_XCONSIDER
   if (d.xG == 0) return;
   d.xRL = K + d.xKBH;
-  d.xPC = d.xG * d.xCAT;
+  // label vector row: the combine lanes' blocks (xG x xCAT) and the helper
+  // lanes' strided sources (xH x ceil(xG xCAT / xH)), whichever is longer
+  d.xPC = std::max(d.xG * d.xCAT, d.xH * ((d.xG * d.xCAT + d.xH - 1) / d.xH));
   d.xRLP = K + d.xH * d.xKBH;
   if (d.xH < 16) d.xRLP += (((d.xH - d.xRLP) % 16) + 16) % 16;
-  if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget) d.xG = 0;
+  // the posterior pass from the kept values must fit too
+  d.pRT = posterior_tile_rows(d, budget);
+  if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget || d.pRT == 0 ||
+      cut_grid_smem_bytes(d) > budget)
+    d.xG = 0;
 }
 
 // Sizes, lane mapping and limits.  Returns a semicrf_status.
@@ -420,20 +427,21 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     // sequences whose rings both ran in the exponential domain: posteriors
     // from the kept values (cut normalisers, then one parallel pass); the
     // others: the checkpoint walk.  Each kernel skips the other's sequences.
-    {
-      ProfScope ps("cut_grid_kernel", st);
-      cut_grid_kernel<<<dim3(d.ngrid, B), 256, 0, st>>>(d, p, lengths, trans, dur);
-    }
-    if ((rc = launched())) return rc;
-    const size_t psm = posterior_smem_bytes(d);
-    if ((rc = set_smem((const void*)posterior_kernel, psm))) return rc;
-    {
-      ProfScope ps("posterior_kernel", st);
-      posterior_kernel<<<dim3(d.nck, B), 512, psm, st>>>(d, p, lengths, trans, dur, grad_logZ,
-                                                         grad_em, start_marg, end_marg);
-    }
-    if ((rc = launched())) return rc;
     cudaError_t e;
+    if (d.xG) {
+      const size_t csm = cut_grid_smem_bytes(d);
+      if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
+      {
+        ProfScope ps("cut_grid_kernel", st);
+        cut_grid_kernel<<<dim3(d.ngrid, B), 256, csm, st>>>(d, p, lengths, trans, dur);
+      }
+      if ((rc = launched())) return rc;
+      {
+        ProfScope ps("posterior_kernel", st);
+        e = launch_posterior(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
+      }
+      if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    }
     {
       ProfScope ps("segment_kernel", st);
       e = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
@@ -461,7 +469,8 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
   const int ne = C * C + K * C;
   {
     ProfScope ps("reduce_partials_kernel", st);
-    reduce_partials_kernel<<<(ne + 255) / 256, 256, 0, st>>>(d, p, lengths, grad_trans, grad_dur);
+    reduce_partials_kernel<<<(ne + RP_E - 1) / RP_E, RP_E * RP_S, 0, st>>>(d, p, lengths, grad_trans,
+                                                                      grad_dur);
   }
   return launched();
 }

@@ -62,6 +62,7 @@ struct XSmem {
   float* Oh;   // [2][C]   k >= 3 sums for the step of that parity (frame Phi_{t-2})
   float* A1;   // [2][C]   k = 1 factors
   float* A2;   // [2][C]   k = 2 factors
+  float* KS;   // [2][2C]  kept values of the step of that parity: p, acc
   float* nsl;  // [2]      frame step n published by the combine warps
   int* aux;    // [4]      block reductions
   int* Sb;     // [C]      label integer bases of the prefix sums
@@ -93,6 +94,8 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   f += 2 * C;
   x.A2 = f;
   f += 2 * C;
+  x.KS = f;
+  f += 4 * C;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
@@ -335,6 +338,14 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       }
       next_ev = next_event(i);
     }
+    if (kv && !comb && i >= 2) {
+      // the helpers write out the kept values the combine staged last step
+      // (rows r - SG: p, r - 2 SG: acc), off the critical path
+      const float* st = xs.KS + ((i - 1) & 1) * 2 * C;
+      for (int x = tid - nwc * 32; x < 2 * C; x += blockDim.x - nwc * 32)
+        kv[(size_t)(x < C ? r - SG : r - 2 * SG) * 2 * C + x] = st[x];
+      if (tid == nwc * 32) kf[r - SG] = F0 + (double)Fph;  // Phi_{i-1}
+    }
     if (comb) {
       // ---------------------------------------------------------- combine
       float acc, mx;
@@ -368,12 +379,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float pn = fmaf(acc * sn, xs.A1[po], R * sn);
       if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
       if (tid == 0) xs.nsl[i & 1] = n;
-      if (kv) {
-        if (leader) {
-          kv[(size_t)r * 2 * C + c] = pn;                       // frame Phi_i
-          kv[(size_t)(r - SG) * 2 * C + C + c] = acc;           // frame Phi_{i-1}
-        }
-        if (tid == 0) kf[r] = F0 + (double)(Fp + n);
+      if (kv && leader) {
+        xs.KS[(i & 1) * 2 * C + c] = pn;        // row r, frame Phi_i
+        xs.KS[(i & 1) * 2 * C + C + c] = acc;   // row r - SG, frame Phi_{i-1}
       }
       if (i >= 2 && leader) {
         // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
@@ -427,6 +435,13 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     }
     __syncthreads();
   }
+  if (kv && !comb) {  // the last step's kept values
+    const int r = UP ? L : 0;
+    const float* st = xs.KS + (L & 1) * 2 * C;
+    for (int x = tid - nwc * 32; x < 2 * C; x += blockDim.x - nwc * 32)
+      kv[(size_t)(x < C ? r : r - SG) * 2 * C + x] = st[x];
+    if (tid == nwc * 32) kf[r] = F0 + (double)(Fph + xs.nsl[L & 1]);
+  }
 
   // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
   if (warp == 0) {
@@ -449,7 +464,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
 
 size_t chain_exp_smem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 7ull * d.C) * 4;
+         (2ull * d.xPC + 11ull * d.C) * 4;
 }
 
 }  // namespace semicrf

@@ -83,28 +83,40 @@ __global__ void __launch_bounds__(256)
 }
 
 // grad_trans (entries 0..C*C-1) and grad_dur (entries C*C..C*C+K*C-1):
-// float64 sums of the per-segment partials in (sequence, segment) order.
-__global__ void __launch_bounds__(256)
+// float64 sums of the per-segment partials.  A block takes RP_E consecutive
+// entries; its RP_S thread rows split the (sequence, segment) list, strided,
+// and the rows' sums are added in row order: a fixed order, so the result
+// does not depend on scheduling.
+__global__ void __launch_bounds__(RP_E * RP_S)
     reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                            float* __restrict__ grad_trans, float* __restrict__ grad_dur) {
+  __shared__ double part[RP_S][RP_E];
   const int C = d.C, K = d.K;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  const int nt = C * C;
-  if (e >= nt + K * C) return;
+  const int ex = threadIdx.x % RP_E, sy = threadIdx.x / RP_E;
+  const int e = blockIdx.x * RP_E + ex;
+  const int nt = C * C, ne = nt + K * C;
   double acc = 0.0;
-  for (int b = 0; b < d.B; ++b) {
-    const int L = lengths[b];
-    if (L <= 0 || L > d.T) continue;
-    const int nseg = (L + d.delta - 1) / d.delta;
-    for (int j = 0; j < nseg; ++j) {
-      const size_t seg = (size_t)b * d.nck + j;
-      acc += (e < nt) ? ws.pgt[seg * nt + e] : ws.pgd[seg * K * C + (e - nt)];
+  if (e < ne) {
+    const double* src = (e < nt) ? ws.pgt + e : ws.pgd + (e - nt);
+    const size_t stride = (e < nt) ? (size_t)nt : (size_t)K * C;
+    const int nrow = d.B * d.nck;
+    for (int r = sy; r < nrow; r += RP_S) {
+      const int b = r / d.nck, j = r - b * d.nck;
+      const int L = lengths[b];
+      if (L <= 0 || L > d.T || j * d.delta >= L) continue;
+      acc += src[(size_t)r * stride];
     }
   }
-  if (e < nt)
-    grad_trans[e] = (float)acc;
-  else
-    grad_dur[e - nt] = (float)acc;
+  part[sy][ex] = acc;
+  __syncthreads();
+  if (sy == 0 && e < ne) {
+    double t = 0.0;
+    for (int q = 0; q < RP_S; ++q) t += part[q][ex];
+    if (e < nt)
+      grad_trans[e] = (float)t;
+    else
+      grad_dur[e - nt] = (float)t;
+  }
 }
 
 }  // namespace semicrf

@@ -37,6 +37,8 @@ __global__ void finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __re
                                           float* __restrict__ start_marg,
                                           float* __restrict__ end_marg);
 
+// reduce_partials_kernel: entries per block, thread rows per entry.
+constexpr int RP_E = 32, RP_S = 8;
 __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                        float* __restrict__ grad_trans, float* __restrict__ grad_dur);
 
@@ -51,12 +53,15 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
 
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                 const float* __restrict__ trans, const float* __restrict__ dur);
-__global__ void posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                                 const float* __restrict__ trans, const float* __restrict__ dur,
-                                 const double* __restrict__ grad_logZ,
-                                 float* __restrict__ grad_em, float* __restrict__ start_marg,
-                                 float* __restrict__ end_marg);
+// The posterior pass (one CTA per checkpoint segment and sequence).
+cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const float* trans, const float* dur, const double* grad_logZ,
+                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st);
 size_t posterior_smem_bytes(const Dims& d);
+// Tile rows for the posterior pass under `budget` bytes of shared memory (0:
+// none fits).
+int posterior_tile_rows(const Dims& d, size_t budget);
+size_t cut_grid_smem_bytes(const Dims& d);
 
 // Sizes, launch geometry and limits for (B, T, C, K); returns a semicrf_status.
 int make_dims(int B, int T, int C, int K, Dims& d);

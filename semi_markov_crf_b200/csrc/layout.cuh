@@ -47,8 +47,9 @@ struct Dims {
   // consecutive entries of different labels fall in distinct banks.
   int xRLP;
   // Posteriors from kept ring values (posterior.cu): cut normaliser every
-  // GS positions, ngrid grid points per sequence.
-  int GS, ngrid;
+  // GS positions, ngrid grid points per sequence; the posterior pass stages
+  // pRT boundaries (plus K rows of halo) of kept values per tile.
+  int GS, ngrid, pRT;
 };
 
 // Device pointers into the caller's workspace.

@@ -21,6 +21,8 @@
 // covering a position) evaluated from the kept values every GS positions --
 // cut_grid_kernel -- and interpolated linearly in between.  At position 0
 // the cut is the backward ring's log Z, at L - 1 the forward ring's.
+#include <algorithm>
+
 #include "ring.cuh"
 
 namespace semicrf {
@@ -59,12 +61,18 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 
 // One CTA per (grid position, sequence): log2 of the cut at position u,
 //   Z(u) = sum over segments [s, t) with s <= u < t, t - s <= K, and labels c of
-//          2^(gamma[s, c] - S[s, c] + dur2[t-s-1, c] + S[t, c] + beta[t, c]),
-// from the kept values; every large quantity (frames, prefix sums) enters as
-// a difference from the reference R = Pf_u + Pb_{u+1} before float32 sees it.
+//          2^(gamma[s, c] - S[s, c] + dur2[t-s-1, c] + S[t, c] + beta[t, c]).
+// The start side (s = u - ia) and the end side (t = u + 1 + jb) are staged
+// once per label as logs relative to R = Pf_u + Pb_{u+1} and S[u, c]:
+//   la[ia, c] = log2 af[s] + (Pf_s - Pf_u) - (S[s, c] - S[u, c])
+//   lb[jb, c] = log2 ab[t] + (Pb_t - Pb_{u+1}) + (S[t, c] - S[u, c])
+// (every large quantity enters as a difference before float32 sees it), and
+// the segment term is la + lb + (2M + dur2[ia + jb, c]), ia + jb < K.  A warp
+// per label sums them (its max first, so the sum cannot overflow).
 __global__ void __launch_bounds__(256)
     cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                     const float* __restrict__ trans, const float* __restrict__ dur) {
+  extern __shared__ float csh[];  // la [K][C], lb [K][C], dd [K][C]
   __shared__ int aux[2];
   __shared__ float lab_M[128], lab_f[128];  // per label: shift, log2 share
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -93,47 +101,57 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     M = ord2f(aux[0]);
   }
+  float* const la = csh;
+  float* const lb = csh + (size_t)K * C;
+  float* const dd = csh + 2 * (size_t)K * C;
   const double Fu = kf_at(ws, d, b, 0, u), Gu = kf_at(ws, d, b, 1, u + 1);
   const int32_t* si = ws.sint + (size_t)b * d.Tstride * C;
   const float* sf = ws.sfrac + (size_t)b * d.Tstride * C;
+  const float* kf0 = kv_row(ws, d, b, 0, 0);
+  const float* kf1 = kv_row(ws, d, b, 1, 0);
+  for (int i = tid; i < K * C; i += blockDim.x) {
+    const int q = i / C, c = i - q * C;
+    const int su = si[(size_t)u * C + c];
+    const float fu = sf[(size_t)u * C + c];
+    float va = NEG_INF, vb = NEG_INF;
+    const int s = u - q, t = u + 1 + q;
+    if (s >= 0) {
+      const float a = kf0[(size_t)s * 2 * C + C + c];
+      if (a > 0.f)
+        va = (lg2(a) + (float)(kf_at(ws, d, b, 0, s) - Fu)) -
+             ((float)(si[(size_t)s * C + c] - su) + (sf[(size_t)s * C + c] - fu));
+    }
+    if (t <= L) {
+      const float bt = kf1[(size_t)t * 2 * C + C + c];
+      if (bt > 0.f)
+        vb = (lg2(bt) + (float)(kf_at(ws, d, b, 1, t) - Gu)) +
+             ((float)(si[(size_t)t * C + c] - su) + (sf[(size_t)t * C + c] - fu));
+    }
+    la[i] = va;
+    lb[i] = vb;
+    dd[i] = 2.f * M + __ldg(dur + i) * l2e();
+  }
+  __syncthreads();
   const int lane = tid & 31, nw = blockDim.x >> 5;
   for (int c = tid >> 5; c < C; c += nw) {
-    // lanes over the start s = u - ia (ia < K), inner loop over the end t
+    // lanes over the start offset ia, inner loop over the end offset jb
     float zmax = NEG_INF, sum = 0.f;
-    for (int pass = 0; pass < 2; ++pass) {
-      const float Mz = (pass == 0) ? 0.f : ((zmax == NEG_INF) ? 0.f : ceilf(zmax));
-      for (int ia = lane; ia < K; ia += 32) {
-        const int s = u - ia;
-        if (s < 0) break;
-        const float a = kv_row(ws, d, b, 0, s)[C + c];
-        if (!(a > 0.f)) continue;
-        const float la = lg2(a) + (float)(kf_at(ws, d, b, 0, s) - Fu);
-        const int sis = si[(size_t)s * C + c];
-        const float sfs = sf[(size_t)s * C + c];
-        const int tmax = min(s + K, L);
-        for (int t = u + 1; t <= tmax; ++t) {
-          const float bt = kv_row(ws, d, b, 1, t)[C + c];
-          if (!(bt > 0.f)) continue;
-          const float z = ((float)(si[(size_t)t * C + c] - sis) +
-                           (la + (lg2(bt) + (float)(kf_at(ws, d, b, 1, t) - Gu)))) +
-                          ((2.f * M + __ldg(dur + (size_t)(t - s - 1) * C + c) * l2e()) +
-                           (sf[(size_t)t * C + c] - sfs));
-          if (pass == 0) {
-            zmax = fmaxf(zmax, z);
-          } else {
-            sum += ex2(z - Mz);
-          }
-        }
-      }
-      if (pass == 0) {
-        zmax = group_max(zmax, 32);
-      } else {
-        sum = group_sum(sum, 32);
-        if (lane == 0) {
-          lab_M[c] = Mz;
-          lab_f[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;
-        }
-      }
+    for (int ia = lane; ia < K; ia += 32) {
+      const float a = la[ia * C + c];
+      if (a == NEG_INF) continue;
+      for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lb[jb * C + c]) + dd[(ia + jb) * C + c]);
+    }
+    zmax = group_max(zmax, 32);
+    const float Mz = (zmax == NEG_INF) ? 0.f : ceilf(zmax);
+    for (int ia = lane; ia < K; ia += 32) {
+      const float a = la[ia * C + c] - Mz;
+      if (a == NEG_INF) continue;
+      for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lb[jb * C + c]) + dd[(ia + jb) * C + c]);
+    }
+    sum = group_sum(sum, 32);
+    if (lane == 0) {
+      lab_M[c] = Mz;
+      lab_f[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;
     }
   }
   __syncthreads();
@@ -150,6 +168,39 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Shared memory of cut_grid_kernel.
+size_t cut_grid_smem_bytes(const Dims& d) { return 3ull * d.K * d.C * sizeof(float); }
+
+namespace {
+
+// Shared memory carve of posterior_kernel for a tile of RT boundaries.
+struct PTile {
+  double* dif;  // [RT][C]   St - E of each boundary and label
+  float* tf;    // [RT][2C]  forward kept rows: p, acc
+  float* pb;    // [RT][C]   backward p
+  float* ab;    // [R][C]    backward acc, R = RT + K rows (segment ends)
+  int* ii;      // [R][C]    (Pb_r - Pb_lo) + S_int[r, c], exact integers
+  float* sf;    // [R][C]    S_frac[r, c]
+  float* vv;    // [RT][C]   suffix sums v of the tile
+  float* fs;    // [RT]      f_s
+};
+__host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int K, int C) {
+  const size_t R = (size_t)RT + K;
+  return (size_t)C * (24ull * RT + 12ull * R) + 4ull * RT;
+}
+__device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, int C) {
+  PTile t;
+  const size_t R = (size_t)RT + K;
+  t.dif = reinterpret_cast<double*>(raw);
+  t.tf = reinterpret_cast<float*>(t.dif + (size_t)RT * C);
+  t.pb = t.tf + (size_t)RT * 2 * C;
+  t.ab = t.pb + (size_t)RT * C;
+  t.ii = reinterpret_cast<int*>(t.ab + R * C);
+  t.sf = reinterpret_cast<float*>(t.ii + R * C);
+  t.vv = t.sf + R * C;
+  t.fs = t.vv + (size_t)RT * C;
+  return t;
+}
 
 // One CTA per (checkpoint segment j, sequence b): every posterior whose start
 // boundary lies in [t0, t1), written in the same per-segment layout as
@@ -157,22 +208,30 @@ __global__ void __launch_bounds__(256)
 // count partials), so finalize and the partial reduction are shared; here
 // the per-segment total is the plain sum over the segment (finalize takes the
 // running sum over segments), because the normaliser is continuous.
-__global__ void __launch_bounds__(512)
+//
+// The segment is cut into tiles of d.pRT boundaries, taken downwards (the
+// suffix sums run that way).  A tile stages its kept rows, and the K rows
+// after it that its segments end on, in shared memory with coalesced loads;
+// then every (boundary, label), (duration, label) and (label, label) item is
+// computed from shared memory.  Each thread keeps the duration and transition
+// sums of its first NID / NIT items in registers across tiles; items beyond
+// (large K C or C C) add their per-tile sums to the float64 partials.
+template <int NID, int NIT>
+__global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                      const float* __restrict__ trans, const float* __restrict__ dur,
                      const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
                      float* __restrict__ start_marg, float* __restrict__ end_marg) {
-  extern __shared__ float fsh[];  // [delta + 1] per-boundary factor f_s
+  extern __shared__ __align__(16) unsigned char psh[];
   __shared__ int aux[1];
-  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int C = d.C, K = d.K;
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
+  const int C = d.C, K = d.K, RT = d.pRT;
   const int L = lengths[b];
   if (L <= 0 || L > d.T) return;
   if (!posterior_from_kept(ws, d, b)) return;  // segment_kernel runs it
   const int t0 = j * d.delta;
   if (t0 >= L) return;
   const int t1 = min(t0 + d.delta, L);
-  const bool last = (t1 == L);
   const size_t seg = (size_t)b * d.nck + j;
   const float gb = (float)(grad_logZ ? grad_logZ[b] : 1.0);
   if (tid == 0) aux[0] = f2ord(NEG_INF);
@@ -180,79 +239,165 @@ __global__ void __launch_bounds__(512)
   float M;
   {
     float m = NEG_INF;
-    for (int i = tid; i < C * C; i += blockDim.x) m = fmaxf(m, __ldg(trans + i) * l2e());
+    for (int i = tid; i < C * C; i += nthr) m = fmaxf(m, __ldg(trans + i) * l2e());
     warp_max_to_shared(&aux[0], f2ord(m));
     __syncthreads();
     M = ord2f(aux[0]);
   }
+  const PTile tl = ptile_carve(psh, RT, K, C);
   const float* pfr = kv_row(ws, d, b, 0, 0);  // row t: pfr + t*2C (p), + C (acc)
   const float* pbr = kv_row(ws, d, b, 1, 0);
   const double* kff = ws.kf + ((size_t)b * 2 + 0) * (d.T + 1);
   const double* kfb = ws.kf + ((size_t)b * 2 + 1) * (d.T + 1);
   const double* nc = ws.ncut + (size_t)b * d.ngrid;
   const int32_t* si = ws.sint + (size_t)b * d.Tstride * C;
-  const float* sf = ws.sfrac + (size_t)b * d.Tstride * C;
-  // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s)), s in [t0, t1] (t1 = L: the end
-  // marginal at L, normalised at position L - 1)
-  const int n = t1 - t0;
-  for (int s = t0 + tid; s <= t1; s += blockDim.x)
-    fsh[s - t0] = ex2((float)(((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1))));
-  __syncthreads();
+  const float* sfp = ws.sfrac + (size_t)b * d.Tstride * C;
+  const int nd = K * C, ntr = C * C;
+  float accd[NID], acct[NIT];
+#pragma unroll
+  for (int m = 0; m < NID; ++m) accd[m] = 0.f;
+#pragma unroll
+  for (int m = 0; m < NIT; ++m) acct[m] = 0.f;
+  double lacc = 0.0, lvs = 0.0;  // thread c < C: running suffix sum, sum of v
 
-  // start / end marginals, suffix sums v and the segment's totals (one
-  // thread per label, walking the segment downwards)
-  for (int c = tid; c < C; c += blockDim.x) {
-    double acc = 0.0, vsum = 0.0;
-    for (int s = t1 - 1; s >= t0; --s) {
-      const float f = fsh[s - t0];
-      const float St = pfr[(size_t)s * 2 * C + C + c] * pbr[(size_t)s * 2 * C + c] * f;
-      const float E = pbr[(size_t)s * 2 * C + C + c] * pfr[(size_t)s * 2 * C + c] * f;
-      const size_t ob = ((size_t)b * (d.T + 1) + s) * C + c;
+  for (int s_hi = t1; s_hi > t0; s_hi -= RT) {
+    const int s_lo = max(t0, s_hi - RT);
+    const int nr = s_hi - s_lo;
+    const int nh = min(s_hi - 1 + K, L) - s_lo + 1;  // rows a segment of the tile ends on
+    const bool first = (s_hi == t1);
+    // ------------------------------------------------------------ stage
+    const double kb0 = kfb[s_lo];
+    for (int i = tid; i < nr * 2 * C; i += nthr) tl.tf[i] = pfr[(size_t)s_lo * 2 * C + i];
+    for (int i = tid; i < nh * C; i += nthr) {
+      const int r = i / C, c = i - r * C;
+      const size_t row = (size_t)(s_lo + r);
+      tl.ab[i] = pbr[row * 2 * C + C + c];
+      tl.ii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
+      tl.sf[i] = sfp[row * C + c];
+      if (r < nr) tl.pb[i] = pbr[row * 2 * C + c];
+    }
+    // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s))
+    for (int s = s_lo + tid; s < s_hi; s += nthr)
+      tl.fs[s - s_lo] = ex2((float)(((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1))));
+    __syncthreads();
+    // ------------------------------------------------------------ start / end marginals
+    for (int i = tid; i < nr * C; i += nthr) {
+      const int r = i / C, c = i - r * C;
+      const float f = tl.fs[r];
+      const float St = tl.tf[r * 2 * C + C + c] * tl.pb[i] * f;
+      const float E = tl.ab[i] * tl.tf[r * 2 * C + c] * f;
+      const size_t ob = ((size_t)b * (d.T + 1) + s_lo + r) * C + c;
       if (start_marg) start_marg[ob] = St;
       if (end_marg) end_marg[ob] = E;
-      grad_em[((size_t)b * d.T + s) * C + c] = (float)acc;  // v[s]: after s
-      vsum += (double)(float)acc;
-      acc += (double)St - (double)E;
+      tl.dif[i] = (double)St - (double)E;
     }
-    ws.segT[seg * C + c] = acc;
-    ws.segV[seg * C + c] = vsum;
-    if (last) {
+    // ------------------------------------------------------------ duration counts
+    // item (k, c): sum over the tile's s of P([s, s+k), c), s + k <= L
+    auto dur_item = [&](int idx) {
+      const int k = idx / C + 1, c = idx - (k - 1) * C;
+      const float dk = M + __ldg(dur + idx) * l2e();
+      const int r_end = min(s_hi, L - k + 1) - s_lo;
+      float a_ = 0.f;
+      for (int r = 0; r < r_end; ++r) {
+        const int o = r * C + c, ok = (r + k) * C + c;
+        const float z = (float)(tl.ii[ok] - tl.ii[o]) + (dk + (tl.sf[ok] - tl.sf[o]));
+        a_ = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a_);
+      }
+      return a_;
+    };
+    // item (c', c): sum over the tile's s of P(c' -> c at s) / w[c', c]
+    auto tr_item = [&](int idx) {
+      const int c1 = idx / C, c = idx - c1 * C;
+      float a_ = 0.f;
+      for (int r = 0; r < nr; ++r) a_ = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a_);
+      return a_;
+    };
+#pragma unroll
+    for (int m = 0; m < NID; ++m)
+      if (tid + m * nthr < nd) accd[m] += dur_item(tid + m * nthr);
+    for (int idx = tid + NID * nthr; idx < nd; idx += nthr) {
+      double* pd = ws.pgd + seg * nd + idx;
+      const double v = (double)(gb * dur_item(idx));
+      *pd = first ? v : *pd + v;
+    }
+#pragma unroll
+    for (int m = 0; m < NIT; ++m)
+      if (tid + m * nthr < ntr) acct[m] += tr_item(tid + m * nthr);
+    for (int idx = tid + NIT * nthr; idx < ntr; idx += nthr) {
+      double* pt = ws.pgt + seg * ntr + idx;
+      const double v = (double)(gb * tr_item(idx) * ex2(__ldg(trans + idx) * l2e() - M));
+      *pt = first ? v : *pt + v;
+    }
+    __syncthreads();
+    // ------------------------------------------------------------ suffix sums
+    // v[s] = sum of (St - E) over the segment's boundaries after s
+    if (tid < C) {
+      for (int r = nr - 1; r >= 0; --r) {
+        tl.vv[r * C + tid] = (float)lacc;
+        lvs += (double)(float)lacc;
+        lacc += tl.dif[r * C + tid];
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < nr * C; i += nthr) grad_em[((size_t)b * d.T + s_lo) * C + i] = tl.vv[i];
+  }
+  // register items: the segment's partials
+#pragma unroll
+  for (int m = 0; m < NID; ++m)
+    if (tid + m * nthr < nd) ws.pgd[seg * nd + tid + m * nthr] = (double)(gb * accd[m]);
+#pragma unroll
+  for (int m = 0; m < NIT; ++m) {
+    const int idx = tid + m * nthr;
+    if (idx < ntr) ws.pgt[seg * ntr + idx] = (double)(gb * acct[m] * ex2(__ldg(trans + idx) * l2e() - M));
+  }
+  if (tid < C) {
+    ws.segT[seg * C + tid] = lacc;
+    ws.segV[seg * C + tid] = lvs;
+  }
+  if (t1 == L) {
+    // boundary L: its end marginal (normalised at position L - 1), no start
+    const float fL = ex2((float)(((kff[L] + kfb[L]) + (double)M) - local_logz(d, nc, L, L - 1)));
+    for (int c = tid; c < C; c += nthr) {
       const size_t ob = ((size_t)b * (d.T + 1) + L) * C + c;
-      if (end_marg)
-        end_marg[ob] = pfr[(size_t)L * 2 * C + c] * pbr[(size_t)L * 2 * C + C + c] * fsh[n];
+      if (end_marg) end_marg[ob] = pfr[(size_t)L * 2 * C + c] * pbr[(size_t)L * 2 * C + C + c] * fL;
       if (start_marg) start_marg[ob] = 0.f;
     }
   }
-
-  // duration counts: thread (k, c) sums P([s, s+k), c) over the segment's s
-  for (int idx = tid; idx < K * C; idx += blockDim.x) {
-    const int k = idx / C + 1, c = idx % C;
-    const float dk = M + __ldg(dur + (size_t)(k - 1) * C + c) * l2e();
-    float accd = 0.f;
-    const int s_end = min(t1, L - k + 1);  // s + k <= L
-    for (int s = t0; s < s_end; ++s) {
-      const float a = pfr[(size_t)s * 2 * C + C + c];
-      const float bt = pbr[(size_t)(s + k) * 2 * C + C + c];
-      const float z = (float)(kfb[s + k] - kfb[s]) + (float)(si[(size_t)(s + k) * C + c] - si[(size_t)s * C + c]) +
-                      (dk + (sf[(size_t)(s + k) * C + c] - sf[(size_t)s * C + c]));
-      accd = fmaf(a * bt, fsh[s - t0] * ex2(z), accd);
-    }
-    ws.pgd[(seg * K + (k - 1)) * C + c] = (double)(gb * accd);
-  }
-
-  // transition counts: thread (c', c) sums P(c' -> c at s) over the
-  // segment's boundaries s >= 1 (pf[0] = 0 takes care of s = 0)
-  for (int idx = tid; idx < C * C; idx += blockDim.x) {
-    const int c1 = idx / C, c = idx % C;
-    float acct = 0.f;
-    for (int s = t0; s < t1; ++s)
-      acct = fmaf(pfr[(size_t)s * 2 * C + c1] * fsh[s - t0], pbr[(size_t)s * 2 * C + c], acct);
-    const float w = ex2(__ldg(trans + (size_t)c1 * C + c) * l2e() - M);
-    ws.pgt[(seg * C + c1) * C + c] = (double)(gb * acct * w);
-  }
 }
 
-// Shared memory of posterior_kernel.
-size_t posterior_smem_bytes(const Dims& d) { return ((size_t)d.delta + 1) * sizeof(float); }
+}  // namespace
+
+// Tile rows of the posterior pass: the largest power of two up to 64 (and
+// not past the segment) whose tile fits `budget` bytes, preferring tiles
+// that leave room for two CTAs per SM; 0 if even 8 rows do not fit.
+int posterior_tile_rows(const Dims& d, size_t budget) {
+  int cap = 64;
+  while (cap > 8 && cap / 2 >= d.delta) cap /= 2;
+  for (const size_t lim : {std::min<size_t>(budget, 100u * 1024u), budget})
+    for (int rt = cap; rt >= 8; rt /= 2)
+      if (ptile_bytes(rt, d.K, d.C) <= lim) return rt;
+  return 0;
+}
+
+size_t posterior_smem_bytes(const Dims& d) { return ptile_bytes(d.pRT, d.K, d.C); }
+
+cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const float* trans, const float* dur, const double* grad_logZ,
+                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st) {
+  const size_t sm = posterior_smem_bytes(d);
+  const bool small = (size_t)d.K * d.C <= 4u * 512u && (size_t)d.C * d.C <= 4u * 512u;
+  const void* fn = small ? (const void*)posterior_kernel<4, 4> : (const void*)posterior_kernel<16, 32>;
+  if (sm > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+  }
+  if (small)
+    posterior_kernel<4, 4><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
+                                                              grad_em, start_marg, end_marg);
+  else
+    posterior_kernel<16, 32><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
+                                                                grad_em, start_marg, end_marg);
+  return cudaGetLastError();
+}
 
 }  // namespace semicrf

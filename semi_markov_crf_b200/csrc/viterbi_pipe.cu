@@ -9,30 +9,31 @@
 // steps before.
 //
 // Roles (one CTA per sequence).  Combine warps (G lanes per label, CAT
-// source labels per lane) run the critical path of step t: read V[t-1, :],
-// take max_{c'} V + trans2 for their label, combine it with the step's
-// precomputed candidates, store V[t] and arrive at the barrier.  The argmax
-// label and the ring write of G[t-1] follow the store, off the path.  Helper
-// warps (H lanes per label, KBH durations per lane, strided over the window
-// so that a label's lanes read consecutive ring entries) compute during step
-// t everything step t+1 needs besides G[t]: the best k >= 3 term and its k,
-// and the additive constants of the k = 1 and k = 2 terms.  One barrier per
-// step.
+// source labels per lane) run only the critical path of step t: read
+// V[t-1, :], take max_{c'} V + trans2 for their label, compare it with the
+// step's precomputed candidates, store V[t] and the chosen duration, write
+// G[t-1] into the label's ring.  Helper warps (H lanes per label, KBH
+// durations per lane, strided over the window so that a label's lanes read
+// consecutive ring entries) compute during step t everything else: the best
+// k >= 3 term of step t+1 and its k, the additive constants of its k = 1 and
+// k = 2 terms, and -- from the same V[t-1, :] -- the argmax label of G[t-1],
+// the max of V[t-1] for the frame, and the backpointer word of boundary t-1.
+// One barrier per step.
 //
-// Frames: V[t, :] is stored relative to Phi_t = Phi_{t-1} + n_t, where n_t =
-// rint(max_c V[t-1, c]) relative to Phi_{t-1} -- taken from the vector every
-// combine lane has just read, so no reduction sits before the barrier.
+// Frames: V[t, :] is stored relative to Phi_t with Phi_t = rint(max V[t-2])
+// (absolute): n_t = rint(m_{t-2}) - n_{t-1}, m published by the helpers, so
+// no reduction sits on the critical path and the frame follows the maximum
+// two steps late without oscillating.
 //
 // Ties: k = 1 before k = 2 before the helpers' best k (itself the smallest
 // k among equal terms), the smallest c' among equal label terms, and the
-// smallest final label; a re-scan finds each argmax once the maximum is
-// known (equal floating-point sums compare bit-exactly).
+// smallest final label.
 //
 // Backpointers: bp[t, c] holds, for the best segment of label c ending at
 // t, its duration k (bits 0-15) and the best label before it (bits 16-31,
-// the argmax of G[t-k, c]).  The argmax labels of recent boundaries live in
-// a K-slot ring per label in shared memory, so the word is complete when step
-// t writes it and the traceback reads one word per decoded segment.
+// the argmax of G[t-k, c]); the argmax labels of recent boundaries live in a
+// K-slot ring per label in shared memory.  The traceback reads one word per
+// decoded segment.
 #include "ring.cuh"
 
 namespace semicrf {
@@ -50,7 +51,10 @@ struct VSmem {
   int* Ok;     // [2][C]    its duration
   float* A1;   // [2][C]    dur2[0] + S[t] - S[t-1]
   float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
+  int* Kd;     // [2][C]    duration chosen by the combine warps at the step
+  int* Bc;     // [2][C]    argmax label of G[t-1] found by the combine at step t
   float* nsl;  // [2]       frame step published by the combine warps
+  float* mx;   // [2]       max V[t-1] published by the helpers at step t
   int* Sb;     // [C]       label integer bases
   int16_t* lab;  // [C][K]  argmax label of G[b, c] for the last K boundaries b
 };
@@ -63,6 +67,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   x.s.maxslot = reinterpret_cast<int*>(p + 16);
   x.s.aux = reinterpret_cast<int*>(p + 32);
   x.nsl = reinterpret_cast<float*>(p + 48);
+  x.mx = reinterpret_cast<float*>(p + 56);
   p += 64;
   x.s.tint = reinterpret_cast<int32_t*>(p);
   p += 2ull * TS * C * sizeof(int32_t);
@@ -82,6 +87,10 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   f += 2 * C;
   x.A2 = f;
   f += 2 * C;
+  x.Kd = reinterpret_cast<int*>(f);
+  f += 2 * C;
+  x.Bc = reinterpret_cast<int*>(f);
+  f += 2 * C;
   x.Sb = reinterpret_cast<int*>(f);
   f += C;
   x.lab = reinterpret_cast<int16_t*>(f);
@@ -96,7 +105,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 9ull * d.C) * 4 + (size_t)d.C * d.K * 2 + 16;
+         (2ull * d.xPC + 13ull * d.C) * 4 + (size_t)d.C * d.K * 2 + 16;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -141,6 +150,7 @@ __global__ void __launch_bounds__(LB, 1)
 
   // ---------------------------------------------------------------- roles
   constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
+  constexpr int CA = (G * CAT + H - 1) / H;  // labels per lane for the frame max
   constexpr int NR = CAT > KBH ? CAT : KBH;
   const int warp = tid >> 5, lane = tid & 31;
   const int nwc = (C + LPWC - 1) / LPWC;
@@ -183,9 +193,11 @@ __global__ void __launch_bounds__(LB, 1)
     vs.Ok[i] = 3;
     vs.A1[i] = NEG_INF;
     vs.A2[i] = NEG_INF;
+    vs.Kd[i] = 1;
   }
   if (tid == 0) {
     vs.nsl[0] = vs.nsl[1] = 0.f;
+    vs.mx[0] = vs.mx[1] = NEG_INF;
     mbar_init(&sm.mbar[0], 1);
     mbar_init(&sm.mbar[1], 1);
     fence_mbar_init();
@@ -222,7 +234,9 @@ __global__ void __launch_bounds__(LB, 1)
     hrow_f = sm.tfrac + 2 * C;
   }
   int hbase = (((-WL) % K) + K) % K;  // window start b_lo = i - 1 - WL, at i = 1
-  // combine state
+  int aslot = 0;                       // argmax ring slot of boundary i - 2
+  int32_t* const bpw = ws.bp + (size_t)b * (T + 1) * C;
+  // combine state: S at row i - 1, ring slot of boundary i - 1
   float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
   int si_p = 0;
   float sf_p = 0.f;
@@ -230,7 +244,6 @@ __global__ void __launch_bounds__(LB, 1)
   const float* crow_f = sm.tfrac + C;
   int wslot = 0;
   double F0 = 0.0;
-  int32_t* bpw = ws.bp + (size_t)b * (T + 1) * C;
   __syncthreads();
   int Sbc = 0;
   int next_rb = VREBASE + 1;
@@ -265,10 +278,10 @@ __global__ void __launch_bounds__(LB, 1)
       if (i == next_rb) {
         // rebase the integer frames to (F0 + Phi_{i-1}, S_int[i-1])
         const float D = comb ? Fp : Fph;
-        if (comb && act) {
-          const float adj = (float)(si_p - Sbc) - D;
-          for (int x = jl; x < RL; x += G) rl[x].y += adj;
-          if (leader) vs.Sb[c] = si_p;
+        if (!comb && act) {
+          const float adj = (float)(hs_p - Sbc) - D;
+          for (int x = jl; x < RL; x += H) rl[x].y += adj;
+          if (leader) vs.Sb[c] = hs_p;
         }
         __syncthreads();
         F0 += (double)D;
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(LB, 1)
     }
     if (comb) {
       // ---------------------------------------------------------- combine
-      float gv, mx = NEG_INF;
+      float gv;
       float sv[CAT];  // this lane's label terms V[x] + trans2[x][c]
       if (i == 1) {
         gv = 0.f;  // G[0] = 0 in frame 0
@@ -293,7 +306,6 @@ __global__ void __launch_bounds__(LB, 1)
       } else {
         const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
         float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
-        float m0 = NEG_INF, m1 = NEG_INF, m2 = NEG_INF, m3 = NEG_INF;
 #pragma unroll
         for (int q = 0; q < CAT; q += 4) {
           const float4 v = *reinterpret_cast<const float4*>(pv + q);
@@ -305,20 +317,15 @@ __global__ void __launch_bounds__(LB, 1)
           b1 = fmaxf(b1, sv[q + 1]);
           b2 = fmaxf(b2, sv[q + 2]);
           b3 = fmaxf(b3, sv[q + 3]);
-          m0 = fmaxf(m0, v.x);
-          m1 = fmaxf(m1, v.y);
-          m2 = fmaxf(m2, v.z);
-          m3 = fmaxf(m3, v.w);
         }
         gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
-        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) {
-          gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
-          mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
-        }
+        for (int o = G / 2; o > 0; o >>= 1) gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
       }
-      const float n = (mx == NEG_INF) ? 0.f : rintf(mx);
+      // frame: Phi_i = Phi_{i-2} + rint(max V[i-2]), the max published by
+      // the helpers a step ago
+      const float mp = vs.mx[(i - 1) & 1];
+      const float n = ((mp == NEG_INF) ? 0.f : rintf(mp)) - nprev;
       const float a1 = vs.A1[(i & 1) * C + cc];
       const float a2 = vs.A2[(i & 1) * C + cc];
       const float om = vs.Om[(i & 1) * C + cc];
@@ -327,41 +334,33 @@ __global__ void __launch_bounds__(LB, 1)
       const float c2 = (g2 + a2) - nprev;
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
-      int kdec = 1;
       if (leader) {
         vs.V[(i & 1) * d.xPC + c] = v - n;
-        const int k = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : vs.Ok[(i & 1) * C + cc]);
-        kdec = k;
+        vs.Kd[(i & 1) * C + c] = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : vs.Ok[(i & 1) * C + c]);
       }
       if (tid == 0) vs.nsl[i & 1] = n;
       if (i >= 2) {
-        // off the path: the best previous label (smallest on ties) and the
-        // ring entry of G[i-1] (frame Phi_{i-1})
-        // bit q of the mask: term q attains the maximum (four independent
-        // chains, then the lowest set bit)
-        static_assert(CAT <= 64, "argmax mask is 64 bits");
-        unsigned long long mk[4] = {0ull, 0ull, 0ull, 0ull};
+        // off the path: the argmax of G[i-1] (smallest label on ties: four
+        // select chains walked downwards, then the lanes of the label), for
+        // the helpers' bookkeeping next step, and G[i-1]'s ring entry
+        int q0 = 0x7fffffff, q1 = 0x7fffffff, q2 = 0x7fffffff, q3 = 0x7fffffff;
 #pragma unroll
-        for (int q = 0; q < CAT; ++q) mk[q & 3] |= (sv[q] == gv ? 1ull : 0ull) << q;
-        const unsigned long long msk = (mk[0] | mk[1]) | (mk[2] | mk[3]);
-        int bc = msk ? jl * CAT + (__ffsll((long long)msk) - 1) : 0x7fffffff;
+        for (int q = CAT - 1; q >= 0; --q) {
+          const bool hit = sv[q] == gv;
+          if ((q & 3) == 0) q0 = hit ? q : q0;
+          if ((q & 3) == 1) q1 = hit ? q : q1;
+          if ((q & 3) == 2) q2 = hit ? q : q2;
+          if ((q & 3) == 3) q3 = hit ? q : q3;
+        }
+        const int qb = min(min(q0, q1), min(q2, q3));
+        int bc = (qb == 0x7fffffff) ? qb : jl * CAT + qb;
 #pragma unroll
         for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
-        bc = min(bc, C - 1);  // every term -inf: an unreachable state, any label
         if (leader) {
-          // the previous label of the best segment ending at i: this step's
-          // argmax for k = 1, the ring's entry of boundary i - k otherwise
-          vs.lab[(size_t)c * K + wslot] = (int16_t)bc;  // boundary i - 1
-          int ps = wslot - kdec + 1;
-          if (ps < 0) ps += K;
-          const int pred = (kdec == 1) ? bc : vs.lab[(size_t)c * K + ps];
-          bpw[(size_t)i * C + c] = kdec | (pred << 16);
+          vs.Bc[(i & 1) * C + c] = min(bc, C - 1);  // all terms -inf: any label
           const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
-          rl[wslot] = e;
-          for (int x = wslot + K; x < RL; x += K) rl[x] = e;
+          for (int x = wslot; x < RL; x += K) rl[x] = e;
         }
-      } else if (leader) {
-        bpw[(size_t)C + c] = kdec;  // segment [0, 1): nothing before it
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
       g2 = gv;
@@ -371,44 +370,86 @@ __global__ void __launch_bounds__(LB, 1)
       sf_p = crow_f[cc];
       crow_i += C;
       crow_f += C;
-    } else if (i < L) {
+    } else {
       // ---------------------------------------------------------- helpers
-      const int sn = hrow_i[cc];
-      const float fn = hrow_f[cc];
-      const float Qh = (float)(sn - Sbc) - Fph;
-      float best = NEG_INF;
-      float tv[KBH];
-#pragma unroll
-      for (int q = 0; q < KBH; ++q) {
-        const float2 e = rl[hbase + q * H + jl];
-        tv[q] = ((e.y + Qh) + e.x) + w[q];
-        best = fmaxf(best, tv[q]);
+      // bookkeeping first, so that its latency hides under the step: the
+      // argmax of G[i-2] the combine found last step enters the label ring
+      // (the slot of boundary i - 2 - K, no longer needed), then the
+      // backpointer word of boundary i - 1, whose duration k was chosen last
+      // step and whose previous label is the argmax kept for boundary i-1-k
+      if (leader && i >= 2) {
+        const int o1 = ((i - 1) & 1) * C + c;
+        if (i >= 3) vs.lab[(size_t)c * K + aslot] = (int16_t)vs.Bc[o1];
+        const int kd = vs.Kd[o1];
+        int ps = aslot + 1 - kd;
+        if (ps < 0) ps += K;
+        bpw[(size_t)(i - 1) * C + c] = kd | ((int)vs.lab[(size_t)c * K + ps] << 16);
       }
+      if (warp == nwc) {
+        // max V[i-1] for the frame of step i + 1 (every label group of the
+        // warp computes it; lane 0 publishes)
+        const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
+        float m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
-      for (int o = H / 2; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
-      // smallest k among equal terms: k falls as the window index grows
-      int kb = 0x7fffffff;
+        for (int q = 0; q < CA; q += 2) {
+          m0 = fmaxf(m0, pv[q * H]);
+          if (q + 1 < CA) m1 = fmaxf(m1, pv[(q + 1) * H]);
+        }
+        float mv = fmaxf(m0, m1);
 #pragma unroll
-      for (int q = 0; q < KBH; ++q)
-        if (tv[q] == best) kb = 2 + WL - (q * H + jl);
-#pragma unroll
-      for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
-      if (leader) {
-        const int o2 = ((i + 1) & 1) * C + c;
-        vs.Om[o2] = best + fn;
-        vs.Ok[o2] = kb;
-        vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
-        vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
+        for (int o = H / 2; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(FULL_MASK, mv, o));
+        if (lane == 0) vs.mx[i & 1] = mv;
       }
-      hs_p = hs_c;
-      hf_p = hf_c;
-      hs_c = sn;
-      hf_c = fn;
-      hrow_i += C;
-      hrow_f += C;
-      hbase = (hbase + 1 == K) ? 0 : hbase + 1;
+      if (i < L) {
+        // the k >= 3 terms of step i + 1 over the window of boundaries
+        // i - 1 - WL .. i - 2, and the constants of its k = 1, 2 terms
+        const int sn = hrow_i[cc];
+        const float fn = hrow_f[cc];
+        const float Qh = (float)(sn - Sbc) - Fph;
+        float best = NEG_INF;
+        float tv[KBH];
+#pragma unroll
+        for (int q = 0; q < KBH; ++q) {
+          const float2 e = rl[hbase + q * H + jl];
+          tv[q] = ((e.y + Qh) + e.x) + w[q];
+          best = fmaxf(best, tv[q]);
+        }
+#pragma unroll
+        for (int o = H / 2; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
+        // smallest k among equal terms: k falls as the window index grows
+        int kb = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < KBH; ++q)
+          if (tv[q] == best) kb = 2 + WL - (q * H + jl);
+#pragma unroll
+        for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
+        if (leader) {
+          const int o2 = ((i + 1) & 1) * C + c;
+          vs.Om[o2] = best + fn;
+          vs.Ok[o2] = kb;
+          vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
+          vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
+        }
+        hs_p = hs_c;
+        hf_p = hf_c;
+        hs_c = sn;
+        hf_c = fn;
+        hrow_i += C;
+        hrow_f += C;
+        hbase = (hbase + 1 == K) ? 0 : hbase + 1;
+      }
+      if (i >= 2) aslot = (aslot + 1 == K) ? 0 : aslot + 1;
     }
     __syncthreads();
+  }
+  // the last bookkeeping: the argmax of G[L-1], then boundary L's word
+  if (!comb && leader) {
+    const int o1 = (L & 1) * C + c;
+    if (L >= 2) vs.lab[(size_t)c * K + aslot] = (int16_t)vs.Bc[o1];
+    const int kd = vs.Kd[o1];
+    int ps = aslot + 1 - kd;
+    if (ps < 0) ps += K;
+    bpw[(size_t)L * C + c] = kd | ((int)vs.lab[(size_t)c * K + ps] << 16);
   }
 
   // best final label (smallest on ties), then the traceback

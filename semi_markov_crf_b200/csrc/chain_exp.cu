@@ -62,7 +62,6 @@ struct XSmem {
   float* Oh;   // [2][C]   k >= 3 sums for the step of that parity (frame Phi_{t-2})
   float* A1;   // [2][C]   k = 1 factors
   float* A2;   // [2][C]   k = 2 factors
-  float* KS;   // [2][2C]  kept values of the step of that parity: p, acc
   float* nsl;  // [2]      frame step n published by the combine warps
   int* aux;    // [4]      block reductions
   int* Sb;     // [C]      label integer bases of the prefix sums
@@ -94,8 +93,6 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   f += 2 * C;
   x.A2 = f;
   f += 2 * C;
-  x.KS = f;
-  f += 4 * C;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
@@ -250,17 +247,15 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
     xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
-  // kept values for the posterior pass: per boundary (row) the vector p and
-  // the label fan-in acc, both relative to the boundary's frame kf
+  // kept values for the posterior pass: per boundary (row) the vector p,
+  // relative to the boundary's frame kf (the label fan-in part of each row is
+  // filled from p afterwards by kept_acc_kernel)
   const int dir = UP ? 0 : 1;
   float* const kv = ws.kv ? ws.kv + (((size_t)b * 2 + dir) * (d.T + 1)) * 2 * C : nullptr;
   double* const kf = ws.kf ? ws.kf + ((size_t)b * 2 + dir) * (d.T + 1) : nullptr;
   if (kv) {
-    const int rL = UP ? L : 0;  // the walk's last row: no label fan-in there
-    for (int x = tid; x < C; x += blockDim.x) {
+    for (int x = tid; x < C; x += blockDim.x)
       kv[(size_t)r0 * 2 * C + x] = 0.f;  // no forward vector at 0, no btil at L
-      kv[(size_t)rL * 2 * C + C + x] = 0.f;
-    }
     if (tid == 0) kf[r0] = 0.0;
   }
   __syncthreads();
@@ -283,6 +278,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   };
   int next_ev = next_event(0);
 
+  const float acc_start = ex2(-M);
   for (int i = 1; i <= L; ++i) {
     const int r = UP ? i : L - i;
     if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
@@ -339,50 +335,51 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       next_ev = next_event(i);
     }
     if (kv && !comb && i >= 2) {
-      // the helpers write out the kept values the combine staged last step
-      // (rows r - SG: p, r - 2 SG: acc), off the critical path
-      const float* st = xs.KS + ((i - 1) & 1) * 2 * C;
-      for (int x = tid - nwc * 32; x < 2 * C; x += blockDim.x - nwc * 32)
-        kv[(size_t)(x < C ? r - SG : r - 2 * SG) * 2 * C + x] = st[x];
-      if (tid == nwc * 32) kf[r - SG] = F0 + (double)Fph;  // Phi_{i-1}
+      // the helpers write out p_{i-1} (row r - SG, frame Phi_{i-1}) from the
+      // vector the combine reads this step, off the critical path
+      const float* pp = xs.P + ((i - 1) & 1) * d.xPC;
+      for (int x = tid - nwc * 32; x < C; x += blockDim.x - nwc * 32)
+        kv[(size_t)(r - SG) * 2 * C + x] = pp[x];
+      if (tid == nwc * 32) kf[r - SG] = F0 + (double)Fph;
     }
+    // Each role issues its shared-memory reads first and its stores last: a
+    // store the compiler cannot separate from later reads keeps those reads
+    // from being issued early, and every access of the step must complete
+    // before the barrier releases.
     if (comb) {
       // ---------------------------------------------------------- combine
-      float acc, mx;
+      const int po = (i & 1) * C + cc;
+      const float a1v = xs.A1[po], a2v = xs.A2[po], ohv = xs.Oh[po];
+      const int si_n = crow_i[cc];  // the walk's row r: the next step's ring entry
+      const float sf_n = crow_f[cc];
+      const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+#pragma unroll
+      for (int q = 0; q < CAT; q += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(pv + q);
+        a0 = fmaf(v.x, w[q], a0);
+        a1 = fmaf(v.y, w[q + 1], a1);
+        a2 = fmaf(v.z, w[q + 2], a2);
+        a3 = fmaf(v.w, w[q + 3], a3);
+        m0 = fmaxf(m0, v.x);
+        m1 = fmaxf(m1, v.y);
+        m2 = fmaxf(m2, v.z);
+        m3 = fmaxf(m3, v.w);
+      }
+      float acc = gsum<G>((a0 + a1) + (a2 + a3));
+      float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
       if (i == 1) {
-        acc = ex2(-M);  // the start boundary: gamma = 0 in frame 0
+        acc = acc_start;  // the start boundary: gamma = 0 in frame 0
         mx = 0.f;
-      } else {
-        const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
-#pragma unroll
-        for (int q = 0; q < CAT; q += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(pv + q);
-          a0 = fmaf(v.x, w[q], a0);
-          a1 = fmaf(v.y, w[q + 1], a1);
-          a2 = fmaf(v.z, w[q + 2], a2);
-          a3 = fmaf(v.w, w[q + 3], a3);
-          m0 = fmaxf(m0, v.x);
-          m1 = fmaxf(m1, v.y);
-          m2 = fmaxf(m2, v.z);
-          m3 = fmaxf(m3, v.w);
-        }
-        acc = gsum<G>((a0 + a1) + (a2 + a3));
-        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-#pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, o));
       }
       const float n = exponent_of(mx);
       const float sn = pow2_neg(n);
-      const int po = (i & 1) * C + cc;
-      const float R = fmaf(acc2, xs.A2[po], xs.Oh[po]) * snprev;  // frame Phi_{i-1}
-      const float pn = fmaf(acc * sn, xs.A1[po], R * sn);
+      const float R = fmaf(acc2, a2v, ohv) * snprev;  // frame Phi_{i-1}
+      const float pn = fmaf(acc * sn, a1v, R * sn);
       if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
       if (tid == 0) xs.nsl[i & 1] = n;
-      if (kv && leader) {
-        xs.KS[(i & 1) * 2 * C + c] = pn;        // row r, frame Phi_i
-        xs.KS[(i & 1) * 2 * C + C + c] = acc;   // row r - SG, frame Phi_{i-1}
-      }
       if (i >= 2 && leader) {
         // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
         const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
@@ -393,8 +390,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       snprev = sn;
       Fp += n;
       si_pp = si_p;
-      si_p = crow_i[cc];
-      sf_p = crow_f[cc];
+      si_p = si_n;
+      sf_p = sf_n;
       crow_i += SG * C;
       crow_f += SG * C;
     } else if (i < L) {
@@ -435,11 +432,10 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     }
     __syncthreads();
   }
-  if (kv && !comb) {  // the last step's kept values
+  if (kv && !comb) {  // the last step's vector
     const int r = UP ? L : 0;
-    const float* st = xs.KS + (L & 1) * 2 * C;
-    for (int x = tid - nwc * 32; x < 2 * C; x += blockDim.x - nwc * 32)
-      kv[(size_t)(x < C ? r : r - SG) * 2 * C + x] = st[x];
+    const float* pp = xs.P + (L & 1) * d.xPC;
+    for (int x = tid - nwc * 32; x < C; x += blockDim.x - nwc * 32) kv[(size_t)r * 2 * C + x] = pp[x];
     if (tid == nwc * 32) kf[r] = F0 + (double)(Fph + xs.nsl[L & 1]);
   }
 
@@ -464,7 +460,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
 
 size_t chain_exp_smem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 11ull * d.C) * 4;
+         (2ull * d.xPC + 7ull * d.C) * 4;
 }
 
 }  // namespace semicrf

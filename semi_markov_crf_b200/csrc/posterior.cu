@@ -59,6 +59,65 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 
 }  // namespace
 
+// The label fan-in part of the kept rows, from their p part: the rings keep
+// only p (one vector per boundary, written off the critical path), and the
+// fan-in of the same boundary and frame is a fixed linear map of it,
+//   forward  af[t, c] = sum_c' pf[t, c'] 2^(trans2[c', c] - M)   (gamma[t])
+//   backward ab[t, c] = sum_c' pb[t, c'] 2^(trans2[c, c'] - M)   (beta[t])
+// except at the walks' start boundaries (gamma[0] = 0, beta[L] = 0), where it
+// is 2^-M.  One CTA per (block of KA_ROWS rows, direction, sequence).
+constexpr int KA_ROWS = 64;
+__global__ void __launch_bounds__(256)
+    kept_acc_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                    const float* __restrict__ trans) {
+  extern __shared__ float ksh[];  // W [C][C], then the p rows [KA_ROWS][C]
+  __shared__ int aux[1];
+  const int rb = blockIdx.x, dir = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int C = d.C;
+  const int L = lengths[b];
+  if (L <= 0 || L > d.T) return;
+  if (!posterior_from_kept(ws, d, b)) return;
+  const int r0 = rb * KA_ROWS;
+  if (r0 > L) return;
+  const int nr = min(r0 + KA_ROWS, L + 1) - r0;
+  if (tid == 0) aux[0] = f2ord(NEG_INF);
+  __syncthreads();
+  float M;
+  {
+    float m = NEG_INF;
+    for (int i = tid; i < C * C; i += blockDim.x) m = fmaxf(m, __ldg(trans + i) * l2e());
+    warp_max_to_shared(&aux[0], f2ord(m));
+    __syncthreads();
+    M = ord2f(aux[0]);
+  }
+  float* const W = ksh;
+  float* const pt = ksh + (size_t)C * C;
+  for (int i = tid; i < C * C; i += blockDim.x) {
+    const int c1 = i / C, c = i - c1 * C;
+    W[i] = ex2(__ldg(trans + (dir == 0 ? (size_t)c1 * C + c : (size_t)c * C + c1)) * l2e() - M);
+  }
+  float* const kv = ws.kv + (((size_t)b * 2 + dir) * (d.T + 1) + r0) * 2 * C;
+  for (int i = tid; i < nr * C; i += blockDim.x) {
+    const int r = i / C, x = i - r * C;
+    pt[i] = kv[(size_t)r * 2 * C + x];
+  }
+  __syncthreads();
+  const int start = (dir == 0) ? 0 : L;  // the walk's start boundary
+  const float a0 = ex2(-M);
+  for (int i = tid; i < nr * C; i += blockDim.x) {
+    const int r = i / C, c = i - r * C;
+    const float* pr = pt + (size_t)r * C;
+    float a = 0.f;
+    for (int c1 = 0; c1 < C; ++c1) a = fmaf(pr[c1], W[c1 * C + c], a);
+    kv[(size_t)r * 2 * C + C + c] = (r0 + r == start) ? a0 : a;
+  }
+}
+
+size_t kept_acc_smem_bytes(const Dims& d) {
+  return ((size_t)d.C * d.C + (size_t)KA_ROWS * d.C) * sizeof(float);
+}
+int kept_acc_rows() { return KA_ROWS; }
+
 // One CTA per (grid position, sequence): log2 of the cut at position u,
 //   Z(u) = sum over segments [s, t) with s <= u < t, t - s <= K, and labels c of
 //          2^(gamma[s, c] - S[s, c] + dur2[t-s-1, c] + S[t, c] + beta[t, c]).

@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(LB, 1)
     vs.A1[i] = NEG_INF;
     vs.A2[i] = NEG_INF;
     vs.Kd[i] = 1;
+    vs.Bc[i] = 0;
   }
   if (tid == 0) {
     vs.nsl[0] = vs.nsl[1] = 0.f;
@@ -295,40 +296,41 @@ __global__ void __launch_bounds__(LB, 1)
       }
       next_ev = next_event(i);
     }
+    // Each role issues all of its shared-memory reads first and its stores
+    // last: a store the compiler cannot separate from later reads keeps
+    // those reads from being issued early, and every access of the step must
+    // complete before the barrier releases.
     if (comb) {
       // ---------------------------------------------------------- combine
-      float gv;
-      float sv[CAT];  // this lane's label terms V[x] + trans2[x][c]
-      if (i == 1) {
-        gv = 0.f;  // G[0] = 0 in frame 0
-#pragma unroll
-        for (int q = 0; q < CAT; ++q) sv[q] = NEG_INF;
-      } else {
-        const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
-        float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
-#pragma unroll
-        for (int q = 0; q < CAT; q += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(pv + q);
-          sv[q] = v.x + w[q];
-          sv[q + 1] = v.y + w[q + 1];
-          sv[q + 2] = v.z + w[q + 2];
-          sv[q + 3] = v.w + w[q + 3];
-          b0 = fmaxf(b0, sv[q]);
-          b1 = fmaxf(b1, sv[q + 1]);
-          b2 = fmaxf(b2, sv[q + 2]);
-          b3 = fmaxf(b3, sv[q + 3]);
-        }
-        gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
-#pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
-      }
-      // frame: Phi_i = Phi_{i-2} + rint(max V[i-2]), the max published by
-      // the helpers a step ago
       const float mp = vs.mx[(i - 1) & 1];
-      const float n = ((mp == NEG_INF) ? 0.f : rintf(mp)) - nprev;
       const float a1 = vs.A1[(i & 1) * C + cc];
       const float a2 = vs.A2[(i & 1) * C + cc];
       const float om = vs.Om[(i & 1) * C + cc];
+      const int okd = vs.Ok[(i & 1) * C + cc];
+      const int si_n = crow_i[cc];  // row i: the next step's ring entry
+      const float sf_n = crow_f[cc];
+      const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
+      float sv[CAT];  // this lane's label terms V[x] + trans2[x][c]
+      float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
+#pragma unroll
+      for (int q = 0; q < CAT; q += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(pv + q);
+        sv[q] = v.x + w[q];
+        sv[q + 1] = v.y + w[q + 1];
+        sv[q + 2] = v.z + w[q + 2];
+        sv[q + 3] = v.w + w[q + 3];
+        b0 = fmaxf(b0, sv[q]);
+        b1 = fmaxf(b1, sv[q + 1]);
+        b2 = fmaxf(b2, sv[q + 2]);
+        b3 = fmaxf(b3, sv[q + 3]);
+      }
+      float gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
+      if (i == 1) gv = 0.f;  // G[0] = 0 in frame 0 (V[0] is all -inf)
+      // frame: Phi_i = Phi_{i-2} + rint(max V[i-2]), the max published by
+      // the helpers a step ago
+      const float n = ((mp == NEG_INF) ? 0.f : rintf(mp)) - nprev;
       // candidates relative to Phi_{i-1}; ties to the smaller k
       const float c1 = gv + a1;
       const float c2 = (g2 + a2) - nprev;
@@ -336,100 +338,97 @@ __global__ void __launch_bounds__(LB, 1)
       const float v = fmaxf(c1, fmaxf(c2, c3));
       if (leader) {
         vs.V[(i & 1) * d.xPC + c] = v - n;
-        vs.Kd[(i & 1) * C + c] = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : vs.Ok[(i & 1) * C + c]);
+        vs.Kd[(i & 1) * C + c] = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
       }
       if (tid == 0) vs.nsl[i & 1] = n;
-      if (i >= 2) {
-        // off the path: the argmax of G[i-1] (smallest label on ties: four
-        // select chains walked downwards, then the lanes of the label), for
-        // the helpers' bookkeeping next step, and G[i-1]'s ring entry
-        int q0 = 0x7fffffff, q1 = 0x7fffffff, q2 = 0x7fffffff, q3 = 0x7fffffff;
+      // off the path: the argmax of G[i-1] (smallest label on ties: four
+      // select chains walked downwards, then the lanes of the label), for
+      // the helpers' bookkeeping next step, and G[i-1]'s ring entry
+      int q0 = 0x7fffffff, q1 = 0x7fffffff, q2 = 0x7fffffff, q3 = 0x7fffffff;
 #pragma unroll
-        for (int q = CAT - 1; q >= 0; --q) {
-          const bool hit = sv[q] == gv;
-          if ((q & 3) == 0) q0 = hit ? q : q0;
-          if ((q & 3) == 1) q1 = hit ? q : q1;
-          if ((q & 3) == 2) q2 = hit ? q : q2;
-          if ((q & 3) == 3) q3 = hit ? q : q3;
-        }
-        const int qb = min(min(q0, q1), min(q2, q3));
-        int bc = (qb == 0x7fffffff) ? qb : jl * CAT + qb;
+      for (int q = CAT - 1; q >= 0; --q) {
+        const bool hit = sv[q] == gv;
+        if ((q & 3) == 0) q0 = hit ? q : q0;
+        if ((q & 3) == 1) q1 = hit ? q : q1;
+        if ((q & 3) == 2) q2 = hit ? q : q2;
+        if ((q & 3) == 3) q3 = hit ? q : q3;
+      }
+      const int qb = min(min(q0, q1), min(q2, q3));
+      int bc = (qb == 0x7fffffff) ? qb : jl * CAT + qb;
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
-        if (leader) {
-          vs.Bc[(i & 1) * C + c] = min(bc, C - 1);  // all terms -inf: any label
-          const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
-          for (int x = wslot; x < RL; x += K) rl[x] = e;
-        }
+      for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
+      if (leader && i >= 2) {
+        vs.Bc[(i & 1) * C + c] = min(bc, C - 1);  // all terms -inf: any label
+        const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
+        for (int x = wslot; x < RL; x += K) rl[x] = e;
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
       g2 = gv;
       nprev = n;
       Fp += n;
-      si_p = crow_i[cc];
-      sf_p = crow_f[cc];
+      si_p = si_n;
+      sf_p = sf_n;
       crow_i += C;
       crow_f += C;
     } else {
       // ---------------------------------------------------------- helpers
-      // bookkeeping first, so that its latency hides under the step: the
-      // argmax of G[i-2] the combine found last step enters the label ring
-      // (the slot of boundary i - 2 - K, no longer needed), then the
-      // backpointer word of boundary i - 1, whose duration k was chosen last
-      // step and whose previous label is the argmax kept for boundary i-1-k
-      if (leader && i >= 2) {
-        const int o1 = ((i - 1) & 1) * C + c;
-        if (i >= 3) vs.lab[(size_t)c * K + aslot] = (int16_t)vs.Bc[o1];
-        const int kd = vs.Kd[o1];
-        int ps = aslot + 1 - kd;
-        if (ps < 0) ps += K;
-        bpw[(size_t)(i - 1) * C + c] = kd | ((int)vs.lab[(size_t)c * K + ps] << 16);
+      // reads: the bookkeeping of boundary i - 1 (its duration, chosen last
+      // step; the argmax of G[i-2] the combine found last step; the argmax
+      // kept for boundary i - 1 - k, which is G[i-2]'s when k = 1), row
+      // V[i-1] for the frame max, the window of the k >= 3 terms of step
+      // i + 1 (boundaries i - 1 - WL .. i - 2) and its prefix-sum row
+      const int o1 = ((i - 1) & 1) * C + cc;
+      const int kd = vs.Kd[o1];
+      const int bcv = vs.Bc[o1];
+      int ps = aslot + 1 - kd;
+      if (ps < 0) ps += K;
+      const int labv = vs.lab[(size_t)cc * K + ps];
+      const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
+      float m0 = NEG_INF, m1 = NEG_INF;
+#pragma unroll
+      for (int q = 0; q < CA; q += 2) {
+        m0 = fmaxf(m0, pv[q * H]);
+        if (q + 1 < CA) m1 = fmaxf(m1, pv[(q + 1) * H]);
       }
-      if (warp == nwc) {
-        // max V[i-1] for the frame of step i + 1 (every label group of the
-        // warp computes it; lane 0 publishes)
-        const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
-        float m0 = NEG_INF, m1 = NEG_INF;
+      const int sn = (i < L) ? hrow_i[cc] : 0;
+      const float fn = (i < L) ? hrow_f[cc] : 0.f;
+      const float Qh = (float)(sn - Sbc) - Fph;
+      float best = NEG_INF;
+      float tv[KBH];
 #pragma unroll
-        for (int q = 0; q < CA; q += 2) {
-          m0 = fmaxf(m0, pv[q * H]);
-          if (q + 1 < CA) m1 = fmaxf(m1, pv[(q + 1) * H]);
-        }
-        float mv = fmaxf(m0, m1);
+      for (int q = 0; q < KBH; ++q) {
+        const float2 e = rl[hbase + q * H + jl];
+        tv[q] = ((e.y + Qh) + e.x) + w[q];
+        best = fmaxf(best, tv[q]);
+      }
+      float mv = fmaxf(m0, m1);
 #pragma unroll
-        for (int o = H / 2; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(FULL_MASK, mv, o));
-        if (lane == 0) vs.mx[i & 1] = mv;
+      for (int o = H / 2; o > 0; o >>= 1) {
+        best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
+        mv = fmaxf(mv, __shfl_xor_sync(FULL_MASK, mv, o));
+      }
+      // smallest k among equal terms: k falls as the window index grows
+      int kb = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < KBH; ++q)
+        if (tv[q] == best) kb = 2 + WL - (q * H + jl);
+#pragma unroll
+      for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
+      // stores
+      if (leader && i >= 2) {
+        if (i >= 3) vs.lab[(size_t)c * K + aslot] = (int16_t)bcv;
+        const int pred = (kd == 1) ? ((i >= 3) ? bcv : 0) : labv;
+        bpw[(size_t)(i - 1) * C + c] = kd | (pred << 16);
+      }
+      if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;  // every group saw all of V[i-1]
+      if (leader && i < L) {
+        const int o2 = ((i + 1) & 1) * C + c;
+        vs.Om[o2] = best + fn;
+        vs.Ok[o2] = kb;
+        vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
+        vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
       }
       if (i < L) {
-        // the k >= 3 terms of step i + 1 over the window of boundaries
-        // i - 1 - WL .. i - 2, and the constants of its k = 1, 2 terms
-        const int sn = hrow_i[cc];
-        const float fn = hrow_f[cc];
-        const float Qh = (float)(sn - Sbc) - Fph;
-        float best = NEG_INF;
-        float tv[KBH];
-#pragma unroll
-        for (int q = 0; q < KBH; ++q) {
-          const float2 e = rl[hbase + q * H + jl];
-          tv[q] = ((e.y + Qh) + e.x) + w[q];
-          best = fmaxf(best, tv[q]);
-        }
-#pragma unroll
-        for (int o = H / 2; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
-        // smallest k among equal terms: k falls as the window index grows
-        int kb = 0x7fffffff;
-#pragma unroll
-        for (int q = 0; q < KBH; ++q)
-          if (tv[q] == best) kb = 2 + WL - (q * H + jl);
-#pragma unroll
-        for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
-        if (leader) {
-          const int o2 = ((i + 1) & 1) * C + c;
-          vs.Om[o2] = best + fn;
-          vs.Ok[o2] = kb;
-          vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
-          vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
-        }
         hs_p = hs_c;
         hf_p = hf_c;
         hs_c = sn;

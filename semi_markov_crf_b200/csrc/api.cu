@@ -101,7 +101,7 @@ void choose_xshape(Dims& d, size_t budget) {
   // the posterior pass from the kept values must fit too
   d.pRT = posterior_tile_rows(d, budget);
   if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget || d.pRT == 0 ||
-      cut_grid_smem_bytes(d) > budget || kept_acc_smem_bytes(d) > budget)
+      cut_grid_smem_bytes(d) > budget || d.C > 128)
     d.xG = 0;
 }
 
@@ -429,14 +429,11 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     // others: the checkpoint walk.  Each kernel skips the other's sequences.
     cudaError_t e;
     if (d.xG) {
-      const size_t ksm = kept_acc_smem_bytes(d);
-      if ((rc = set_smem((const void*)kept_acc_kernel, ksm))) return rc;
       {
         ProfScope ps("kept_acc_kernel", st);
-        kept_acc_kernel<<<dim3((T + kept_acc_rows()) / kept_acc_rows(), 2, B), 256, ksm, st>>>(
-            d, p, lengths, trans);
+        e = launch_kept_acc(d, p, lengths, trans, st);
       }
-      if ((rc = launched())) return rc;
+      if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
       const size_t csm = cut_grid_smem_bytes(d);
       if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
       {

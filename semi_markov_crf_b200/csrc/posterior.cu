@@ -67,10 +67,13 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 // except at the walks' start boundaries (gamma[0] = 0, beta[L] = 0), where it
 // is 2^-M.  One CTA per (block of KA_ROWS rows, direction, sequence).
 constexpr int KA_ROWS = 64;
+// NW >= C: the weight column a thread keeps in registers (padded with 0) and
+// the padded row length of the staged p rows (16-byte vector reads).
+template <int NW>
 __global__ void __launch_bounds__(256)
     kept_acc_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                     const float* __restrict__ trans) {
-  extern __shared__ float ksh[];  // W [C][C], then the p rows [KA_ROWS][C]
+  __shared__ __align__(16) float pt[KA_ROWS * NW];  // p rows, zero padded
   __shared__ int aux[1];
   const int rb = blockIdx.x, dir = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int C = d.C;
@@ -90,33 +93,55 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     M = ord2f(aux[0]);
   }
-  float* const W = ksh;
-  float* const pt = ksh + (size_t)C * C;
-  for (int i = tid; i < C * C; i += blockDim.x) {
-    const int c1 = i / C, c = i - c1 * C;
-    W[i] = ex2(__ldg(trans + (dir == 0 ? (size_t)c1 * C + c : (size_t)c * C + c1)) * l2e() - M);
-  }
   float* const kv = ws.kv + (((size_t)b * 2 + dir) * (d.T + 1) + r0) * 2 * C;
-  for (int i = tid; i < nr * C; i += blockDim.x) {
-    const int r = i / C, x = i - r * C;
-    pt[i] = kv[(size_t)r * 2 * C + x];
+  for (int i = tid; i < nr * NW; i += blockDim.x) {
+    const int r = i / NW, x = i - r * NW;
+    pt[i] = (x < C) ? kv[(size_t)r * 2 * C + x] : 0.f;
   }
+  // thread (column c, row phase g): rows g, g + ng, ...
+  const int ng = blockDim.x / C;
+  const int c = tid % C, g = tid / C;
+  float w[NW];
+#pragma unroll
+  for (int q = 0; q < NW; ++q)
+    w[q] = (q < C && g < ng)
+               ? ex2(__ldg(trans + (dir == 0 ? (size_t)q * C + c : (size_t)c * C + q)) * l2e() - M)
+               : 0.f;
   __syncthreads();
+  if (g >= ng) return;
   const int start = (dir == 0) ? 0 : L;  // the walk's start boundary
   const float a0 = ex2(-M);
-  for (int i = tid; i < nr * C; i += blockDim.x) {
-    const int r = i / C, c = i - r * C;
-    const float* pr = pt + (size_t)r * C;
-    float a = 0.f;
-    for (int c1 = 0; c1 < C; ++c1) a = fmaf(pr[c1], W[c1 * C + c], a);
-    kv[(size_t)r * 2 * C + C + c] = (r0 + r == start) ? a0 : a;
+  for (int r = g; r < nr; r += ng) {
+    const float4* pr = reinterpret_cast<const float4*>(pt + (size_t)r * NW);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int q = 0; q < NW / 4; ++q) {
+      const float4 v = pr[q];
+      s0 = fmaf(v.x, w[4 * q], s0);
+      s1 = fmaf(v.y, w[4 * q + 1], s1);
+      s2 = fmaf(v.z, w[4 * q + 2], s2);
+      s3 = fmaf(v.w, w[4 * q + 3], s3);
+    }
+    kv[(size_t)r * 2 * C + C + c] = (r0 + r == start) ? a0 : (s0 + s1) + (s2 + s3);
   }
 }
 
-size_t kept_acc_smem_bytes(const Dims& d) {
-  return ((size_t)d.C * d.C + (size_t)KA_ROWS * d.C) * sizeof(float);
-}
+#define SEMICRF_KA_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
+
 int kept_acc_rows() { return KA_ROWS; }
+
+cudaError_t launch_kept_acc(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                            const float* trans, cudaStream_t st) {
+  const dim3 grid((d.T + KA_ROWS) / KA_ROWS, 2, d.B);
+#define SEMICRF_KA_LAUNCH(nw)                                                  \
+  if (d.C <= nw) {                                                             \
+    kept_acc_kernel<nw><<<grid, 256, 0, st>>>(d, ws, lengths, trans);          \
+    return cudaGetLastError();                                                 \
+  }
+  SEMICRF_KA_WIDTHS(SEMICRF_KA_LAUNCH)
+#undef SEMICRF_KA_LAUNCH
+  return cudaErrorInvalidConfiguration;
+}
 
 // One CTA per (grid position, sequence): log2 of the cut at position u,
 //   Z(u) = sum over segments [s, t) with s <= u < t, t - s <= K, and labels c of
@@ -168,6 +193,7 @@ __global__ void __launch_bounds__(256)
   const float* sf = ws.sfrac + (size_t)b * d.Tstride * C;
   const float* kf0 = kv_row(ws, d, b, 0, 0);
   const float* kf1 = kv_row(ws, d, b, 1, 0);
+  #pragma unroll 4
   for (int i = tid; i < K * C; i += blockDim.x) {
     const int q = i / C, c = i - q * C;
     const int su = si[(size_t)u * C + c];
@@ -326,7 +352,9 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     const bool first = (s_hi == t1);
     // ------------------------------------------------------------ stage
     const double kb0 = kfb[s_lo];
+    #pragma unroll 4
     for (int i = tid; i < nr * 2 * C; i += nthr) tl.tf[i] = pfr[(size_t)s_lo * 2 * C + i];
+    #pragma unroll 4
     for (int i = tid; i < nh * C; i += nthr) {
       const int r = i / C, c = i - r * C;
       const size_t row = (size_t)(s_lo + r);

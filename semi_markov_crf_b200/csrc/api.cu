@@ -208,6 +208,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_segT = take(B * nck * C * 8);
   const size_t o_segV = take(B * nck * C * 8);
   const size_t o_bp = take(B * (size_t)(d.T + 1) * C * 4);
+  const size_t o_vrow = take(d.xG ? B * (size_t)(d.T + 1) * C * 4 : 0);
   const size_t o_kv = take(B * 2ull * (d.T + 1) * 2 * C * 4);
   const size_t o_kf = take(B * 2ull * (d.T + 1) * 8);
   const size_t o_ncut = take(B * (size_t)d.ngrid * 8);
@@ -231,6 +232,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segT = reinterpret_cast<double*>(c + o_segT);
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
+    p->vrow = reinterpret_cast<float*>(c + o_vrow);
     p->kv = reinterpret_cast<float*>(c + o_kv);
     p->kf = reinterpret_cast<double*>(c + o_kf);
     p->ncut = reinterpret_cast<double*>(c + o_ncut);
@@ -497,8 +499,19 @@ extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const fl
   if (rc) return rc;
   cudaError_t e;
   if (d.xG) {
-    ProfScope ps("viterbi_pipe_kernel", st);
-    e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st);
+    {
+      ProfScope ps("viterbi_pipe_kernel", st);
+      e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st);
+    }
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    {
+      ProfScope ps("viterbi_words_kernel", st);
+      e = launch_viterbi_words(d, p, lengths, trans, st);
+    }
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    ProfScope ps("viterbi_walk_kernel", st);
+    e = launch_viterbi_walk(d, p, lengths, labels, seg_start,
+                            viterbi_walk_smem_bytes(d, (size_t)max_smem_optin() - 256), st);
   } else {
     ProfScope ps("viterbi_kernel", st);
     e = launch_viterbi(d, p, lengths, trans, dur, score, labels, seg_start, st);

@@ -114,6 +114,13 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
 
 size_t chain_exp_smem_bytes(const Dims& d);
 size_t viterbi_pipe_smem_bytes(const Dims& d);
+// After viterbi_pipe: the backpointer words from the kept rows (grid-wide),
+// then the traceback (one CTA per sequence, `sm` bytes of shared memory).
+cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                 const float* trans, cudaStream_t st);
+size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget);
+cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                int32_t* labels, uint8_t* seg_start, size_t sm, cudaStream_t st);
 // Viterbi with the pipelined schedule (shapes of SEMICRF_FOR_EACH_XSHAPE).
 cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 const float* trans, const float* dur, double* score,

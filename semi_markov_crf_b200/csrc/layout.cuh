@@ -69,7 +69,8 @@ struct WsPtrs {
   double* pgd;     // [B][nck][K][C] duration-count partials
   double* segT;    // [B][nck][C] per-segment sum of (start - end) marginals
   double* segV;    // [B][nck][C] per-segment sum of the within-segment suffix sums
-  int32_t* bp;     // [B][T+1][C] Viterbi backpointers
+  int32_t* bp;     // [B][T+1][C] Viterbi backpointers (viterbi_pipe: the chosen duration only)
+  float* vrow;     // [B][T+1][C] viterbi_pipe: V per boundary, relative to its frame
   float* kv;       // [B][2][T+1][2][C] exponential-domain ring values per boundary:
                    //   direction (forward, backward) x (p, acc), relative to the frame
   double* kf;      // [B][2][T+1] that frame (absolute, log2 units)

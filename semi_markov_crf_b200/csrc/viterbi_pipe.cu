@@ -16,9 +16,7 @@
 // durations per lane, strided over the window so that a label's lanes read
 // consecutive ring entries) compute during step t everything else: the best
 // k >= 3 term of step t+1 and its k, the additive constants of its k = 1 and
-// k = 2 terms, and -- from the same V[t-1, :] -- the argmax label of G[t-1],
-// the max of V[t-1] for the frame, and the backpointer word of boundary t-1.
-// One barrier per step.
+// k = 2 terms, and the max of V[t-1] for the frame.  One barrier per step.
 //
 // Frames: V[t, :] is stored relative to Phi_t with Phi_t = rint(max V[t-2])
 // (absolute): n_t = rint(m_{t-2}) - n_{t-1}, m published by the helpers, so
@@ -29,11 +27,15 @@
 // k among equal terms), the smallest c' among equal label terms, and the
 // smallest final label.
 //
-// Backpointers: bp[t, c] holds, for the best segment of label c ending at
-// t, its duration k (bits 0-15) and the best label before it (bits 16-31,
-// the argmax of G[t-k, c]); the argmax labels of recent boundaries live in a
-// K-slot ring per label in shared memory.  The traceback reads one word per
-// decoded segment.
+// Decoding: no argmax label is computed during the recursion.  The helpers
+// write out, one step late, each boundary's row of V (relative to its frame)
+// and of chosen durations.  The traceback needs the best previous label only
+// where a decoded segment starts, and recomputes it there from the kept row:
+// argmax_{c'} V[s, c'] + trans2[c', c] is the same float sum the combine
+// compared (the frame shifts every term alike), so the result, ties
+// included, is the recursion's own.
+#include <algorithm>
+
 #include "ring.cuh"
 
 namespace semicrf {
@@ -52,11 +54,9 @@ struct VSmem {
   float* A1;   // [2][C]    dur2[0] + S[t] - S[t-1]
   float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
   int* Kd;     // [2][C]    duration chosen by the combine warps at the step
-  int* Bc;     // [2][C]    argmax label of G[t-1] found by the combine at step t
   float* nsl;  // [2]       frame step published by the combine warps
   float* mx;   // [2]       max V[t-1] published by the helpers at step t
   int* Sb;     // [C]       label integer bases
-  int16_t* lab;  // [C][K]  argmax label of G[b, c] for the last K boundaries b
 };
 
 __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
@@ -89,11 +89,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   f += 2 * C;
   x.Kd = reinterpret_cast<int*>(f);
   f += 2 * C;
-  x.Bc = reinterpret_cast<int*>(f);
-  f += 2 * C;
   x.Sb = reinterpret_cast<int*>(f);
-  f += C;
-  x.lab = reinterpret_cast<int16_t*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
   x.s.tmp = nullptr;
@@ -105,7 +101,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 13ull * d.C) * 4 + (size_t)d.C * d.K * 2 + 16;
+         (2ull * d.xPC + 11ull * d.C) * 4;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -187,14 +183,12 @@ __global__ void __launch_bounds__(LB, 1)
   // ---------------------------------------------------------------- shared state
   for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) vs.V[i] = NEG_INF;
-  for (int i = tid; i < C * K; i += blockDim.x) vs.lab[i] = 0;
   for (int i = tid; i < 2 * C; i += blockDim.x) {
     vs.Om[i] = NEG_INF;
     vs.Ok[i] = 3;
     vs.A1[i] = NEG_INF;
     vs.A2[i] = NEG_INF;
     vs.Kd[i] = 1;
-    vs.Bc[i] = 0;
   }
   if (tid == 0) {
     vs.nsl[0] = vs.nsl[1] = 0.f;
@@ -235,8 +229,10 @@ __global__ void __launch_bounds__(LB, 1)
     hrow_f = sm.tfrac + 2 * C;
   }
   int hbase = (((-WL) % K) + K) % K;  // window start b_lo = i - 1 - WL, at i = 1
-  int aslot = 0;                       // argmax ring slot of boundary i - 2
-  int32_t* const bpw = ws.bp + (size_t)b * (T + 1) * C;
+  // kept rows of boundaries 1..L: V (frame-relative) and the chosen duration
+  float* const vrw = ws.vrow + (size_t)b * (T + 1) * C;
+  int32_t* const kdw = ws.bp + (size_t)b * (T + 1) * C;
+  const int hx = tid - nwc * 32, nh = blockDim.x - nwc * 32;  // helper thread index, count
   // combine state: S at row i - 1, ring slot of boundary i - 1
   float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
   int si_p = 0;
@@ -310,19 +306,14 @@ __global__ void __launch_bounds__(LB, 1)
       const int si_n = crow_i[cc];  // row i: the next step's ring entry
       const float sf_n = crow_f[cc];
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
-      float sv[CAT];  // this lane's label terms V[x] + trans2[x][c]
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
 #pragma unroll
       for (int q = 0; q < CAT; q += 4) {
         const float4 v = *reinterpret_cast<const float4*>(pv + q);
-        sv[q] = v.x + w[q];
-        sv[q + 1] = v.y + w[q + 1];
-        sv[q + 2] = v.z + w[q + 2];
-        sv[q + 3] = v.w + w[q + 3];
-        b0 = fmaxf(b0, sv[q]);
-        b1 = fmaxf(b1, sv[q + 1]);
-        b2 = fmaxf(b2, sv[q + 2]);
-        b3 = fmaxf(b3, sv[q + 3]);
+        b0 = fmaxf(b0, v.x + w[q]);
+        b1 = fmaxf(b1, v.y + w[q + 1]);
+        b2 = fmaxf(b2, v.z + w[q + 2]);
+        b3 = fmaxf(b3, v.w + w[q + 3]);
       }
       float gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
 #pragma unroll
@@ -341,24 +332,8 @@ __global__ void __launch_bounds__(LB, 1)
         vs.Kd[(i & 1) * C + c] = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
       }
       if (tid == 0) vs.nsl[i & 1] = n;
-      // off the path: the argmax of G[i-1] (smallest label on ties: four
-      // select chains walked downwards, then the lanes of the label), for
-      // the helpers' bookkeeping next step, and G[i-1]'s ring entry
-      int q0 = 0x7fffffff, q1 = 0x7fffffff, q2 = 0x7fffffff, q3 = 0x7fffffff;
-#pragma unroll
-      for (int q = CAT - 1; q >= 0; --q) {
-        const bool hit = sv[q] == gv;
-        if ((q & 3) == 0) q0 = hit ? q : q0;
-        if ((q & 3) == 1) q1 = hit ? q : q1;
-        if ((q & 3) == 2) q2 = hit ? q : q2;
-        if ((q & 3) == 3) q3 = hit ? q : q3;
-      }
-      const int qb = min(min(q0, q1), min(q2, q3));
-      int bc = (qb == 0x7fffffff) ? qb : jl * CAT + qb;
-#pragma unroll
-      for (int o = G / 2; o > 0; o >>= 1) bc = min(bc, __shfl_xor_sync(FULL_MASK, bc, o));
+      // off the path: G[i-1]'s ring entry (frame Phi_{i-1})
       if (leader && i >= 2) {
-        vs.Bc[(i & 1) * C + c] = min(bc, C - 1);  // all terms -inf: any label
         const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
         for (int x = wslot; x < RL; x += K) rl[x] = e;
       }
@@ -372,17 +347,16 @@ __global__ void __launch_bounds__(LB, 1)
       crow_f += C;
     } else {
       // ---------------------------------------------------------- helpers
-      // reads: the bookkeeping of boundary i - 1 (its duration, chosen last
-      // step; the argmax of G[i-2] the combine found last step; the argmax
-      // kept for boundary i - 1 - k, which is G[i-2]'s when k = 1), row
-      // V[i-1] for the frame max, the window of the k >= 3 terms of step
-      // i + 1 (boundaries i - 1 - WL .. i - 2) and its prefix-sum row
-      const int o1 = ((i - 1) & 1) * C + cc;
-      const int kd = vs.Kd[o1];
-      const int bcv = vs.Bc[o1];
-      int ps = aslot + 1 - kd;
-      if (ps < 0) ps += K;
-      const int labv = vs.lab[(size_t)cc * K + ps];
+      // reads: boundary i - 1's kept rows (V[i-1] and its chosen durations,
+      // both written last step; a helper thread holds at most two of the
+      // 2C values, nh >= C), row V[i-1] for the frame max, the window of the
+      // k >= 3 terms of step i + 1 (boundaries i - 1 - WL .. i - 2) and its
+      // prefix-sum row
+      const float* vpr = vs.V + ((i - 1) & 1) * d.xPC;
+      const int* kpr = vs.Kd + ((i - 1) & 1) * C;
+      const int x1 = hx + nh;
+      const float kv0 = (hx < C) ? vpr[hx] : __int_as_float(kpr[min(hx - C, C - 1)]);
+      const float kv1 = (x1 < C) ? vpr[x1] : __int_as_float(kpr[min(max(x1 - C, 0), C - 1)]);
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
       float m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
@@ -414,13 +388,22 @@ __global__ void __launch_bounds__(LB, 1)
         if (tv[q] == best) kb = 2 + WL - (q * H + jl);
 #pragma unroll
       for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
-      // stores
-      if (leader && i >= 2) {
-        if (i >= 3) vs.lab[(size_t)c * K + aslot] = (int16_t)bcv;
-        const int pred = (kd == 1) ? ((i >= 3) ? bcv : 0) : labv;
-        bpw[(size_t)(i - 1) * C + c] = kd | (pred << 16);
+      // stores (every label group saw all of V[i-1]: the first one publishes)
+      if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;
+      if (i >= 2) {
+        if (hx < 2 * C) {
+          if (hx < C)
+            vrw[(size_t)(i - 1) * C + hx] = kv0;
+          else
+            kdw[(size_t)(i - 1) * C + hx - C] = __float_as_int(kv0);
+        }
+        if (x1 < 2 * C) {
+          if (x1 < C)
+            vrw[(size_t)(i - 1) * C + x1] = kv1;
+          else
+            kdw[(size_t)(i - 1) * C + x1 - C] = __float_as_int(kv1);
+        }
       }
-      if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;  // every group saw all of V[i-1]
       if (leader && i < L) {
         const int o2 = ((i + 1) & 1) * C + c;
         vs.Om[o2] = best + fn;
@@ -437,28 +420,130 @@ __global__ void __launch_bounds__(LB, 1)
         hrow_f += C;
         hbase = (hbase + 1 == K) ? 0 : hbase + 1;
       }
-      if (i >= 2) aslot = (aslot + 1 == K) ? 0 : aslot + 1;
     }
     __syncthreads();
   }
-  // the last bookkeeping: the argmax of G[L-1], then boundary L's word
-  if (!comb && leader) {
-    const int o1 = (L & 1) * C + c;
-    if (L >= 2) vs.lab[(size_t)c * K + aslot] = (int16_t)vs.Bc[o1];
-    const int kd = vs.Kd[o1];
-    int ps = aslot + 1 - kd;
-    if (ps < 0) ps += K;
-    bpw[(size_t)L * C + c] = kd | ((int)vs.lab[(size_t)c * K + ps] << 16);
+  // boundary L's kept rows
+  if (!comb) {
+    const float* vp = vs.V + (L & 1) * d.xPC;
+    const int* kp = vs.Kd + (L & 1) * C;
+    for (int x = hx; x < 2 * C; x += nh) {
+      if (x < C)
+        vrw[(size_t)L * C + x] = vp[x];
+      else
+        kdw[(size_t)L * C + x - C] = kp[x - C];
+    }
   }
 
-  // best final label (smallest on ties), then the traceback
-  __shared__ int s_tb[2];  // walk state shared by the block: row, label
+  // the optimum: max over the final labels of V[L] in frame Phi_L
   if (tid < 32) {
     const float* V = vs.V + (L & 1) * d.xPC;
     float best = NEG_INF;
+    for (int x = tid; x < C; x += 32) best = fmaxf(best, V[x]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
+    if (tid == 0) score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
+  }
+}
+
+// Backpointer words, in parallel over (boundary, label): for boundary t in
+// [1, L] and label c with k = kd[t, c] and s = t - k >= 1, the word is
+// k | argmax_{c'} (V[s, c'] + trans2[c', c]) << 16 (smallest c' on ties),
+// written over kd[t, c]; for s = 0 the word is k.  One CTA per block of
+// VW_ROWS boundaries of a sequence: the V rows its segments start at are
+// staged in shared memory (rows of VS = C rounded up to 4 floats, -inf
+// padded), and thread (label c, row phase) keeps trans2[., c] in registers.
+// The argmax runs four independent compare chains (c' mod 4) and merges
+// them by value, then index, so it is the smallest c' among equal maxima,
+// as the recursion's own comparisons would give.
+constexpr int VW_ROWS = 64;
+template <int NW>
+__global__ void __launch_bounds__(256)
+    viterbi_words_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                         const float* __restrict__ trans) {
+  extern __shared__ __align__(16) float vsh[];  // [VW_ROWS + K][VS]
+  const int C = d.C, K = d.K, tid = threadIdx.x, b = blockIdx.y;
+  const int L = lengths[b];
+  if (L < 1 || L > d.T) return;
+  const int t0 = blockIdx.x * VW_ROWS + 1;
+  if (t0 > L) return;
+  const int t1 = min(t0 + VW_ROWS - 1, L);
+  const int VS = (C + 3) & ~3;
+  const int vlo = max(1, t0 - K);  // V rows [vlo, t1 - 1]
+  const float* vrw = ws.vrow + (size_t)b * (d.T + 1) * C;
+  int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
+  const int nv = (t1 - vlo) * VS;
+#pragma unroll 4
+  for (int i = tid; i < nv; i += blockDim.x) {
+    const int r = i / VS, x = i - r * VS;
+    vsh[i] = (x < C) ? vrw[(size_t)(vlo + r) * C + x] : NEG_INF;
+  }
+  const int pc = tid % C, pg = tid / C, png = blockDim.x / C;
+  float w2[NW];
+#pragma unroll
+  for (int q = 0; q < NW; ++q)
+    w2[q] = (q < C && pg < png) ? __ldg(trans + (size_t)q * C + pc) * l2e() : NEG_INF;
+  __syncthreads();
+  if (pg >= png) return;
+  for (int t = t0 + pg; t <= t1; t += png) {
+    const int k = kdw[(size_t)t * C + pc];
+    const int sb = t - k;
+    int word = k;
+    if (k >= 1 && k <= K && sb >= 1) {
+      const float4* vr = reinterpret_cast<const float4*>(vsh + (size_t)(sb - vlo) * VS);
+      float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
+      int q0 = 0, q1 = 1, q2 = 2, q3 = 3;
+#pragma unroll
+      for (int q4 = 0; q4 < NW / 4; ++q4) {
+        if (4 * q4 < VS) {
+          const float4 v = vr[q4];
+          const float e0 = v.x + w2[4 * q4], e1 = v.y + w2[4 * q4 + 1];
+          const float e2 = v.z + w2[4 * q4 + 2], e3 = v.w + w2[4 * q4 + 3];
+          if (e0 > b0) { b0 = e0; q0 = 4 * q4; }
+          if (e1 > b1) { b1 = e1; q1 = 4 * q4 + 1; }
+          if (e2 > b2) { b2 = e2; q2 = 4 * q4 + 2; }
+          if (e3 > b3) { b3 = e3; q3 = 4 * q4 + 3; }
+        }
+      }
+      // a chain that never improved on -inf keeps its first index, so an
+      // all -inf row yields label 0 (the smallest)
+      if (b1 > b0 || (b1 == b0 && q1 < q0)) { b0 = b1; q0 = q1; }
+      if (b3 > b2 || (b3 == b2 && q3 < q2)) { b2 = b3; q2 = q3; }
+      if (b2 > b0 || (b2 == b0 && q2 < q0)) { b0 = b2; q0 = q2; }
+      word = k | (q0 << 16);
+    }
+    kdw[(size_t)t * C + pc] = word;
+  }
+}
+
+// The traceback, one CTA per sequence.  Start: the best final label
+// (argmax of the kept row V[L], smallest on ties).  In stages over the
+// dynamic shared memory: the block stages the word rows [lo, tt0]
+// (coalesced), thread 0 follows the words -- one shared-memory read per
+// decoded segment -- and marks each segment's start position with its
+// label, then warp 0 fills every position of the stage with the label of
+// the last mark at or below it (a running "last mark" scan, 32 positions per
+// shuffle round) and writes labels and start flags out coalesced.  The next
+// stage starts where the walk left the staged rows.  A word with a duration
+// outside [1, t] or a previous label >= C ends the walk with the positions
+// not reached labelled -1.
+__global__ void __launch_bounds__(256)
+    viterbi_walk_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                        int32_t* __restrict__ labels, uint8_t* __restrict__ seg_start, int WR) {
+  extern __shared__ __align__(16) int wsh[];  // words [WR][C], marks [WR + K]
+  __shared__ int s_tb[2];
+  const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x, lane = tid & 31, b = blockIdx.x;
+  const int L = lengths[b];
+  if (L < 1 || L > T) return;
+  const int32_t* kdw = ws.bp + (size_t)b * (T + 1) * C;
+  const float* vrw = ws.vrow + (size_t)b * (T + 1) * C;
+  int* const kbuf = wsh;
+  int* const lbuf = wsh + (size_t)WR * C;
+  if (tid < 32) {
+    float best = NEG_INF;
     int bc = 0x7fffffff;
     for (int x = tid; x < C; x += 32) {
-      const float v = V[x];
+      const float v = vrw[(size_t)L * C + x];
       if (v > best || bc == 0x7fffffff) {
         best = v;
         bc = x;
@@ -466,58 +551,116 @@ __global__ void __launch_bounds__(LB, 1)
     }
     gargmax<32>(best, bc);
     if (tid == 0) {
-      score[b] = (F0 + (double)Fp + (double)best) * LN2_D;
       s_tb[0] = L;
       s_tb[1] = bc;
     }
   }
   __syncthreads();
-  // Traceback.  The whole dynamic shared memory is free now: the block
-  // stages as many backpointer rows as fit (coalesced, every thread), warp 0
-  // walks them -- one word per decoded segment -- and the block stages the
-  // next rows where the walk left off.  A duration outside [1, t] or a
-  // previous label >= C (impossible for backpointers this kernel wrote) ends
-  // the walk with the positions not reached labelled -1.
-  const int32_t* bp = ws.bp + (size_t)b * (T + 1) * C;
-  int32_t* buf = reinterpret_cast<int32_t*>(smem_raw + 64);
-  const int WR = (int)((vsmem_bytes(d) - 64) / ((size_t)C * 4));
   for (;;) {
     const int tt0 = s_tb[0];
     if (tt0 <= 0) break;
-    const int lo = max(0, tt0 - WR + 1);
-    for (int idx = tid; idx < (tt0 - lo + 1) * C; idx += blockDim.x) buf[idx] = bp[(size_t)lo * C + idx];
-    __syncthreads();
-    if (tid < 32) {
-      int tt = tt0, cl = s_tb[1];
-      while (tt >= lo && tt > 0) {
-        const int w = buf[(tt - lo) * C + cl];
-        const int k = w & 0xffff, pred = (w >> 16) & 0xffff;
-        if (k < 1 || k > tt || (tt - k > 0 && pred >= C)) {
-          for (int u = tid; u < tt; u += 32) labels[(size_t)b * T + u] = -1;
-          tt = 0;
-          break;
-        }
-        const int sb = tt - k;
-        for (int u = sb + tid; u < tt; u += 32) {
-          labels[(size_t)b * T + u] = cl;
-          seg_start[(size_t)b * T + u] = (u == sb) ? 1 : 0;
-        }
-        tt = sb;
-        cl = pred;
-      }
-      __syncwarp();
-      if (tid == 0) {
-        s_tb[0] = tt;
-        s_tb[1] = cl;
-      }
+    const int lo = max(1, tt0 - WR + 1);
+    const int pb = lo - K;  // mark of position u at lbuf[u - pb]
+    {
+      const int nk = (tt0 - lo + 1) * C;
+      const int32_t* ksrc = kdw + (size_t)lo * C;
+#pragma unroll 8
+      for (int i = tid; i < nk; i += blockDim.x) kbuf[i] = ksrc[i];
+      for (int i = tid; i < WR + K; i += blockDim.x) lbuf[i] = -1;
     }
     __syncthreads();
+    if (tid == 0) {
+      int tt = tt0, cl = s_tb[1];
+      bool broken = false;
+      while (tt >= lo) {
+        const int w = kbuf[(tt - lo) * C + cl];
+        const int k = w & 0xffff, pred = (w >> 16) & 0xffff;
+        if (k < 1 || k > tt || (tt - k > 0 && pred >= C)) {
+          broken = true;
+          break;
+        }
+        tt -= k;
+        lbuf[tt - pb] = cl;
+        cl = pred;
+      }
+      s_tb[0] = broken ? -tt : tt;  // -tt: stop, positions below tt get -1
+      s_tb[1] = cl;
+    }
+    __syncthreads();
+    const int te = s_tb[0];
+    const int end = te < 0 ? -te : te;
+    if (tid < 32) {
+      int carry = -1;
+      for (int u0 = end; u0 < tt0; u0 += 32) {
+        const int u = u0 + lane;
+        const int m = (u < tt0) ? lbuf[u - pb] : -1;
+        int v = m;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int up = __shfl_up_sync(FULL_MASK, v, o);
+          if (lane >= o && v < 0) v = up;
+        }
+        if (v < 0) v = carry;
+        carry = __shfl_sync(FULL_MASK, v, 31);
+        if (u < tt0) {
+          labels[(size_t)b * T + u] = v;
+          seg_start[(size_t)b * T + u] = (m >= 0) ? 1 : 0;
+        }
+      }
+    }
+    if (te < 0)
+      for (int u = tid; u < end; u += blockDim.x) labels[(size_t)b * T + u] = -1;
+    __syncthreads();  // every thread has read s_tb and the marks before the next stage
+    if (te < 0) break;
   }
 }
 
 }  // namespace
 
 size_t viterbi_pipe_smem_bytes(const Dims& d) { return vsmem_bytes(d); }
+
+#define SEMICRF_VW_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
+
+cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                 const float* trans, cudaStream_t st) {
+  const size_t sm = (size_t)(VW_ROWS + d.K) * ((d.C + 3) & ~3) * sizeof(float);
+  const dim3 grid((d.T + VW_ROWS - 1) / VW_ROWS, d.B);
+  if (d.T == 0) return cudaSuccess;
+#define SEMICRF_VW_LAUNCH(nw)                                                                   \
+  if (d.C <= nw) {                                                                              \
+    if (sm > 48 * 1024) {                                                                       \
+      const cudaError_t e = cudaFuncSetAttribute(viterbi_words_kernel<nw>,                      \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                                 (int)sm);                                      \
+      if (e != cudaSuccess) return e;                                                           \
+    }                                                                                           \
+    viterbi_words_kernel<nw><<<grid, 256, sm, st>>>(d, ws, lengths, trans);                     \
+    return cudaGetLastError();                                                                  \
+  }
+  SEMICRF_VW_WIDTHS(SEMICRF_VW_LAUNCH)
+#undef SEMICRF_VW_LAUNCH
+  return cudaErrorInvalidConfiguration;
+}
+
+// Shared memory of the walk: about 96 KB (fewer stages), at least the K
+// marks and one row.
+size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget) {
+  const size_t want = std::min<size_t>(budget, 96u * 1024u);
+  const size_t need = ((size_t)d.K + 1 + 2 * (size_t)d.C) * sizeof(int);
+  return std::max(want, need);
+}
+
+cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                int32_t* labels, uint8_t* seg_start, size_t sm, cudaStream_t st) {
+  const int WR = (int)((sm / sizeof(int) - (size_t)d.K) / ((size_t)d.C + 1));
+  if (sm > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(viterbi_walk_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+  }
+  viterbi_walk_kernel<<<d.B, 256, sm, st>>>(d, ws, lengths, labels, seg_start, WR);
+  return cudaGetLastError();
+}
 
 }  // namespace semicrf
 

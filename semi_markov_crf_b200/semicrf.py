@@ -23,7 +23,8 @@ __all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi",
 KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "chain_kernel",
            "kept_acc_kernel", "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
-           "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel")
+           "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
+           "viterbi_walk_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2

@@ -33,6 +33,22 @@ int isqrt_ceil(long long v) {
   return (int)r;
 }
 
+int sm_count() {
+  static int cached = -1;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (cached < 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1) {
+      cudaGetLastError();
+      v = 148;  // B200
+    }
+    cached = v;
+  }
+  return cached;
+}
+
 int max_smem_optin() {
   static int cached = -1;
   static std::mutex mu;
@@ -116,14 +132,14 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   d.K = K;
   // Checkpoint spacing: ceil(sqrt(T K)) balances checkpoint memory against
   // recompute, but memory is not what binds here -- the posterior pass runs
-  // one CTA per (segment, sequence) and each CTA walks 2 Delta serial steps.
-  // So Delta is also capped at what gives the batch about SEGMENTS_WANTED
-  // segments (two CTAs per SM), though never below 2K.  Any spacing gives the
+  // one CTA per (segment, sequence).  So Delta is also capped at what gives
+  // the batch at most two segment CTAs per SM in all (one wave), each
+  // sequence an equal share, though never below 2K.  Any spacing gives the
   // same results in exact arithmetic.
-  constexpr long long SEGMENTS_WANTED = 320;
   d.delta = T > 0 ? isqrt_ceil((long long)T * K) : 1;
   if (T > 0) {
-    const long long par = ((long long)B * T + SEGMENTS_WANTED - 1) / SEGMENTS_WANTED;
+    const long long per_seq = std::max<long long>(1, 2LL * sm_count() / std::max(B, 1));
+    const long long par = (T + per_seq - 1) / per_seq;
     d.delta = (int)std::min<long long>(d.delta, std::max<long long>(2LL * K, par));
   }
   if (d.delta < 1) d.delta = 1;
@@ -214,6 +230,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_ncut = take(B * (size_t)d.ngrid * 8);
   const size_t o_emax = take(B * 4);
   const size_t o_mode = take(2 * B * 4);
+  const size_t o_tmax = take(4);
   if (base && p) {
     char* c = static_cast<char*>(base);
     p->status = reinterpret_cast<int*>(c + o_status);
@@ -238,6 +255,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->ncut = reinterpret_cast<double*>(c + o_ncut);
     p->emax = reinterpret_cast<float*>(c + o_emax);
     p->mode = reinterpret_cast<int*>(c + o_mode);
+    p->tmax = reinterpret_cast<float*>(c + o_tmax);
   }
   return off;
 }

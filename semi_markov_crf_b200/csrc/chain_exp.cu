@@ -507,6 +507,7 @@ __global__ void __launch_bounds__(LB, 1)
   for (int i = tid; i < K * C; i += blockDim.x) bad |= !isfinite(__ldg(dur + i));
   bad = __syncthreads_or(bad);  // also orders the aux reset
   const float M = block_max(&xs.aux[0], C * C, [&](int i) { return __ldg(trans + i) * l2e(); });
+  if (ws.tmax && threadIdx.x == 0 && blockIdx.x == 0) *ws.tmax = M;  // for the posterior pass
   const float tmin = -block_max(&xs.aux[1], C * C, [&](int i) { return -__ldg(trans + i) * l2e(); });
   const float dmax = block_max(&xs.aux[2], K * C, [&](int i) { return __ldg(dur + i) * l2e(); });
   const float dmin = -block_max(&xs.aux[3], K * C, [&](int i) { return -__ldg(dur + i) * l2e(); });

@@ -109,32 +109,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// One-dimensional TMA bulk copy shared -> global in the issuing thread's bulk
-// group (no multicast).  dst, src 16-byte aligned; bytes a multiple of 16.
-// The copy does not hold up the CTA's barriers; the issuing thread tracks it
-// with bulk_commit and the bulk_wait_* calls.
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_addr(src)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Until every committed group of this thread has read its shared source.
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Until every committed group of this thread has written its destination.
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-// Orders async-proxy accesses (any state space) with this thread's later
-// generic-proxy accesses.
-__device__ __forceinline__ void fence_proxy_async_all() {
-  asm volatile("fence.proxy.async;" ::: "memory");
-}
-
 // Bounded wait for phase `parity` of `bar`.  Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int spins) {
   const uint32_t a = smem_addr(bar);

@@ -54,7 +54,6 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
 // The label fan-in part of the kept rows (C <= 128).
 cudaError_t launch_kept_acc(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                             const float* trans, cudaStream_t st);
-int kept_acc_rows();
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                 const float* __restrict__ trans, const float* __restrict__ dur);
 // The posterior pass (one CTA per checkpoint segment and sequence).

@@ -77,6 +77,7 @@ struct WsPtrs {
   double* ncut;    // [B][ngrid] log2 of the cut normaliser at the grid positions
   float* emax;     // [B] largest |centred emission| * log2(e) over the valid positions
   int* mode;       // [2][B] ring path per (direction, sequence): 1 exponential, 2 log domain
+  float* tmax;     // [1] M = max trans * log2(e), written by the exponential-domain rings
 };
 
 }  // namespace semicrf

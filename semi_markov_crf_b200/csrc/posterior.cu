@@ -66,15 +66,17 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 //   backward ab[t, c] = sum_c' pb[t, c'] 2^(trans2[c, c'] - M)   (beta[t])
 // except at the walks' start boundaries (gamma[0] = 0, beta[L] = 0), where it
 // is 2^-M.  One CTA per (block of KA_ROWS rows, direction, sequence).
-constexpr int KA_ROWS = 64;
+// rows per CTA: 128, or 64 for the widest columns (static shared memory <= 48 KB)
+template <int NW>
+constexpr int ka_rows() { return NW <= 64 ? 128 : 64; }
 // NW >= C: the weight column a thread keeps in registers (padded with 0) and
 // the padded row length of the staged p rows (16-byte vector reads).
 template <int NW>
 __global__ void __launch_bounds__(256)
     kept_acc_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                     const float* __restrict__ trans) {
+  constexpr int KA_ROWS = ka_rows<NW>();
   __shared__ __align__(16) float pt[KA_ROWS * NW];  // p rows, zero padded
-  __shared__ int aux[1];
   const int rb = blockIdx.x, dir = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int C = d.C;
   const int L = lengths[b];
@@ -83,16 +85,7 @@ __global__ void __launch_bounds__(256)
   const int r0 = rb * KA_ROWS;
   if (r0 > L) return;
   const int nr = min(r0 + KA_ROWS, L + 1) - r0;
-  if (tid == 0) aux[0] = f2ord(NEG_INF);
-  __syncthreads();
-  float M;
-  {
-    float m = NEG_INF;
-    for (int i = tid; i < C * C; i += blockDim.x) m = fmaxf(m, __ldg(trans + i) * l2e());
-    warp_max_to_shared(&aux[0], f2ord(m));
-    __syncthreads();
-    M = ord2f(aux[0]);
-  }
+  const float M = *ws.tmax;  // max trans2, written by the rings
   float* const kv = ws.kv + (((size_t)b * 2 + dir) * (d.T + 1) + r0) * 2 * C;
   for (int i = tid; i < nr * NW; i += blockDim.x) {
     const int r = i / NW, x = i - r * NW;
@@ -128,13 +121,12 @@ __global__ void __launch_bounds__(256)
 
 #define SEMICRF_KA_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
 
-int kept_acc_rows() { return KA_ROWS; }
-
 cudaError_t launch_kept_acc(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                             const float* trans, cudaStream_t st) {
-  const dim3 grid((d.T + KA_ROWS) / KA_ROWS, 2, d.B);
 #define SEMICRF_KA_LAUNCH(nw)                                                  \
   if (d.C <= nw) {                                                             \
+    constexpr int rows = ka_rows<nw>();                                        \
+    const dim3 grid((d.T + rows) / rows, 2, d.B);                              \
     kept_acc_kernel<nw><<<grid, 256, 0, st>>>(d, ws, lengths, trans);          \
     return cudaGetLastError();                                                 \
   }
@@ -157,7 +149,6 @@ __global__ void __launch_bounds__(256)
     cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                     const float* __restrict__ trans, const float* __restrict__ dur) {
   extern __shared__ float csh[];  // la [K][C], lb [K][C], dd [K][C]
-  __shared__ int aux[2];
   __shared__ float lab_M[128], lab_f[128];  // per label: shift, log2 share
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int C = d.C, K = d.K;
@@ -175,16 +166,7 @@ __global__ void __launch_bounds__(256)
     if (tid == 0) *out = ws.logz2[b];
     return;
   }
-  if (tid == 0) aux[0] = f2ord(NEG_INF);
-  __syncthreads();
-  float M;
-  {
-    float m = NEG_INF;
-    for (int i = tid; i < C * C; i += blockDim.x) m = fmaxf(m, __ldg(trans + i) * l2e());
-    warp_max_to_shared(&aux[0], f2ord(m));
-    __syncthreads();
-    M = ord2f(aux[0]);
-  }
+  const float M = *ws.tmax;  // max trans2, written by the rings
   float* const la = csh;
   float* const lb = csh + (size_t)K * C;
   float* const dd = csh + 2 * (size_t)K * C;
@@ -308,7 +290,6 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
                      const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
                      float* __restrict__ start_marg, float* __restrict__ end_marg) {
   extern __shared__ __align__(16) unsigned char psh[];
-  __shared__ int aux[1];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
   const int C = d.C, K = d.K, RT = d.pRT;
   const int L = lengths[b];
@@ -319,16 +300,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
   const int t1 = min(t0 + d.delta, L);
   const size_t seg = (size_t)b * d.nck + j;
   const float gb = (float)(grad_logZ ? grad_logZ[b] : 1.0);
-  if (tid == 0) aux[0] = f2ord(NEG_INF);
-  __syncthreads();
-  float M;
-  {
-    float m = NEG_INF;
-    for (int i = tid; i < C * C; i += nthr) m = fmaxf(m, __ldg(trans + i) * l2e());
-    warp_max_to_shared(&aux[0], f2ord(m));
-    __syncthreads();
-    M = ord2f(aux[0]);
-  }
+  const float M = *ws.tmax;  // max trans2, written by the rings
   const PTile tl = ptile_carve(psh, RT, K, C);
   const float* pfr = kv_row(ws, d, b, 0, 0);  // row t: pfr + t*2C (p), + C (acc)
   const float* pbr = kv_row(ws, d, b, 1, 0);
@@ -460,7 +432,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
 int posterior_tile_rows(const Dims& d, size_t budget) {
   int cap = 64;
   while (cap > 8 && cap / 2 >= d.delta) cap /= 2;
-  for (const size_t lim : {std::min<size_t>(budget, 100u * 1024u), budget})
+  for (const size_t lim : {std::min<size_t>(budget, 112u * 1024u), budget})
     for (int rt = cap; rt >= 8; rt /= 2)
       if (ptile_bytes(rt, d.K, d.C) <= lim) return rt;
   return 0;

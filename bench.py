@@ -363,8 +363,13 @@ def run_ours(args):
     # takes its own sequences): positions per ring kernel, both directions
     dom = semicrf.ring_domains(ws)
     lens = [int(x) for x in w["lengths"]]
+    kept = [dom[b] == 1 and dom[B + b] == 1 for b in range(B)]
     ring_pos = {"chain_exp_kernel": sum(lens[i % B] for i, m in enumerate(dom) if m == 1) / 2,
-                "chain_kernel": sum(lens[i % B] for i, m in enumerate(dom) if m == 2) / 2}
+                "chain_kernel": sum(lens[i % B] for i, m in enumerate(dom) if m == 2) / 2,
+                # the posterior pass takes the sequences both of whose rings
+                # kept their values, the checkpoint walk the others
+                "posterior_kernel": sum(l for l, k in zip(lens, kept) if k),
+                "segment_kernel": sum(l for l, k in zip(lens, kept) if not k)}
 
     stream = torch.cuda.current_stream(dev)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]

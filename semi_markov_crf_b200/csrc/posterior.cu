@@ -281,8 +281,10 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, 
 // after it that its segments end on, in shared memory with coalesced loads;
 // then every (boundary, label), (duration, label) and (label, label) item is
 // computed from shared memory.  Each thread keeps the duration and transition
-// sums of its first NID / NIT items in registers across tiles; items beyond
-// (large K C or C C) add their per-tile sums to the float64 partials.
+// sums of its first NID / NIT items in registers across tiles (with 512
+// threads that is every item within this build's limits: K C <= 8192, where
+// the log-domain kernels' shared memory ends, and C <= 128); items beyond
+// would add their per-tile sums to the float64 partials.
 template <int NID, int NIT>
 __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,

@@ -28,6 +28,9 @@ def _cases():
         "mixed_with_empty": lambda: synth.make_custom(4, 80, 9, 5, seed=9, lengths=[80, 0, 1, 57]),
         "delta_not_multiple_of_K": lambda: synth.make_custom(1, 501, 7, 3, seed=10),
         "many_segments_small_K": lambda: synth.make_custom(2, 1200, 3, 4, seed=11, lengths=[1200, 999]),
+        # C = 64: the traceback stages a few hundred rows at a time, so these
+        # lengths take several stages
+        "traceback_in_stages": lambda: synth.make_custom(2, 900, 16, 64, seed=13, lengths=[900, 777]),
     }
 
 

@@ -248,8 +248,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
   // kept values for the posterior pass: per boundary (row) the vector p,
-  // relative to the boundary's frame kf (the label fan-in part of each row is
-  // filled from p afterwards by kept_acc_kernel)
+  // relative to the boundary's frame kf, stored by the combine leaders at the
+  // end of their step (the label fan-in part of each row is filled from p
+  // afterwards by kept_acc_kernel)
   const int dir = UP ? 0 : 1;
   float* const kv = ws.kv ? ws.kv + (((size_t)b * 2 + dir) * (d.T + 1)) * 2 * C : nullptr;
   double* const kf = ws.kf ? ws.kf + ((size_t)b * 2 + dir) * (d.T + 1) : nullptr;
@@ -334,14 +335,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       }
       next_ev = next_event(i);
     }
-    if (kv && !comb && i >= 2) {
-      // the helpers write out p_{i-1} (row r - SG, frame Phi_{i-1}) from the
-      // vector the combine reads this step, off the critical path
-      const float* pp = xs.P + ((i - 1) & 1) * d.xPC;
-      for (int x = tid - nwc * 32; x < C; x += blockDim.x - nwc * 32)
-        kv[(size_t)(r - SG) * 2 * C + x] = pp[x];
-      if (tid == nwc * 32) kf[r - SG] = F0 + (double)Fph;
-    }
+    // the frame of the row the combine kept last step (Phi_{i-1})
+    if (kv && tid == nwc * 32 && i >= 2) kf[r - SG] = F0 + (double)Fph;
     // Each role issues its shared-memory reads first and its stores last: a
     // store the compiler cannot separate from later reads keeps those reads
     // from being issued early, and every access of the step must complete
@@ -385,6 +380,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
         put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
       }
+      // the kept row of this boundary, last: a global store at the end of the
+      // step costs the path least (measured against the helpers copying it)
+      if (kv && leader) kv[(size_t)r * 2 * C + c] = pn;
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;
@@ -432,12 +430,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     }
     __syncthreads();
   }
-  if (kv && !comb) {  // the last step's vector
-    const int r = UP ? L : 0;
-    const float* pp = xs.P + (L & 1) * d.xPC;
-    for (int x = tid - nwc * 32; x < C; x += blockDim.x - nwc * 32) kv[(size_t)r * 2 * C + x] = pp[x];
-    if (tid == nwc * 32) kf[r] = F0 + (double)(Fph + xs.nsl[L & 1]);
-  }
+  if (kv && tid == nwc * 32)  // the last row's frame (its vector was kept at step L)
+    kf[UP ? L : 0] = F0 + (double)(Fph + xs.nsl[L & 1]);
 
   // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
   if (warp == 0) {

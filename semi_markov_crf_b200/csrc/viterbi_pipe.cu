@@ -27,9 +27,10 @@
 // k among equal terms), the smallest c' among equal label terms, and the
 // smallest final label.
 //
-// Decoding: no argmax label is computed during the recursion.  The helpers
-// write out, one step late, each boundary's row of V (relative to its frame)
-// and of chosen durations.  The traceback needs the best previous label only
+// Decoding: no argmax label is computed during the recursion.  The combine
+// leaders write out, at the end of each step, the boundary's row of V
+// (relative to its frame) and of chosen durations.  The traceback needs the
+// best previous label only
 // where a decoded segment starts, and recomputes it there from the kept row:
 // argmax_{c'} V[s, c'] + trans2[c', c] is the same float sum the combine
 // compared (the frame shifts every term alike), so the result, ties
@@ -53,7 +54,6 @@ struct VSmem {
   int* Ok;     // [2][C]    its duration
   float* A1;   // [2][C]    dur2[0] + S[t] - S[t-1]
   float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
-  int* Kd;     // [2][C]    duration chosen by the combine warps at the step
   float* nsl;  // [2]       frame step published by the combine warps
   float* mx;   // [2]       max V[t-1] published by the helpers at step t
   int* Sb;     // [C]       label integer bases
@@ -87,8 +87,6 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   f += 2 * C;
   x.A2 = f;
   f += 2 * C;
-  x.Kd = reinterpret_cast<int*>(f);
-  f += 2 * C;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
@@ -101,7 +99,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
   return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 11ull * d.C) * 4;
+         (2ull * d.xPC + 9ull * d.C) * 4;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -188,7 +186,6 @@ __global__ void __launch_bounds__(LB, 1)
     vs.Ok[i] = 3;
     vs.A1[i] = NEG_INF;
     vs.A2[i] = NEG_INF;
-    vs.Kd[i] = 1;
   }
   if (tid == 0) {
     vs.nsl[0] = vs.nsl[1] = 0.f;
@@ -232,7 +229,6 @@ __global__ void __launch_bounds__(LB, 1)
   // kept rows of boundaries 1..L: V (frame-relative) and the chosen duration
   float* const vrw = ws.vrow + (size_t)b * (T + 1) * C;
   int32_t* const kdw = ws.bp + (size_t)b * (T + 1) * C;
-  const int hx = tid - nwc * 32, nh = blockDim.x - nwc * 32;  // helper thread index, count
   // combine state: S at row i - 1, ring slot of boundary i - 1
   float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
   int si_p = 0;
@@ -327,15 +323,19 @@ __global__ void __launch_bounds__(LB, 1)
       const float c2 = (g2 + a2) - nprev;
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
-      if (leader) {
-        vs.V[(i & 1) * d.xPC + c] = v - n;
-        vs.Kd[(i & 1) * C + c] = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
-      }
+      const int kdec = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
+      if (leader) vs.V[(i & 1) * d.xPC + c] = v - n;
       if (tid == 0) vs.nsl[i & 1] = n;
       // off the path: G[i-1]'s ring entry (frame Phi_{i-1})
       if (leader && i >= 2) {
         const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
         for (int x = wslot; x < RL; x += K) rl[x] = e;
+      }
+      // boundary i's kept rows (V relative to Phi_i, the chosen duration),
+      // last: a global store at the end of the step costs the path least
+      if (leader) {
+        vrw[(size_t)i * C + c] = v - n;
+        kdw[(size_t)i * C + c] = kdec;
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
       g2 = gv;
@@ -347,16 +347,8 @@ __global__ void __launch_bounds__(LB, 1)
       crow_f += C;
     } else {
       // ---------------------------------------------------------- helpers
-      // reads: boundary i - 1's kept rows (V[i-1] and its chosen durations,
-      // both written last step; a helper thread holds at most two of the
-      // 2C values, nh >= C), row V[i-1] for the frame max, the window of the
-      // k >= 3 terms of step i + 1 (boundaries i - 1 - WL .. i - 2) and its
-      // prefix-sum row
-      const float* vpr = vs.V + ((i - 1) & 1) * d.xPC;
-      const int* kpr = vs.Kd + ((i - 1) & 1) * C;
-      const int x1 = hx + nh;
-      const float kv0 = (hx < C) ? vpr[hx] : __int_as_float(kpr[min(hx - C, C - 1)]);
-      const float kv1 = (x1 < C) ? vpr[x1] : __int_as_float(kpr[min(max(x1 - C, 0), C - 1)]);
+      // reads: row V[i-1] for the frame max, the window of the k >= 3 terms
+      // of step i + 1 (boundaries i - 1 - WL .. i - 2) and its prefix-sum row
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
       float m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
@@ -390,20 +382,6 @@ __global__ void __launch_bounds__(LB, 1)
       for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
       // stores (every label group saw all of V[i-1]: the first one publishes)
       if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;
-      if (i >= 2) {
-        if (hx < 2 * C) {
-          if (hx < C)
-            vrw[(size_t)(i - 1) * C + hx] = kv0;
-          else
-            kdw[(size_t)(i - 1) * C + hx - C] = __float_as_int(kv0);
-        }
-        if (x1 < 2 * C) {
-          if (x1 < C)
-            vrw[(size_t)(i - 1) * C + x1] = kv1;
-          else
-            kdw[(size_t)(i - 1) * C + x1 - C] = __float_as_int(kv1);
-        }
-      }
       if (leader && i < L) {
         const int o2 = ((i + 1) & 1) * C + c;
         vs.Om[o2] = best + fn;
@@ -423,18 +401,6 @@ __global__ void __launch_bounds__(LB, 1)
     }
     __syncthreads();
   }
-  // boundary L's kept rows
-  if (!comb) {
-    const float* vp = vs.V + (L & 1) * d.xPC;
-    const int* kp = vs.Kd + (L & 1) * C;
-    for (int x = hx; x < 2 * C; x += nh) {
-      if (x < C)
-        vrw[(size_t)L * C + x] = vp[x];
-      else
-        kdw[(size_t)L * C + x - C] = kp[x - C];
-    }
-  }
-
   // the optimum: max over the final labels of V[L] in frame Phi_L
   if (tid < 32) {
     const float* V = vs.V + (L & 1) * d.xPC;

@@ -303,6 +303,46 @@ std::mutex prof_mu;
 bool prof_on = false;
 std::vector<ProfRec> prof_recs;
 
+// A second stream, per host thread and device, for the kernels of the
+// backward pass that do not depend on each other; forked from and joined
+// back into the caller's stream with events (which stream capture also
+// records), so the call stays ordered on the caller's stream.  nullptr if
+// it cannot be created: the caller's stream then runs everything.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream* side_stream() {
+  thread_local std::vector<SideStream> per_dev;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if ((int)per_dev.size() <= dev) per_dev.resize(dev + 1);
+  SideStream& ss = per_dev[dev];
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      ss = SideStream{};
+      return nullptr;
+    }
+  }
+  return &ss;
+}
+// The side stream waits for everything queued on st so far.
+bool side_fork(SideStream* ss, cudaStream_t st) {
+  return !ss || (cudaEventRecord(ss->fork, st) == cudaSuccess &&
+                 cudaStreamWaitEvent(ss->s, ss->fork, 0) == cudaSuccess);
+}
+// st waits for everything queued on the side stream so far.
+bool side_join(SideStream* ss, cudaStream_t st) {
+  return !ss || (cudaEventRecord(ss->join, ss->s) == cudaSuccess &&
+                 cudaStreamWaitEvent(st, ss->join, 0) == cudaSuccess);
+}
+
 struct ProfScope {
   cudaStream_t st;
   ProfRec rec{nullptr, nullptr, nullptr};
@@ -476,6 +516,17 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     const size_t fsm = ((size_t)C + (size_t)nj * C) * sizeof(double);
     rc = set_smem((const void*)finalize_positions_kernel, fsm);
     if (rc) return rc;
+    // the parameter-gradient sums (side stream) and the per-position outputs
+    // read different partials
+    SideStream* ss = side_stream();
+    const cudaStream_t s2 = ss ? ss->s : st;
+    if (!side_fork(ss, st)) return SEMICRF_ERR_CUDA;
+    {
+      ProfScope ps("reduce_partials_kernel", s2);
+      reduce_partials_kernel<<<(C * C + K * C + RP_E - 1) / RP_E, RP_E * RP_S, 0, s2>>>(
+          d, p, lengths, grad_trans, grad_dur);
+    }
+    const int rc_red = launched();
     {
       ProfScope ps("finalize_positions_kernel", st);
       finalize_positions_kernel<<<dim3((T + FIN_ROWS_HOST - 1) / FIN_ROWS_HOST, B), 256, fsm,
@@ -483,7 +534,9 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
                                         (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, grad_em,
                                         pos_marg, start_marg, end_marg);
     }
-    if ((rc = launched())) return rc;
+    rc = launched();
+    if (!side_join(ss, st)) return SEMICRF_ERR_CUDA;
+    return rc_red ? rc_red : rc;
   } else {
     // T == 0: only boundary row 0 exists, and nothing starts or ends there
     if (start_marg && cudaMemsetAsync(start_marg, 0, (size_t)B * C * 4, st) != cudaSuccess)

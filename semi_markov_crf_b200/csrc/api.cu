@@ -225,6 +225,9 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_segV = take(B * nck * C * 8);
   const size_t o_bp = take(B * (size_t)(d.T + 1) * C * 4);
   const size_t o_vrow = take(d.xG ? B * (size_t)(d.T + 1) * C * 4 : 0);
+  const size_t CP = (C + 3) / 4 * 4;
+  const size_t o_wrd = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
+  const size_t o_wdl = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
   const size_t o_kv = take(B * 2ull * (d.T + 1) * 2 * C * 4);
   const size_t o_kf = take(B * 2ull * (d.T + 1) * 8);
   const size_t o_ncut = take(B * (size_t)d.ngrid * 8);
@@ -250,6 +253,8 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->segV = reinterpret_cast<double*>(c + o_segV);
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
     p->vrow = reinterpret_cast<float*>(c + o_vrow);
+    p->wrd = reinterpret_cast<int32_t*>(c + o_wrd);
+    p->wdl = reinterpret_cast<int32_t*>(c + o_wdl);
     p->kv = reinterpret_cast<float*>(c + o_kv);
     p->kf = reinterpret_cast<double*>(c + o_kf);
     p->ncut = reinterpret_cast<double*>(c + o_ncut);

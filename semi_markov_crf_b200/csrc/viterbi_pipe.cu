@@ -414,8 +414,10 @@ __global__ void __launch_bounds__(LB, 1)
 
 // Backpointer words, in parallel over (boundary, label): for boundary t in
 // [1, L] and label c with k = kd[t, c] and s = t - k >= 1, the word is
-// k | argmax_{c'} (V[s, c'] + trans2[c', c]) << 16 (smallest c' on ties),
-// written over kd[t, c]; for s = 0 the word is k.  One CTA per block of
+// k | argmax_{c'} (V[s, c'] + trans2[c', c]) << 16 (smallest c' on ties);
+// for s = 0 the word is k.  Beside it goes the step from this word's index
+// to the previous segment's, -k * CP + (c' - c), for a walk over rows CP =
+// C rounded up to 4 apart (16-byte rows, copied to shared memory in bulk).  One CTA per block of
 // VW_ROWS boundaries of a sequence: the V rows its segments start at are
 // staged in shared memory (rows of VS = C rounded up to 4 floats, -inf
 // padded), and thread (label c, row phase) keeps trans2[., c] in registers.
@@ -437,7 +439,9 @@ __global__ void __launch_bounds__(256)
   const int VS = (C + 3) & ~3;
   const int vlo = max(1, t0 - K);  // V rows [vlo, t1 - 1]
   const float* vrw = ws.vrow + (size_t)b * (d.T + 1) * C;
-  int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
+  const int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
+  int32_t* wrd = ws.wrd + (size_t)b * (d.T + 1) * VS;
+  int32_t* wdl = ws.wdl + (size_t)b * (d.T + 1) * VS;
   const int nv = (t1 - vlo) * VS;
 #pragma unroll 4
   for (int i = tid; i < nv; i += blockDim.x) {
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(256)
   for (int t = t0 + pg; t <= t1; t += png) {
     const int k = kdw[(size_t)t * C + pc];
     const int sb = t - k;
-    int word = k;
+    int word = k, step = 0;
     if (k >= 1 && k <= K && sb >= 1) {
       const float4* vr = reinterpret_cast<const float4*>(vsh + (size_t)(sb - vlo) * VS);
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
@@ -477,34 +481,45 @@ __global__ void __launch_bounds__(256)
       if (b3 > b2 || (b3 == b2 && q3 < q2)) { b2 = b3; q2 = q3; }
       if (b2 > b0 || (b2 == b0 && q2 < q0)) { b0 = b2; q0 = q2; }
       word = k | (q0 << 16);
+      step = -k * VS + (q0 - pc);
     }
-    kdw[(size_t)t * C + pc] = word;
+    wrd[(size_t)t * VS + pc] = word;
+    wdl[(size_t)t * VS + pc] = step;
   }
 }
 
 // The traceback, one CTA per sequence.  Start: the best final label
 // (argmax of the kept row V[L], smallest on ties).  In stages over the
-// dynamic shared memory: the block stages the word rows [lo, tt0]
-// (coalesced), thread 0 follows the words -- one shared-memory read per
+// dynamic shared memory: thread 0 copies the word rows [lo, tt0] and their
+// index steps in with two bulk copies (TMA, completion on an mbarrier, a
+// bounded wait), follows the words -- one shared-memory read and an add per
 // decoded segment -- and marks each segment's start position with its
-// label, then warp 0 fills every position of the stage with the label of
-// the last mark at or below it (a running "last mark" scan, 32 positions per
+// label; then warp 0 fills every position of the stage with the label of the
+// last mark at or below it (a running "last mark" scan, 32 positions per
 // shuffle round) and writes labels and start flags out coalesced.  The next
 // stage starts where the walk left the staged rows.  A word with a duration
-// outside [1, t] or a previous label >= C ends the walk with the positions
-// not reached labelled -1.
+// outside [1, t], a previous label >= C or a step leaving the staged rows
+// ends the walk with the positions not reached labelled -1.
 __global__ void __launch_bounds__(256)
     viterbi_walk_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                         int32_t* __restrict__ labels, uint8_t* __restrict__ seg_start, int WR) {
-  extern __shared__ __align__(16) int wsh[];  // words [WR][C], marks [WR + K]
+  extern __shared__ __align__(16) int wsh[];  // words [WR][CP], steps [WR][CP], marks [WR + K]
   __shared__ int s_tb[2];
+  __shared__ __align__(8) uint64_t wbar;
   const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x, lane = tid & 31, b = blockIdx.x;
+  const int CP = (C + 3) & ~3;
   const int L = lengths[b];
   if (L < 1 || L > T) return;
-  const int32_t* kdw = ws.bp + (size_t)b * (T + 1) * C;
+  const int32_t* wrd = ws.wrd + (size_t)b * (T + 1) * CP;
+  const int32_t* wdl = ws.wdl + (size_t)b * (T + 1) * CP;
   const float* vrw = ws.vrow + (size_t)b * (T + 1) * C;
   int* const kbuf = wsh;
-  int* const lbuf = wsh + (size_t)WR * C;
+  int* const dbuf = wsh + (size_t)WR * CP;
+  int* const lbuf = wsh + 2 * (size_t)WR * CP;
+  if (tid == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+  }
   if (tid < 32) {
     float best = NEG_INF;
     int bc = 0x7fffffff;
@@ -522,24 +537,37 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
+  uint32_t phase = 0;
   for (;;) {
     const int tt0 = s_tb[0];
     if (tt0 <= 0) break;
     const int lo = max(1, tt0 - WR + 1);
     const int pb = lo - K;  // mark of position u at lbuf[u - pb]
-    {
-      const int nk = (tt0 - lo + 1) * C;
-      const int32_t* ksrc = kdw + (size_t)lo * C;
-#pragma unroll 8
-      for (int i = tid; i < nk; i += blockDim.x) kbuf[i] = ksrc[i];
-      for (int i = tid; i < WR + K; i += blockDim.x) lbuf[i] = -1;
+    const uint32_t bytes = (uint32_t)((tt0 - lo + 1) * CP * 4);
+    if (tid == 0) {
+      fence_proxy_async();  // the last stage's reads come before the copies' writes
+      mbar_expect_tx(&wbar, 2 * bytes);
+      bulk_g2s(kbuf, wrd + (size_t)lo * CP, bytes, &wbar);
+      bulk_g2s(dbuf, wdl + (size_t)lo * CP, bytes, &wbar);
     }
-    __syncthreads();
+    for (int i = tid; i < WR + K; i += blockDim.x) lbuf[i] = -1;
+    const bool ok = mbar_wait(&wbar, phase, WAIT_SPIN_LIMIT);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) {
+        set_status(ws.status, ST_DEVICE_TIMEOUT);
+        mbar_wait(&wbar, phase ^ 1u, WAIT_SPIN_LIMIT);  // let the copies land before exit
+      }
+      return;
+    }
     if (tid == 0) {
       int tt = tt0, cl = s_tb[1];
+      int idx = (tt - lo) * CP + cl;
+      const int nidx = (tt0 - lo + 1) * CP;
       bool broken = false;
       while (tt >= lo) {
-        const int w = kbuf[(tt - lo) * C + cl];
+        const int w = kbuf[idx];
+        const int step = dbuf[idx];
         const int k = w & 0xffff, pred = (w >> 16) & 0xffff;
         if (k < 1 || k > tt || (tt - k > 0 && pred >= C)) {
           broken = true;
@@ -548,6 +576,11 @@ __global__ void __launch_bounds__(256)
         tt -= k;
         lbuf[tt - pb] = cl;
         cl = pred;
+        idx += step;
+        if (tt >= lo && (idx < 0 || idx >= nidx)) {
+          broken = true;
+          break;
+        }
       }
       s_tb[0] = broken ? -tt : tt;  // -tt: stop, positions below tt get -1
       s_tb[1] = cl;
@@ -609,16 +642,18 @@ cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t*
 }
 
 // Shared memory of the walk: about 96 KB (fewer stages), at least the K
-// marks and one row.
+// marks and one row of words and steps.
 size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget) {
+  const size_t CP = (d.C + 3) & ~3;
   const size_t want = std::min<size_t>(budget, 96u * 1024u);
-  const size_t need = ((size_t)d.K + 1 + 2 * (size_t)d.C) * sizeof(int);
+  const size_t need = ((size_t)d.K + 1 + 2 * CP) * sizeof(int);
   return std::max(want, need);
 }
 
 cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 int32_t* labels, uint8_t* seg_start, size_t sm, cudaStream_t st) {
-  const int WR = (int)((sm / sizeof(int) - (size_t)d.K) / ((size_t)d.C + 1));
+  const size_t CP = (d.C + 3) & ~3;
+  const int WR = (int)((sm / sizeof(int) - (size_t)d.K) / (2 * CP + 1));
   if (sm > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(viterbi_walk_kernel,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

@@ -494,11 +494,6 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     // others: the checkpoint walk.  Each kernel skips the other's sequences.
     cudaError_t e;
     if (d.xG) {
-      {
-        ProfScope ps("kept_acc_kernel", st);
-        e = launch_kept_acc(d, p, lengths, trans, st);
-      }
-      if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
       const size_t csm = cut_grid_smem_bytes(d);
       if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
       {

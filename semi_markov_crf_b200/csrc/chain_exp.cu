@@ -102,17 +102,6 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   return x;
 }
 
-// Block-wide max of f(i) over i < n (all threads; one barrier; aux slot must
-// hold f2ord(-inf) beforehand and is left holding the result).
-template <typename F>
-__device__ __forceinline__ float block_max(int* slot, int n, F f) {
-  float m = NEG_INF;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, f(i));
-  warp_max_to_shared(slot, f2ord(m));
-  __syncthreads();
-  return ord2f(*slot);
-}
-
 // 2^-n for an integer-valued n in [-126, 127] (exact, no rounding).
 __device__ __forceinline__ float pow2_neg(float n) {
   return __int_as_float((127 - (int)n) << 23);
@@ -247,16 +236,18 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
     xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
-  // kept values for the posterior pass: per boundary (row) the vector p,
-  // relative to the boundary's frame kf, stored by the combine leaders at the
-  // end of their step (the label fan-in part of each row is filled from p
-  // afterwards by kept_acc_kernel)
+  // kept values for the posterior pass: per boundary (row) the vector p and
+  // the label fan-in acc, relative to the boundary's frame kf, stored by the
+  // combine leaders at the end of their step
   const int dir = UP ? 0 : 1;
   float* const kv = ws.kv ? ws.kv + (((size_t)b * 2 + dir) * (d.T + 1)) * 2 * C : nullptr;
   double* const kf = ws.kf ? ws.kf + ((size_t)b * 2 + dir) * (d.T + 1) : nullptr;
   if (kv) {
-    for (int x = tid; x < C; x += blockDim.x)
+    const int rL = UP ? L : 0;  // the walk's last row: no label fan-in there
+    for (int x = tid; x < C; x += blockDim.x) {
       kv[(size_t)r0 * 2 * C + x] = 0.f;  // no forward vector at 0, no btil at L
+      kv[(size_t)rL * 2 * C + C + x] = 0.f;
+    }
     if (tid == 0) kf[r0] = 0.0;
   }
   __syncthreads();
@@ -382,7 +373,10 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       }
       // the kept row of this boundary, last: a global store at the end of the
       // step costs the path least (measured against the helpers copying it)
-      if (kv && leader) kv[(size_t)r * 2 * C + c] = pn;
+      if (kv && leader) {
+        kv[(size_t)r * 2 * C + c] = pn;                // row r, frame Phi_i
+        kv[(size_t)(r - SG) * 2 * C + C + c] = acc;    // row r - SG, frame Phi_{i-1}
+      }
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;
@@ -494,17 +488,34 @@ __global__ void __launch_bounds__(LB, 1)
     }
     return;
   }
-  // ---- the fast-path test (identical in every CTA of the sequence)
+  // ---- the fast-path test (identical in every CTA of the sequence): one
+  // pass over trans and one over dur for finiteness and both extremes
   if (tid < 4) xs.aux[tid] = f2ord(NEG_INF);
+  __syncthreads();
   bool bad = false;
-  for (int i = tid; i < C * C; i += blockDim.x) bad |= !isfinite(__ldg(trans + i));
-  for (int i = tid; i < K * C; i += blockDim.x) bad |= !isfinite(__ldg(dur + i));
-  bad = __syncthreads_or(bad);  // also orders the aux reset
-  const float M = block_max(&xs.aux[0], C * C, [&](int i) { return __ldg(trans + i) * l2e(); });
+  float tmx = NEG_INF, tmn = INFINITY, dmx = NEG_INF, dmn = INFINITY;
+  for (int i = tid; i < C * C; i += blockDim.x) {
+    const float raw = __ldg(trans + i);
+    bad |= !isfinite(raw);
+    tmx = fmaxf(tmx, raw * l2e());
+    tmn = fminf(tmn, raw * l2e());
+  }
+  for (int i = tid; i < K * C; i += blockDim.x) {
+    const float raw = __ldg(dur + i);
+    bad |= !isfinite(raw);
+    dmx = fmaxf(dmx, raw * l2e());
+    dmn = fminf(dmn, raw * l2e());
+  }
+  warp_max_to_shared(&xs.aux[0], f2ord(tmx));
+  warp_max_to_shared(&xs.aux[1], f2ord(-tmn));
+  warp_max_to_shared(&xs.aux[2], f2ord(dmx));
+  warp_max_to_shared(&xs.aux[3], f2ord(-dmn));
+  bad = __syncthreads_or(bad);  // also completes the four reductions
+  const float M = ord2f(xs.aux[0]);
   if (ws.tmax && threadIdx.x == 0 && blockIdx.x == 0) *ws.tmax = M;  // for the posterior pass
-  const float tmin = -block_max(&xs.aux[1], C * C, [&](int i) { return -__ldg(trans + i) * l2e(); });
-  const float dmax = block_max(&xs.aux[2], K * C, [&](int i) { return __ldg(dur + i) * l2e(); });
-  const float dmin = -block_max(&xs.aux[3], K * C, [&](int i) { return -__ldg(dur + i) * l2e(); });
+  const float tmin = -ord2f(xs.aux[1]);
+  const float dmax = ord2f(xs.aux[2]);
+  const float dmin = -ord2f(xs.aux[3]);
   const float span = fabsf(M) + (M - tmin) + fabsf(dmax) + fabsf(dmin) + 2.f * ws.emax[b] +
                      lg2((float)(K * C));
   if (bad || !(span < FAST_BOUND)) {

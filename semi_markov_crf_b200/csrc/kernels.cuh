@@ -51,9 +51,6 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
   return ws.kv != nullptr && ws.mode != nullptr && ws.mode[b] == 1 && ws.mode[d.B + b] == 1;
 }
 
-// The label fan-in part of the kept rows (C <= 128).
-cudaError_t launch_kept_acc(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                            const float* trans, cudaStream_t st);
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                 const float* __restrict__ trans, const float* __restrict__ dur);
 // The posterior pass (one CTA per checkpoint segment and sequence).

@@ -59,82 +59,6 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 
 }  // namespace
 
-// The label fan-in part of the kept rows, from their p part: the rings keep
-// only p (one vector per boundary, written off the critical path), and the
-// fan-in of the same boundary and frame is a fixed linear map of it,
-//   forward  af[t, c] = sum_c' pf[t, c'] 2^(trans2[c', c] - M)   (gamma[t])
-//   backward ab[t, c] = sum_c' pb[t, c'] 2^(trans2[c, c'] - M)   (beta[t])
-// except at the walks' start boundaries (gamma[0] = 0, beta[L] = 0), where it
-// is 2^-M.  One CTA per (block of KA_ROWS rows, direction, sequence).
-// rows per CTA: 128, or 64 for the widest columns (static shared memory <= 48 KB)
-template <int NW>
-constexpr int ka_rows() { return NW <= 64 ? 128 : 64; }
-// NW >= C: the weight column a thread keeps in registers (padded with 0) and
-// the padded row length of the staged p rows (16-byte vector reads).
-template <int NW>
-__global__ void __launch_bounds__(256)
-    kept_acc_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                    const float* __restrict__ trans) {
-  constexpr int KA_ROWS = ka_rows<NW>();
-  __shared__ __align__(16) float pt[KA_ROWS * NW];  // p rows, zero padded
-  const int rb = blockIdx.x, dir = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int C = d.C;
-  const int L = lengths[b];
-  if (L <= 0 || L > d.T) return;
-  if (!posterior_from_kept(ws, d, b)) return;
-  const int r0 = rb * KA_ROWS;
-  if (r0 > L) return;
-  const int nr = min(r0 + KA_ROWS, L + 1) - r0;
-  const float M = *ws.tmax;  // max trans2, written by the rings
-  float* const kv = ws.kv + (((size_t)b * 2 + dir) * (d.T + 1) + r0) * 2 * C;
-  for (int i = tid; i < nr * NW; i += blockDim.x) {
-    const int r = i / NW, x = i - r * NW;
-    pt[i] = (x < C) ? kv[(size_t)r * 2 * C + x] : 0.f;
-  }
-  // thread (column c, row phase g): rows g, g + ng, ...
-  const int ng = blockDim.x / C;
-  const int c = tid % C, g = tid / C;
-  float w[NW];
-#pragma unroll
-  for (int q = 0; q < NW; ++q)
-    w[q] = (q < C && g < ng)
-               ? ex2(__ldg(trans + (dir == 0 ? (size_t)q * C + c : (size_t)c * C + q)) * l2e() - M)
-               : 0.f;
-  __syncthreads();
-  if (g >= ng) return;
-  const int start = (dir == 0) ? 0 : L;  // the walk's start boundary
-  const float a0 = ex2(-M);
-  for (int r = g; r < nr; r += ng) {
-    const float4* pr = reinterpret_cast<const float4*>(pt + (size_t)r * NW);
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-    for (int q = 0; q < NW / 4; ++q) {
-      const float4 v = pr[q];
-      s0 = fmaf(v.x, w[4 * q], s0);
-      s1 = fmaf(v.y, w[4 * q + 1], s1);
-      s2 = fmaf(v.z, w[4 * q + 2], s2);
-      s3 = fmaf(v.w, w[4 * q + 3], s3);
-    }
-    kv[(size_t)r * 2 * C + C + c] = (r0 + r == start) ? a0 : (s0 + s1) + (s2 + s3);
-  }
-}
-
-#define SEMICRF_KA_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
-
-cudaError_t launch_kept_acc(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                            const float* trans, cudaStream_t st) {
-#define SEMICRF_KA_LAUNCH(nw)                                                  \
-  if (d.C <= nw) {                                                             \
-    constexpr int rows = ka_rows<nw>();                                        \
-    const dim3 grid((d.T + rows) / rows, 2, d.B);                              \
-    kept_acc_kernel<nw><<<grid, 256, 0, st>>>(d, ws, lengths, trans);          \
-    return cudaGetLastError();                                                 \
-  }
-  SEMICRF_KA_WIDTHS(SEMICRF_KA_LAUNCH)
-#undef SEMICRF_KA_LAUNCH
-  return cudaErrorInvalidConfiguration;
-}
-
 // One CTA per (grid position, sequence): log2 of the cut at position u,
 //   Z(u) = sum over segments [s, t) with s <= u < t, t - s <= K, and labels c of
 //          2^(gamma[s, c] - S[s, c] + dur2[t-s-1, c] + S[t, c] + beta[t, c]).

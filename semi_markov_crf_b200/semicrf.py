@@ -21,7 +21,7 @@ __all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi",
 
 # every kernel the library launches (names used by the profiler)
 KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "chain_kernel",
-           "kept_acc_kernel", "cut_grid_kernel", "posterior_kernel", "segment_kernel",
+           "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
            "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
            "viterbi_walk_kernel")

@@ -360,23 +360,23 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         acc = acc_start;  // the start boundary: gamma = 0 in frame 0
         mx = 0.f;
       }
+      // gamma (beta) of the previous row's boundary, frame Phi_{i-1}: its
+      // logarithm is issued first so that its latency hides under the path
+      const float gprev = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
       const float n = exponent_of(mx);
       const float sn = pow2_neg(n);
       const float R = fmaf(acc2, a2v, ohv) * snprev;  // frame Phi_{i-1}
       const float pn = fmaf(acc * sn, a1v, R * sn);
       if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
       if (tid == 0) xs.nsl[i & 1] = n;
-      if (i >= 2 && leader) {
-        // gamma (beta) of the previous row's boundary, frame Phi_{i-1}
-        const float g = (acc > 0.f) ? M + lg2(acc) : NEG_INF;
-        put(wslot, make_float2(g - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
-      }
-      // the kept row of this boundary, last: a global store at the end of the
-      // step costs the path least (measured against the helpers copying it)
+      // the kept row of this boundary, then the ring entry: global stores
+      // after the critical store cost the path least (measured against the
+      // helpers copying the row, and against storing after the ring entry)
       if (kv && leader) {
         kv[(size_t)r * 2 * C + c] = pn;                // row r, frame Phi_i
         kv[(size_t)(r - SG) * 2 * C + C + c] = acc;    // row r - SG, frame Phi_{i-1}
       }
+      if (i >= 2 && leader) put(wslot, make_float2(gprev - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;

@@ -326,16 +326,16 @@ __global__ void __launch_bounds__(LB, 1)
       const int kdec = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
       if (leader) vs.V[(i & 1) * d.xPC + c] = v - n;
       if (tid == 0) vs.nsl[i & 1] = n;
-      // off the path: G[i-1]'s ring entry (frame Phi_{i-1})
-      if (leader && i >= 2) {
-        const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
-        for (int x = wslot; x < RL; x += K) rl[x] = e;
-      }
-      // boundary i's kept rows (V relative to Phi_i, the chosen duration),
-      // last: a global store at the end of the step costs the path least
+      // off the path: boundary i's kept rows (V relative to Phi_i, the chosen
+      // duration; global stores after the critical store cost the path
+      // least), then G[i-1]'s ring entry (frame Phi_{i-1})
       if (leader) {
         vrw[(size_t)i * C + c] = v - n;
         kdw[(size_t)i * C + c] = kdec;
+      }
+      if (leader && i >= 2) {
+        const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
+        for (int x = wslot; x < RL; x += K) rl[x] = e;
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
       g2 = gv;

@@ -492,7 +492,16 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     // sequences whose rings both ran in the exponential domain: posteriors
     // from the kept values (cut normalisers, then one parallel pass); the
     // others: the checkpoint walk.  Each kernel skips the other's sequences.
-    cudaError_t e;
+    cudaError_t e = cudaSuccess, e_seg;
+    // the checkpoint walk (side stream) and the posterior pass take
+    // different sequences
+    SideStream* ss = side_stream();
+    const cudaStream_t s2 = ss ? ss->s : st;
+    if (!side_fork(ss, st)) return SEMICRF_ERR_CUDA;
+    {
+      ProfScope ps("segment_kernel", s2);
+      e_seg = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, s2);
+    }
     if (d.xG) {
       const size_t csm = cut_grid_smem_bytes(d);
       if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
@@ -505,21 +514,15 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
         ProfScope ps("posterior_kernel", st);
         e = launch_posterior(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
       }
-      if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
     }
-    {
-      ProfScope ps("segment_kernel", st);
-      e = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
-    }
-    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    if (!side_join(ss, st)) return SEMICRF_ERR_CUDA;
+    if (e != cudaSuccess || e_seg != cudaSuccess) return SEMICRF_ERR_CUDA;
     const int nj = FIN_ROWS_HOST / d.delta + 2;
     const size_t fsm = ((size_t)C + (size_t)nj * C) * sizeof(double);
     rc = set_smem((const void*)finalize_positions_kernel, fsm);
     if (rc) return rc;
     // the parameter-gradient sums (side stream) and the per-position outputs
     // read different partials
-    SideStream* ss = side_stream();
-    const cudaStream_t s2 = ss ? ss->s : st;
     if (!side_fork(ss, st)) return SEMICRF_ERR_CUDA;
     {
       ProfScope ps("reduce_partials_kernel", s2);

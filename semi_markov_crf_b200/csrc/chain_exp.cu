@@ -292,27 +292,19 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         crow_f = sm.tfrac + o;
       }
       if (i == next_ck) {
-        // rebase the ring to (F0 + D, S_int at the boundary) and save it
-        const int bnd = UP ? i - 1 : r + 2;
-        const int j = UP ? bnd / delta : bnd / delta - 1;
+        // rebase the ring to (F0 + D, S_int at the boundary): keeps the
+        // integer parts small over long walks.  (No checkpoint is saved: both
+        // rings of a sequence take the same domain, so the posteriors of this
+        // kernel's sequences come from the kept rows, never from a walk.)
         const float D = comb ? Fp : Fph;  // both are Phi_{i-1} - F0
         if (comb) {
           const int sit = UP ? si_p : si_pp;
           if (act) {
             const float adj = sg * (float)(sit - Sbc) - D;
             for (int x = jl; x < RL; x += G) rl[x].y += adj;
-          }
-          __syncwarp();  // every lane of the warp, labels >= C included
-          if (act) {
-            float2* dst = (UP ? ws.ack : ws.bck) + (((size_t)b * d.nck + j) * K) * C + c;
-            for (int q = jl; q < K; q += G) {
-              const int bb = UP ? bnd - K + q : bnd + q;
-              if (UP ? bb >= 0 : bb <= L) dst[(size_t)q * C] = rl[bb % K];
-            }
             if (leader) xs.Sb[c] = sit;
           }
         }
-        if (tid == 0) (UP ? ws.acf : ws.bcf)[(size_t)b * d.nck + j] = F0 + (double)D;
         __syncthreads();
         F0 += (double)D;
         if (comb) {

@@ -402,6 +402,40 @@ def run_ours(args):
     launches_per_step = sum(v["launches"] for v in kern.values()) / args.steps
     peak_mem = torch.cuda.max_memory_allocated(dev)
 
+    # --- the loss: log Z - score(gold) with its gradient (the gold-path part
+    # subtracted from the step's gradients), timed on its own: it is not part
+    # of the fwd+bwd metric
+    gold = torch.from_numpy(w["gold"]).to(dev)
+    gold_start = torch.from_numpy(w["gold_start"]).to(dev)
+    nll_grads = {k: torch.zeros_like(out[k]) for k in ("grad_em", "grad_trans", "grad_dur")}
+    gscore = torch.empty(B, dtype=torch.float64, device=dev)
+
+    def nll_step():
+        semicrf.path_score(em, lengths, trans, dur, gold, gold_start, ws=ws, negate=True,
+                           grads=nll_grads, score=gscore)
+
+    for _ in range(max(args.warmup, 3)):
+        nll_step()
+    torch.cuda.synchronize(dev)
+    n_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    n_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    semicrf.profile_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        n_s[i].record(stream)
+        nll_step()
+        n_e[i].record(stream)
+    torch.cuda.synchronize(dev)
+    semicrf.profile_enable(False)
+    nll_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(n_s, n_e)), dev) / args.steps
+    nll_kern = {}
+    for name in ("path_terms_kernel", "path_final_kernel", "path_grad_em_kernel",
+                 "path_grad_param_kernel"):
+        tot, n = semicrf.profile_read(name)
+        if n:
+            nll_kern[name] = {"ms_total": tot, "launches": n, "ms_per_launch": tot / n}
+    nll_ok = bool(torch.isfinite(gscore).all().item()) and semicrf.get_status(ws) == 0
+
     # --- end to end: host (pinned) inputs -> device -> results back to host
     h_em = torch.from_numpy(w["em"]).pin_memory()
     h_len = torch.from_numpy(w["lengths"]).pin_memory()
@@ -490,6 +524,28 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "results_checked": bool(ok)},
             "clocks": clocks,
+        }
+        # algorithmic bytes per position: the terms pass reads the emission
+        # row (4C, for nu), the label (4) and the start flag (1); the
+        # emission-gradient pass reads and writes its row (8C) and the label
+        nll_bytes = {"path_terms_kernel": (4 * C + 5) * positions,
+                     "path_grad_em_kernel": (8 * C + 4) * positions}
+        nll_roofs = {}
+        for k, nb in nll_bytes.items():
+            if k in nll_kern:
+                per = nll_kern[k]["ms_per_launch"]
+                nll_roofs[k] = {"bound": "hbm", "achieved": nb / (per * 1e-3) / 1e9,
+                                "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
+                                "frac": (nb / (per * 1e-3) / 1e9) / peaks["hbm_gbs"]
+                                if peaks.get("hbm_gbs") else None,
+                                "bytes_per_launch": nb}
+        line["nll"] = {
+            "what": "loss log Z - score(gold) and its gradient: semicrf_path_score with "
+                    "SEMICRF_FLAG_NEGATE_GRAD on the gradient buffers (gold = the generating "
+                    "segmentation), timed alone with L2 flushed between steps",
+            "ms_per_step": nll_ms, "kernels": nll_kern, "roofline": nll_roofs,
+            "gpu_launches_per_step": sum(v["launches"] for v in nll_kern.values()) / args.steps,
+            "scores_finite": nll_ok,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)

@@ -11,6 +11,8 @@
  *   3. a checkpointed backward pass giving exact
  *      marginals and gradients                       semicrf_backward
  *   4. max-semiring (Viterbi) decoding               semicrf_viterbi
+ *   and the score of a given segmentation with its
+ *   gradient, for the training loss                  semicrf_path_score
  *
  * Model.  A sequence b has length L_b (0 <= L_b <= T).  A segmentation
  * splits its positions 0..L_b-1 into consecutive segments [s, t) of duration
@@ -85,6 +87,9 @@ enum semicrf_status {
                                           keep every step within float32's exponent
                                           range runs in the faster exponential domain;
                                           results agree to rounding) */
+#define SEMICRF_FLAG_NEGATE_GRAD 0x8u  /* semicrf_path_score subtracts its gradient
+                                          (w_b = -grad_score[b]); the other calls
+                                          ignore it */
 
 /*
  * Bytes of device workspace needed by forward/backward/viterbi for these
@@ -159,6 +164,41 @@ SEMICRF_API int semicrf_backward(const int32_t *lengths, const float *trans, con
 SEMICRF_API int semicrf_viterbi(const float *em, const int32_t *lengths, const float *trans, const float *dur,
                     int B, int T, int C, int K, unsigned flags, void *ws, size_t ws_bytes,
                     double *score, int32_t *labels, uint8_t *seg_start, semicrf_stream_t stream);
+
+/*
+ * Score of given segmentations, for the training loss (explainer section 4,
+ * "Results and Benchmarks", Correctness: the model is trained to the CRF loss,
+ * the negative log-likelihood log Z - score(gold)).  The path of sequence b is
+ * labels[b, u] (int32) and seg_start[b, u] (uint8, nonzero where a segment
+ * starts), u < L_b, the form semicrf_viterbi writes; entries u >= L_b are
+ * never read.  Writes score[b] (float64, nullable): the model score of that
+ * segmentation, the same sum as in the model above (centred unless
+ * SEMICRF_FLAG_NO_CENTER).  A malformed path -- no start at u = 0, a label
+ * outside [0, C), a label that changes inside a segment, a segment longer
+ * than K -- gets score NaN and no gradient; L_b = 0 scores 0.
+ *
+ * Gradients are ACCUMULATED: for each non-null output,
+ *   grad_em    [B, T, C] += w_b * d score_b / d em[b, u, c]
+ *                           = w_b * ([labels[b,u] = c] - n_bc / L_b)  (u < L_b;
+ *                             n_bc positions labelled c, the second term
+ *                             through the centring mean)
+ *   grad_trans [C, C]    += sum_b w_b * (#c' -> c transitions on path b)
+ *   grad_dur   [K, C]    += sum_b w_b * (#label-c segments of length k)
+ * with w_b = grad_score[b] (device float64 [B]; NULL means all ones), negated
+ * under SEMICRF_FLAG_NEGATE_GRAD.  For the NLL log Z - score, run
+ * semicrf_backward with grad_logZ = g (gradients of log Z) and then this call
+ * with grad_score = g and SEMICRF_FLAG_NEGATE_GRAD on the same output buffers.  The path-score part of the
+ * workspace is its own, so the call may sit between semicrf_forward and
+ * semicrf_backward.  (B, T, C, K) and the workspace are as for
+ * semicrf_forward; a length outside [0, T] sets SEMICRF_ERR_BAD_LENGTH.
+ * Deterministic: counts use integer atomics, every float sum a fixed order.
+ */
+SEMICRF_API int semicrf_path_score(const float *em, const int32_t *lengths, const float *trans,
+                                   const float *dur, const int32_t *labels,
+                                   const uint8_t *seg_start, int B, int T, int C, int K,
+                                   unsigned flags, void *ws, size_t ws_bytes,
+                                   const double *grad_score, double *score, float *grad_em,
+                                   float *grad_trans, float *grad_dur, semicrf_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the device status word of workspace

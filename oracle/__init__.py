@@ -64,6 +64,9 @@ def _load():
             lib.oracle_path_score.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
                                               ctypes.c_int, _ip, _u8p]
             lib.oracle_path_score.restype = ctypes.c_double
+            lib.oracle_path_counts.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, _ip, _u8p, _dp, _dp, _dp]
+            lib.oracle_path_counts.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -244,3 +247,37 @@ def path_score(em, lengths, trans, dur, labels, seg_start, K: int | None = None,
         out[b] = lib.oracle_path_score(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), int(center),
                                        _ptr(lab, _ip), _ptr(ss, _u8p))
     return out
+
+
+def path_counts(lengths, labels, seg_start, C: int, K: int, center: bool = True):
+    """Derivatives of the path score of given segmentations (float64).
+
+    Returns ``grad_em`` [B, T, C] (d score_b / d em[b, u, c], zero past L_b),
+    ``trans_count`` [B, C, C], ``dur_count`` [B, K, C] (per sequence, not
+    weighted) and ``valid`` [B] (False where the path is malformed; its
+    counts are zero).  Their weighted sums are the gold-score part of the
+    gradient of the loss log Z - score.
+    """
+    lib = _load()
+    labels = np.asarray(labels)
+    seg_start = np.asarray(seg_start)
+    B, T = labels.shape
+    grad_em = np.zeros((B, T, C))
+    tc = np.zeros((B, C, C))
+    dc = np.zeros((B, K, C))
+    valid = np.ones(B, dtype=bool)
+    for b in range(B):
+        L = int(lengths[b])
+        lab = np.ascontiguousarray(np.asarray(labels[b, :max(L, 1)], dtype=np.int32))
+        ss = np.ascontiguousarray(np.asarray(seg_start[b, :max(L, 1)], dtype=np.uint8))
+        de = np.zeros((max(L, 1), C))
+        dt = np.zeros((C, C))
+        dd = np.zeros((K, C))
+        rc = lib.oracle_path_counts(L, C, K, int(center), _ptr(lab, _ip), _ptr(ss, _u8p),
+                                    _ptr(de), _ptr(dt), _ptr(dd))
+        valid[b] = rc == 0
+        if L > 0:
+            grad_em[b, :L] = de[:L]
+        tc[b] = dt
+        dc[b] = dd
+    return dict(grad_em=grad_em, trans_count=tc, dur_count=dc, valid=valid)

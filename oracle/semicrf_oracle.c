@@ -388,3 +388,58 @@ double oracle_path_score(const double *e, int L, int C, int K, const double *tra
     free(et); free(nu);
     return total;
 }
+
+/*
+ * Derivatives of the path score above with respect to the parameters, for
+ * the training loss log Z - score(gold) ("Streaming Structured Inference with
+ * Flash-SemiCRF", explainer section 4, Correctness: training to the CRF loss).
+ * The score is linear in every parameter, so each derivative is a count read
+ * off the segmentation:
+ *   de[u, c]     = [labels[u] = c] - (centred ? n_c / L : 0), u < L,
+ *                  where n_c counts the positions labelled c (the second term
+ *                  is the derivative through the centring mean nu[c]);
+ *   dtrans[c',c] = number of consecutive segment pairs labelled c' then c;
+ *   ddur[k-1, c] = number of label-c segments of length k.
+ * The outputs are overwritten.  Returns 0, or -1 (outputs zero) if the
+ * segmentation is malformed in the sense of oracle_path_score.
+ */
+int oracle_path_counts(int L, int C, int K, int center, const int32_t *labels,
+                       const uint8_t *seg_start, double *de, double *dtrans, double *ddur)
+{
+    memset(dtrans, 0, sizeof(double) * (size_t)C * C);
+    memset(ddur, 0, sizeof(double) * (size_t)K * C);
+    if (L <= 0) return 0;
+    memset(de, 0, sizeof(double) * (size_t)L * C);
+    if (!seg_start[0]) return -1;
+    double *n = calloc((size_t)C, sizeof(double));
+    if (!n) return -1;
+    int prev = -1, s = 0, bad = 0;
+    while (s < L && !bad) {
+        const int c = labels[s];
+        if (c < 0 || c >= C) { bad = 1; break; }
+        int t = s + 1;
+        while (t < L && !seg_start[t]) {
+            if (labels[t] != c) { bad = 1; break; }
+            ++t;
+        }
+        if (bad || t - s > K) { bad = 1; break; }
+        for (int u = s; u < t; ++u) de[(size_t)u * C + c] += 1.0;
+        n[c] += (double)(t - s);
+        ddur[(size_t)(t - s - 1) * C + c] += 1.0;
+        if (prev >= 0) dtrans[(size_t)prev * C + c] += 1.0;
+        prev = c;
+        s = t;
+    }
+    if (bad) {
+        memset(de, 0, sizeof(double) * (size_t)L * C);
+        memset(dtrans, 0, sizeof(double) * (size_t)C * C);
+        memset(ddur, 0, sizeof(double) * (size_t)K * C);
+        free(n);
+        return -1;
+    }
+    if (center)
+        for (int u = 0; u < L; ++u)
+            for (int c = 0; c < C; ++c) de[(size_t)u * C + c] -= n[c] / (double)L;
+    free(n);
+    return 0;
+}

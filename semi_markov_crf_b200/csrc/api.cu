@@ -147,6 +147,7 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
   d.GS = 128;
   d.ngrid = T > 0 ? (T - 1) / d.GS + 2 : 1;  // positions 0, GS, 2GS, ... and L - 1
+  d.npch = std::max(1, (T + PATH_ROWS - 1) / PATH_ROWS);
   // Kernel shape: G lanes per label (a power of two), each with KBT durations
   // and CAT labels, picked from the instantiated menu by a latency model.
   // Per step about one warp runs per scheduler and the step is latency
@@ -234,6 +235,13 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_emax = take(B * 4);
   const size_t o_mode = take(2 * B * 4);
   const size_t o_tmax = take(4);
+  const size_t o_pcnt = take(B * (C * C + K * C) * 4);
+  const size_t o_psum = take(B * (size_t)d.npch * C * 8);
+  const size_t o_plab = take(B * (size_t)d.npch * C * 4);
+  const size_t o_pscr = take(B * (size_t)d.npch * 8);
+  const size_t o_pfr = take(B * C * 8);
+  const size_t o_pw = take(B * 8);
+  const size_t o_pbad = take(B * 4);
   if (base && p) {
     char* c = static_cast<char*>(base);
     p->status = reinterpret_cast<int*>(c + o_status);
@@ -261,12 +269,19 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->emax = reinterpret_cast<float*>(c + o_emax);
     p->mode = reinterpret_cast<int*>(c + o_mode);
     p->tmax = reinterpret_cast<float*>(c + o_tmax);
+    p->pcnt = reinterpret_cast<int32_t*>(c + o_pcnt);
+    p->psum = reinterpret_cast<double*>(c + o_psum);
+    p->plab = reinterpret_cast<int32_t*>(c + o_plab);
+    p->pscr = reinterpret_cast<double*>(c + o_pscr);
+    p->pfr = reinterpret_cast<double*>(c + o_pfr);
+    p->pw = reinterpret_cast<double*>(c + o_pw);
+    p->pbad = reinterpret_cast<int32_t*>(c + o_pbad);
   }
   return off;
 }
 
-constexpr unsigned KNOWN_FLAGS =
-    SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY | SEMICRF_FLAG_LOG_DOMAIN;
+constexpr unsigned KNOWN_FLAGS = SEMICRF_FLAG_NO_CENTER | SEMICRF_FLAG_FORWARD_ONLY |
+                                  SEMICRF_FLAG_LOG_DOMAIN | SEMICRF_FLAG_NEGATE_GRAD;
 
 int prepare(int B, int T, int C, int K, unsigned flags, void* ws, size_t ws_bytes, Dims& d,
             WsPtrs& p) {
@@ -589,6 +604,49 @@ extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const fl
   } else {
     ProfScope ps("viterbi_kernel", st);
     e = launch_viterbi(d, p, lengths, trans, dur, score, labels, seg_start, st);
+  }
+  return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
+}
+
+extern "C" int semicrf_path_score(const float* em, const int32_t* lengths, const float* trans,
+                                  const float* dur, const int32_t* labels,
+                                  const uint8_t* seg_start, int B, int T, int C, int K,
+                                  unsigned flags, void* ws, size_t ws_bytes,
+                                  const double* grad_score, double* score, float* grad_em,
+                                  float* grad_trans, float* grad_dur, semicrf_stream_t stream) {
+  if (!lengths || !trans || !dur || (B > 0 && T > 0 && (!em || !labels || !seg_start)))
+    return SEMICRF_ERR_INVALID_ARG;
+  Dims d;
+  WsPtrs p;
+  int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
+  if (rc) return rc;
+  if (B == 0) return SEMICRF_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned center = (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u;
+  const size_t ncnt = (size_t)B * ((size_t)C * C + (size_t)K * C);
+  if (cudaMemsetAsync(p.pcnt, 0, ncnt * sizeof(int32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(p.pbad, 0, (size_t)B * sizeof(int32_t), st) != cudaSuccess)
+    return SEMICRF_ERR_CUDA;
+  cudaError_t e;
+  {
+    ProfScope ps("path_terms_kernel", st);
+    e = launch_path_terms(d, p, em, lengths, trans, dur, labels, seg_start, center, st);
+  }
+  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+  {
+    ProfScope ps("path_final_kernel", st);
+    e = launch_path_final(d, p, lengths, center, grad_score,
+                          (flags & SEMICRF_FLAG_NEGATE_GRAD) ? 1 : 0, score, st);
+  }
+  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+  if (grad_em) {
+    ProfScope ps("path_grad_em_kernel", st);
+    e = launch_path_grad_em(d, p, lengths, labels, grad_em, sm_count(), st);
+  }
+  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+  if (grad_trans || grad_dur) {
+    ProfScope ps("path_grad_param_kernel", st);
+    e = launch_path_grad_param(d, p, grad_trans, grad_dur, st);
   }
   return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }

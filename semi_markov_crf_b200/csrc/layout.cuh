@@ -14,6 +14,7 @@ constexpr int KC_MAX = 16384;
 constexpr int NT_MAX = 512;  // threads per CTA
 constexpr int TS = 32;       // prefix-sum rows per TMA tile
 constexpr int FLUSH_EVERY = 64;  // positions between fp32 -> fp64 partial flushes
+constexpr int PATH_ROWS = 1024;  // positions per CTA of the path-score pass
 
 // Problem sizes and the lane mapping chosen for them.
 //
@@ -50,6 +51,7 @@ struct Dims {
   // GS positions, ngrid grid points per sequence; the posterior pass stages
   // pRT boundaries (plus K rows of halo) of kept values per tile.
   int GS, ngrid, pRT;
+  int npch;      // path-score chunks per sequence, ceil(T / PATH_ROWS)
 };
 
 // Device pointers into the caller's workspace.
@@ -80,6 +82,15 @@ struct WsPtrs {
   float* emax;     // [B] largest |centred emission| * log2(e) over the valid positions
   int* mode;       // [2][B] ring path per (direction, sequence): 1 exponential, 2 log domain
   float* tmax;     // [1] M = max trans * log2(e), written by the exponential-domain rings
+  // Path score (path.cu); a region of its own, so that it may run between a
+  // forward and its backward on the same workspace.
+  int32_t* pcnt;   // [B][C*C + K*C] gold transition then duration counts
+  double* psum;    // [B][npch][C] per-chunk emission column sums
+  int32_t* plab;   // [B][npch][C] per-chunk label counts
+  double* pscr;    // [B][npch] per-chunk sum of the gold terms
+  double* pfr;     // [B][C] n_c / L_b (0 without centering)
+  double* pw;      // [B] gradient weight (0 for a malformed path)
+  int32_t* pbad;   // [B] malformed-path bits
 };
 
 }  // namespace semicrf

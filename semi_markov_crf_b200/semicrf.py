@@ -13,7 +13,8 @@ import os
 
 import torch
 
-__all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "get_status",
+__all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "path_score",
+           "get_status", "FLAG_NEGATE_GRAD",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
            "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "ring_domains", "profile_enable", "profile_read",
            "forward_noalloc", "NOALLOC_SCRATCH_BYTES",
@@ -24,11 +25,13 @@ KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "ch
            "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
            "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
-           "viterbi_walk_kernel")
+           "viterbi_walk_kernel", "path_terms_kernel", "path_final_kernel", "path_grad_em_kernel",
+           "path_grad_param_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2
 FLAG_LOG_DOMAIN = 0x4
+FLAG_NEGATE_GRAD = 0x8
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SEMICRF_NOALLOC_SCRATCH_BYTES
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsemicrf_b200.so")
@@ -49,6 +52,8 @@ lib.semicrf_backward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _v
                                  _vp, _vp, _vp, _vp]
 lib.semicrf_viterbi.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp,
                                 _vp]
+lib.semicrf_path_score.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz,
+                                   _vp, _vp, _vp, _vp, _vp, _vp]
 lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
@@ -58,7 +63,7 @@ lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.P
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
 for _f in ("semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
-           "semicrf_backward", "semicrf_viterbi", "semicrf_get_status",
+           "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
            "semicrf_selftest_bounded_wait", "semicrf_ring_domains"):
     getattr(lib, _f).restype = _i
 
@@ -224,6 +229,49 @@ def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None =
                                ws.ptr, ws.nbytes, _ptr(score), _ptr(labels), _ptr(seg), _stream(dev)),
            "semicrf_viterbi")
     return score, labels, seg
+
+
+def path_score(em, lengths, trans, dur, labels, seg_start, center: bool = True,
+               ws: Workspace | None = None, grad_score=None, negate: bool = False,
+               grads: dict | None = None, score=None):
+    """Score [B] (float64) of given segmentations, NaN where malformed.
+
+    ``labels`` [B,T] int32 and ``seg_start`` [B,T] uint8 as :func:`viterbi`
+    returns them.  ``grads`` may hold any of grad_em [B,T,C], grad_trans
+    [C,C], grad_dur [K,C] (float32): w_b * d score_b / d x is ADDED into
+    them, w_b = grad_score[b] (float64 [B], None = ones), negated when
+    ``negate``.  For the NLL log Z - score: :func:`backward` with grad_logZ=g,
+    then this call with grad_score=g, negate=True and the same dict.  ``ws``
+    may be the workspace of a :func:`forward` with the same sizes (the path
+    score has a region of its own)."""
+    dev = em.device
+    _need(em, torch.float32, "em", dev)
+    _need(lengths, torch.int32, "lengths", dev)
+    _need(trans, torch.float32, "trans", dev)
+    _need(dur, torch.float32, "dur", dev)
+    _need(labels, torch.int32, "labels", dev)
+    _need(seg_start, torch.uint8, "seg_start", dev)
+    B, T, C = em.shape
+    K = dur.shape[0]
+    flags = _flags(center) | (FLAG_NEGATE_GRAD if negate else 0)
+    if ws is None or ws.dims != (B, T, C, K):
+        ws = Workspace(B, T, C, K, _flags(center), dev)
+    if grad_score is not None:
+        _need(grad_score, torch.float64, "grad_score", dev)
+    if score is None:
+        score = torch.empty(B, dtype=torch.float64, device=dev)
+    g = {} if grads is None else grads
+    for name, shape in (("grad_em", (B, T, C)), ("grad_trans", (C, C)), ("grad_dur", (K, C))):
+        if g.get(name) is not None:
+            _need(g[name], torch.float32, name, dev)
+            if tuple(g[name].shape) != shape:
+                raise TypeError(f"{name} must have shape {shape}")
+    _check(lib.semicrf_path_score(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), _ptr(labels),
+                                  _ptr(seg_start), B, T, C, K, flags, ws.ptr, ws.nbytes,
+                                  _ptr(grad_score), _ptr(score), _ptr(g.get("grad_em")),
+                                  _ptr(g.get("grad_trans")), _ptr(g.get("grad_dur")),
+                                  _stream(dev)), "semicrf_path_score")
+    return score
 
 
 def get_status(ws: Workspace) -> int:

@@ -84,6 +84,7 @@ def _draw(rng, w: Workload, B: int, T: int, K: int, C: int, pad_value):
         lengths = rng.integers(w.len_lo, T + 1, size=B).astype(np.int32)
     em = np.zeros((B, T, C), dtype=np.float32)
     gold = np.full((B, T), -1, dtype=np.int32)
+    gold_start = np.zeros((B, T), dtype=np.uint8)
     for b in range(B):
         L = int(lengths[b])
         if w.mode == "noise":
@@ -99,6 +100,7 @@ def _draw(rng, w: Workload, B: int, T: int, K: int, C: int, pad_value):
                 d = int(rng.geometric(1.0 / w.dur_mean))
                 d = min(d, K, L - pos)
                 labels[pos:pos + d] = c
+                gold_start[b, pos] = 1
                 pos += d
             noise = rng.standard_normal((L, C))
             x = noise
@@ -109,7 +111,8 @@ def _draw(rng, w: Workload, B: int, T: int, K: int, C: int, pad_value):
             em[b, L:] = pad_value
     trans = (w.param_std * rng.standard_normal((C, C))).astype(np.float32)
     dur = (w.param_std * rng.standard_normal((K, C))).astype(np.float32)
-    return dict(em=em, lengths=lengths, trans=trans, dur=dur, K=K, gold=gold)
+    return dict(em=em, lengths=lengths, trans=trans, dur=dur, K=K, gold=gold,
+                gold_start=gold_start)
 
 
 def make(name: str, pad_value=None, B: int | None = None, T: int | None = None,
@@ -121,7 +124,9 @@ def make(name: str, pad_value=None, B: int | None = None, T: int | None = None,
     to get oracle-sized cases of the same distribution.  Returns a dict with
     ``em`` [B,T,C] float32, ``lengths`` [B] int32, ``trans`` [C,C] float32
     (trans[c_prev, c]), ``dur`` [K,C] float32 (dur[k-1, c] scores duration
-    k), ``K`` and the generating segmentation ``gold`` [B,T] (-1 = padding).
+    k), ``K`` and the generating segmentation: labels ``gold`` [B,T] (-1 =
+    padding) and ``gold_start`` [B,T] uint8 (1 where a drawn segment starts;
+    two adjacent drawn segments may share a label).
     """
     w = CONFIGS[name]
     B_ = w.B if B is None else int(B)
@@ -158,6 +163,7 @@ def make_custom(B: int, T: int, K: int, C: int, seed: int, *, lengths=None,
             if L < T:
                 em[b, L:] = 0.0 if pad_value is None else pad_value
                 out["gold"][b, L:] = -1
+                out["gold_start"][b, L:] = 0
         out["lengths"] = lengths
     out["name"] = "custom"
     return out

@@ -97,3 +97,48 @@ def test_fullsize_viterbi_is_optimal(full):
                                  got["labels"], got["seg_start"], K=case["dur"].shape[0])
     assert np.all(np.isfinite(rescored))
     assert np.all(rescored >= best - LOGZ_RTOL * np.maximum(1.0, np.abs(best))), (rescored - best)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_fullsize_gold_path_score_and_counts(name):
+    """The path score of the generating segmentation (a random one for the
+    noise-only tiny workload) and the counts it adds to the gradients, at the
+    full size, against the oracle (cheap: one pass over the path)."""
+    from gpu_common import to_dev
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make(name)
+    B, T, C = case["em"].shape
+    K = case["dur"].shape[0]
+    labels, seg = case["gold"], case["gold_start"]
+    if not np.any(labels >= 0):
+        rng = np.random.default_rng(5)
+        labels = np.full((B, T), -1, dtype=np.int32)
+        seg = np.zeros((B, T), dtype=np.uint8)
+        for b, L in enumerate(case["lengths"]):
+            pos = 0
+            while pos < L:
+                d = int(rng.integers(1, min(K, L - pos) + 1))
+                labels[b, pos:pos + d] = rng.integers(0, C)
+                seg[b, pos] = 1
+                pos += d
+    em, lengths, trans, dur = to_dev(case)
+    grads = dict(grad_em=torch.zeros((B, T, C), dtype=torch.float32, device="cuda"),
+                 grad_trans=torch.zeros((C, C), dtype=torch.float32, device="cuda"),
+                 grad_dur=torch.zeros((K, C), dtype=torch.float32, device="cuda"))
+    g = np.linspace(-1.0, 2.0, B) if B > 1 else np.array([0.75])
+    score = semicrf.path_score(em, lengths, trans, dur, torch.from_numpy(labels).cuda(),
+                               torch.from_numpy(seg).cuda(),
+                               grad_score=torch.as_tensor(g, device="cuda"), grads=grads)
+    score = score.cpu().numpy()
+    ref = oracle.path_score(case["em"], case["lengths"], case["trans"], case["dur"], labels, seg, K)
+    assert np.all(np.isfinite(ref))
+    err = np.abs(score - ref) / np.maximum(1.0, np.abs(ref))
+    print(name, "path score rel err", err.max())
+    assert err.max() <= 1e-9
+    cnt = oracle.path_counts(case["lengths"], labels, seg, C, K)
+    e = float(np.max(np.abs(grads["grad_em"].cpu().numpy() - cnt["grad_em"] * g[:, None, None])))
+    assert e <= MARG_ATOL, e
+    for key, ck in (("grad_trans", "trans_count"), ("grad_dur", "dur_count")):
+        ref_c = np.einsum("b,bij->ij", g, cnt[ck])
+        d = np.abs(grads[key].cpu().numpy().astype(np.float64) - ref_c)
+        assert np.max(d / np.maximum(1.0, np.abs(ref_c))) <= COUNT_RTOL, key

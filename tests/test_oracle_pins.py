@@ -320,3 +320,114 @@ def test_synthetic_generator_is_reproducible_and_shaped():
     assert freq[0] > 0.4 and freq[5] < 0.1
     assert synth.checkpoint_interval(1_000_000, 200) == 14143
     assert synth.checkpoint_interval(800, 30) == 155
+
+
+# ------------------------------------------------------- path score and loss
+def _as_arrays(segs, L):
+    lab = np.full(L, -1, dtype=np.int32)
+    ss = np.zeros(L, dtype=np.uint8)
+    for (s, t, c) in segs:
+        lab[s:t] = c
+        ss[s] = 1
+    return lab, ss
+
+
+@pytest.mark.parametrize("L,K,C,center,seed", BRUTE_CASES[:4])
+def test_path_scores_of_all_segmentations_give_logZ_and_expected_counts(L, K, C, center, seed):
+    # log Z is the log-sum-exp of the scores of every segmentation, and the
+    # gradient of log Z is the posterior expectation of the path counts.
+    rng = np.random.default_rng(300 + seed)
+    em, lengths, trans, dur = _rand_case(rng, 1, L, K, C, pstd=0.7)
+    segs = list(brute.segmentations(L, K, C))
+    labs = np.stack([_as_arrays(sg, L)[0] for sg in segs])
+    sss = np.stack([_as_arrays(sg, L)[1] for sg in segs])
+    n = len(segs)
+    emb = np.repeat(em, n, axis=0)
+    scores = oracle.path_score(emb, np.full(n, L), trans, dur, labs, sss, K, center=center)
+    m = scores.max()
+    logZ = m + math.log(np.exp(scores - m).sum())
+    fb = oracle.forward_backward(em, lengths, trans, dur, K, center=center, threads=1)
+    assert abs(logZ - fb["logZ"][0]) < 1e-12 * max(1.0, abs(logZ))
+    cnt = oracle.path_counts(np.full(n, L), labs, sss, C, K, center=center)
+    assert cnt["valid"].all()
+    p = np.exp(scores - logZ)
+    assert np.max(np.abs(np.einsum("n,nij->ij", p, cnt["trans_count"]) - fb["grad_trans"])) < 1e-12
+    assert np.max(np.abs(np.einsum("n,nij->ij", p, cnt["dur_count"]) - fb["grad_dur"])) < 1e-12
+    assert np.max(np.abs(np.einsum("n,nuc->uc", p, cnt["grad_em"][:, :L])
+                         - fb["grad_e"][0, :L])) < 1e-12
+
+
+def _random_path(rng, L, K, C):
+    lab = np.empty(L, dtype=np.int32)
+    ss = np.zeros(L, dtype=np.uint8)
+    pos = 0
+    while pos < L:
+        d = int(rng.integers(1, min(K, L - pos) + 1))
+        lab[pos:pos + d] = rng.integers(0, C)
+        ss[pos] = 1
+        pos += d
+    return lab, ss
+
+
+@pytest.mark.parametrize("center", [True, False])
+def test_path_counts_are_the_finite_differences_of_the_path_score(center):
+    # The path score is linear in em, trans and dur, so a central difference
+    # with a large step is exact up to rounding.
+    rng = np.random.default_rng(311)
+    T, K, C = 17, 5, 4
+    em, lengths, trans, dur = _rand_case(rng, 1, T, K, C, lengths=[14])
+    lab, ss = _random_path(rng, 14, K, C)
+    labels = np.full((1, T), -1, dtype=np.int32); labels[0, :14] = lab
+    seg = np.zeros((1, T), dtype=np.uint8); seg[0, :14] = ss
+    cnt = oracle.path_counts(lengths, labels, seg, C, K, center=center)
+    h = 0.25
+
+    def sc(e=em, t=trans, d=dur):
+        return oracle.path_score(e, lengths, t, d, labels, seg, K, center=center)[0]
+
+    for (u, c) in [(0, 0), (3, 1), (7, 2), (13, 3), (10, 0)]:
+        ep, emn = em.copy(), em.copy()
+        ep[0, u, c] += h; emn[0, u, c] -= h
+        assert abs((sc(e=ep) - sc(e=emn)) / (2 * h) - cnt["grad_em"][0, u, c]) < 1e-9
+    for (a, c) in [(0, 1), (2, 3), (1, 1), (3, 0)]:
+        tp, tm = trans.copy(), trans.copy()
+        tp[a, c] += h; tm[a, c] -= h
+        assert abs((sc(t=tp) - sc(t=tm)) / (2 * h) - cnt["trans_count"][0, a, c]) < 1e-9
+    for (k, c) in [(0, 0), (1, 2), (4, 3), (2, 1)]:
+        dp, dm = dur.copy(), dur.copy()
+        dp[k, c] += h; dm[k, c] -= h
+        assert abs((sc(d=dp) - sc(d=dm)) / (2 * h) - cnt["dur_count"][0, k, c]) < 1e-9
+    # the rows past L_b carry no gradient
+    assert np.all(cnt["grad_em"][0, 14:] == 0)
+
+
+def test_path_counts_reject_what_the_path_score_rejects():
+    rng = np.random.default_rng(312)
+    T, K, C = 12, 3, 3
+    em, lengths, trans, dur = _rand_case(rng, 1, T, K, C)
+    lab, ss = _random_path(rng, T, K, C)
+    cases = []
+    s0 = ss.copy(); s0[0] = 0; cases.append((lab, s0))            # no start at 0
+    l1 = lab.copy(); l1[5] = C; cases.append((l1, ss))             # label out of range
+    one = np.zeros(T, dtype=np.uint8); one[0] = 1                  # one segment longer than K
+    cases.append((np.zeros(T, dtype=np.int32), one))
+    for (a, s) in cases:
+        out = oracle.path_counts(lengths, a[None], s[None], C, K)
+        assert not out["valid"][0] and np.all(out["trans_count"] == 0)
+        assert math.isnan(oracle.path_score(em, lengths, trans, dur, a[None], s[None], K)[0])
+    ok = oracle.path_counts(lengths, lab[None], ss[None], C, K)
+    assert ok["valid"][0]
+    # segments - transitions = 1; durations sum to L; centred emission rows sum to 0
+    assert ok["dur_count"].sum() - ok["trans_count"].sum() == 1
+    assert (ok["dur_count"][0] * np.arange(1, K + 1)[:, None]).sum() == T
+    assert np.max(np.abs(ok["grad_em"][0].sum(axis=1))) < 1e-12
+
+
+def test_gold_segmentation_of_the_generator_is_a_valid_path():
+    w = synth.make("genomic", B=2, T=3000)
+    cnt = oracle.path_counts(w["lengths"], w["gold"], w["gold_start"], 6, w["K"])
+    assert cnt["valid"].all()
+    nll = (oracle.log_partition(w["em"], w["lengths"], w["trans"], w["dur"], w["K"])
+           - oracle.path_score(w["em"], w["lengths"], w["trans"], w["dur"], w["gold"],
+                               w["gold_start"], w["K"]))
+    assert np.all(nll > 0)

@@ -429,8 +429,7 @@ def run_ours(args):
     semicrf.profile_enable(False)
     nll_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(n_s, n_e)), dev) / args.steps
     nll_kern = {}
-    for name in ("path_terms_kernel", "path_final_kernel", "path_grad_em_kernel",
-                 "path_grad_param_kernel"):
+    for name in ("path_terms_kernel", "path_grad_kernel"):
         tot, n = semicrf.profile_read(name)
         if n:
             nll_kern[name] = {"ms_total": tot, "launches": n, "ms_per_launch": tot / n}
@@ -527,9 +526,10 @@ def run_ours(args):
         }
         # algorithmic bytes per position: the terms pass reads the emission
         # row (4C, for nu), the label (4) and the start flag (1); the
-        # emission-gradient pass reads and writes its row (8C) and the label
+        # gradient pass reads and writes the emission-gradient row (8C) and
+        # reads the label (4); the count tables are O(C^2 + KC) per sequence
         nll_bytes = {"path_terms_kernel": (4 * C + 5) * positions,
-                     "path_grad_em_kernel": (8 * C + 4) * positions}
+                     "path_grad_kernel": (8 * C + 4) * positions}
         nll_roofs = {}
         for k, nb in nll_bytes.items():
             if k in nll_kern:

@@ -235,13 +235,13 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_emax = take(B * 4);
   const size_t o_mode = take(2 * B * 4);
   const size_t o_tmax = take(4);
-  const size_t o_pcnt = take(B * (C * C + K * C) * 4);
+  const size_t pz = (B * (C * C + K * C) + 2 * B) * 4;  // pcnt | pbad | pdone
+  const size_t o_pcnt = take(pz);
   const size_t o_psum = take(B * (size_t)d.npch * C * 8);
   const size_t o_plab = take(B * (size_t)d.npch * C * 4);
   const size_t o_pscr = take(B * (size_t)d.npch * 8);
   const size_t o_pfr = take(B * C * 8);
   const size_t o_pw = take(B * 8);
-  const size_t o_pbad = take(B * 4);
   if (base && p) {
     char* c = static_cast<char*>(base);
     p->status = reinterpret_cast<int*>(c + o_status);
@@ -275,7 +275,9 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->pscr = reinterpret_cast<double*>(c + o_pscr);
     p->pfr = reinterpret_cast<double*>(c + o_pfr);
     p->pw = reinterpret_cast<double*>(c + o_pw);
-    p->pbad = reinterpret_cast<int32_t*>(c + o_pbad);
+    p->pbad = p->pcnt + B * (C * C + K * C);
+    p->pdone = p->pbad + B;
+    p->pzero_bytes = pz;
   }
   return off;
 }
@@ -623,30 +625,17 @@ extern "C" int semicrf_path_score(const float* em, const int32_t* lengths, const
   if (B == 0) return SEMICRF_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const unsigned center = (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u;
-  const size_t ncnt = (size_t)B * ((size_t)C * C + (size_t)K * C);
-  if (cudaMemsetAsync(p.pcnt, 0, ncnt * sizeof(int32_t), st) != cudaSuccess ||
-      cudaMemsetAsync(p.pbad, 0, (size_t)B * sizeof(int32_t), st) != cudaSuccess)
-    return SEMICRF_ERR_CUDA;
+  if (cudaMemsetAsync(p.pcnt, 0, p.pzero_bytes, st) != cudaSuccess) return SEMICRF_ERR_CUDA;
   cudaError_t e;
   {
     ProfScope ps("path_terms_kernel", st);
-    e = launch_path_terms(d, p, em, lengths, trans, dur, labels, seg_start, center, st);
-  }
-  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
-  {
-    ProfScope ps("path_final_kernel", st);
-    e = launch_path_final(d, p, lengths, center, grad_score,
+    e = launch_path_terms(d, p, em, lengths, trans, dur, labels, seg_start, center, grad_score,
                           (flags & SEMICRF_FLAG_NEGATE_GRAD) ? 1 : 0, score, st);
   }
   if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
-  if (grad_em) {
-    ProfScope ps("path_grad_em_kernel", st);
-    e = launch_path_grad_em(d, p, lengths, labels, grad_em, sm_count(), st);
-  }
-  if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
-  if (grad_trans || grad_dur) {
-    ProfScope ps("path_grad_param_kernel", st);
-    e = launch_path_grad_param(d, p, grad_trans, grad_dur, st);
+  if (grad_em || grad_trans || grad_dur) {
+    ProfScope ps("path_grad_kernel", st);
+    e = launch_path_grad(d, p, lengths, labels, grad_em, grad_trans, grad_dur, st);
   }
   return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }

@@ -129,17 +129,15 @@ cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* len
                              int n_beta, cudaStream_t st);
 
 // Score of given segmentations and its gradient (path.cu).  The caller zeroes
-// ws.pcnt and ws.pbad first.
+// the ws.pzero_bytes region at ws.pcnt first.  The terms pass writes score[b]
+// (nullable) and the weights; the gradient pass adds into the non-null outputs.
 cudaError_t launch_path_terms(const Dims& d, const WsPtrs& ws, const float* em,
                               const int32_t* lengths, const float* trans, const float* dur,
                               const int32_t* labels, const uint8_t* seg_start, unsigned center,
+                              const double* grad_score, int negate, double* score,
                               cudaStream_t st);
-cudaError_t launch_path_final(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                              unsigned center, const double* grad_score, int negate,
-                              double* score, cudaStream_t st);
-cudaError_t launch_path_grad_em(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                                const int32_t* labels, float* grad_em, int sms, cudaStream_t st);
-cudaError_t launch_path_grad_param(const Dims& d, const WsPtrs& ws, float* grad_trans,
-                                   float* grad_dur, cudaStream_t st);
+cudaError_t launch_path_grad(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const int32_t* labels, float* grad_em, float* grad_trans,
+                             float* grad_dur, cudaStream_t st);
 
 }  // namespace semicrf

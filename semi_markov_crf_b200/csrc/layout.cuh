@@ -14,7 +14,7 @@ constexpr int KC_MAX = 16384;
 constexpr int NT_MAX = 512;  // threads per CTA
 constexpr int TS = 32;       // prefix-sum rows per TMA tile
 constexpr int FLUSH_EVERY = 64;  // positions between fp32 -> fp64 partial flushes
-constexpr int PATH_ROWS = 1024;  // positions per CTA of the path-score pass
+constexpr int PATH_ROWS = 256;  // positions per CTA of the path-score pass (one per thread)
 
 // Problem sizes and the lane mapping chosen for them.
 //
@@ -84,6 +84,8 @@ struct WsPtrs {
   float* tmax;     // [1] M = max trans * log2(e), written by the exponential-domain rings
   // Path score (path.cu); a region of its own, so that it may run between a
   // forward and its backward on the same workspace.
+  // pcnt, pbad and pdone are one contiguous region, zeroed by one memset
+  // before every call (pzero_bytes).
   int32_t* pcnt;   // [B][C*C + K*C] gold transition then duration counts
   double* psum;    // [B][npch][C] per-chunk emission column sums
   int32_t* plab;   // [B][npch][C] per-chunk label counts
@@ -91,6 +93,8 @@ struct WsPtrs {
   double* pfr;     // [B][C] n_c / L_b (0 without centering)
   double* pw;      // [B] gradient weight (0 for a malformed path)
   int32_t* pbad;   // [B] malformed-path bits
+  int32_t* pdone;  // [B] chunks of the sequence finished (the last one reduces)
+  size_t pzero_bytes;
 };
 
 }  // namespace semicrf

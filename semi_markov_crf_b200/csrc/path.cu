@@ -19,17 +19,19 @@
 // The path comes as two per-position arrays, the form the decoder writes:
 // labels[b, u] (int32) and seg_start[b, u] (1 where a segment starts).
 //
-// Three passes, each coalesced over positions:
-//   path_terms_kernel  one CTA per (chunk of PATH_ROWS positions, sequence):
-//                      the chunk's emission column sums (for nu), its gold
-//                      emission, duration and transition terms, its label
-//                      counts, and the gold duration / transition counts,
-//                      added to per-sequence int32 tables by integer atomics
-//                      (exact, so their order does not matter);
-//   path_final_kernel  one CTA per sequence: nu, the centred score, n_c / L;
-//   path_grad_*        grad += w_b * d score_b / d x for the emissions and
-//                      for the transition / duration tables (summed over b in
-//                      a fixed order).
+// Two launches, each coalesced over positions:
+//   path_terms_kernel  one CTA per (chunk of PATH_ROWS positions, sequence),
+//                      one position per thread: the chunk's emission column
+//                      sums (for nu), its gold emission, duration and
+//                      transition terms and its label counts; the gold
+//                      duration / transition counts go to per-sequence int32
+//                      tables by integer atomics (exact, so their order does
+//                      not matter).  The last CTA of a sequence to finish
+//                      (a per-sequence counter) reduces the chunks in order:
+//                      nu, the centred score, n_c / L and the weight w_b.
+//   path_grad_kernel   grad += w_b * d score_b / d x: the emission gradient
+//                      element by element, the transition / duration tables
+//                      summed over b in a fixed order (the last CTAs).
 // Every floating-point sum runs in float64 in a fixed order.
 #include "kernels.cuh"
 
@@ -64,212 +66,209 @@ __global__ void __launch_bounds__(PT_THREADS) path_terms_kernel(
     const float* __restrict__ em, const int32_t* __restrict__ lengths,
     const float* __restrict__ trans, const float* __restrict__ dur,
     const int32_t* __restrict__ labels, const uint8_t* __restrict__ seg_start, Dims d,
-    WsPtrs ws, unsigned center) {
-  const int b = blockIdx.y, j = blockIdx.x;
+    WsPtrs ws, unsigned center, const double* __restrict__ grad_score, int negate,
+    double* __restrict__ score) {
+  const int b = blockIdx.y, j = blockIdx.x, tid = threadIdx.x;
   const int C = d.C, K = d.K, T = d.T;
-  int L = lengths[b];
-  if (L < 0 || L > T) {
-    if (j == 0 && threadIdx.x == 0) {
-      set_status(ws.status, ST_BAD_LENGTH);
-      atomicOr(ws.pbad + b, PB_LEN);
+  const int L = lengths[b];
+  const double g = (grad_score ? grad_score[b] : 1.0) * (negate ? -1.0 : 1.0);
+  if (L <= 0 || L > T) {
+    // Nothing to sum: chunk 0 alone reports the sequence.
+    if (j == 0 && tid == 0) {
+      const bool bad = L != 0;
+      if (bad) set_status(ws.status, ST_BAD_LENGTH);
+      if (score) score[b] = bad ? __longlong_as_double(0x7ff8000000000000ll) : 0.0;
+      ws.pw[b] = bad ? 0.0 : g;
     }
     return;
   }
   const int u0 = j * PATH_ROWS;
   if (u0 >= L) return;
   const int u1 = min(u0 + PATH_ROWS, L);
+  const int nchb = (L + PATH_ROWS - 1) / PATH_ROWS;
 
   __shared__ double part[PT_THREADS];
   __shared__ double red[PT_THREADS / 32];
   __shared__ int cnt[C_MAX];
-  for (int c = threadIdx.x; c < C; c += PT_THREADS) cnt[c] = 0;
+  __shared__ unsigned char fl[PATH_ROWS + K_MAX];  // start flags of [u0, u0 + PATH_ROWS + K)
+  __shared__ int last;
 
   const float* eb = em + (size_t)b * T * C;
   const int32_t* yb = labels + (size_t)b * T;
   const uint8_t* sb = seg_start + (size_t)b * T;
 
+  for (int c = tid; c < C; c += PT_THREADS) cnt[c] = 0;
+  const int nfl = min(PATH_ROWS + K, L - u0);
+  for (int q = tid; q < nfl; q += PT_THREADS) fl[q] = sb[u0 + q];
+
   // Emission column sums of the chunk: thread (g, c) sums rows u0+g, u0+g+G, ...
+  double es = 0.0;
   if (center) {
     const int G = PT_THREADS / C;
-    const int g = threadIdx.x / C, c = threadIdx.x % C;
-    double acc = 0.0;
-    if (g < G)
-      for (int u = u0 + g; u < u1; u += G) acc += (double)eb[(size_t)u * C + c];
-    part[threadIdx.x] = acc;
+    const int gi = tid / C, c = tid - (tid / C) * C;
+    if (gi < G) {
+      const float* col = eb + c;
+      // independent loads, many in flight: the chain is one add per row
+#pragma unroll 16
+      for (int u = u0 + gi; u < u1; u += G) es += (double)col[(size_t)u * C];
+    }
   }
-  __syncthreads();  // part[] ready, cnt[] zeroed
-  if (center && threadIdx.x < C) {
-    const int G = PT_THREADS / C;
-    double s = 0.0;
-    for (int g = 0; g < G; ++g) s += part[g * C + threadIdx.x];
-    ws.psum[((size_t)b * d.npch + j) * C + threadIdx.x] = s;
-  }
+  part[tid] = es;
 
-  // Gold terms, one position per thread and pass.
+  // The gold terms of position u = u0 + tid.
   int* cnt_t = ws.pcnt + (size_t)b * (C * C + K * C);
   int* cnt_d = cnt_t + C * C;
+  const int u = u0 + tid;
   double acc = 0.0;
   int bad = 0;
-  for (int u = u0 + threadIdx.x; u < u1; u += PT_THREADS) {
-    const int y = yb[u];
-    const bool st = sb[u] != 0;
+  int y = -1, yp = -1;
+  if (u < u1) {
+    y = yb[u];
+    if (u > 0) yp = yb[u - 1];
+  }
+  __syncthreads();  // fl[], cnt[] and part[] ready
+  if (u < u1) {
+    const bool st = fl[tid] != 0;
     if (y < 0 || y >= C) {
       bad |= PB_LABEL;
-      continue;
-    }
-    if (u == 0 && !st) bad |= PB_START;
-    if (u > 0 && !st && yb[u - 1] != y) bad |= PB_CHANGE;
-    acc += (double)eb[(size_t)u * C + y];
-    atomicAdd(&cnt[y], 1);
-    if (st) {
-      // Duration: distance to the next start, or to the end of the sequence.
-      int k = 0;
-      for (int q = 1; q <= K; ++q) {
-        if (u + q >= L || sb[u + q]) {
-          k = q;
-          break;
+    } else {
+      if (u == 0 && !st) bad |= PB_START;
+      if (u > 0 && !st && yp != y) bad |= PB_CHANGE;
+      acc = (double)eb[(size_t)u * C + y];
+      atomicAdd(&cnt[y], 1);
+      if (st) {
+        // Duration: distance to the next start, or to the end of the sequence.
+        int k = 0;
+        for (int q = 1; q <= K; ++q) {
+          if (u + q >= L || fl[tid + q]) {
+            k = q;
+            break;
+          }
         }
-      }
-      if (k == 0) {
-        bad |= PB_LONG;
-        continue;
-      }
-      acc += (double)dur[(k - 1) * C + y];
-      atomicAdd(cnt_d + (k - 1) * C + y, 1);
-      if (u > 0) {
-        const int yp = yb[u - 1];
-        if (yp >= 0 && yp < C) {
-          acc += (double)trans[yp * C + y];
-          atomicAdd(cnt_t + yp * C + y, 1);
+        if (k == 0) {
+          bad |= PB_LONG;
+        } else {
+          acc += (double)dur[(k - 1) * C + y];
+          atomicAdd(cnt_d + (k - 1) * C + y, 1);
+          if (u > 0 && yp >= 0 && yp < C) {
+            acc += (double)trans[yp * C + y];
+            atomicAdd(cnt_t + yp * C + y, 1);
+          }
         }
       }
     }
   }
   if (bad) atomicOr(ws.pbad + b, bad);
+  if (center && tid < C) {
+    const int G = PT_THREADS / C;
+    double s = 0.0;
+    for (int gi = 0; gi < G; ++gi) s += part[gi * C + tid];
+    ws.psum[((size_t)b * d.npch + j) * C + tid] = s;
+  }
   const double tot = block_sum_fixed(acc, red);
   __syncthreads();  // cnt[] complete
-  if (threadIdx.x == 0) ws.pscr[(size_t)b * d.npch + j] = tot;
-  for (int c = threadIdx.x; c < C; c += PT_THREADS)
-    ws.plab[((size_t)b * d.npch + j) * C + c] = cnt[c];
-}
+  if (tid == 0) ws.pscr[(size_t)b * d.npch + j] = tot;
+  for (int c = tid; c < C; c += PT_THREADS) ws.plab[((size_t)b * d.npch + j) * C + c] = cnt[c];
 
-// One CTA per sequence: nu[c] = (sum of the chunk column sums) / L, the score
-// sum_chunks(partial) - sum_c n_c nu[c], the fractions n_c / L for the
-// emission gradient and the weight w_b = +-grad_score[b] (0 for a malformed
-// path).
-__global__ void __launch_bounds__(C_MAX) path_final_kernel(const int32_t* __restrict__ lengths,
-                                                           Dims d, WsPtrs ws, unsigned center,
-                                                           const double* __restrict__ grad_score,
-                                                           int negate, double* __restrict__ score) {
-  const int b = blockIdx.x, C = d.C;
-  __shared__ double corr[C_MAX];
-  const int bad = ws.pbad[b];
-  int L = lengths[b];
-  if (L < 0 || L > d.T) L = 0;
-  const int nch = (L + PATH_ROWS - 1) / PATH_ROWS;
-  const int c = threadIdx.x;
-  double cr = 0.0;
-  if (c < C) {
-    double es = 0.0;
-    long long n = 0;
-    for (int j = 0; j < nch; ++j) {
-      const size_t o = ((size_t)b * d.npch + j) * C + c;
-      if (center) es += ws.psum[o];
-      n += ws.plab[o];
-    }
-    const double nu = (center && L > 0) ? es / (double)L : 0.0;
-    cr = (double)n * nu;
-    ws.pfr[(size_t)b * C + c] = (center && L > 0) ? (double)n / (double)L : 0.0;
-  }
-  corr[c] = cr;
+  // The last chunk of the sequence to finish reduces all of them.
+  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int j = 0; j < nch; ++j) s += ws.pscr[(size_t)b * d.npch + j];
-    for (int cc = 0; cc < C; ++cc) s -= corr[cc];
-    double g = grad_score ? grad_score[b] : 1.0;
-    if (negate) g = -g;
-    if (bad) {
-      if (score) score[b] = __longlong_as_double(0x7ff8000000000000ll);  // NaN
-      ws.pw[b] = 0.0;
-    } else {
-      if (score) score[b] = s;
-      ws.pw[b] = g;
+  if (tid == 0) last = (atomicAdd(ws.pdone + b, 1) == nchb - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  double cr = 0.0;
+  if (tid < C) {
+    double e = 0.0;
+    long long n = 0;
+    for (int jj = 0; jj < nchb; ++jj) {
+      const size_t o = ((size_t)b * d.npch + jj) * C + tid;
+      if (center) e += __ldcg(ws.psum + o);
+      n += __ldcg(ws.plab + o);
     }
+    cr = center ? (double)n * (e / (double)L) : 0.0;
+    ws.pfr[(size_t)b * C + tid] = center ? (double)n / (double)L : 0.0;
+  }
+  part[tid] = cr;
+  __syncthreads();
+  if (tid == 0) {
+    double sc = 0.0;
+    for (int jj = 0; jj < nchb; ++jj) sc += __ldcg(ws.pscr + (size_t)b * d.npch + jj);
+    for (int c = 0; c < C; ++c) sc -= part[c];
+    const int anybad = __ldcg(ws.pbad + b);
+    if (score) score[b] = anybad ? __longlong_as_double(0x7ff8000000000000ll) : sc;
+    ws.pw[b] = anybad ? 0.0 : g;
   }
 }
 
-// grad_em[b, u, c] += w_b * ([y_u = c] - n_c / L) for u < L_b.
-__global__ void __launch_bounds__(PT_THREADS) path_grad_em_kernel(
+// grad_em[b, u, c] += w_b * ([y_u = c] - n_c / L) for u < L_b, four elements
+// per thread (blocks [0, nbe)); then grad_trans[c', c] += sum_b w_b *
+// (#c' -> c transitions of path b) and grad_dur[k-1, c] += sum_b w_b *
+// (#label-c segments of length k) in a fixed order (blocks [nbe, gridDim.x)).
+__global__ void __launch_bounds__(PT_THREADS) path_grad_kernel(
     const int32_t* __restrict__ lengths, const int32_t* __restrict__ labels, Dims d, WsPtrs ws,
-    float* __restrict__ grad_em) {
-  const int b = blockIdx.y, C = d.C;
-  const double w = ws.pw[b];
-  if (w == 0.0) return;
-  int L = lengths[b];
-  if (L < 0 || L > d.T) return;
-  const size_t n = (size_t)L * C;
-  const int32_t* yb = labels + (size_t)b * d.T;
-  const double* fr = ws.pfr + (size_t)b * C;
-  float* gb = grad_em + (size_t)b * d.T * C;
-  for (size_t i = (size_t)blockIdx.x * PT_THREADS + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * PT_THREADS) {
-    const int u = (int)(i / C), c = (int)(i - (size_t)u * C);
-    const double v = ((yb[u] == c) ? 1.0 : 0.0) - fr[c];
-    gb[i] += (float)(w * v);
+    float* __restrict__ grad_em, float* __restrict__ grad_trans, float* __restrict__ grad_dur,
+    int nbe) {
+  const int C = d.C, K = d.K, T = d.T;
+  if ((int)blockIdx.x < nbe) {
+    const size_t per_seq = (size_t)T * C;
+    const size_t base = (size_t)blockIdx.x * (4 * PT_THREADS) + threadIdx.x;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const size_t i = base + (size_t)q * PT_THREADS;
+      if (i >= (size_t)d.B * per_seq) break;
+      const int b = (int)(i / per_seq);
+      const size_t r = i - (size_t)b * per_seq;
+      const int u = (int)(r / C), c = (int)(r - (size_t)u * C);
+      const int L = __ldg(lengths + b);
+      const double w = ws.pw[b];
+      if (u >= L || w == 0.0) continue;
+      const double v = ((labels[(size_t)b * T + u] == c) ? 1.0 : 0.0) - ws.pfr[(size_t)b * C + c];
+      grad_em[i] += (float)(w * v);
+    }
+    return;
   }
-}
-
-// grad_trans[c', c] += sum_b w_b * (#c' -> c transitions of path b) and
-// grad_dur[k-1, c] += sum_b w_b * (#label-c segments of length k), b in order.
-__global__ void __launch_bounds__(PT_THREADS) path_grad_param_kernel(Dims d, WsPtrs ws,
-                                                                     float* __restrict__ grad_trans,
-                                                                     float* __restrict__ grad_dur) {
-  const int C = d.C, K = d.K;
+  // Count tables: 32 entries per block, the 8 warps take every 8th sequence
+  // and their sums are added in warp order.
+  __shared__ double ps[PT_THREADS / 32][32];
   const int nt = C * C, nall = C * C + K * C;
-  const int i = blockIdx.x * PT_THREADS + threadIdx.x;
-  if (i >= nall) return;
-  float* out = (i < nt) ? grad_trans : grad_dur;
-  if (!out) return;
+  const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
+  const int i = (blockIdx.x - nbe) * 32 + lane;
   double s = 0.0;
-  for (int b = 0; b < d.B; ++b) {
-    const int v = ws.pcnt[(size_t)b * nall + i];
-    if (v) s += ws.pw[b] * (double)v;
+  if (i < nall)
+#pragma unroll 4
+    for (int b = wg; b < d.B; b += PT_THREADS / 32)
+      s += ws.pw[b] * (double)ws.pcnt[(size_t)b * nall + i];
+  ps[wg][lane] = s;
+  __syncthreads();
+  if (wg == 0 && i < nall) {
+    double t = 0.0;
+    for (int w = 0; w < PT_THREADS / 32; ++w) t += ps[w][lane];
+    float* out = (i < nt) ? grad_trans : grad_dur;
+    if (out) out[i < nt ? i : i - nt] += (float)t;
   }
-  out[i < nt ? i : i - nt] += (float)s;
 }
 
 cudaError_t launch_path_terms(const Dims& d, const WsPtrs& ws, const float* em,
                               const int32_t* lengths, const float* trans, const float* dur,
                               const int32_t* labels, const uint8_t* seg_start, unsigned center,
+                              const double* grad_score, int negate, double* score,
                               cudaStream_t st) {
-  path_terms_kernel<<<dim3(d.npch, d.B), PT_THREADS, 0, st>>>(em, lengths, trans, dur, labels,
-                                                               seg_start, d, ws, center);
+  path_terms_kernel<<<dim3(d.npch, d.B), PT_THREADS, 0, st>>>(
+      em, lengths, trans, dur, labels, seg_start, d, ws, center, grad_score, negate, score);
   return cudaGetLastError();
 }
 
-cudaError_t launch_path_final(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                              unsigned center, const double* grad_score, int negate,
-                              double* score, cudaStream_t st) {
-  path_final_kernel<<<d.B, C_MAX, 0, st>>>(lengths, d, ws, center, grad_score, negate, score);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_path_grad_em(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                                const int32_t* labels, float* grad_em, int sms, cudaStream_t st) {
-  // At most about four waves of 2048 threads per SM over the whole batch.
-  const size_t per_seq_full = ((size_t)d.T * d.C + PT_THREADS - 1) / PT_THREADS;
-  const size_t cap = (size_t)std::max(1, 4 * 8 * sms / std::max(d.B, 1));
-  const int per_seq = (int)std::max<size_t>(1, std::min(per_seq_full, cap));
-  path_grad_em_kernel<<<dim3(per_seq, d.B), PT_THREADS, 0, st>>>(lengths, labels, d, ws, grad_em);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_path_grad_param(const Dims& d, const WsPtrs& ws, float* grad_trans,
-                                   float* grad_dur, cudaStream_t st) {
+cudaError_t launch_path_grad(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                             const int32_t* labels, float* grad_em, float* grad_trans,
+                             float* grad_dur, cudaStream_t st) {
+  const size_t nem = (size_t)d.B * d.T * d.C;
+  const int nbe = grad_em ? (int)((nem + 4 * PT_THREADS - 1) / (4 * PT_THREADS)) : 0;
   const int nall = d.C * d.C + d.K * d.C;
-  path_grad_param_kernel<<<(nall + PT_THREADS - 1) / PT_THREADS, PT_THREADS, 0, st>>>(
-      d, ws, grad_trans, grad_dur);
+  const int nbp = (grad_trans || grad_dur) ? (nall + 31) / 32 : 0;
+  if (nbe + nbp == 0) return cudaSuccess;
+  path_grad_kernel<<<nbe + nbp, PT_THREADS, 0, st>>>(lengths, labels, d, ws, grad_em, grad_trans,
+                                                     grad_dur, nbe);
   return cudaGetLastError();
 }
 

@@ -25,8 +25,7 @@ KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "ch
            "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
            "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
-           "viterbi_walk_kernel", "path_terms_kernel", "path_final_kernel", "path_grad_em_kernel",
-           "path_grad_param_kernel")
+           "viterbi_walk_kernel", "path_terms_kernel", "path_grad_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2

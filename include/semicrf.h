@@ -43,8 +43,10 @@
  *    a bounded wait that gave up) are recorded in the workspace status word,
  *    read with semicrf_get_status.
  *  - Limits of this build: 1 <= C <= 128, T <= 2^26, B <= 2^20, and
- *    K <= 512 (C <= 16), K <= 256 (C <= 32), K <= 128 (C <= 64),
- *    K <= 64 (C <= 128).  Larger values return SEMICRF_ERR_UNSUPPORTED.
+ *    K <= 2048 (C <= 8), K <= 512 (C <= 16), K <= 256 (C <= 32),
+ *    K <= 128 (C <= 64), K <= 64 (C <= 128).  Larger values return
+ *    SEMICRF_ERR_UNSUPPORTED.  (Durations up to K = 2000 on sequences of
+ *    10^6 positions are the pages' genomic regime, explainer section 4.)
  *  - Numbers are computed in float32 in base-2 log units with exactly
  *    representable integer frames and float64 normalisers; results are
  *    deterministic (no floating-point atomics).

@@ -85,14 +85,16 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
 
 // Every kernel shape the library instantiates: (durations per lane KBT,
 // labels per lane CAT, lanes per label G, launch bound LB).  The (16, 32, G,
-// 512) family alone covers every supported size; the others are tuned for
-// smaller problems (fewer wasted terms, fewer registers).
+// 512) family alone covers every size with K <= 512; the others are tuned for
+// smaller problems (fewer wasted terms, fewer registers), and (64, 1, 32, 256)
+// takes long durations, K <= 2048 with C <= 8.
 #define SEMICRF_FOR_EACH_SHAPE(X)                                                        \
   X(4, 4, 1, 256) X(8, 4, 1, 256) X(4, 8, 1, 256) X(8, 8, 1, 256) X(16, 8, 1, 256)       \
   X(16, 32, 1, 256) X(4, 4, 2, 256) X(8, 8, 2, 256) X(16, 32, 2, 256) X(4, 8, 4, 256)    \
   X(8, 16, 4, 256) X(16, 32, 4, 512) X(4, 8, 8, 512) X(8, 4, 8, 256) X(8, 8, 8, 512)     \
   X(16, 8, 8, 512) X(16, 32, 8, 512) X(8, 1, 16, 256) X(16, 1, 16, 256) X(16, 4, 16, 512) \
-  X(16, 32, 16, 512) X(8, 1, 32, 256) X(16, 1, 32, 512) X(16, 32, 32, 512)
+  X(16, 32, 16, 512) X(8, 1, 32, 256) X(16, 1, 32, 512) X(16, 32, 32, 512)              \
+  X(64, 1, 32, 256)
 
 // Pipelined exponential-domain rings (chain_exp.cu): shapes (combine lanes
 // per label G, weights per combine lane CAT, helper lanes per label H,

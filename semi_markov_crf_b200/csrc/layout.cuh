@@ -9,7 +9,7 @@
 namespace semicrf {
 
 constexpr int C_MAX = 128;
-constexpr int K_MAX = 512;
+constexpr int K_MAX = 2048;
 constexpr int KC_MAX = 16384;
 constexpr int NT_MAX = 512;  // threads per CTA
 constexpr int TS = 32;       // prefix-sum rows per TMA tile

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float s;
         const float lse =
-            k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
+            k_fanin<KBT, G>(rl + base, ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float ssum;
         const float lse =
-            k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
+            k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
         const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = Bt;
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(LB, 1)
         const int si = ri[ln.cc];
         const float sf = rf[ln.cc];
         float s;
-        const float lse = k_fanin<KBT, G>(rl + base, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
+        const float lse = k_fanin<KBT, G>(rl + base, ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(LB, 1)
 #pragma unroll
   for (int i = 0; i < KBT; ++i) {
     accd[i] = 0.f;
-    const int k = ln.k_of(i, false);
+    const int k = ln.k_of(ln.widx(i), false);
     if (ln.act && k <= K) ws.pgd[(seg * K + (k - 1)) * C + ln.c] = 0.0;
   }
 #pragma unroll
@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(LB, 1)
       const int si = ri[ln.cc];
       const float sf = rf[ln.cc];
       float ksum;
-      const float lse = k_fanin<KBT, G>(rl + base, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
+      const float lse = k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
       const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
       float St = 0.f;
       if (ln.leader) {
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(LB, 1)
         if (ln.act) {
 #pragma unroll
           for (int i = 0; i < KBT; ++i) {
-            const int k = ln.k_of(i, false);
+            const int k = ln.k_of(ln.widx(i), false);
             if (k <= K) ws.pgd[(seg * K + (k - 1)) * C + ln.c] += (double)accd[i];
             accd[i] = 0.f;
           }

@@ -204,9 +204,15 @@ __device__ __forceinline__ void gargmax(float& v, int& i) {
 
 // ----------------------------------------------------------------------------- lanes
 
-// One lane of a label group: label c, lane j of G.  Durations of lane term i:
-//   up   (forward, terms at t - k):  k_i = (j + 1) * KBT - i
-//   down (backward, terms at s + k): k_i = j * KBT + 1 + i
+// One lane of a label group: label c, lane j of G.  Durations of window
+// element w of the lane (its ring entries r[0..KBT), contiguous):
+//   up   (forward, terms at t - k):  k_w = (j + 1) * KBT - w
+//   down (backward, terms at s + k): k_w = j * KBT + 1 + w
+// The lane visits its window in rotated order, element widx(i) = (i + j) mod
+// KBT at term i: lanes of a label start KBT entries apart, so in plain order
+// a half warp's 64-bit reads would all fall in the same shared-memory banks
+// (16-way for KBT >= 16); rotated, consecutive lanes read consecutive banks.
+// The duration scores d[i] are stored in the same rotated order.
 // Label-fan-in operands e[i] = 2^(trans2 - max) for the other side's labels
 // j*CAT + i: column-normalised for the forward side (sum over c' into c),
 // row-normalised for the backward side (sum over c out of c').
@@ -217,9 +223,11 @@ struct Lane {
   float tmax;
   float d[KBT];
   float e[CAT];
-  __device__ __forceinline__ int k_of(int i, bool up) const {
-    return up ? (j + 1) * KBT - i : j * KBT + 1 + i;
+  __device__ __forceinline__ int k_of(int w, bool up) const {
+    return up ? (j + 1) * KBT - w : j * KBT + 1 + w;
   }
+  // window element visited at term i
+  __device__ __forceinline__ int widx(int i) const { return (i + j) & (KBT - 1); }
   __device__ __forceinline__ void init_ids(const Dims& dm) {
     c = threadIdx.x / G;
     j = threadIdx.x % G;
@@ -230,7 +238,7 @@ struct Lane {
   __device__ __forceinline__ void init_dur(const Dims& dm, const float* dur, bool up) {
 #pragma unroll
     for (int i = 0; i < KBT; ++i) {
-      const int k = k_of(i, up);
+      const int k = k_of(widx(i), up);
       d[i] = (act && k <= dm.K) ? __ldg(dur + (size_t)(k - 1) * dm.C + cc) * l2e() : NEG_INF;
     }
   }
@@ -282,7 +290,9 @@ __device__ __forceinline__ void load_block(const float* p, float (&v)[CAT]) {
 }
 
 // ----------------------------------------------------------------------------- fan-ins
-// k fan-in over a lane's window r[0..KBT), y_i = ((P + Q) + v) + dur2.
+// k fan-in over a lane's window r[0..KBT), visited in the lane's rotated
+// order (term i reads r[(i + rot) mod KBT], d[i] is its duration score),
+// y_i = ((P + Q) + v) + dur2.
 // The exponentials are taken against an exact-integer shift m (a prediction
 // of the group LSE: no max pass, no max reduction): e[i] = 2^(y_i - m) and
 // s = group sum.  If s leaves [2^-64, 2^64] the group redoes the fan-in
@@ -292,14 +302,15 @@ __device__ __forceinline__ void load_block(const float* p, float (&v)[CAT]) {
 // >= C: their sum is 0 by construction and must not take the fallback, which
 // would hold up the rest of their warp every step.
 template <int KBT, int G>
-__device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (&d)[KBT], float& m,
-                                         float& s, float (&e)[KBT], bool live = true) {
+__device__ __forceinline__ float k_fanin(const float2* r, int rot, float Q, const float (&d)[KBT],
+                                         float& m, float& s, float (&e)[KBT], bool live = true) {
+  static_assert((KBT & (KBT - 1)) == 0, "KBT must be a power of two");
   {
     const float Qm = Q - m;  // exact: both integers
     float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < KBT; ++i) {
-      const float2 v = r[i];
+      const float2 v = r[(i + rot) & (KBT - 1)];
       e[i] = ex2(((v.y + Qm) + v.x) + d[i]);
       sp[i & 3] += e[i];
     }
@@ -311,7 +322,7 @@ __device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (
     float mx = NEG_INF;
 #pragma unroll
     for (int i = 0; i < KBT; ++i) {
-      const float2 v = r[i];
+      const float2 v = r[(i + rot) & (KBT - 1)];
       mx = fmaxf(mx, ((v.y + Q) + v.x) + d[i]);
     }
 #pragma unroll
@@ -321,7 +332,7 @@ __device__ __forceinline__ float k_fanin(const float2* r, float Q, const float (
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < KBT; ++i) {
-      const float2 v = r[i];
+      const float2 v = r[(i + rot) & (KBT - 1)];
       e[i] = ex2(((v.y + Qm) + v.x) + d[i]);
       ss += e[i];
     }

@@ -112,16 +112,19 @@ __global__ void __launch_bounds__(LB, 1)
       {
         const float Q = (float)(si - Sb) - Frel;
         const float2* r = rl + base;
-        // lane term i has k = (j+1)*KBT - i: walk i downwards for ascending k
+        // the lane's window in its rotated order (Lane::widx); ties go to
+        // the smallest k
         float best = NEG_INF;
         bk = 0x7fffffff;
 #pragma unroll
-        for (int i = KBT - 1; i >= 0; --i) {
-          const float2 v = r[i];
+        for (int i = 0; i < KBT; ++i) {
+          const int w = ln.widx(i);
+          const float2 v = r[w];
           const float y = ((v.y + Q) + v.x) + ln.d[i];
-          if (y > best || bk == 0x7fffffff) {
+          const int k = ln.k_of(w, true);
+          if (y > best || (y == best && k < bk) || bk == 0x7fffffff) {
             best = y;
-            bk = ln.k_of(i, true);
+            bk = k;
           }
         }
         gargmax<G>(best, bk);

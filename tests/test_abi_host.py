@@ -54,6 +54,9 @@ def test_workspace_bytes_and_limits(lib):
     assert _ws_bytes(lib, 1, 10, 128, 65)[0] == 2         # K above the limit for C=128
     assert _ws_bytes(lib, 1, 10, 16, 512)[0] == 0
     assert _ws_bytes(lib, 1, 10, 16, 513)[0] == 2
+    assert _ws_bytes(lib, 1, 10, 8, 2048)[0] == 0          # long durations, few labels
+    assert _ws_bytes(lib, 1, 10, 8, 2049)[0] == 2
+    assert _ws_bytes(lib, 1, 10, 9, 1024)[0] == 2
     assert _ws_bytes(lib, -1, 10, 4, 4)[0] == 1
     assert _ws_bytes(lib, 1, 10, 0, 4)[0] == 1
     assert _ws_bytes(lib, 1, 10, 4, 4, flags=0x80)[0] == 1

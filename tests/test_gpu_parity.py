@@ -31,6 +31,12 @@ def _cases():
         # C = 64: the traceback stages a few hundred rows at a time, so these
         # lengths take several stages
         "traceback_in_stages": lambda: synth.make_custom(2, 900, 16, 64, seed=13, lengths=[900, 777]),
+        # long durations: K above 512 takes the 64-durations-per-lane shape
+        "k_700": lambda: synth.make_custom(2, 2600, 700, 4, seed=42, lengths=[2600, 1900],
+                                           dur_mean=100.0, amp=2.0),
+        "k_2000_genomic_like": lambda: synth.make_custom(
+            2, 5000, 2000, 6, seed=41, lengths=[5000, 3333], dur_mean=50.0, amp=2.0,
+            label_p=(0.6, 0.2, 0.1, 0.05, 0.03, 0.02)),
     }
 
 

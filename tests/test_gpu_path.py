@@ -93,6 +93,8 @@ CASES = {
     "mixed_with_empty": lambda: synth.make_custom(4, 80, 9, 5, seed=9, lengths=[80, 0, 1, 57]),
     "k_equals_1": lambda: synth.make_custom(2, 90, 1, 7, seed=7, lengths=[90, 41]),
     "several_chunks": lambda: synth.make_custom(3, 2600, 12, 3, seed=21, lengths=[2600, 1025, 1024]),
+    "k_2000": lambda: synth.make_custom(2, 5000, 2000, 6, seed=41, lengths=[5000, 3333],
+                                        dur_mean=400.0, amp=2.0),
 }
 
 

@@ -108,7 +108,8 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(1, 32, 16, 16, 544) X(2, 24, 4, 8, 288) X(2, 24, 4, 16, 288) X(2, 24, 8, 16, 480) \
   X(2, 32, 4, 8, 384) X(2, 32, 4, 16, 384) X(2, 32, 8, 16, 640) X(4, 24, 4, 8, 768)   \
   X(4, 12, 4, 8, 384) X(4, 12, 4, 16, 384) X(2, 48, 2, 32, 384) X(2, 64, 2, 32, 512)  \
-  X(4, 24, 2, 32, 576) X(4, 32, 4, 8, 1024) X(4, 32, 2, 32, 768)
+  X(4, 24, 2, 32, 576) X(4, 32, 4, 8, 1024) X(4, 32, 2, 32, 768) X(1, 8, 32, 64, 224) \
+  X(1, 8, 32, 64, 288)
 
 size_t chain_exp_smem_bytes(const Dims& d);
 size_t viterbi_pipe_smem_bytes(const Dims& d);

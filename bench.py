@@ -538,7 +538,7 @@ def run_ours(args):
                                 "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
                                 "frac": (nb / (per * 1e-3) / 1e9) / peaks["hbm_gbs"]
                                 if peaks.get("hbm_gbs") else None,
-                                "bytes_per_launch": nb}
+                                "bytes_per_launch": nb, "traffic": stored_traffic(k)}
         line["nll"] = {
             "what": "loss log Z - score(gold) and its gradient: semicrf_path_score with "
                     "SEMICRF_FLAG_NEGATE_GRAD on the gradient buffers (gold = the generating "

@@ -54,14 +54,14 @@ def _load():
             lib.oracle_center.restype = None
             lib.oracle_prefix.argtypes = [_dp, ctypes.c_int, ctypes.c_int, _dp]
             lib.oracle_prefix.restype = None
-            lib.oracle_fb.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
+            lib.oracle_fb.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp,
                                       ctypes.c_int, ctypes.c_double, _dp, _dp,
                                       _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
             lib.oracle_fb.restype = ctypes.c_int
-            lib.oracle_viterbi.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
+            lib.oracle_viterbi.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp,
                                            ctypes.c_int, _dp, _ip, _u8p]
             lib.oracle_viterbi.restype = ctypes.c_int
-            lib.oracle_path_score.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
+            lib.oracle_path_score.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp,
                                               ctypes.c_int, _ip, _u8p]
             lib.oracle_path_score.restype = ctypes.c_double
             lib.oracle_path_counts.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -85,6 +85,13 @@ def _threads(n_items: int, threads: int | None) -> int:
     if threads is None:
         threads = os.cpu_count() or 1
     return max(1, min(int(threads), n_items))
+
+
+def _proj(P, b, L, C):
+    """Contiguous float64 [L, C] slice of a [B, T, C] projection array, or None."""
+    if P is None:
+        return None
+    return np.ascontiguousarray(np.asarray(P[b, :max(L, 1)], dtype=np.float64)) if L > 0 else np.zeros((1, C))
 
 
 def prefix_center(em, lengths, center: bool = True):
@@ -111,8 +118,12 @@ def prefix_center(em, lengths, center: bool = True):
 
 
 def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool = True,
-                     grad_logZ=None, threads: int | None = None, want_alpha_beta: bool = False):
+                     grad_logZ=None, threads: int | None = None, want_alpha_beta: bool = False,
+                     p_start=None, p_end=None):
     """Exact log Z, marginals and gradients for a batch.
+
+    ``p_start`` / ``p_end`` [B, T, C] (optional) are boundary projection
+    scores: segment [s, t) with label c gains p_start[b, s, c] + p_end[b, t-1, c].
 
     Returns a dict of float64 arrays:
       logZ [B], logZ_beta [B], start_marg / end_marg [B, T+1, C],
@@ -151,7 +162,8 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
         ge = np.zeros((max(L, 1), C))
         al = np.zeros((L + 1, C)) if want_alpha_beta else None
         be = np.zeros((L + 1, C)) if want_alpha_beta else None
-        rc = lib.oracle_fb(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), int(center), float(g[b]),
+        rc = lib.oracle_fb(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), _ptr(_proj(p_start, b, L, C)),
+                           _ptr(_proj(p_end, b, L, C)), int(center), float(g[b]),
                            _ptr(lz), _ptr(lzb), _ptr(al), _ptr(be), _ptr(St), _ptr(En),
                            _ptr(mu), _ptr(ge), _ptr(gt[b]), _ptr(gd[b]))
         if rc != 0:
@@ -183,13 +195,14 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
 
 
 def log_partition(em, lengths, trans, dur, K: int | None = None, center: bool = True,
-                  threads: int | None = None):
+                  threads: int | None = None, p_start=None, p_end=None):
     """log Z [B] only (still the full explicit-edge forward-backward)."""
-    return forward_backward(em, lengths, trans, dur, K, center, threads=threads)["logZ"]
+    return forward_backward(em, lengths, trans, dur, K, center, threads=threads,
+                            p_start=p_start, p_end=p_end)["logZ"]
 
 
 def viterbi(em, lengths, trans, dur, K: int | None = None, center: bool = True,
-            threads: int | None = None):
+            threads: int | None = None, p_start=None, p_end=None):
     """Best segmentation: score [B] float64, labels [B, T] int32 (-1 past the
     length) and seg_start [B, T] uint8 (1 where a segment starts)."""
     lib = _load()
@@ -209,7 +222,9 @@ def viterbi(em, lengths, trans, dur, K: int | None = None, center: bool = True,
         sc = np.zeros(1)
         lab = np.full(max(L, 1), -1, dtype=np.int32)
         ss = np.zeros(max(L, 1), dtype=np.uint8)
-        rc = lib.oracle_viterbi(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), int(center), _ptr(sc),
+        rc = lib.oracle_viterbi(_ptr(e), L, C, K, _ptr(trans), _ptr(dur),
+                                _ptr(_proj(p_start, b, L, C)), _ptr(_proj(p_end, b, L, C)),
+                                int(center), _ptr(sc),
                                 _ptr(lab, _ip), _ptr(ss, _u8p))
         if rc != 0:
             raise MemoryError("oracle_viterbi: allocation failed")
@@ -229,7 +244,7 @@ def viterbi(em, lengths, trans, dur, K: int | None = None, center: bool = True,
 
 
 def path_score(em, lengths, trans, dur, labels, seg_start, K: int | None = None,
-               center: bool = True):
+               center: bool = True, p_start=None, p_end=None):
     """float64 score [B] of the given segmentations (NaN where malformed)."""
     lib = _load()
     em = _f64(em)
@@ -244,7 +259,9 @@ def path_score(em, lengths, trans, dur, labels, seg_start, K: int | None = None,
         e = np.ascontiguousarray(em[b, :L]) if L > 0 else np.zeros((1, C))
         lab = np.ascontiguousarray(np.asarray(labels[b, :max(L, 1)], dtype=np.int32))
         ss = np.ascontiguousarray(np.asarray(seg_start[b, :max(L, 1)], dtype=np.uint8))
-        out[b] = lib.oracle_path_score(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), int(center),
+        out[b] = lib.oracle_path_score(_ptr(e), L, C, K, _ptr(trans), _ptr(dur),
+                                       _ptr(_proj(p_start, b, L, C)), _ptr(_proj(p_end, b, L, C)),
+                                       int(center),
                                        _ptr(lab, _ip), _ptr(ss, _u8p))
     return out
 
@@ -253,8 +270,9 @@ def path_counts(lengths, labels, seg_start, C: int, K: int, center: bool = True)
     """Derivatives of the path score of given segmentations (float64).
 
     Returns ``grad_em`` [B, T, C] (d score_b / d em[b, u, c], zero past L_b),
-    ``trans_count`` [B, C, C], ``dur_count`` [B, K, C] (per sequence, not
-    weighted) and ``valid`` [B] (False where the path is malformed; its
+    ``trans_count`` [B, C, C], ``dur_count`` [B, K, C], ``p_start_count`` /
+    ``p_end_count`` [B, T, C] (derivatives with respect to boundary
+    projections; per sequence, not weighted) and ``valid`` [B] (False where the path is malformed; its
     counts are zero).  Their weighted sums are the gold-score part of the
     gradient of the loss log Z - score.
     """
@@ -280,4 +298,18 @@ def path_counts(lengths, labels, seg_start, C: int, K: int, center: bool = True)
             grad_em[b, :L] = de[:L]
         tc[b] = dt
         dc[b] = dd
-    return dict(grad_em=grad_em, trans_count=tc, dur_count=dc, valid=valid)
+    # boundary projections: the path score gains p_start at each segment's
+    # first position and p_end at its last, so those are its derivatives
+    ps_c = np.zeros((B, T, C))
+    pe_c = np.zeros((B, T, C))
+    for b in range(B):
+        L = int(lengths[b])
+        if not valid[b]:
+            continue
+        for u in range(L):
+            if seg_start[b, u]:
+                ps_c[b, u, labels[b, u]] = 1.0
+            if u == L - 1 or seg_start[b, u + 1]:
+                pe_c[b, u, labels[b, u]] = 1.0
+    return dict(grad_em=grad_em, trans_count=tc, dur_count=dc, valid=valid,
+                p_start_count=ps_c, p_end_count=pe_c)

@@ -19,7 +19,10 @@
  *   is no start or end transition (the first segment carries no trans term).
  *   content(s, t, c) is the sum of the (centred) emissions of label c over the
  *   positions s..t-1 (explainer section 2, "On-the-Fly Edge Computation via
- *   Prefix Sums": the segment content score).
+ *   Prefix Sums": the segment content score).  Optional boundary projections
+ *   (explainer section 2, "Boundary Projections") add P_start[s, c] +
+ *   P_end[t-1, c] to the segment: a score for starting at position s and one
+ *   for ending at position t-1.
  *
  *   Centering (explainer section 2, "Emission Baseline Centering"): a
  *   per-sequence, per-label baseline nu[c] = mean over the L valid positions
@@ -116,18 +119,31 @@ static void contents_starting_at(const double *et, int C, int s, int kmax, doubl
                 content[(size_t)(k - 2) * C + c] + et[(size_t)(s + k - 1) * C + c];
 }
 
+/* Boundary projection terms of segment [s, t) with label c
+ * ("Streaming Structured Inference with Flash-SemiCRF", explainer section 2,
+ * "Boundary Projections": start and end features added to the edge
+ * potential): ps[s, c] + pe[t-1, c], either array may be NULL (no term). */
+static double proj(const double *ps, const double *pe, int C, int s, int t, int c)
+{
+    double v = 0.0;
+    if (ps) v += ps[(size_t)s * C + c];
+    if (pe) v += pe[(size_t)(t - 1) * C + c];
+    return v;
+}
+
 /* The explicit edge block for segments ending at boundary t:
- *   W[k-1, c', c] = content(t-k, t, c) + dur[k-1, c] + trans[c', c]   (t-k >= 1)
- *   W[k-1, 0,  c] = content(0,   t, c) + dur[k-1, c]                  (t-k == 0)
+ *   W[k-1, c', c] = content(t-k, t, c) + dur[k-1, c] + proj + trans[c', c]   (t-k >= 1)
+ *   W[k-1, 0,  c] = content(0,   t, c) + dur[k-1, c] + proj                  (t-k == 0)
  */
 static void edge_block(const double *content, const double *trans, const double *dur,
-                       int C, int t, int kmax, double *W)
+                       const double *ps, const double *pe, int C, int t, int kmax, double *W)
 {
     for (int k = 1; k <= kmax; ++k) {
         double *Wk = W + (size_t)(k - 1) * C * C;
         for (int cp = 0; cp < C; ++cp)
             for (int c = 0; c < C; ++c) {
-                double v = content[(size_t)(k - 1) * C + c] + dur[(size_t)(k - 1) * C + c];
+                double v = content[(size_t)(k - 1) * C + c] + dur[(size_t)(k - 1) * C + c] +
+                           proj(ps, pe, C, t - k, t, c);
                 if (t - k >= 1) v += trans[(size_t)cp * C + c];
                 Wk[(size_t)cp * C + c] = v;
             }
@@ -139,6 +155,7 @@ static void edge_block(const double *content, const double *trans, const double 
  * e [L, C] raw emissions; trans [C, C] (trans[c', c]); dur [K, C].
  * g is d loss / d logZ for this sequence (scales the three gradients only).
  *
+ * ps, pe [L, C] boundary projection scores (NULL: none), see proj().
  * Outputs (each may be NULL except logZ):
  *   alpha, beta        [(L+1), C]  full float64 forward / backward arrays
  *                                  (beta row 0 is left at 0: no segment
@@ -150,7 +167,7 @@ static void edge_block(const double *content, const double *trans, const double 
  * Returns 0, or -1 if the scratch allocation failed.
  */
 int oracle_fb(const double *e, int L, int C, int K, const double *trans, const double *dur,
-              int center, double g, double *logZ, double *logZ_beta,
+              const double *ps, const double *pe, int center, double g, double *logZ, double *logZ_beta,
               double *alpha_out, double *beta_out, double *start_marg, double *end_marg,
               double *pos_marg, double *grad_e, double *grad_trans, double *grad_dur)
 {
@@ -186,7 +203,7 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
     for (int t = 1; t <= L; ++t) {
         int kmax = t < K ? t : K;
         contents_ending_at(et, C, t, kmax, content);
-        edge_block(content, trans, dur, C, t, kmax, W);
+        edge_block(content, trans, dur, ps, pe, C, t, kmax, W);
         for (int c = 0; c < C; ++c) {
             int n = 0;
             for (int k = 1; k <= kmax; ++k) {
@@ -214,7 +231,8 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
                 for (int k = 1; k <= kmax; ++k)
                     for (int c = 0; c < C; ++c)
                         terms[n++] = trans[(size_t)cp * C + c] + content[(size_t)(k - 1) * C + c] +
-                                     dur[(size_t)(k - 1) * C + c] + beta[(size_t)(s + k) * C + c];
+                                     dur[(size_t)(k - 1) * C + c] + proj(ps, pe, C, s, s + k, c) +
+                                     beta[(size_t)(s + k) * C + c];
                 beta[(size_t)s * C + cp] = lse(terms, n);
             }
         } else {
@@ -222,7 +240,7 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
             for (int k = 1; k <= kmax; ++k)
                 for (int c = 0; c < C; ++c)
                     terms[n++] = content[(size_t)(k - 1) * C + c] + dur[(size_t)(k - 1) * C + c] +
-                                 beta[(size_t)k * C + c];
+                                 proj(ps, pe, C, 0, k, c) + beta[(size_t)k * C + c];
             if (logZ_beta) *logZ_beta = lse(terms, n);
             for (int c = 0; c < C; ++c) beta[c] = 0.0;
         }
@@ -233,7 +251,7 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
     for (int t = 1; t <= L; ++t) {
         int kmax = t < K ? t : K;
         contents_ending_at(et, C, t, kmax, content);
-        edge_block(content, trans, dur, C, t, kmax, W);
+        edge_block(content, trans, dur, ps, pe, C, t, kmax, W);
         for (int k = 1; k <= kmax; ++k) {
             const int s = t - k;
             const double *Wk = W + (size_t)(k - 1) * C * C;
@@ -283,7 +301,7 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
  * smallest final label.  Returns 0, or -1 on allocation failure.
  */
 int oracle_viterbi(const double *e, int L, int C, int K, const double *trans, const double *dur,
-                   int center, double *score, int32_t *labels, uint8_t *seg_start)
+                   const double *ps, const double *pe, int center, double *score, int32_t *labels, uint8_t *seg_start)
 {
     if (L <= 0) {
         *score = 0.0;
@@ -305,7 +323,7 @@ int oracle_viterbi(const double *e, int L, int C, int K, const double *trans, co
     for (int t = 1; t <= L; ++t) {
         int kmax = t < K ? t : K;
         contents_ending_at(et, C, t, kmax, content);
-        edge_block(content, trans, dur, C, t, kmax, W);
+        edge_block(content, trans, dur, ps, pe, C, t, kmax, W);
         for (int c = 0; c < C; ++c) {
             double best = -INFINITY;
             int best_k = 0, best_c = -1, have = 0;
@@ -354,7 +372,7 @@ int oracle_viterbi(const double *e, int L, int C, int K, const double *trans, co
  * or a segment longer than K.
  */
 double oracle_path_score(const double *e, int L, int C, int K, const double *trans,
-                         const double *dur, int center, const int32_t *labels,
+                         const double *dur, const double *ps, const double *pe, int center, const int32_t *labels,
                          const uint8_t *seg_start)
 {
     if (L <= 0) return 0.0;
@@ -379,7 +397,7 @@ double oracle_path_score(const double *e, int L, int C, int K, const double *tra
         if (k > K) { total = NAN; break; }
         double seg = 0.0;
         for (int u = s; u < t; ++u) seg += et[(size_t)u * C + c];
-        seg += dur[(size_t)(k - 1) * C + c];
+        seg += dur[(size_t)(k - 1) * C + c] + proj(ps, pe, C, s, t, c);
         if (prev >= 0) seg += trans[(size_t)prev * C + c];
         total += seg;
         prev = c;

@@ -30,19 +30,23 @@ def segmentations(L: int, K: int, C: int):
     yield from rec(0)
 
 
-def score(segs, et, trans, dur):
+def score(segs, et, trans, dur, ps=None, pe=None):
     total = 0.0
     prev = None
     for (s, t, c) in segs:
         total += float(sum(et[u, c] for u in range(s, t)))
         total += float(dur[t - s - 1, c])
+        if ps is not None:
+            total += float(ps[s, c])      # boundary projections: start at s,
+        if pe is not None:
+            total += float(pe[t - 1, c])  # end at position t-1
         if prev is not None:
             total += float(trans[prev, c])
         prev = c
     return total
 
 
-def enumerate_all(e, L, trans, dur, center=True, tie_tol=1e-9):
+def enumerate_all(e, L, trans, dur, center=True, tie_tol=1e-9, ps=None, pe=None):
     """Everything the oracle reports, by enumeration, for one sequence."""
     e = np.asarray(e, dtype=np.float64)[:L]
     trans = np.asarray(trans, dtype=np.float64)
@@ -51,7 +55,7 @@ def enumerate_all(e, L, trans, dur, center=True, tie_tol=1e-9):
     nu = e.mean(axis=0) if (center and L > 0) else np.zeros(C)
     et = e - nu
     segs_all = list(segmentations(L, K, C))
-    scores = np.array([score(sg, et, trans, dur) for sg in segs_all])
+    scores = np.array([score(sg, et, trans, dur, ps, pe) for sg in segs_all])
     m = scores.max()
     logZ = m + math.log(np.exp(scores - m).sum())
     probs = np.exp(scores - logZ)

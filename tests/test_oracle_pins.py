@@ -399,6 +399,21 @@ def test_path_counts_are_the_finite_differences_of_the_path_score(center):
         assert abs((sc(d=dp) - sc(d=dm)) / (2 * h) - cnt["dur_count"][0, k, c]) < 1e-9
     # the rows past L_b carry no gradient
     assert np.all(cnt["grad_em"][0, 14:] == 0)
+    # boundary projections enter the score linearly too
+    ps = rng.normal(0, 1, size=(1, T, C))
+    pe = rng.normal(0, 1, size=(1, T, C))
+
+    def scp(a, z):
+        return oracle.path_score(em, lengths, trans, dur, labels, seg, K, center=center,
+                                 p_start=a, p_end=z)[0]
+
+    for (u, c) in [(0, lab[0]), (5, 1), (13, 2), (9, 0)]:
+        a, z = ps.copy(), ps.copy()
+        a[0, u, c] += h; z[0, u, c] -= h
+        assert abs((scp(a, pe) - scp(z, pe)) / (2 * h) - cnt["p_start_count"][0, u, c]) < 1e-9
+        a, z = pe.copy(), pe.copy()
+        a[0, u, c] += h; z[0, u, c] -= h
+        assert abs((scp(ps, a) - scp(ps, z)) / (2 * h) - cnt["p_end_count"][0, u, c]) < 1e-9
 
 
 def test_path_counts_reject_what_the_path_score_rejects():
@@ -431,3 +446,70 @@ def test_gold_segmentation_of_the_generator_is_a_valid_path():
            - oracle.path_score(w["em"], w["lengths"], w["trans"], w["dur"], w["gold"],
                                w["gold_start"], w["K"]))
     assert np.all(nll > 0)
+
+
+# ------------------------------------------------------- boundary projections
+@pytest.mark.parametrize("L,K,C,center,seed", BRUTE_CASES[:5])
+def test_projections_bruteforce(L, K, C, center, seed):
+    rng = np.random.default_rng(400 + seed)
+    em, lengths, trans, dur = _rand_case(rng, 1, L, K, C, pstd=0.7)
+    ps = rng.normal(0, 0.8, size=(1, L, C))
+    pe = rng.normal(0, 0.8, size=(1, L, C))
+    ref = brute.enumerate_all(em[0], L, trans, dur, center=center, ps=ps[0], pe=pe[0])
+    out = oracle.forward_backward(em, lengths, trans, dur, K, center=center, threads=1,
+                                  p_start=ps, p_end=pe)
+    assert abs(out["logZ"][0] - ref["logZ"]) <= 1e-12 * max(1.0, abs(ref["logZ"]))
+    assert abs(out["logZ_beta"][0] - ref["logZ"]) <= 1e-12 * max(1.0, abs(ref["logZ"]))
+    for key in ("start_marg", "end_marg", "pos_marg"):
+        assert np.max(np.abs(out[key][0][: ref[key].shape[0]] - ref[key])) < 1e-12, key
+    assert np.max(np.abs(out["grad_dur"] - ref["grad_dur"])) < 1e-12
+    assert np.max(np.abs(out["grad_trans"] - ref["grad_trans"])) < 1e-12
+    vit = oracle.viterbi(em, lengths, trans, dur, K, center=center, threads=1, p_start=ps, p_end=pe)
+    assert abs(vit["score"][0] - ref["best_score"]) < 1e-12
+    assert any(np.array_equal(vit["labels"][0, :L], lab) and np.array_equal(vit["seg_start"][0, :L], ss)
+               for lab, ss in ref["optimal"])
+    rs = oracle.path_score(em, lengths, trans, dur, vit["labels"], vit["seg_start"], K,
+                           center=center, p_start=ps, p_end=pe)
+    assert abs(rs[0] - ref["best_score"]) < 1e-12
+
+
+def test_projection_gradients_are_the_boundary_marginals():
+    # d log Z / d p_start[s, c] = P(a label-c segment starts at s) and
+    # d log Z / d p_end[u, c] = P(a label-c segment ends after position u).
+    rng = np.random.default_rng(411)
+    T, K, C = 15, 4, 3
+    em, lengths, trans, dur = _rand_case(rng, 1, T, K, C, lengths=[13])
+    ps = rng.normal(0, 0.5, size=(1, T, C))
+    pe = rng.normal(0, 0.5, size=(1, T, C))
+    out = oracle.forward_backward(em, lengths, trans, dur, K, threads=1, p_start=ps, p_end=pe)
+
+    def lz(a, b_):
+        return oracle.log_partition(em, lengths, trans, dur, K, threads=1, p_start=a, p_end=b_)[0]
+
+    for (u, c) in [(0, 0), (4, 2), (12, 1), (7, 0)]:
+        a, b_ = ps.copy(), ps.copy()
+        a[0, u, c] += 1e-5; b_[0, u, c] -= 1e-5
+        assert abs((lz(a, pe) - lz(b_, pe)) / 2e-5 - out["start_marg"][0, u, c]) < 1e-6
+        a, b_ = pe.copy(), pe.copy()
+        a[0, u, c] += 1e-5; b_[0, u, c] -= 1e-5
+        assert abs((lz(ps, a) - lz(ps, b_)) / 2e-5 - out["end_marg"][0, u + 1, c]) < 1e-6
+    # entries past the length change nothing
+    a = ps.copy(); a[0, 13:] += 5.0
+    assert lz(a, pe) == lz(ps, pe)
+
+
+def test_label_constant_projections_are_a_duration_shift():
+    # p_start[s, c] = a[c] and p_end[u, c] = z[c] for every position add
+    # a[c] + z[c] to every label-c segment, which is dur[k-1, c] + a[c] + z[c].
+    rng = np.random.default_rng(412)
+    B, T, K, C = 2, 40, 6, 4
+    em, lengths, trans, dur = _rand_case(rng, B, T, K, C, lengths=[40, 23])
+    a = rng.normal(0, 1, size=C)
+    z = rng.normal(0, 1, size=C)
+    ps = np.broadcast_to(a, (B, T, C)).copy()
+    pe = np.broadcast_to(z, (B, T, C)).copy()
+    got = oracle.forward_backward(em, lengths, trans, dur, K, threads=1, p_start=ps, p_end=pe)
+    ref = oracle.forward_backward(em, lengths, trans, dur + a + z, K, threads=1)
+    assert np.max(np.abs(got["logZ"] - ref["logZ"])) < 1e-10
+    assert np.max(np.abs(got["pos_marg"] - ref["pos_marg"])) < 1e-10
+    assert np.max(np.abs(got["grad_dur"] - ref["grad_dur"])) < 1e-10

@@ -13,6 +13,7 @@
  *   4. max-semiring (Viterbi) decoding               semicrf_viterbi
  *   and the score of a given segmentation with its
  *   gradient, for the training loss                  semicrf_path_score
+ *   with boundary projections                        semicrf_*_proj
  *
  * Model.  A sequence b has length L_b (0 <= L_b <= T).  A segmentation
  * splits its positions 0..L_b-1 into consecutive segments [s, t) of duration
@@ -201,6 +202,54 @@ SEMICRF_API int semicrf_path_score(const float *em, const int32_t *lengths, cons
                                    unsigned flags, void *ws, size_t ws_bytes,
                                    const double *grad_score, double *score, float *grad_em,
                                    float *grad_trans, float *grad_dur, semicrf_stream_t stream);
+
+/*
+ * Boundary projections ("Streaming Structured Inference with Flash-SemiCRF",
+ * explainer section 2, "Boundary Projections": separately computed start and
+ * end features added to the edge potentials).  p_start and p_end are
+ * [B, T, C] float32 device arrays (either may be NULL): a segment [s, t) with
+ * label c scores p_start[b, s, c] + p_end[b, t-1, c] on top of the model
+ * above.  Entries u >= L_b are never read.
+ *
+ * semicrf_forward_proj: as semicrf_forward.  The rings run in the log domain
+ *   (the exponential-domain kernels have no projection term); the workspace
+ *   records that projections are on for the backward that consumes it.
+ * semicrf_backward_proj: as semicrf_backward, after semicrf_forward_proj on
+ *   the same workspace; additionally writes (each nullable)
+ *     grad_p_start [B, T, C] = g_b * start_marg[b, u, c]
+ *     grad_p_end   [B, T, C] = g_b * end_marg[b, u + 1, c]   (0 for u >= L_b),
+ *   the gradients of g_b * log Z_b.  The marginal outputs stay optional.
+ * semicrf_viterbi_proj: as semicrf_viterbi with the projection terms.
+ * semicrf_path_score_proj: as semicrf_path_score with the projection terms;
+ *   also ADDS w_b to grad_p_start[b, s, c] at the first position s and to
+ *   grad_p_end[b, u, c] at the last position u of each label-c segment
+ *   (each nullable).
+ * A plain call (semicrf_forward, semicrf_viterbi) clears the record.
+ */
+SEMICRF_API int semicrf_forward_proj(const float *em, const int32_t *lengths, const float *trans,
+                                     const float *dur, const float *p_start, const float *p_end,
+                                     int B, int T, int C, int K, unsigned flags, void *ws,
+                                     size_t ws_bytes, double *logZ, semicrf_stream_t stream);
+SEMICRF_API int semicrf_backward_proj(const int32_t *lengths, const float *trans, const float *dur,
+                                      int B, int T, int C, int K, unsigned flags, void *ws,
+                                      size_t ws_bytes, const double *grad_logZ, float *grad_em,
+                                      float *grad_trans, float *grad_dur, float *grad_p_start,
+                                      float *grad_p_end, float *pos_marg, float *start_marg,
+                                      float *end_marg, semicrf_stream_t stream);
+SEMICRF_API int semicrf_viterbi_proj(const float *em, const int32_t *lengths, const float *trans,
+                                     const float *dur, const float *p_start, const float *p_end,
+                                     int B, int T, int C, int K, unsigned flags, void *ws,
+                                     size_t ws_bytes, double *score, int32_t *labels,
+                                     uint8_t *seg_start, semicrf_stream_t stream);
+SEMICRF_API int semicrf_path_score_proj(const float *em, const int32_t *lengths,
+                                        const float *trans, const float *dur,
+                                        const float *p_start, const float *p_end,
+                                        const int32_t *labels, const uint8_t *seg_start, int B,
+                                        int T, int C, int K, unsigned flags, void *ws,
+                                        size_t ws_bytes, const double *grad_score, double *score,
+                                        float *grad_em, float *grad_trans, float *grad_dur,
+                                        float *grad_p_start, float *grad_p_end,
+                                        semicrf_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the device status word of workspace

@@ -237,6 +237,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
   const size_t o_tmax = take(4);
   const size_t pz = (B * (C * C + K * C) + 2 * B) * 4;  // pcnt | pbad | pdone
   const size_t o_pcnt = take(pz);
+  const size_t o_pd = take(B * d.Tstride * C * 4);
   const size_t o_psum = take(B * (size_t)d.npch * C * 8);
   const size_t o_plab = take(B * (size_t)d.npch * C * 4);
   const size_t o_pscr = take(B * (size_t)d.npch * 8);
@@ -278,6 +279,8 @@ size_t layout(const Dims& d, void* base, WsPtrs* p) {
     p->pbad = p->pcnt + B * (C * C + K * C);
     p->pdone = p->pbad + B;
     p->pzero_bytes = pz;
+    p->pon = p->status + 1;
+    p->pd = reinterpret_cast<float*>(c + o_pd);
   }
   return off;
 }
@@ -413,7 +416,8 @@ int run_chains(const Dims& d, WsPtrs p, const int32_t* lengths, const float* tra
 }
 
 int run_prefix(const float* em, const int32_t* lengths, const Dims& d, const WsPtrs& p,
-               unsigned flags, int mode, double* S64, float* nu, cudaStream_t st) {
+               unsigned flags, int mode, double* S64, float* nu, cudaStream_t st,
+               const float* p_start = nullptr, const float* p_end = nullptr) {
   if (d.B == 0 || d.T == 0) return SEMICRF_OK;
   const dim3 grid(d.nchunk, d.B);
   {
@@ -427,7 +431,7 @@ int run_prefix(const float* em, const int32_t* lengths, const Dims& d, const WsP
     ProfScope ps("prefix_scan_kernel", st);
     prefix_scan_kernel<<<grid, 256, sm, st>>>(em, lengths, d, p,
                                               (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, mode,
-                                              S64, nu);
+                                              S64, nu, p_start, p_end);
   }
   return launched();
 }
@@ -466,35 +470,76 @@ extern "C" int semicrf_prefix_center(const float* em, const int32_t* lengths, in
   return run_prefix(em, lengths, d, p, flags, 0, S, nu, st);
 }
 
-extern "C" int semicrf_forward(const float* em, const int32_t* lengths, const float* trans,
-                               const float* dur, int B, int T, int C, int K, unsigned flags,
-                               void* ws, size_t ws_bytes, double* logZ, semicrf_stream_t stream) {
+namespace {
+
+// Status word and projection switch: every forward / decode starts with both
+// cleared; a call with boundary projections then sets the switch, which the
+// kernels of this call and of the backward that consumes it read.
+int reset_status(const WsPtrs& p, bool proj, cudaStream_t st) {
+  if (cudaMemsetAsync(p.status, 0, 2 * sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
+  if (proj && cudaMemsetAsync(p.pon, 1, 1, st) != cudaSuccess) return SEMICRF_ERR_CUDA;
+  return SEMICRF_OK;
+}
+
+int forward_impl(const float* em, const int32_t* lengths, const float* trans, const float* dur,
+                 const float* p_start, const float* p_end, int B, int T, int C, int K,
+                 unsigned flags, void* ws, size_t ws_bytes, double* logZ, cudaStream_t st) {
   if (!lengths || !trans || !dur || !logZ || (B > 0 && T > 0 && !em)) return SEMICRF_ERR_INVALID_ARG;
   Dims d;
   WsPtrs p;
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
+  const bool proj = p_start || p_end;
+  // projections run on the log-domain rings (the exponential-domain kernels
+  // have no projection term)
+  if (proj) flags |= SEMICRF_FLAG_LOG_DOMAIN;
+  if ((rc = reset_status(p, proj, st))) return rc;
   if (B == 0) return SEMICRF_OK;
-  rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
+  rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st, p_start, p_end);
   if (rc) return rc;
   const int nbeta = (flags & SEMICRF_FLAG_FORWARD_ONLY) ? 0 : B;
   return run_chains(d, p, lengths, trans, dur, logZ, B, nbeta, flags, st);
 }
 
-extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, const float* dur,
-                                int B, int T, int C, int K, unsigned flags, void* ws,
-                                size_t ws_bytes, const double* grad_logZ, float* grad_em,
-                                float* grad_trans, float* grad_dur, float* pos_marg,
-                                float* start_marg, float* end_marg, semicrf_stream_t stream) {
+}  // namespace
+
+extern "C" int semicrf_forward(const float* em, const int32_t* lengths, const float* trans,
+                               const float* dur, int B, int T, int C, int K, unsigned flags,
+                               void* ws, size_t ws_bytes, double* logZ, semicrf_stream_t stream) {
+  return forward_impl(em, lengths, trans, dur, nullptr, nullptr, B, T, C, K, flags, ws, ws_bytes,
+                      logZ, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int semicrf_forward_proj(const float* em, const int32_t* lengths, const float* trans,
+                                    const float* dur, const float* p_start, const float* p_end,
+                                    int B, int T, int C, int K, unsigned flags, void* ws,
+                                    size_t ws_bytes, double* logZ, semicrf_stream_t stream) {
+  return forward_impl(em, lengths, trans, dur, p_start, p_end, B, T, C, K, flags, ws, ws_bytes,
+                      logZ, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+int backward_impl(const int32_t* lengths, const float* trans, const float* dur, int B, int T,
+                  int C, int K, unsigned flags, void* ws, size_t ws_bytes,
+                  const double* grad_logZ, float* grad_em, float* grad_trans, float* grad_dur,
+                  float* grad_p_start, float* grad_p_end, float* pos_marg, float* start_marg,
+                  float* end_marg, bool proj, cudaStream_t st) {
   if (!lengths || !trans || !dur || !grad_trans || !grad_dur || (B > 0 && T > 0 && !grad_em))
     return SEMICRF_ERR_INVALID_ARG;
   Dims d;
   WsPtrs p;
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (proj) flags |= SEMICRF_FLAG_LOG_DOMAIN;  // as the forward with projections ran
+  const bool want_pg = (grad_p_start || grad_p_end) && T > 0;
+  if (want_pg) {
+    // the projection gradients are g times the boundary marginals; without
+    // caller buffers those go to the exponential-domain rows of the
+    // workspace, which a run with projections does not use
+    if (!start_marg) start_marg = p.kv;
+    if (!end_marg) end_marg = p.kv + (size_t)B * (T + 1) * C;
+  }
   if (B == 0) {
     if (cudaMemsetAsync(grad_trans, 0, (size_t)C * C * 4, st) != cudaSuccess ||
         cudaMemsetAsync(grad_dur, 0, (size_t)K * C * 4, st) != cudaSuccess)
@@ -556,7 +601,14 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
     }
     rc = launched();
     if (!side_join(ss, st)) return SEMICRF_ERR_CUDA;
-    return rc_red ? rc_red : rc;
+    if (rc_red || rc) return rc_red ? rc_red : rc;
+    if (want_pg) {
+      ProfScope ps("proj_grad_kernel", st);
+      if (launch_proj_grad(d, lengths, grad_logZ, start_marg, end_marg, grad_p_start, grad_p_end,
+                           st) != cudaSuccess)
+        return SEMICRF_ERR_CUDA;
+    }
+    return SEMICRF_OK;
   } else {
     // T == 0: only boundary row 0 exists, and nothing starts or ends there
     if (start_marg && cudaMemsetAsync(start_marg, 0, (size_t)B * C * 4, st) != cudaSuccess)
@@ -573,23 +625,50 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
   return launched();
 }
 
-extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const float* trans,
-                               const float* dur, int B, int T, int C, int K, unsigned flags,
-                               void* ws, size_t ws_bytes, double* score, int32_t* labels,
-                               uint8_t* seg_start, semicrf_stream_t stream) {
+}  // namespace
+
+extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, const float* dur,
+                                int B, int T, int C, int K, unsigned flags, void* ws,
+                                size_t ws_bytes, const double* grad_logZ, float* grad_em,
+                                float* grad_trans, float* grad_dur, float* pos_marg,
+                                float* start_marg, float* end_marg, semicrf_stream_t stream) {
+  return backward_impl(lengths, trans, dur, B, T, C, K, flags, ws, ws_bytes, grad_logZ, grad_em,
+                       grad_trans, grad_dur, nullptr, nullptr, pos_marg, start_marg, end_marg,
+                       false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int semicrf_backward_proj(const int32_t* lengths, const float* trans, const float* dur,
+                                     int B, int T, int C, int K, unsigned flags, void* ws,
+                                     size_t ws_bytes, const double* grad_logZ, float* grad_em,
+                                     float* grad_trans, float* grad_dur, float* grad_p_start,
+                                     float* grad_p_end, float* pos_marg, float* start_marg,
+                                     float* end_marg, semicrf_stream_t stream) {
+  return backward_impl(lengths, trans, dur, B, T, C, K, flags, ws, ws_bytes, grad_logZ, grad_em,
+                       grad_trans, grad_dur, grad_p_start, grad_p_end, pos_marg, start_marg,
+                       end_marg, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+int viterbi_impl(const float* em, const int32_t* lengths, const float* trans, const float* dur,
+                 const float* p_start, const float* p_end, int B, int T, int C, int K,
+                 unsigned flags, void* ws, size_t ws_bytes, double* score, int32_t* labels,
+                 uint8_t* seg_start, cudaStream_t st) {
   if (!lengths || !trans || !dur || !score || (B > 0 && T > 0 && (!em || !labels || !seg_start)))
     return SEMICRF_ERR_INVALID_ARG;
   Dims d;
   WsPtrs p;
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
+  const bool proj = p_start || p_end;
+  if ((rc = reset_status(p, proj, st))) return rc;
   if (B == 0) return SEMICRF_OK;
-  rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st);
+  rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st, p_start, p_end);
   if (rc) return rc;
   cudaError_t e;
-  if (d.xG) {
+  // the pipelined decoder has no projection term: with projections the
+  // one-role kernel decodes
+  if (d.xG && !proj) {
     {
       ProfScope ps("viterbi_pipe_kernel", st);
       e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st);
@@ -610,12 +689,33 @@ extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const fl
   return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
 }
 
-extern "C" int semicrf_path_score(const float* em, const int32_t* lengths, const float* trans,
-                                  const float* dur, const int32_t* labels,
-                                  const uint8_t* seg_start, int B, int T, int C, int K,
-                                  unsigned flags, void* ws, size_t ws_bytes,
-                                  const double* grad_score, double* score, float* grad_em,
-                                  float* grad_trans, float* grad_dur, semicrf_stream_t stream) {
+}  // namespace
+
+extern "C" int semicrf_viterbi(const float* em, const int32_t* lengths, const float* trans,
+                               const float* dur, int B, int T, int C, int K, unsigned flags,
+                               void* ws, size_t ws_bytes, double* score, int32_t* labels,
+                               uint8_t* seg_start, semicrf_stream_t stream) {
+  return viterbi_impl(em, lengths, trans, dur, nullptr, nullptr, B, T, C, K, flags, ws, ws_bytes,
+                      score, labels, seg_start, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int semicrf_viterbi_proj(const float* em, const int32_t* lengths, const float* trans,
+                                    const float* dur, const float* p_start, const float* p_end,
+                                    int B, int T, int C, int K, unsigned flags, void* ws,
+                                    size_t ws_bytes, double* score, int32_t* labels,
+                                    uint8_t* seg_start, semicrf_stream_t stream) {
+  return viterbi_impl(em, lengths, trans, dur, p_start, p_end, B, T, C, K, flags, ws, ws_bytes,
+                      score, labels, seg_start, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+int path_score_impl(const float* em, const int32_t* lengths, const float* trans, const float* dur,
+                    const float* p_start, const float* p_end, const int32_t* labels,
+                    const uint8_t* seg_start, int B, int T, int C, int K, unsigned flags, void* ws,
+                    size_t ws_bytes, const double* grad_score, double* score, float* grad_em,
+                    float* grad_trans, float* grad_dur, float* grad_p_start, float* grad_p_end,
+                    cudaStream_t st) {
   if (!lengths || !trans || !dur || (B > 0 && T > 0 && (!em || !labels || !seg_start)))
     return SEMICRF_ERR_INVALID_ARG;
   Dims d;
@@ -623,21 +723,47 @@ extern "C" int semicrf_path_score(const float* em, const int32_t* lengths, const
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
   if (B == 0) return SEMICRF_OK;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const unsigned center = (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u;
   if (cudaMemsetAsync(p.pcnt, 0, p.pzero_bytes, st) != cudaSuccess) return SEMICRF_ERR_CUDA;
   cudaError_t e;
   {
     ProfScope ps("path_terms_kernel", st);
     e = launch_path_terms(d, p, em, lengths, trans, dur, labels, seg_start, center, grad_score,
-                          (flags & SEMICRF_FLAG_NEGATE_GRAD) ? 1 : 0, score, st);
+                          (flags & SEMICRF_FLAG_NEGATE_GRAD) ? 1 : 0, score, p_start, p_end, st);
   }
   if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
-  if (grad_em || grad_trans || grad_dur) {
+  if (grad_em || grad_trans || grad_dur || grad_p_start || grad_p_end) {
     ProfScope ps("path_grad_kernel", st);
-    e = launch_path_grad(d, p, lengths, labels, grad_em, grad_trans, grad_dur, st);
+    e = launch_path_grad(d, p, lengths, labels, seg_start, grad_em, grad_trans, grad_dur,
+                         grad_p_start, grad_p_end, st);
   }
   return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int semicrf_path_score(const float* em, const int32_t* lengths, const float* trans,
+                                  const float* dur, const int32_t* labels,
+                                  const uint8_t* seg_start, int B, int T, int C, int K,
+                                  unsigned flags, void* ws, size_t ws_bytes,
+                                  const double* grad_score, double* score, float* grad_em,
+                                  float* grad_trans, float* grad_dur, semicrf_stream_t stream) {
+  return path_score_impl(em, lengths, trans, dur, nullptr, nullptr, labels, seg_start, B, T, C, K,
+                         flags, ws, ws_bytes, grad_score, score, grad_em, grad_trans, grad_dur,
+                         nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int semicrf_path_score_proj(const float* em, const int32_t* lengths, const float* trans,
+                                       const float* dur, const float* p_start, const float* p_end,
+                                       const int32_t* labels, const uint8_t* seg_start, int B,
+                                       int T, int C, int K, unsigned flags, void* ws,
+                                       size_t ws_bytes, const double* grad_score, double* score,
+                                       float* grad_em, float* grad_trans, float* grad_dur,
+                                       float* grad_p_start, float* grad_p_end,
+                                       semicrf_stream_t stream) {
+  return path_score_impl(em, lengths, trans, dur, p_start, p_end, labels, seg_start, B, T, C, K,
+                         flags, ws, ws_bytes, grad_score, score, grad_em, grad_trans, grad_dur,
+                         grad_p_start, grad_p_end, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int semicrf_get_status(const void* ws, semicrf_stream_t stream, int* status) {

@@ -15,6 +15,8 @@
 // gradient is g_b * (pos_marg[u,c] - mean_v pos_marg[v,c]) (the Jacobian of
 // subtracting the per-label mean; "Emission Baseline Centering", explainer
 // section 2).
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace semicrf {
@@ -117,6 +119,45 @@ __global__ void __launch_bounds__(RP_E * RP_S)
     else
       grad_dur[e - nt] = (float)t;
   }
+}
+
+// Gradients of g_b * log Z_b with respect to the boundary projections
+// ("Streaming Structured Inference with Flash-SemiCRF", explainer section 2,
+// "Boundary Projections"): log Z depends on P_start[b, u, c] through the
+// segments that start at u with label c, and on P_end[b, u, c] through those
+// that end after position u, so
+//   grad_p_start[b, u, c] = g_b * start_marg[b, u, c]
+//   grad_p_end[b, u, c]   = g_b * end_marg[b, u + 1, c]      (u < L_b; else 0).
+__global__ void __launch_bounds__(256) proj_grad_kernel(Dims d, const int32_t* __restrict__ lengths,
+                                                        const double* __restrict__ grad_logZ,
+                                                        const float* __restrict__ start_marg,
+                                                        const float* __restrict__ end_marg,
+                                                        float* __restrict__ grad_p_start,
+                                                        float* __restrict__ grad_p_end) {
+  const int b = blockIdx.y, C = d.C, T = d.T;
+  int L = lengths[b];
+  if (L < 0 || L > T) L = 0;
+  const float g = (float)(grad_logZ ? grad_logZ[b] : 1.0);
+  const size_t n = (size_t)T * C;
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
+    const int u = (int)(i / C);
+    const bool in = u < L;
+    const size_t o = (size_t)b * n + i;
+    const size_t m = (size_t)b * (T + 1) * C + i;  // row u of the [T+1] marginals
+    if (grad_p_start) grad_p_start[o] = in ? g * start_marg[m] : 0.f;
+    if (grad_p_end) grad_p_end[o] = in ? g * end_marg[m + C] : 0.f;
+  }
+}
+
+cudaError_t launch_proj_grad(const Dims& d, const int32_t* lengths, const double* grad_logZ,
+                             const float* start_marg, const float* end_marg, float* grad_p_start,
+                             float* grad_p_end, cudaStream_t st) {
+  if (d.T == 0 || d.B == 0) return cudaSuccess;
+  const size_t n = (size_t)d.T * d.C;
+  const int gx = (int)std::min<size_t>((n + 255) / 256, 1024);
+  proj_grad_kernel<<<dim3(gx, d.B), 256, 0, st>>>(d, lengths, grad_logZ, start_marg, end_marg,
+                                                 grad_p_start, grad_p_end);
+  return cudaGetLastError();
 }
 
 }  // namespace semicrf

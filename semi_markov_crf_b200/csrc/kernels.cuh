@@ -29,7 +29,8 @@ __global__ void prefix_reduce_kernel(const float* __restrict__ em, const int32_t
                                      Dims d, WsPtrs ws);
 __global__ void prefix_scan_kernel(const float* __restrict__ em, const int32_t* __restrict__ lengths,
                                    Dims d, WsPtrs ws, unsigned center, int mode,
-                                   double* __restrict__ S64, float* __restrict__ nu_out);
+                                   double* __restrict__ S64, float* __restrict__ nu_out,
+                                   const float* __restrict__ p_start, const float* __restrict__ p_end);
 
 __global__ void finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                           const double* __restrict__ grad_logZ, unsigned center,
@@ -131,6 +132,12 @@ cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* len
                              const float* trans, const float* dur, double* logZ_out, int n_alpha,
                              int n_beta, cudaStream_t st);
 
+// g_b times the boundary marginals as the boundary-projection gradients
+// (finalize.cu); start_marg / end_marg are [B][T+1][C].
+cudaError_t launch_proj_grad(const Dims& d, const int32_t* lengths, const double* grad_logZ,
+                             const float* start_marg, const float* end_marg, float* grad_p_start,
+                             float* grad_p_end, cudaStream_t st);
+
 // Score of given segmentations and its gradient (path.cu).  The caller zeroes
 // the ws.pzero_bytes region at ws.pcnt first.  The terms pass writes score[b]
 // (nullable) and the weights; the gradient pass adds into the non-null outputs.
@@ -138,9 +145,10 @@ cudaError_t launch_path_terms(const Dims& d, const WsPtrs& ws, const float* em,
                               const int32_t* lengths, const float* trans, const float* dur,
                               const int32_t* labels, const uint8_t* seg_start, unsigned center,
                               const double* grad_score, int negate, double* score,
-                              cudaStream_t st);
+                              const float* p_start, const float* p_end, cudaStream_t st);
 cudaError_t launch_path_grad(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                             const int32_t* labels, float* grad_em, float* grad_trans,
-                             float* grad_dur, cudaStream_t st);
+                             const int32_t* labels, const uint8_t* seg_start, float* grad_em,
+                             float* grad_trans, float* grad_dur, float* grad_p_start,
+                             float* grad_p_end, cudaStream_t st);
 
 }  // namespace semicrf

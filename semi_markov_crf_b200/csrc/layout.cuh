@@ -94,6 +94,12 @@ struct WsPtrs {
   double* pw;      // [B] gradient weight (0 for a malformed path)
   int32_t* pbad;   // [B] malformed-path bits
   int32_t* pdone;  // [B] chunks of the sequence finished (the last one reduces)
+  // Boundary projections: pd[b][t][c] = P_end[t-1, c] + P_start[t, c] in
+  // base-2 units (the start side of boundary t; the end side P_end[t-1] is
+  // folded into the stored prefix sums), read when *pon != 0 (pon is the
+  // word after the status word, cleared with it by every forward / decode).
+  int* pon;
+  float* pd;       // [B][Tstride][C]
   size_t pzero_bytes;
 };
 

@@ -119,7 +119,7 @@ extern "C" int semicrf_forward_noalloc(const float* em, const int32_t* lengths, 
       return SEMICRF_ERR_CUDA;
     prefix_scan_kernel<<<grid, 256, sm, st>>>(em, lengths, d, p,
                                               (flags & SEMICRF_FLAG_NO_CENTER) ? 0u : 1u, 1,
-                                              nullptr, nullptr);
+                                              nullptr, nullptr, nullptr, nullptr);
     if (cudaGetLastError() != cudaSuccess) return SEMICRF_ERR_CUDA;
   }
   // exponential-domain ring where the scores allow it, log domain for the rest

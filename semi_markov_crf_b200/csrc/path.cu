@@ -67,7 +67,8 @@ __global__ void __launch_bounds__(PT_THREADS) path_terms_kernel(
     const float* __restrict__ trans, const float* __restrict__ dur,
     const int32_t* __restrict__ labels, const uint8_t* __restrict__ seg_start, Dims d,
     WsPtrs ws, unsigned center, const double* __restrict__ grad_score, int negate,
-    double* __restrict__ score) {
+    double* __restrict__ score, const float* __restrict__ p_start,
+    const float* __restrict__ p_end) {
   const int b = blockIdx.y, j = blockIdx.x, tid = threadIdx.x;
   const int C = d.C, K = d.K, T = d.T;
   const int L = lengths[b];
@@ -136,6 +137,9 @@ __global__ void __launch_bounds__(PT_THREADS) path_terms_kernel(
       if (u > 0 && !st && yp != y) bad |= PB_CHANGE;
       acc = (double)eb[(size_t)u * C + y];
       atomicAdd(&cnt[y], 1);
+      // boundary projections: a segment's first and last positions
+      if (p_start && st) acc += (double)p_start[((size_t)b * T + u) * C + y];
+      if (p_end && (u + 1 >= L || fl[tid + 1])) acc += (double)p_end[((size_t)b * T + u) * C + y];
       if (st) {
         // Duration: distance to the next start, or to the end of the sequence.
         int k = 0;
@@ -201,14 +205,17 @@ __global__ void __launch_bounds__(PT_THREADS) path_terms_kernel(
   }
 }
 
-// grad_em[b, u, c] += w_b * ([y_u = c] - n_c / L) for u < L_b, four elements
+// grad_em[b, u, c] += w_b * ([y_u = c] - n_c / L) for u < L_b (and, with
+// boundary projections, grad_p_start / grad_p_end += w_b at each segment's
+// first / last position and label), four elements
 // per thread (blocks [0, nbe)); then grad_trans[c', c] += sum_b w_b *
 // (#c' -> c transitions of path b) and grad_dur[k-1, c] += sum_b w_b *
 // (#label-c segments of length k) in a fixed order (blocks [nbe, gridDim.x)).
 __global__ void __launch_bounds__(PT_THREADS) path_grad_kernel(
-    const int32_t* __restrict__ lengths, const int32_t* __restrict__ labels, Dims d, WsPtrs ws,
-    float* __restrict__ grad_em, float* __restrict__ grad_trans, float* __restrict__ grad_dur,
-    int nbe) {
+    const int32_t* __restrict__ lengths, const int32_t* __restrict__ labels,
+    const uint8_t* __restrict__ seg_start, Dims d, WsPtrs ws, float* __restrict__ grad_em,
+    float* __restrict__ grad_trans, float* __restrict__ grad_dur, float* __restrict__ grad_p_start,
+    float* __restrict__ grad_p_end, int nbe) {
   const int C = d.C, K = d.K, T = d.T;
   if ((int)blockIdx.x < nbe) {
     const size_t per_seq = (size_t)T * C;
@@ -223,8 +230,11 @@ __global__ void __launch_bounds__(PT_THREADS) path_grad_kernel(
       const int L = __ldg(lengths + b);
       const double w = ws.pw[b];
       if (u >= L || w == 0.0) continue;
-      const double v = ((labels[(size_t)b * T + u] == c) ? 1.0 : 0.0) - ws.pfr[(size_t)b * C + c];
-      grad_em[i] += (float)(w * v);
+      const bool is_y = labels[(size_t)b * T + u] == c;
+      if (grad_em) grad_em[i] += (float)(w * ((is_y ? 1.0 : 0.0) - ws.pfr[(size_t)b * C + c]));
+      if (is_y && grad_p_start && seg_start[(size_t)b * T + u]) grad_p_start[i] += (float)w;
+      if (is_y && grad_p_end && (u + 1 >= L || seg_start[(size_t)b * T + u + 1]))
+        grad_p_end[i] += (float)w;
     }
     return;
   }
@@ -253,22 +263,26 @@ cudaError_t launch_path_terms(const Dims& d, const WsPtrs& ws, const float* em,
                               const int32_t* lengths, const float* trans, const float* dur,
                               const int32_t* labels, const uint8_t* seg_start, unsigned center,
                               const double* grad_score, int negate, double* score,
-                              cudaStream_t st) {
+                              const float* p_start, const float* p_end, cudaStream_t st) {
   path_terms_kernel<<<dim3(d.npch, d.B), PT_THREADS, 0, st>>>(
-      em, lengths, trans, dur, labels, seg_start, d, ws, center, grad_score, negate, score);
+      em, lengths, trans, dur, labels, seg_start, d, ws, center, grad_score, negate, score, p_start,
+      p_end);
   return cudaGetLastError();
 }
 
 cudaError_t launch_path_grad(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                             const int32_t* labels, float* grad_em, float* grad_trans,
-                             float* grad_dur, cudaStream_t st) {
+                             const int32_t* labels, const uint8_t* seg_start, float* grad_em,
+                             float* grad_trans, float* grad_dur, float* grad_p_start,
+                             float* grad_p_end, cudaStream_t st) {
   const size_t nem = (size_t)d.B * d.T * d.C;
-  const int nbe = grad_em ? (int)((nem + 4 * PT_THREADS - 1) / (4 * PT_THREADS)) : 0;
+  const bool per_pos = grad_em || grad_p_start || grad_p_end;
+  const int nbe = per_pos ? (int)((nem + 4 * PT_THREADS - 1) / (4 * PT_THREADS)) : 0;
   const int nall = d.C * d.C + d.K * d.C;
   const int nbp = (grad_trans || grad_dur) ? (nall + 31) / 32 : 0;
   if (nbe + nbp == 0) return cudaSuccess;
-  path_grad_kernel<<<nbe + nbp, PT_THREADS, 0, st>>>(lengths, labels, d, ws, grad_em, grad_trans,
-                                                     grad_dur, nbe);
+  path_grad_kernel<<<nbe + nbp, PT_THREADS, 0, st>>>(lengths, labels, seg_start, d, ws, grad_em,
+                                                     grad_trans, grad_dur, grad_p_start,
+                                                     grad_p_end, nbe);
   return cudaGetLastError();
 }
 

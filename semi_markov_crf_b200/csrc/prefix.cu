@@ -49,7 +49,9 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
                                                           const int32_t* __restrict__ lengths,
                                                           Dims d, WsPtrs ws, unsigned center,
                                                           int mode, double* __restrict__ S64,
-                                                          float* __restrict__ nu_out) {
+                                                          float* __restrict__ nu_out,
+                                                          const float* __restrict__ p_start,
+                                                          const float* __restrict__ p_end) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int b = blockIdx.y, j = blockIdx.x;
   const int C = d.C, R = d.prefR, T = d.T;
@@ -130,9 +132,17 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
       if (mode == 0) {
         S64[((size_t)b * (T + 1) + t) * C + c] = valid ? val : 0.0;
       } else {
-        const double s2 = valid ? val * LOG2E_D : 0.0;
-        const double ip = rint(s2);
         const size_t o = ((size_t)b * d.Tstride + t) * C + c;
+        double pe = 0.0;
+        if (p_start || p_end) {
+          // boundary projections: P_end[t-1] joins S[t]; pd[t] is the start side
+          const size_t q = ((size_t)b * T + (t - 1)) * C + c;
+          pe = (valid && p_end) ? (double)__ldg(p_end + q) : 0.0;
+          const double ps = (t < L && p_start) ? (double)__ldg(p_start + q + C) : 0.0;
+          ws.pd[o] = (float)((pe + ps) * LOG2E_D);
+        }
+        const double s2 = valid ? (val + pe) * LOG2E_D : 0.0;
+        const double ip = rint(s2);
         ws.sint[o] = (int32_t)ip;
         ws.sfrac[o] = (float)(s2 - ip);
       }
@@ -144,6 +154,8 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
         const size_t o = ((size_t)b * d.Tstride) * C + c;
         ws.sint[o] = 0;
         ws.sfrac[o] = 0.f;
+        if (p_start || p_end)
+          ws.pd[o] = (p_start && L > 0) ? (float)((double)__ldg(p_start + (size_t)b * T * C + c) * LOG2E_D) : 0.f;
       }
     }
   }

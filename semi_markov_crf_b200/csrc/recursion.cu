@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(LB, 1)
   ln.init_dur(d, dur, is_alpha);
   float2* const rl = sm.ring + (size_t)ln.cc * d.RL;  // this lane's label ring
   float e[KBT], p[CAT];
+  const bool pj = proj_on(ws);  // boundary projections
   init_smem(sm, d);
   __syncthreads();
   ln.init_trans(d, trans, !is_alpha, block_trans_max(sm, d, trans));
@@ -222,7 +223,8 @@ __global__ void __launch_bounds__(LB, 1)
   if (is_alpha) {
     // ---------------------------------------------------------------- forward
     for (int c = tid; c < C; c += blockDim.x) {
-      ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));  // boundary 0
+      ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0,
+                    make_float2(proj_d(ws, d, pj, b, 0, c), 0.f));  // boundary 0
       sm.Sbase[c] = 0;
     }
     tile_start(sm, d, ws, b, ts, 1, 1, L, +1);
@@ -291,7 +293,8 @@ __global__ void __launch_bounds__(LB, 1)
         const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
-          ring_put<KBT>(rl, d, wslot, make_float2(g - sf, (Frel + n) - (float)(si - Sb)));
+          ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
+                                                  (Frel + n) - (float)(si - Sb)));
         }
         __syncwarp();
         Frel += n;
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(LB, 1)
         float ssum;
         const float lse =
             k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
-        const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
+        const float Bt = (lse == NEG_INF) ? NEG_INF : (lse - sf) + proj_d(ws, d, pj, b, s, ln.cc);
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = Bt;
           sm.pcur[par * PC + ln.c] = ex2(Bt);
@@ -430,6 +433,7 @@ __global__ void __launch_bounds__(LB, 1)
   ln.init_ids(d);
   float2* const rl = sm.ring + (size_t)ln.cc * d.RL;
   float e[KBT], p[CAT];
+  const bool pj = proj_on(ws);  // boundary projections
   TileStream ts;
   ts.ph[0] = ts.ph[1] = 0;
   double F0 = 0.0;
@@ -455,7 +459,7 @@ __global__ void __launch_bounds__(LB, 1)
     int t_start, Sb;
     if (j == 0) {
       for (int c = tid; c < C; c += blockDim.x) {
-        ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));
+        ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(proj_d(ws, d, pj, b, 0, c), 0.f));
         store[c] = NEG_INF;  // no alpha at boundary 0
         store[C + c] = 0.f;  // gamma[0] = 0 in frame 0
       }
@@ -532,7 +536,8 @@ __global__ void __launch_bounds__(LB, 1)
         float* row = store + (size_t)(t - t0) * SW;
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
-          ring_put<KBT>(rl, d, wslot, make_float2(g - sf, (Frel + n) - (float)(si - Sb)));
+          ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
+                                                  (Frel + n) - (float)(si - Sb)));
           row[ln.c] = A;
           row[C + ln.c] = g;
         }
@@ -631,7 +636,7 @@ __global__ void __launch_bounds__(LB, 1)
       const float sf = rf[ln.cc];
       float ksum;
       const float lse = k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
-      const float Bt = (lse == NEG_INF) ? NEG_INF : lse - sf;
+      const float Bt = (lse == NEG_INF) ? NEG_INF : (lse - sf) + proj_d(ws, d, pj, b, s, ln.cc);
       float St = 0.f;
       if (ln.leader) {
         const float Xs = (float)(Xc + (double)row[2 * C + 1] + (double)Grel);

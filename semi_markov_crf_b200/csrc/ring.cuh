@@ -202,6 +202,19 @@ __device__ __forceinline__ void gargmax(float& v, int& i) {
   }
 }
 
+// ----------------------------------------------------------------------------- projections
+// Start-side boundary projection term of boundary t for label c, base-2
+// units ("Streaming Structured Inference with Flash-SemiCRF", explainer
+// section 2, "Boundary Projections"): a segment [s, t) scores
+// P_start[s] + P_end[t-1] on top of its content.  The end side P_end[t-1]
+// is part of the stored prefix sum S'[t] = S[t] + P_end[t-1]; the start side
+// uses S'[s] - pd[s] with pd[s] = P_end[s-1] + P_start[s], so a ring entry
+// (the start role of its boundary) adds pd.  0 when the call has none.
+__device__ __forceinline__ bool proj_on(const WsPtrs& ws) { return ws.pon && *ws.pon != 0; }
+__device__ __forceinline__ float proj_d(const WsPtrs& ws, const Dims& d, bool on, int b, int t, int c) {
+  return on ? ws.pd[((size_t)b * d.Tstride + t) * d.C + c] : 0.f;
+}
+
 // ----------------------------------------------------------------------------- lanes
 
 // One lane of a label group: label c, lane j of G.  Durations of window

@@ -51,10 +51,11 @@ __global__ void __launch_bounds__(LB, 1)
     tr[i] = (ln.act && x < C) ? __ldg(trans + (size_t)x * C + ln.cc) * l2e() : NEG_INF;
   }
   float2* const rl = sm.ring + (size_t)ln.cc * d.RL;
+  const bool pj = proj_on(ws);  // boundary projections
   init_smem(sm, d);
   __syncthreads();
   for (int c = tid; c < C; c += blockDim.x) {
-    ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(0.f, 0.f));
+    ring_put<KBT>(sm.ring + (size_t)c * d.RL, d, 0, make_float2(proj_d(ws, d, pj, b, 0, c), 0.f));
     sm.Sbase[c] = 0;
   }
   __syncthreads();
@@ -154,7 +155,8 @@ __global__ void __launch_bounds__(LB, 1)
         }
         gargmax<G>(best, bc);
         if (ln.leader) {
-          ring_put<KBT>(rl, d, wslot, make_float2((best - n) - sf, (Frel + n) - (float)(si - Sb)));
+          ring_put<KBT>(rl, d, wslot, make_float2(((best - n) - sf) + proj_d(ws, d, pj, b, t, ln.c),
+                                                  (Frel + n) - (float)(si - Sb)));
           bp[(size_t)t * C + ln.c] = (bk & 0xffff) | (bc << 16);
         }
       }

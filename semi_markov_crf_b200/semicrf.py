@@ -25,7 +25,8 @@ KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "ch
            "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
            "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
-           "viterbi_walk_kernel", "path_terms_kernel", "path_grad_kernel")
+           "viterbi_walk_kernel", "path_terms_kernel", "path_grad_kernel",
+           "proj_grad_kernel")
 
 FLAG_NO_CENTER = 0x1
 FLAG_FORWARD_ONLY = 0x2
@@ -53,6 +54,14 @@ lib.semicrf_viterbi.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz
                                 _vp]
 lib.semicrf_path_score.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz,
                                    _vp, _vp, _vp, _vp, _vp, _vp]
+lib.semicrf_forward_proj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz,
+                                     _vp, _vp]
+lib.semicrf_backward_proj.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.semicrf_viterbi_proj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz,
+                                     _vp, _vp, _vp, _vp]
+lib.semicrf_path_score_proj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u,
+                                        _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
@@ -63,6 +72,8 @@ lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
 for _f in ("semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
+           "semicrf_forward_proj", "semicrf_backward_proj", "semicrf_viterbi_proj",
+           "semicrf_path_score_proj",
            "semicrf_selftest_bounded_wait", "semicrf_ring_domains"):
     getattr(lib, _f).restype = _i
 
@@ -117,6 +128,7 @@ class Workspace:
         self.flags = flags
         self.nbytes = workspace_bytes(B, T, C, K, flags)
         self.buf = torch.empty(max(self.nbytes, 256), dtype=torch.uint8, device=device or "cuda")
+        self.proj = False  # the last forward on it had boundary projections
 
     def matches(self, B, T, C, K, flags) -> bool:
         return self.dims == (B, T, C, K) and self.flags == flags
@@ -124,6 +136,15 @@ class Workspace:
     @property
     def ptr(self) -> int:
         return self.buf.data_ptr()
+
+
+def _projections(p_start, p_end, shape, device):
+    for name, t in (("p_start", p_start), ("p_end", p_end)):
+        if t is not None:
+            _need(t, torch.float32, name, device)
+            if tuple(t.shape) != tuple(shape):
+                raise TypeError(f"{name} must have shape {tuple(shape)}")
+    return p_start is not None or p_end is not None
 
 
 def _flags(center: bool, forward_only: bool = False, log_domain: bool = False) -> int:
@@ -148,10 +169,13 @@ def prefix_center(em, lengths, center: bool = True, ws: Workspace | None = None)
 
 
 def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = False,
-            ws: Workspace | None = None, logZ=None, log_domain: bool = False):
+            ws: Workspace | None = None, logZ=None, log_domain: bool = False,
+            p_start=None, p_end=None):
     """Steps 1-2: log Z [B] (float64).  Returns (logZ, workspace); pass the
     workspace to :func:`backward`.  log_domain=True runs every sequence's
-    rings in the log domain (SEMICRF_FLAG_LOG_DOMAIN)."""
+    rings in the log domain (SEMICRF_FLAG_LOG_DOMAIN).  ``p_start`` /
+    ``p_end`` [B,T,C] float32 are boundary projection scores
+    (semicrf_forward_proj)."""
     dev = em.device
     _need(em, torch.float32, "em", dev)
     _need(lengths, torch.int32, "lengths", dev)
@@ -164,8 +188,16 @@ def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = F
         ws = Workspace(B, T, C, K, flags, dev)
     if logZ is None:
         logZ = torch.empty(B, dtype=torch.float64, device=dev)
-    _check(lib.semicrf_forward(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, flags,
-                               ws.ptr, ws.nbytes, _ptr(logZ), _stream(dev)), "semicrf_forward")
+    if _projections(p_start, p_end, (B, T, C), dev):
+        _check(lib.semicrf_forward_proj(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur),
+                                        _ptr(p_start), _ptr(p_end), B, T, C, K, flags, ws.ptr,
+                                        ws.nbytes, _ptr(logZ), _stream(dev)), "semicrf_forward_proj")
+        ws.proj = True
+    else:
+        _check(lib.semicrf_forward(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K,
+                                   flags, ws.ptr, ws.nbytes, _ptr(logZ), _stream(dev)),
+               "semicrf_forward")
+        ws.proj = False
     return logZ, ws
 
 
@@ -175,7 +207,9 @@ def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool
 
     Returns a dict with grad_em [B,T,C], grad_trans [C,C], grad_dur [K,C]
     (float32) and, when ``marginals``, pos_marg [B,T,C], start_marg and
-    end_marg [B,T+1,C].  ``out`` may supply preallocated tensors."""
+    end_marg [B,T+1,C]; after a forward with boundary projections also
+    grad_p_start and grad_p_end [B,T,C] (semicrf_backward_proj).  ``out``
+    may supply preallocated tensors."""
     B, T, C, K = ws.dims
     dev = ws.buf.device
     _need(lengths, torch.int32, "lengths", dev)
@@ -192,6 +226,18 @@ def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool
         o["pos_marg"] = torch.empty((B, T, C), dtype=torch.float32, device=dev)
         o["start_marg"] = torch.empty((B, T + 1, C), dtype=torch.float32, device=dev)
         o["end_marg"] = torch.empty((B, T + 1, C), dtype=torch.float32, device=dev)
+    if ws.proj:
+        for name in ("grad_p_start", "grad_p_end"):
+            if name not in o:
+                o[name] = torch.empty((B, T, C), dtype=torch.float32, device=dev)
+        _check(lib.semicrf_backward_proj(
+            _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, ws.flags, ws.ptr, ws.nbytes,
+            _ptr(grad_logZ), _ptr(o["grad_em"]), _ptr(o["grad_trans"]), _ptr(o["grad_dur"]),
+            _ptr(o["grad_p_start"]), _ptr(o["grad_p_end"]),
+            _ptr(o.get("pos_marg") if marginals else None),
+            _ptr(o.get("start_marg") if marginals else None),
+            _ptr(o.get("end_marg") if marginals else None), _stream(dev)), "semicrf_backward_proj")
+        return o
     _check(lib.semicrf_backward(_ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, ws.flags, ws.ptr,
                                 ws.nbytes, _ptr(grad_logZ), _ptr(o["grad_em"]), _ptr(o["grad_trans"]),
                                 _ptr(o["grad_dur"]), _ptr(o.get("pos_marg") if marginals else None),
@@ -202,9 +248,10 @@ def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool
 
 
 def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None = None,
-            out=None):
+            out=None, p_start=None, p_end=None):
     """Step 4: (score [B] float64, labels [B,T] int32, seg_start [B,T] uint8).
-    ``out`` may supply that triple preallocated."""
+    ``out`` may supply that triple preallocated; ``p_start`` / ``p_end``
+    [B,T,C] are boundary projection scores (semicrf_viterbi_proj)."""
     dev = em.device
     _need(em, torch.float32, "em", dev)
     _need(lengths, torch.int32, "lengths", dev)
@@ -224,15 +271,23 @@ def viterbi(em, lengths, trans, dur, center: bool = True, ws: Workspace | None =
         _need(score, torch.float64, "score", dev)
         _need(labels, torch.int32, "labels", dev)
         _need(seg, torch.uint8, "seg_start", dev)
+    if _projections(p_start, p_end, (B, T, C), dev):
+        _check(lib.semicrf_viterbi_proj(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur),
+                                        _ptr(p_start), _ptr(p_end), B, T, C, K, flags, ws.ptr,
+                                        ws.nbytes, _ptr(score), _ptr(labels), _ptr(seg),
+                                        _stream(dev)), "semicrf_viterbi_proj")
+        ws.proj = True
+        return score, labels, seg
     _check(lib.semicrf_viterbi(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, flags,
                                ws.ptr, ws.nbytes, _ptr(score), _ptr(labels), _ptr(seg), _stream(dev)),
            "semicrf_viterbi")
+    ws.proj = False
     return score, labels, seg
 
 
 def path_score(em, lengths, trans, dur, labels, seg_start, center: bool = True,
                ws: Workspace | None = None, grad_score=None, negate: bool = False,
-               grads: dict | None = None, score=None):
+               grads: dict | None = None, score=None, p_start=None, p_end=None):
     """Score [B] (float64) of given segmentations, NaN where malformed.
 
     ``labels`` [B,T] int32 and ``seg_start`` [B,T] uint8 as :func:`viterbi`
@@ -242,7 +297,9 @@ def path_score(em, lengths, trans, dur, labels, seg_start, center: bool = True,
     ``negate``.  For the NLL log Z - score: :func:`backward` with grad_logZ=g,
     then this call with grad_score=g, negate=True and the same dict.  ``ws``
     may be the workspace of a :func:`forward` with the same sizes (the path
-    score has a region of its own)."""
+    score has a region of its own).  ``p_start`` / ``p_end`` [B,T,C] add the
+    boundary projection terms (semicrf_path_score_proj), and ``grads`` may
+    then also hold grad_p_start / grad_p_end [B,T,C]."""
     dev = em.device
     _need(em, torch.float32, "em", dev)
     _need(lengths, torch.int32, "lengths", dev)
@@ -260,11 +317,21 @@ def path_score(em, lengths, trans, dur, labels, seg_start, center: bool = True,
     if score is None:
         score = torch.empty(B, dtype=torch.float64, device=dev)
     g = {} if grads is None else grads
-    for name, shape in (("grad_em", (B, T, C)), ("grad_trans", (C, C)), ("grad_dur", (K, C))):
+    for name, shape in (("grad_em", (B, T, C)), ("grad_trans", (C, C)), ("grad_dur", (K, C)),
+                        ("grad_p_start", (B, T, C)), ("grad_p_end", (B, T, C))):
         if g.get(name) is not None:
             _need(g[name], torch.float32, name, dev)
             if tuple(g[name].shape) != shape:
                 raise TypeError(f"{name} must have shape {shape}")
+    if _projections(p_start, p_end, (B, T, C), dev) or g.get("grad_p_start") is not None \
+            or g.get("grad_p_end") is not None:
+        _check(lib.semicrf_path_score_proj(
+            _ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), _ptr(p_start), _ptr(p_end),
+            _ptr(labels), _ptr(seg_start), B, T, C, K, flags, ws.ptr, ws.nbytes, _ptr(grad_score),
+            _ptr(score), _ptr(g.get("grad_em")), _ptr(g.get("grad_trans")), _ptr(g.get("grad_dur")),
+            _ptr(g.get("grad_p_start")), _ptr(g.get("grad_p_end")), _stream(dev)),
+            "semicrf_path_score_proj")
+        return score
     _check(lib.semicrf_path_score(_ptr(em), _ptr(lengths), _ptr(trans), _ptr(dur), _ptr(labels),
                                   _ptr(seg_start), B, T, C, K, flags, ws.ptr, ws.nbytes,
                                   _ptr(grad_score), _ptr(score), _ptr(g.get("grad_em")),

@@ -84,7 +84,7 @@ def errors(got, ref):
     return out
 
 
-def assert_viterbi_ok(got, ref, case, center=True, label=""):
+def assert_viterbi_ok(got, ref, case, center=True, label="", p_start=None, p_end=None):
     """Scores agree; paths are bit-exact or, where they differ, the GPU path is
     a valid segmentation whose float64 re-score is optimal within the
     tolerance (a tie in the model, resolved differently by float32 rounding)."""
@@ -94,7 +94,8 @@ def assert_viterbi_ok(got, ref, case, center=True, label=""):
     err = np.abs(got["score"] - sc_r) / np.maximum(1.0, np.abs(sc_r))
     assert np.all(err <= LOGZ_RTOL), f"{label} viterbi score rel err {err.max():.3e}"
     rescored = oracle.path_score(case["em"], lengths, case["trans"], case["dur"], got["labels"],
-                                 got["seg_start"], K=case["dur"].shape[0], center=center)
+                                 got["seg_start"], K=case["dur"].shape[0], center=center,
+                                 p_start=p_start, p_end=p_end)
     n_diff = 0
     for b in range(len(lengths)):
         L = int(lengths[b])

@@ -146,3 +146,43 @@ def test_plain_call_after_a_projection_call_clears_the_switch():
     assert torch.equal(lz0, lz1)
     for k in ref:
         assert torch.equal(ref[k], got[k]), k
+
+
+def test_projections_without_centering_and_forward_only():
+    from semi_markov_crf_b200 import semicrf
+    case = CASES["speech_small"]()
+    B, T, C = case["em"].shape
+    K = case["dur"].shape[0]
+    ps, pe = _proj(case, 54)
+    g = np.linspace(-1.0, 2.0, B)
+    em, lengths, trans, dur = to_dev(case)
+    tp, te = torch.from_numpy(ps).cuda(), torch.from_numpy(pe).cuda()
+    gt = torch.as_tensor(g, device="cuda")
+    ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"], K,
+                                  center=False, grad_logZ=g, p_start=ps, p_end=pe)
+    for fo in (False, True):
+        logZ, ws = semicrf.forward(em, lengths, trans, dur, center=False, forward_only=fo,
+                                   p_start=tp, p_end=te)
+        out = semicrf.backward(ws, lengths, trans, dur, marginals=True, grad_logZ=gt)
+        assert semicrf.get_status(ws) == 0
+        got = {k: v.cpu().numpy() for k, v in out.items()}
+        got["logZ"] = logZ.cpu().numpy()
+        assert_fb_close(got, ref, case["lengths"], f"no_center forward_only={fo}")
+        eps = _masked(g[:, None, None] * ref["start_marg"][:, :T], case["lengths"])
+        assert max_abs(got["grad_p_start"], eps) <= MARG_ATOL
+
+
+def test_projections_with_a_bad_length():
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make_custom(3, 40, 5, 3, seed=3, lengths=[40, 20, 10])
+    ps, pe = _proj(case, 55)
+    case["lengths"] = np.array([40, 41, 10], dtype=np.int32)
+    em, lengths, trans, dur = to_dev(case)
+    logZ, ws = semicrf.forward(em, lengths, trans, dur, p_start=torch.from_numpy(ps).cuda(),
+                               p_end=torch.from_numpy(pe).cuda())
+    out = semicrf.backward(ws, lengths, trans, dur)
+    assert semicrf.get_status(ws) == 6
+    lz = logZ.cpu().numpy()
+    assert np.isnan(lz[1]) and np.isfinite(lz[0]) and np.isfinite(lz[2])
+    assert np.all(out["grad_p_start"][1].cpu().numpy() == 0)
+    assert np.all(out["grad_p_end"][1].cpu().numpy() == 0)

@@ -43,7 +43,7 @@
  *    host before anything is launched.  Device-side conditions (bad lengths,
  *    a bounded wait that gave up) are recorded in the workspace status word,
  *    read with semicrf_get_status.
- *  - Limits of this build: 1 <= C <= 128, T <= 2^26, B <= 2^20, and
+ *  - Limits of the library: 1 <= C <= 128, T <= 2^26, B <= 2^20, and
  *    K <= 2048 (C <= 8), K <= 512 (C <= 16), K <= 256 (C <= 32),
  *    K <= 128 (C <= 64), K <= 64 (C <= 128).  Larger values return
  *    SEMICRF_ERR_UNSUPPORTED.  (Durations up to K = 2000 on sequences of

@@ -801,7 +801,7 @@ extern "C" const char* semicrf_strerror(int code) {
   switch (code) {
     case SEMICRF_OK: return "ok";
     case SEMICRF_ERR_INVALID_ARG: return "invalid argument";
-    case SEMICRF_ERR_UNSUPPORTED: return "unsupported size (above this build's limits)";
+    case SEMICRF_ERR_UNSUPPORTED: return "unsupported size (above the library's limits)";
     case SEMICRF_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case SEMICRF_ERR_CUDA: return "CUDA launch or copy failed";
     case SEMICRF_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";

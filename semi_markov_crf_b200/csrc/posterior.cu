@@ -206,9 +206,9 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, 
 // then every (boundary, label), (duration, label) and (label, label) item is
 // computed from shared memory.  Each thread keeps the duration and transition
 // sums of its first NID / NIT items in registers across tiles (with 512
-// threads that is every item within this build's limits: K C <= 8192, where
-// the log-domain kernels' shared memory ends, and C <= 128); items beyond
-// would add their per-tile sums to the float64 partials.
+// threads that covers K C <= 8192 and C <= 128); the items beyond (long
+// durations: K C up to 16384) add their per-tile sums to the float64
+// partials.
 template <int NID, int NIT>
 __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,

@@ -407,22 +407,28 @@ def run_ours(args):
     graph, launch_mode = None, "eager"
     if not args.no_graph:
         try:
-            ref_logz = logZ.clone()
-            ref_gt = out["grad_trans"].clone()
+            # rank-local outputs of the last eager step (grad_trans / grad_dur
+            # are all-reduced across ranks, the replay below is not)
+            ref_logz, ref_gem = logZ.clone(), out["grad_em"].clone()
             torch.cuda.synchronize(dev)
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, capture_error_mode="relaxed"):
                 lib_step(em, lengths, trans, dur)
             graph.replay()
-            allreduce_param_grads([out["grad_trans"], out["grad_dur"]])
             torch.cuda.synchronize(dev)
             if semicrf.get_status(ws) != 0 or not torch.equal(logZ, ref_logz) \
-                    or not torch.equal(out["grad_trans"], ref_gt):
+                    or not torch.equal(out["grad_em"], ref_gem):
                 raise RuntimeError("graph replay differs from the eager step")
             launch_mode = "cuda graph (the step captured once, replayed)"
         except Exception as exc:  # keep the eager number
             graph = None
             launch_mode = f"eager (graph capture failed: {str(exc).splitlines()[0][:120]})"
+    if world > 1:
+        # every rank times the same way: the graph only if all captured it
+        ok = torch.tensor([1 if graph is not None else 0], dtype=torch.int32, device=dev)
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+        if graph is not None and int(ok.item()) == 0:
+            graph, launch_mode = None, "eager (graph capture failed on another rank)"
     if graph is not None:
         g_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         g_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]

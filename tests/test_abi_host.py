@@ -84,6 +84,36 @@ def test_host_side_argument_errors_launch_nothing(lib):
                                ctypes.c_size_t(1 << 30), fake, None) == 1
 
 
+def test_host_side_argument_errors_of_the_loss_and_projection_calls(lib):
+    vp = ctypes.c_void_p
+    fake = vp(256 * 1024)  # never dereferenced: every call below fails validation first
+    big = ctypes.c_size_t(1 << 30)
+    u0 = ctypes.c_uint(0)
+    # path score: missing labels / workspace too small / unknown flag
+    assert lib.semicrf_path_score(fake, fake, fake, fake, None, fake, 1, 8, 2, 2, u0, fake, big,
+                                  None, fake, None, None, None, None) == 1
+    assert lib.semicrf_path_score(fake, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0, fake,
+                                  ctypes.c_size_t(16), None, fake, None, None, None, None) == 3
+    assert lib.semicrf_path_score(fake, fake, fake, fake, fake, fake, 1, 8, 2, 2,
+                                  ctypes.c_uint(0x40), fake, big, None, fake, None, None, None,
+                                  None) == 1
+    assert lib.semicrf_path_score_proj(fake, None, fake, fake, fake, fake, fake, fake, 1, 8, 2, 2,
+                                       u0, fake, big, None, fake, None, None, None, None, None,
+                                       None) == 1
+    # projection entry points: null inputs, unsupported sizes, misaligned workspace
+    assert lib.semicrf_forward_proj(None, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0, fake, big,
+                                    fake, None) == 1
+    assert lib.semicrf_forward_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 4000, u0, fake,
+                                    big, fake, None) == 2
+    assert lib.semicrf_forward_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0,
+                                    vp(256 * 1024 + 8), big, fake, None) == 1
+    assert lib.semicrf_viterbi_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0, fake, big,
+                                    None, fake, fake, None) == 1
+    assert lib.semicrf_backward_proj(fake, fake, fake, 1, 8, 2, 2, u0, fake, ctypes.c_size_t(16),
+                                     None, fake, fake, fake, None, None, None, None, None,
+                                     None) == 3
+
+
 def test_strerror_names_every_status(lib):
     lib.semicrf_strerror.restype = ctypes.c_char_p
     seen = {lib.semicrf_strerror(i).decode() for i in range(7)}

@@ -215,7 +215,10 @@ SEMICRF_API int semicrf_path_score(const float *em, const int32_t *lengths, cons
  *   (the exponential-domain kernels have no projection term); the workspace
  *   records that projections are on for the backward that consumes it.
  * semicrf_backward_proj: as semicrf_backward, after semicrf_forward_proj on
- *   the same workspace; additionally writes (each nullable)
+ *   the same workspace (a workspace filled by semicrf_forward_proj must be
+ *   consumed by semicrf_backward_proj: under SEMICRF_FLAG_FORWARD_ONLY the
+ *   plain semicrf_backward would run the backward ring without the
+ *   projection terms); additionally writes (each nullable)
  *     grad_p_start [B, T, C] = g_b * start_marg[b, u, c]
  *     grad_p_end   [B, T, C] = g_b * end_marg[b, u + 1, c]   (0 for u >= L_b),
  *   the gradients of g_b * log Z_b.  The marginal outputs stay optional.

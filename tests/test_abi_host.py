@@ -119,3 +119,19 @@ def test_strerror_names_every_status(lib):
     seen = {lib.semicrf_strerror(i).decode() for i in range(7)}
     assert len(seen) == 7 and "unknown status" not in seen
     assert lib.semicrf_strerror(99).decode() == "unknown status"
+
+
+def test_binding_argument_lists_match_the_header():
+    import re
+    torch = pytest.importorskip("torch")  # noqa: F841  (the binding imports it)
+    from semi_markov_crf_b200 import semicrf
+    header = open(os.path.join(ROOT, "include", "semicrf.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    decls = re.findall(r"SEMICRF_API\s+[\w\s\*]+?\b(semicrf_\w+)\s*\(([^;]*?)\)\s*;", header, flags=re.S)
+    assert len(decls) >= 15
+    for name, params in decls:
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        fn = getattr(semicrf.lib, name)
+        if fn.argtypes is None:
+            continue  # declared but not bound by the Python layer
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)

@@ -106,6 +106,28 @@ enum semicrf_status {
 SEMICRF_API int semicrf_workspace_bytes(int B, int T, int C, int K, unsigned flags, size_t *bytes);
 
 /*
+ * Where the workspace bytes go (host-only, launches nothing; no counterpart
+ * on the pages: it itemises the memory the pages' "Memory Complexity
+ * Breakthrough" discussion counts, explainer section 3).  Writes
+ * bytes[i] for i < n, the size of workspace group i below (0 for
+ * i >= SEMICRF_WS_GROUPS); the groups add up to semicrf_workspace_bytes.
+ * Returns the same codes as semicrf_workspace_bytes.
+ */
+enum semicrf_ws_group {
+    SEMICRF_WS_OTHER = 0,        /* status word, log Z, per-sequence flags and bounds */
+    SEMICRF_WS_PREFIX = 1,       /* split prefix sums [B][T+1][C] x 8 bytes, chunk sums */
+    SEMICRF_WS_CHECKPOINTS = 2,  /* ring checkpoints every Delta positions, both directions */
+    SEMICRF_WS_RECOMPUTE = 3,    /* per-segment recompute store and count partials */
+    SEMICRF_WS_VITERBI = 4,      /* decoder rows: chosen durations, V, backpointer words */
+    SEMICRF_WS_KEPT_ROWS = 5,    /* exponential-domain ring values kept per boundary */
+    SEMICRF_WS_PATH = 6,         /* path-score counts and partial sums */
+    SEMICRF_WS_PROJ = 7,         /* boundary-projection start terms */
+    SEMICRF_WS_GROUPS = 8
+};
+SEMICRF_API int semicrf_workspace_itemize(int B, int T, int C, int K, unsigned flags, size_t *bytes,
+                                          int n);
+
+/*
  * Step 1 (explainer section 2, "On-the-Fly Edge Computation via Prefix Sums"
  * and "Emission Baseline Centering"): nu[b, c] = mean of em[b, :L_b, c]
  * (0 with SEMICRF_FLAG_NO_CENTER) and the float64 prefix sums

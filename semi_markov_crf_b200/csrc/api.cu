@@ -201,43 +201,56 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
 namespace {
 
 // Workspace layout; fills `p` when base != nullptr.  Returns total bytes.
-size_t layout(const Dims& d, void* base, WsPtrs* p) {
+size_t layout(const Dims& d, void* base, WsPtrs* p, size_t* groups = nullptr) {
   size_t off = 0;
+  int group = 0;  // SEMICRF_WS_* group of the regions taken next
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = align256(off + bytes);
+    if (groups) groups[group] += off - o;
     return o;
   };
   const size_t B = d.B, C = d.C, K = d.K, nck = d.nck;
+  group = SEMICRF_WS_OTHER;
   const size_t o_status = take(256);
+  group = SEMICRF_WS_PREFIX;
   const size_t o_sint = take(B * d.Tstride * C * 4);
   const size_t o_sfrac = take(B * d.Tstride * C * 4);
   const size_t o_chunk = take(B * d.nchunk * C * 8);
+  group = SEMICRF_WS_OTHER;
   const size_t o_lz = take(B * 8);
   const size_t o_lzb = take(B * 8);
+  group = SEMICRF_WS_CHECKPOINTS;
   const size_t o_ack = take(B * nck * K * C * 8);
   const size_t o_acf = take(B * nck * 8);
   const size_t o_bck = take(B * nck * K * C * 8);
   const size_t o_bcf = take(B * nck * 8);
+  group = SEMICRF_WS_RECOMPUTE;
   const size_t o_store = take(d.store_smem ? 0 : B * nck * (size_t)d.delta * d.store_w * 4);
   const size_t o_pgt = take(B * nck * C * C * 8);
   const size_t o_pgd = take(B * nck * K * C * 8);
   const size_t o_segT = take(B * nck * C * 8);
   const size_t o_segV = take(B * nck * C * 8);
+  group = SEMICRF_WS_VITERBI;
   const size_t o_bp = take(B * (size_t)(d.T + 1) * C * 4);
   const size_t o_vrow = take(d.xG ? B * (size_t)(d.T + 1) * C * 4 : 0);
   const size_t CP = (C + 3) / 4 * 4;
   const size_t o_wrd = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
   const size_t o_wdl = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
+  group = SEMICRF_WS_KEPT_ROWS;
   const size_t o_kv = take(B * 2ull * (d.T + 1) * 2 * C * 4);
   const size_t o_kf = take(B * 2ull * (d.T + 1) * 8);
   const size_t o_ncut = take(B * (size_t)d.ngrid * 8);
+  group = SEMICRF_WS_OTHER;
   const size_t o_emax = take(B * 4);
   const size_t o_mode = take(2 * B * 4);
   const size_t o_tmax = take(4);
   const size_t pz = (B * (C * C + K * C) + 2 * B) * 4;  // pcnt | pbad | pdone
+  group = SEMICRF_WS_PATH;
   const size_t o_pcnt = take(pz);
+  group = SEMICRF_WS_PROJ;
   const size_t o_pd = take(B * d.Tstride * C * 4);
+  group = SEMICRF_WS_PATH;
   const size_t o_psum = take(B * (size_t)d.npch * C * 8);
   const size_t o_plab = take(B * (size_t)d.npch * C * 4);
   const size_t o_pscr = take(B * (size_t)d.npch * 8);
@@ -447,6 +460,18 @@ extern "C" int semicrf_workspace_bytes(int B, int T, int C, int K, unsigned flag
   const int rc = make_dims(B, T, C, K, d);
   if (rc != SEMICRF_OK) return rc;
   *bytes = layout(d, nullptr, nullptr);
+  return SEMICRF_OK;
+}
+
+extern "C" int semicrf_workspace_itemize(int B, int T, int C, int K, unsigned flags,
+                                         size_t* bytes, int n) {
+  if (!bytes || n < 0 || (flags & ~KNOWN_FLAGS)) return SEMICRF_ERR_INVALID_ARG;
+  Dims d;
+  const int rc = make_dims(B, T, C, K, d);
+  if (rc != SEMICRF_OK) return rc;
+  size_t g[SEMICRF_WS_GROUPS] = {};
+  layout(d, nullptr, nullptr, g);
+  for (int i = 0; i < n; ++i) bytes[i] = i < SEMICRF_WS_GROUPS ? g[i] : 0;
   return SEMICRF_OK;
 }
 

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["workspace_bytes", "prefix_center", "forward", "backward", "viterbi", "path_score",
+__all__ = ["workspace_bytes", "workspace_itemize", "WS_GROUPS", "prefix_center", "forward", "backward", "viterbi", "path_score",
            "get_status", "FLAG_NEGATE_GRAD",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
            "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "ring_domains", "profile_enable", "profile_read",
@@ -46,6 +46,7 @@ _u = ctypes.c_uint
 _sz = ctypes.c_size_t
 
 lib.semicrf_workspace_bytes.argtypes = [_i, _i, _i, _i, _u, ctypes.POINTER(_sz)]
+lib.semicrf_workspace_itemize.argtypes = [_i, _i, _i, _i, _u, ctypes.POINTER(_sz), _i]
 lib.semicrf_prefix_center.argtypes = [_vp, _vp, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp]
 lib.semicrf_forward.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
 lib.semicrf_backward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp, _vp,
@@ -70,7 +71,7 @@ lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, 
 lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.POINTER(ctypes.c_int32)]
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
-for _f in ("semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+for _f in ("semicrf_workspace_itemize", "semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
            "semicrf_forward_proj", "semicrf_backward_proj", "semicrf_viterbi_proj",
            "semicrf_path_score_proj",
@@ -102,6 +103,20 @@ def workspace_bytes(B: int, T: int, C: int, K: int, flags: int = 0) -> int:
     n = _sz(0)
     _check(lib.semicrf_workspace_bytes(B, T, C, K, flags, ctypes.byref(n)), "semicrf_workspace_bytes")
     return int(n.value)
+
+
+# workspace groups of semicrf_workspace_itemize, in the header's order
+WS_GROUPS = ("other", "prefix_sums", "checkpoints", "recompute", "viterbi", "kept_rows",
+             "path_score", "projections")
+
+
+def workspace_itemize(B: int, T: int, C: int, K: int, flags: int = 0) -> dict:
+    """Bytes of each workspace group (names of WS_GROUPS); they add up to
+    :func:`workspace_bytes`."""
+    arr = (_sz * len(WS_GROUPS))()
+    _check(lib.semicrf_workspace_itemize(B, T, C, K, flags, arr, len(WS_GROUPS)),
+           "semicrf_workspace_itemize")
+    return {name: int(arr[i]) for i, name in enumerate(WS_GROUPS)}
 
 
 def _stream(device) -> int:

@@ -63,4 +63,4 @@ def test_single_process_helpers_are_identities():
     bench.allreduce_param_grads([t])
     assert t.tolist() == [1.0, 1.0]
     assert bench.edges_of([10, 5], 3, 2) == 15 * 3 * 4
-    assert bench.mufu_ops_per_position("chain_kernel", 30, 39) == 2 * (30 * 39 + 3 * 39)
+    assert bench.algorithmic_ops_per_position("chain_kernel", 30, 39) == (2 * 30 * 39, "mufu")

@@ -1,16 +1,34 @@
-"""Writes the float64 oracle's expected values for the five full-size workloads.
+"""Writes the float64 oracle's expected values for the full-size workloads.
 
-Usage:  python tests/golden/make_golden.py [tiny speech genomic ultra large]
+Usage:  python tests/golden/make_golden.py [genomic ultra large ...]
 
 Calls only the oracle (``oracle/``) on inputs drawn by the seeded generator
 (``semi_markov_crf_b200.synth``), and stores, per workload, in
 ``tests/golden/<name>.npz``:
 
-  logZ [B], grad_trans [C, C], grad_dur [K, C]          exact, in full
-  viterbi_score [B]                                     the optimum
-  sample_b, sample_u [S]                                seeded sampled positions
-  pos_marg, grad_e [S, C]       at (b, u)               sampled outputs
-  start_marg, end_marg [S, C]   at boundary (b, u)
+  logZ [B], logZ_beta [B], grad_trans [C, C], grad_dur [K, C]   in full
+  viterbi_score [B]                                  the optimum
+  viterbi_labels [B, T] int8/int16, viterbi_seg [B, T] packed bits
+                                                     the oracle's decoded path, in full
+  row_b, row_u [R]              targeted positions (b, u), u < L_b
+  q_pos_marg, q_grad_e [R, C]   outputs there
+  brow_b, brow_u [S]            targeted boundaries (b, t), t <= L_b
+  q_start_marg, q_end_marg [S, C]
+                                boundary marginals there
+
+Marginals and emission gradients are stored quantised, round(x * 2^17) as
+int32 (error <= 2^-18, far below the 1e-4 tolerance), so that values near
+zero compress.  The targeted rows are the positions around the points where
+the kernels change state -- both sides of every 8th prefix-sum tile edge
+(multiples of 256) and of every cut-normaliser grid point (multiples of
+128), two rows either side of every checkpoint at the checkpoint spacing
+ceil(sqrt(T K)) and at the library's capped spacing, with the rows K before
+and after each checkpoint (segments that straddle it), and the first and
+last K + 2 rows of each sequence -- plus seeded random rows.  For wide label
+sets (C > 64) only the first and last sequence get the targeted rows.
+
+The tiny and speech workloads are not stored: the GPU tests run the oracle on
+them at test time (seconds) and compare every element.
 
 The GPU parity tests regenerate the same inputs, run the CUDA path at the
 benchmark's launch configuration and compare against these values, so the
@@ -19,6 +37,7 @@ oracle (minutes per workload at these sizes) does not run on the GPU machine.
 
 from __future__ import annotations
 
+import math
 import os
 import sys
 import time
@@ -32,36 +51,87 @@ sys.path.insert(0, ROOT)
 import oracle  # noqa: E402
 from semi_markov_crf_b200 import synth  # noqa: E402
 
-NAMES = ("tiny", "speech", "genomic", "ultra", "large")
+NAMES = ("genomic", "ultra", "large")
+QSCALE = float(1 << 17)
+SMS = 148  # B200: the library's checkpoint cap depends on the SM count
 
 
-def sample_positions(lengths, C, seed):
-    """Seeded (b, u) pairs with 0 <= u < L_b, about 1 MB of samples at most."""
+def spacings(T: int, K: int, B: int):
+    """Checkpoint spacings the rows are aimed at: the pages' ceil(sqrt(T K))
+    and the library's spacing on a 148-SM GPU (capped so the posterior pass
+    is one wave)."""
+    pages = math.isqrt(T * K)
+    if pages * pages < T * K:
+        pages += 1
+    per_seq = max(1, 2 * SMS // max(B, 1))
+    lib = min(pages, max(2 * K, -(-T // per_seq)))
+    return sorted({pages, max(lib, 1)})
+
+
+def target_rows(lengths, T: int, K: int, seed: int, n_random: int, targeted):
+    """Sorted unique (b, u) position rows and (b, t) boundary rows; the
+    sequences in `targeted` get the state-change rows, every sequence the
+    random ones."""
     rng = np.random.default_rng(1000 + seed)
-    n = int(min(4000, max(64, 32000 // C)))
-    bs = rng.integers(0, len(lengths), size=n)
-    us = np.array([rng.integers(0, max(1, int(lengths[b]))) for b in bs], dtype=np.int64)
-    return bs.astype(np.int64), us
+    B = len(lengths)
+    pos_b, pos_u, bnd_b, bnd_u = [], [], [], []
+    for b in range(B):
+        L = int(lengths[b])
+        pts = set()
+        if b in targeted:
+            for p in range(256, L, 256):                  # prefix-sum tile edges (every 8th)
+                pts.update((p - 1, p))
+            for p in range(128, L + 1, 128):              # cut-normaliser grid
+                pts.update((p - 1, p))
+            for s in spacings(T, K, B):                   # checkpoints, and segments across them
+                for p in range(s, L + 1, s):
+                    pts.update(range(p - 2, p + 2))
+                    pts.update((p - K, p - K + 1, p + K - 1, p + K))
+            pts.update(range(0, min(L, K + 2)))
+            pts.update(range(max(0, L - K - 2), L + 1))
+        pts.update(int(x) for x in rng.integers(0, L + 1, size=n_random))
+        rows = sorted(x for x in pts if 0 <= x < L)
+        bnds = sorted(x for x in pts if 0 <= x <= L)
+        pos_b += [b] * len(rows)
+        pos_u += rows
+        bnd_b += [b] * len(bnds)
+        bnd_u += bnds
+    return (np.array(pos_b, np.int32), np.array(pos_u, np.int32),
+            np.array(bnd_b, np.int32), np.array(bnd_u, np.int32))
+
+
+def quantise(x):
+    return np.rint(np.asarray(x, np.float64) * QSCALE).astype(np.int32)
 
 
 def make(name: str):
     w = synth.make(name)
     K = w["dur"].shape[0]
+    B, T, C = w["em"].shape
     t0 = time.time()
     fb = oracle.forward_backward(w["em"], w["lengths"], w["trans"], w["dur"], K)
     vit = oracle.viterbi(w["em"], w["lengths"], w["trans"], w["dur"], K)
     dt = time.time() - t0
-    C = w["em"].shape[2]
-    bs, us = sample_positions(w["lengths"], C, synth.CONFIGS[name].seed)
+    # wide label sets: the state-change rows of the first and last sequence
+    targeted = {0, B - 1} if C > 64 else set(range(B))
+    n_random = 100 if C > 64 else 300
+    rb, ru, bb, bu = target_rows(w["lengths"], T, K, synth.CONFIGS[name].seed, n_random,
+                                 targeted)
+    lab_dtype = np.int8 if C <= 127 else np.int16
     out = dict(
         logZ=fb["logZ"], logZ_beta=fb["logZ_beta"], grad_trans=fb["grad_trans"],
-        grad_dur=fb["grad_dur"], viterbi_score=vit["score"], sample_b=bs, sample_u=us,
-        pos_marg=fb["pos_marg"][bs, us], grad_e=fb["grad_e"][bs, us],
-        start_marg=fb["start_marg"][bs, us], end_marg=fb["end_marg"][bs, us],
-        lengths=w["lengths"], oracle_seconds=np.array(dt))
+        grad_dur=fb["grad_dur"], viterbi_score=vit["score"],
+        viterbi_labels=vit["labels"].astype(lab_dtype),
+        viterbi_seg=np.packbits(vit["seg_start"].astype(np.uint8), axis=1),
+        row_b=rb, row_u=ru, q_pos_marg=quantise(fb["pos_marg"][rb, ru]),
+        q_grad_e=quantise(fb["grad_e"][rb, ru]),
+        brow_b=bb, brow_u=bu, q_start_marg=quantise(fb["start_marg"][bb, bu]),
+        q_end_marg=quantise(fb["end_marg"][bb, bu]),
+        qscale=np.array(QSCALE), lengths=w["lengths"], oracle_seconds=np.array(dt))
     path = os.path.join(HERE, f"{name}.npz")
     np.savez_compressed(path, **out)
-    print(f"{name}: oracle {dt:.1f} s -> {path} ({os.path.getsize(path)} bytes)", flush=True)
+    print(f"{name}: oracle {dt:.1f} s, {len(rb)} position rows, {len(bb)} boundary rows -> "
+          f"{path} ({os.path.getsize(path)} bytes)", flush=True)
 
 
 if __name__ == "__main__":

@@ -128,6 +128,21 @@ SEMICRF_API int semicrf_workspace_itemize(int B, int T, int C, int K, unsigned f
                                           int n);
 
 /*
+ * Launch geometry the library picks for these sizes (host-only diagnostic,
+ * launches nothing; no counterpart on the pages).  Writes shape[i] for
+ * i < n (0 past the fields): CTAs per ring of the exponential-domain rings
+ * and pipelined decoder (0: those kernels do not serve these sizes; 1: one
+ * CTA per ring; more: a thread-block cluster), labels per CTA, combine lanes
+ * per label, weights per combine lane, helper lanes per label, durations per
+ * helper lane, threads per CTA, checkpoint spacing Delta, checkpoint
+ * segments per sequence, posterior tile rows, and the log-domain kernels'
+ * durations per lane, lanes per label, labels per lane and threads per CTA.
+ * Returns the same codes as semicrf_workspace_bytes.
+ */
+#define SEMICRF_SHAPE_FIELDS 14
+SEMICRF_API int semicrf_launch_shape(int B, int T, int C, int K, int32_t *shape, int n);
+
+/*
  * Step 1 (explainer section 2, "On-the-Fly Edge Computation via Prefix Sums"
  * and "Emission Baseline Centering"): nu[b, c] = mean of em[b, :L_b, c]
  * (0 with SEMICRF_FLAG_NO_CENTER) and the float64 prefix sums

@@ -71,13 +71,23 @@ int max_smem_optin() {
 // sequence takes the log-domain kernel).  The step's latency is the longer of
 // the combine path (CAT multiply-adds, log2 G shuffle levels) and the helper
 // path (KBH exponentials, log2 H shuffle levels), plus issue time for the
-// warps that share a scheduler.  SEMICRF_XSHAPE=i forces the i-th fitting
-// shape of the menu (tuning).
+// warps that share a scheduler.  One CTA per ring serves narrow label sets
+// best; from C >= CLUSTER_MIN_C labels a ring is split over a thread-block
+// cluster (N CTAs, C / N labels each): the per-step work of one SM shrinks
+// N-fold and each step pays a cluster barrier (about 500 cycles measured on
+// B200 against about 150 for a CTA barrier), which pays when one SM's step
+// is several thousand cycles (C = 128: about 4300 cycles on one CTA).
+// SEMICRF_XSHAPE=i forces the i-th fitting shape of the menu and
+// SEMICRF_XCLUSTER=n restricts the choice to clusters of n CTAs (tuning).
+constexpr int CLUSTER_MIN_C = 96;
 void choose_xshape(Dims& d, size_t budget) {
   const int C = d.C, K = d.K;
-  int forced = -1;
+  int forced = -1, forced_n = 0;
   if (const char* env = std::getenv("SEMICRF_XSHAPE")) forced = std::atoi(env);
+  if (const char* env = std::getenv("SEMICRF_XCLUSTER")) forced_n = std::atoi(env);
   d.xG = 0;
+  d.xN = 1;
+  d.xCr = C;
   d.pRT = 0;
   double best = 1e30;
   int idx = 0;
@@ -86,15 +96,21 @@ void choose_xshape(Dims& d, size_t budget) {
     while ((1 << l) < v) ++l;
     return l;
   };
-#define SEMICRF_XCONSIDER(g, cat, h, kbh, lb)                                             \
+  const int want_n = forced_n > 0 ? forced_n : 0;
+#define SEMICRF_XCONSIDER(n, g, cat, h, kbh, lb)                                          \
   {                                                                                       \
-    const int nwc = (C + 32 / g - 1) / (32 / g), nwh = (C + 32 / h - 1) / (32 / h);       \
+    const int cr = (C + n - 1) / n;                                                       \
+    const int nwc = (cr + 32 / g - 1) / (32 / g), nwh = (cr + 32 / h - 1) / (32 / h);     \
     const int nt = 32 * (nwc + nwh);                                                      \
-    if (C <= g * cat && K <= h * kbh + 2 && nt <= lb) {                                   \
+    const bool cl_ok = want_n ? (n == want_n) : ((n > 1) == (C >= CLUSTER_MIN_C));        \
+    if (C <= g * cat && K <= h * kbh + 2 && nt <= lb && cl_ok && (n == 1 || cr * n - C < cr)) { \
       const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +        \
-                          10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0);       \
+                          10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0) +      \
+                          (n > 1 ? 100.0 + 10.0 * n : 0.0);                               \
       if ((forced < 0 && cost < best) || forced == idx) {                                 \
         best = cost;                                                                      \
+        d.xN = n;                                                                         \
+        d.xCr = cr;                                                                       \
         d.xG = g;                                                                         \
         d.xCAT = cat;                                                                     \
         d.xH = h;                                                                         \
@@ -117,8 +133,11 @@ void choose_xshape(Dims& d, size_t budget) {
   // the posterior pass from the kept values must fit too
   d.pRT = posterior_tile_rows(d, budget);
   if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget || d.pRT == 0 ||
-      cut_grid_smem_bytes(d) > budget || d.C > 128)
+      cut_grid_smem_bytes(d) > budget || d.C > 128) {
     d.xG = 0;
+    d.xN = 1;
+    d.xCr = C;
+  }
 }
 
 // Sizes, lane mapping and limits.  Returns a semicrf_status.
@@ -460,6 +479,17 @@ extern "C" int semicrf_workspace_bytes(int B, int T, int C, int K, unsigned flag
   const int rc = make_dims(B, T, C, K, d);
   if (rc != SEMICRF_OK) return rc;
   *bytes = layout(d, nullptr, nullptr);
+  return SEMICRF_OK;
+}
+
+extern "C" int semicrf_launch_shape(int B, int T, int C, int K, int32_t* shape, int n) {
+  if (!shape || n < 0) return SEMICRF_ERR_INVALID_ARG;
+  Dims d;
+  const int rc = make_dims(B, T, C, K, d);
+  if (rc != SEMICRF_OK) return rc;
+  const int32_t v[SEMICRF_SHAPE_FIELDS] = {d.xG ? d.xN : 0, d.xCr, d.xG, d.xCAT, d.xH, d.xKBH,
+                                           d.xNT, d.delta, d.nck, d.pRT, d.KBT, d.GB, d.CAT, d.NT};
+  for (int i = 0; i < n; ++i) shape[i] = i < SEMICRF_SHAPE_FIELDS ? v[i] : 0;
   return SEMICRF_OK;
 }
 

@@ -56,20 +56,22 @@ namespace {
 
 constexpr float FAST_BOUND = 60.f;  // log2 units; two steps stay inside fp32's 126
 
+// Per-label arrays cover the CTA's own labels (Cr = xCr of them, local
+// index); P holds the whole label vector in every CTA of a cluster.
 struct XSmem {
-  Smem s;      // mbar, tint, tfrac, ring (tile stream and ring helpers)
-  float* P;    // [2][xPC] exp-domain label vector, by step parity
-  float* Oh;   // [2][C]   k >= 3 sums for the step of that parity (frame Phi_{t-2})
-  float* A1;   // [2][C]   k = 1 factors
-  float* A2;   // [2][C]   k = 2 factors
+  Smem s;      // mbar, tint, tfrac (every label), ring (own labels)
+  float* P;    // [2][xPC] exp-domain label vector, by step parity (all labels)
+  float* Oh;   // [2][Cr]  k >= 3 sums for the step of that parity (frame Phi_{t-2})
+  float* A1;   // [2][Cr]  k = 1 factors
+  float* A2;   // [2][Cr]  k = 2 factors
   float* nsl;  // [2]      frame step n published by the combine warps
   int* aux;    // [4]      block reductions
-  int* Sb;     // [C]      label integer bases of the prefix sums
+  int* Sb;     // [Cr]     label integer bases of the prefix sums
 };
 
 __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   XSmem x;
-  const int C = d.C;
+  const int C = d.C, Cr = d.xCr;  // tile rows hold every label, the rest this CTA's
   unsigned char* p = raw;
   x.s.mbar = reinterpret_cast<uint64_t*>(p);
   x.s.maxslot = reinterpret_cast<int*>(p + 16);
@@ -82,17 +84,17 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   x.s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
   x.s.ring = reinterpret_cast<float2*>(p);
-  p += (size_t)d.xRLP * C * sizeof(float2);
+  p += (size_t)d.xRLP * Cr * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
   float* f = reinterpret_cast<float*>(p);
   x.P = f;
   f += 2 * d.xPC;
   x.Oh = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.A1 = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.A2 = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
@@ -128,27 +130,46 @@ __device__ __forceinline__ int next_mod(int i, int rem) {
 
 // One ring (direction UP: forward over rows 1..L; else backward over rows
 // L-1..0) of sequence b, after the fast-path test has passed.
-template <bool UP, int G, int CAT, int H, int KBH>
+//
+// With a cluster of N > 1 CTAs per ring, CTA `rank` owns labels
+// [rank*Cr, rank*Cr + Cr): its ring, its k fan-in and its label fan-in
+// outputs.  The label fan-in of every label needs the whole vector p_{t-1},
+// so each combine group stores its p_t into the P buffer of every CTA of the
+// cluster (plain distributed-shared-memory stores, the group's lanes taking
+// different destination CTAs) and the step ends with a cluster barrier
+// (release / acquire) instead of the CTA barrier.  Every CTA then holds the
+// same full vector and computes the same frame step n from it.
+template <bool UP, int N, int G, int CAT, int H, int KBH>
 __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPtrs& ws, int b,
                                       int L, const float* __restrict__ trans,
                                       const float* __restrict__ dur, float M,
-                                      double* __restrict__ logZ_out) {
+                                      double* __restrict__ logZ_out, int rank) {
   const Smem& sm = xs.s;
-  const int C = d.C, K = d.K, tid = threadIdx.x;
+  const int C = d.C, K = d.K, Cr = d.xCr, tid = threadIdx.x;
   constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
   constexpr int NR = CAT > KBH ? CAT : KBH;
   constexpr int SG = UP ? 1 : -1;  // walk direction over rows
   const float sg = UP ? 1.f : -1.f;
   const int warp = tid >> 5, lane = tid & 31;
-  const int nwc = (C + LPWC - 1) / LPWC;
+  const int nwc = (Cr + LPWC - 1) / LPWC;
   const bool comb = warp < nwc;
-  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
+  const int c0 = rank * Cr;  // first label of this CTA
+  const int cl = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;  // local label
+  const int c = c0 + cl;     // global label
+  const bool act = cl < Cr && c < C;
+  const int cc = act ? c : 0;     // global label (tile rows, parameters, outputs)
+  const int ccl = act ? cl : 0;   // local label (ring, per-label arrays)
   const int jl = comb ? lane % G : lane % H;
-  const bool act = c < C;
-  const int cc = act ? c : 0;
   const bool leader = act && jl == 0;
   const int RL = K + WL, RLP = d.xRLP;
-  float2* const rl = sm.ring + (size_t)cc * RLP;
+  float2* const rl = sm.ring + (size_t)ccl * RLP;
+  auto step_sync = [&]() {
+    if constexpr (N > 1) {
+      cluster_sync();
+    } else {
+      __syncthreads();
+    }
+  };
   auto put = [&](int slot, float2 v) {  // slot and its mirrors slot + mK < RL
     for (int x = slot; x < RL; x += K) rl[x] = v;
   };
@@ -178,9 +199,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   }
 
   // ---------------------------------------------------------------- shared state
-  for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  for (int i = tid; i < RLP * Cr; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) xs.P[i] = 0.f;
-  for (int i = tid; i < 2 * C; i += blockDim.x) {
+  for (int i = tid; i < 2 * Cr; i += blockDim.x) {
     xs.Oh[i] = 0.f;
     xs.A1[i] = 0.f;
     xs.A2[i] = 0.f;
@@ -201,20 +222,27 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   ts.dir = SG;
   tile_issue(sm, d, ws, b, ts, r0 / TS);
   tile_issue(sm, d, ws, b, ts, r0 / TS + SG);
+  // A wait that gives up records the timeout and drains the copies in
+  // flight.  One CTA returns at once; in a cluster the CTA instead stops
+  // waiting and issuing copies (`dead`) and keeps taking part in the
+  // cluster barriers until the last step, so that no CTA waits for one that
+  // left (its results are then meaningless; the status word says so).
+  bool dead = false;
   bool ok = xtile_wait(sm, ts, r0 / TS);
   if (ok && r1 / TS != r0 / TS) ok = xtile_wait(sm, ts, r1 / TS);
   if (!ok) {
     if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
     tile_drain(sm, ts);
-    return;
+    if constexpr (N == 1) return;
+    dead = true;
   }
   const size_t o0 = tile_row_off(r0, C), o1 = tile_row_off(r1, C);
-  for (int x = tid; x < C; x += blockDim.x) {
+  for (int x = tid; x < Cr && c0 + x < C; x += blockDim.x) {
     // gamma[0] = 0 at S = 0 (forward); beta[L] = 0 at S[L] (backward)
-    const float2 v = make_float2(UP ? 0.f : sm.tfrac[o0 + x], 0.f);
+    const float2 v = make_float2(UP ? 0.f : sm.tfrac[o0 + c0 + x], 0.f);
     float2* r = sm.ring + (size_t)x * RLP;
     for (int y = r0 % K; y < RL; y += K) r[y] = v;
-    xs.Sb[x] = UP ? 0 : sm.tint[o0 + x];
+    xs.Sb[x] = UP ? 0 : sm.tint[o0 + c0 + x];
   }
   // combine state: rows r-1 and r-2 (walk order) of S_int, row r-1 of S_frac,
   // acc and n of the last step, the frame of p_{i-1} relative to F0
@@ -234,7 +262,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   int hbase = UP ? -WL : L + 1;  // window start boundary at step 1
   hbase = ((hbase % K) + K) % K;
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
-    xs.A1[C + c] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
+    xs.A1[Cr + cl] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
   // kept values for the posterior pass: per boundary (row) the vector p and
   // the label fan-in acc, relative to the boundary's frame kf, stored by the
@@ -244,14 +272,16 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   double* const kf = ws.kf ? ws.kf + ((size_t)b * 2 + dir) * (d.T + 1) : nullptr;
   if (kv) {
     const int rL = UP ? L : 0;  // the walk's last row: no label fan-in there
-    for (int x = tid; x < C; x += blockDim.x) {
+    for (int x = c0 + tid; x < c0 + Cr && x < C; x += blockDim.x) {
       kv[(size_t)r0 * 2 * C + x] = 0.f;  // no forward vector at 0, no btil at L
       kv[(size_t)rL * 2 * C + C + x] = 0.f;
     }
-    if (tid == 0) kf[r0] = 0.0;
+    if (tid == 0 && rank == 0) kf[r0] = 0.0;
   }
-  __syncthreads();
-  int Sbc = xs.Sb[cc];
+  // every CTA of a cluster has initialised its P buffer before any other
+  // stores into it
+  step_sync();
+  int Sbc = xs.Sb[ccl];
   // checkpoint steps: forward boundary t = i - 1 at step i; backward
   // boundary t1 = r + 2 at step i
   const int delta = d.delta;
@@ -276,17 +306,18 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
     if (i == next_ev) {
       if (i < L && i % TS == rem_w) {
-        if (!xtile_wait(sm, ts, (r + SG) / TS)) {
+        if (!dead && !xtile_wait(sm, ts, (r + SG) / TS)) {
           if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
           tile_drain(sm, ts);
-          return;
+          if constexpr (N == 1) return;
+          dead = true;
         }
         const size_t o = tile_row_off(r + SG, C);
         hrow_i = sm.tint + o;
         hrow_f = sm.tfrac + o;
       }
       if (i % TS == rem_i) {
-        tile_issue(sm, d, ws, b, ts, r / TS + SG);
+        if (!dead) tile_issue(sm, d, ws, b, ts, r / TS + SG);
         const size_t o = tile_row_off(r, C);
         crow_i = sm.tint + o;
         crow_f = sm.tfrac + o;
@@ -302,7 +333,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
           if (act) {
             const float adj = sg * (float)(sit - Sbc) - D;
             for (int x = jl; x < RL; x += G) rl[x].y += adj;
-            if (leader) xs.Sb[c] = sit;
+            if (leader) xs.Sb[cl] = sit;
           }
         }
         __syncthreads();
@@ -312,21 +343,21 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         } else {
           Fph -= D;
         }
-        Sbc = xs.Sb[cc];
+        Sbc = xs.Sb[ccl];
         next_ck += delta;
         if (UP ? next_ck - 1 >= L : L + 2 - next_ck < delta) next_ck = INT_MAX;
       }
       next_ev = next_event(i);
     }
     // the frame of the row the combine kept last step (Phi_{i-1})
-    if (kv && tid == nwc * 32 && i >= 2) kf[r - SG] = F0 + (double)Fph;
+    if (kv && rank == 0 && tid == nwc * 32 && i >= 2) kf[r - SG] = F0 + (double)Fph;
     // Each role issues its shared-memory reads first and its stores last: a
     // store the compiler cannot separate from later reads keeps those reads
     // from being issued early, and every access of the step must complete
     // before the barrier releases.
     if (comb) {
       // ---------------------------------------------------------- combine
-      const int po = (i & 1) * C + cc;
+      const int po = (i & 1) * Cr + ccl;
       const float a1v = xs.A1[po], a2v = xs.A2[po], ohv = xs.Oh[po];
       const int si_n = crow_i[cc];  // the walk's row r: the next step's ring entry
       const float sf_n = crow_f[cc];
@@ -359,7 +390,13 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float sn = pow2_neg(n);
       const float R = fmaf(acc2, a2v, ohv) * snprev;  // frame Phi_{i-1}
       const float pn = fmaf(acc * sn, a1v, R * sn);
-      if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
+      if constexpr (N > 1) {
+        // into every CTA of the cluster (this one included)
+        if (act)
+          for (int q = jl; q < N; q += G) st_cluster(xs.P + (i & 1) * d.xPC + c, q, pn);
+      } else {
+        if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
+      }
       if (tid == 0) xs.nsl[i & 1] = n;
       // the kept row of this boundary, then the ring entry: global stores
       // after the critical store cost the path least (measured against the
@@ -392,7 +429,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float aO = m + sg * fn;
       const float aA1 = (M + d1) + sg * ((float)(sn - hs_c) + (fn - hf_c));
       const float aA2 = (M + d2) + sg * ((float)(sn - hs_p) + (fn - hf_p));
-      const int o2 = ((i + 1) & 1) * C + c;
+      const int o2 = ((i + 1) & 1) * Cr + ccl;
       if constexpr (H >= 3) {
         const float e = ex2(jl == 0 ? aO : (jl == 1 ? aA1 : aA2));
         if (act && jl == 0) xs.Oh[o2] = (s > 0.f) ? s * e : 0.f;
@@ -414,13 +451,13 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       hrow_f += SG * C;
       hbase = UP ? (hbase + 1 == K ? 0 : hbase + 1) : (hbase == 0 ? K - 1 : hbase - 1);
     }
-    __syncthreads();
+    step_sync();
   }
-  if (kv && tid == nwc * 32)  // the last row's frame (its vector was kept at step L)
+  if (kv && rank == 0 && tid == nwc * 32)  // the last row's frame (its vector was kept at step L)
     kf[UP ? L : 0] = F0 + (double)(Fph + xs.nsl[L & 1]);
 
   // log2 Z = F0 + Phi_L + log2 sum_c p_L[c]
-  if (warp == 0) {
+  if (warp == 0 && rank == 0) {
     float s = 0.f;
     for (int x = lane; x < C; x += 32) s += xs.P[(L & 1) * d.xPC + x];
     s = group_sum(s, 32);
@@ -439,8 +476,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
 }  // namespace
 
 size_t chain_exp_smem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 7ull * d.C) * 4;
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
+         (2ull * d.xPC + 7ull * d.xCr) * 4;
 }
 
 }  // namespace semicrf
@@ -449,12 +486,14 @@ namespace semicrf {
 namespace {
 
 // ===========================================================================
-// One CTA per (direction, sequence): blockIdx.x < n_alpha runs the forward
-// ring of sequence blockIdx.x, the others the backward ring of sequence
-// blockIdx.x - n_alpha.  Writes mode[direction][b]; returns at once (mode 2)
-// when the sequence needs the log-domain kernel.
+// One CTA, or one cluster of N CTAs, per (direction, sequence): ring q =
+// blockIdx.x / N < n_alpha runs the forward ring of sequence q, the others
+// the backward ring of sequence q - n_alpha.  Writes mode[direction][b];
+// returns at once (mode 2) when the sequence needs the log-domain kernel.
+// Every CTA of a cluster takes the same early exits (they depend only on the
+// inputs), before any of them touches another's shared memory.
 // ===========================================================================
-template <int G, int CAT, int H, int KBH, int LB>
+template <int N, int G, int CAT, int H, int KBH, int LB>
 __global__ void __launch_bounds__(LB, 1)
     chain_exp_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                      const float* __restrict__ trans, const float* __restrict__ dur,
@@ -462,12 +501,14 @@ __global__ void __launch_bounds__(LB, 1)
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const XSmem xs = xcarve(smem_raw, d);
   const int C = d.C, K = d.K, tid = threadIdx.x;
-  const bool up = (int)blockIdx.x < n_alpha;
-  const int b = up ? blockIdx.x : blockIdx.x - n_alpha;
+  const int rank = N > 1 ? (int)cluster_ctarank() : 0;
+  const int q = (int)blockIdx.x / N;
+  const bool up = q < n_alpha;
+  const int b = up ? q : q - n_alpha;
   const int L = lengths[b];
   int* const mode = ws.mode + (up ? 0 : d.B) + b;
   if (L < 0 || L > d.T || L == 0) {
-    if (tid == 0) {
+    if (tid == 0 && rank == 0) {
       const double v = (L == 0) ? 0.0 : __longlong_as_double(0x7ff8000000000000ll);
       if (L != 0) set_status(ws.status, ST_BAD_LENGTH);
       if (up) {
@@ -511,21 +552,21 @@ __global__ void __launch_bounds__(LB, 1)
   const float span = fabsf(M) + (M - tmin) + fabsf(dmax) + fabsf(dmin) + 2.f * ws.emax[b] +
                      lg2((float)(K * C));
   if (bad || !(span < FAST_BOUND)) {
-    if (tid == 0) *mode = 2;
+    if (tid == 0 && rank == 0) *mode = 2;
     return;
   }
-  if (tid == 0) *mode = 1;
+  if (tid == 0 && rank == 0) *mode = 1;
   if (up)
-    xring<true, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out);
+    xring<true, N, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out, rank);
   else
-    xring<false, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out);
+    xring<false, N, G, CAT, H, KBH>(xs, d, ws, b, L, trans, dur, M, logZ_out, rank);
 }
 
 }  // namespace
 
-bool xshape_supported(int G, int CAT, int H, int KBH, int LB) {
-#define SEMICRF_XSHAPE_OK(g, cat, h, kbh, lb) \
-  if (G == g && CAT == cat && H == h && KBH == kbh && LB == lb) return true;
+bool xshape_supported(int N, int G, int CAT, int H, int KBH, int LB) {
+#define SEMICRF_XSHAPE_OK(n, g, cat, h, kbh, lb) \
+  if (N == n && G == g && CAT == cat && H == h && KBH == kbh && LB == lb) return true;
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_XSHAPE_OK)
 #undef SEMICRF_XSHAPE_OK
   return false;
@@ -535,18 +576,10 @@ cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* len
                              const float* trans, const float* dur, double* logZ_out, int n_alpha,
                              int n_beta, cudaStream_t st) {
   const size_t sm = chain_exp_smem_bytes(d);
-#define SEMICRF_LAUNCH_XCHAIN(g, cat, h, kbh, lb)                                              \
-  if (d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb) {               \
-    if (sm > 48 * 1024) {                                                                      \
-      const cudaError_t e = cudaFuncSetAttribute(chain_exp_kernel<g, cat, h, kbh, lb>,         \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                                 (int)sm);                                     \
-      if (e != cudaSuccess) return e;                                                          \
-    }                                                                                          \
-    chain_exp_kernel<g, cat, h, kbh, lb><<<n_alpha + n_beta, d.xNT, sm, st>>>(                 \
-        d, ws, lengths, trans, dur, logZ_out, n_alpha);                                        \
-    return cudaGetLastError();                                                                 \
-  }
+#define SEMICRF_LAUNCH_XCHAIN(n, g, cat, h, kbh, lb)                                           \
+  if (d.xN == n && d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb)    \
+    return launch_clustered(chain_exp_kernel<n, g, cat, h, kbh, lb>, n, (n_alpha + n_beta) * n, \
+                            d.xNT, sm, st, d, ws, lengths, trans, dur, logZ_out, n_alpha);
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_XCHAIN)
 #undef SEMICRF_LAUNCH_XCHAIN
   return cudaErrorInvalidConfiguration;

@@ -109,6 +109,33 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// ----------------------------------------------------------------------------- clusters
+// Rank of this CTA in its thread-block cluster.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Cluster-wide barrier: every thread of every CTA of the cluster arrives
+// (release: its earlier shared-memory stores, local or remote, are ordered
+// before) and waits (acquire).  All threads of a warp execute it together.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+
+// Plain store of one float into the shared memory of CTA `rank` of this
+// cluster, at the offset `local` has in this CTA's shared memory (the same
+// carve in every CTA).  No multicast.
+__device__ __forceinline__ void st_cluster(const float* local, uint32_t rank, float v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
 // Bounded wait for phase `parity` of `bar`.  Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int spins) {
   const uint32_t a = smem_addr(bar);

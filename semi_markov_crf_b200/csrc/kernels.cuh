@@ -97,20 +97,53 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(16, 32, 16, 512) X(8, 1, 32, 256) X(16, 1, 32, 512) X(16, 32, 32, 512)              \
   X(64, 1, 32, 256)
 
-// Pipelined exponential-domain rings (chain_exp.cu): shapes (combine lanes
-// per label G, weights per combine lane CAT, helper lanes per label H,
-// durations per helper lane KBH, launch bound LB).  A shape serves C <= G*CAT
-// and K <= H*KBH + 2 with 32*(ceil(C*G/32) + ceil(C*H/32)) <= LB threads
-// (labels never straddle a warp).
+// Pipelined exponential-domain rings (chain_exp.cu) and decoder
+// (viterbi_pipe.cu): shapes (CTAs per ring N, combine lanes per label G,
+// weights per combine lane CAT, helper lanes per label H, durations per
+// helper lane KBH, launch bound LB).  Each CTA owns Cr = ceil(C / N) labels;
+// a shape serves C <= G*CAT and K <= H*KBH + 2 with
+// 32*(ceil(Cr*G/32) + ceil(Cr*H/32)) <= LB threads (labels never straddle a
+// warp).  N > 1 runs each ring on a thread-block cluster of N CTAs.
 #define SEMICRF_FOR_EACH_XSHAPE(X)                                                     \
-  X(1, 8, 1, 8, 64) X(1, 8, 4, 8, 64) X(1, 8, 8, 16, 96) X(1, 8, 16, 16, 160)          \
-  X(1, 8, 32, 16, 288) X(1, 16, 1, 8, 64) X(1, 16, 4, 8, 96) X(1, 16, 8, 16, 160)      \
-  X(1, 16, 16, 16, 288) X(1, 16, 32, 16, 544) X(1, 32, 4, 8, 160) X(1, 32, 8, 16, 288) \
-  X(1, 32, 16, 16, 544) X(2, 24, 4, 8, 288) X(2, 24, 4, 16, 288) X(2, 24, 8, 16, 480) \
-  X(2, 32, 4, 8, 384) X(2, 32, 4, 16, 384) X(2, 32, 8, 16, 640) X(4, 24, 4, 8, 768)   \
-  X(4, 12, 4, 8, 384) X(4, 12, 4, 16, 384) X(2, 48, 2, 32, 384) X(2, 64, 2, 32, 512)  \
-  X(4, 24, 2, 32, 576) X(4, 32, 4, 8, 1024) X(4, 32, 2, 32, 768) X(1, 8, 32, 64, 224) \
-  X(1, 8, 32, 64, 288)
+  X(1, 1, 8, 1, 8, 64) X(1, 1, 8, 4, 8, 64) X(1, 1, 8, 8, 16, 96) X(1, 1, 8, 16, 16, 160)          \
+  X(1, 1, 8, 32, 16, 288) X(1, 1, 16, 1, 8, 64) X(1, 1, 16, 4, 8, 96) X(1, 1, 16, 8, 16, 160)      \
+  X(1, 1, 16, 16, 16, 288) X(1, 1, 16, 32, 16, 544) X(1, 1, 32, 4, 8, 160) X(1, 1, 32, 8, 16, 288) \
+  X(1, 1, 32, 16, 16, 544) X(1, 2, 24, 4, 8, 288) X(1, 2, 24, 4, 16, 288) X(1, 2, 24, 8, 16, 480) \
+  X(1, 2, 32, 4, 8, 384) X(1, 2, 32, 4, 16, 384) X(1, 2, 32, 8, 16, 640) X(1, 4, 24, 4, 8, 768)   \
+  X(1, 4, 12, 4, 8, 384) X(1, 4, 12, 4, 16, 384) X(1, 2, 48, 2, 32, 384) X(1, 2, 64, 2, 32, 512)  \
+  X(1, 4, 24, 2, 32, 576) X(1, 4, 32, 4, 8, 1024) X(1, 4, 32, 2, 32, 768) X(1, 1, 8, 32, 64, 224) \
+  X(1, 1, 8, 32, 64, 288) \
+  X(2, 2, 24, 4, 8, 160) X(2, 4, 32, 4, 16, 512) X(4, 4, 32, 4, 16, 256) X(8, 4, 32, 4, 16, 128)
+
+// Launches `kern` on `grid` CTAs of `threads` threads grouped in clusters of
+// n_cluster CTAs (grid a multiple of n_cluster; n_cluster = 1: a plain
+// launch), with `smem` bytes of dynamic shared memory each.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_clustered(void (*kern)(KArgs...), int n_cluster, int grid, int threads,
+                             size_t smem, cudaStream_t st, Args... args) {
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  if (n_cluster <= 1) {
+    kern<<<grid, threads, smem, st>>>(args...);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = n_cluster;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 size_t chain_exp_smem_bytes(const Dims& d);
 size_t viterbi_pipe_smem_bytes(const Dims& d);
@@ -125,7 +158,7 @@ cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* 
 cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 const float* trans, const float* dur, double* score,
                                 int32_t* labels, uint8_t* seg_start, cudaStream_t st);
-bool xshape_supported(int G, int CAT, int H, int KBH, int LB);
+bool xshape_supported(int N, int G, int CAT, int H, int KBH, int LB);
 // Same grid and outputs as launch_chain for the sequences whose scores fit
 // the exponential domain; writes ws.mode for every (direction, sequence).
 cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* lengths,

@@ -42,6 +42,10 @@ struct Dims {
   // durations each (k = 3..K), xNT threads (launch bound xLB), ring of
   // xRL = K + xKBH entries per label, label vector padded to xPC = xG * xCAT.
   int xG, xCAT, xH, xKBH, xNT, xLB, xRL, xPC;
+  // Thread-block cluster of the pipelined rings: xN CTAs per ring (1: one
+  // CTA), each owning xCr = ceil(C / xN) consecutive labels; the label
+  // vector is exchanged through distributed shared memory every step.
+  int xN, xCr;
   // Pipelined Viterbi (viterbi_pipe.cu): helper lanes stride over a window
   // of xH * xKBH ring entries; the label rows of its ring are xRLP >= K +
   // xH * xKBH entries apart, padded so that a half warp's 64-bit reads of

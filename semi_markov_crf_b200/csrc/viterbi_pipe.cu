@@ -47,21 +47,23 @@ namespace {
 
 constexpr int VREBASE = 4096;  // steps between integer rebases (keeps y exact)
 
+// Per-label arrays cover the CTA's own labels (Cr = xCr of them, local
+// index); V holds the whole row in every CTA of a cluster.
 struct VSmem {
-  Smem s;      // mbar, tint, tfrac, ring
-  float* V;    // [2][xPC]  V of the step of that parity (-inf padded)
-  float* Om;   // [2][C]    helpers' best k >= 3 candidate, frame Phi_{t-2}
-  int* Ok;     // [2][C]    its duration
-  float* A1;   // [2][C]    dur2[0] + S[t] - S[t-1]
-  float* A2;   // [2][C]    dur2[1] + S[t] - S[t-2]
+  Smem s;      // mbar, tint, tfrac (every label), ring (own labels)
+  float* V;    // [2][xPC]  V of the step of that parity (-inf padded, all labels)
+  float* Om;   // [2][Cr]   helpers' best k >= 3 candidate, frame Phi_{t-2}
+  int* Ok;     // [2][Cr]   its duration
+  float* A1;   // [2][Cr]   dur2[0] + S[t] - S[t-1]
+  float* A2;   // [2][Cr]   dur2[1] + S[t] - S[t-2]
   float* nsl;  // [2]       frame step published by the combine warps
   float* mx;   // [2]       max V[t-1] published by the helpers at step t
-  int* Sb;     // [C]       label integer bases
+  int* Sb;     // [Cr]      label integer bases
 };
 
 __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   VSmem x;
-  const int C = d.C;
+  const int C = d.C, Cr = d.xCr;
   unsigned char* p = raw;
   x.s.mbar = reinterpret_cast<uint64_t*>(p);
   x.s.maxslot = reinterpret_cast<int*>(p + 16);
@@ -74,19 +76,19 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   x.s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
   x.s.ring = reinterpret_cast<float2*>(p);
-  p += (size_t)d.xRLP * C * sizeof(float2);
+  p += (size_t)d.xRLP * Cr * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
   float* f = reinterpret_cast<float*>(p);
   x.V = f;
   f += 2 * d.xPC;
   x.Om = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.Ok = reinterpret_cast<int*>(f);
-  f += 2 * C;
+  f += 2 * Cr;
   x.A1 = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.A2 = f;
-  f += 2 * C;
+  f += 2 * Cr;
   x.Sb = reinterpret_cast<int*>(f);
   x.s.pcur = nullptr;
   x.s.Acur = nullptr;
@@ -98,8 +100,8 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.C * 8 + 16 +
-         (2ull * d.xPC + 9ull * d.C) * 4;
+  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
+         (2ull * d.xPC + 9ull * d.xCr) * 4;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -116,7 +118,14 @@ __device__ __forceinline__ int next_with_rem(int i, int rem) {
   return x > i ? x : x + TS;
 }
 
-template <int G, int CAT, int H, int KBH, int LB>
+//
+// With a cluster of N > 1 CTAs per sequence, CTA `rank` owns labels
+// [rank*Cr, rank*Cr + Cr) (ring, k fan-in, label fan-in outputs); each
+// combine group stores its V[t] into the V buffer of every CTA of the
+// cluster (plain distributed-shared-memory stores) and each step ends with a
+// cluster barrier, so every CTA holds the whole row and takes the same frame.
+// Every CTA takes the same early exits (they depend only on the inputs).
+template <int N, int G, int CAT, int H, int KBH, int LB>
 __global__ void __launch_bounds__(LB, 1)
     viterbi_pipe_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                         const float* __restrict__ trans, const float* __restrict__ dur,
@@ -125,17 +134,19 @@ __global__ void __launch_bounds__(LB, 1)
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const VSmem vs = vcarve(smem_raw, d);
   const Smem& sm = vs.s;
-  const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x;
-  const int b = blockIdx.x;
+  const int C = d.C, K = d.K, T = d.T, Cr = d.xCr, tid = threadIdx.x;
+  const int rank = N > 1 ? (int)cluster_ctarank() : 0;
+  const int b = (int)blockIdx.x / N;
   const int L = lengths[b];
   const bool bad = (L < 0 || L > T);
   // positions past the length (all of them for a bad length)
-  for (int u = (bad ? 0 : L) + tid; u < T; u += blockDim.x) {
-    labels[(size_t)b * T + u] = -1;
-    seg_start[(size_t)b * T + u] = 0;
-  }
+  if (rank == 0)
+    for (int u = (bad ? 0 : L) + tid; u < T; u += blockDim.x) {
+      labels[(size_t)b * T + u] = -1;
+      seg_start[(size_t)b * T + u] = 0;
+    }
   if (bad || L == 0) {
-    if (tid == 0) {
+    if (tid == 0 && rank == 0) {
       if (bad) set_status(ws.status, ST_BAD_LENGTH);
       score[b] = bad ? __longlong_as_double(0x7ff8000000000000ll) : 0.0;
     }
@@ -147,15 +158,25 @@ __global__ void __launch_bounds__(LB, 1)
   constexpr int CA = (G * CAT + H - 1) / H;  // labels per lane for the frame max
   constexpr int NR = CAT > KBH ? CAT : KBH;
   const int warp = tid >> 5, lane = tid & 31;
-  const int nwc = (C + LPWC - 1) / LPWC;
+  const int nwc = (Cr + LPWC - 1) / LPWC;
   const bool comb = warp < nwc;
-  const int c = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;
+  const int c0 = rank * Cr;  // first label of this CTA
+  const int cl = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;  // local label
+  const int c = c0 + cl;     // global label
   const int jl = comb ? lane % G : lane % H;
-  const bool act = c < C;
-  const int cc = act ? c : 0;
+  const bool act = cl < Cr && c < C;
+  const int cc = act ? c : 0;     // global label (tile rows, parameters, outputs)
+  const int ccl = act ? cl : 0;   // local label (ring, per-label arrays)
   const bool leader = act && jl == 0;
   const int RL = K + WL, RLP = d.xRLP;
-  float2* const rl = sm.ring + (size_t)cc * RLP;
+  float2* const rl = sm.ring + (size_t)ccl * RLP;
+  auto step_sync = [&]() {
+    if constexpr (N > 1) {
+      cluster_sync();
+    } else {
+      __syncthreads();
+    }
+  };
 
   // combine lanes: trans2[x][c] of their sources x = jl*CAT + q (-inf past C);
   // helper lanes: dur2 of window index q*H + jl, k = 2 + WL - (q*H + jl)
@@ -179,9 +200,9 @@ __global__ void __launch_bounds__(LB, 1)
   }
 
   // ---------------------------------------------------------------- shared state
-  for (int i = tid; i < RLP * C; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
+  for (int i = tid; i < RLP * Cr; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) vs.V[i] = NEG_INF;
-  for (int i = tid; i < 2 * C; i += blockDim.x) {
+  for (int i = tid; i < 2 * Cr; i += blockDim.x) {
     vs.Om[i] = NEG_INF;
     vs.Ok[i] = 3;
     vs.A1[i] = NEG_INF;
@@ -202,13 +223,20 @@ __global__ void __launch_bounds__(LB, 1)
   ts.dir = 1;
   tile_issue(sm, d, ws, b, ts, 0);
   tile_issue(sm, d, ws, b, ts, 1);
+  // A wait that gives up records the timeout and drains the copies in
+  // flight.  One CTA returns at once; in a cluster the CTA instead stops
+  // waiting and issuing copies (`dead`) and keeps taking part in the
+  // cluster barriers until the last step (its results are then meaningless;
+  // the status word says so).
+  bool dead = false;
   if (!vtile_wait(sm, ts, 0)) {
     if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
     tile_drain(sm, ts);
-    return;
+    if constexpr (N == 1) return;
+    dead = true;
   }
   // boundary 0: G = 0 at S = 0, base 0; helpers set step 1's k = 1 constant
-  for (int x = tid; x < C; x += blockDim.x) {
+  for (int x = tid; x < Cr; x += blockDim.x) {
     float2* r = sm.ring + (size_t)x * RLP;
     for (int y = 0; y < RL; y += K) r[y] = make_float2(0.f, 0.f);
     vs.Sb[x] = 0;
@@ -221,7 +249,7 @@ __global__ void __launch_bounds__(LB, 1)
   if (!comb) {
     hs_c = sm.tint[C + cc];  // row 1
     hf_c = sm.tfrac[C + cc];
-    if (leader) vs.A1[1 * C + c] = d1 + ((float)hs_c + hf_c);  // S[1] - S[0]
+    if (leader) vs.A1[1 * Cr + cl] = d1 + ((float)hs_c + hf_c);  // S[1] - S[0]
     hrow_i = sm.tint + 2 * C;  // row 2 for step 1
     hrow_f = sm.tfrac + 2 * C;
   }
@@ -237,7 +265,9 @@ __global__ void __launch_bounds__(LB, 1)
   const float* crow_f = sm.tfrac + C;
   int wslot = 0;
   double F0 = 0.0;
-  __syncthreads();
+  // every CTA of a cluster has initialised its V buffer before any other
+  // stores into it
+  step_sync();
   int Sbc = 0;
   int next_rb = VREBASE + 1;
   // next step with an event: a tile to wait for (row i+1 opens a tile), a
@@ -253,17 +283,18 @@ __global__ void __launch_bounds__(LB, 1)
     if (!comb && i >= 2) Fph += vs.nsl[(i - 1) & 1];
     if (i == next_ev) {
       if (i < L && (i + 1) % TS == 0) {
-        if (!vtile_wait(sm, ts, (i + 1) / TS)) {
+        if (!dead && !vtile_wait(sm, ts, (i + 1) / TS)) {
           if (tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
           tile_drain(sm, ts);
-          return;
+          if constexpr (N == 1) return;
+          dead = true;
         }
         const size_t o = tile_row_off(i + 1, C);
         hrow_i = sm.tint + o;
         hrow_f = sm.tfrac + o;
       }
       if (i % TS == 0) {
-        tile_issue(sm, d, ws, b, ts, i / TS + 1);
+        if (!dead) tile_issue(sm, d, ws, b, ts, i / TS + 1);
         const size_t o = tile_row_off(i, C);
         crow_i = sm.tint + o;
         crow_f = sm.tfrac + o;
@@ -274,7 +305,7 @@ __global__ void __launch_bounds__(LB, 1)
         if (!comb && act) {
           const float adj = (float)(hs_p - Sbc) - D;
           for (int x = jl; x < RL; x += H) rl[x].y += adj;
-          if (leader) vs.Sb[c] = hs_p;
+          if (leader) vs.Sb[cl] = hs_p;
         }
         __syncthreads();
         F0 += (double)D;
@@ -283,7 +314,7 @@ __global__ void __launch_bounds__(LB, 1)
         } else {
           Fph -= D;
         }
-        Sbc = vs.Sb[cc];
+        Sbc = vs.Sb[ccl];
         next_rb += VREBASE;
       }
       next_ev = next_event(i);
@@ -295,10 +326,10 @@ __global__ void __launch_bounds__(LB, 1)
     if (comb) {
       // ---------------------------------------------------------- combine
       const float mp = vs.mx[(i - 1) & 1];
-      const float a1 = vs.A1[(i & 1) * C + cc];
-      const float a2 = vs.A2[(i & 1) * C + cc];
-      const float om = vs.Om[(i & 1) * C + cc];
-      const int okd = vs.Ok[(i & 1) * C + cc];
+      const float a1 = vs.A1[(i & 1) * Cr + ccl];
+      const float a2 = vs.A2[(i & 1) * Cr + ccl];
+      const float om = vs.Om[(i & 1) * Cr + ccl];
+      const int okd = vs.Ok[(i & 1) * Cr + ccl];
       const int si_n = crow_i[cc];  // row i: the next step's ring entry
       const float sf_n = crow_f[cc];
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
@@ -324,7 +355,13 @@ __global__ void __launch_bounds__(LB, 1)
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
       const int kdec = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
-      if (leader) vs.V[(i & 1) * d.xPC + c] = v - n;
+      if constexpr (N > 1) {
+        // into every CTA of the cluster (this one included)
+        if (act)
+          for (int q = jl; q < N; q += G) st_cluster(vs.V + (i & 1) * d.xPC + c, q, v - n);
+      } else {
+        if (leader) vs.V[(i & 1) * d.xPC + c] = v - n;
+      }
       if (tid == 0) vs.nsl[i & 1] = n;
       // off the path: boundary i's kept rows (V relative to Phi_i, the chosen
       // duration; global stores after the critical store cost the path
@@ -383,7 +420,7 @@ __global__ void __launch_bounds__(LB, 1)
       // stores (every label group saw all of V[i-1]: the first one publishes)
       if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;
       if (leader && i < L) {
-        const int o2 = ((i + 1) & 1) * C + c;
+        const int o2 = ((i + 1) & 1) * Cr + cl;
         vs.Om[o2] = best + fn;
         vs.Ok[o2] = kb;
         vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
@@ -399,10 +436,10 @@ __global__ void __launch_bounds__(LB, 1)
         hbase = (hbase + 1 == K) ? 0 : hbase + 1;
       }
     }
-    __syncthreads();
+    step_sync();
   }
   // the optimum: max over the final labels of V[L] in frame Phi_L
-  if (tid < 32) {
+  if (tid < 32 && rank == 0) {
     const float* V = vs.V + (L & 1) * d.xPC;
     float best = NEG_INF;
     for (int x = tid; x < C; x += 32) best = fmaxf(best, V[x]);
@@ -671,18 +708,10 @@ cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* 
                                 const float* trans, const float* dur, double* score,
                                 int32_t* labels, uint8_t* seg_start, cudaStream_t st) {
   const size_t sm = viterbi_pipe_smem_bytes(d);
-#define SEMICRF_LAUNCH_VPIPE(g, cat, h, kbh, lb)                                               \
-  if (d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb) {               \
-    if (sm > 48 * 1024) {                                                                      \
-      const cudaError_t e = cudaFuncSetAttribute(viterbi_pipe_kernel<g, cat, h, kbh, lb>,      \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                                 (int)sm);                                     \
-      if (e != cudaSuccess) return e;                                                          \
-    }                                                                                          \
-    viterbi_pipe_kernel<g, cat, h, kbh, lb><<<d.B, d.xNT, sm, st>>>(d, ws, lengths, trans, dur,  \
-                                                                    score, labels, seg_start); \
-    return cudaGetLastError();                                                                 \
-  }
+#define SEMICRF_LAUNCH_VPIPE(n, g, cat, h, kbh, lb)                                            \
+  if (d.xN == n && d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb)    \
+    return launch_clustered(viterbi_pipe_kernel<n, g, cat, h, kbh, lb>, n, d.B * n, d.xNT, sm,  \
+                            st, d, ws, lengths, trans, dur, score, labels, seg_start);
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_VPIPE)
 #undef SEMICRF_LAUNCH_VPIPE
   return cudaErrorInvalidConfiguration;

@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["workspace_bytes", "workspace_itemize", "WS_GROUPS", "prefix_center", "forward", "backward", "viterbi", "path_score",
+__all__ = ["workspace_bytes", "workspace_itemize", "WS_GROUPS", "launch_shape", "prefix_center", "forward", "backward", "viterbi", "path_score",
            "get_status", "FLAG_NEGATE_GRAD",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
            "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "ring_domains", "profile_enable", "profile_read",
@@ -47,6 +47,7 @@ _sz = ctypes.c_size_t
 
 lib.semicrf_workspace_bytes.argtypes = [_i, _i, _i, _i, _u, ctypes.POINTER(_sz)]
 lib.semicrf_workspace_itemize.argtypes = [_i, _i, _i, _i, _u, ctypes.POINTER(_sz), _i]
+lib.semicrf_launch_shape.argtypes = [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_int32), _i]
 lib.semicrf_prefix_center.argtypes = [_vp, _vp, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp]
 lib.semicrf_forward.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
 lib.semicrf_backward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp, _vp,
@@ -71,7 +72,7 @@ lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, 
 lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.POINTER(ctypes.c_int32)]
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
-for _f in ("semicrf_workspace_itemize", "semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+for _f in ("semicrf_launch_shape", "semicrf_workspace_itemize", "semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
            "semicrf_forward_proj", "semicrf_backward_proj", "semicrf_viterbi_proj",
            "semicrf_path_score_proj",
@@ -117,6 +118,19 @@ def workspace_itemize(B: int, T: int, C: int, K: int, flags: int = 0) -> dict:
     _check(lib.semicrf_workspace_itemize(B, T, C, K, flags, arr, len(WS_GROUPS)),
            "semicrf_workspace_itemize")
     return {name: int(arr[i]) for i, name in enumerate(WS_GROUPS)}
+
+
+SHAPE_FIELDS = ("ring_ctas", "labels_per_cta", "combine_lanes", "combine_weights",
+                "helper_lanes", "helper_durations", "ring_threads", "delta", "n_checkpoints",
+                "posterior_tile_rows", "log_durations_per_lane", "log_lanes_per_label",
+                "log_labels_per_lane", "log_threads")
+
+
+def launch_shape(B: int, T: int, C: int, K: int) -> dict:
+    """The launch geometry the library picks for these sizes (diagnostic)."""
+    arr = (ctypes.c_int32 * len(SHAPE_FIELDS))()
+    _check(lib.semicrf_launch_shape(B, T, C, K, arr, len(SHAPE_FIELDS)), "semicrf_launch_shape")
+    return {name: int(arr[i]) for i, name in enumerate(SHAPE_FIELDS)}
 
 
 def _stream(device) -> int:

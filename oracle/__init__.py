@@ -56,7 +56,7 @@ def _load():
             lib.oracle_prefix.restype = None
             lib.oracle_fb.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp,
                                       ctypes.c_int, ctypes.c_double, _dp, _dp,
-                                      _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+                                      _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
             lib.oracle_fb.restype = ctypes.c_int
             lib.oracle_viterbi.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp,
                                            ctypes.c_int, _dp, _ip, _u8p]
@@ -119,7 +119,7 @@ def prefix_center(em, lengths, center: bool = True):
 
 def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool = True,
                      grad_logZ=None, threads: int | None = None, want_alpha_beta: bool = False,
-                     p_start=None, p_end=None):
+                     p_start=None, p_end=None, want_segments: bool = False):
     """Exact log Z, marginals and gradients for a batch.
 
     ``p_start`` / ``p_end`` [B, T, C] (optional) are boundary projection
@@ -128,7 +128,9 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
     Returns a dict of float64 arrays:
       logZ [B], logZ_beta [B], start_marg / end_marg [B, T+1, C],
       pos_marg / grad_e [B, T, C], grad_trans [C, C], grad_dur [K, C]
-    (and alpha / beta [B, T+1, C] when ``want_alpha_beta``).  Entries past a
+    (and alpha / beta [B, T+1, C] when ``want_alpha_beta``; seg_marg
+    [B, T, K, C] when ``want_segments``: P(segment [s, s+k) with label c) at
+    [b, s, k-1, c], zero where s + k > L_b).  Entries past a
     sequence's length are zero.  ``grad_logZ`` [B] (default ones) scales the
     three gradients; grad_trans / grad_dur are summed over the batch in batch
     order.
@@ -148,6 +150,8 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
     if want_alpha_beta:
         out["alpha"] = np.zeros((B, T + 1, C))
         out["beta"] = np.zeros((B, T + 1, C))
+    if want_segments:
+        out["seg_marg"] = np.zeros((B, T, K, C))
     gt = np.zeros((B, C, C))
     gd = np.zeros((B, K, C))
 
@@ -162,10 +166,11 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
         ge = np.zeros((max(L, 1), C))
         al = np.zeros((L + 1, C)) if want_alpha_beta else None
         be = np.zeros((L + 1, C)) if want_alpha_beta else None
+        sg = np.zeros((max(L, 1), K, C)) if want_segments else None
         rc = lib.oracle_fb(_ptr(e), L, C, K, _ptr(trans), _ptr(dur), _ptr(_proj(p_start, b, L, C)),
                            _ptr(_proj(p_end, b, L, C)), int(center), float(g[b]),
                            _ptr(lz), _ptr(lzb), _ptr(al), _ptr(be), _ptr(St), _ptr(En),
-                           _ptr(mu), _ptr(ge), _ptr(gt[b]), _ptr(gd[b]))
+                           _ptr(mu), _ptr(ge), _ptr(gt[b]), _ptr(gd[b]), _ptr(sg))
         if rc != 0:
             raise MemoryError("oracle_fb: allocation failed")
         out["logZ"][b] = lz[0]
@@ -178,6 +183,8 @@ def forward_backward(em, lengths, trans, dur, K: int | None = None, center: bool
         if want_alpha_beta:
             out["alpha"][b, :L + 1] = al
             out["beta"][b, :L + 1] = be
+        if want_segments and L > 0:
+            out["seg_marg"][b, :L] = sg[:L]
 
     n = _threads(B, threads)
     if n == 1:

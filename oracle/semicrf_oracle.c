@@ -163,13 +163,19 @@ static void edge_block(const double *content, const double *trans, const double 
  *   start_marg, end_marg [(L+1), C]
  *   pos_marg, grad_e   [L, C]
  *   grad_trans [C, C], grad_dur [K, C]: ADDED to (so a batch can share them)
+ *   seg_marg  [L, K, C]  P(segment [s, s+k) with label c) at [s, k-1, c], the
+ *                        explicit edge posteriors summed over the previous
+ *                        label (explainer section 4, "Correctness": the
+ *                        boundary and segment probabilities); entries with
+ *                        s + k > L are left as passed (zero)
  * logZ_beta receives log Z recomputed from the backward side.
  * Returns 0, or -1 if the scratch allocation failed.
  */
 int oracle_fb(const double *e, int L, int C, int K, const double *trans, const double *dur,
               const double *ps, const double *pe, int center, double g, double *logZ, double *logZ_beta,
               double *alpha_out, double *beta_out, double *start_marg, double *end_marg,
-              double *pos_marg, double *grad_e, double *grad_trans, double *grad_dur)
+              double *pos_marg, double *grad_e, double *grad_trans, double *grad_dur,
+              double *seg_marg)
 {
     if (L <= 0) {
         *logZ = 0.0;
@@ -268,6 +274,7 @@ int oracle_fb(const double *e, int L, int C, int K, const double *trans, const d
                     P = exp(Wk[c] + beta[(size_t)t * C + c] - lz);
                 }
                 if (grad_dur) grad_dur[(size_t)(k - 1) * C + c] += g * P;
+                if (seg_marg) seg_marg[((size_t)s * K + (k - 1)) * C + c] = P;
                 St[(size_t)s * C + c] += P;
                 En[(size_t)t * C + c] += P;
                 for (int u = s; u < t; ++u) mu[(size_t)u * C + c] += P;

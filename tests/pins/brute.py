@@ -64,9 +64,11 @@ def enumerate_all(e, L, trans, dur, center=True, tie_tol=1e-9, ps=None, pe=None)
     mu = np.zeros((L, C))
     gdur = np.zeros((K, C))
     gtrans = np.zeros((C, C))
+    segm = np.zeros((max(L, 1), K, C))
     for p, sg in zip(probs, segs_all):
         prev = None
         for (s, t, c) in sg:
+            segm[s, t - s - 1, c] += p
             St[s, c] += p
             En[t, c] += p
             mu[s:t, c] += p
@@ -89,7 +91,7 @@ def enumerate_all(e, L, trans, dur, center=True, tie_tol=1e-9, ps=None, pe=None)
             out.append(sg[i - 1][2] if i > 0 else -1)
         return out
     chosen = min(optimal, key=key)
-    return dict(logZ=logZ, start_marg=St, end_marg=En, pos_marg=mu, grad_dur=gdur,
+    return dict(logZ=logZ, start_marg=St, end_marg=En, pos_marg=mu, grad_dur=gdur, seg_marg=segm[:L],
                 grad_trans=gtrans, best_score=best, optimal=[to_arrays(sg, L) for sg in optimal],
                 tie_broken=to_arrays(chosen, L), n_segmentations=len(segs_all))
 

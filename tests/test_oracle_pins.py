@@ -81,6 +81,32 @@ def test_bruteforce_logZ_and_marginals(L, K, C, center, seed):
 
 
 @pytest.mark.parametrize("L,K,C,center,seed", BRUTE_CASES)
+def test_bruteforce_segment_marginals(L, K, C, center, seed):
+    """P(segment [s, s+k) with label c), the quantity behind the pages'
+    "boundary probabilities are valid" check (explainer section 4,
+    Correctness), against enumeration; and its bookkeeping: summed over
+    durations it is the start marginal, over starts the duration count,
+    over the segments covering u the position marginal."""
+    rng = np.random.default_rng(seed)
+    em, lengths, trans, dur = _rand_case(rng, 1, L, K, C, pstd=0.7)
+    ref = brute.enumerate_all(em[0], L, trans, dur, center=center)
+    out = oracle.forward_backward(em, lengths, trans, dur, K, center=center, threads=1,
+                                  want_segments=True)
+    sm = out["seg_marg"][0]
+    assert sm.shape == (L, K, C)
+    assert np.max(np.abs(sm - ref["seg_marg"])) < 1e-12
+    assert np.max(np.abs(sm.sum(axis=1) - out["start_marg"][0, :L])) < 1e-12
+    assert np.max(np.abs(sm.sum(axis=0) - out["grad_dur"])) < 1e-12
+    cover = np.zeros((L, C))
+    for s_ in range(L):
+        for k in range(1, K + 1):
+            cover[s_:s_ + k] += sm[s_, k - 1]
+    assert np.max(np.abs(cover - out["pos_marg"][0, :L])) < 1e-12
+    for s_ in range(L):   # no segment runs past the end
+        assert np.all(sm[s_, L - s_:] == 0)
+
+
+@pytest.mark.parametrize("L,K,C,center,seed", BRUTE_CASES)
 def test_bruteforce_viterbi(L, K, C, center, seed):
     rng = np.random.default_rng(100 + seed)
     em, lengths, trans, dur = _rand_case(rng, 1, L, K, C, pstd=0.7)

@@ -194,6 +194,26 @@ SEMICRF_API int semicrf_backward(const int32_t *lengths, const float *trans, con
                      semicrf_stream_t stream);
 
 /*
+ * Step 3 with the segment marginals (explainer section 4, "Correctness --
+ * Self-Consistency": the boundary and segment probabilities are valid
+ * distributions): everything semicrf_backward computes, plus
+ *   seg_marg [B, T, K, C]  P(a label-c segment covers exactly [s, s+k)) at
+ *                          [b, s, k-1, c]; zero where s >= L_b or s + k > L_b
+ * (float32, not scaled by g_b).  Summed over k it is start_marg, over s (and
+ * times g) grad_dur.  The array is O(T K C): meant for moderate sizes (the
+ * speech-scale batch needs 150 MB).  seg_marg must not be NULL when B, T > 0
+ * (SEMICRF_ERR_INVALID_ARG); the other arguments and errors are those of
+ * semicrf_backward.  Not for a workspace filled by semicrf_forward_proj.
+ */
+SEMICRF_API int semicrf_backward_segments(const int32_t *lengths, const float *trans,
+                                          const float *dur, int B, int T, int C, int K,
+                                          unsigned flags, void *ws, size_t ws_bytes,
+                                          const double *grad_logZ, float *grad_em,
+                                          float *grad_trans, float *grad_dur, float *pos_marg,
+                                          float *start_marg, float *end_marg, float *seg_marg,
+                                          semicrf_stream_t stream);
+
+/*
  * Step 4: max-semiring decoding with the same recursion (max in place of
  * log-sum-exp).  Ties go to the smallest duration k, then the smallest
  * previous label c', and at the end to the smallest final label.  Writes
@@ -348,6 +368,9 @@ SEMICRF_API int semicrf_profile_read(const char *kernel, double *total_ms, int *
  *    checkpoints) return SEMICRF_ERR_UNSUPPORTED before anything runs.
  *  - The first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
+ *    The address is kept for the life of the process: after a device reset
+ *    (which unloads the library's device image) restart the process before
+ *    calling this again.
  *  - No cudaMalloc, cudaFree or allocating library call is made.
  *  - Every call on a device shares the array and leaves its contents behind;
  *    only the status word is cleared per call.  Calls that overlap on the GPU

@@ -76,7 +76,9 @@ int max_smem_optin() {
 // cluster (N CTAs, C / N labels each): the per-step work of one SM shrinks
 // N-fold and each step pays a cluster barrier (about 500 cycles measured on
 // B200 against about 150 for a CTA barrier), which pays when one SM's step
-// is several thousand cycles (C = 128: about 4300 cycles on one CTA).
+// is several thousand cycles (C = 128: about 4300 cycles on one CTA, 2400 on
+// a cluster of 4, 2500 on 8).  Clusters of 4 are preferred: the two rings
+// and the decoder of a batch then fit the GPU side by side (B = 8: 96 SMs).
 // SEMICRF_XSHAPE=i forces the i-th fitting shape of the menu and
 // SEMICRF_XCLUSTER=n restricts the choice to clusters of n CTAs (tuning).
 constexpr int CLUSTER_MIN_C = 96;
@@ -106,7 +108,7 @@ void choose_xshape(Dims& d, size_t budget) {
     if (C <= g * cat && K <= h * kbh + 2 && nt <= lb && cl_ok && (n == 1 || cr * n - C < cr)) { \
       const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +        \
                           10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0) +      \
-                          (n > 1 ? 100.0 + 10.0 * n : 0.0);                               \
+                          (n > 1 ? 100.0 + 25.0 * std::abs(n - 4) : 0.0);                 \
       if ((forced < 0 && cost < best) || forced == idx) {                                 \
         best = cost;                                                                      \
         d.xN = n;                                                                         \
@@ -579,7 +581,7 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
                   int C, int K, unsigned flags, void* ws, size_t ws_bytes,
                   const double* grad_logZ, float* grad_em, float* grad_trans, float* grad_dur,
                   float* grad_p_start, float* grad_p_end, float* pos_marg, float* start_marg,
-                  float* end_marg, bool proj, cudaStream_t st) {
+                  float* end_marg, bool proj, cudaStream_t st, float* seg_marg = nullptr) {
   if (!lengths || !trans || !dur || !grad_trans || !grad_dur || (B > 0 && T > 0 && !grad_em))
     return SEMICRF_ERR_INVALID_ARG;
   Dims d;
@@ -605,6 +607,11 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
     rc = run_chains(d, p, lengths, trans, dur, nullptr, 0, B, flags, st);
     if (rc) return rc;
   }
+  // segment marginals: every entry the posterior kernels do not write (past
+  // a length, segments running past the end) is zero
+  if (seg_marg && T > 0 &&
+      cudaMemsetAsync(seg_marg, 0, (size_t)B * T * K * C * sizeof(float), st) != cudaSuccess)
+    return SEMICRF_ERR_CUDA;
   if (T > 0) {
     // sequences whose rings both ran in the exponential domain: posteriors
     // from the kept values (cut normalisers, then one parallel pass); the
@@ -617,7 +624,8 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
     if (!side_fork(ss, st)) return SEMICRF_ERR_CUDA;
     {
       ProfScope ps("segment_kernel", s2);
-      e_seg = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, s2);
+      e_seg = launch_segment(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, s2,
+                             seg_marg);
     }
     if (d.xG) {
       const size_t csm = cut_grid_smem_bytes(d);
@@ -629,7 +637,8 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
       if ((rc = launched())) return rc;
       {
         ProfScope ps("posterior_kernel", st);
-        e = launch_posterior(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st);
+        e = launch_posterior(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st,
+                             seg_marg);
       }
     }
     if (!side_join(ss, st)) return SEMICRF_ERR_CUDA;
@@ -690,6 +699,19 @@ extern "C" int semicrf_backward(const int32_t* lengths, const float* trans, cons
   return backward_impl(lengths, trans, dur, B, T, C, K, flags, ws, ws_bytes, grad_logZ, grad_em,
                        grad_trans, grad_dur, nullptr, nullptr, pos_marg, start_marg, end_marg,
                        false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int semicrf_backward_segments(const int32_t* lengths, const float* trans,
+                                         const float* dur, int B, int T, int C, int K,
+                                         unsigned flags, void* ws, size_t ws_bytes,
+                                         const double* grad_logZ, float* grad_em,
+                                         float* grad_trans, float* grad_dur, float* pos_marg,
+                                         float* start_marg, float* end_marg, float* seg_marg,
+                                         semicrf_stream_t stream) {
+  if (!seg_marg && B > 0 && T > 0) return SEMICRF_ERR_INVALID_ARG;
+  return backward_impl(lengths, trans, dur, B, T, C, K, flags, ws, ws_bytes, grad_logZ, grad_em,
+                       grad_trans, grad_dur, nullptr, nullptr, pos_marg, start_marg, end_marg,
+                       false, reinterpret_cast<cudaStream_t>(stream), seg_marg);
 }
 
 extern "C" int semicrf_backward_proj(const int32_t* lengths, const float* trans, const float* dur,

@@ -21,6 +21,23 @@ constexpr float NEG_INF = -__builtin_huge_valf();
 constexpr int ST_DEVICE_TIMEOUT = 5;
 constexpr int ST_BAD_LENGTH = 6;
 
+// Bounds-checking debug build (-DSEMICRF_BOUNDS_CHECK; libsemicrf_b200_check.so).
+// SEMICRF_INB(status, cond, site) is true in the release build; in the
+// debug build a false `cond` records ST_BOUNDS | site << 8 in the status
+// word (the first failure wins) and the caller skips the access it guards.
+// Sites are numbered per file (see the SITE_* constants at each use); no
+// trap, no fault: the kernel carries on and the host reads the status.
+constexpr int ST_BOUNDS = 7;
+#ifdef SEMICRF_BOUNDS_CHECK
+__device__ __noinline__ inline void bounds_fail(int* status, int site) {
+  if (status) atomicCAS(status, 0, ST_BOUNDS | (site << 8));
+}
+#define SEMICRF_INB(status, cond, site) \
+  ((cond) ? true : (::semicrf::bounds_fail((status), (site)), false))
+#else
+#define SEMICRF_INB(status, cond, site) true
+#endif
+
 // Polls of an mbarrier before a wait gives up (each try_wait may itself
 // suspend for a bounded, hardware-defined time).
 constexpr int WAIT_SPIN_LIMIT = 1 << 22;

@@ -55,9 +55,12 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                 const float* __restrict__ trans, const float* __restrict__ dur);
 // The posterior pass (one CTA per checkpoint segment and sequence).
+// seg_marg (nullable) [B][T][K][C]: the segment marginals of the sequences
+// the kernel takes (the caller zeroes the array first).
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,
-                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st);
+                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
+                             float* seg_marg = nullptr);
 size_t posterior_smem_bytes(const Dims& d);
 // Tile rows for the posterior pass under `budget` bytes of shared memory (0:
 // none fits).
@@ -79,7 +82,8 @@ cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths
 // One CTA per (checkpoint segment, sequence).
 cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                            const float* trans, const float* dur, const double* grad_logZ,
-                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st);
+                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
+                           float* seg_marg = nullptr);
 cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                            const float* trans, const float* dur, double* score, int32_t* labels,
                            uint8_t* seg_start, cudaStream_t st);

@@ -29,7 +29,10 @@ std::mutex scratch_mu;
 void* scratch_ptr[MAX_DEVICES] = {};
 
 // Device address of the array on the current device.  Looked up once per
-// device (host code cannot use the array's name as an address).
+// device (host code cannot use the array's name as an address) and kept for
+// the life of the process; a device reset unloads the module the address
+// belongs to, so a process that resets a device must restart before calling
+// the entry point again.
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {

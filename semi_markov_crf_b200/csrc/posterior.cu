@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                      const float* __restrict__ trans, const float* __restrict__ dur,
                      const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
-                     float* __restrict__ start_marg, float* __restrict__ end_marg) {
+                     float* __restrict__ start_marg, float* __restrict__ end_marg,
+                     float* __restrict__ seg_marg) {
   extern __shared__ __align__(16) unsigned char psh[];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
   const int C = d.C, K = d.K, RT = d.pRT;
@@ -275,6 +276,21 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
       if (start_marg) start_marg[ob] = St;
       if (end_marg) end_marg[ob] = E;
       tl.dif[i] = (double)St - (double)E;
+    }
+    // ------------------------------------------------------------ segment marginals
+    // (optional output) P([s, s+k), c) for every start of the tile, the same
+    // product as the duration counts below, not scaled by g (a marginal)
+    if (seg_marg) {
+      for (int i = tid; i < nr * nd; i += nthr) {
+        const int r = i / nd, idx = i - r * nd;
+        const int k = idx / C + 1, c = idx - (k - 1) * C;
+        if (s_lo + r + k > L) continue;
+        const int o = r * C + c, ok = (r + k) * C + c;
+        const float z = (float)(tl.ii[ok] - tl.ii[o]) +
+                        ((M + __ldg(dur + idx) * l2e()) + (tl.sf[ok] - tl.sf[o]));
+        seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] =
+            tl.tf[r * 2 * C + C + c] * tl.ab[ok] * (tl.fs[r] * ex2(z));
+      }
     }
     // ------------------------------------------------------------ duration counts
     // item (k, c): sum over the tile's s of P([s, s+k), c), s + k <= L
@@ -368,7 +384,8 @@ size_t posterior_smem_bytes(const Dims& d) { return ptile_bytes(d.pRT, d.K, d.C)
 
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,
-                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st) {
+                             float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
+                             float* seg_marg) {
   const size_t sm = posterior_smem_bytes(d);
   const bool small = (size_t)d.K * d.C <= 4u * 512u && (size_t)d.C * d.C <= 4u * 512u;
   const void* fn = small ? (const void*)posterior_kernel<4, 4> : (const void*)posterior_kernel<16, 32>;
@@ -378,10 +395,12 @@ cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* len
   }
   if (small)
     posterior_kernel<4, 4><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
-                                                              grad_em, start_marg, end_marg);
+                                                              grad_em, start_marg, end_marg,
+                                                              seg_marg);
   else
     posterior_kernel<16, 32><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
-                                                                grad_em, start_marg, end_marg);
+                                                                grad_em, start_marg, end_marg,
+                                                                seg_marg);
   return cudaGetLastError();
 }
 

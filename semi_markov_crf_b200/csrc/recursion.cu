@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(LB, 1)
     segment_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                    const float* __restrict__ trans, const float* __restrict__ dur,
                    const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
-                   float* __restrict__ start_marg, float* __restrict__ end_marg) {
+                   float* __restrict__ start_marg, float* __restrict__ end_marg,
+                   float* __restrict__ seg_marg) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const Smem sm = carve(smem_raw, d, d.store_smem != 0);
   const int C = d.C, K = d.K, PC = d.PC, tid = threadIdx.x;
@@ -652,6 +653,17 @@ __global__ void __launch_bounds__(LB, 1)
         const float coef = (ksum > 0.f) ? gbf * Stg / ksum : 0.f;
 #pragma unroll
         for (int i = 0; i < KBT; ++i) accd[i] = fmaf(coef, e[i], accd[i]);
+        if (seg_marg && ln.act) {
+          // P([s, s+k), c) = start marginal x normalised k term (not scaled
+          // by g: a marginal); rescaled with the rest below
+          const float cs = (ksum > 0.f) ? Stg / ksum : 0.f;
+          float* const row = seg_marg + ((size_t)b * d.T + s) * K * C + ln.c;
+#pragma unroll
+          for (int i = 0; i < KBT; ++i) {
+            const int k = ln.k_of(ln.widx(i), false);
+            if (k <= K && s + k <= L) row[(size_t)(k - 1) * C] = cs * e[i];
+          }
+        }
       }
       __syncthreads();
       bool slow;
@@ -738,6 +750,9 @@ __global__ void __launch_bounds__(LB, 1)
   if (last && end_marg)
     for (int c = tid; c < C; c += blockDim.x) end_marg[((size_t)b * (d.T + 1) + L) * C + c] *= rs;
   for (int idx = tid; idx < K * C; idx += blockDim.x) ws.pgd[seg * K * C + idx] *= (double)rs;
+  if (seg_marg)
+    for (size_t idx = tid; idx < (size_t)(t1 - t0) * K * C; idx += blockDim.x)
+      seg_marg[((size_t)b * d.T + t0) * K * C + idx] *= rs;
   for (int idx = tid; idx < C * C; idx += blockDim.x) ws.pgt[seg * C * C + idx] *= (double)rs;
   if (ln.leader) {
     ws.segT[seg * C + ln.c] = (double)sm.tmp[ln.c] + (double)rs * accmu;  // mu[t0 - 1] + total
@@ -794,14 +809,15 @@ cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths
 
 cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                            const float* trans, const float* dur, const double* grad_logZ,
-                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st) {
+                           float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
+                           float* seg_marg) {
   const size_t sm = recursion_smem_bytes(d, d.store_smem != 0);
 #define SEMICRF_LAUNCH_SEG(a, b, g, lb)                                                      \
   if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \
     const cudaError_t e = allow_smem(segment_kernel<a, b, g, lb>, sm);                       \
     if (e != cudaSuccess) return e;                                                          \
     segment_kernel<a, b, g, lb><<<dim3(d.nck, d.B), d.NT, sm, st>>>(                         \
-        d, ws, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg);               \
+        d, ws, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, seg_marg);     \
     return cudaGetLastError();                                                               \
   }
   SEMICRF_FOR_EACH_SHAPE(SEMICRF_LAUNCH_SEG)

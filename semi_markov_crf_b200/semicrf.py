@@ -52,6 +52,8 @@ lib.semicrf_prefix_center.argtypes = [_vp, _vp, _i, _i, _i, _u, _vp, _sz, _vp, _
 lib.semicrf_forward.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
 lib.semicrf_backward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp, _vp,
                                  _vp, _vp, _vp, _vp]
+lib.semicrf_backward_segments.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.semicrf_viterbi.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp, _vp,
                                 _vp]
 lib.semicrf_path_score.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _sz,
@@ -72,7 +74,7 @@ lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, 
 lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.POINTER(ctypes.c_int32)]
 lib.semicrf_profile_enable.argtypes = [_i]
 lib.semicrf_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
-for _f in ("semicrf_launch_shape", "semicrf_workspace_itemize", "semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
+for _f in ("semicrf_backward_segments", "semicrf_launch_shape", "semicrf_workspace_itemize", "semicrf_forward_noalloc", "semicrf_profile_enable", "semicrf_profile_read", "semicrf_workspace_bytes", "semicrf_prefix_center", "semicrf_forward",
            "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
            "semicrf_forward_proj", "semicrf_backward_proj", "semicrf_viterbi_proj",
            "semicrf_path_score_proj",
@@ -231,14 +233,16 @@ def forward(em, lengths, trans, dur, center: bool = True, forward_only: bool = F
 
 
 def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool = False,
-             out: dict | None = None):
+             out: dict | None = None, segments: bool = False):
     """Step 3 on the workspace of the preceding :func:`forward`.
 
     Returns a dict with grad_em [B,T,C], grad_trans [C,C], grad_dur [K,C]
     (float32) and, when ``marginals``, pos_marg [B,T,C], start_marg and
     end_marg [B,T+1,C]; after a forward with boundary projections also
-    grad_p_start and grad_p_end [B,T,C] (semicrf_backward_proj).  ``out``
-    may supply preallocated tensors."""
+    grad_p_start and grad_p_end [B,T,C] (semicrf_backward_proj).  With
+    ``segments`` also seg_marg [B,T,K,C], P(segment [s, s+k) with label c)
+    at [b, s, k-1, c] (semicrf_backward_segments; not after a forward with
+    projections).  ``out`` may supply preallocated tensors."""
     B, T, C, K = ws.dims
     dev = ws.buf.device
     _need(lengths, torch.int32, "lengths", dev)
@@ -266,6 +270,19 @@ def backward(ws: Workspace, lengths, trans, dur, grad_logZ=None, marginals: bool
             _ptr(o.get("pos_marg") if marginals else None),
             _ptr(o.get("start_marg") if marginals else None),
             _ptr(o.get("end_marg") if marginals else None), _stream(dev)), "semicrf_backward_proj")
+        return o
+    if segments:
+        if ws.proj:
+            raise ValueError("segment marginals are not available after a forward with projections")
+        if "seg_marg" not in o:
+            o["seg_marg"] = torch.empty((B, T, K, C), dtype=torch.float32, device=dev)
+        _check(lib.semicrf_backward_segments(
+            _ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, ws.flags, ws.ptr, ws.nbytes,
+            _ptr(grad_logZ), _ptr(o["grad_em"]), _ptr(o["grad_trans"]), _ptr(o["grad_dur"]),
+            _ptr(o.get("pos_marg") if marginals else None),
+            _ptr(o.get("start_marg") if marginals else None),
+            _ptr(o.get("end_marg") if marginals else None), _ptr(o["seg_marg"]), _stream(dev)),
+            "semicrf_backward_segments")
         return o
     _check(lib.semicrf_backward(_ptr(lengths), _ptr(trans), _ptr(dur), B, T, C, K, ws.flags, ws.ptr,
                                 ws.nbytes, _ptr(grad_logZ), _ptr(o["grad_em"]), _ptr(o["grad_trans"]),

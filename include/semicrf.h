@@ -78,7 +78,9 @@ enum semicrf_status {
     SEMICRF_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < semicrf_workspace_bytes(...) */
     SEMICRF_ERR_CUDA = 4,                /* a CUDA launch or copy failed */
     SEMICRF_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device wait gave up */
-    SEMICRF_ERR_BAD_LENGTH = 6           /* some lengths[b] outside [0, T] */
+    SEMICRF_ERR_BAD_LENGTH = 6,          /* some lengths[b] outside [0, T] */
+    SEMICRF_ERR_BOUNDS = 7               /* bounds-checking build only: an index check
+                                            failed; (status >> 8) names the check site */
 };
 
 /* flags */
@@ -340,6 +342,17 @@ SEMICRF_API const char *semicrf_strerror(int code);
  * the pages.
  */
 SEMICRF_API int semicrf_selftest_bounded_wait(void *ws, size_t ws_bytes, int spins, semicrf_stream_t stream);
+
+/*
+ * Self-test of the bounds-checking debug build (libsemicrf_b200_check.so,
+ * compiled with -DSEMICRF_BOUNDS_CHECK; no counterpart on the pages): clears
+ * the status word of `ws` and launches one CTA whose only guarded store uses
+ * an index one past its 32-entry shared array; the check records
+ * SEMICRF_ERR_BOUNDS | site << 8 and skips the store, so nothing is written
+ * out of bounds.  Read the result with semicrf_get_status.  The release
+ * build returns SEMICRF_ERR_UNSUPPORTED and launches nothing.
+ */
+SEMICRF_API int semicrf_selftest_bounds(void *ws, size_t ws_bytes, semicrf_stream_t stream);
 
 /*
  * Diagnostic timing (no counterpart on the pages).  semicrf_profile_enable(1)

@@ -1,6 +1,11 @@
 """Build the C-ABI library ``libsemicrf_b200.so`` in-tree with nvcc (sm_100a).
 
-Usage:  python -m semi_markov_crf_b200.build [--force] [--verbose]
+Usage:  python -m semi_markov_crf_b200.build [--force] [--verbose] [--bounds-check]
+
+``--bounds-check`` builds the debug variant ``libsemicrf_b200_check.so``
+(-DSEMICRF_BOUNDS_CHECK): index checks in the kernels record the first
+failing site in the workspace status word instead of making the access.
+The binding loads it when SEMICRF_LIBRARY=check.
 
 Compiles every ``csrc/*.cu`` for ``-gencode arch=compute_100a,code=sm_100a``
 (with -lineinfo) and links a shared library with the CUDA runtime linked
@@ -21,6 +26,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsemicrf_b200.so")
+LIB_CHECK = os.path.join(PKG, "libsemicrf_b200_check.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
 NVCC_FLAGS = [
@@ -43,24 +49,27 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, bounds_check: bool = False) -> str:
+    lib = LIB_CHECK if bounds_check else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = _nvcc()
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    bdir = BUILD_DIR + ("_check" if bounds_check else "")
+    os.makedirs(bdir, exist_ok=True)
+    extra = ["-DSEMICRF_BOUNDS_CHECK"] if bounds_check else []
     from concurrent.futures import ThreadPoolExecutor
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         res = subprocess.run(cmd, capture_output=True, text=True)
@@ -73,16 +82,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
            "-Xcompiler", "-fPIC", *objs, "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                bounds_check="--bounds-check" in sys.argv))

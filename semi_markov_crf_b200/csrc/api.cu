@@ -883,7 +883,10 @@ extern "C" const char* semicrf_strerror(int code) {
     case SEMICRF_ERR_CUDA: return "CUDA launch or copy failed";
     case SEMICRF_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
     case SEMICRF_ERR_BAD_LENGTH: return "a sequence length is outside [0, T]";
-    default: return "unknown status";
+    default:
+      if ((code & 0xff) == SEMICRF_ERR_BOUNDS)
+        return "an index check failed (bounds-checking build; status >> 8 is the site)";
+      return "unknown status";
   }
 }
 
@@ -895,6 +898,22 @@ extern "C" int semicrf_selftest_bounded_wait(void* ws, size_t ws_bytes, int spin
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
   selftest_wait_kernel<<<1, 32, 0, st>>>(status, spins);
   return launched();
+}
+
+extern "C" int semicrf_selftest_bounds(void* ws, size_t ws_bytes, semicrf_stream_t stream) {
+#ifdef SEMICRF_BOUNDS_CHECK
+  if (!ws || ws_bytes < 256) return SEMICRF_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SEMICRF_ERR_CUDA;
+  selftest_bounds_kernel<<<1, 32, 0, st>>>(status, 32);
+  return launched();
+#else
+  (void)ws;
+  (void)ws_bytes;
+  (void)stream;
+  return SEMICRF_ERR_UNSUPPORTED;  // the release build has no index checks to exercise
+#endif
 }
 
 extern "C" int semicrf_profile_enable(int on) {

@@ -173,6 +173,11 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   auto put = [&](int slot, float2 v) {  // slot and its mirrors slot + mK < RL
     for (int x = slot; x < RL; x += K) rl[x] = v;
   };
+  // bounds-check build: a row pointer lies inside the two tile buffers
+  auto row_ok = [&](const int32_t* row) {
+    const ptrdiff_t o = row - sm.tint;
+    return o >= 0 && o + C <= 2 * TS * C;
+  };
 
   // One register array serves both roles: combine lanes keep the transition
   // weights 2^(trans2 - M) of their CAT source labels (forward trans[x][c],
@@ -359,8 +364,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       // ---------------------------------------------------------- combine
       const int po = (i & 1) * Cr + ccl;
       const float a1v = xs.A1[po], a2v = xs.A2[po], ohv = xs.Oh[po];
-      const int si_n = crow_i[cc];  // the walk's row r: the next step's ring entry
-      const float sf_n = crow_f[cc];
+      const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
+      const int si_n = rok ? crow_i[cc] : 0;  // the walk's row r: the next step's ring entry
+      const float sf_n = rok ? crow_f[cc] : 0.f;
       const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
 #pragma unroll
@@ -390,22 +396,25 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float sn = pow2_neg(n);
       const float R = fmaf(acc2, a2v, ohv) * snprev;  // frame Phi_{i-1}
       const float pn = fmaf(acc * sn, a1v, R * sn);
+      const bool pok = SEMICRF_INB(ws.status, c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
-        if (act)
+        if (act && pok)
           for (int q = jl; q < N; q += G) st_cluster(xs.P + (i & 1) * d.xPC + c, q, pn);
       } else {
-        if (leader) xs.P[(i & 1) * d.xPC + c] = pn;
+        if (leader && pok) xs.P[(i & 1) * d.xPC + c] = pn;
       }
       if (tid == 0) xs.nsl[i & 1] = n;
       // the kept row of this boundary, then the ring entry: global stores
       // after the critical store cost the path least (measured against the
       // helpers copying the row, and against storing after the ring entry)
-      if (kv && leader) {
+      if (kv && leader &&
+          SEMICRF_INB(ws.status, r >= 0 && r <= d.T && r - SG >= 0 && r - SG <= d.T, SITE_KEPT_ROW)) {
         kv[(size_t)r * 2 * C + c] = pn;                // row r, frame Phi_i
         kv[(size_t)(r - SG) * 2 * C + C + c] = acc;    // row r - SG, frame Phi_{i-1}
       }
-      if (i >= 2 && leader) put(wslot, make_float2(gprev - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
+      if (i >= 2 && leader && SEMICRF_INB(ws.status, wslot >= 0 && wslot < K, SITE_RING_SLOT))
+        put(wslot, make_float2(gprev - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;
@@ -417,12 +426,15 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       crow_f += SG * C;
     } else if (i < L) {
       // ---------------------------------------------------------- helpers
-      const int sn = hrow_i[cc];
-      const float fn = hrow_f[cc];
+      const bool hok = SEMICRF_INB(ws.status, row_ok(hrow_i), SITE_TILE_ROW);
+      const int sn = hok ? hrow_i[cc] : 0;
+      const float fn = hok ? hrow_f[cc] : 0.f;
+      const bool wok = SEMICRF_INB(ws.status, hbase >= 0 && hbase + jl + (KBH - 1) * H < RLP,
+                                   SITE_RING_WINDOW);
       const float Qh = sg * (float)(sn - Sbc) - Fph;
       float m = Qh + rel;
       float s;
-      const float lse = k_fanin_strided<KBH, H>(rl + hbase + jl, Qh, w, m, s, act);
+      const float lse = k_fanin_strided<KBH, H>(rl + (wok ? hbase : 0) + jl, Qh, w, m, s, act);
       if (isfinite(lse)) rel = rintf(lse - Qh);
       // the three values step i+1 reads: lanes 0, 1, 2 of the group take one
       // exponential each (no divergent branches); narrower groups take all

@@ -44,6 +44,9 @@ __global__ void reduce_partials_kernel(Dims d, WsPtrs ws, const int32_t* __restr
                                        float* __restrict__ grad_trans, float* __restrict__ grad_dur);
 
 __global__ void selftest_wait_kernel(int* status, int spins);
+#ifdef SEMICRF_BOUNDS_CHECK
+__global__ void selftest_bounds_kernel(int* status, int idx);
+#endif
 
 // Posteriors of sequence b come from the values both exponential-domain
 // rings kept (posterior.cu) rather than from the checkpoint walk

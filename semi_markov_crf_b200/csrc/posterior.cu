@@ -249,6 +249,8 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     const int nr = s_hi - s_lo;
     const int nh = min(s_hi - 1 + K, L) - s_lo + 1;  // rows a segment of the tile ends on
     const bool first = (s_hi == t1);
+    // bounds-check build: the tile and its halo fit the staged rows
+    if (!SEMICRF_INB(ws.status, nr >= 1 && nr <= RT && nh <= RT + K, SITE_POST_TILE)) break;
     // ------------------------------------------------------------ stage
     const double kb0 = kfb[s_lo];
     #pragma unroll 4
@@ -285,6 +287,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
         const int r = i / nd, idx = i - r * nd;
         const int k = idx / C + 1, c = idx - (k - 1) * C;
         if (s_lo + r + k > L) continue;
+        if (!SEMICRF_INB(ws.status, r + k < nh, SITE_POST_ITEM)) continue;
         const int o = r * C + c, ok = (r + k) * C + c;
         const float z = (float)(tl.ii[ok] - tl.ii[o]) +
                         ((M + __ldg(dur + idx) * l2e()) + (tl.sf[ok] - tl.sf[o]));
@@ -297,7 +300,8 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     auto dur_item = [&](int idx) {
       const int k = idx / C + 1, c = idx - (k - 1) * C;
       const float dk = M + __ldg(dur + idx) * l2e();
-      const int r_end = min(s_hi, L - k + 1) - s_lo;
+      int r_end = min(s_hi, L - k + 1) - s_lo;
+      if (!SEMICRF_INB(ws.status, r_end <= 0 || r_end - 1 + k < nh, SITE_POST_ITEM)) r_end = 0;
       float a_ = 0.f;
       for (int r = 0; r < r_end; ++r) {
         const int o = r * C + c, ok = (r + k) * C + c;

@@ -270,7 +270,8 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float s;
         const float lse =
-            k_fanin<KBT, G>(rl + base, ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
+            k_fanin<KBT, G>(rl + checked_base(ws, base, K),
+                            ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -293,8 +294,9 @@ __global__ void __launch_bounds__(LB, 1)
         const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
-          ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
-                                                  (Frel + n) - (float)(si - Sb)));
+          if (checked_slot(ws, wslot, K))
+            ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
+                                                    (Frel + n) - (float)(si - Sb)));
         }
         __syncwarp();
         Frel += n;
@@ -359,7 +361,8 @@ __global__ void __launch_bounds__(LB, 1)
         const float sf = rf[ln.cc];
         float ssum;
         const float lse =
-            k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
+            k_fanin<KBT, G>(rl + checked_base(ws, base, K),
+                            ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ssum, e, ln.act);
         const float Bt = (lse == NEG_INF) ? NEG_INF : (lse - sf) + proj_d(ws, d, pj, b, s, ln.cc);
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = Bt;
@@ -382,7 +385,8 @@ __global__ void __launch_bounds__(LB, 1)
         const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, true);
-          ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
+          if (checked_slot(ws, wslot, K))
+            ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
         }
         __syncwarp();
         Grel += n;
@@ -513,7 +517,8 @@ __global__ void __launch_bounds__(LB, 1)
         const int si = ri[ln.cc];
         const float sf = rf[ln.cc];
         float s;
-        const float lse = k_fanin<KBT, G>(rl + base, ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
+        const float lse = k_fanin<KBT, G>(rl + checked_base(ws, base, K),
+                                          ln.j, (float)(si - Sb) - Frel, ln.d, mk, s, e, ln.act);
         const float A = (lse == NEG_INF) ? NEG_INF : sf + lse;
         if (ln.leader) {
           sm.Acur[par * C + ln.c] = A;
@@ -537,8 +542,9 @@ __global__ void __launch_bounds__(LB, 1)
         float* row = store + (size_t)(t - t0) * SW;
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, false);
-          ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
-                                                  (Frel + n) - (float)(si - Sb)));
+          if (checked_slot(ws, wslot, K))
+            ring_put<KBT>(rl, d, wslot, make_float2((g - sf) + proj_d(ws, d, pj, b, t, ln.c),
+                                                    (Frel + n) - (float)(si - Sb)));
           row[ln.c] = A;
           row[C + ln.c] = g;
         }
@@ -636,7 +642,8 @@ __global__ void __launch_bounds__(LB, 1)
       const int si = ri[ln.cc];
       const float sf = rf[ln.cc];
       float ksum;
-      const float lse = k_fanin<KBT, G>(rl + base, ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
+      const float lse = k_fanin<KBT, G>(rl + checked_base(ws, base, K),
+                                        ln.j, -(float)(si - Sb) - Grel, ln.d, mk, ksum, e, ln.act);
       const float Bt = (lse == NEG_INF) ? NEG_INF : (lse - sf) + proj_d(ws, d, pj, b, s, ln.cc);
       float St = 0.f;
       if (ln.leader) {
@@ -679,7 +686,8 @@ __global__ void __launch_bounds__(LB, 1)
         const float acc = label_fanin<CAT, G>(sm.pcur + par * PC + ln.j * CAT, ln.e, p);
         if (ln.leader) {
           const float g = label_log(acc, ln.tmax, shift, C, sm.Acur + par * C, n, trans, ln.c, true);
-          ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
+          if (checked_slot(ws, wslot, K))
+            ring_put<KBT>(rl, d, wslot, make_float2(g + sf, (Grel + n) + (float)(si - Sb)));
           const float Ys = (float)(Xc + (double)row[2 * C] + (double)(Grel + n));
           E = (g == NEG_INF || row[ln.c] == NEG_INF) ? 0.f : ex2(row[ln.c] + g + Ys);
           if (end_marg) end_marg[((size_t)b * (d.T + 1) + s) * C + ln.c] = E;
@@ -772,6 +780,20 @@ __global__ void selftest_wait_kernel(int* status, int spins) {
   if (!__syncthreads_or(!ok)) return;
   if (threadIdx.x == 0) set_status(status, ST_DEVICE_TIMEOUT);
 }
+
+#ifdef SEMICRF_BOUNDS_CHECK
+// One guarded store whose index is one past a 32-entry shared array: the
+// check records SITE_SELFTEST and skips the store (debug build only).
+__global__ void selftest_bounds_kernel(int* status, int idx) {
+  __shared__ int buf[32];
+  buf[threadIdx.x & 31] = 0;
+  __syncthreads();
+  if (threadIdx.x == 0 && SEMICRF_INB(status, idx >= 0 && idx < 32, ring::SITE_SELFTEST))
+    buf[idx] = 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && buf[0] == 12345) set_status(status, 0x7fffffff);  // keeps buf live
+}
+#endif
 
 // ----------------------------------------------------------------------------- launchers
 bool shape_supported(int KBT, int CAT, int G, int LB) {

@@ -25,6 +25,23 @@
 namespace semicrf {
 namespace ring {
 
+// Bounds-check sites (status >> 8 in the debug build), one per guarded access.
+enum BoundsSite {
+  SITE_TILE_ISSUE = 1,    // TMA prefix-sum tile: source rows inside the sequence
+  SITE_TILE_ROW = 2,      // a row pointer into the tile buffers
+  SITE_RING_WINDOW = 3,   // a lane's k fan-in window inside its label's ring row
+  SITE_RING_SLOT = 4,     // a ring write slot
+  SITE_VECTOR = 5,        // label-vector (p or V) store, local or in a cluster peer
+  SITE_KEPT_ROW = 6,      // kept per-boundary rows (p, acc, V, durations, frames)
+  SITE_STEP_ARRAYS = 7,   // per-label step arrays written by the helpers
+  SITE_WALK_STAGE = 8,    // traceback stage: rows copied fit the staging buffer
+  SITE_WALK_MARK = 9,     // traceback: a segment-start mark inside the stage
+  SITE_POST_TILE = 10,    // posterior pass: tile rows and halo inside the staged tile
+  SITE_POST_ITEM = 11,    // posterior pass: a segment end inside the staged rows
+  SITE_SEG_STORE = 12,    // checkpoint walk: the per-position store
+  SITE_SELFTEST = 13      // semicrf_selftest_bounds: an index past its array on purpose
+};
+
 // Per-step buffers are double-buffered by step parity (pcur, Acur) or
 // triple-buffered (maxslot): with one CTA barrier per step, a fast warp may
 // write the next step's copy while a slow one still reads this step's.
@@ -110,6 +127,15 @@ __device__ __forceinline__ void ring_put(float2* rl, const Dims& d, int slot, fl
     for (int x = slot + d.K; x < d.RL; x += d.K) rl[x] = v;
 }
 
+// A lane's ring window base and a ring write slot, after the bounds-check
+// build's test (in the release build: the base itself, and true).
+__device__ __forceinline__ int checked_base(const WsPtrs& ws, int base, int K) {
+  return SEMICRF_INB(ws.status, base >= 0 && base < K, SITE_RING_WINDOW) ? base : 0;
+}
+__device__ __forceinline__ bool checked_slot(const WsPtrs& ws, int slot, int K) {
+  return SEMICRF_INB(ws.status, slot >= 0 && slot < K, SITE_RING_SLOT);
+}
+
 // Ring entry of boundary `bnd` (0 <= bnd) for label c.
 __device__ __forceinline__ float2& ring_at(const Smem& sm, const Dims& d, int c, int bnd) {
   return sm.ring[(size_t)c * d.RL + (bnd % d.K)];
@@ -129,6 +155,10 @@ __device__ __forceinline__ void tile_issue(const Smem& sm, const Dims& d, const 
   const int buf = i & 1;
   const uint32_t bytes = (uint32_t)(TS * d.C * 4);
   const size_t row0 = (size_t)b * d.Tstride + (size_t)i * TS;
+  // bounds-check build: the tile's rows lie in sequence b's rows
+  if (!SEMICRF_INB(ws.status, i >= 0 && b >= 0 && b < d.B && (size_t)(i + 1) * TS <= (size_t)d.Tstride,
+                   SITE_TILE_ISSUE))
+    return;
   fence_proxy_async();
   mbar_expect_tx(&sm.mbar[buf], 2 * bytes);
   bulk_g2s(sm.tint + (size_t)buf * TS * d.C, ws.sint + row0 * d.C, bytes, &sm.mbar[buf]);

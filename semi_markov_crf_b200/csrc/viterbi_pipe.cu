@@ -177,6 +177,11 @@ __global__ void __launch_bounds__(LB, 1)
       __syncthreads();
     }
   };
+  // bounds-check build: a row pointer lies inside the two tile buffers
+  auto row_ok = [&](const int32_t* row) {
+    const ptrdiff_t o = row - sm.tint;
+    return o >= 0 && o + C <= 2 * TS * C;
+  };
 
   // combine lanes: trans2[x][c] of their sources x = jl*CAT + q (-inf past C);
   // helper lanes: dur2 of window index q*H + jl, k = 2 + WL - (q*H + jl)
@@ -330,8 +335,9 @@ __global__ void __launch_bounds__(LB, 1)
       const float a2 = vs.A2[(i & 1) * Cr + ccl];
       const float om = vs.Om[(i & 1) * Cr + ccl];
       const int okd = vs.Ok[(i & 1) * Cr + ccl];
-      const int si_n = crow_i[cc];  // row i: the next step's ring entry
-      const float sf_n = crow_f[cc];
+      const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
+      const int si_n = rok ? crow_i[cc] : 0;  // row i: the next step's ring entry
+      const float sf_n = rok ? crow_f[cc] : 0.f;
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
 #pragma unroll
@@ -355,22 +361,23 @@ __global__ void __launch_bounds__(LB, 1)
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
       const int kdec = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
+      const bool pok = SEMICRF_INB(ws.status, c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
-        if (act)
+        if (act && pok)
           for (int q = jl; q < N; q += G) st_cluster(vs.V + (i & 1) * d.xPC + c, q, v - n);
       } else {
-        if (leader) vs.V[(i & 1) * d.xPC + c] = v - n;
+        if (leader && pok) vs.V[(i & 1) * d.xPC + c] = v - n;
       }
       if (tid == 0) vs.nsl[i & 1] = n;
       // off the path: boundary i's kept rows (V relative to Phi_i, the chosen
       // duration; global stores after the critical store cost the path
       // least), then G[i-1]'s ring entry (frame Phi_{i-1})
-      if (leader) {
+      if (leader && SEMICRF_INB(ws.status, i <= T, SITE_KEPT_ROW)) {
         vrw[(size_t)i * C + c] = v - n;
         kdw[(size_t)i * C + c] = kdec;
       }
-      if (leader && i >= 2) {
+      if (leader && i >= 2 && SEMICRF_INB(ws.status, wslot >= 0 && wslot < K, SITE_RING_SLOT)) {
         const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
         for (int x = wslot; x < RL; x += K) rl[x] = e;
       }
@@ -393,14 +400,17 @@ __global__ void __launch_bounds__(LB, 1)
         m0 = fmaxf(m0, pv[q * H]);
         if (q + 1 < CA) m1 = fmaxf(m1, pv[(q + 1) * H]);
       }
-      const int sn = (i < L) ? hrow_i[cc] : 0;
-      const float fn = (i < L) ? hrow_f[cc] : 0.f;
+      const bool hok = i < L && SEMICRF_INB(ws.status, row_ok(hrow_i), SITE_TILE_ROW);
+      const int sn = hok ? hrow_i[cc] : 0;
+      const float fn = hok ? hrow_f[cc] : 0.f;
       const float Qh = (float)(sn - Sbc) - Fph;
+      const int hb = SEMICRF_INB(ws.status, hbase >= 0 && hbase + jl + (KBH - 1) * H < RLP,
+                                 SITE_RING_WINDOW) ? hbase : 0;
       float best = NEG_INF;
       float tv[KBH];
 #pragma unroll
       for (int q = 0; q < KBH; ++q) {
-        const float2 e = rl[hbase + q * H + jl];
+        const float2 e = rl[hb + q * H + jl];
         tv[q] = ((e.y + Qh) + e.x) + w[q];
         best = fmaxf(best, tv[q]);
       }
@@ -581,6 +591,8 @@ __global__ void __launch_bounds__(256)
     const int lo = max(1, tt0 - WR + 1);
     const int pb = lo - K;  // mark of position u at lbuf[u - pb]
     const uint32_t bytes = (uint32_t)((tt0 - lo + 1) * CP * 4);
+    // bounds-check build: the stage's rows fit the staging buffers
+    if (!SEMICRF_INB(ws.status, tt0 - lo + 1 <= WR && tt0 <= T, SITE_WALK_STAGE)) break;
     if (tid == 0) {
       fence_proxy_async();  // the last stage's reads come before the copies' writes
       mbar_expect_tx(&wbar, 2 * bytes);
@@ -611,7 +623,8 @@ __global__ void __launch_bounds__(256)
           break;
         }
         tt -= k;
-        lbuf[tt - pb] = cl;
+        if (SEMICRF_INB(ws.status, tt - pb >= 0 && tt - pb < WR + K, SITE_WALK_MARK))
+          lbuf[tt - pb] = cl;
         cl = pred;
         idx += step;
         if (tt >= lo && (idx < 0 || idx >= nidx)) {

@@ -16,7 +16,7 @@ import torch
 __all__ = ["workspace_bytes", "workspace_itemize", "WS_GROUPS", "launch_shape", "prefix_center", "forward", "backward", "viterbi", "path_score",
            "get_status", "FLAG_NEGATE_GRAD",
            "strerror", "SemiCRFError", "library_path", "Workspace", "FLAG_NO_CENTER",
-           "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "ring_domains", "profile_enable", "profile_read",
+           "FLAG_FORWARD_ONLY", "FLAG_LOG_DOMAIN", "selftest_bounded_wait", "selftest_bounds", "ring_domains", "profile_enable", "profile_read",
            "forward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "KERNELS", "lib"]
 
@@ -34,7 +34,10 @@ FLAG_LOG_DOMAIN = 0x4
 FLAG_NEGATE_GRAD = 0x8
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SEMICRF_NOALLOC_SCRATCH_BYTES
 
-library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsemicrf_b200.so")
+# SEMICRF_LIBRARY=check loads the bounds-checking debug build instead
+_LIBNAME = ("libsemicrf_b200_check.so" if os.environ.get("SEMICRF_LIBRARY") == "check"
+            else "libsemicrf_b200.so")
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIBNAME)
 if not os.path.exists(library_path):
     raise ImportError(f"{library_path} is missing: build it with `python -m semi_markov_crf_b200.build`")
 
@@ -70,6 +73,7 @@ lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
 lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
+lib.semicrf_selftest_bounds.argtypes = [_vp, _sz, _vp]
 lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _vp]
 lib.semicrf_ring_domains.argtypes = [_vp, _sz, _i, _i, _i, _i, _u, _vp, ctypes.POINTER(ctypes.c_int32)]
 lib.semicrf_profile_enable.argtypes = [_i]
@@ -78,7 +82,7 @@ for _f in ("semicrf_backward_segments", "semicrf_launch_shape", "semicrf_workspa
            "semicrf_backward", "semicrf_viterbi", "semicrf_path_score", "semicrf_get_status",
            "semicrf_forward_proj", "semicrf_backward_proj", "semicrf_viterbi_proj",
            "semicrf_path_score_proj",
-           "semicrf_selftest_bounded_wait", "semicrf_ring_domains"):
+           "semicrf_selftest_bounded_wait", "semicrf_selftest_bounds", "semicrf_ring_domains"):
     getattr(lib, _f).restype = _i
 
 
@@ -411,6 +415,18 @@ def selftest_bounded_wait(ws: Workspace, spins: int) -> int:
     _check(lib.semicrf_selftest_bounded_wait(ws.ptr, ws.nbytes, int(spins), _stream(ws.buf.device)),
            "semicrf_selftest_bounded_wait")
     return get_status(ws)
+
+
+def selftest_bounds(ws: Workspace) -> int:
+    """Bounds-checking build: runs one deliberately out-of-range guarded store
+    (skipped by its check) and returns the status word it leaves.  The
+    release build raises SemiCRFError(SEMICRF_ERR_UNSUPPORTED)."""
+    _check(lib.semicrf_selftest_bounds(ws.ptr, ws.nbytes, _stream(ws.buf.device)),
+           "semicrf_selftest_bounds")
+    st = _i(0)
+    _check(lib.semicrf_get_status(ws.ptr, _stream(ws.buf.device), ctypes.byref(st)),
+           "semicrf_get_status")
+    return int(st.value)
 
 
 def profile_enable(on: bool = True):

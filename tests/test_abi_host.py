@@ -116,8 +116,8 @@ def test_host_side_argument_errors_of_the_loss_and_projection_calls(lib):
 
 def test_strerror_names_every_status(lib):
     lib.semicrf_strerror.restype = ctypes.c_char_p
-    seen = {lib.semicrf_strerror(i).decode() for i in range(7)}
-    assert len(seen) == 7 and "unknown status" not in seen
+    seen = {lib.semicrf_strerror(i).decode() for i in range(8)}
+    assert len(seen) == 8 and "unknown status" not in seen
     assert lib.semicrf_strerror(99).decode() == "unknown status"
 
 

@@ -396,7 +396,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float sn = pow2_neg(n);
       const float R = fmaf(acc2, a2v, ohv) * snprev;  // frame Phi_{i-1}
       const float pn = fmaf(acc * sn, a1v, R * sn);
-      const bool pok = SEMICRF_INB(ws.status, c < d.xPC, SITE_VECTOR);
+      const bool pok = SEMICRF_INB(ws.status, !act || c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
         if (act && pok)

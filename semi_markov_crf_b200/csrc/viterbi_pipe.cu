@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(LB, 1)
       const float c3 = om - nprev;
       const float v = fmaxf(c1, fmaxf(c2, c3));
       const int kdec = (c1 >= c2 && c1 >= c3) ? 1 : (c2 >= c3 ? 2 : okd);
-      const bool pok = SEMICRF_INB(ws.status, c < d.xPC, SITE_VECTOR);
+      const bool pok = SEMICRF_INB(ws.status, !act || c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
         if (act && pok)

@@ -67,9 +67,10 @@ struct XSmem {
   float* nsl;  // [2]      frame step n published by the combine warps
   int* aux;    // [4]      block reductions
   int* Sb;     // [Cr]     label integer bases of the prefix sums
+  uint64_t* pbar;  // [2]  cluster: arrival of the step's label vector, by step parity
 };
 
-__device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
+__device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d, bool pj) {
   XSmem x;
   const int C = d.C, Cr = d.xCr;  // tile rows hold every label, the rest this CTA's
   unsigned char* p = raw;
@@ -78,11 +79,17 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d) {
   x.aux = reinterpret_cast<int*>(p + 32);
   x.s.aux = x.aux;
   x.nsl = reinterpret_cast<float*>(p + 48);
-  p += 64;
+  x.pbar = reinterpret_cast<uint64_t*>(p + 64);
+  p += 96;
   x.s.tint = reinterpret_cast<int32_t*>(p);
   p += 2ull * TS * C * sizeof(int32_t);
   x.s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
+  x.s.tpd = nullptr;
+  if (pj) {  // boundary projections: start terms stream with the prefix sums
+    x.s.tpd = reinterpret_cast<float*>(p);
+    p += 2ull * TS * C * sizeof(float);
+  }
   x.s.ring = reinterpret_cast<float2*>(p);
   p += (size_t)d.xRLP * Cr * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
@@ -134,11 +141,17 @@ __device__ __forceinline__ int next_mod(int i, int rem) {
 // With a cluster of N > 1 CTAs per ring, CTA `rank` owns labels
 // [rank*Cr, rank*Cr + Cr): its ring, its k fan-in and its label fan-in
 // outputs.  The label fan-in of every label needs the whole vector p_{t-1},
-// so each combine group stores its p_t into the P buffer of every CTA of the
-// cluster (plain distributed-shared-memory stores, the group's lanes taking
-// different destination CTAs) and the step ends with a cluster barrier
-// (release / acquire) instead of the CTA barrier.  Every CTA then holds the
-// same full vector and computes the same frame step n from it.
+// so each combine group sends its p_t into the P buffer of every CTA of the
+// cluster with asynchronous distributed-shared-memory stores (the group's
+// lanes taking different destination CTAs) that count against the
+// destination's arrival barrier pbar[t & 1] (4 C bytes per step).  A combine
+// lane waits on its own CTA's barrier before reading p_{t-1}, then its CTA
+// re-arms that barrier for step t+1; steps still end with the CTA barrier
+// only.  No release fence sits in the step (a cluster barrier's release
+// would also wait for the kept rows' global stores).  Every CTA holds the
+// same full vector and computes the same frame step n from it.  A barrier
+// phase is reused two steps later, by which time every CTA has read the
+// vector it held (the senders of step t+1 have received step t from all).
 template <bool UP, int N, int G, int CAT, int H, int KBH>
 __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPtrs& ws, int b,
                                       int L, const float* __restrict__ trans,
@@ -163,13 +176,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   const bool leader = act && jl == 0;
   const int RL = K + WL, RLP = d.xRLP;
   float2* const rl = sm.ring + (size_t)ccl * RLP;
-  auto step_sync = [&]() {
-    if constexpr (N > 1) {
-      cluster_sync();
-    } else {
-      __syncthreads();
-    }
-  };
+  const uint32_t vbytes = 4u * (uint32_t)C;  // label-vector bytes arriving per step (clusters)
   auto put = [&](int slot, float2 v) {  // slot and its mirrors slot + mK < RL
     for (int x = slot; x < RL; x += K) rl[x] = v;
   };
@@ -215,7 +222,15 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     xs.nsl[0] = xs.nsl[1] = 0.f;
     mbar_init(&sm.mbar[0], 1);
     mbar_init(&sm.mbar[1], 1);
+    if constexpr (N > 1) {
+      mbar_init(&xs.pbar[0], 1);
+      mbar_init(&xs.pbar[1], 1);
+    }
     fence_mbar_init();
+    if constexpr (N > 1) {
+      mbar_expect_tx(&xs.pbar[1], vbytes);  // step 1's vector
+      mbar_expect_tx(&xs.pbar[0], vbytes);  // step 2's vector
+    }
   }
   __syncthreads();
   const int r0 = UP ? 0 : L;  // the walk's start boundary
@@ -243,8 +258,10 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   }
   const size_t o0 = tile_row_off(r0, C), o1 = tile_row_off(r1, C);
   for (int x = tid; x < Cr && c0 + x < C; x += blockDim.x) {
-    // gamma[0] = 0 at S = 0 (forward); beta[L] = 0 at S[L] (backward)
-    const float2 v = make_float2(UP ? 0.f : sm.tfrac[o0 + c0 + x], 0.f);
+    // gamma[0] = 0 at S = 0 (forward; with projections the start term of
+    // boundary 0); beta[L] = 0 at S[L] (backward)
+    const float2 v = make_float2(UP ? (sm.tpd ? sm.tpd[o0 + c0 + x] : 0.f) : sm.tfrac[o0 + c0 + x],
+                                 0.f);
     float2* r = sm.ring + (size_t)x * RLP;
     for (int y = r0 % K; y < RL; y += K) r[y] = v;
     xs.Sb[x] = UP ? 0 : sm.tint[o0 + c0 + x];
@@ -253,21 +270,30 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   // acc and n of the last step, the frame of p_{i-1} relative to F0
   int si_p = UP ? 0 : sm.tint[o0 + cc], si_pp = si_p;
   float sf_p = UP ? 0.f : sm.tfrac[o0 + cc];
+  // boundary projections (sm.tpd set): the start term pd of a row, added
+  // wherever its boundary takes the start role -- forward ring entries and
+  // the k = 1, 2 factors (rows r-1, r-2 of the step); backward every term
+  // of the step's own row
+  float pd_p = sm.tpd ? sm.tpd[o0 + cc] : 0.f;
   float acc2 = 0.f, snprev = 1.f, Fp = 0.f;
   int wslot = r0 % K;
   const int32_t* crow_i = sm.tint + o1;
   const float* crow_f = sm.tfrac + o1;
+  const float* crow_d = sm.tpd ? sm.tpd + o1 : nullptr;
   // helper state: rows r (cur) and r-1 (prev) of S, frame Phi_{i-1} - F0,
   // predicted shift relative to Q, window base
   int hs_c = sm.tint[o1 + cc], hs_p = si_p;
   float hf_c = sm.tfrac[o1 + cc], hf_p = sf_p;
+  float hd_c = sm.tpd ? sm.tpd[o1 + cc] : 0.f, hd_p = pd_p;
   float Fph = 0.f, rel = 0.f;
   const int32_t* hrow_i = sm.tint + o1 + SG * C;  // row r + SG of step 1
   const float* hrow_f = sm.tfrac + o1 + SG * C;
+  const float* hrow_d = sm.tpd ? sm.tpd + o1 + SG * C : nullptr;
   int hbase = UP ? -WL : L + 1;  // window start boundary at step 1
   hbase = ((hbase % K) + K) % K;
   if (!comb && leader)  // step 1's k = 1 factor (no k = 2 term, no k >= 3 terms)
-    xs.A1[Cr + cl] = ex2((M + d1) + sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
+    xs.A1[Cr + cl] = ex2(((M + d1) + (UP ? hd_p : hd_c)) +
+                         sg * ((float)(hs_c - hs_p) + (hf_c - hf_p)));
   double F0 = 0.0;
   // kept values for the posterior pass: per boundary (row) the vector p and
   // the label fan-in acc, relative to the boundary's frame kf, stored by the
@@ -283,9 +309,14 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     }
     if (tid == 0 && rank == 0) kf[r0] = 0.0;
   }
-  // every CTA of a cluster has initialised its P buffer before any other
-  // stores into it
-  step_sync();
+  // every CTA of a cluster has initialised its P buffer and arrival
+  // barriers before any other CTA stores into them
+  if constexpr (N > 1) {
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
+  bool xdead = false;  // cluster: an arrival wait gave up (results are then meaningless)
   int Sbc = xs.Sb[ccl];
   // checkpoint steps: forward boundary t = i - 1 at step i; backward
   // boundary t1 = r + 2 at step i
@@ -320,12 +351,14 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         const size_t o = tile_row_off(r + SG, C);
         hrow_i = sm.tint + o;
         hrow_f = sm.tfrac + o;
+        if (sm.tpd) hrow_d = sm.tpd + o;
       }
       if (i % TS == rem_i) {
         if (!dead) tile_issue(sm, d, ws, b, ts, r / TS + SG);
         const size_t o = tile_row_off(r, C);
         crow_i = sm.tint + o;
         crow_f = sm.tfrac + o;
+        if (sm.tpd) crow_d = sm.tpd + o;
       }
       if (i == next_ck) {
         // rebase the ring to (F0 + D, S_int at the boundary): keeps the
@@ -362,11 +395,23 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
     // before the barrier releases.
     if (comb) {
       // ---------------------------------------------------------- combine
+      if constexpr (N > 1) {
+        if (i >= 2) {
+          // p_{i-1} from every CTA of the cluster, then re-arm for step i+1
+          const int pb = (i - 1) & 1;
+          if (!xdead && !mbar_wait_cluster(&xs.pbar[pb], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
+            set_status(ws.status, ST_DEVICE_TIMEOUT);
+            xdead = true;
+          }
+          if (tid == 0 && i + 1 <= L) mbar_expect_tx(&xs.pbar[pb], vbytes);
+        }
+      }
       const int po = (i & 1) * Cr + ccl;
       const float a1v = xs.A1[po], a2v = xs.A2[po], ohv = xs.Oh[po];
       const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
       const int si_n = rok ? crow_i[cc] : 0;  // the walk's row r: the next step's ring entry
       const float sf_n = rok ? crow_f[cc] : 0.f;
+      const float pd_n = (UP && crow_d && rok) ? crow_d[cc] : 0.f;
       const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
 #pragma unroll
@@ -400,7 +445,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
         if (act && pok)
-          for (int q = jl; q < N; q += G) st_cluster(xs.P + (i & 1) * d.xPC + c, q, pn);
+          for (int q = jl; q < N; q += G)
+            st_async_cluster(xs.P + (i & 1) * d.xPC + c, xs.pbar + (i & 1), q, pn);
       } else {
         if (leader && pok) xs.P[(i & 1) * d.xPC + c] = pn;
       }
@@ -414,7 +460,7 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         kv[(size_t)(r - SG) * 2 * C + C + c] = acc;    // row r - SG, frame Phi_{i-1}
       }
       if (i >= 2 && leader && SEMICRF_INB(ws.status, wslot >= 0 && wslot < K, SITE_RING_SLOT))
-        put(wslot, make_float2(gprev - sg * sf_p, Fp - sg * (float)(si_p - Sbc)));
+        put(wslot, make_float2((gprev - sg * sf_p) + pd_p, Fp - sg * (float)(si_p - Sbc)));
       wslot = UP ? (wslot + 1 == K ? 0 : wslot + 1) : (wslot == 0 ? K - 1 : wslot - 1);
       acc2 = acc;
       snprev = sn;
@@ -422,13 +468,16 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       si_pp = si_p;
       si_p = si_n;
       sf_p = sf_n;
+      pd_p = pd_n;
       crow_i += SG * C;
       crow_f += SG * C;
+      if (crow_d) crow_d += SG * C;
     } else if (i < L) {
       // ---------------------------------------------------------- helpers
       const bool hok = SEMICRF_INB(ws.status, row_ok(hrow_i), SITE_TILE_ROW);
       const int sn = hok ? hrow_i[cc] : 0;
       const float fn = hok ? hrow_f[cc] : 0.f;
+      const float dn = (hrow_d && hok) ? hrow_d[cc] : 0.f;
       const bool wok = SEMICRF_INB(ws.status, hbase >= 0 && hbase + jl + (KBH - 1) * H < RLP,
                                    SITE_RING_WINDOW);
       const float Qh = sg * (float)(sn - Sbc) - Fph;
@@ -438,9 +487,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       if (isfinite(lse)) rel = rintf(lse - Qh);
       // the three values step i+1 reads: lanes 0, 1, 2 of the group take one
       // exponential each (no divergent branches); narrower groups take all
-      const float aO = m + sg * fn;
-      const float aA1 = (M + d1) + sg * ((float)(sn - hs_c) + (fn - hf_c));
-      const float aA2 = (M + d2) + sg * ((float)(sn - hs_p) + (fn - hf_p));
+      const float aO = (m + (UP ? 0.f : dn)) + sg * fn;
+      const float aA1 = ((M + d1) + (UP ? hd_c : dn)) + sg * ((float)(sn - hs_c) + (fn - hf_c));
+      const float aA2 = ((M + d2) + (UP ? hd_p : dn)) + sg * ((float)(sn - hs_p) + (fn - hf_p));
       const int o2 = ((i + 1) & 1) * Cr + ccl;
       if constexpr (H >= 3) {
         const float e = ex2(jl == 0 ? aO : (jl == 1 ? aA1 : aA2));
@@ -457,13 +506,24 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       }
       hs_p = hs_c;
       hf_p = hf_c;
+      hd_p = hd_c;
       hs_c = sn;
       hf_c = fn;
+      hd_c = dn;
       hrow_i += SG * C;
       hrow_f += SG * C;
+      if (hrow_d) hrow_d += SG * C;
       hbase = UP ? (hbase + 1 == K ? 0 : hbase + 1) : (hbase == 0 ? K - 1 : hbase - 1);
     }
-    step_sync();
+    __syncthreads();
+  }
+  if constexpr (N > 1) {
+    // the last vector has arrived here (log Z reads it; no store into this
+    // CTA is left in flight), then no CTA leaves before every CTA is done
+    if (comb && !xdead &&
+        !mbar_wait_cluster(&xs.pbar[L & 1], ((L - 1) >> 1) & 1, WAIT_SPIN_LIMIT))
+      set_status(ws.status, ST_DEVICE_TIMEOUT);
+    cluster_sync();
   }
   if (kv && rank == 0 && tid == nwc * 32)  // the last row's frame (its vector was kept at step L)
     kf[UP ? L : 0] = F0 + (double)(Fph + xs.nsl[L & 1]);
@@ -487,8 +547,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
 
 }  // namespace
 
-size_t chain_exp_smem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
+size_t chain_exp_smem_bytes(const Dims& d, bool pj) {
+  return 96 + 2ull * TS * d.C * (pj ? 12 : 8) + (size_t)d.xRLP * d.xCr * 8 + 16 +
          (2ull * d.xPC + 7ull * d.xCr) * 4;
 }
 
@@ -509,9 +569,9 @@ template <int N, int G, int CAT, int H, int KBH, int LB>
 __global__ void __launch_bounds__(LB, 1)
     chain_exp_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                      const float* __restrict__ trans, const float* __restrict__ dur,
-                     double* __restrict__ logZ_out, int n_alpha) {
+                     double* __restrict__ logZ_out, int n_alpha, int pj) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const XSmem xs = xcarve(smem_raw, d);
+  const XSmem xs = xcarve(smem_raw, d, pj != 0);
   const int C = d.C, K = d.K, tid = threadIdx.x;
   const int rank = N > 1 ? (int)cluster_ctarank() : 0;
   const int q = (int)blockIdx.x / N;
@@ -586,12 +646,12 @@ bool xshape_supported(int N, int G, int CAT, int H, int KBH, int LB) {
 
 cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, double* logZ_out, int n_alpha,
-                             int n_beta, cudaStream_t st) {
-  const size_t sm = chain_exp_smem_bytes(d);
+                             int n_beta, cudaStream_t st, int pj) {
+  const size_t sm = chain_exp_smem_bytes(d, pj != 0);
 #define SEMICRF_LAUNCH_XCHAIN(n, g, cat, h, kbh, lb)                                           \
   if (d.xN == n && d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb)    \
     return launch_clustered(chain_exp_kernel<n, g, cat, h, kbh, lb>, n, (n_alpha + n_beta) * n, \
-                            d.xNT, sm, st, d, ws, lengths, trans, dur, logZ_out, n_alpha);
+                            d.xNT, sm, st, d, ws, lengths, trans, dur, logZ_out, n_alpha, pj);
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_XCHAIN)
 #undef SEMICRF_LAUNCH_XCHAIN
   return cudaErrorInvalidConfiguration;

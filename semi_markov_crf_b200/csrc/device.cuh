@@ -153,6 +153,39 @@ __device__ __forceinline__ void st_cluster(const float* local, uint32_t rank, fl
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
+// Asynchronous store of one float into the shared memory of CTA `rank` of
+// this cluster (the offset `local` has here), completing `bytes` = 4 of the
+// transaction count of that CTA's mbarrier at the offset of `bar`.  The
+// receiver learns of the data by waiting on its own mbarrier; no memory
+// fence is involved on either side.  No multicast.
+__device__ __forceinline__ void st_async_cluster(const float* local, const uint64_t* bar,
+                                                 uint32_t rank, float v) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_addr(bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(ra),
+               "r"(__float_as_uint(v)), "r"(rb)
+               : "memory");
+}
+
+// Bounded wait, with cluster-scope acquire, for phase `parity` of `bar`
+// (data delivered by st_async_cluster from any CTA of the cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int spins) {
+  const uint32_t a = smem_addr(bar);
+  for (int i = 0; i < spins; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 // Bounded wait for phase `parity` of `bar`.  Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int spins) {
   const uint32_t a = smem_addr(bar);

@@ -152,7 +152,9 @@ cudaError_t launch_clustered(void (*kern)(KArgs...), int n_cluster, int grid, in
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-size_t chain_exp_smem_bytes(const Dims& d);
+// pj: the call has boundary projections (the tile stream carries their
+// start terms; the kernels add them where a boundary takes the start role).
+size_t chain_exp_smem_bytes(const Dims& d, bool pj = false);
 size_t viterbi_pipe_smem_bytes(const Dims& d);
 // After viterbi_pipe: the backpointer words from the kept rows (grid-wide),
 // then the traceback (one CTA per sequence, `sm` bytes of shared memory).
@@ -170,7 +172,7 @@ bool xshape_supported(int N, int G, int CAT, int H, int KBH, int LB);
 // the exponential domain; writes ws.mode for every (direction, sequence).
 cudaError_t launch_chain_exp(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, double* logZ_out, int n_alpha,
-                             int n_beta, cudaStream_t st);
+                             int n_beta, cudaStream_t st, int pj = 0);
 
 // g_b times the boundary marginals as the boundary-projection gradients
 // (finalize.cu); start_marg / end_marg are [B][T+1][C].

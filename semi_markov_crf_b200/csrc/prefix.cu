@@ -121,12 +121,13 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
     for (int r = g * RB; r < min((g + 1) * RB, R); ++r) {
       const int t = r0 + r + 1;
       if (t > T) break;
-      double val = 0.0;
+      double val = 0.0, xa = 0.0;
       if (r < nrows) {
         const double x = (double)tile[r * C + c] - nuc;
         run += x;
         val = run;
-        emx = fmaxf(emx, (float)fabs(x));
+        xa = fabs(x);
+        emx = fmaxf(emx, (float)xa);
       }
       const bool valid = (t <= L);
       if (mode == 0) {
@@ -140,6 +141,9 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
           pe = (valid && p_end) ? (double)__ldg(p_end + q) : 0.0;
           const double ps = (t < L && p_start) ? (double)__ldg(p_start + q + C) : 0.0;
           ws.pd[o] = (float)((pe + ps) * LOG2E_D);
+          // the exponential-domain test bounds a step's swing: with
+          // projections a position's terms include both of them
+          if (valid) emx = fmaxf(emx, (float)(xa + fabs(pe) + fabs(ps)));
         }
         const double s2 = valid ? (val + pe) * LOG2E_D : 0.0;
         const double ip = rint(s2);

@@ -51,6 +51,8 @@ struct Smem {
   int* aux;         // [1] block-wide max of the transition scores
   int32_t* tint;    // [2][TS][C]
   float* tfrac;     // [2][TS][C]
+  float* tpd;       // [2][TS][C] projection start terms (pipelined kernels with
+                    // boundary projections; nullptr otherwise)
   float2* ring;     // [C][RL]
   float* pcur;      // [2][PC] exp-domain label vector (zero padded)
   float* Acur;      // [2][C]
@@ -73,6 +75,7 @@ __device__ __forceinline__ Smem carve(unsigned char* raw, const Dims& d, bool wi
   p += 2ull * TS * C * sizeof(int32_t);
   s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
+  s.tpd = nullptr;
   s.ring = reinterpret_cast<float2*>(p);
   p += (size_t)d.RL * C * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
@@ -160,9 +163,10 @@ __device__ __forceinline__ void tile_issue(const Smem& sm, const Dims& d, const 
                    SITE_TILE_ISSUE))
     return;
   fence_proxy_async();
-  mbar_expect_tx(&sm.mbar[buf], 2 * bytes);
+  mbar_expect_tx(&sm.mbar[buf], (sm.tpd ? 3 : 2) * bytes);
   bulk_g2s(sm.tint + (size_t)buf * TS * d.C, ws.sint + row0 * d.C, bytes, &sm.mbar[buf]);
   bulk_g2s(sm.tfrac + (size_t)buf * TS * d.C, ws.sfrac + row0 * d.C, bytes, &sm.mbar[buf]);
+  if (sm.tpd) bulk_g2s(sm.tpd + (size_t)buf * TS * d.C, ws.pd + row0 * d.C, bytes, &sm.mbar[buf]);
 }
 
 // Rows lo_row..hi_row will be visited starting at first_row.

@@ -59,6 +59,7 @@ struct VSmem {
   float* nsl;  // [2]       frame step published by the combine warps
   float* mx;   // [2]       max V[t-1] published by the helpers at step t
   int* Sb;     // [Cr]      label integer bases
+  uint64_t* vbar;  // [2]   cluster: arrival of the step's V row, by step parity
 };
 
 __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
@@ -70,7 +71,8 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   x.s.aux = reinterpret_cast<int*>(p + 32);
   x.nsl = reinterpret_cast<float*>(p + 48);
   x.mx = reinterpret_cast<float*>(p + 56);
-  p += 64;
+  x.vbar = reinterpret_cast<uint64_t*>(p + 64);
+  p += 96;
   x.s.tint = reinterpret_cast<int32_t*>(p);
   p += 2ull * TS * C * sizeof(int32_t);
   x.s.tfrac = reinterpret_cast<float*>(p);
@@ -100,7 +102,7 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
-  return 64 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
+  return 96 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
          (2ull * d.xPC + 9ull * d.xCr) * 4;
 }
 
@@ -121,10 +123,13 @@ __device__ __forceinline__ int next_with_rem(int i, int rem) {
 //
 // With a cluster of N > 1 CTAs per sequence, CTA `rank` owns labels
 // [rank*Cr, rank*Cr + Cr) (ring, k fan-in, label fan-in outputs); each
-// combine group stores its V[t] into the V buffer of every CTA of the
-// cluster (plain distributed-shared-memory stores) and each step ends with a
-// cluster barrier, so every CTA holds the whole row and takes the same frame.
-// Every CTA takes the same early exits (they depend only on the inputs).
+// combine group sends its V[t] into the V buffer of every CTA of the cluster
+// with asynchronous distributed-shared-memory stores counted by the
+// destination's arrival barrier vbar[t & 1] (4 C bytes per step); a combine
+// lane waits on it before reading V[t-1] and the CTA re-arms it for step t+1
+// (the same exchange as the exponential-domain rings), so every CTA holds the
+// whole row and takes the same frame.  Every CTA takes the same early exits
+// (they depend only on the inputs).
 template <int N, int G, int CAT, int H, int KBH, int LB>
 __global__ void __launch_bounds__(LB, 1)
     viterbi_pipe_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
@@ -170,13 +175,7 @@ __global__ void __launch_bounds__(LB, 1)
   const bool leader = act && jl == 0;
   const int RL = K + WL, RLP = d.xRLP;
   float2* const rl = sm.ring + (size_t)ccl * RLP;
-  auto step_sync = [&]() {
-    if constexpr (N > 1) {
-      cluster_sync();
-    } else {
-      __syncthreads();
-    }
-  };
+  const uint32_t vbytes = 4u * (uint32_t)C;  // V-row bytes arriving per step (clusters)
   // bounds-check build: a row pointer lies inside the two tile buffers
   auto row_ok = [&](const int32_t* row) {
     const ptrdiff_t o = row - sm.tint;
@@ -218,7 +217,15 @@ __global__ void __launch_bounds__(LB, 1)
     vs.mx[0] = vs.mx[1] = NEG_INF;
     mbar_init(&sm.mbar[0], 1);
     mbar_init(&sm.mbar[1], 1);
+    if constexpr (N > 1) {
+      mbar_init(&vs.vbar[0], 1);
+      mbar_init(&vs.vbar[1], 1);
+    }
     fence_mbar_init();
+    if constexpr (N > 1) {
+      mbar_expect_tx(&vs.vbar[1], vbytes);  // step 1's row
+      mbar_expect_tx(&vs.vbar[0], vbytes);  // step 2's row
+    }
   }
   __syncthreads();
   TileStream ts;
@@ -270,9 +277,14 @@ __global__ void __launch_bounds__(LB, 1)
   const float* crow_f = sm.tfrac + C;
   int wslot = 0;
   double F0 = 0.0;
-  // every CTA of a cluster has initialised its V buffer before any other
-  // stores into it
-  step_sync();
+  // every CTA of a cluster has initialised its V buffer and arrival barriers
+  // before any other CTA stores into them
+  if constexpr (N > 1) {
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
+  bool xdead = false;  // cluster: an arrival wait gave up (results are then meaningless)
   int Sbc = 0;
   int next_rb = VREBASE + 1;
   // next step with an event: a tile to wait for (row i+1 opens a tile), a
@@ -330,6 +342,17 @@ __global__ void __launch_bounds__(LB, 1)
     // complete before the barrier releases.
     if (comb) {
       // ---------------------------------------------------------- combine
+      if constexpr (N > 1) {
+        if (i >= 2) {
+          // V[i-1] from every CTA of the cluster, then re-arm for step i+1
+          const int pb = (i - 1) & 1;
+          if (!xdead && !mbar_wait_cluster(&vs.vbar[pb], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
+            set_status(ws.status, ST_DEVICE_TIMEOUT);
+            xdead = true;
+          }
+          if (tid == 0 && i + 1 <= L) mbar_expect_tx(&vs.vbar[pb], vbytes);
+        }
+      }
       const float mp = vs.mx[(i - 1) & 1];
       const float a1 = vs.A1[(i & 1) * Cr + ccl];
       const float a2 = vs.A2[(i & 1) * Cr + ccl];
@@ -365,7 +388,8 @@ __global__ void __launch_bounds__(LB, 1)
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
         if (act && pok)
-          for (int q = jl; q < N; q += G) st_cluster(vs.V + (i & 1) * d.xPC + c, q, v - n);
+          for (int q = jl; q < N; q += G)
+            st_async_cluster(vs.V + (i & 1) * d.xPC + c, vs.vbar + (i & 1), q, v - n);
       } else {
         if (leader && pok) vs.V[(i & 1) * d.xPC + c] = v - n;
       }
@@ -393,6 +417,14 @@ __global__ void __launch_bounds__(LB, 1)
       // ---------------------------------------------------------- helpers
       // reads: row V[i-1] for the frame max, the window of the k >= 3 terms
       // of step i + 1 (boundaries i - 1 - WL .. i - 2) and its prefix-sum row
+      if constexpr (N > 1) {
+        // V[i-1] from every CTA of the cluster (the combine lanes re-arm)
+        if (i >= 2 && !xdead &&
+            !mbar_wait_cluster(&vs.vbar[(i - 1) & 1], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
+          set_status(ws.status, ST_DEVICE_TIMEOUT);
+          xdead = true;
+        }
+      }
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
       float m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
@@ -446,7 +478,15 @@ __global__ void __launch_bounds__(LB, 1)
         hbase = (hbase + 1 == K) ? 0 : hbase + 1;
       }
     }
-    step_sync();
+    __syncthreads();
+  }
+  if constexpr (N > 1) {
+    // the last row has arrived here (the score reads it; no store into this
+    // CTA is left in flight), then no CTA leaves before every CTA is done
+    if (comb && !xdead &&
+        !mbar_wait_cluster(&vs.vbar[L & 1], ((L - 1) >> 1) & 1, WAIT_SPIN_LIMIT))
+      set_status(ws.status, ST_DEVICE_TIMEOUT);
+    cluster_sync();
   }
   // the optimum: max over the final labels of V[L] in frame Phi_L
   if (tid < 32 && rank == 0) {

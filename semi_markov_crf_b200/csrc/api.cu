@@ -427,13 +427,24 @@ struct ProfScope {
 // Both rings (forward of n_alpha sequences, backward of n_beta): the
 // exponential-domain kernel takes every sequence whose scores fit it and
 // marks the rest, which the log-domain kernel then runs.
+// Whether the pipelined exponential-domain kernels serve this call: their
+// shape exists, the log domain is not forced, and with boundary projections
+// their larger tile stream still fits shared memory.
+bool pipelined(const Dims& d, unsigned flags, bool proj) {
+  if (!d.xG || (flags & SEMICRF_FLAG_LOG_DOMAIN)) return false;
+  if (!proj) return true;
+  const size_t budget = (size_t)max_smem_optin() - 256;
+  return chain_exp_smem_bytes(d, true) <= budget && viterbi_pipe_smem_bytes(d, true) <= budget &&
+         posterior_smem_bytes(d) <= budget;
+}
+
 int run_chains(const Dims& d, WsPtrs p, const int32_t* lengths, const float* trans,
                const float* dur, double* logZ, int n_alpha, int n_beta, unsigned flags,
-               cudaStream_t st) {
+               cudaStream_t st, bool proj = false) {
   cudaError_t e = cudaSuccess;
-  if (d.xG && !(flags & SEMICRF_FLAG_LOG_DOMAIN)) {
+  if (pipelined(d, flags, proj)) {
     ProfScope ps("chain_exp_kernel", st);
-    e = launch_chain_exp(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st);
+    e = launch_chain_exp(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st, proj ? 1 : 0);
   } else {
     // no ring kept anything: the posterior pass must not trust a record left
     // in the workspace by an earlier call
@@ -547,15 +558,12 @@ int forward_impl(const float* em, const int32_t* lengths, const float* trans, co
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
   const bool proj = p_start || p_end;
-  // projections run on the log-domain rings (the exponential-domain kernels
-  // have no projection term)
-  if (proj) flags |= SEMICRF_FLAG_LOG_DOMAIN;
   if ((rc = reset_status(p, proj, st))) return rc;
   if (B == 0) return SEMICRF_OK;
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st, p_start, p_end);
   if (rc) return rc;
   const int nbeta = (flags & SEMICRF_FLAG_FORWARD_ONLY) ? 0 : B;
-  return run_chains(d, p, lengths, trans, dur, logZ, B, nbeta, flags, st);
+  return run_chains(d, p, lengths, trans, dur, logZ, B, nbeta, flags, st, proj);
 }
 
 }  // namespace
@@ -588,14 +596,21 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
   WsPtrs p;
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
-  if (proj) flags |= SEMICRF_FLAG_LOG_DOMAIN;  // as the forward with projections ran
+  if (proj && !pipelined(d, flags, true)) flags |= SEMICRF_FLAG_LOG_DOMAIN;  // as the forward ran
   const bool want_pg = (grad_p_start || grad_p_end) && T > 0;
   if (want_pg) {
     // the projection gradients are g times the boundary marginals; without
-    // caller buffers those go to the exponential-domain rows of the
-    // workspace, which a run with projections does not use
-    if (!start_marg) start_marg = p.kv;
-    if (!end_marg) end_marg = p.kv + (size_t)B * (T + 1) * C;
+    // caller buffers those go to the decoder's rows of the workspace
+    // ([B][T+1][C] four-byte entries each, unused between a forward and its
+    // backward), or, without a pipelined shape, to the exponential-domain
+    // rows (then unused too)
+    if (d.xG) {
+      if (!start_marg) start_marg = p.vrow;
+      if (!end_marg) end_marg = reinterpret_cast<float*>(p.bp);
+    } else {
+      if (!start_marg) start_marg = p.kv;
+      if (!end_marg) end_marg = p.kv + (size_t)B * (T + 1) * C;
+    }
   }
   if (B == 0) {
     if (cudaMemsetAsync(grad_trans, 0, (size_t)C * C * 4, st) != cudaSuccess ||
@@ -604,7 +619,7 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
     return SEMICRF_OK;
   }
   if (flags & SEMICRF_FLAG_FORWARD_ONLY) {
-    rc = run_chains(d, p, lengths, trans, dur, nullptr, 0, B, flags, st);
+    rc = run_chains(d, p, lengths, trans, dur, nullptr, 0, B, flags, st, proj);
     if (rc) return rc;
   }
   // segment marginals: every entry the posterior kernels do not write (past
@@ -632,13 +647,14 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
       if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
       {
         ProfScope ps("cut_grid_kernel", st);
-        cut_grid_kernel<<<dim3(d.ngrid, B), 256, csm, st>>>(d, p, lengths, trans, dur);
+        cut_grid_kernel<<<dim3(d.ngrid, B), 256, csm, st>>>(d, p, lengths, trans, dur,
+                                                            proj ? 1 : 0);
       }
       if ((rc = launched())) return rc;
       {
         ProfScope ps("posterior_kernel", st);
         e = launch_posterior(d, p, lengths, trans, dur, grad_logZ, grad_em, start_marg, end_marg, st,
-                             seg_marg);
+                             seg_marg, proj ? 1 : 0);
       }
     }
     if (!side_join(ss, st)) return SEMICRF_ERR_CUDA;
@@ -743,12 +759,12 @@ int viterbi_impl(const float* em, const int32_t* lengths, const float* trans, co
   rc = run_prefix(em, lengths, d, p, flags, 1, nullptr, nullptr, st, p_start, p_end);
   if (rc) return rc;
   cudaError_t e;
-  // the pipelined decoder has no projection term: with projections the
-  // one-role kernel decodes
-  if (d.xG && !proj) {
+  // the pipelined decoder, unless no shape fits (then the one-role kernel)
+  if (pipelined(d, 0, proj)) {
     {
       ProfScope ps("viterbi_pipe_kernel", st);
-      e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st);
+      e = launch_viterbi_pipe(d, p, lengths, trans, dur, score, labels, seg_start, st,
+                              proj ? 1 : 0);
     }
     if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
     {

@@ -56,14 +56,15 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
 }
 
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                                const float* __restrict__ trans, const float* __restrict__ dur);
+                                const float* __restrict__ trans, const float* __restrict__ dur,
+                                int pj);
 // The posterior pass (one CTA per checkpoint segment and sequence).
 // seg_marg (nullable) [B][T][K][C]: the segment marginals of the sequences
 // the kernel takes (the caller zeroes the array first).
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,
                              float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
-                             float* seg_marg = nullptr);
+                             float* seg_marg = nullptr, int pj = 0);
 size_t posterior_smem_bytes(const Dims& d);
 // Tile rows for the posterior pass under `budget` bytes of shared memory (0:
 // none fits).
@@ -155,7 +156,7 @@ cudaError_t launch_clustered(void (*kern)(KArgs...), int n_cluster, int grid, in
 // pj: the call has boundary projections (the tile stream carries their
 // start terms; the kernels add them where a boundary takes the start role).
 size_t chain_exp_smem_bytes(const Dims& d, bool pj = false);
-size_t viterbi_pipe_smem_bytes(const Dims& d);
+size_t viterbi_pipe_smem_bytes(const Dims& d, bool pj = false);
 // After viterbi_pipe: the backpointer words from the kept rows (grid-wide),
 // then the traceback (one CTA per sequence, `sm` bytes of shared memory).
 cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
@@ -166,7 +167,7 @@ cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* 
 // Viterbi with the pipelined schedule (shapes of SEMICRF_FOR_EACH_XSHAPE).
 cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 const float* trans, const float* dur, double* score,
-                                int32_t* labels, uint8_t* seg_start, cudaStream_t st);
+                                int32_t* labels, uint8_t* seg_start, cudaStream_t st, int pj = 0);
 bool xshape_supported(int N, int G, int CAT, int H, int KBH, int LB);
 // Same grid and outputs as launch_chain for the sequences whose scores fit
 // the exponential domain; writes ws.mode for every (direction, sequence).

@@ -71,7 +71,7 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 // per label sums them (its max first, so the sum cannot overflow).
 __global__ void __launch_bounds__(256)
     cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                    const float* __restrict__ trans, const float* __restrict__ dur) {
+                    const float* __restrict__ trans, const float* __restrict__ dur, int pj) {
   extern __shared__ float csh[];  // la [K][C], lb [K][C], dd [K][C]
   __shared__ float lab_M[128], lab_f[128];  // per label: shift, log2 share
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -110,7 +110,8 @@ __global__ void __launch_bounds__(256)
       const float a = kf0[(size_t)s * 2 * C + C + c];
       if (a > 0.f)
         va = (lg2(a) + (float)(kf_at(ws, d, b, 0, s) - Fu)) -
-             ((float)(si[(size_t)s * C + c] - su) + (sf[(size_t)s * C + c] - fu));
+             ((float)(si[(size_t)s * C + c] - su) + (sf[(size_t)s * C + c] - fu)) +
+             (pj ? ws.pd[((size_t)b * d.Tstride + s) * C + c] : 0.f);  // start-side projection
     }
     if (t <= L) {
       const float bt = kf1[(size_t)t * 2 * C + C + c];
@@ -165,6 +166,7 @@ size_t cut_grid_smem_bytes(const Dims& d) { return 3ull * d.K * d.C * sizeof(flo
 namespace {
 
 // Shared memory carve of posterior_kernel for a tile of RT boundaries.
+// (With boundary projections pd holds the start terms of the tile's rows.)
 struct PTile {
   double* dif;  // [RT][C]   St - E of each boundary and label
   float* tf;    // [RT][2C]  forward kept rows: p, acc
@@ -174,10 +176,11 @@ struct PTile {
   float* sf;    // [R][C]    S_frac[r, c]
   float* vv;    // [RT][C]   suffix sums v of the tile
   float* fs;    // [RT]      f_s
+  float* pd;    // [RT][C]   projection start terms of the tile's rows (0 without)
 };
 __host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int K, int C) {
   const size_t R = (size_t)RT + K;
-  return (size_t)C * (24ull * RT + 12ull * R) + 4ull * RT;
+  return (size_t)C * (28ull * RT + 12ull * R) + 4ull * RT;
 }
 __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, int C) {
   PTile t;
@@ -190,6 +193,7 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, 
   t.sf = reinterpret_cast<float*>(t.ii + R * C);
   t.vv = t.sf + R * C;
   t.fs = t.vv + (size_t)RT * C;
+  t.pd = t.fs + RT;
   return t;
 }
 
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
                      const float* __restrict__ trans, const float* __restrict__ dur,
                      const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
                      float* __restrict__ start_marg, float* __restrict__ end_marg,
-                     float* __restrict__ seg_marg) {
+                     float* __restrict__ seg_marg, int pj) {
   extern __shared__ __align__(16) unsigned char psh[];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
   const int C = d.C, K = d.K, RT = d.pRT;
@@ -262,7 +266,10 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
       tl.ab[i] = pbr[row * 2 * C + C + c];
       tl.ii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
       tl.sf[i] = sfp[row * C + c];
-      if (r < nr) tl.pb[i] = pbr[row * 2 * C + c];
+      if (r < nr) {
+        tl.pb[i] = pbr[row * 2 * C + c];
+        tl.pd[i] = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
+      }
     }
     // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s))
     for (int s = s_lo + tid; s < s_hi; s += nthr)
@@ -290,7 +297,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
         if (!SEMICRF_INB(ws.status, r + k < nh, SITE_POST_ITEM)) continue;
         const int o = r * C + c, ok = (r + k) * C + c;
         const float z = (float)(tl.ii[ok] - tl.ii[o]) +
-                        ((M + __ldg(dur + idx) * l2e()) + (tl.sf[ok] - tl.sf[o]));
+                        ((M + __ldg(dur + idx) * l2e()) + ((tl.sf[ok] - tl.sf[o]) + tl.pd[o]));
         seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] =
             tl.tf[r * 2 * C + C + c] * tl.ab[ok] * (tl.fs[r] * ex2(z));
       }
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
       float a_ = 0.f;
       for (int r = 0; r < r_end; ++r) {
         const int o = r * C + c, ok = (r + k) * C + c;
-        const float z = (float)(tl.ii[ok] - tl.ii[o]) + (dk + (tl.sf[ok] - tl.sf[o]));
+        const float z = (float)(tl.ii[ok] - tl.ii[o]) + (dk + ((tl.sf[ok] - tl.sf[o]) + tl.pd[o]));
         a_ = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a_);
       }
       return a_;
@@ -389,7 +396,7 @@ size_t posterior_smem_bytes(const Dims& d) { return ptile_bytes(d.pRT, d.K, d.C)
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,
                              float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
-                             float* seg_marg) {
+                             float* seg_marg, int pj) {
   const size_t sm = posterior_smem_bytes(d);
   const bool small = (size_t)d.K * d.C <= 4u * 512u && (size_t)d.C * d.C <= 4u * 512u;
   const void* fn = small ? (const void*)posterior_kernel<4, 4> : (const void*)posterior_kernel<16, 32>;
@@ -400,11 +407,11 @@ cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* len
   if (small)
     posterior_kernel<4, 4><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
                                                               grad_em, start_marg, end_marg,
-                                                              seg_marg);
+                                                              seg_marg, pj);
   else
     posterior_kernel<16, 32><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
                                                                 grad_em, start_marg, end_marg,
-                                                                seg_marg);
+                                                                seg_marg, pj);
   return cudaGetLastError();
 }
 

@@ -158,8 +158,11 @@ __global__ void __launch_bounds__(256) prefix_scan_kernel(const float* __restric
         const size_t o = ((size_t)b * d.Tstride) * C + c;
         ws.sint[o] = 0;
         ws.sfrac[o] = 0.f;
-        if (p_start || p_end)
-          ws.pd[o] = (p_start && L > 0) ? (float)((double)__ldg(p_start + (size_t)b * T * C + c) * LOG2E_D) : 0.f;
+        if (p_start || p_end) {
+          const double ps0 = (p_start && L > 0) ? (double)__ldg(p_start + (size_t)b * T * C + c) : 0.0;
+          ws.pd[o] = (float)(ps0 * LOG2E_D);
+          emx = fmaxf(emx, (float)fabs(ps0));
+        }
       }
     }
   }

@@ -62,7 +62,7 @@ struct VSmem {
   uint64_t* vbar;  // [2]   cluster: arrival of the step's V row, by step parity
 };
 
-__device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
+__device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d, bool pj) {
   VSmem x;
   const int C = d.C, Cr = d.xCr;
   unsigned char* p = raw;
@@ -77,6 +77,11 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
   p += 2ull * TS * C * sizeof(int32_t);
   x.s.tfrac = reinterpret_cast<float*>(p);
   p += 2ull * TS * C * sizeof(float);
+  x.s.tpd = nullptr;
+  if (pj) {  // boundary projections: start terms stream with the prefix sums
+    x.s.tpd = reinterpret_cast<float*>(p);
+    p += 2ull * TS * C * sizeof(float);
+  }
   x.s.ring = reinterpret_cast<float2*>(p);
   p += (size_t)d.xRLP * Cr * sizeof(float2);
   p = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
@@ -101,8 +106,8 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d) {
 }
 
 // Dynamic shared memory of the kernel (carve order of vcarve).
-__host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d) {
-  return 96 + 2ull * TS * d.C * 8 + (size_t)d.xRLP * d.xCr * 8 + 16 +
+__host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d, bool pj) {
+  return 96 + 2ull * TS * d.C * (pj ? 12 : 8) + (size_t)d.xRLP * d.xCr * 8 + 16 +
          (2ull * d.xPC + 9ull * d.xCr) * 4;
 }
 
@@ -135,9 +140,9 @@ __global__ void __launch_bounds__(LB, 1)
     viterbi_pipe_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                         const float* __restrict__ trans, const float* __restrict__ dur,
                         double* __restrict__ score, int32_t* __restrict__ labels,
-                        uint8_t* __restrict__ seg_start) {
+                        uint8_t* __restrict__ seg_start, int pj) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const VSmem vs = vcarve(smem_raw, d);
+  const VSmem vs = vcarve(smem_raw, d, pj != 0);
   const Smem& sm = vs.s;
   const int C = d.C, K = d.K, T = d.T, Cr = d.xCr, tid = threadIdx.x;
   const int rank = N > 1 ? (int)cluster_ctarank() : 0;
@@ -247,21 +252,31 @@ __global__ void __launch_bounds__(LB, 1)
     if constexpr (N == 1) return;
     dead = true;
   }
-  // boundary 0: G = 0 at S = 0, base 0; helpers set step 1's k = 1 constant
+  // boundary 0: G = 0 at S = 0, base 0 (with boundary projections: the
+  // start term of boundary 0); helpers set step 1's k = 1 constant
   for (int x = tid; x < Cr; x += blockDim.x) {
     float2* r = sm.ring + (size_t)x * RLP;
-    for (int y = 0; y < RL; y += K) r[y] = make_float2(0.f, 0.f);
+    const float v0 = (sm.tpd && c0 + x < C) ? sm.tpd[c0 + x] : 0.f;
+    for (int y = 0; y < RL; y += K) r[y] = make_float2(v0, 0.f);
     vs.Sb[x] = 0;
   }
-  // helper state: rows i (cur) and i-1 (prev) of S, frame Phi_{i-1} - F0
+  // helper state: rows i (cur) and i-1 (prev) of S, frame Phi_{i-1} - F0;
+  // with boundary projections the start terms pd of those rows (the k = 1
+  // and k = 2 factors' start boundaries)
   int hs_c = 0, hs_p = 0;
-  float hf_c = 0.f, hf_p = 0.f, Fph = 0.f;
+  float hf_c = 0.f, hf_p = 0.f, Fph = 0.f, hd_c = 0.f, hd_p = 0.f;
   const int32_t* hrow_i = sm.tint;  // row i+1 of the current step (set below)
   const float* hrow_f = sm.tfrac;
+  const float* hrow_d = nullptr;
   if (!comb) {
     hs_c = sm.tint[C + cc];  // row 1
     hf_c = sm.tfrac[C + cc];
-    if (leader) vs.A1[1 * Cr + cl] = d1 + ((float)hs_c + hf_c);  // S[1] - S[0]
+    if (sm.tpd) {
+      hd_p = sm.tpd[cc];      // row 0
+      hd_c = sm.tpd[C + cc];  // row 1
+      hrow_d = sm.tpd + 2 * C;
+    }
+    if (leader) vs.A1[1 * Cr + cl] = (d1 + hd_p) + ((float)hs_c + hf_c);  // S[1] - S[0]
     hrow_i = sm.tint + 2 * C;  // row 2 for step 1
     hrow_f = sm.tfrac + 2 * C;
   }
@@ -272,9 +287,10 @@ __global__ void __launch_bounds__(LB, 1)
   // combine state: S at row i - 1, ring slot of boundary i - 1
   float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
   int si_p = 0;
-  float sf_p = 0.f;
+  float sf_p = 0.f, pd_p = sm.tpd ? sm.tpd[cc] : 0.f;  // row i - 1 (pd: start term)
   const int32_t* crow_i = sm.tint + C;  // row i of the current step
   const float* crow_f = sm.tfrac + C;
+  const float* crow_d = sm.tpd ? sm.tpd + C : nullptr;
   int wslot = 0;
   double F0 = 0.0;
   // every CTA of a cluster has initialised its V buffer and arrival barriers
@@ -309,12 +325,14 @@ __global__ void __launch_bounds__(LB, 1)
         const size_t o = tile_row_off(i + 1, C);
         hrow_i = sm.tint + o;
         hrow_f = sm.tfrac + o;
+        if (sm.tpd) hrow_d = sm.tpd + o;
       }
       if (i % TS == 0) {
         if (!dead) tile_issue(sm, d, ws, b, ts, i / TS + 1);
         const size_t o = tile_row_off(i, C);
         crow_i = sm.tint + o;
         crow_f = sm.tfrac + o;
+        if (sm.tpd) crow_d = sm.tpd + o;
       }
       if (i == next_rb) {
         // rebase the integer frames to (F0 + Phi_{i-1}, S_int[i-1])
@@ -360,6 +378,7 @@ __global__ void __launch_bounds__(LB, 1)
       const int okd = vs.Ok[(i & 1) * Cr + ccl];
       const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
       const int si_n = rok ? crow_i[cc] : 0;  // row i: the next step's ring entry
+      const float pd_n = (crow_d && rok) ? crow_d[cc] : 0.f;
       const float sf_n = rok ? crow_f[cc] : 0.f;
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(LB, 1)
         kdw[(size_t)i * C + c] = kdec;
       }
       if (leader && i >= 2 && SEMICRF_INB(ws.status, wslot >= 0 && wslot < K, SITE_RING_SLOT)) {
-        const float2 e = make_float2(gv - sf_p, Fp - (float)(si_p - Sbc));
+        const float2 e = make_float2((gv - sf_p) + pd_p, Fp - (float)(si_p - Sbc));
         for (int x = wslot; x < RL; x += K) rl[x] = e;
       }
       wslot = (wslot + 1 == K) ? 0 : wslot + 1;
@@ -411,6 +430,8 @@ __global__ void __launch_bounds__(LB, 1)
       Fp += n;
       si_p = si_n;
       sf_p = sf_n;
+      pd_p = pd_n;
+      if (crow_d) crow_d += C;
       crow_i += C;
       crow_f += C;
     } else {
@@ -465,14 +486,19 @@ __global__ void __launch_bounds__(LB, 1)
         const int o2 = ((i + 1) & 1) * Cr + cl;
         vs.Om[o2] = best + fn;
         vs.Ok[o2] = kb;
-        vs.A1[o2] = d1 + ((float)(sn - hs_c) + (fn - hf_c));
-        vs.A2[o2] = d2 + ((float)(sn - hs_p) + (fn - hf_p));
+        vs.A1[o2] = (d1 + hd_c) + ((float)(sn - hs_c) + (fn - hf_c));
+        vs.A2[o2] = (d2 + hd_p) + ((float)(sn - hs_p) + (fn - hf_p));
       }
       if (i < L) {
         hs_p = hs_c;
         hf_p = hf_c;
         hs_c = sn;
         hf_c = fn;
+        hd_p = hd_c;
+        if (hrow_d) {
+          hd_c = hok ? hrow_d[cc] : 0.f;
+          hrow_d += C;
+        }
         hrow_i += C;
         hrow_f += C;
         hbase = (hbase + 1 == K) ? 0 : hbase + 1;
@@ -706,7 +732,7 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-size_t viterbi_pipe_smem_bytes(const Dims& d) { return vsmem_bytes(d); }
+size_t viterbi_pipe_smem_bytes(const Dims& d, bool pj) { return vsmem_bytes(d, pj); }
 
 #define SEMICRF_VW_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
 
@@ -759,12 +785,12 @@ namespace semicrf {
 
 cudaError_t launch_viterbi_pipe(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 const float* trans, const float* dur, double* score,
-                                int32_t* labels, uint8_t* seg_start, cudaStream_t st) {
-  const size_t sm = viterbi_pipe_smem_bytes(d);
+                                int32_t* labels, uint8_t* seg_start, cudaStream_t st, int pj) {
+  const size_t sm = viterbi_pipe_smem_bytes(d, pj != 0);
 #define SEMICRF_LAUNCH_VPIPE(n, g, cat, h, kbh, lb)                                            \
   if (d.xN == n && d.xG == g && d.xCAT == cat && d.xH == h && d.xKBH == kbh && d.xLB == lb)    \
     return launch_clustered(viterbi_pipe_kernel<n, g, cat, h, kbh, lb>, n, d.B * n, d.xNT, sm,  \
-                            st, d, ws, lengths, trans, dur, score, labels, seg_start);
+                            st, d, ws, lengths, trans, dur, score, labels, seg_start, pj);
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_LAUNCH_VPIPE)
 #undef SEMICRF_LAUNCH_VPIPE
   return cudaErrorInvalidConfiguration;

@@ -2,7 +2,10 @@
 against the float64 oracle: log Z, marginals and every gradient (the
 projection gradients included), decoding, the path score and its counts,
 and that a plain call after a projection call on the same workspace is a
-plain call again.  Tolerances as in gpu_common."""
+plain call again.  Every forward-backward case runs twice: on the default
+path (exponential-domain rings, the kept-row posterior pass and the
+pipelined decoder, which carry the projection terms) and with the rings
+forced into the log domain.  Tolerances as in gpu_common."""
 
 import numpy as np
 import pytest
@@ -42,8 +45,9 @@ def _masked(x, lengths):
     return x
 
 
+@pytest.mark.parametrize("log_domain", [False, True])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_forward_backward_with_projections_match_oracle(name):
+def test_forward_backward_with_projections_match_oracle(name, log_domain):
     from semi_markov_crf_b200 import semicrf
     case = CASES[name]()
     B, T, C = case["em"].shape
@@ -52,10 +56,15 @@ def test_forward_backward_with_projections_match_oracle(name):
     g = np.linspace(0.5, 1.5, B)
     em, lengths, trans, dur = to_dev(case)
     tp, te = torch.from_numpy(ps).cuda(), torch.from_numpy(pe).cuda()
-    logZ, ws = semicrf.forward(em, lengths, trans, dur, p_start=tp, p_end=te)
+    logZ, ws = semicrf.forward(em, lengths, trans, dur, p_start=tp, p_end=te,
+                               log_domain=log_domain)
     out = semicrf.backward(ws, lengths, trans, dur, marginals=True,
                            grad_logZ=torch.as_tensor(g, device="cuda"))
     assert semicrf.get_status(ws) == 0
+    dom = semicrf.ring_domains(ws)
+    nonempty = [b for b in range(B) if case["lengths"][b] > 0]
+    want = 2 if log_domain else 1
+    assert all(dom[b] == want and dom[B + b] == want for b in nonempty), dom
     got = {k: v.cpu().numpy() for k, v in out.items()}
     got["logZ"] = logZ.cpu().numpy()
     ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"], K,
@@ -68,7 +77,8 @@ def test_forward_backward_with_projections_match_oracle(name):
     assert max_abs(got["grad_p_start"], eps) <= MARG_ATOL
     assert max_abs(got["grad_p_end"], epe) <= MARG_ATOL
     # the same without the caller's marginal buffers
-    logZ2, ws2 = semicrf.forward(em, lengths, trans, dur, p_start=tp, p_end=te)
+    logZ2, ws2 = semicrf.forward(em, lengths, trans, dur, p_start=tp, p_end=te,
+                                 log_domain=log_domain)
     out2 = semicrf.backward(ws2, lengths, trans, dur, grad_logZ=torch.as_tensor(g, device="cuda"))
     assert torch.equal(out2["grad_p_start"], out["grad_p_start"])
     assert torch.equal(out2["grad_p_end"], out["grad_p_end"])
@@ -116,19 +126,48 @@ def test_viterbi_and_path_score_with_projections_match_oracle(name):
         assert np.max(d / np.maximum(1.0, np.abs(r))) <= COUNT_RTOL, key
 
 
-def test_zero_projections_equal_the_plain_log_domain_run():
+@pytest.mark.parametrize("log_domain", [False, True])
+def test_zero_projections_equal_the_plain_run(log_domain):
     from semi_markov_crf_b200 import semicrf
     case = CASES["speech_small"]()
     B, T, C = case["em"].shape
     em, lengths, trans, dur = to_dev(case)
     z = torch.zeros((B, T, C), dtype=torch.float32, device="cuda")
-    lz_p, ws_p = semicrf.forward(em, lengths, trans, dur, p_start=z, p_end=z)
+    lz_p, ws_p = semicrf.forward(em, lengths, trans, dur, p_start=z, p_end=z, log_domain=log_domain)
     out_p = semicrf.backward(ws_p, lengths, trans, dur, marginals=True)
-    lz, ws = semicrf.forward(em, lengths, trans, dur, log_domain=True)
+    lz, ws = semicrf.forward(em, lengths, trans, dur, log_domain=log_domain)
     out = semicrf.backward(ws, lengths, trans, dur, marginals=True)
     assert torch.equal(lz_p, lz)
     for k in ("grad_em", "grad_trans", "grad_dur", "pos_marg", "start_marg", "end_marg"):
         assert torch.equal(out_p[k], out[k]), k
+    # decoding: zero projections change nothing either
+    a = semicrf.viterbi(em, lengths, trans, dur, p_start=z, p_end=z)
+    b = semicrf.viterbi(em, lengths, trans, dur)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_loud_projections_leave_the_exponential_domain():
+    """Projections of several hundred nats per position exceed the
+    exponential-domain kernels' exponent head-room: those sequences run in
+    the log domain and still match the oracle."""
+    from semi_markov_crf_b200 import semicrf
+    case = synth.make("speech", B=3, T=60, seed=23)
+    B, T, C = case["em"].shape
+    K = case["dur"].shape[0]
+    ps, pe = _proj(case, 56, scale=30.0)
+    em, lengths, trans, dur = to_dev(case)
+    tp, te = torch.from_numpy(ps).cuda(), torch.from_numpy(pe).cuda()
+    logZ, ws = semicrf.forward(em, lengths, trans, dur, p_start=tp, p_end=te)
+    out = semicrf.backward(ws, lengths, trans, dur, marginals=True)
+    assert semicrf.get_status(ws) == 0
+    assert all(v == 2 for v in semicrf.ring_domains(ws))
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    got["logZ"] = logZ.cpu().numpy()
+    ref = oracle.forward_backward(case["em"], case["lengths"], case["trans"], case["dur"], K,
+                                  p_start=ps, p_end=pe)
+    err = np.abs(got["logZ"] - ref["logZ"]) / np.maximum(1.0, np.abs(ref["logZ"]))
+    assert np.all(err <= 1e-5), err
 
 
 def test_plain_call_after_a_projection_call_clears_the_switch():

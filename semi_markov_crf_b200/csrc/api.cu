@@ -147,6 +147,7 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (B < 0 || T < 0 || C < 1 || K < 1) return SEMICRF_ERR_INVALID_ARG;
   if (C > C_MAX || K > K_MAX || (long long)K * C > KC_MAX || T > (1 << 26) || B > (1 << 20))
     return SEMICRF_ERR_UNSUPPORTED;
+  d = Dims{};
   d.B = B;
   d.T = T;
   d.C = C;

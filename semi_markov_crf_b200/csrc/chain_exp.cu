@@ -195,7 +195,10 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   if (comb) {
 #pragma unroll
     for (int q = 0; q < NR; ++q) {
-      const int x = jl * CAT + q;
+      // interleaved 16-byte chunks: chunk q/4 of lane jl is label block
+      // (q/4) * G + jl, so a group's lanes read consecutive chunks (no shared
+      // memory bank conflicts on the critical path's vector loads)
+      const int x = 4 * ((q >> 2) * G + jl) + (q & 3);
       w[q] = (q < CAT && act && x < C)
                  ? ex2(__ldg(trans + (UP ? (size_t)x * C + cc : (size_t)cc * C + x)) * l2e() - M)
                  : 0.f;
@@ -412,11 +415,11 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const int si_n = rok ? crow_i[cc] : 0;  // the walk's row r: the next step's ring entry
       const float sf_n = rok ? crow_f[cc] : 0.f;
       const float pd_n = (UP && crow_d && rok) ? crow_d[cc] : 0.f;
-      const float* pv = xs.P + ((i - 1) & 1) * d.xPC + jl * CAT;
+      const float* pv = xs.P + ((i - 1) & 1) * d.xPC + 4 * jl;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
 #pragma unroll
       for (int q = 0; q < CAT; q += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(pv + q);
+        const float4 v = *reinterpret_cast<const float4*>(pv + q * G);
         a0 = fmaf(v.x, w[q], a0);
         a1 = fmaf(v.y, w[q + 1], a1);
         a2 = fmaf(v.z, w[q + 2], a2);

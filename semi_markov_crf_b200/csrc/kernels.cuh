@@ -121,7 +121,8 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(1, 4, 12, 4, 8, 384) X(1, 4, 12, 4, 16, 384) X(1, 2, 48, 2, 32, 384) X(1, 2, 64, 2, 32, 512)  \
   X(1, 4, 24, 2, 32, 576) X(1, 4, 32, 4, 8, 1024) X(1, 4, 32, 2, 32, 768) X(1, 1, 8, 32, 64, 224) \
   X(1, 1, 8, 32, 64, 288) \
-  X(2, 2, 24, 4, 8, 160) X(2, 4, 32, 4, 16, 512) X(4, 4, 32, 4, 16, 256) X(8, 4, 32, 4, 16, 128)
+  X(2, 2, 24, 4, 8, 160) X(2, 4, 32, 4, 16, 512) X(4, 4, 32, 4, 16, 256) X(8, 4, 32, 4, 16, 128) \
+  X(4, 8, 16, 4, 16, 384) X(4, 4, 32, 8, 8, 384) X(8, 8, 16, 8, 8, 256) X(8, 4, 32, 8, 8, 192)
 
 // Launches `kern` on `grid` CTAs of `threads` threads grouped in clusters of
 // n_cluster CTAs (grid a multiple of n_cluster; n_cluster = 1: a plain

@@ -194,7 +194,10 @@ __global__ void __launch_bounds__(LB, 1)
   if (comb) {
 #pragma unroll
     for (int q = 0; q < NR; ++q) {
-      const int x = jl * CAT + q;
+      // interleaved 16-byte chunks: chunk q/4 of lane jl is label block
+      // (q/4) * G + jl, so a group's lanes read consecutive chunks (no shared
+      // memory bank conflicts on the critical path's vector loads)
+      const int x = 4 * ((q >> 2) * G + jl) + (q & 3);
       w[q] = (q < CAT && act && x < C) ? __ldg(trans + (size_t)x * C + cc) * l2e() : NEG_INF;
     }
   } else {
@@ -380,11 +383,11 @@ __global__ void __launch_bounds__(LB, 1)
       const int si_n = rok ? crow_i[cc] : 0;  // row i: the next step's ring entry
       const float pd_n = (crow_d && rok) ? crow_d[cc] : 0.f;
       const float sf_n = rok ? crow_f[cc] : 0.f;
-      const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl * CAT;
+      const float* pv = vs.V + ((i - 1) & 1) * d.xPC + 4 * jl;
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
 #pragma unroll
       for (int q = 0; q < CAT; q += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(pv + q);
+        const float4 v = *reinterpret_cast<const float4*>(pv + q * G);
         b0 = fmaxf(b0, v.x + w[q]);
         b1 = fmaxf(b1, v.y + w[q + 1]);
         b2 = fmaxf(b2, v.z + w[q + 2]);

@@ -82,6 +82,18 @@ int max_smem_optin() {
 // SEMICRF_XSHAPE=i forces the i-th fitting shape of the menu and
 // SEMICRF_XCLUSTER=n restricts the choice to clusters of n CTAs (tuning).
 constexpr int CLUSTER_MIN_C = 96;
+constexpr int LONG_K = 2050;  // above: helper lanes of a label span several warps
+// Fills the derived fields of a pipelined shape (ring rows, label-vector
+// length, bank padding).
+void xshape_derive(Dims& d) {
+  d.xRL = d.K + d.xKBH;
+  // label vector row: the combine lanes' blocks (xG x xCAT) and the helper
+  // lanes' strided sources (xH x ceil(xG xCAT / xH)), whichever is longer
+  d.xPC = std::max(d.xG * d.xCAT, d.xH * ((d.xG * d.xCAT + d.xH - 1) / d.xH));
+  d.xRLP = d.K + d.xH * d.xKBH;
+  if (d.xH < 16) d.xRLP += (((d.xH - d.xRLP) % 16) + 16) % 16;
+}
+
 void choose_xshape(Dims& d, size_t budget) {
   const int C = d.C, K = d.K;
   int forced = -1, forced_n = 0;
@@ -99,43 +111,47 @@ void choose_xshape(Dims& d, size_t budget) {
     return l;
   };
   const int want_n = forced_n > 0 ? forced_n : 0;
+  // wide label sets, and long durations (a label's ring and window then fill
+  // one SM's shared memory: one label per CTA)
+  const bool needs_cluster = C >= CLUSTER_MIN_C || (K > LONG_K && C > 1);
+  Dims pick = d;
 #define SEMICRF_XCONSIDER(n, g, cat, h, kbh, lb)                                          \
   {                                                                                       \
     const int cr = (C + n - 1) / n;                                                       \
-    const int nwc = (cr + 32 / g - 1) / (32 / g), nwh = (cr + 32 / h - 1) / (32 / h);     \
+    const int nwc = (cr + 32 / g - 1) / (32 / g);                                         \
+    const int nwh = h > 32 ? cr * (h / 32) : (cr + 32 / h - 1) / (32 / h);                \
     const int nt = 32 * (nwc + nwh);                                                      \
-    const bool cl_ok = want_n ? (n == want_n) : ((n > 1) == (C >= CLUSTER_MIN_C));        \
+    const bool cl_ok = want_n ? (n == want_n) : ((n > 1) == needs_cluster);              \
     if (C <= g * cat && K <= h * kbh + 2 && nt <= lb && cl_ok && (n == 1 || cr * n - C < cr)) { \
-      const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +        \
-                          10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0) +      \
-                          (n > 1 ? 100.0 + 25.0 * std::abs(n - 4) : 0.0);                 \
-      if ((forced < 0 && cost < best) || forced == idx) {                                 \
-        best = cost;                                                                      \
-        d.xN = n;                                                                         \
-        d.xCr = cr;                                                                       \
-        d.xG = g;                                                                         \
-        d.xCAT = cat;                                                                     \
-        d.xH = h;                                                                         \
-        d.xKBH = kbh;                                                                     \
-        d.xLB = lb;                                                                       \
-        d.xNT = nt;                                                                       \
+      Dims t = d;                                                                         \
+      t.xN = n;                                                                           \
+      t.xCr = cr;                                                                         \
+      t.xG = g;                                                                           \
+      t.xCAT = cat;                                                                       \
+      t.xH = h;                                                                           \
+      t.xKBH = kbh;                                                                       \
+      t.xLB = lb;                                                                         \
+      t.xNT = nt;                                                                         \
+      xshape_derive(t);                                                                   \
+      if (chain_exp_smem_bytes(t) <= budget && viterbi_pipe_smem_bytes(t) <= budget) {   \
+        const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +      \
+                            10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0) +    \
+                            (n > 1 ? 100.0 + 25.0 * std::abs(n - 4) : 0.0);               \
+        if ((forced < 0 && cost < best) || forced == idx) {                               \
+          best = cost;                                                                    \
+          pick = t;                                                                       \
+        }                                                                                 \
+        ++idx;                                                                            \
       }                                                                                   \
-      ++idx;                                                                              \
     }                                                                                     \
   }
   SEMICRF_FOR_EACH_XSHAPE(SEMICRF_XCONSIDER)
 #undef SEMICRF_XCONSIDER
-  if (d.xG == 0) return;
-  d.xRL = K + d.xKBH;
-  // label vector row: the combine lanes' blocks (xG x xCAT) and the helper
-  // lanes' strided sources (xH x ceil(xG xCAT / xH)), whichever is longer
-  d.xPC = std::max(d.xG * d.xCAT, d.xH * ((d.xG * d.xCAT + d.xH - 1) / d.xH));
-  d.xRLP = K + d.xH * d.xKBH;
-  if (d.xH < 16) d.xRLP += (((d.xH - d.xRLP) % 16) + 16) % 16;
-  // the posterior pass from the kept values must fit too
+  if (pick.xG == 0) return;
+  d = pick;
+  // the posterior pass from the kept values and the cut normaliser must fit too
   d.pRT = posterior_tile_rows(d, budget);
-  if (chain_exp_smem_bytes(d) > budget || viterbi_pipe_smem_bytes(d) > budget || d.pRT == 0 ||
-      cut_grid_smem_bytes(d) > budget || d.C > 128) {
+  if (d.pRT == 0 || cut_grid_smem_bytes(d) > budget || d.C > 128) {
     d.xG = 0;
     d.xN = 1;
     d.xCr = C;
@@ -167,7 +183,12 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
+  // Cut-normaliser grid: every 128 positions, sparser for long durations (a
+  // grid point costs K(K+1)/2 C terms; the two rings' rounding drifts by about
+  // 1e-7 per position, so linear interpolation over 2048 positions still
+  // keeps the marginals' error far below 1e-4)
   d.GS = 128;
+  while (d.GS < 2048 && d.GS * 4 < K) d.GS *= 2;
   d.ngrid = T > 0 ? (T - 1) / d.GS + 2 : 1;  // positions 0, GS, 2GS, ... and L - 1
   d.npch = std::max(1, (T + PATH_ROWS - 1) / PATH_ROWS);
   // Kernel shape: G lanes per label (a power of two), each with KBT durations
@@ -205,18 +226,26 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
     SEMICRF_FOR_EACH_SHAPE(SEMICRF_CONSIDER)
 #undef SEMICRF_CONSIDER
   }
-  if (d.KBT == 0) return SEMICRF_ERR_UNSUPPORTED;
-  d.GA = d.GB;
-  d.RL = K + d.KBT;
-  d.PC = ((std::max(C, d.GB * d.CAT) + 3) / 4) * 4;
   d.prefR = std::max(16, pow2floor(8192 / C));
   d.nchunk = T > 0 ? (T + d.prefR - 1) / d.prefR : 1;
   d.store_w = 2 * C + 2;
   // the per-block limit covers static shared memory too (a few bytes here)
   const size_t budget = (size_t)max_smem_optin() - 256;
-  d.store_smem = recursion_smem_bytes(d, true) <= budget ? 1 : 0;
-  if (recursion_smem_bytes(d, false) > budget) return SEMICRF_ERR_UNSUPPORTED;
+  if (d.KBT) {
+    d.GA = d.GB;
+    d.RL = K + d.KBT;
+    d.PC = ((std::max(C, d.GB * d.CAT) + 3) / 4) * 4;
+    d.store_smem = recursion_smem_bytes(d, true) <= budget ? 1 : 0;
+    if (recursion_smem_bytes(d, false) > budget) d.KBT = 0;
+  }
+  if (!d.KBT) {  // no log-domain kernels for these sizes (long durations)
+    d.KBT = d.GB = d.CAT = d.GA = d.RL = d.NT = d.LB = 0;
+    d.PC = ((C + 3) / 4) * 4;
+    d.store_smem = 1;  // nothing to store
+  }
   choose_xshape(d, budget);
+  // a size needs the pipelined kernels or the log-domain ones
+  if (!d.KBT && !d.xG) return SEMICRF_ERR_UNSUPPORTED;
   return SEMICRF_OK;
 }
 

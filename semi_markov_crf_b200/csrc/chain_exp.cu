@@ -61,7 +61,8 @@ constexpr float FAST_BOUND = 60.f;  // log2 units; two steps stay inside fp32's 
 struct XSmem {
   Smem s;      // mbar, tint, tfrac (every label), ring (own labels)
   float* P;    // [2][xPC] exp-domain label vector, by step parity (all labels)
-  float* Oh;   // [2][Cr]  k >= 3 sums for the step of that parity (frame Phi_{t-2})
+  float* Oh;   // [HW][2][Cr] k >= 3 sums for the step of that parity (frame Phi_{t-2}),
+               // one partial per helper warp of a label (HW = ceil(xH / 32))
   float* A1;   // [2][Cr]  k = 1 factors
   float* A2;   // [2][Cr]  k = 2 factors
   float* nsl;  // [2]      frame step n published by the combine warps
@@ -97,7 +98,7 @@ __device__ __forceinline__ XSmem xcarve(unsigned char* raw, const Dims& d, bool 
   x.P = f;
   f += 2 * d.xPC;
   x.Oh = f;
-  f += 2 * Cr;
+  f += 2 * Cr * ((d.xH + 31) / 32);
   x.A1 = f;
   f += 2 * Cr;
   x.A2 = f;
@@ -159,7 +160,12 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
                                       double* __restrict__ logZ_out, int rank) {
   const Smem& sm = xs.s;
   const int C = d.C, K = d.K, Cr = d.xCr, tid = threadIdx.x;
-  constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
+  // Long durations: H > 32 lanes per label spread over HW = H / 32 helper
+  // warps; each warp sums its share of the window (its own predicted shift)
+  // and publishes a partial k >= 3 sum, which the combine adds up.
+  constexpr int HG = H > 32 ? 32 : H;       // lanes per reduction group
+  constexpr int HW = H > 32 ? H / 32 : 1;   // helper warps per label
+  constexpr int LPWC = 32 / G, LPWH = 32 / HG, WL = H * KBH;
   constexpr int NR = CAT > KBH ? CAT : KBH;
   constexpr int SG = UP ? 1 : -1;  // walk direction over rows
   const float sg = UP ? 1.f : -1.f;
@@ -167,12 +173,15 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   const int nwc = (Cr + LPWC - 1) / LPWC;
   const bool comb = warp < nwc;
   const int c0 = rank * Cr;  // first label of this CTA
-  const int cl = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;  // local label
+  const int hwi = warp - nwc;  // helper warp index
+  const int cl = comb ? warp * LPWC + lane / G
+                      : (HW > 1 ? hwi / HW : hwi * LPWH + lane / H);  // local label
+  const int hwarp = HW > 1 && !comb ? hwi % HW : 0;  // this lane's warp among its label's
   const int c = c0 + cl;     // global label
   const bool act = cl < Cr && c < C;
   const int cc = act ? c : 0;     // global label (tile rows, parameters, outputs)
   const int ccl = act ? cl : 0;   // local label (ring, per-label arrays)
-  const int jl = comb ? lane % G : lane % H;
+  const int jl = comb ? lane % G : (HW > 1 ? hwarp * 32 + lane : lane % H);
   const bool leader = act && jl == 0;
   const int RL = K + WL, RLP = d.xRLP;
   float2* const rl = sm.ring + (size_t)ccl * RLP;
@@ -216,8 +225,8 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   // ---------------------------------------------------------------- shared state
   for (int i = tid; i < RLP * Cr; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) xs.P[i] = 0.f;
+  for (int i = tid; i < 2 * Cr * HW; i += blockDim.x) xs.Oh[i] = 0.f;
   for (int i = tid; i < 2 * Cr; i += blockDim.x) {
-    xs.Oh[i] = 0.f;
     xs.A1[i] = 0.f;
     xs.A2[i] = 0.f;
   }
@@ -410,7 +419,10 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
         }
       }
       const int po = (i & 1) * Cr + ccl;
-      const float a1v = xs.A1[po], a2v = xs.A2[po], ohv = xs.Oh[po];
+      const float a1v = xs.A1[po], a2v = xs.A2[po];
+      float ohv = xs.Oh[po];
+#pragma unroll
+      for (int hw = 1; hw < HW; ++hw) ohv += xs.Oh[hw * 2 * Cr + po];  // long durations
       const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
       const int si_n = rok ? crow_i[cc] : 0;  // the walk's row r: the next step's ring entry
       const float sf_n = rok ? crow_f[cc] : 0.f;
@@ -495,8 +507,11 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const float aA2 = ((M + d2) + (UP ? hd_p : dn)) + sg * ((float)(sn - hs_p) + (fn - hf_p));
       const int o2 = ((i + 1) & 1) * Cr + ccl;
       if constexpr (H >= 3) {
-        const float e = ex2(jl == 0 ? aO : (jl == 1 ? aA1 : aA2));
-        if (act && jl == 0) xs.Oh[o2] = (s > 0.f) ? s * e : 0.f;
+        // (several helper warps per label: each warp's lane 0 its partial
+        // k >= 3 sum, the label's first warp the k = 1, 2 factors)
+        const int ln = jl % HG;
+        const float e = ex2(ln == 0 ? aO : (jl == 1 ? aA1 : aA2));
+        if (act && ln == 0) xs.Oh[hwarp * 2 * Cr + o2] = (s > 0.f) ? s * e : 0.f;
         if (act && jl == 1) xs.A1[o2] = e;
         if (act && jl == 2) xs.A2[o2] = e;
       } else {
@@ -551,8 +566,9 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
 }  // namespace
 
 size_t chain_exp_smem_bytes(const Dims& d, bool pj) {
+  const size_t hw = (d.xH + 31) / 32;  // helper warps per label (long durations: > 1)
   return 96 + 2ull * TS * d.C * (pj ? 12 : 8) + (size_t)d.xRLP * d.xCr * 8 + 16 +
-         (2ull * d.xPC + 7ull * d.xCr) * 4;
+         (2ull * d.xPC + (5ull + 2 * hw) * d.xCr) * 4;
 }
 
 }  // namespace semicrf

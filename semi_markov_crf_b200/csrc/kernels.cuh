@@ -111,7 +111,10 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
 // helper lane KBH, launch bound LB).  Each CTA owns Cr = ceil(C / N) labels;
 // a shape serves C <= G*CAT and K <= H*KBH + 2 with
 // 32*(ceil(Cr*G/32) + ceil(Cr*H/32)) <= LB threads (labels never straddle a
-// warp).  N > 1 runs each ring on a thread-block cluster of N CTAs.
+// warp).  N > 1 runs each ring on a thread-block cluster of N CTAs.  H = 128
+// (long durations, K up to 8194): a label's helper lanes span four warps,
+// one label per CTA (its ring of K + 8192 entries fills the CTA's shared
+// memory).
 #define SEMICRF_FOR_EACH_XSHAPE(X)                                                     \
   X(1, 1, 8, 1, 8, 64) X(1, 1, 8, 4, 8, 64) X(1, 1, 8, 8, 16, 96) X(1, 1, 8, 16, 16, 160)          \
   X(1, 1, 8, 32, 16, 288) X(1, 1, 16, 1, 8, 64) X(1, 1, 16, 4, 8, 96) X(1, 1, 16, 8, 16, 160)      \
@@ -122,7 +125,10 @@ cudaError_t launch_viterbi(const Dims& d, const WsPtrs& ws, const int32_t* lengt
   X(1, 4, 24, 2, 32, 576) X(1, 4, 32, 4, 8, 1024) X(1, 4, 32, 2, 32, 768) X(1, 1, 8, 32, 64, 224) \
   X(1, 1, 8, 32, 64, 288) \
   X(2, 2, 24, 4, 8, 160) X(2, 4, 32, 4, 16, 512) X(4, 4, 32, 4, 16, 256) X(8, 4, 32, 4, 16, 128) \
-  X(4, 8, 16, 4, 16, 384) X(4, 4, 32, 8, 8, 384) X(8, 8, 16, 8, 8, 256) X(8, 4, 32, 8, 8, 192)
+  X(4, 8, 16, 4, 16, 384) X(4, 4, 32, 8, 8, 384) X(8, 8, 16, 8, 8, 256) X(8, 4, 32, 8, 8, 192) \
+  X(1, 1, 8, 128, 64, 160) X(2, 1, 8, 128, 64, 160) X(3, 1, 8, 128, 64, 160)                 \
+  X(4, 1, 8, 128, 64, 160) X(5, 1, 8, 128, 64, 160) X(6, 1, 8, 128, 64, 160)                 \
+  X(7, 1, 8, 128, 64, 160) X(8, 1, 8, 128, 64, 160)
 
 // Launches `kern` on `grid` CTAs of `threads` threads grouped in clusters of
 // n_cluster CTAs (grid a multiple of n_cluster; n_cluster = 1: a plain

@@ -9,8 +9,10 @@
 namespace semicrf {
 
 constexpr int C_MAX = 128;
-constexpr int K_MAX = 2048;
-constexpr int KC_MAX = 16384;
+constexpr int K_MAX = 8192;      // long durations (K > LOG_K_MAX) need C <= 8 ...
+constexpr int KC_MAX = 65536;    // ... and run on the pipelined kernels only
+constexpr int LOG_K_MAX = 2048;  // largest K of the log-domain kernels' shapes
+constexpr int LOG_KC_MAX = 16384;
 constexpr int NT_MAX = 512;  // threads per CTA
 constexpr int TS = 32;       // prefix-sum rows per TMA tile
 constexpr int FLUSH_EVERY = 64;  // positions between fp32 -> fp64 partial flushes
@@ -27,7 +29,8 @@ struct Dims {
   int delta;     // checkpoint spacing ceil(sqrt(T*K))
   int nck;       // checkpoint segments per sequence, ceil(T / delta)
   int Tstride;   // rows per sequence in the prefix-sum arrays (>= T+1, multiple of TS)
-  int KBT, GB;   // durations per lane, lanes per label (k fan-in)
+  int KBT, GB;   // durations per lane, lanes per label (k fan-in); KBT = 0: no
+                 // log-domain shape (long durations), see logok
   int CAT, GA;   // labels per lane, lanes per output label (label fan-in)
   int RL;        // ring entries per label: K + KBT (the first KBT slots are mirrored)
   int PC;        // padded length of the exp-domain label vector (>= GA * CAT)

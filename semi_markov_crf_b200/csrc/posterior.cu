@@ -72,7 +72,7 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 __global__ void __launch_bounds__(256)
     cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                     const float* __restrict__ trans, const float* __restrict__ dur, int pj) {
-  extern __shared__ float csh[];  // la [K][C], lb [K][C], dd [K][C]
+  extern __shared__ float csh[];  // la, lb, dd: [C][K + 1] each
   __shared__ float lab_M[128], lab_f[128];  // per label: shift, log2 share
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int C = d.C, K = d.K;
@@ -91,9 +91,13 @@ __global__ void __launch_bounds__(256)
     return;
   }
   const float M = *ws.tmax;  // max trans2, written by the rings
+  // label-major rows of KP = K + 1 floats (the odd stride keeps both the
+  // staging stores, consecutive labels, and the sums' reads, consecutive
+  // offsets of one label, free of bank conflicts)
+  const int KP = K + 1;
   float* const la = csh;
-  float* const lb = csh + (size_t)K * C;
-  float* const dd = csh + 2 * (size_t)K * C;
+  float* const lb = csh + (size_t)KP * C;
+  float* const dd = csh + 2 * (size_t)KP * C;
   const double Fu = kf_at(ws, d, b, 0, u), Gu = kf_at(ws, d, b, 1, u + 1);
   const int32_t* si = ws.sint + (size_t)b * d.Tstride * C;
   const float* sf = ws.sfrac + (size_t)b * d.Tstride * C;
@@ -119,26 +123,29 @@ __global__ void __launch_bounds__(256)
         vb = (lg2(bt) + (float)(kf_at(ws, d, b, 1, t) - Gu)) +
              ((float)(si[(size_t)t * C + c] - su) + (sf[(size_t)t * C + c] - fu));
     }
-    la[i] = va;
-    lb[i] = vb;
-    dd[i] = 2.f * M + __ldg(dur + i) * l2e();
+    la[c * KP + q] = va;
+    lb[c * KP + q] = vb;
+    dd[c * KP + q] = 2.f * M + __ldg(dur + i) * l2e();
   }
   __syncthreads();
   const int lane = tid & 31, nw = blockDim.x >> 5;
   for (int c = tid >> 5; c < C; c += nw) {
     // lanes over the start offset ia, inner loop over the end offset jb
     float zmax = NEG_INF, sum = 0.f;
+    const float* const lac = la + c * KP;
+    const float* const lbc = lb + c * KP;
+    const float* const ddc = dd + c * KP;
     for (int ia = lane; ia < K; ia += 32) {
-      const float a = la[ia * C + c];
+      const float a = lac[ia];
       if (a == NEG_INF) continue;
-      for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lb[jb * C + c]) + dd[(ia + jb) * C + c]);
+      for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lbc[jb]) + ddc[ia + jb]);
     }
     zmax = group_max(zmax, 32);
     const float Mz = (zmax == NEG_INF) ? 0.f : ceilf(zmax);
     for (int ia = lane; ia < K; ia += 32) {
-      const float a = la[ia * C + c] - Mz;
+      const float a = lac[ia] - Mz;
       if (a == NEG_INF) continue;
-      for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lb[jb * C + c]) + dd[(ia + jb) * C + c]);
+      for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lbc[jb]) + ddc[ia + jb]);
     }
     sum = group_sum(sum, 32);
     if (lane == 0) {
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // Shared memory of cut_grid_kernel.
-size_t cut_grid_smem_bytes(const Dims& d) { return 3ull * d.K * d.C * sizeof(float); }
+size_t cut_grid_smem_bytes(const Dims& d) { return 3ull * (d.K + 1) * d.C * sizeof(float); }
 
 namespace {
 

@@ -394,10 +394,14 @@ __device__ __forceinline__ float k_fanin(const float2* r, int rot, float Q, cons
 // group interleave over consecutive ring entries, so a group's reads of one q
 // are contiguous), y_q = ((P + Q) + v) + dur2.  Same predicted-shift scheme
 // and fallback as k_fanin; returns the group LSE, m and s describe the sum.
+// With H > 32 (long durations) the lanes of a label span H / 32 warps and
+// every sum, max and shift here is per warp: the caller adds the warps'
+// partial sums, each in the linear domain of the same frame.
 template <int KBH, int H, int N>
 __device__ __forceinline__ float k_fanin_strided(const float2* r, float Q, const float (&d)[N],
                                                  float& m, float& s, bool live) {
   static_assert(N >= KBH, "duration array shorter than the lane's terms");
+  constexpr int HG = H > 32 ? 32 : H;
   {
     const float Qm = Q - m;  // exact: both integers
     float sp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -406,10 +410,10 @@ __device__ __forceinline__ float k_fanin_strided(const float2* r, float Q, const
       const float2 v = r[q * H];
       sp[q & 3] += ex2(((v.y + Qm) + v.x) + d[q]);
     }
-    s = gsum<H>((sp[0] + sp[1]) + (sp[2] + sp[3]));
+    s = gsum<HG>((sp[0] + sp[1]) + (sp[2] + sp[3]));
   }
   if (live && !(s >= 0x1p-64f && s <= 0x1p64f)) {
-    const unsigned gm = gmask<H>();
+    const unsigned gm = gmask<HG>();
     float mx = NEG_INF;
 #pragma unroll
     for (int q = 0; q < KBH; ++q) {
@@ -417,7 +421,7 @@ __device__ __forceinline__ float k_fanin_strided(const float2* r, float Q, const
       mx = fmaxf(mx, ((v.y + Q) + v.x) + d[q]);
     }
 #pragma unroll
-    for (int o = H / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gm, mx, o));
+    for (int o = HG / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(gm, mx, o));
     m = (mx == NEG_INF) ? 0.f : ceilf(mx);
     const float Qm = Q - m;
     float ss = 0.f;
@@ -427,7 +431,7 @@ __device__ __forceinline__ float k_fanin_strided(const float2* r, float Q, const
       ss += ex2(((v.y + Qm) + v.x) + d[q]);
     }
 #pragma unroll
-    for (int o = H / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gm, ss, o);
+    for (int o = HG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gm, ss, o);
     s = ss;
   }
   return (s > 0.f) ? m + lg2(s) : NEG_INF;

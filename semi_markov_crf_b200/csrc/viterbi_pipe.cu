@@ -52,8 +52,9 @@ constexpr int VREBASE = 4096;  // steps between integer rebases (keeps y exact)
 struct VSmem {
   Smem s;      // mbar, tint, tfrac (every label), ring (own labels)
   float* V;    // [2][xPC]  V of the step of that parity (-inf padded, all labels)
-  float* Om;   // [2][Cr]   helpers' best k >= 3 candidate, frame Phi_{t-2}
-  int* Ok;     // [2][Cr]   its duration
+  float* Om;   // [HW][2][Cr] helpers' best k >= 3 candidate, frame Phi_{t-2}, one per
+               // helper warp of a label (HW = ceil(xH / 32))
+  int* Ok;     // [HW][2][Cr] its duration
   float* A1;   // [2][Cr]   dur2[0] + S[t] - S[t-1]
   float* A2;   // [2][Cr]   dur2[1] + S[t] - S[t-2]
   float* nsl;  // [2]       frame step published by the combine warps
@@ -88,10 +89,11 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d, bool 
   float* f = reinterpret_cast<float*>(p);
   x.V = f;
   f += 2 * d.xPC;
+  const int hw = (d.xH + 31) / 32;
   x.Om = f;
-  f += 2 * Cr;
+  f += 2 * Cr * hw;
   x.Ok = reinterpret_cast<int*>(f);
-  f += 2 * Cr;
+  f += 2 * Cr * hw;
   x.A1 = f;
   f += 2 * Cr;
   x.A2 = f;
@@ -107,8 +109,9 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d, bool 
 
 // Dynamic shared memory of the kernel (carve order of vcarve).
 __host__ __device__ __forceinline__ size_t vsmem_bytes(const Dims& d, bool pj) {
+  const size_t hw = (d.xH + 31) / 32;  // helper warps per label (long durations: > 1)
   return 96 + 2ull * TS * d.C * (pj ? 12 : 8) + (size_t)d.xRLP * d.xCr * 8 + 16 +
-         (2ull * d.xPC + 9ull * d.xCr) * 4;
+         (2ull * d.xPC + (5ull + 4 * hw) * d.xCr) * 4;
 }
 
 // Bounded wait for prefix-sum tile `ti`; false (uniformly) if it gave up.
@@ -164,16 +167,24 @@ __global__ void __launch_bounds__(LB, 1)
   }
 
   // ---------------------------------------------------------------- roles
-  constexpr int LPWC = 32 / G, LPWH = 32 / H, WL = H * KBH;
+  // Long durations: H > 32 lanes per label spread over HW = H / 32 helper
+  // warps; each warp finds the best k >= 3 candidate of its share of the
+  // window and the combine takes the best of the warps' candidates.
+  constexpr int HG = H > 32 ? 32 : H;       // lanes per reduction group
+  constexpr int HW = H > 32 ? H / 32 : 1;   // helper warps per label
+  constexpr int LPWC = 32 / G, LPWH = 32 / HG, WL = H * KBH;
   constexpr int CA = (G * CAT + H - 1) / H;  // labels per lane for the frame max
   constexpr int NR = CAT > KBH ? CAT : KBH;
   const int warp = tid >> 5, lane = tid & 31;
   const int nwc = (Cr + LPWC - 1) / LPWC;
   const bool comb = warp < nwc;
   const int c0 = rank * Cr;  // first label of this CTA
-  const int cl = comb ? warp * LPWC + lane / G : (warp - nwc) * LPWH + lane / H;  // local label
+  const int hwi = warp - nwc;  // helper warp index
+  const int cl = comb ? warp * LPWC + lane / G
+                      : (HW > 1 ? hwi / HW : hwi * LPWH + lane / H);  // local label
+  const int hwarp = HW > 1 && !comb ? hwi % HW : 0;  // this lane's warp among its label's
   const int c = c0 + cl;     // global label
-  const int jl = comb ? lane % G : lane % H;
+  const int jl = comb ? lane % G : (HW > 1 ? hwarp * 32 + lane : lane % H);
   const bool act = cl < Cr && c < C;
   const int cc = act ? c : 0;     // global label (tile rows, parameters, outputs)
   const int ccl = act ? cl : 0;   // local label (ring, per-label arrays)
@@ -214,9 +225,11 @@ __global__ void __launch_bounds__(LB, 1)
   // ---------------------------------------------------------------- shared state
   for (int i = tid; i < RLP * Cr; i += blockDim.x) sm.ring[i] = make_float2(NEG_INF, 0.f);
   for (int i = tid; i < 2 * d.xPC; i += blockDim.x) vs.V[i] = NEG_INF;
-  for (int i = tid; i < 2 * Cr; i += blockDim.x) {
+  for (int i = tid; i < 2 * Cr * HW; i += blockDim.x) {
     vs.Om[i] = NEG_INF;
     vs.Ok[i] = 3;
+  }
+  for (int i = tid; i < 2 * Cr; i += blockDim.x) {
     vs.A1[i] = NEG_INF;
     vs.A2[i] = NEG_INF;
   }
@@ -377,8 +390,17 @@ __global__ void __launch_bounds__(LB, 1)
       const float mp = vs.mx[(i - 1) & 1];
       const float a1 = vs.A1[(i & 1) * Cr + ccl];
       const float a2 = vs.A2[(i & 1) * Cr + ccl];
-      const float om = vs.Om[(i & 1) * Cr + ccl];
-      const int okd = vs.Ok[(i & 1) * Cr + ccl];
+      float om = vs.Om[(i & 1) * Cr + ccl];
+      int okd = vs.Ok[(i & 1) * Cr + ccl];
+#pragma unroll
+      for (int hw = 1; hw < HW; ++hw) {  // long durations: the warps' best, smallest k on ties
+        const float o2 = vs.Om[hw * 2 * Cr + (i & 1) * Cr + ccl];
+        const int k2 = vs.Ok[hw * 2 * Cr + (i & 1) * Cr + ccl];
+        if (o2 > om || (o2 == om && k2 < okd)) {
+          om = o2;
+          okd = k2;
+        }
+      }
       const bool rok = SEMICRF_INB(ws.status, row_ok(crow_i), SITE_TILE_ROW);
       const int si_n = rok ? crow_i[cc] : 0;  // row i: the next step's ring entry
       const float pd_n = (crow_d && rok) ? crow_d[cc] : 0.f;
@@ -472,7 +494,7 @@ __global__ void __launch_bounds__(LB, 1)
       }
       float mv = fmaxf(m0, m1);
 #pragma unroll
-      for (int o = H / 2; o > 0; o >>= 1) {
+      for (int o = HG / 2; o > 0; o >>= 1) {
         best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
         mv = fmaxf(mv, __shfl_xor_sync(FULL_MASK, mv, o));
       }
@@ -482,13 +504,16 @@ __global__ void __launch_bounds__(LB, 1)
       for (int q = 0; q < KBH; ++q)
         if (tv[q] == best) kb = 2 + WL - (q * H + jl);
 #pragma unroll
-      for (int o = H / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
+      for (int o = HG / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
       // stores (every label group saw all of V[i-1]: the first one publishes)
       if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;
+      if (act && lane % HG == 0 && i < L) {  // each helper warp's candidate
+        const int o2 = ((i + 1) & 1) * Cr + cl;
+        vs.Om[hwarp * 2 * Cr + o2] = best + fn;
+        vs.Ok[hwarp * 2 * Cr + o2] = kb;
+      }
       if (leader && i < L) {
         const int o2 = ((i + 1) & 1) * Cr + cl;
-        vs.Om[o2] = best + fn;
-        vs.Ok[o2] = kb;
         vs.A1[o2] = (d1 + hd_c) + ((float)(sn - hs_c) + (fn - hf_c));
         vs.A2[o2] = (d2 + hd_p) + ((float)(sn - hs_p) + (fn - hf_p));
       }
@@ -544,7 +569,9 @@ constexpr int VW_ROWS = 64;
 template <int NW>
 __global__ void __launch_bounds__(256)
     viterbi_words_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                         const float* __restrict__ trans) {
+                         const float* __restrict__ trans, int staged) {
+  // staged = 0 (long durations: the rows a block's segments start on do not
+  // fit shared memory): the V rows are read from global memory instead
   extern __shared__ __align__(16) float vsh[];  // [VW_ROWS + K][VS]
   const int C = d.C, K = d.K, tid = threadIdx.x, b = blockIdx.y;
   const int L = lengths[b];
@@ -558,7 +585,7 @@ __global__ void __launch_bounds__(256)
   const int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
   int32_t* wrd = ws.wrd + (size_t)b * (d.T + 1) * VS;
   int32_t* wdl = ws.wdl + (size_t)b * (d.T + 1) * VS;
-  const int nv = (t1 - vlo) * VS;
+  const int nv = staged ? (t1 - vlo) * VS : 0;
 #pragma unroll 4
   for (int i = tid; i < nv; i += blockDim.x) {
     const int r = i / VS, x = i - r * VS;
@@ -575,7 +602,30 @@ __global__ void __launch_bounds__(256)
     const int k = kdw[(size_t)t * C + pc];
     const int sb = t - k;
     int word = k, step = 0;
-    if (k >= 1 && k <= K && sb >= 1) {
+    if (k >= 1 && k <= K && sb >= 1 && !staged) {
+      // the same compare order as the staged path below (chains q mod 4,
+      // merged by value then index), reading row sb from global memory
+      const float* vg = vrw + (size_t)sb * C;
+      float bq[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      int qq[4] = {0, 1, 2, 3};
+#pragma unroll
+      for (int q = 0; q < NW; ++q) {
+        if (q < C) {
+          const float e = vg[q] + w2[q];
+          if (e > bq[q & 3]) {
+            bq[q & 3] = e;
+            qq[q & 3] = q;
+          }
+        }
+      }
+      float b0 = bq[0], b2 = bq[2];
+      int q0 = qq[0], q2 = qq[2];
+      if (bq[1] > b0 || (bq[1] == b0 && qq[1] < q0)) { b0 = bq[1]; q0 = qq[1]; }
+      if (bq[3] > b2 || (bq[3] == b2 && qq[3] < q2)) { b2 = bq[3]; q2 = qq[3]; }
+      if (b2 > b0 || (b2 == b0 && q2 < q0)) { b0 = b2; q0 = q2; }
+      word = k | (q0 << 16);
+      step = -k * VS + (q0 - pc);
+    } else if (k >= 1 && k <= K && sb >= 1) {
       const float4* vr = reinterpret_cast<const float4*>(vsh + (size_t)(sb - vlo) * VS);
       float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
       int q0 = 0, q1 = 1, q2 = 2, q3 = 3;
@@ -741,7 +791,14 @@ size_t viterbi_pipe_smem_bytes(const Dims& d, bool pj) { return vsmem_bytes(d, p
 
 cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                  const float* trans, cudaStream_t st) {
-  const size_t sm = (size_t)(VW_ROWS + d.K) * ((d.C + 3) & ~3) * sizeof(float);
+  size_t sm = (size_t)(VW_ROWS + d.K) * ((d.C + 3) & ~3) * sizeof(float);
+  int max_optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+          cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int staged = sm + 256 <= (size_t)max_optin ? 1 : 0;
+  if (!staged) sm = 0;
   const dim3 grid((d.T + VW_ROWS - 1) / VW_ROWS, d.B);
   if (d.T == 0) return cudaSuccess;
 #define SEMICRF_VW_LAUNCH(nw)                                                                   \
@@ -752,7 +809,7 @@ cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t*
                                                  (int)sm);                                      \
       if (e != cudaSuccess) return e;                                                           \
     }                                                                                           \
-    viterbi_words_kernel<nw><<<grid, 256, sm, st>>>(d, ws, lengths, trans);                     \
+    viterbi_words_kernel<nw><<<grid, 256, sm, st>>>(d, ws, lengths, trans, staged);             \
     return cudaGetLastError();                                                                  \
   }
   SEMICRF_VW_WIDTHS(SEMICRF_VW_LAUNCH)

@@ -44,10 +44,16 @@
  *    a bounded wait that gave up) are recorded in the workspace status word,
  *    read with semicrf_get_status.
  *  - Limits of the library: 1 <= C <= 128, T <= 2^26, B <= 2^20, and
- *    K <= 2048 (C <= 8), K <= 512 (C <= 16), K <= 256 (C <= 32),
+ *    K <= 8192 (C <= 8), K <= 512 (C <= 16), K <= 256 (C <= 32),
  *    K <= 128 (C <= 64), K <= 64 (C <= 128).  Larger values return
- *    SEMICRF_ERR_UNSUPPORTED.  (Durations up to K = 2000 on sequences of
- *    10^6 positions are the pages' genomic regime, explainer section 4.)
+ *    SEMICRF_ERR_UNSUPPORTED.  (Durations of K = 2000-8000 on sequences of
+ *    10^6 positions are the pages' genomic regime, explainer section 4 and
+ *    the Chinese explainer's section 4.)  Long durations, 2048 < K <= 8192,
+ *    run on the exponential-domain rings and the pipelined decoder only:
+ *    a sequence whose scores leave those rings' exponent range (see
+ *    SEMICRF_FLAG_LOG_DOMAIN) is reported through the status word as
+ *    SEMICRF_ERR_UNSUPPORTED with log Z = NaN and zero posteriors, and
+ *    SEMICRF_FLAG_LOG_DOMAIN itself returns SEMICRF_ERR_UNSUPPORTED.
  *  - Numbers are computed in float32 in base-2 log units with exactly
  *    representable integer frames and float64 normalisers; results are
  *    deterministic (no floating-point atomics).
@@ -137,11 +143,13 @@ SEMICRF_API int semicrf_workspace_itemize(int B, int T, int C, int K, unsigned f
  * CTA per ring; more: a thread-block cluster), labels per CTA, combine lanes
  * per label, weights per combine lane, helper lanes per label, durations per
  * helper lane, threads per CTA, checkpoint spacing Delta, checkpoint
- * segments per sequence, posterior tile rows, and the log-domain kernels'
- * durations per lane, lanes per label, labels per lane and threads per CTA.
+ * segments per sequence, posterior tile rows, the log-domain kernels'
+ * durations per lane, lanes per label, labels per lane and threads per CTA
+ * (0: no log-domain kernel for these sizes), the segment-end rows the
+ * posterior pass stages at once, and the cut-normaliser grid spacing.
  * Returns the same codes as semicrf_workspace_bytes.
  */
-#define SEMICRF_SHAPE_FIELDS 14
+#define SEMICRF_SHAPE_FIELDS 16
 SEMICRF_API int semicrf_launch_shape(int B, int T, int C, int K, int32_t *shape, int n);
 
 /*

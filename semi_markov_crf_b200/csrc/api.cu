@@ -151,7 +151,7 @@ void choose_xshape(Dims& d, size_t budget) {
   d = pick;
   // the posterior pass from the kept values and the cut normaliser must fit too
   d.pRT = posterior_tile_rows(d, budget);
-  if (d.pRT == 0 || cut_grid_smem_bytes(d) > budget || d.C > 128) {
+  if (d.pRT == 0 || cut_grid_smem_bytes(d, budget) > budget || d.C > 128) {
     d.xG = 0;
     d.xN = 1;
     d.xCr = C;
@@ -238,6 +238,9 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
     d.store_smem = recursion_smem_bytes(d, true) <= budget ? 1 : 0;
     if (recursion_smem_bytes(d, false) > budget) d.KBT = 0;
   }
+  // sizes without a log-domain shape are served only in the long-duration
+  // regime (K > LOG_K_MAX, C <= 8: the pipelined kernels alone)
+  if (!d.KBT && K <= LOG_K_MAX) return SEMICRF_ERR_UNSUPPORTED;
   if (!d.KBT) {  // no log-domain kernels for these sizes (long durations)
     d.KBT = d.GB = d.CAT = d.GA = d.RL = d.NT = d.LB = 0;
     d.PC = ((C + 3) / 4) * 4;
@@ -472,6 +475,8 @@ int run_chains(const Dims& d, WsPtrs p, const int32_t* lengths, const float* tra
                const float* dur, double* logZ, int n_alpha, int n_beta, unsigned flags,
                cudaStream_t st, bool proj = false) {
   cudaError_t e = cudaSuccess;
+  // long durations have only the pipelined kernels
+  if (!d.KBT && !pipelined(d, flags, proj)) return SEMICRF_ERR_UNSUPPORTED;
   if (pipelined(d, flags, proj)) {
     ProfScope ps("chain_exp_kernel", st);
     e = launch_chain_exp(d, p, lengths, trans, dur, logZ, n_alpha, n_beta, st, proj ? 1 : 0);
@@ -531,7 +536,8 @@ extern "C" int semicrf_launch_shape(int B, int T, int C, int K, int32_t* shape, 
   const int rc = make_dims(B, T, C, K, d);
   if (rc != SEMICRF_OK) return rc;
   const int32_t v[SEMICRF_SHAPE_FIELDS] = {d.xG ? d.xN : 0, d.xCr, d.xG, d.xCAT, d.xH, d.xKBH,
-                                           d.xNT, d.delta, d.nck, d.pRT, d.KBT, d.GB, d.CAT, d.NT};
+                                           d.xNT, d.delta, d.nck, d.pRT, d.KBT, d.GB, d.CAT, d.NT,
+                                           d.pKH, d.GS};
   for (int i = 0; i < n; ++i) shape[i] = i < SEMICRF_SHAPE_FIELDS ? v[i] : 0;
   return SEMICRF_OK;
 }
@@ -673,12 +679,14 @@ int backward_impl(const int32_t* lengths, const float* trans, const float* dur, 
                              seg_marg);
     }
     if (d.xG) {
-      const size_t csm = cut_grid_smem_bytes(d);
+      const size_t budget = (size_t)max_smem_optin() - 256;
+      const size_t csm = cut_grid_smem_bytes(d, budget);
       if ((rc = set_smem((const void*)cut_grid_kernel, csm))) return rc;
       {
         ProfScope ps("cut_grid_kernel", st);
         cut_grid_kernel<<<dim3(d.ngrid, B), 256, csm, st>>>(d, p, lengths, trans, dur,
-                                                            proj ? 1 : 0);
+                                                            proj ? 1 : 0,
+                                                            cut_grid_per_label(d, budget) ? 1 : 0);
       }
       if ((rc = launched())) return rc;
       {
@@ -790,6 +798,7 @@ int viterbi_impl(const float* em, const int32_t* lengths, const float* trans, co
   if (rc) return rc;
   cudaError_t e;
   // the pipelined decoder, unless no shape fits (then the one-role kernel)
+  if (!d.KBT && !pipelined(d, 0, proj)) return SEMICRF_ERR_UNSUPPORTED;
   if (pipelined(d, 0, proj)) {
     {
       ProfScope ps("viterbi_pipe_kernel", st);

@@ -57,7 +57,7 @@ __device__ __forceinline__ bool posterior_from_kept(const WsPtrs& ws, const Dims
 
 __global__ void cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                                 const float* __restrict__ trans, const float* __restrict__ dur,
-                                int pj);
+                                int pj, int per_label);
 // The posterior pass (one CTA per checkpoint segment and sequence).
 // seg_marg (nullable) [B][T][K][C]: the segment marginals of the sequences
 // the kernel takes (the caller zeroes the array first).
@@ -68,8 +68,9 @@ cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* len
 size_t posterior_smem_bytes(const Dims& d);
 // Tile rows for the posterior pass under `budget` bytes of shared memory (0:
 // none fits).
-int posterior_tile_rows(const Dims& d, size_t budget);
-size_t cut_grid_smem_bytes(const Dims& d);
+int posterior_tile_rows(Dims& d, size_t budget);
+bool cut_grid_per_label(const Dims& d, size_t budget);
+size_t cut_grid_smem_bytes(const Dims& d, size_t budget);
 
 // Sizes, launch geometry and limits for (B, T, C, K); returns a semicrf_status.
 int make_dims(int B, int T, int C, int K, Dims& d);

@@ -58,6 +58,8 @@ struct Dims {
   // GS positions, ngrid grid points per sequence; the posterior pass stages
   // pRT boundaries (plus K rows of halo) of kept values per tile.
   int GS, ngrid, pRT;
+  int pKH;       // segment-end rows staged at once by the posterior pass (K, or a
+                 // chunk of the durations for long durations)
   int npch;      // path-score chunks per sequence, ceil(T / PATH_ROWS)
 };
 

@@ -126,6 +126,8 @@ extern "C" int semicrf_forward_noalloc(const float* em, const int32_t* lengths, 
     if (cudaGetLastError() != cudaSuccess) return SEMICRF_ERR_CUDA;
   }
   // exponential-domain ring where the scores allow it, log domain for the rest
+  // (long durations have no log-domain kernel: declined rings are reported)
+  if (!d.KBT && (!d.xG || (flags & SEMICRF_FLAG_LOG_DOMAIN))) return SEMICRF_ERR_UNSUPPORTED;
   if (d.xG && !(flags & SEMICRF_FLAG_LOG_DOMAIN)) {
     if (launch_chain_exp(d, p, lengths, trans, dur, logZ, B, 0, st) != cudaSuccess)
       return SEMICRF_ERR_CUDA;

@@ -71,9 +71,13 @@ __device__ __forceinline__ double local_logz(const Dims& d, const double* nc, in
 // per label sums them (its max first, so the sum cannot overflow).
 __global__ void __launch_bounds__(256)
     cut_grid_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                    const float* __restrict__ trans, const float* __restrict__ dur, int pj) {
-  extern __shared__ float csh[];  // la, lb, dd: [C][K + 1] each
+                    const float* __restrict__ trans, const float* __restrict__ dur, int pj,
+                    int per_label) {
+  // la, lb, dd: [C][K + 1] each; per_label (long durations): [K + 1] each,
+  // one label at a time, every thread of the block on that label
+  extern __shared__ float csh[];
   __shared__ float lab_M[128], lab_f[128];  // per label: shift, log2 share
+  __shared__ float red[32];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int C = d.C, K = d.K;
   const int L = lengths[b];
@@ -95,17 +99,17 @@ __global__ void __launch_bounds__(256)
   // staging stores, consecutive labels, and the sums' reads, consecutive
   // offsets of one label, free of bank conflicts)
   const int KP = K + 1;
+  const int CB = per_label ? 1 : C;  // labels staged at once
   float* const la = csh;
-  float* const lb = csh + (size_t)KP * C;
-  float* const dd = csh + 2 * (size_t)KP * C;
+  float* const lb = csh + (size_t)KP * CB;
+  float* const dd = csh + 2 * (size_t)KP * CB;
   const double Fu = kf_at(ws, d, b, 0, u), Gu = kf_at(ws, d, b, 1, u + 1);
   const int32_t* si = ws.sint + (size_t)b * d.Tstride * C;
   const float* sf = ws.sfrac + (size_t)b * d.Tstride * C;
   const float* kf0 = kv_row(ws, d, b, 0, 0);
   const float* kf1 = kv_row(ws, d, b, 1, 0);
-  #pragma unroll 4
-  for (int i = tid; i < K * C; i += blockDim.x) {
-    const int q = i / C, c = i - q * C;
+  // the start side (s = u - q) and end side (t = u + 1 + q) of label c
+  auto stage = [&](int i, int q, int c, int slot) {
     const int su = si[(size_t)u * C + c];
     const float fu = sf[(size_t)u * C + c];
     float va = NEG_INF, vb = NEG_INF;
@@ -123,12 +127,55 @@ __global__ void __launch_bounds__(256)
         vb = (lg2(bt) + (float)(kf_at(ws, d, b, 1, t) - Gu)) +
              ((float)(si[(size_t)t * C + c] - su) + (sf[(size_t)t * C + c] - fu));
     }
-    la[c * KP + q] = va;
-    lb[c * KP + q] = vb;
-    dd[c * KP + q] = 2.f * M + __ldg(dur + i) * l2e();
+    la[slot * KP + q] = va;
+    lb[slot * KP + q] = vb;
+    dd[slot * KP + q] = 2.f * M + __ldg(dur + i) * l2e();
+  };
+  const int lane = tid & 31;
+  if (per_label) {
+    // long durations: label by label, all threads over the start offset ia
+    const int nw = blockDim.x >> 5, wid = tid >> 5;
+    for (int c = 0; c < C; ++c) {
+      for (int q = tid; q < K; q += blockDim.x) stage(q * C + c, q, c, 0);
+      __syncthreads();
+      float zmax = NEG_INF;
+      for (int ia = tid; ia < K; ia += blockDim.x) {
+        const float a = la[ia];
+        if (a == NEG_INF) continue;
+        for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lb[jb]) + dd[ia + jb]);
+      }
+      zmax = group_max(zmax, 32);
+      if (lane == 0) red[wid] = zmax;
+      __syncthreads();
+      float mz = NEG_INF;
+      for (int w2 = 0; w2 < nw; ++w2) mz = fmaxf(mz, red[w2]);
+      const float Mz = (mz == NEG_INF) ? 0.f : ceilf(mz);
+      __syncthreads();
+      float sum = 0.f;
+      for (int ia = tid; ia < K; ia += blockDim.x) {
+        const float a = la[ia] - Mz;
+        if (a == NEG_INF) continue;
+        for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lb[jb]) + dd[ia + jb]);
+      }
+      sum = group_sum(sum, 32);
+      if (lane == 0) red[wid] = sum;
+      __syncthreads();
+      if (tid == 0) {
+        float tot = 0.f;
+        for (int w2 = 0; w2 < nw; ++w2) tot += red[w2];  // fixed order: deterministic
+        lab_M[c] = Mz;
+        lab_f[c] = (tot > 0.f) ? lg2(tot) : NEG_INF;
+      }
+      __syncthreads();
+    }
+  } else {
+  #pragma unroll 4
+  for (int i = tid; i < K * C; i += blockDim.x) {
+    const int q = i / C, c = i - q * C;
+    stage(i, q, c, c);
   }
   __syncthreads();
-  const int lane = tid & 31, nw = blockDim.x >> 5;
+  const int nw = blockDim.x >> 5;
   for (int c = tid >> 5; c < C; c += nw) {
     // lanes over the start offset ia, inner loop over the end offset jb
     float zmax = NEG_INF, sum = 0.f;
@@ -154,6 +201,7 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
+  }
   if (tid < 32) {
     float Mz = NEG_INF;
     for (int c = lane; c < C; c += 32)
@@ -168,30 +216,45 @@ __global__ void __launch_bounds__(256)
 }
 
 // Shared memory of cut_grid_kernel.
-size_t cut_grid_smem_bytes(const Dims& d) { return 3ull * (d.K + 1) * d.C * sizeof(float); }
+// Shared memory of cut_grid_kernel: every label's rows when they fit the
+// budget, else one label's (cut_grid_per_label).
+bool cut_grid_per_label(const Dims& d, size_t budget) {
+  return 3ull * (d.K + 1) * d.C * sizeof(float) > budget;
+}
+size_t cut_grid_smem_bytes(const Dims& d, size_t budget) {
+  return 3ull * (d.K + 1) * (cut_grid_per_label(d, budget) ? 1 : d.C) * sizeof(float);
+}
 
 namespace {
 
 // Shared memory carve of posterior_kernel for a tile of RT boundaries.
 // (With boundary projections pd holds the start terms of the tile's rows.)
+// Segment ends: a tile's segments end on up to RT + K rows.  Those rows are
+// staged KH at a time (KH = K: all at once; long durations: chunks of the
+// duration range, each staging RT + KH rows), so the halo arrays hold
+// R = RT + KH rows and, when chunked, the tile rows' own integer and
+// fractional prefix sums have arrays of their own (tii, tsf).
 struct PTile {
   double* dif;  // [RT][C]   St - E of each boundary and label
   float* tf;    // [RT][2C]  forward kept rows: p, acc
   float* pb;    // [RT][C]   backward p
-  float* ab;    // [R][C]    backward acc, R = RT + K rows (segment ends)
+  float* ab;    // [R][C]    backward acc of the staged segment-end rows
   int* ii;      // [R][C]    (Pb_r - Pb_lo) + S_int[r, c], exact integers
   float* sf;    // [R][C]    S_frac[r, c]
   float* vv;    // [RT][C]   suffix sums v of the tile
   float* fs;    // [RT]      f_s
   float* pd;    // [RT][C]   projection start terms of the tile's rows (0 without)
+  int* tii;     // [RT][C]   ii of the tile rows (aliases ii when not chunked)
+  float* tsf;   // [RT][C]   sf of the tile rows (aliases sf when not chunked)
 };
-__host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int K, int C) {
-  const size_t R = (size_t)RT + K;
-  return (size_t)C * (28ull * RT + 12ull * R) + 4ull * RT;
+__host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int KH, int C, bool chunked) {
+  const size_t R = (size_t)RT + KH;
+  return (size_t)C * (28ull * RT + 12ull * R + (chunked ? 8ull * RT : 0)) + 4ull * RT;
 }
-__device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, int C) {
+__device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH, int C,
+                                             bool chunked) {
   PTile t;
-  const size_t R = (size_t)RT + K;
+  const size_t R = (size_t)RT + KH;
   t.dif = reinterpret_cast<double*>(raw);
   t.tf = reinterpret_cast<float*>(t.dif + (size_t)RT * C);
   t.pb = t.tf + (size_t)RT * 2 * C;
@@ -201,6 +264,12 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int K, 
   t.vv = t.sf + R * C;
   t.fs = t.vv + (size_t)RT * C;
   t.pd = t.fs + RT;
+  t.tii = t.ii;
+  t.tsf = t.sf;
+  if (chunked) {
+    t.tii = reinterpret_cast<int*>(t.pd + (size_t)RT * C);
+    t.tsf = reinterpret_cast<float*>(t.tii + (size_t)RT * C);
+  }
   return t;
 }
 
@@ -229,7 +298,8 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
                      float* __restrict__ seg_marg, int pj) {
   extern __shared__ __align__(16) unsigned char psh[];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
-  const int C = d.C, K = d.K, RT = d.pRT;
+  const int C = d.C, K = d.K, RT = d.pRT, KH = d.pKH;
+  const bool chunked = KH < K;  // long durations: the segment ends come KH rows at a time
   const int L = lengths[b];
   if (L <= 0 || L > d.T) return;
   if (!posterior_from_kept(ws, d, b)) return;  // segment_kernel runs it
@@ -239,7 +309,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
   const size_t seg = (size_t)b * d.nck + j;
   const float gb = (float)(grad_logZ ? grad_logZ[b] : 1.0);
   const float M = *ws.tmax;  // max trans2, written by the rings
-  const PTile tl = ptile_carve(psh, RT, K, C);
+  const PTile tl = ptile_carve(psh, RT, KH, C, chunked);
   const float* pfr = kv_row(ws, d, b, 0, 0);  // row t: pfr + t*2C (p), + C (acc)
   const float* pbr = kv_row(ws, d, b, 1, 0);
   const double* kff = ws.kf + ((size_t)b * 2 + 0) * (d.T + 1);
@@ -260,70 +330,101 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     const int nr = s_hi - s_lo;
     const int nh = min(s_hi - 1 + K, L) - s_lo + 1;  // rows a segment of the tile ends on
     const bool first = (s_hi == t1);
-    // bounds-check build: the tile and its halo fit the staged rows
+    // bounds-check build: the tile fits its rows
     if (!SEMICRF_INB(ws.status, nr >= 1 && nr <= RT && nh <= RT + K, SITE_POST_TILE)) break;
-    // ------------------------------------------------------------ stage
+    // ------------------------------------------------------------ stage the tile rows
     const double kb0 = kfb[s_lo];
     #pragma unroll 4
     for (int i = tid; i < nr * 2 * C; i += nthr) tl.tf[i] = pfr[(size_t)s_lo * 2 * C + i];
     #pragma unroll 4
-    for (int i = tid; i < nh * C; i += nthr) {
+    for (int i = tid; i < nr * C; i += nthr) {
       const int r = i / C, c = i - r * C;
       const size_t row = (size_t)(s_lo + r);
-      tl.ab[i] = pbr[row * 2 * C + C + c];
-      tl.ii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
-      tl.sf[i] = sfp[row * C + c];
-      if (r < nr) {
-        tl.pb[i] = pbr[row * 2 * C + c];
-        tl.pd[i] = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
+      tl.pb[i] = pbr[row * 2 * C + c];
+      tl.pd[i] = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
+      if (chunked) {
+        tl.tii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
+        tl.tsf[i] = sfp[row * C + c];
       }
     }
     // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s))
     for (int s = s_lo + tid; s < s_hi; s += nthr)
       tl.fs[s - s_lo] = ex2((float)(((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1))));
-    __syncthreads();
-    // ------------------------------------------------------------ start / end marginals
-    for (int i = tid; i < nr * C; i += nthr) {
-      const int r = i / C, c = i - r * C;
-      const float f = tl.fs[r];
-      const float St = tl.tf[r * 2 * C + C + c] * tl.pb[i] * f;
-      const float E = tl.ab[i] * tl.tf[r * 2 * C + c] * f;
-      const size_t ob = ((size_t)b * (d.T + 1) + s_lo + r) * C + c;
-      if (start_marg) start_marg[ob] = St;
-      if (end_marg) end_marg[ob] = E;
-      tl.dif[i] = (double)St - (double)E;
-    }
-    // ------------------------------------------------------------ segment marginals
-    // (optional output) P([s, s+k), c) for every start of the tile, the same
-    // product as the duration counts below, not scaled by g (a marginal)
-    if (seg_marg) {
-      for (int i = tid; i < nr * nd; i += nthr) {
-        const int r = i / nd, idx = i - r * nd;
+    // ------------------------------------------------------------ segment ends, by chunk
+    // chunk kc: durations [kc, kc + KH), staged rows at offsets [kc - 1, kc - 1 + nr + KH)
+    // from s_lo (the first chunk includes the tile rows themselves)
+    for (int kc = 1; kc <= K; kc += KH) {
+      const int base = kc - 1;
+      const int nst = max(0, min(base + nr + KH, nh) - base);
+      if (kc > 1) __syncthreads();  // the previous chunk's reads are done
+      #pragma unroll 4
+      for (int i = tid; i < nst * C; i += nthr) {
+        const int r = i / C, c = i - r * C;
+        const size_t row = (size_t)(s_lo + base + r);
+        tl.ab[i] = pbr[row * 2 * C + C + c];
+        tl.ii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
+        tl.sf[i] = sfp[row * C + c];
+      }
+      __syncthreads();
+      if (kc == 1) {
+        // ---------------------------------------------------------- start / end marginals
+        for (int i = tid; i < nr * C; i += nthr) {
+          const int r = i / C, c = i - r * C;
+          const float f = tl.fs[r];
+          const float St = tl.tf[r * 2 * C + C + c] * tl.pb[i] * f;
+          const float E = tl.ab[i] * tl.tf[r * 2 * C + c] * f;
+          const size_t ob = ((size_t)b * (d.T + 1) + s_lo + r) * C + c;
+          if (start_marg) start_marg[ob] = St;
+          if (end_marg) end_marg[ob] = E;
+          tl.dif[i] = (double)St - (double)E;
+        }
+      }
+      const int lo_i = base * C, hi_i = min(nd, (base + KH) * C);  // this chunk's (k, c) items
+      // -------------------------------------------------------- segment marginals
+      // (optional output) P([s, s+k), c) for every start of the tile, the same
+      // product as the duration counts below, not scaled by g (a marginal)
+      if (seg_marg) {
+        const int nci = hi_i - lo_i;
+        for (int i = tid; i < nr * nci; i += nthr) {
+          const int r = i / nci, idx = lo_i + (i - r * nci);
+          const int k = idx / C + 1, c = idx - (k - 1) * C;
+          if (s_lo + r + k > L) continue;
+          if (!SEMICRF_INB(ws.status, r + k - base < nst, SITE_POST_ITEM)) continue;
+          const int o = r * C + c, ok = (r + k - base) * C + c;
+          const float z = (float)(tl.ii[ok] - tl.tii[o]) +
+                          ((M + __ldg(dur + idx) * l2e()) + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
+          seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] =
+              tl.tf[r * 2 * C + C + c] * tl.ab[ok] * (tl.fs[r] * ex2(z));
+        }
+      }
+      // -------------------------------------------------------- duration counts
+      // item (k, c): sum over the tile's s of P([s, s+k), c), s + k <= L
+      auto dur_item = [&](int idx) {
         const int k = idx / C + 1, c = idx - (k - 1) * C;
-        if (s_lo + r + k > L) continue;
-        if (!SEMICRF_INB(ws.status, r + k < nh, SITE_POST_ITEM)) continue;
-        const int o = r * C + c, ok = (r + k) * C + c;
-        const float z = (float)(tl.ii[ok] - tl.ii[o]) +
-                        ((M + __ldg(dur + idx) * l2e()) + ((tl.sf[ok] - tl.sf[o]) + tl.pd[o]));
-        seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] =
-            tl.tf[r * 2 * C + C + c] * tl.ab[ok] * (tl.fs[r] * ex2(z));
+        const float dk = M + __ldg(dur + idx) * l2e();
+        int r_end = min(s_hi, L - k + 1) - s_lo;
+        if (!SEMICRF_INB(ws.status, r_end <= 0 || r_end - 1 + k - base < nst, SITE_POST_ITEM))
+          r_end = 0;
+        float a_ = 0.f;
+        for (int r = 0; r < r_end; ++r) {
+          const int o = r * C + c, ok = (r + k - base) * C + c;
+          const float z = (float)(tl.ii[ok] - tl.tii[o]) + (dk + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
+          a_ = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a_);
+        }
+        return a_;
+      };
+#pragma unroll
+      for (int m = 0; m < NID; ++m) {
+        const int idx = tid + m * nthr;
+        if (idx >= lo_i && idx < hi_i) accd[m] += dur_item(idx);
+      }
+      for (int idx = tid + NID * nthr; idx < hi_i; idx += nthr) {
+        if (idx < lo_i) continue;
+        double* pd = ws.pgd + seg * nd + idx;
+        const double v = (double)(gb * dur_item(idx));
+        *pd = first ? v : *pd + v;
       }
     }
-    // ------------------------------------------------------------ duration counts
-    // item (k, c): sum over the tile's s of P([s, s+k), c), s + k <= L
-    auto dur_item = [&](int idx) {
-      const int k = idx / C + 1, c = idx - (k - 1) * C;
-      const float dk = M + __ldg(dur + idx) * l2e();
-      int r_end = min(s_hi, L - k + 1) - s_lo;
-      if (!SEMICRF_INB(ws.status, r_end <= 0 || r_end - 1 + k < nh, SITE_POST_ITEM)) r_end = 0;
-      float a_ = 0.f;
-      for (int r = 0; r < r_end; ++r) {
-        const int o = r * C + c, ok = (r + k) * C + c;
-        const float z = (float)(tl.ii[ok] - tl.ii[o]) + (dk + ((tl.sf[ok] - tl.sf[o]) + tl.pd[o]));
-        a_ = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a_);
-      }
-      return a_;
-    };
     // item (c', c): sum over the tile's s of P(c' -> c at s) / w[c', c]
     auto tr_item = [&](int idx) {
       const int c1 = idx / C, c = idx - c1 * C;
@@ -331,14 +432,6 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
       for (int r = 0; r < nr; ++r) a_ = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a_);
       return a_;
     };
-#pragma unroll
-    for (int m = 0; m < NID; ++m)
-      if (tid + m * nthr < nd) accd[m] += dur_item(tid + m * nthr);
-    for (int idx = tid + NID * nthr; idx < nd; idx += nthr) {
-      double* pd = ws.pgd + seg * nd + idx;
-      const double v = (double)(gb * dur_item(idx));
-      *pd = first ? v : *pd + v;
-    }
 #pragma unroll
     for (int m = 0; m < NIT; ++m)
       if (tid + m * nthr < ntr) acct[m] += tr_item(tid + m * nthr);
@@ -387,18 +480,32 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
 }  // namespace
 
 // Tile rows of the posterior pass: the largest power of two up to 64 (and
-// not past the segment) whose tile fits `budget` bytes, preferring tiles
-// that leave room for two CTAs per SM; 0 if even 8 rows do not fit.
-int posterior_tile_rows(const Dims& d, size_t budget) {
+// not past the segment) whose tile, with all K segment-end rows, fits
+// `budget` bytes, preferring tiles that leave room for two CTAs per SM.
+// Long durations: the segment ends are staged in chunks of KH rows (a
+// multiple of 64), the tile as tall as fits.  Sets d.pKH; 0 if nothing fits.
+int posterior_tile_rows(Dims& d, size_t budget) {
   int cap = 64;
   while (cap > 8 && cap / 2 >= d.delta) cap /= 2;
+  d.pKH = d.K;
   for (const size_t lim : {std::min<size_t>(budget, 112u * 1024u), budget})
     for (int rt = cap; rt >= 8; rt /= 2)
-      if (ptile_bytes(rt, d.K, d.C) <= lim) return rt;
+      if (ptile_bytes(rt, d.K, d.C, false) <= lim) return rt;
+  for (int rt = cap; rt >= 8; rt /= 2) {
+    const size_t fixed = ptile_bytes(rt, 0, d.C, true);
+    if (fixed >= budget) continue;
+    const long long kh = ((long long)((budget - fixed) / (12ull * d.C)) - rt) / 64 * 64;
+    if (kh >= 64) {
+      d.pKH = (int)std::min<long long>(kh, d.K);
+      return rt;
+    }
+  }
   return 0;
 }
 
-size_t posterior_smem_bytes(const Dims& d) { return ptile_bytes(d.pRT, d.K, d.C); }
+size_t posterior_smem_bytes(const Dims& d) {
+  return ptile_bytes(d.pRT, d.pKH, d.C, d.pKH < d.K);
+}
 
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,

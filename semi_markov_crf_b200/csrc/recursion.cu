@@ -812,9 +812,68 @@ cudaError_t allow_smem(F fn, size_t sm) {
 }
 }  // namespace
 
+namespace {
+
+// Long durations have no log-domain kernel: a ring the exponential-domain
+// kernel declined (mode 2: a score outside its exponent range) is reported
+// as SEMICRF_ERR_UNSUPPORTED in the status word and its log Z is NaN.
+__global__ void declined_chain_kernel(Dims d, WsPtrs ws, double* __restrict__ logZ_out,
+                                      int n_alpha) {
+  const bool up = (int)blockIdx.x < n_alpha;
+  const int b = up ? blockIdx.x : blockIdx.x - n_alpha;
+  if (threadIdx.x != 0 || !ws.mode || ws.mode[(up ? 0 : d.B) + b] != 2) return;
+  set_status(ws.status, 2);  // SEMICRF_ERR_UNSUPPORTED
+  const double nan = __longlong_as_double(0x7ff8000000000000ll);
+  if (up) {
+    if (logZ_out) logZ_out[b] = nan;
+    ws.logz2[b] = nan;
+  } else {
+    ws.logz2b[b] = nan;
+  }
+}
+
+// ... and its posteriors are zero: the per-segment partials, the emission
+// gradient's suffix sums and the boundary marginals of the declined
+// sequences (every other sequence took the posterior pass).
+__global__ void declined_segment_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                                        float* __restrict__ grad_em, float* __restrict__ start_marg,
+                                        float* __restrict__ end_marg, float* __restrict__ seg_marg) {
+  const int j = blockIdx.x, b = blockIdx.y, C = d.C, K = d.K;
+  const int L = lengths[b];
+  if (L <= 0 || L > d.T || posterior_from_kept(ws, d, b)) return;
+  const int t0 = j * d.delta;
+  if (t0 >= L) return;
+  const int t1 = min(t0 + d.delta, L);
+  const size_t seg = (size_t)b * d.nck + j;
+  for (int i = threadIdx.x; i < K * C; i += blockDim.x) ws.pgd[seg * K * C + i] = 0.0;
+  for (int i = threadIdx.x; i < C * C; i += blockDim.x) ws.pgt[seg * C * C + i] = 0.0;
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    ws.segT[seg * C + i] = 0.0;
+    ws.segV[seg * C + i] = 0.0;
+  }
+  const int t_end = (t1 == L) ? L + 1 : t1;  // the last segment also clears boundary L
+  for (int i = threadIdx.x; i < (t1 - t0) * C; i += blockDim.x)
+    grad_em[((size_t)b * d.T + t0) * C + i] = 0.f;
+  for (int i = threadIdx.x; i < (t_end - t0) * C; i += blockDim.x) {
+    const size_t ob = ((size_t)b * (d.T + 1) + t0) * C + i;
+    if (start_marg) start_marg[ob] = 0.f;
+    if (end_marg) end_marg[ob] = 0.f;
+  }
+  if (seg_marg)
+    for (size_t i = threadIdx.x; i < (size_t)(t1 - t0) * K * C; i += blockDim.x)
+      seg_marg[((size_t)b * d.T + t0) * K * C + i] = 0.f;
+}
+
+}  // namespace
+
 cudaError_t launch_chain(const Dims& d, const WsPtrs& ws, const int32_t* lengths, const float* trans,
                          const float* dur, double* logZ_out, int n_alpha, int n_beta,
                          cudaStream_t st) {
+  if (d.KBT == 0) {  // long durations: no log-domain kernel
+    if (n_alpha + n_beta > 0)
+      declined_chain_kernel<<<n_alpha + n_beta, 32, 0, st>>>(d, ws, logZ_out, n_alpha);
+    return cudaGetLastError();
+  }
   const size_t sm = recursion_smem_bytes(d, false);
 #define SEMICRF_LAUNCH_CHAIN(a, b, g, lb)                                                    \
   if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \
@@ -833,6 +892,11 @@ cudaError_t launch_segment(const Dims& d, const WsPtrs& ws, const int32_t* lengt
                            const float* trans, const float* dur, const double* grad_logZ,
                            float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
                            float* seg_marg) {
+  if (d.KBT == 0) {  // long durations: zero the declined sequences' posteriors
+    declined_segment_kernel<<<dim3(d.nck, d.B), 256, 0, st>>>(d, ws, lengths, grad_em, start_marg,
+                                                               end_marg, seg_marg);
+    return cudaGetLastError();
+  }
   const size_t sm = recursion_smem_bytes(d, d.store_smem != 0);
 #define SEMICRF_LAUNCH_SEG(a, b, g, lb)                                                      \
   if (d.KBT == a && d.CAT == b && d.GB == g && d.LB == lb) {                                 \

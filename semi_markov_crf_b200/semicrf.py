@@ -129,7 +129,7 @@ def workspace_itemize(B: int, T: int, C: int, K: int, flags: int = 0) -> dict:
 SHAPE_FIELDS = ("ring_ctas", "labels_per_cta", "combine_lanes", "combine_weights",
                 "helper_lanes", "helper_durations", "ring_threads", "delta", "n_checkpoints",
                 "posterior_tile_rows", "log_durations_per_lane", "log_lanes_per_label",
-                "log_labels_per_lane", "log_threads")
+                "log_labels_per_lane", "log_threads", "posterior_halo_rows", "cut_grid_spacing")
 
 
 def launch_shape(B: int, T: int, C: int, K: int) -> dict:

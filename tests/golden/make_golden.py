@@ -28,7 +28,8 @@ last K + 2 rows of each sequence -- plus seeded random rows.  For wide label
 sets (C > 64) only the first and last sequence get the targeted rows.
 
 The tiny and speech workloads are not stored: the GPU tests run the oracle on
-them at test time (seconds) and compare every element.
+them at test time (seconds) and compare every element.  ``long_k`` is the
+long-duration case (B=2, T=20,000, K=8000, C=6), stored at every position.
 
 The GPU parity tests regenerate the same inputs, run the CUDA path at the
 benchmark's launch configuration and compare against these values, so the
@@ -51,7 +52,20 @@ sys.path.insert(0, ROOT)
 import oracle  # noqa: E402
 from semi_markov_crf_b200 import synth  # noqa: E402
 
-NAMES = ("genomic", "ultra", "large")
+NAMES = ("genomic", "ultra", "large", "long_k")
+
+
+def long_k_case():
+    """Long durations (the pages' genomic regime of K = 2000-8000): B=2,
+    T=20,000 (lengths 20,000 and 13,000), K=8000, C=6, the genomic label
+    frequencies with segments of mean length 500."""
+    return synth.make_custom(2, 20_000, 8000, 6, seed=43, lengths=[20_000, 13_000],
+                             dur_mean=500.0, amp=2.0,
+                             label_p=(0.6, 0.2, 0.1, 0.05, 0.03, 0.02))
+
+
+def workload(name: str):
+    return long_k_case() if name == "long_k" else synth.make(name)
 QSCALE = float(1 << 17)
 SMS = 148  # B200: the library's checkpoint cap depends on the SM count
 
@@ -105,7 +119,7 @@ def quantise(x):
 
 
 def make(name: str):
-    w = synth.make(name)
+    w = workload(name)
     K = w["dur"].shape[0]
     B, T, C = w["em"].shape
     t0 = time.time()
@@ -115,8 +129,13 @@ def make(name: str):
     # wide label sets: the state-change rows of the first and last sequence
     targeted = {0, B - 1} if C > 64 else set(range(B))
     n_random = 100 if C > 64 else 300
-    rb, ru, bb, bu = target_rows(w["lengths"], T, K, synth.CONFIGS[name].seed, n_random,
-                                 targeted)
+    seed = 43 if name == "long_k" else synth.CONFIGS[name].seed
+    if name == "long_k":  # every position
+        rb, ru = np.nonzero(np.arange(T)[None, :] < w["lengths"][:, None])
+        bb, bu = np.nonzero(np.arange(T + 1)[None, :] <= w["lengths"][:, None])
+        rb, ru, bb, bu = (x.astype(np.int32) for x in (rb, ru, bb, bu))
+    else:
+        rb, ru, bb, bu = target_rows(w["lengths"], T, K, seed, n_random, targeted)
     lab_dtype = np.int8 if C <= 127 else np.int16
     out = dict(
         logZ=fb["logZ"], logZ_beta=fb["logZ_beta"], grad_trans=fb["grad_trans"],

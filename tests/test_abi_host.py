@@ -47,20 +47,43 @@ def test_workspace_bytes_and_limits(lib):
     assert rc == 0 and n > 32 * 801 * 39 * 8  # at least the split prefix sums
     rc2, n2 = _ws_bytes(lib, 1, 1_000_000, 6, 200)
     assert rc2 == 0
-    # checkpoint memory grows like sqrt(T): 4x T -> about 2x checkpoint bytes
-    _, a = _ws_bytes(lib, 1, 100_000, 6, 200)
-    assert n2 < 12 * a
     assert _ws_bytes(lib, 1, 10, 129, 4)[0] == 2          # C above the limit
     assert _ws_bytes(lib, 1, 10, 128, 65)[0] == 2         # K above the limit for C=128
     assert _ws_bytes(lib, 1, 10, 16, 512)[0] == 0
     assert _ws_bytes(lib, 1, 10, 16, 513)[0] == 2
     assert _ws_bytes(lib, 1, 10, 8, 2048)[0] == 0          # long durations, few labels
-    assert _ws_bytes(lib, 1, 10, 8, 2049)[0] == 2
+    assert _ws_bytes(lib, 1, 10, 8, 8192)[0] == 0          # ... up to 8192 (pipelined kernels)
+    assert _ws_bytes(lib, 1, 10, 8, 8193)[0] == 2
     assert _ws_bytes(lib, 1, 10, 9, 1024)[0] == 2
+    assert _ws_bytes(lib, 1, 10, 9, 2049)[0] == 2
     assert _ws_bytes(lib, -1, 10, 4, 4)[0] == 1
     assert _ws_bytes(lib, 1, 10, 0, 4)[0] == 1
     assert _ws_bytes(lib, 1, 10, 4, 4, flags=0x80)[0] == 1
     assert lib.semicrf_workspace_bytes(1, 10, 4, 4, ctypes.c_uint(0), None) == 1
+
+
+def _groups(B, T, C, K):
+    from semi_markov_crf_b200 import semicrf
+    return semicrf.workspace_itemize(B, T, C, K)
+
+
+def test_workspace_groups_add_up_and_scale_as_designed(lib):
+    """Where the workspace goes, from semicrf_workspace_itemize: the groups
+    add up to semicrf_workspace_bytes; the checkpoints of the log-domain
+    walk grow like the number of checkpoint segments (their K x C rings,
+    about sqrt(T) of them at the pages' spacing) while the per-position
+    arrays (prefix sums, kept ring rows, decoder rows) grow like T."""
+    for B, T, C, K in ((32, 800, 39, 30), (1, 1_000_000, 6, 200), (8, 10_000, 128, 64)):
+        g = _groups(B, T, C, K)
+        assert sum(g.values()) == _ws_bytes(lib, B, T, C, K)[1]
+        assert g["prefix_sums"] >= B * (T + 1) * C * 8
+    small, big = _groups(1, 250_000, 6, 200), _groups(1, 1_000_000, 6, 200)
+    for key in ("prefix_sums", "kept_rows", "viterbi"):      # O(T C)
+        assert 3.9 < big[key] / small[key] < 4.1, key
+    # checkpoints: one K x C ring pair per segment; segments grow more slowly
+    # than T (sqrt(T K), capped for one wave of the posterior pass)
+    assert big["checkpoints"] / small["checkpoints"] < 3.0
+    assert big["checkpoints"] < big["prefix_sums"] / 4
 
 
 def test_host_side_argument_errors_launch_nothing(lib):
@@ -103,7 +126,7 @@ def test_host_side_argument_errors_of_the_loss_and_projection_calls(lib):
     # projection entry points: null inputs, unsupported sizes, misaligned workspace
     assert lib.semicrf_forward_proj(None, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0, fake, big,
                                     fake, None) == 1
-    assert lib.semicrf_forward_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 4000, u0, fake,
+    assert lib.semicrf_forward_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 9000, u0, fake,
                                     big, fake, None) == 2
     assert lib.semicrf_forward_proj(fake, fake, fake, fake, fake, fake, 1, 8, 2, 2, u0,
                                     vp(256 * 1024 + 8), big, fake, None) == 1

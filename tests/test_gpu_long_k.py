@@ -4,16 +4,18 @@ These sizes run on the exponential-domain rings and the pipelined decoder,
 one label per CTA of a thread-block cluster, with the posterior pass staging
 the segment ends in chunks and the cut normaliser label by label.
 
-- K = 8000, C = 6, T = 20,000 (lengths 20,000 and 13,000) against the
-  float64 oracle at every position (tests/golden/long_k.npz): log Z,
+- K = 8000, C = 6, T = 6,000 (lengths 6,000 and 4,500: segments up to the
+  whole sequence) against the float64 oracle at every position
+  (tests/golden/long_k.npz; the oracle's explicit covering sums make larger
+  T a matter of hours): log Z,
   marginals, emission gradients, transition and duration gradients, and the
   decoded path (bit-exact except at ties of the model).
 - K = 3000 at C = 1 and C = 3 (one CTA, and a cluster of three) against the
   oracle computed now.
 - T = 10^6, K = 8000, C = 6: the any-size invariants.
-- A sequence outside the exponent range (a forbidden transition) is reported
-  as unsupported (status 2, log Z NaN, zero posteriors) next to a normal one;
-  forcing the log domain is refused on the host.
+- A sequence outside the exponent range is reported as unsupported (status
+  2, log Z NaN, zero posteriors) next to a normal one, which still matches
+  the oracle; forcing the log domain is refused on the host.
 """
 
 import os
@@ -34,7 +36,7 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "lon
 
 
 def _long_k_case():
-    return synth.make_custom(2, 20_000, 8000, 6, seed=43, lengths=[20_000, 13_000],
+    return synth.make_custom(2, 6_000, 8000, 6, seed=43, lengths=[6_000, 4_500],
                              dur_mean=500.0, amp=2.0, label_p=(0.6, 0.2, 0.1, 0.05, 0.03, 0.02))
 
 
@@ -75,7 +77,7 @@ def test_k8000_matches_the_oracle_everywhere():
 
 @pytest.mark.parametrize("C,n", [(1, 1), (3, 3)])
 def test_k3000_small_label_sets_match_oracle(C, n):
-    case = synth.make_custom(2, 4000, 3000, C, seed=44 + C, lengths=[4000, 2600],
+    case = synth.make_custom(2, 3200, 3000, C, seed=44 + C, lengths=[3200, 2100],
                              dur_mean=400.0, amp=2.0)
     B, T, _ = case["em"].shape
     K = case["dur"].shape[0]
@@ -111,20 +113,27 @@ def test_k8000_million_positions_invariants():
     assert abs(resc[0] - vit["score"][0]) <= 1e-8 * abs(resc[0]), (resc[0], vit["score"][0])
 
 
-def test_k8000_outside_the_exponent_range_is_reported():
+def test_k4000_outside_the_exponent_range_is_reported():
+    """Sequence 1's emissions are scaled far outside the exponential-domain
+    rings' head-room: it is reported (status 2, log Z NaN, zero posteriors)
+    while sequence 0 is computed as usual."""
     case = synth.make_custom(2, 3000, 4000, 4, seed=46, dur_mean=300.0, amp=2.0)
-    case["trans"][1, 2] = -np.inf          # both sequences leave the exponent range
-    ok = synth.make_custom(2, 3000, 4000, 4, seed=46, dur_mean=300.0, amp=2.0)
+    case["em"][1] *= 60.0
+    K = case["dur"].shape[0]
     em, lengths, trans, dur = to_dev(case)
     logZ, ws = semicrf.forward(em, lengths, trans, dur)
     out = semicrf.backward(ws, lengths, trans, dur, marginals=True)
     assert semicrf.get_status(ws) == 2
-    assert np.all(np.isnan(logZ.cpu().numpy()))
-    for k in ("grad_em", "pos_marg", "start_marg", "end_marg", "grad_trans", "grad_dur"):
-        assert torch.count_nonzero(out[k]) == 0, k
+    assert semicrf.ring_domains(ws) == [1, 2, 1, 2]
+    lz = logZ.cpu().numpy()
+    assert np.isnan(lz[1]) and np.isfinite(lz[0])
+    for k in ("grad_em", "pos_marg", "start_marg", "end_marg"):
+        assert torch.count_nonzero(out[k][1]) == 0, k
+    one = dict(case, em=case["em"][:1], lengths=case["lengths"][:1])
+    ref = oracle.forward_backward(one["em"], one["lengths"], case["trans"], case["dur"], K)
+    got = {k: v[:1].cpu().numpy() if v.dim() == 3 else v.cpu().numpy() for k, v in out.items()}
+    got["logZ"] = lz[:1]
+    assert_fb_close(got, ref, one["lengths"], "K=4000 with a declined sequence")
     with pytest.raises(semicrf.SemiCRFError) as info:
-        semicrf.forward(*to_dev(ok), log_domain=True)
+        semicrf.forward(em, lengths, trans, dur, log_domain=True)
     assert info.value.code == 2
-    # the same sizes inside the range run
-    got = gpu_fb(ok)
-    assert got["status"] == 0 and np.isfinite(got["logZ"]).all()

@@ -405,13 +405,25 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
         int r_end = min(s_hi, L - k + 1) - s_lo;
         if (!SEMICRF_INB(ws.status, r_end <= 0 || r_end - 1 + k - base < nst, SITE_POST_ITEM))
           r_end = 0;
-        float a_ = 0.f;
-        for (int r = 0; r < r_end; ++r) {
+        // two accumulators and an unrolled loop: independent terms overlap
+        // their shared-memory loads and exponentials
+        float a0 = 0.f, a1 = 0.f;
+        int r = 0;
+#pragma unroll 2
+        for (; r + 1 < r_end; r += 2) {
+          const int o = r * C + c, ok = (r + k - base) * C + c;
+          const float z0 = (float)(tl.ii[ok] - tl.tii[o]) + (dk + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
+          const float z1 = (float)(tl.ii[ok + C] - tl.tii[o + C]) +
+                           (dk + ((tl.sf[ok + C] - tl.tsf[o + C]) + tl.pd[o + C]));
+          a0 = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z0), a0);
+          a1 = fmaf(tl.tf[(r + 1) * 2 * C + C + c] * tl.ab[ok + C], tl.fs[r + 1] * ex2(z1), a1);
+        }
+        if (r < r_end) {
           const int o = r * C + c, ok = (r + k - base) * C + c;
           const float z = (float)(tl.ii[ok] - tl.tii[o]) + (dk + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
-          a_ = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a_);
+          a0 = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a0);
         }
-        return a_;
+        return a0 + a1;
       };
 #pragma unroll
       for (int m = 0; m < NID; ++m) {
@@ -428,9 +440,15 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
     // item (c', c): sum over the tile's s of P(c' -> c at s) / w[c', c]
     auto tr_item = [&](int idx) {
       const int c1 = idx / C, c = idx - c1 * C;
-      float a_ = 0.f;
-      for (int r = 0; r < nr; ++r) a_ = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a_);
-      return a_;
+      float a0 = 0.f, a1 = 0.f;
+      int r = 0;
+#pragma unroll 4
+      for (; r + 1 < nr; r += 2) {
+        a0 = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a0);
+        a1 = fmaf(tl.tf[(r + 1) * 2 * C + c1] * tl.fs[r + 1], tl.pb[(r + 1) * C + c], a1);
+      }
+      if (r < nr) a0 = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a0);
+      return a0 + a1;
     };
 #pragma unroll
     for (int m = 0; m < NIT; ++m)

@@ -215,7 +215,6 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Shared memory of cut_grid_kernel.
 // Shared memory of cut_grid_kernel: every label's rows when they fit the
 // budget, else one label's (cut_grid_per_label).
 bool cut_grid_per_label(const Dims& d, size_t budget) {
@@ -227,50 +226,78 @@ size_t cut_grid_smem_bytes(const Dims& d, size_t budget) {
 
 namespace {
 
-// Shared memory carve of posterior_kernel for a tile of RT boundaries.
-// (With boundary projections pd holds the start terms of the tile's rows.)
-// Segment ends: a tile's segments end on up to RT + K rows.  Those rows are
-// staged KH at a time (KH = K: all at once; long durations: chunks of the
-// duration range, each staging RT + KH rows), so the halo arrays hold
-// R = RT + KH rows and, when chunked, the tile rows' own integer and
-// fractional prefix sums have arrays of their own (tii, tsf).
+// Shared memory of posterior_kernel for a tile of RT boundaries (Cp = C
+// rounded up to a multiple of 4, R = RT + KH staged segment-end rows).
+//
+// Every duration term is one power of two,
+//   P([s, s+k), c) = 2^(Y[s+k, c] - X[s, c] + dur2'[k-1, c])        (dur2' = M + dur2)
+//   Y[t, c] = I[t, c] + S_frac[t, c] + log2 ab[t, c]                 (end side)
+//   X[s, c] = I[s, c] + S_frac[s, c] - pd[s, c] - log2 af[s, c] - log2 f_s   (start side)
+// with I[t, c] = (Pb_t - Pb_lo) + S_int[t, c] the exact integer part of the
+// prefix sum.  Both sides are stored split into an integer (held exactly in a
+// float: the integers are taken relative to the tile's first row, so they
+// stay far below 2^24) and a fraction in [-1/2, 1/2], so the large values
+// only ever meet as an exact integer difference.  A side whose kept value is
+// zero is stored as an infinite integer part (its terms are 0).
 struct PTile {
+  float* pa;    // [RT][Cp]  forward p of the tile rows times f_s (transition items)
+  float* pbt;   // [RT][Cp]  backward p of the tile rows (transition items)
   double* dif;  // [RT][C]   St - E of each boundary and label
-  float* tf;    // [RT][2C]  forward kept rows: p, acc
-  float* pb;    // [RT][C]   backward p
-  float* ab;    // [R][C]    backward acc of the staged segment-end rows
-  int* ii;      // [R][C]    (Pb_r - Pb_lo) + S_int[r, c], exact integers
-  float* sf;    // [R][C]    S_frac[r, c]
-  float* vv;    // [RT][C]   suffix sums v of the tile
+  float* xi;    // [RT][C]   start side X: integer part
+  float* xf;    // [RT][C]   start side X: fraction
+  float* yi;    // [R][C]    end side Y of the staged rows: integer part
+  float* yf;    // [R][C]    end side Y: fraction
+  int* li;      // [RT]      log2 f_s: integer part
+  float* lf;    // [RT]      log2 f_s: remainder
   float* fs;    // [RT]      f_s
-  float* pd;    // [RT][C]   projection start terms of the tile's rows (0 without)
-  int* tii;     // [RT][C]   ii of the tile rows (aliases ii when not chunked)
-  float* tsf;   // [RT][C]   sf of the tile rows (aliases sf when not chunked)
 };
-__host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int KH, int C, bool chunked) {
+__host__ __device__ __forceinline__ int pad4(int C) { return (C + 3) & ~3; }
+__host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int KH, int C) {
   const size_t R = (size_t)RT + KH;
-  return (size_t)C * (28ull * RT + 12ull * R + (chunked ? 8ull * RT : 0)) + 4ull * RT;
+  return 8ull * RT * pad4(C) + 16ull * RT * C + 8ull * R * C + 12ull * RT;
 }
-__device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH, int C,
-                                             bool chunked) {
+__device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH, int C) {
   PTile t;
-  const size_t R = (size_t)RT + KH;
-  t.dif = reinterpret_cast<double*>(raw);
-  t.tf = reinterpret_cast<float*>(t.dif + (size_t)RT * C);
-  t.pb = t.tf + (size_t)RT * 2 * C;
-  t.ab = t.pb + (size_t)RT * C;
-  t.ii = reinterpret_cast<int*>(t.ab + R * C);
-  t.sf = reinterpret_cast<float*>(t.ii + R * C);
-  t.vv = t.sf + R * C;
-  t.fs = t.vv + (size_t)RT * C;
-  t.pd = t.fs + RT;
-  t.tii = t.ii;
-  t.tsf = t.sf;
-  if (chunked) {
-    t.tii = reinterpret_cast<int*>(t.pd + (size_t)RT * C);
-    t.tsf = reinterpret_cast<float*>(t.tii + (size_t)RT * C);
-  }
+  const size_t R = (size_t)RT + KH, Cp = pad4(C);
+  t.pa = reinterpret_cast<float*>(raw);  // 16-byte aligned: read as float4
+  t.pbt = t.pa + RT * Cp;
+  t.dif = reinterpret_cast<double*>(t.pbt + RT * Cp);
+  t.xi = reinterpret_cast<float*>(t.dif + (size_t)RT * C);
+  t.xf = t.xi + (size_t)RT * C;
+  t.yi = t.xf + (size_t)RT * C;
+  t.yf = t.yi + R * C;
+  t.li = reinterpret_cast<int*>(t.yf + R * C);
+  t.lf = reinterpret_cast<float*>(t.li + RT);
+  t.fs = t.lf + RT;
   return t;
+}
+
+// log2 that keeps subnormal inputs (the ftz form would send them to -inf)
+__device__ __forceinline__ float lg2_sub(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Split v into an integer (added to the exact integer base ib) and a
+// fraction in [-1/2, 1/2] and store both; a value too large to split (an
+// infinite side: a kept value of 0) is stored whole as the integer part.
+__device__ __forceinline__ void split_store(float v, int ib, float* pi, float* pf) {
+  if (fabsf(v) < 1e7f) {
+    const float n = rintf(v);
+    *pi = (float)(ib + (int)n);
+    *pf = v - n;
+  } else {
+    *pi = v;
+    *pf = 0.f;
+  }
+}
+
+// The kernel variant: two CTAs per SM (one quad and one transition block per
+// thread) when the items fit that, else one.
+inline bool posterior_pair(const Dims& d) {
+  const long long nq = (long long)((d.K + 3) / 4) * d.C, nbk = pad4(d.C) / 4;
+  return nq <= 512 && nbk * nbk <= 512;
 }
 
 // One CTA per (checkpoint segment j, sequence b): every posterior whose start
@@ -281,16 +308,21 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH,
 // running sum over segments), because the normaliser is continuous.
 //
 // The segment is cut into tiles of d.pRT boundaries, taken downwards (the
-// suffix sums run that way).  A tile stages its kept rows, and the K rows
-// after it that its segments end on, in shared memory with coalesced loads;
-// then every (boundary, label), (duration, label) and (label, label) item is
-// computed from shared memory.  Each thread keeps the duration and transition
-// sums of its first NID / NIT items in registers across tiles (with 512
-// threads that covers K C <= 8192 and C <= 128); the items beyond (long
-// durations: K C up to 16384) add their per-tile sums to the float64
-// partials.
-template <int NID, int NIT>
-__global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
+// suffix sums run that way).  A tile stages, with coalesced loads, its start
+// sides X and its transition operands, and the end sides Y of the rows its
+// segments end on (KH rows at a time: all K at once, or chunks of the
+// duration range for long durations).  Then:
+//   duration counts -- a thread owns quads (4 consecutive durations, one
+//     label) and slides a 4-row window of Y down the tile's starts: per term
+//     one exponential and four adds, one new Y row per start;
+//   transition counts -- sum over s of pa[s, c'] pb[s, c], a rank-RT update
+//     of a C x C matrix, in 4 x 4 register blocks;
+//   suffix sums -- one thread per label, running up the tile.
+// Each thread keeps its first NQ quads and NB blocks in registers across
+// tiles (512 threads: K C <= 8192, C <= 128); the quads beyond (long
+// durations) add per-tile sums to the float64 partials.
+template <int NQ, int NB>
+__global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
     posterior_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                      const float* __restrict__ trans, const float* __restrict__ dur,
                      const double* __restrict__ grad_logZ, float* __restrict__ grad_em,
@@ -298,8 +330,8 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
                      float* __restrict__ seg_marg, int pj) {
   extern __shared__ __align__(16) unsigned char psh[];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
-  const int C = d.C, K = d.K, RT = d.pRT, KH = d.pKH;
-  const bool chunked = KH < K;  // long durations: the segment ends come KH rows at a time
+  const int C = d.C, K = d.K, RT = d.pRT, KH = d.pKH, Cp = pad4(C);
+  [[maybe_unused]] const int R = RT + KH;  // staged rows (bounds-check build)
   const int L = lengths[b];
   if (L <= 0 || L > d.T) return;
   if (!posterior_from_kept(ws, d, b)) return;  // segment_kernel runs it
@@ -309,7 +341,7 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
   const size_t seg = (size_t)b * d.nck + j;
   const float gb = (float)(grad_logZ ? grad_logZ[b] : 1.0);
   const float M = *ws.tmax;  // max trans2, written by the rings
-  const PTile tl = ptile_carve(psh, RT, KH, C, chunked);
+  const PTile tl = ptile_carve(psh, RT, KH, C);
   const float* pfr = kv_row(ws, d, b, 0, 0);  // row t: pfr + t*2C (p), + C (acc)
   const float* pbr = kv_row(ws, d, b, 1, 0);
   const double* kff = ws.kf + ((size_t)b * 2 + 0) * (d.T + 1);
@@ -318,38 +350,65 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
   const int32_t* si = ws.sint + (size_t)b * d.Tstride * C;
   const float* sfp = ws.sfrac + (size_t)b * d.Tstride * C;
   const int nd = K * C, ntr = C * C;
-  float accd[NID], acct[NIT];
+  const int nq = ((K + 3) >> 2) * C;  // quads
+  const int nbk = Cp >> 2, nblk = nbk * nbk;
+  float accq[NQ][4], acct[NB][16];
 #pragma unroll
-  for (int m = 0; m < NID; ++m) accd[m] = 0.f;
+  for (int m = 0; m < NQ; ++m)
 #pragma unroll
-  for (int m = 0; m < NIT; ++m) acct[m] = 0.f;
+    for (int u = 0; u < 4; ++u) accq[m][u] = 0.f;
+#pragma unroll
+  for (int m = 0; m < NB; ++m)
+#pragma unroll
+    for (int u = 0; u < 16; ++u) acct[m][u] = 0.f;
   double lacc = 0.0, lvs = 0.0;  // thread c < C: running suffix sum, sum of v
 
   for (int s_hi = t1; s_hi > t0; s_hi -= RT) {
     const int s_lo = max(t0, s_hi - RT);
     const int nr = s_hi - s_lo;
+    const int Lr = L - s_lo;                         // a segment [s_lo + r, s_lo + r + k) needs r + k <= Lr
     const int nh = min(s_hi - 1 + K, L) - s_lo + 1;  // rows a segment of the tile ends on
     const bool first = (s_hi == t1);
     // bounds-check build: the tile fits its rows
     if (!SEMICRF_INB(ws.status, nr >= 1 && nr <= RT && nh <= RT + K, SITE_POST_TILE)) break;
-    // ------------------------------------------------------------ stage the tile rows
     const double kb0 = kfb[s_lo];
-    #pragma unroll 4
-    for (int i = tid; i < nr * 2 * C; i += nthr) tl.tf[i] = pfr[(size_t)s_lo * 2 * C + i];
-    #pragma unroll 4
-    for (int i = tid; i < nr * C; i += nthr) {
-      const int r = i / C, c = i - r * C;
-      const size_t row = (size_t)(s_lo + r);
-      tl.pb[i] = pbr[row * 2 * C + c];
-      tl.pd[i] = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
-      if (chunked) {
-        tl.tii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
-        tl.tsf[i] = sfp[row * C + c];
-      }
+    // ------------------------------------------------------------ f_s of the tile rows
+    // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s)), also split for the start sides
+    for (int r = tid; r < nr; r += nthr) {
+      const int s = s_lo + r;
+      const double l = ((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1));
+      const double n = fabs(l) < 1e9 ? rint(l) : 0.0;
+      tl.li[r] = (int)n;
+      tl.lf[r] = (float)(l - n);
+      tl.fs[r] = ex2((float)l);
     }
-    // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s))
-    for (int s = s_lo + tid; s < s_hi; s += nthr)
-      tl.fs[s - s_lo] = ex2((float)(((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1))));
+    __syncthreads();
+    // ------------------------------------------------------------ stage the tile rows
+    // start / end marginals and St - E; transition operands; start sides X
+    for (int i = tid; i < nr * Cp; i += nthr) {
+      const int r = i / Cp, c = i - r * Cp;
+      if (c >= C) {
+        tl.pa[i] = 0.f;
+        tl.pbt[i] = 0.f;
+        continue;
+      }
+      const size_t row = (size_t)(s_lo + r);
+      const float f = tl.fs[r];
+      const float tp = pfr[row * 2 * C + c], ta = pfr[row * 2 * C + C + c];
+      const float bp = pbr[row * 2 * C + c], ba = pbr[row * 2 * C + C + c];
+      const float St = ta * bp * f, E = ba * tp * f;
+      const size_t ob = ((size_t)b * (d.T + 1) + row) * C + c;
+      if (start_marg) start_marg[ob] = St;
+      if (end_marg) end_marg[ob] = E;
+      const int o = r * C + c;
+      tl.dif[o] = (double)St - (double)E;
+      tl.pa[i] = tp * f;
+      tl.pbt[i] = bp;
+      const float pdv = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
+      const int ib = (int)(kfb[row] - kb0) + (si[row * C + c] - si[(size_t)s_lo * C + c]);
+      split_store((sfp[row * C + c] - pdv) - (lg2_sub(ta) + tl.lf[r]), ib - tl.li[r], tl.xi + o,
+                  tl.xf + o);
+    }
     // ------------------------------------------------------------ segment ends, by chunk
     // chunk kc: durations [kc, kc + KH), staged rows at offsets [kc - 1, kc - 1 + nr + KH)
     // from s_lo (the first chunk includes the tile rows themselves)
@@ -357,128 +416,174 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
       const int base = kc - 1;
       const int nst = max(0, min(base + nr + KH, nh) - base);
       if (kc > 1) __syncthreads();  // the previous chunk's reads are done
-      #pragma unroll 4
       for (int i = tid; i < nst * C; i += nthr) {
         const int r = i / C, c = i - r * C;
         const size_t row = (size_t)(s_lo + base + r);
-        tl.ab[i] = pbr[row * 2 * C + C + c];
-        tl.ii[i] = (int)(kfb[row] - kb0) + si[row * C + c];
-        tl.sf[i] = sfp[row * C + c];
+        const int ib = (int)(kfb[row] - kb0) + (si[row * C + c] - si[(size_t)s_lo * C + c]);
+        split_store(sfp[row * C + c] + lg2_sub(pbr[row * 2 * C + C + c]), ib, tl.yi + i, tl.yf + i);
       }
       __syncthreads();
-      if (kc == 1) {
-        // ---------------------------------------------------------- start / end marginals
-        for (int i = tid; i < nr * C; i += nthr) {
-          const int r = i / C, c = i - r * C;
-          const float f = tl.fs[r];
-          const float St = tl.tf[r * 2 * C + C + c] * tl.pb[i] * f;
-          const float E = tl.ab[i] * tl.tf[r * 2 * C + c] * f;
-          const size_t ob = ((size_t)b * (d.T + 1) + s_lo + r) * C + c;
-          if (start_marg) start_marg[ob] = St;
-          if (end_marg) end_marg[ob] = E;
-          tl.dif[i] = (double)St - (double)E;
-        }
-      }
-      const int lo_i = base * C, hi_i = min(nd, (base + KH) * C);  // this chunk's (k, c) items
       // -------------------------------------------------------- segment marginals
-      // (optional output) P([s, s+k), c) for every start of the tile, the same
-      // product as the duration counts below, not scaled by g (a marginal)
+      // (optional output) P([s, s+k), c) for every start of the tile and
+      // every duration of the chunk, not scaled by g (a marginal)
       if (seg_marg) {
-        const int nci = hi_i - lo_i;
+        const int lo_i = base * C, nci = min(nd, (base + KH) * C) - lo_i;
         for (int i = tid; i < nr * nci; i += nthr) {
           const int r = i / nci, idx = lo_i + (i - r * nci);
           const int k = idx / C + 1, c = idx - (k - 1) * C;
-          if (s_lo + r + k > L) continue;
+          if (r + k > Lr) continue;
           if (!SEMICRF_INB(ws.status, r + k - base < nst, SITE_POST_ITEM)) continue;
           const int o = r * C + c, ok = (r + k - base) * C + c;
-          const float z = (float)(tl.ii[ok] - tl.tii[o]) +
-                          ((M + __ldg(dur + idx) * l2e()) + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
-          seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] =
-              tl.tf[r * 2 * C + C + c] * tl.ab[ok] * (tl.fs[r] * ex2(z));
+          const float z = (tl.yi[ok] - tl.xi[o]) +
+                          ((tl.yf[ok] - tl.xf[o]) + (M + __ldg(dur + idx) * l2e()));
+          seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] = ex2(z);
         }
       }
       // -------------------------------------------------------- duration counts
-      // item (k, c): sum over the tile's s of P([s, s+k), c), s + k <= L
-      auto dur_item = [&](int idx) {
-        const int k = idx / C + 1, c = idx - (k - 1) * C;
-        const float dk = M + __ldg(dur + idx) * l2e();
-        int r_end = min(s_hi, L - k + 1) - s_lo;
-        if (!SEMICRF_INB(ws.status, r_end <= 0 || r_end - 1 + k - base < nst, SITE_POST_ITEM))
-          r_end = 0;
-        // two accumulators and an unrolled loop: independent terms overlap
-        // their shared-memory loads and exponentials
-        float a0 = 0.f, a1 = 0.f;
+      // quad q = (kq, c): durations k0 .. k0 + 3 (k0 = 4 kq + 1) of label c, each
+      // summed over the tile's starts r with r + k <= Lr
+      const int q_lo = (base >> 2) * C, q_hi = min(nq, ((base + KH + 3) >> 2) * C);
+      auto quad = [&](int q, float (&a)[4]) {
+        const int kq = q / C, c = q - kq * C, k0 = 4 * kq + 1;
+        float dk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          dk[u] = (k0 + u <= K) ? M + __ldg(dur + (k0 + u - 1) * C + c) * l2e() : -INFINITY;
+        const int h0 = k0 - base;  // staged row of (r = 0, u = 0)
+        const int r_all = max(0, min(nr, Lr - (k0 + 3) + 1));  // every k0 + u valid
+        const int r_any = max(0, min(nr, Lr - k0 + 1));        // k0 valid
+        // bounds-check build: the window stays in the staged rows
+        if (!SEMICRF_INB(ws.status, h0 >= 1 && h0 + nr + 2 < R &&
+                                        (r_any == 0 || r_any - 1 + k0 - base < nst),
+                         SITE_POST_ITEM))
+          return;
+        const float* yi = tl.yi + c;
+        const float* yf = tl.yf + c;
+        float w0i = yi[h0 * C], w0f = yf[h0 * C];
+        float w1i = yi[(h0 + 1) * C], w1f = yf[(h0 + 1) * C];
+        float w2i = yi[(h0 + 2) * C], w2f = yf[(h0 + 2) * C];
         int r = 0;
-#pragma unroll 2
-        for (; r + 1 < r_end; r += 2) {
-          const int o = r * C + c, ok = (r + k - base) * C + c;
-          const float z0 = (float)(tl.ii[ok] - tl.tii[o]) + (dk + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
-          const float z1 = (float)(tl.ii[ok + C] - tl.tii[o + C]) +
-                           (dk + ((tl.sf[ok + C] - tl.tsf[o + C]) + tl.pd[o + C]));
-          a0 = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z0), a0);
-          a1 = fmaf(tl.tf[(r + 1) * 2 * C + C + c] * tl.ab[ok + C], tl.fs[r + 1] * ex2(z1), a1);
+#pragma unroll 4
+        for (; r < r_all; ++r) {
+          const int h3 = (h0 + r + 3) * C;
+          const float w3i = yi[h3], w3f = yf[h3];
+          const float oi = tl.xi[r * C + c], of = tl.xf[r * C + c];
+          a[0] += ex2((w0i - oi) + ((w0f - of) + dk[0]));
+          a[1] += ex2((w1i - oi) + ((w1f - of) + dk[1]));
+          a[2] += ex2((w2i - oi) + ((w2f - of) + dk[2]));
+          a[3] += ex2((w3i - oi) + ((w3f - of) + dk[3]));
+          w0i = w1i; w0f = w1f;
+          w1i = w2i; w1f = w2f;
+          w2i = w3i; w2f = w3f;
         }
-        if (r < r_end) {
-          const int o = r * C + c, ok = (r + k - base) * C + c;
-          const float z = (float)(tl.ii[ok] - tl.tii[o]) + (dk + ((tl.sf[ok] - tl.tsf[o]) + tl.pd[o]));
-          a0 = fmaf(tl.tf[r * 2 * C + C + c] * tl.ab[ok], tl.fs[r] * ex2(z), a0);
+        // the last starts of a sequence: the longer durations run past L
+        for (; r < r_any; ++r) {
+          const float oi = tl.xi[r * C + c], of = tl.xf[r * C + c];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (r + k0 + u > Lr) break;
+            const int h = (h0 + r + u) * C;
+            a[u] += ex2((yi[h] - oi) + ((yf[h] - of) + dk[u]));
+          }
         }
-        return a0 + a1;
       };
 #pragma unroll
-      for (int m = 0; m < NID; ++m) {
-        const int idx = tid + m * nthr;
-        if (idx >= lo_i && idx < hi_i) accd[m] += dur_item(idx);
+      for (int m = 0; m < NQ; ++m) {
+        const int q = tid + m * nthr;
+        if (q >= q_lo && q < q_hi) quad(q, accq[m]);
       }
-      for (int idx = tid + NID * nthr; idx < hi_i; idx += nthr) {
-        if (idx < lo_i) continue;
-        double* pd = ws.pgd + seg * nd + idx;
-        const double v = (double)(gb * dur_item(idx));
-        *pd = first ? v : *pd + v;
+      for (int q = tid + NQ * nthr; q < q_hi; q += nthr) {
+        if (q < q_lo) continue;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        quad(q, a);
+        const int kq = q / C, c = q - kq * C;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = 4 * kq + 1 + u;
+          if (k > K) break;
+          double* pd = ws.pgd + seg * nd + (size_t)(k - 1) * C + c;
+          const double v = (double)(gb * a[u]);
+          *pd = first ? v : *pd + v;
+        }
       }
     }
-    // item (c', c): sum over the tile's s of P(c' -> c at s) / w[c', c]
-    auto tr_item = [&](int idx) {
-      const int c1 = idx / C, c = idx - c1 * C;
-      float a0 = 0.f, a1 = 0.f;
-      int r = 0;
-#pragma unroll 4
-      for (; r + 1 < nr; r += 2) {
-        a0 = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a0);
-        a1 = fmaf(tl.tf[(r + 1) * 2 * C + c1] * tl.fs[r + 1], tl.pb[(r + 1) * C + c], a1);
+    // ------------------------------------------------------------ transition counts
+    // block (bi, bj): labels c' in 4 bi .. 4 bi + 3, c in 4 bj .. 4 bj + 3
+    auto tblock = [&](int q, float (&a)[16]) {
+      const int bi = q / nbk, bj = q - bi * nbk;
+      const float4* pa4 = reinterpret_cast<const float4*>(tl.pa) + bi;
+      const float4* pb4 = reinterpret_cast<const float4*>(tl.pbt) + bj;
+#pragma unroll 2
+      for (int r = 0; r < nr; ++r) {
+        const float4 x = pa4[r * nbk], y = pb4[r * nbk];
+        const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) a[u * 4 + v] = fmaf(xs[u], ys[v], a[u * 4 + v]);
       }
-      if (r < nr) a0 = fmaf(tl.tf[r * 2 * C + c1] * tl.fs[r], tl.pb[r * C + c], a0);
-      return a0 + a1;
+    };
+    auto tblock_out = [&](int q, const float (&a)[16], bool to_partials) {
+      const int bi = q / nbk, bj = q - bi * nbk;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int c1 = 4 * bi + u, c = 4 * bj + v;
+          if (c1 >= C || c >= C) continue;
+          const int idx = c1 * C + c;
+          const double val = (double)(gb * a[u * 4 + v] * ex2(__ldg(trans + idx) * l2e() - M));
+          double* pt = ws.pgt + seg * ntr + idx;
+          *pt = (to_partials && !first) ? *pt + val : val;
+        }
     };
 #pragma unroll
-    for (int m = 0; m < NIT; ++m)
-      if (tid + m * nthr < ntr) acct[m] += tr_item(tid + m * nthr);
-    for (int idx = tid + NIT * nthr; idx < ntr; idx += nthr) {
-      double* pt = ws.pgt + seg * ntr + idx;
-      const double v = (double)(gb * tr_item(idx) * ex2(__ldg(trans + idx) * l2e() - M));
-      *pt = first ? v : *pt + v;
+    for (int m = 0; m < NB; ++m)
+      if (tid + m * nthr < nblk) tblock(tid + m * nthr, acct[m]);
+    for (int q = tid + NB * nthr; q < nblk; q += nthr) {
+      float a[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) a[u] = 0.f;
+      tblock(q, a);
+      tblock_out(q, a, true);
     }
-    __syncthreads();
     // ------------------------------------------------------------ suffix sums
     // v[s] = sum of (St - E) over the segment's boundaries after s
     if (tid < C) {
       for (int r = nr - 1; r >= 0; --r) {
-        tl.vv[r * C + tid] = (float)lacc;
+        grad_em[((size_t)b * d.T + s_lo + r) * C + tid] = (float)lacc;
         lvs += (double)(float)lacc;
         lacc += tl.dif[r * C + tid];
       }
     }
-    __syncthreads();
-    for (int i = tid; i < nr * C; i += nthr) grad_em[((size_t)b * d.T + s_lo) * C + i] = tl.vv[i];
+    __syncthreads();  // the next tile overwrites the staged rows
   }
   // register items: the segment's partials
 #pragma unroll
-  for (int m = 0; m < NID; ++m)
-    if (tid + m * nthr < nd) ws.pgd[seg * nd + tid + m * nthr] = (double)(gb * accd[m]);
+  for (int m = 0; m < NQ; ++m) {
+    const int q = tid + m * nthr;
+    if (q >= nq) continue;
+    const int kq = q / C, c = q - kq * C;
 #pragma unroll
-  for (int m = 0; m < NIT; ++m) {
-    const int idx = tid + m * nthr;
-    if (idx < ntr) ws.pgt[seg * ntr + idx] = (double)(gb * acct[m] * ex2(__ldg(trans + idx) * l2e() - M));
+    for (int u = 0; u < 4; ++u) {
+      const int k = 4 * kq + 1 + u;
+      if (k <= K) ws.pgd[seg * nd + (size_t)(k - 1) * C + c] = (double)(gb * accq[m][u]);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NB; ++m) {
+    const int q = tid + m * nthr;
+    if (q >= nblk) continue;
+    const int bi = q / nbk, bj = q - bi * nbk;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int c1 = 4 * bi + u, c = 4 * bj + v;
+        if (c1 < C && c < C)
+          ws.pgt[seg * ntr + c1 * C + c] =
+              (double)(gb * acct[m][u * 4 + v] * ex2(__ldg(trans + c1 * C + c) * l2e() - M));
+      }
   }
   if (tid < C) {
     ws.segT[seg * C + tid] = lacc;
@@ -499,20 +604,25 @@ __global__ void __launch_bounds__(512, NID > 4 ? 1 : 2)
 
 // Tile rows of the posterior pass: the largest power of two up to 64 (and
 // not past the segment) whose tile, with all K segment-end rows, fits
-// `budget` bytes, preferring tiles that leave room for two CTAs per SM.
-// Long durations: the segment ends are staged in chunks of KH rows (a
-// multiple of 64), the tile as tall as fits.  Sets d.pKH; 0 if nothing fits.
+// `budget` bytes; with `pair` (the kernel that runs two CTAs per SM) a tile
+// that fits half the SM first, unless that halves the rows.  Long
+// durations: the segment ends are staged in chunks of KH rows (a multiple of
+// 64), the tile as tall as fits.  Sets d.pKH; 0 if nothing fits.
 int posterior_tile_rows(Dims& d, size_t budget) {
   int cap = 64;
   while (cap > 8 && cap / 2 >= d.delta) cap /= 2;
   d.pKH = d.K;
-  for (const size_t lim : {std::min<size_t>(budget, 112u * 1024u), budget})
-    for (int rt = cap; rt >= 8; rt /= 2)
-      if (ptile_bytes(rt, d.K, d.C, false) <= lim) return rt;
+  int best = 0;
+  for (int rt = cap; rt >= 8 && !best; rt /= 2)
+    if (ptile_bytes(rt, d.K, d.C) <= budget) best = rt;
+  if (best && posterior_pair(d))
+    for (int rt = best; rt >= 8 && rt * 2 > best; rt /= 2)
+      if (ptile_bytes(rt, d.K, d.C) <= std::min<size_t>(budget, 112u * 1024u)) return rt;
+  if (best) return best;
   for (int rt = cap; rt >= 8; rt /= 2) {
-    const size_t fixed = ptile_bytes(rt, 0, d.C, true);
+    const size_t fixed = ptile_bytes(rt, 0, d.C);
     if (fixed >= budget) continue;
-    const long long kh = ((long long)((budget - fixed) / (12ull * d.C)) - rt) / 64 * 64;
+    const long long kh = ((long long)((budget - fixed) / (8ull * d.C)) - rt) / 64 * 64;
     if (kh >= 64) {
       d.pKH = (int)std::min<long long>(kh, d.K);
       return rt;
@@ -521,29 +631,27 @@ int posterior_tile_rows(Dims& d, size_t budget) {
   return 0;
 }
 
-size_t posterior_smem_bytes(const Dims& d) {
-  return ptile_bytes(d.pRT, d.pKH, d.C, d.pKH < d.K);
-}
+size_t posterior_smem_bytes(const Dims& d) { return ptile_bytes(d.pRT, d.pKH, d.C); }
 
 cudaError_t launch_posterior(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                              const float* trans, const float* dur, const double* grad_logZ,
                              float* grad_em, float* start_marg, float* end_marg, cudaStream_t st,
                              float* seg_marg, int pj) {
   const size_t sm = posterior_smem_bytes(d);
-  const bool small = (size_t)d.K * d.C <= 4u * 512u && (size_t)d.C * d.C <= 4u * 512u;
-  const void* fn = small ? (const void*)posterior_kernel<4, 4> : (const void*)posterior_kernel<16, 32>;
+  const bool pair = posterior_pair(d);
+  const void* fn = pair ? (const void*)posterior_kernel<1, 1> : (const void*)posterior_kernel<4, 2>;
   if (sm > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
   }
-  if (small)
-    posterior_kernel<4, 4><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
+  if (pair)
+    posterior_kernel<1, 1><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
                                                               grad_em, start_marg, end_marg,
                                                               seg_marg, pj);
   else
-    posterior_kernel<16, 32><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
-                                                                grad_em, start_marg, end_marg,
-                                                                seg_marg, pj);
+    posterior_kernel<4, 2><<<dim3(d.nck, d.B), 512, sm, st>>>(d, ws, lengths, trans, dur, grad_logZ,
+                                                              grad_em, start_marg, end_marg,
+                                                              seg_marg, pj);
   return cudaGetLastError();
 }
 

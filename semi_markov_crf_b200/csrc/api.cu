@@ -290,7 +290,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p, size_t* groups = nullptr) {
   const size_t o_vrow = take(d.xG ? B * (size_t)(d.T + 1) * C * 4 : 0);
   const size_t CP = (C + 3) / 4 * 4;
   const size_t o_wrd = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
-  const size_t o_wdl = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
+  const size_t o_varg = take(d.xG ? B * (size_t)(d.T + 1) * CP * 4 : 0);
   group = SEMICRF_WS_KEPT_ROWS;
   const size_t o_kv = take(B * 2ull * (d.T + 1) * 2 * C * 4);
   const size_t o_kf = take(B * 2ull * (d.T + 1) * 8);
@@ -330,7 +330,7 @@ size_t layout(const Dims& d, void* base, WsPtrs* p, size_t* groups = nullptr) {
     p->bp = reinterpret_cast<int32_t*>(c + o_bp);
     p->vrow = reinterpret_cast<float*>(c + o_vrow);
     p->wrd = reinterpret_cast<int32_t*>(c + o_wrd);
-    p->wdl = reinterpret_cast<int32_t*>(c + o_wdl);
+    p->varg = reinterpret_cast<int32_t*>(c + o_varg);
     p->kv = reinterpret_cast<float*>(c + o_kv);
     p->kf = reinterpret_cast<double*>(c + o_kf);
     p->ncut = reinterpret_cast<double*>(c + o_ncut);
@@ -807,8 +807,13 @@ int viterbi_impl(const float* em, const int32_t* lengths, const float* trans, co
     }
     if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
     {
+      ProfScope ps("viterbi_argmax_kernel", st);
+      e = launch_viterbi_argmax(d, p, lengths, trans, st);
+    }
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    {
       ProfScope ps("viterbi_words_kernel", st);
-      e = launch_viterbi_words(d, p, lengths, trans, st);
+      e = launch_viterbi_words(d, p, lengths, st);
     }
     if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
     ProfScope ps("viterbi_walk_kernel", st);

@@ -165,10 +165,13 @@ cudaError_t launch_clustered(void (*kern)(KArgs...), int n_cluster, int grid, in
 // start terms; the kernels add them where a boundary takes the start role).
 size_t chain_exp_smem_bytes(const Dims& d, bool pj = false);
 size_t viterbi_pipe_smem_bytes(const Dims& d, bool pj = false);
-// After viterbi_pipe: the backpointer words from the kept rows (grid-wide),
-// then the traceback (one CTA per sequence, `sm` bytes of shared memory).
+// After viterbi_pipe: the label argmax of every segment start and the
+// backpointer words from the kept rows (grid-wide), then the traceback (one
+// CTA per sequence, `sm` bytes of shared memory).
+cudaError_t launch_viterbi_argmax(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                  const float* trans, cudaStream_t st);
 cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                                 const float* trans, cudaStream_t st);
+                                 cudaStream_t st);
 size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget);
 cudaError_t launch_viterbi_walk(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
                                 int32_t* labels, uint8_t* seg_start, size_t sm, cudaStream_t st);

@@ -83,7 +83,7 @@ struct WsPtrs {
   int32_t* bp;     // [B][T+1][C] Viterbi backpointers (viterbi_pipe: the chosen duration only)
   float* vrow;     // [B][T+1][C] viterbi_pipe: V per boundary, relative to its frame
   int32_t* wrd;    // [B][T+1][CP] viterbi_pipe: backpointer words, CP = C rounded up to 4
-  int32_t* wdl;    // [B][T+1][CP] viterbi_pipe: index step to the previous segment's word
+  int32_t* varg;   // [B][T+1][CP] viterbi_pipe: label argmax A[s, c] of a segment starting at s
   float* kv;       // [B][2][T+1][2][C] exponential-domain ring values per boundary:
                    //   direction (forward, backward) x (p, acc), relative to the frame
   double* kf;      // [B][2][T+1] that frame (absolute, log2 units)

@@ -553,43 +553,38 @@ __global__ void __launch_bounds__(LB, 1)
   }
 }
 
-// Backpointer words, in parallel over (boundary, label): for boundary t in
-// [1, L] and label c with k = kd[t, c] and s = t - k >= 1, the word is
-// k | argmax_{c'} (V[s, c'] + trans2[c', c]) << 16 (smallest c' on ties);
-// for s = 0 the word is k.  Beside it goes the step from this word's index
-// to the previous segment's, -k * CP + (c' - c), for a walk over rows CP =
-// C rounded up to 4 apart (16-byte rows, copied to shared memory in bulk).  One CTA per block of
-// VW_ROWS boundaries of a sequence: the V rows its segments start at are
-// staged in shared memory (rows of VS = C rounded up to 4 floats, -inf
-// padded), and thread (label c, row phase) keeps trans2[., c] in registers.
+// Label argmax rows, in parallel over (boundary, label): for boundary s in
+// [1, L - 1] and label c,
+//   A[s, c] = argmax_{c'} (V[s, c'] + trans2[c', c])   (smallest c' on ties),
+// the label before a segment of label c that starts at s.  It depends on s
+// and c only, not on where the segment ends, so it is computed once per
+// boundary.  One CTA per block of VA_ROWS boundaries of a sequence stages
+// those rows of V (rows of VS = C rounded up to 4 floats, -inf padded);
+// thread (label c, row phase) keeps trans2[., c] in registers and reads each
+// row as float4 broadcasts (the lanes of one row phase read the same row).
 // The argmax runs four independent compare chains (c' mod 4) and merges
-// them by value, then index, so it is the smallest c' among equal maxima,
-// as the recursion's own comparisons would give.
-constexpr int VW_ROWS = 64;
+// them by value, then index, so it is the smallest c' among equal maxima, as
+// the recursion's own comparisons would give.
+constexpr int VA_ROWS = 64;
 template <int NW>
 __global__ void __launch_bounds__(256)
-    viterbi_words_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
-                         const float* __restrict__ trans, int staged) {
-  // staged = 0 (long durations: the rows a block's segments start on do not
-  // fit shared memory): the V rows are read from global memory instead
-  extern __shared__ __align__(16) float vsh[];  // [VW_ROWS + K][VS]
-  const int C = d.C, K = d.K, tid = threadIdx.x, b = blockIdx.y;
+    viterbi_argmax_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
+                          const float* __restrict__ trans) {
+  __shared__ __align__(16) float vsh[VA_ROWS * NW];
+  const int C = d.C, tid = threadIdx.x, b = blockIdx.y;
   const int L = lengths[b];
   if (L < 1 || L > d.T) return;
-  const int t0 = blockIdx.x * VW_ROWS + 1;
-  if (t0 > L) return;
-  const int t1 = min(t0 + VW_ROWS - 1, L);
+  const int s0 = blockIdx.x * VA_ROWS + 1;
+  if (s0 >= L) return;  // boundaries [1, L - 1] start a segment with a predecessor
+  const int s1 = min(s0 + VA_ROWS - 1, L - 1);
   const int VS = (C + 3) & ~3;
-  const int vlo = max(1, t0 - K);  // V rows [vlo, t1 - 1]
   const float* vrw = ws.vrow + (size_t)b * (d.T + 1) * C;
-  const int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
-  int32_t* wrd = ws.wrd + (size_t)b * (d.T + 1) * VS;
-  int32_t* wdl = ws.wdl + (size_t)b * (d.T + 1) * VS;
-  const int nv = staged ? (t1 - vlo) * VS : 0;
+  int32_t* arg = ws.varg + (size_t)b * (d.T + 1) * VS;
+  const int nv = (s1 - s0 + 1) * VS;
 #pragma unroll 4
   for (int i = tid; i < nv; i += blockDim.x) {
     const int r = i / VS, x = i - r * VS;
-    vsh[i] = (x < C) ? vrw[(size_t)(vlo + r) * C + x] : NEG_INF;
+    vsh[i] = (x < C) ? vrw[(size_t)(s0 + r) * C + x] : NEG_INF;
   }
   const int pc = tid % C, pg = tid / C, png = blockDim.x / C;
   float w2[NW];
@@ -598,92 +593,100 @@ __global__ void __launch_bounds__(256)
     w2[q] = (q < C && pg < png) ? __ldg(trans + (size_t)q * C + pc) * l2e() : NEG_INF;
   __syncthreads();
   if (pg >= png) return;
-  for (int t = t0 + pg; t <= t1; t += png) {
-    const int k = kdw[(size_t)t * C + pc];
-    const int sb = t - k;
-    int word = k, step = 0;
-    if (k >= 1 && k <= K && sb >= 1 && !staged) {
-      // the same compare order as the staged path below (chains q mod 4,
-      // merged by value then index), reading row sb from global memory
-      const float* vg = vrw + (size_t)sb * C;
-      float bq[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
-      int qq[4] = {0, 1, 2, 3};
+  // two rows at a time (eight independent chains); per element an add, a
+  // compare-select of the index and a max of the value, so a chain's value
+  // update does not wait on its compare
+  for (int s = s0 + pg; s <= s1; s += 2 * png) {
+    const int sB = min(s + png, s1);  // the second row (the first again past s1)
+    const float4* va = reinterpret_cast<const float4*>(vsh + (size_t)(s - s0) * VS);
+    const float4* vb = reinterpret_cast<const float4*>(vsh + (size_t)(sB - s0) * VS);
+    float bA[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF}, bB[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+    int qA[4] = {0, 1, 2, 3}, qB[4] = {0, 1, 2, 3};
 #pragma unroll
-      for (int q = 0; q < NW; ++q) {
-        if (q < C) {
-          const float e = vg[q] + w2[q];
-          if (e > bq[q & 3]) {
-            bq[q & 3] = e;
-            qq[q & 3] = q;
-          }
+    for (int q4 = 0; q4 < NW / 4; ++q4) {
+      if (4 * q4 < VS) {
+        const float4 x = va[q4], y = vb[q4];
+        const float ex[4] = {x.x, x.y, x.z, x.w}, ey[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float e = ex[u] + w2[4 * q4 + u], f = ey[u] + w2[4 * q4 + u];
+          qA[u] = (e > bA[u]) ? 4 * q4 + u : qA[u];
+          bA[u] = fmaxf(bA[u], e);
+          qB[u] = (f > bB[u]) ? 4 * q4 + u : qB[u];
+          bB[u] = fmaxf(bB[u], f);
         }
       }
-      float b0 = bq[0], b2 = bq[2];
-      int q0 = qq[0], q2 = qq[2];
-      if (bq[1] > b0 || (bq[1] == b0 && qq[1] < q0)) { b0 = bq[1]; q0 = qq[1]; }
-      if (bq[3] > b2 || (bq[3] == b2 && qq[3] < q2)) { b2 = bq[3]; q2 = qq[3]; }
-      if (b2 > b0 || (b2 == b0 && q2 < q0)) { b0 = b2; q0 = q2; }
-      word = k | (q0 << 16);
-      step = -k * VS + (q0 - pc);
-    } else if (k >= 1 && k <= K && sb >= 1) {
-      const float4* vr = reinterpret_cast<const float4*>(vsh + (size_t)(sb - vlo) * VS);
-      float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
-      int q0 = 0, q1 = 1, q2 = 2, q3 = 3;
-#pragma unroll
-      for (int q4 = 0; q4 < NW / 4; ++q4) {
-        if (4 * q4 < VS) {
-          const float4 v = vr[q4];
-          const float e0 = v.x + w2[4 * q4], e1 = v.y + w2[4 * q4 + 1];
-          const float e2 = v.z + w2[4 * q4 + 2], e3 = v.w + w2[4 * q4 + 3];
-          if (e0 > b0) { b0 = e0; q0 = 4 * q4; }
-          if (e1 > b1) { b1 = e1; q1 = 4 * q4 + 1; }
-          if (e2 > b2) { b2 = e2; q2 = 4 * q4 + 2; }
-          if (e3 > b3) { b3 = e3; q3 = 4 * q4 + 3; }
-        }
-      }
-      // a chain that never improved on -inf keeps its first index, so an
-      // all -inf row yields label 0 (the smallest)
-      if (b1 > b0 || (b1 == b0 && q1 < q0)) { b0 = b1; q0 = q1; }
-      if (b3 > b2 || (b3 == b2 && q3 < q2)) { b2 = b3; q2 = q3; }
-      if (b2 > b0 || (b2 == b0 && q2 < q0)) { b0 = b2; q0 = q2; }
-      word = k | (q0 << 16);
-      step = -k * VS + (q0 - pc);
     }
-    wrd[(size_t)t * VS + pc] = word;
-    wdl[(size_t)t * VS + pc] = step;
+    // merge the chains by value, then index: the smallest c' among equal
+    // maxima (a chain that never improved on -inf keeps its first index, so
+    // an all -inf row yields label 0)
+    auto merge = [](float (&bv)[4], int (&qv)[4]) {
+      if (bv[1] > bv[0] || (bv[1] == bv[0] && qv[1] < qv[0])) { bv[0] = bv[1]; qv[0] = qv[1]; }
+      if (bv[3] > bv[2] || (bv[3] == bv[2] && qv[3] < qv[2])) { bv[2] = bv[3]; qv[2] = qv[3]; }
+      if (bv[2] > bv[0] || (bv[2] == bv[0] && qv[2] < qv[0])) { bv[0] = bv[2]; qv[0] = qv[2]; }
+      return qv[0];
+    };
+    arg[(size_t)s * VS + pc] = merge(bA, qA);
+    const int qb = merge(bB, qB);
+    if (s + png <= s1) arg[(size_t)sB * VS + pc] = qb;
+  }
+}
+
+// Backpointer words, in parallel over (boundary, label): for boundary t in
+// [1, L] and label c with k = kd[t, c] in [1, K] and s = t - k >= 1, the word
+// is k | A[s, c] << 16; otherwise (s = 0, or a duration the recursion never
+// set) it is k.  Rows of CP = C rounded up to 4 words (16-byte rows, copied
+// to shared memory in bulk by the walk).
+__global__ void __launch_bounds__(256)
+    viterbi_words_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths) {
+  const int C = d.C, CP = (C + 3) & ~3, b = blockIdx.y;
+  const int L = lengths[b];
+  if (L < 1 || L > d.T) return;
+  const int32_t* kdw = ws.bp + (size_t)b * (d.T + 1) * C;
+  const int32_t* arg = ws.varg + (size_t)b * (d.T + 1) * CP;
+  int32_t* wrd = ws.wrd + (size_t)b * (d.T + 1) * CP;
+  const size_t n = (size_t)L * C;  // boundaries [1, L]
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / C) + 1, c = (int)(i - (size_t)(t - 1) * C);
+    const int k = kdw[(size_t)t * C + c];
+    const int s = t - k;
+    int word = k;
+    if (k >= 1 && k <= d.K && s >= 1) word = k | (arg[(size_t)s * CP + c] << 16);
+    wrd[(size_t)t * CP + c] = word;
   }
 }
 
 // The traceback, one CTA per sequence.  Start: the best final label
-// (argmax of the kept row V[L], smallest on ties).  In stages over the
-// dynamic shared memory: thread 0 copies the word rows [lo, tt0] and their
-// index steps in with two bulk copies (TMA, completion on an mbarrier, a
-// bounded wait), follows the words -- one shared-memory read and an add per
-// decoded segment -- and marks each segment's start position with its
-// label; then warp 0 fills every position of the stage with the label of the
-// last mark at or below it (a running "last mark" scan, 32 positions per
-// shuffle round) and writes labels and start flags out coalesced.  The next
-// stage starts where the walk left the staged rows.  A word with a duration
-// outside [1, t], a previous label >= C or a step leaving the staged rows
-// ends the walk with the positions not reached labelled -1.
+// (argmax of the kept row V[L], smallest on ties).  The word rows are cut
+// into fixed windows of WR rows, [1 + w WR, (w + 1) WR], taken downwards
+// through two buffers: while the walk reads window w, a bulk copy (TMA,
+// completion on that buffer's mbarrier, bounded waits) brings window w - 1
+// into the other.  Thread 0 follows the words through the window -- one
+// shared-memory read per decoded segment -- and marks each segment's start
+// position with its label; then warp 0 fills every position from where the
+// walk left the window up to where it entered it with the label of the last
+// mark at or below it (a running "last mark" scan, 32 positions per shuffle
+// round) and writes labels and start flags out coalesced.  A segment that
+// jumps past the prefetched window has its window copied in before the walk
+// goes on.  A word with a duration outside [1, min(t, K)] or a previous
+// label >= C ends the walk with the positions not reached labelled -1.
 __global__ void __launch_bounds__(256)
     viterbi_walk_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
                         int32_t* __restrict__ labels, uint8_t* __restrict__ seg_start, int WR) {
-  extern __shared__ __align__(16) int wsh[];  // words [WR][CP], steps [WR][CP], marks [WR + K]
+  extern __shared__ __align__(16) int wsh[];  // words [2][WR][CP], marks [WR + K]
   __shared__ int s_tb[2];
-  __shared__ __align__(8) uint64_t wbar;
+  __shared__ __align__(8) uint64_t wbar[2];
   const int C = d.C, K = d.K, T = d.T, tid = threadIdx.x, lane = tid & 31, b = blockIdx.x;
   const int CP = (C + 3) & ~3;
   const int L = lengths[b];
   if (L < 1 || L > T) return;
   const int32_t* wrd = ws.wrd + (size_t)b * (T + 1) * CP;
-  const int32_t* wdl = ws.wdl + (size_t)b * (T + 1) * CP;
   const float* vrw = ws.vrow + (size_t)b * (T + 1) * C;
-  int* const kbuf = wsh;
-  int* const dbuf = wsh + (size_t)WR * CP;
   int* const lbuf = wsh + 2 * (size_t)WR * CP;
   if (tid == 0) {
-    mbar_init(&wbar, 1);
+    mbar_init(&wbar[0], 1);
+    mbar_init(&wbar[1], 1);
     fence_mbar_init();
   }
   if (tid < 32) {
@@ -703,41 +706,53 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
-  uint32_t phase = 0;
+  // copy window w (its rows up to L) into buffer p; thread 0
+  auto issue = [&](int w, int p) {
+    const int lo = 1 + w * WR, hi = min(L, lo + WR - 1);
+    const uint32_t bytes = (uint32_t)((hi - lo + 1) * CP * 4);
+    fence_proxy_async();  // earlier reads of the buffer come before the copy's writes
+    mbar_expect_tx(&wbar[p], bytes);
+    bulk_g2s(wsh + (size_t)p * WR * CP, wrd + (size_t)lo * CP, bytes, &wbar[p]);
+  };
+  uint32_t ph[2] = {0u, 0u};    // every thread tracks both barriers' phases
+  bool busy[2] = {true, false};  // a copy into the buffer is in flight
+  // a bounded wait for buffer p's copy, by every thread together; false: a
+  // thread gave up (the state is left as it was, the same in every thread)
+  bool timed_out = false;
+  auto land = [&](int p) {
+    const bool ok = mbar_wait(&wbar[p], ph[p], WAIT_SPIN_LIMIT);
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      return false;
+    }
+    ph[p] ^= 1u;
+    busy[p] = false;
+    return true;
+  };
+  int w = (L - 1) / WR, p = 0;
+  if (tid == 0) issue(w, 0);
   for (;;) {
-    const int tt0 = s_tb[0];
-    if (tt0 <= 0) break;
-    const int lo = max(1, tt0 - WR + 1);
+    const int tt0 = s_tb[0];  // 1 <= tt0, inside window w
+    const int lo = 1 + w * WR;
     const int pb = lo - K;  // mark of position u at lbuf[u - pb]
-    const uint32_t bytes = (uint32_t)((tt0 - lo + 1) * CP * 4);
-    // bounds-check build: the stage's rows fit the staging buffers
-    if (!SEMICRF_INB(ws.status, tt0 - lo + 1 <= WR && tt0 <= T, SITE_WALK_STAGE)) break;
-    if (tid == 0) {
-      fence_proxy_async();  // the last stage's reads come before the copies' writes
-      mbar_expect_tx(&wbar, 2 * bytes);
-      bulk_g2s(kbuf, wrd + (size_t)lo * CP, bytes, &wbar);
-      bulk_g2s(dbuf, wdl + (size_t)lo * CP, bytes, &wbar);
+    // bounds-check build: the walk starts inside the window
+    if (!SEMICRF_INB(ws.status, tt0 >= lo && tt0 - lo < WR && tt0 <= L, SITE_WALK_STAGE)) break;
+    if (!land(p)) break;
+    const bool pre = w > 0;
+    if (pre) {
+      if (tid == 0) issue(w - 1, p ^ 1);
+      busy[p ^ 1] = true;
     }
     for (int i = tid; i < WR + K; i += blockDim.x) lbuf[i] = -1;
-    const bool ok = mbar_wait(&wbar, phase, WAIT_SPIN_LIMIT);
-    phase ^= 1u;
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) {
-        set_status(ws.status, ST_DEVICE_TIMEOUT);
-        mbar_wait(&wbar, phase ^ 1u, WAIT_SPIN_LIMIT);  // let the copies land before exit
-      }
-      return;
-    }
+    __syncthreads();
     if (tid == 0) {
+      const int* kb = wsh + (size_t)p * WR * CP;
       int tt = tt0, cl = s_tb[1];
-      int idx = (tt - lo) * CP + cl;
-      const int nidx = (tt0 - lo + 1) * CP;
       bool broken = false;
       while (tt >= lo) {
-        const int w = kbuf[idx];
-        const int step = dbuf[idx];
-        const int k = w & 0xffff, pred = (w >> 16) & 0xffff;
-        if (k < 1 || k > tt || (tt - k > 0 && pred >= C)) {
+        const int wd = kb[(tt - lo) * CP + cl];
+        const int k = wd & 0xffff, pred = (wd >> 16) & 0xffff;
+        if (k < 1 || k > tt || k > K || (tt - k > 0 && pred >= C)) {
           broken = true;
           break;
         }
@@ -745,11 +760,6 @@ __global__ void __launch_bounds__(256)
         if (SEMICRF_INB(ws.status, tt - pb >= 0 && tt - pb < WR + K, SITE_WALK_MARK))
           lbuf[tt - pb] = cl;
         cl = pred;
-        idx += step;
-        if (tt >= lo && (idx < 0 || idx >= nidx)) {
-          broken = true;
-          break;
-        }
       }
       s_tb[0] = broken ? -tt : tt;  // -tt: stop, positions below tt get -1
       s_tb[1] = cl;
@@ -778,47 +788,56 @@ __global__ void __launch_bounds__(256)
     }
     if (te < 0)
       for (int u = tid; u < end; u += blockDim.x) labels[(size_t)b * T + u] = -1;
-    __syncthreads();  // every thread has read s_tb and the marks before the next stage
-    if (te < 0) break;
+    __syncthreads();  // every thread has read s_tb and the marks before the next window
+    if (te <= 0) break;
+    // the next window: the one holding te (the prefetched one unless a
+    // segment jumped past it)
+    const int wn = (te - 1) / WR;
+    if (wn != w - 1) {
+      if (!land(p ^ 1)) break;
+      if (tid == 0) issue(wn, p ^ 1);
+      busy[p ^ 1] = true;
+    }
+    w = wn;
+    p ^= 1;
   }
+  // leave no copy in flight into this CTA's shared memory
+  for (int q = 0; q < 2; ++q)
+    if (busy[q]) land(q);
+  if (timed_out && tid == 0) set_status(ws.status, ST_DEVICE_TIMEOUT);
 }
 
 }  // namespace
 
 size_t viterbi_pipe_smem_bytes(const Dims& d, bool pj) { return vsmem_bytes(d, pj); }
 
-#define SEMICRF_VW_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
+#define SEMICRF_VA_WIDTHS(X) X(8) X(16) X(32) X(48) X(64) X(96) X(128)
 
-cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
-                                 const float* trans, cudaStream_t st) {
-  size_t sm = (size_t)(VW_ROWS + d.K) * ((d.C + 3) & ~3) * sizeof(float);
-  int max_optin = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-          cudaSuccess)
-    return cudaErrorInvalidValue;
-  const int staged = sm + 256 <= (size_t)max_optin ? 1 : 0;
-  if (!staged) sm = 0;
-  const dim3 grid((d.T + VW_ROWS - 1) / VW_ROWS, d.B);
-  if (d.T == 0) return cudaSuccess;
-#define SEMICRF_VW_LAUNCH(nw)                                                                   \
-  if (d.C <= nw) {                                                                              \
-    if (sm > 48 * 1024) {                                                                       \
-      const cudaError_t e = cudaFuncSetAttribute(viterbi_words_kernel<nw>,                      \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                                 (int)sm);                                      \
-      if (e != cudaSuccess) return e;                                                           \
-    }                                                                                           \
-    viterbi_words_kernel<nw><<<grid, 256, sm, st>>>(d, ws, lengths, trans, staged);             \
-    return cudaGetLastError();                                                                  \
+cudaError_t launch_viterbi_argmax(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                  const float* trans, cudaStream_t st) {
+  if (d.T == 0 || d.B == 0) return cudaSuccess;
+  const dim3 grid((d.T + VA_ROWS - 1) / VA_ROWS, d.B);
+#define SEMICRF_VA_LAUNCH(nw)                                                 \
+  if (d.C <= nw) {                                                            \
+    viterbi_argmax_kernel<nw><<<grid, 256, 0, st>>>(d, ws, lengths, trans);   \
+    return cudaGetLastError();                                                \
   }
-  SEMICRF_VW_WIDTHS(SEMICRF_VW_LAUNCH)
-#undef SEMICRF_VW_LAUNCH
+  SEMICRF_VA_WIDTHS(SEMICRF_VA_LAUNCH)
+#undef SEMICRF_VA_LAUNCH
   return cudaErrorInvalidConfiguration;
 }
 
-// Shared memory of the walk: about 96 KB (fewer stages), at least the K
-// marks and one row of words and steps.
+cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t* lengths,
+                                 cudaStream_t st) {
+  if (d.T == 0 || d.B == 0) return cudaSuccess;
+  const size_t items = (size_t)d.T * d.C;
+  const dim3 grid((unsigned)std::min<size_t>((items + 255) / 256, 1184), d.B);
+  viterbi_words_kernel<<<grid, 256, 0, st>>>(d, ws, lengths);
+  return cudaGetLastError();
+}
+
+// Shared memory of the walk: about 96 KB (longer windows), at least the K
+// marks and one row of words per buffer.
 size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget) {
   const size_t CP = (d.C + 3) & ~3;
   const size_t want = std::min<size_t>(budget, 96u * 1024u);

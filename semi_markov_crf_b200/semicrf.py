@@ -24,8 +24,8 @@ __all__ = ["workspace_bytes", "workspace_itemize", "WS_GROUPS", "launch_shape", 
 KERNELS = ("prefix_reduce_kernel", "prefix_scan_kernel", "chain_exp_kernel", "chain_kernel",
            "cut_grid_kernel", "posterior_kernel", "segment_kernel",
            "finalize_positions_kernel",
-           "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_words_kernel",
-           "viterbi_walk_kernel", "path_terms_kernel", "path_grad_kernel",
+           "reduce_partials_kernel", "viterbi_kernel", "viterbi_pipe_kernel", "viterbi_argmax_kernel",
+           "viterbi_words_kernel", "viterbi_walk_kernel", "path_terms_kernel", "path_grad_kernel",
            "proj_grad_kernel")
 
 FLAG_NO_CENTER = 0x1

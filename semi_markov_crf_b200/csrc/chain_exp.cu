@@ -146,9 +146,10 @@ __device__ __forceinline__ int next_mod(int i, int rem) {
 // cluster with asynchronous distributed-shared-memory stores (the group's
 // lanes taking different destination CTAs) that count against the
 // destination's arrival barrier pbar[t & 1] (4 C bytes per step).  A combine
-// lane waits on its own CTA's barrier before reading p_{t-1}, then its CTA
-// re-arms that barrier for step t+1; steps still end with the CTA barrier
-// only.  No release fence sits in the step (a cluster barrier's release
+// lane waits on its own CTA's barrier before reading p_{t-1}; a thread off
+// the combine path re-arms it at the top of step t+1 (for step t+1's
+// vector); steps still end with the CTA barrier only.  The send addresses
+// in the other CTAs are mapped once, before the walk.  No release fence sits in the step (a cluster barrier's release
 // would also wait for the kept rows' global stores).  Every CTA holds the
 // same full vector and computes the same frame step n from it.  A barrier
 // phase is reused two steps later, by which time every CTA has read the
@@ -186,6 +187,21 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   const int RL = K + WL, RLP = d.xRLP;
   float2* const rl = sm.ring + (size_t)ccl * RLP;
   const uint32_t vbytes = 4u * (uint32_t)C;  // label-vector bytes arriving per step (clusters)
+  // clusters: the destinations of this combine lane's sends (CTAs jl,
+  // jl + G, ...), their buffer and barrier mapped once
+  constexpr int ND = (N + G - 1) / G;
+  uint32_t rbuf[ND], rbar[ND];
+#pragma unroll
+  for (int u = 0; u < ND; ++u) {
+    rbuf[u] = rbar[u] = 0u;
+    if constexpr (N > 1) {
+      const int q = jl + u * G;
+      if (comb && q < N) {
+        rbuf[u] = cluster_addr(xs.P, (uint32_t)q);
+        rbar[u] = cluster_addr(xs.pbar, (uint32_t)q);
+      }
+    }
+  }
   auto put = [&](int slot, float2 v) {  // slot and its mirrors slot + mK < RL
     for (int x = slot; x < RL; x += K) rl[x] = v;
   };
@@ -351,6 +367,12 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
   const float acc_start = ex2(-M);
   for (int i = 1; i <= L; ++i) {
     const int r = UP ? i : L - i;
+    // clusters: re-arm the arrival barrier of step i's vector (its previous
+    // phase, step i-2's, completed before step i-1's label fan-in) for this
+    // step's arrivals, by a thread off the combine path (bytes arriving
+    // before the arm only take the count below zero)
+    if constexpr (N > 1)
+      if (tid == (int)blockDim.x - 32 && i >= 3) mbar_expect_tx(&xs.pbar[i & 1], vbytes);
     if (!comb && i >= 2) Fph += xs.nsl[(i - 1) & 1];
     if (i == next_ev) {
       if (i < L && i % TS == rem_w) {
@@ -409,13 +431,12 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       // ---------------------------------------------------------- combine
       if constexpr (N > 1) {
         if (i >= 2) {
-          // p_{i-1} from every CTA of the cluster, then re-arm for step i+1
+          // p_{i-1} from every CTA of the cluster
           const int pb = (i - 1) & 1;
           if (!xdead && !mbar_wait_cluster(&xs.pbar[pb], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
             set_status(ws.status, ST_DEVICE_TIMEOUT);
             xdead = true;
           }
-          if (tid == 0 && i + 1 <= L) mbar_expect_tx(&xs.pbar[pb], vbytes);
         }
       }
       const int po = (i & 1) * Cr + ccl;
@@ -459,9 +480,12 @@ __device__ __forceinline__ void xring(const XSmem& xs, const Dims& d, const WsPt
       const bool pok = SEMICRF_INB(ws.status, !act || c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
-        if (act && pok)
-          for (int q = jl; q < N; q += G)
-            st_async_cluster(xs.P + (i & 1) * d.xPC + c, xs.pbar + (i & 1), q, pn);
+        if (act && pok) {
+          const uint32_t po = 4u * (uint32_t)((i & 1) * d.xPC + c), bo = 8u * (uint32_t)(i & 1);
+#pragma unroll
+          for (int u = 0; u < ND; ++u)
+            if (jl + u * G < N) st_async_mapped(rbuf[u] + po, rbar[u] + bo, pn);
+        }
       } else {
         if (leader && pok) xs.P[(i & 1) * d.xPC + c] = pn;
       }

@@ -168,6 +168,23 @@ __device__ __forceinline__ void st_async_cluster(const float* local, const uint6
                : "memory");
 }
 
+// The address of `local` (a shared-memory location of this CTA) in the
+// shared memory of cluster CTA `rank`.  A CTA's window is linear, so the
+// address of local + off there is this plus off.
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
+  return ra;
+}
+
+// st_async_cluster with the remote addresses already mapped (cluster_addr):
+// v to ra, completing 4 bytes on the mbarrier at rb.
+__device__ __forceinline__ void st_async_mapped(uint32_t ra, uint32_t rb, float v) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(ra),
+               "r"(__float_as_uint(v)), "r"(rb)
+               : "memory");
+}
+
 // Bounded wait, with cluster-scope acquire, for phase `parity` of `bar`
 // (data delivered by st_async_cluster from any CTA of the cluster).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int spins) {

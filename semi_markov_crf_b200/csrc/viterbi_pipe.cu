@@ -134,8 +134,8 @@ __device__ __forceinline__ int next_with_rem(int i, int rem) {
 // combine group sends its V[t] into the V buffer of every CTA of the cluster
 // with asynchronous distributed-shared-memory stores counted by the
 // destination's arrival barrier vbar[t & 1] (4 C bytes per step); a combine
-// lane waits on it before reading V[t-1] and the CTA re-arms it for step t+1
-// (the same exchange as the exponential-domain rings), so every CTA holds the
+// lane waits on it before reading V[t-1] and a thread off the combine path
+// re-arms it at the top of step t+1 (the same exchange as the exponential-domain rings), so every CTA holds the
 // whole row and takes the same frame.  Every CTA takes the same early exits
 // (they depend only on the inputs).
 template <int N, int G, int CAT, int H, int KBH, int LB>
@@ -192,6 +192,21 @@ __global__ void __launch_bounds__(LB, 1)
   const int RL = K + WL, RLP = d.xRLP;
   float2* const rl = sm.ring + (size_t)ccl * RLP;
   const uint32_t vbytes = 4u * (uint32_t)C;  // V-row bytes arriving per step (clusters)
+  // clusters: the destinations of this combine lane's sends (CTAs jl,
+  // jl + G, ...), their buffer and barrier mapped once
+  constexpr int ND = (N + G - 1) / G;
+  uint32_t rbuf[ND], rbar[ND];
+#pragma unroll
+  for (int u = 0; u < ND; ++u) {
+    rbuf[u] = rbar[u] = 0u;
+    if constexpr (N > 1) {
+      const int q = jl + u * G;
+      if (comb && q < N) {
+        rbuf[u] = cluster_addr(vs.V, (uint32_t)q);
+        rbar[u] = cluster_addr(vs.vbar, (uint32_t)q);
+      }
+    }
+  }
   // bounds-check build: a row pointer lies inside the two tile buffers
   auto row_ok = [&](const int32_t* row) {
     const ptrdiff_t o = row - sm.tint;
@@ -329,6 +344,12 @@ __global__ void __launch_bounds__(LB, 1)
   int next_ev = next_event(0);
 
   for (int i = 1; i <= L; ++i) {
+    // clusters: re-arm the arrival barrier of step i's vector (its previous
+    // phase, step i-2's, completed before step i-1's label fan-in) for this
+    // step's arrivals, by a thread off the combine path (bytes arriving
+    // before the arm only take the count below zero)
+    if constexpr (N > 1)
+      if (tid == (int)blockDim.x - 32 && i >= 3) mbar_expect_tx(&vs.vbar[i & 1], vbytes);
     if (!comb && i >= 2) Fph += vs.nsl[(i - 1) & 1];
     if (i == next_ev) {
       if (i < L && (i + 1) % TS == 0) {
@@ -378,13 +399,12 @@ __global__ void __launch_bounds__(LB, 1)
       // ---------------------------------------------------------- combine
       if constexpr (N > 1) {
         if (i >= 2) {
-          // V[i-1] from every CTA of the cluster, then re-arm for step i+1
+          // V[i-1] from every CTA of the cluster
           const int pb = (i - 1) & 1;
           if (!xdead && !mbar_wait_cluster(&vs.vbar[pb], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
             set_status(ws.status, ST_DEVICE_TIMEOUT);
             xdead = true;
           }
-          if (tid == 0 && i + 1 <= L) mbar_expect_tx(&vs.vbar[pb], vbytes);
         }
       }
       const float mp = vs.mx[(i - 1) & 1];
@@ -431,9 +451,12 @@ __global__ void __launch_bounds__(LB, 1)
       const bool pok = SEMICRF_INB(ws.status, !act || c < d.xPC, SITE_VECTOR);
       if constexpr (N > 1) {
         // into every CTA of the cluster (this one included)
-        if (act && pok)
-          for (int q = jl; q < N; q += G)
-            st_async_cluster(vs.V + (i & 1) * d.xPC + c, vs.vbar + (i & 1), q, v - n);
+        if (act && pok) {
+          const uint32_t po = 4u * (uint32_t)((i & 1) * d.xPC + c), bo = 8u * (uint32_t)(i & 1);
+#pragma unroll
+          for (int u = 0; u < ND; ++u)
+            if (jl + u * G < N) st_async_mapped(rbuf[u] + po, rbar[u] + bo, v - n);
+        }
       } else {
         if (leader && pok) vs.V[(i & 1) * d.xPC + c] = v - n;
       }

@@ -15,13 +15,15 @@
 // G[t-1] into the label's ring.  Helper warps (H lanes per label, KBH
 // durations per lane, strided over the window so that a label's lanes read
 // consecutive ring entries) compute during step t everything else: the best
-// k >= 3 term of step t+1 and its k, the additive constants of its k = 1 and
-// k = 2 terms, and the max of V[t-1] for the frame.  One barrier per step.
+// k >= 3 term of step t+1 and its k and the additive constants of its k = 1
+// and k = 2 terms; they never read the row V[t-1], so in a cluster they
+// finish before the exchange brings it.  One barrier per step.
 //
 // Frames: V[t, :] is stored relative to Phi_t with Phi_t = rint(max V[t-2])
-// (absolute): n_t = rint(m_{t-2}) - n_{t-1}, m published by the helpers, so
-// no reduction sits on the critical path and the frame follows the maximum
-// two steps late without oscillating.
+// (absolute): n_t = rint(m_{t-2}) - n_{t-1}, m the max every combine group
+// takes of the row it reads for the label fan-in (one step before it is
+// used), so the reduction runs beside the fan-in's and the frame follows the
+// maximum two steps late without oscillating.
 //
 // Ties: k = 1 before k = 2 before the helpers' best k (itself the smallest
 // k among equal terms), the smallest c' among equal label terms, and the
@@ -58,7 +60,6 @@ struct VSmem {
   float* A1;   // [2][Cr]   dur2[0] + S[t] - S[t-1]
   float* A2;   // [2][Cr]   dur2[1] + S[t] - S[t-2]
   float* nsl;  // [2]       frame step published by the combine warps
-  float* mx;   // [2]       max V[t-1] published by the helpers at step t
   int* Sb;     // [Cr]      label integer bases
   uint64_t* vbar;  // [2]   cluster: arrival of the step's V row, by step parity
 };
@@ -71,7 +72,6 @@ __device__ __forceinline__ VSmem vcarve(unsigned char* raw, const Dims& d, bool 
   x.s.maxslot = reinterpret_cast<int*>(p + 16);
   x.s.aux = reinterpret_cast<int*>(p + 32);
   x.nsl = reinterpret_cast<float*>(p + 48);
-  x.mx = reinterpret_cast<float*>(p + 56);
   x.vbar = reinterpret_cast<uint64_t*>(p + 64);
   p += 96;
   x.s.tint = reinterpret_cast<int32_t*>(p);
@@ -135,8 +135,9 @@ __device__ __forceinline__ int next_with_rem(int i, int rem) {
 // with asynchronous distributed-shared-memory stores counted by the
 // destination's arrival barrier vbar[t & 1] (4 C bytes per step); a combine
 // lane waits on it before reading V[t-1] and a thread off the combine path
-// re-arms it at the top of step t+1 (the same exchange as the exponential-domain rings), so every CTA holds the
-// whole row and takes the same frame.  Every CTA takes the same early exits
+// re-arms it at the top of step t+1 (the same exchange as the
+// exponential-domain rings), so every CTA holds the whole row and takes the
+// same frame.  Every CTA takes the same early exits
 // (they depend only on the inputs).
 template <int N, int G, int CAT, int H, int KBH, int LB>
 __global__ void __launch_bounds__(LB, 1)
@@ -173,7 +174,6 @@ __global__ void __launch_bounds__(LB, 1)
   constexpr int HG = H > 32 ? 32 : H;       // lanes per reduction group
   constexpr int HW = H > 32 ? H / 32 : 1;   // helper warps per label
   constexpr int LPWC = 32 / G, LPWH = 32 / HG, WL = H * KBH;
-  constexpr int CA = (G * CAT + H - 1) / H;  // labels per lane for the frame max
   constexpr int NR = CAT > KBH ? CAT : KBH;
   const int warp = tid >> 5, lane = tid & 31;
   const int nwc = (Cr + LPWC - 1) / LPWC;
@@ -250,7 +250,6 @@ __global__ void __launch_bounds__(LB, 1)
   }
   if (tid == 0) {
     vs.nsl[0] = vs.nsl[1] = 0.f;
-    vs.mx[0] = vs.mx[1] = NEG_INF;
     mbar_init(&sm.mbar[0], 1);
     mbar_init(&sm.mbar[1], 1);
     if constexpr (N > 1) {
@@ -316,7 +315,7 @@ __global__ void __launch_bounds__(LB, 1)
   float* const vrw = ws.vrow + (size_t)b * (T + 1) * C;
   int32_t* const kdw = ws.bp + (size_t)b * (T + 1) * C;
   // combine state: S at row i - 1, ring slot of boundary i - 1
-  float g2 = NEG_INF, nprev = 0.f, Fp = 0.f;
+  float g2 = NEG_INF, nprev = 0.f, Fp = 0.f, mp = NEG_INF;
   int si_p = 0;
   float sf_p = 0.f, pd_p = sm.tpd ? sm.tpd[cc] : 0.f;  // row i - 1 (pd: start term)
   const int32_t* crow_i = sm.tint + C;  // row i of the current step
@@ -407,7 +406,6 @@ __global__ void __launch_bounds__(LB, 1)
           }
         }
       }
-      const float mp = vs.mx[(i - 1) & 1];
       const float a1 = vs.A1[(i & 1) * Cr + ccl];
       const float a2 = vs.A2[(i & 1) * Cr + ccl];
       float om = vs.Om[(i & 1) * Cr + ccl];
@@ -426,7 +424,9 @@ __global__ void __launch_bounds__(LB, 1)
       const float pd_n = (crow_d && rok) ? crow_d[cc] : 0.f;
       const float sf_n = rok ? crow_f[cc] : 0.f;
       const float* pv = vs.V + ((i - 1) & 1) * d.xPC + 4 * jl;
-      float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF;
+      // the label fan-in and, beside it, max V[i-1] (a group's lanes read
+      // the whole row; padding entries hold -inf): the frame of step i+1
+      float b0 = NEG_INF, b1 = NEG_INF, b2 = NEG_INF, b3 = NEG_INF, m0 = NEG_INF, m1 = NEG_INF;
 #pragma unroll
       for (int q = 0; q < CAT; q += 4) {
         const float4 v = *reinterpret_cast<const float4*>(pv + q * G);
@@ -434,14 +434,21 @@ __global__ void __launch_bounds__(LB, 1)
         b1 = fmaxf(b1, v.y + w[q + 1]);
         b2 = fmaxf(b2, v.z + w[q + 2]);
         b3 = fmaxf(b3, v.w + w[q + 3]);
+        m0 = fmaxf(m0, fmaxf(v.x, v.y));
+        m1 = fmaxf(m1, fmaxf(v.z, v.w));
       }
       float gv = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
+      float mcur = fmaxf(m0, m1);
 #pragma unroll
-      for (int o = G / 2; o > 0; o >>= 1) gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
+      for (int o = G / 2; o > 0; o >>= 1) {
+        gv = fmaxf(gv, __shfl_xor_sync(FULL_MASK, gv, o));
+        mcur = fmaxf(mcur, __shfl_xor_sync(FULL_MASK, mcur, o));
+      }
       if (i == 1) gv = 0.f;  // G[0] = 0 in frame 0 (V[0] is all -inf)
-      // frame: Phi_i = Phi_{i-2} + rint(max V[i-2]), the max published by
-      // the helpers a step ago
+      // frame: Phi_i = Phi_{i-2} + rint(max V[i-2]), the max this lane took
+      // a step ago
       const float n = ((mp == NEG_INF) ? 0.f : rintf(mp)) - nprev;
+      mp = mcur;
       // candidates relative to Phi_{i-1}; ties to the smaller k
       const float c1 = gv + a1;
       const float c2 = (g2 + a2) - nprev;
@@ -484,23 +491,9 @@ __global__ void __launch_bounds__(LB, 1)
       crow_f += C;
     } else {
       // ---------------------------------------------------------- helpers
-      // reads: row V[i-1] for the frame max, the window of the k >= 3 terms
-      // of step i + 1 (boundaries i - 1 - WL .. i - 2) and its prefix-sum row
-      if constexpr (N > 1) {
-        // V[i-1] from every CTA of the cluster (the combine lanes re-arm)
-        if (i >= 2 && !xdead &&
-            !mbar_wait_cluster(&vs.vbar[(i - 1) & 1], ((i - 2) >> 1) & 1, WAIT_SPIN_LIMIT)) {
-          set_status(ws.status, ST_DEVICE_TIMEOUT);
-          xdead = true;
-        }
-      }
-      const float* pv = vs.V + ((i - 1) & 1) * d.xPC + jl;
-      float m0 = NEG_INF, m1 = NEG_INF;
-#pragma unroll
-      for (int q = 0; q < CA; q += 2) {
-        m0 = fmaxf(m0, pv[q * H]);
-        if (q + 1 < CA) m1 = fmaxf(m1, pv[(q + 1) * H]);
-      }
+      // reads: the window of the k >= 3 terms of step i + 1 (boundaries
+      // i - 1 - WL .. i - 2) and its prefix-sum row (not the row V[i-1]: in a
+      // cluster the helpers never wait for the exchange)
       const bool hok = i < L && SEMICRF_INB(ws.status, row_ok(hrow_i), SITE_TILE_ROW);
       const int sn = hok ? hrow_i[cc] : 0;
       const float fn = hok ? hrow_f[cc] : 0.f;
@@ -515,12 +508,8 @@ __global__ void __launch_bounds__(LB, 1)
         tv[q] = ((e.y + Qh) + e.x) + w[q];
         best = fmaxf(best, tv[q]);
       }
-      float mv = fmaxf(m0, m1);
 #pragma unroll
-      for (int o = HG / 2; o > 0; o >>= 1) {
-        best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
-        mv = fmaxf(mv, __shfl_xor_sync(FULL_MASK, mv, o));
-      }
+      for (int o = HG / 2; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(FULL_MASK, best, o));
       // smallest k among equal terms: k falls as the window index grows
       int kb = 0x7fffffff;
 #pragma unroll
@@ -528,8 +517,7 @@ __global__ void __launch_bounds__(LB, 1)
         if (tv[q] == best) kb = 2 + WL - (q * H + jl);
 #pragma unroll
       for (int o = HG / 2; o > 0; o >>= 1) kb = min(kb, __shfl_xor_sync(FULL_MASK, kb, o));
-      // stores (every label group saw all of V[i-1]: the first one publishes)
-      if (warp == nwc && lane == 0) vs.mx[i & 1] = mv;
+      // stores
       if (act && lane % HG == 0 && i < L) {  // each helper warp's candidate
         const int o2 = ((i + 1) & 1) * Cr + cl;
         vs.Om[hwarp * 2 * Cr + o2] = best + fn;

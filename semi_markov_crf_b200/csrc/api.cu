@@ -74,11 +74,14 @@ int max_smem_optin() {
 // warps that share a scheduler.  One CTA per ring serves narrow label sets
 // best; from C >= CLUSTER_MIN_C labels a ring is split over a thread-block
 // cluster (N CTAs, C / N labels each): the per-step work of one SM shrinks
-// N-fold and each step pays a cluster barrier (about 500 cycles measured on
-// B200 against about 150 for a CTA barrier), which pays when one SM's step
-// is several thousand cycles (C = 128: about 4300 cycles on one CTA, 2400 on
-// a cluster of 4, 2500 on 8).  Clusters of 4 are preferred: the two rings
-// and the decoder of a batch then fit the GPU side by side (B = 8: 96 SMs).
+// N-fold and each step pays the label vector's exchange through distributed
+// shared memory (about 400 cycles measured on B200, beside about 200 for a
+// CTA barrier), which pays when one SM's step is several thousand cycles.
+// At C = 128, K = 64 a step measured about 4300 cycles on one CTA; 1270 on
+// a cluster of 4 and 1240 on 8 (forward-backward), 1280 and 1020 (the
+// decoder, whose helpers are lighter).  Forward-backward prefers clusters of
+// 4 and the decoder 8 where its clusters fit the GPU at once: at B = 8 the
+// two rings (64 SMs) and the decoder (64) then run side by side.
 // SEMICRF_XSHAPE=i forces the i-th fitting shape of the menu and
 // SEMICRF_XCLUSTER=n restricts the choice to clusters of n CTAs (tuning).
 constexpr int CLUSTER_MIN_C = 96;
@@ -94,7 +97,7 @@ void xshape_derive(Dims& d) {
   if (d.xH < 16) d.xRLP += (((d.xH - d.xRLP) % 16) + 16) % 16;
 }
 
-void choose_xshape(Dims& d, size_t budget) {
+void choose_xshape(Dims& d, size_t budget, int prefer_n) {
   const int C = d.C, K = d.K;
   int forced = -1, forced_n = 0;
   if (const char* env = std::getenv("SEMICRF_XSHAPE")) forced = std::atoi(env);
@@ -136,7 +139,7 @@ void choose_xshape(Dims& d, size_t budget) {
       if (chain_exp_smem_bytes(t) <= budget && viterbi_pipe_smem_bytes(t) <= budget) {   \
         const double cost = std::max(cat + 25.0 * lg(g), 2.0 * kbh + 25.0 * lg(h)) +      \
                             10.0 * ((nwc + nwh + 3) / 4) + (lb > 512 ? 1000.0 : 0.0) +    \
-                            (n > 1 ? 100.0 + 25.0 * std::abs(n - 4) : 0.0);               \
+                            (n > 1 ? 100.0 + 25.0 * std::abs(n - prefer_n) : 0.0);        \
         if ((forced < 0 && cost < best) || forced == idx) {                               \
           best = cost;                                                                    \
           pick = t;                                                                       \
@@ -246,7 +249,7 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
     d.PC = ((C + 3) / 4) * 4;
     d.store_smem = 1;  // nothing to store
   }
-  choose_xshape(d, budget);
+  choose_xshape(d, budget, 4);
   // a size needs the pipelined kernels or the log-domain ones
   if (!d.KBT && !d.xG) return SEMICRF_ERR_UNSUPPORTED;
   return SEMICRF_OK;
@@ -791,6 +794,14 @@ int viterbi_impl(const float* em, const int32_t* lengths, const float* trans, co
   WsPtrs p;
   int rc = prepare(B, T, C, K, flags, ws, ws_bytes, d, p);
   if (rc) return rc;
+  // The decoder's ring prefers clusters of 8 where all 8 B CTAs fit the GPU
+  // at once: its helpers are light, so splitting the labels finer shortens
+  // the step (the workspace layout does not depend on the cluster shape).
+  if (d.xG && d.xN > 1 && 8LL * B <= sm_count()) {
+    Dims e = d;
+    choose_xshape(e, (size_t)max_smem_optin() - 256, 8);
+    if (e.xG) d = e;
+  }
   const bool proj = p_start || p_end;
   if ((rc = reset_status(p, proj, st))) return rc;
   if (B == 0) return SEMICRF_OK;

@@ -847,11 +847,11 @@ cudaError_t launch_viterbi_words(const Dims& d, const WsPtrs& ws, const int32_t*
   return cudaGetLastError();
 }
 
-// Shared memory of the walk: about 96 KB (longer windows), at least the K
-// marks and one row of words per buffer.
+// Shared memory of the walk: up to 200 KB (long windows: fewer of them), at
+// least the K marks and one row of words per buffer.
 size_t viterbi_walk_smem_bytes(const Dims& d, size_t budget) {
   const size_t CP = (d.C + 3) & ~3;
-  const size_t want = std::min<size_t>(budget, 96u * 1024u);
+  const size_t want = std::min<size_t>(budget, 200u * 1024u);
   const size_t need = ((size_t)d.K + 1 + 2 * CP) * sizeof(int);
   return std::max(want, need);
 }

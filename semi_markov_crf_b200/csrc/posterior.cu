@@ -177,24 +177,54 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int nw = blockDim.x >> 5;
   for (int c = tid >> 5; c < C; c += nw) {
-    // lanes over the start offset ia, inner loop over the end offset jb
-    float zmax = NEG_INF, sum = 0.f;
+    // a warp per label: lanes over pairs of start offsets (ia, K-1-ia), so
+    // every lane sums about K + 1 terms, the inner loop over the end offset
     const float* const lac = la + c * KP;
     const float* const lbc = lb + c * KP;
     const float* const ddc = dd + c * KP;
-    for (int ia = lane; ia < K; ia += 32) {
-      const float a = lac[ia];
-      if (a == NEG_INF) continue;
-      for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lbc[jb]) + ddc[ia + jb]);
+    auto pair_sum = [&](float Mz) {
+      float sum = 0.f;
+      for (int p = lane; p < (K + 1) / 2; p += 32) {
+        for (int h = 0; h < 2; ++h) {
+          const int ia = h ? K - 1 - p : p;
+          if (h && ia == p) break;
+          const float a = lac[ia] - Mz;
+          if (a == NEG_INF) continue;
+          for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lbc[jb]) + ddc[ia + jb]);
+        }
+      }
+      return group_sum(sum, 32);
+    };
+    // the shift: a bound on every term, max la + max lb + max dd; only when
+    // the sum then falls below 2^-60 (the bound far above the largest term)
+    // is the exact largest term found and the sum taken again
+    float ma = NEG_INF, mb = NEG_INF, md = NEG_INF;
+    for (int q = lane; q < K; q += 32) {
+      ma = fmaxf(ma, lac[q]);
+      mb = fmaxf(mb, lbc[q]);
+      md = fmaxf(md, ddc[q]);
     }
-    zmax = group_max(zmax, 32);
-    const float Mz = (zmax == NEG_INF) ? 0.f : ceilf(zmax);
-    for (int ia = lane; ia < K; ia += 32) {
-      const float a = lac[ia] - Mz;
-      if (a == NEG_INF) continue;
-      for (int jb = 0; jb < K - ia; ++jb) sum += ex2((a + lbc[jb]) + ddc[ia + jb]);
+    ma = group_max(ma, 32);
+    mb = group_max(mb, 32);
+    md = group_max(md, 32);
+    const bool any = ma != NEG_INF && mb != NEG_INF && md != NEG_INF;
+    float Mz = any ? ceilf((ma + mb) + md) : 0.f;
+    float sum = any ? pair_sum(Mz) : 0.f;
+    if (any && !(sum >= 0x1p-60f)) {
+      float zmax = NEG_INF;
+      for (int p = lane; p < (K + 1) / 2; p += 32) {
+        for (int h = 0; h < 2; ++h) {
+          const int ia = h ? K - 1 - p : p;
+          if (h && ia == p) break;
+          const float a = lac[ia];
+          if (a == NEG_INF) continue;
+          for (int jb = 0; jb < K - ia; ++jb) zmax = fmaxf(zmax, (a + lbc[jb]) + ddc[ia + jb]);
+        }
+      }
+      zmax = group_max(zmax, 32);
+      Mz = (zmax == NEG_INF) ? 0.f : ceilf(zmax);
+      sum = pair_sum(Mz);
     }
-    sum = group_sum(sum, 32);
     if (lane == 0) {
       lab_M[c] = Mz;
       lab_f[c] = (sum > 0.f) ? lg2(sum) : NEG_INF;
@@ -233,11 +263,11 @@ namespace {
 //   P([s, s+k), c) = 2^(Y[s+k, c] - X[s, c] + dur2'[k-1, c])        (dur2' = M + dur2)
 //   Y[t, c] = I[t, c] + S_frac[t, c] + log2 ab[t, c]                 (end side)
 //   X[s, c] = I[s, c] + S_frac[s, c] - pd[s, c] - log2 af[s, c] - log2 f_s   (start side)
-// with I[t, c] = (Pb_t - Pb_lo) + S_int[t, c] the exact integer part of the
+// with I[t, c] = (Pb_t - Pb_t0) + S_int[t, c] the exact integer part of the
 // prefix sum.  Both sides are stored split into an integer (held exactly in a
-// float: the integers are taken relative to the tile's first row, so they
-// stay far below 2^24) and a fraction in [-1/2, 1/2], so the large values
-// only ever meet as an exact integer difference.  A side whose kept value is
+// float: the integers are taken relative to the segment's first row t0, so
+// they stay far below 2^24) and a fraction in [-1/2, 1/2], so the large
+// values only ever meet as an exact integer difference.  A side whose kept value is
 // zero is stored as an infinite integer part (its terms are 0).
 struct PTile {
   float* pa;    // [RT][Cp]  forward p of the tile rows times f_s (transition items)
@@ -247,14 +277,14 @@ struct PTile {
   float* xf;    // [RT][C]   start side X: fraction
   float* yi;    // [R][C]    end side Y of the staged rows: integer part
   float* yf;    // [R][C]    end side Y: fraction
-  int* li;      // [RT]      log2 f_s: integer part
-  float* lf;    // [RT]      log2 f_s: remainder
-  float* fs;    // [RT]      f_s
+  int* li;      // [2][RT]   log2 f_s: integer part (this tile's and the next's)
+  float* lf;    // [2][RT]   log2 f_s: remainder
+  float* fs;    // [2][RT]   f_s
 };
 __host__ __device__ __forceinline__ int pad4(int C) { return (C + 3) & ~3; }
 __host__ __device__ __forceinline__ size_t ptile_bytes(int RT, int KH, int C) {
   const size_t R = (size_t)RT + KH;
-  return 8ull * RT * pad4(C) + 16ull * RT * C + 8ull * R * C + 12ull * RT;
+  return 8ull * RT * pad4(C) + 16ull * RT * C + 8ull * R * C + 24ull * RT;
 }
 __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH, int C) {
   PTile t;
@@ -267,8 +297,8 @@ __device__ __forceinline__ PTile ptile_carve(unsigned char* raw, int RT, int KH,
   t.yi = t.xf + (size_t)RT * C;
   t.yf = t.yi + R * C;
   t.li = reinterpret_cast<int*>(t.yf + R * C);
-  t.lf = reinterpret_cast<float*>(t.li + RT);
-  t.fs = t.lf + RT;
+  t.lf = reinterpret_cast<float*>(t.li + 2 * RT);
+  t.fs = t.lf + 2 * RT;
   return t;
 }
 
@@ -331,7 +361,7 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
   extern __shared__ __align__(16) unsigned char psh[];
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nthr = blockDim.x;
   const int C = d.C, K = d.K, RT = d.pRT, KH = d.pKH, Cp = pad4(C);
-  [[maybe_unused]] const int R = RT + KH;  // staged rows (bounds-check build)
+  const int R = RT + KH;  // staged segment-end rows
   const int L = lengths[b];
   if (L <= 0 || L > d.T) return;
   if (!posterior_from_kept(ws, d, b)) return;  // segment_kernel runs it
@@ -362,6 +392,36 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
 #pragma unroll
     for (int u = 0; u < 16; ++u) acct[m][u] = 0.f;
   double lacc = 0.0, lvs = 0.0;  // thread c < C: running suffix sum, sum of v
+  // integer bases of the segment: every staged integer is relative to row t0
+  const double kbase = kfb[t0];
+  const int32_t* sib = si + (size_t)t0 * C;
+  // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s)) of a tile's rows, also split for
+  // the start sides, into buffer slot fb (the next tile's are taken while
+  // this one computes)
+  auto stage_f = [&](int lo, int n, int fb) {
+    for (int r = tid; r < n; r += nthr) {
+      const int s = lo + r;
+      const double l = ((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1));
+      const double nn = fabs(l) < 1e9 ? rint(l) : 0.0;
+      tl.li[fb * RT + r] = (int)nn;
+      tl.lf[fb * RT + r] = (float)(l - nn);
+      tl.fs[fb * RT + r] = ex2((float)l);
+    }
+  };
+  // the end side Y of row `row`, label c, into staged slot p
+  auto stage_y = [&](size_t row, int c, int p) {
+    const int ib = (int)(kfb[row] - kbase) + (si[row * C + c] - sib[c]);
+    split_store(sfp[row * C + c] + lg2_sub(pbr[row * 2 * C + C + c]), ib, tl.yi + (size_t)p * C + c,
+                tl.yf + (size_t)p * C + c);
+  };
+  // All segment ends staged at once (KH = K): the staged rows roll.  Row t
+  // sits in slot (t - t0) mod R; a tile needs rows [s_lo, s_lo + nr + K), so
+  // the next tile down (s_lo - RT) stages only its RT new rows, whose slots
+  // held rows at least RT + K above them, past what it reads.
+  const bool roll = KH == K;
+  int fb = 0;
+  stage_f(max(t0, t1 - RT), t1 - max(t0, t1 - RT), 0);
+  __syncthreads();
 
   for (int s_hi = t1; s_hi > t0; s_hi -= RT) {
     const int s_lo = max(t0, s_hi - RT);
@@ -371,18 +431,15 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
     const bool first = (s_hi == t1);
     // bounds-check build: the tile fits its rows
     if (!SEMICRF_INB(ws.status, nr >= 1 && nr <= RT && nh <= RT + K, SITE_POST_TILE)) break;
-    const double kb0 = kfb[s_lo];
-    // ------------------------------------------------------------ f_s of the tile rows
-    // f_s = 2^(Pf_s + Pb_s + M - log2 Z(s)), also split for the start sides
-    for (int r = tid; r < nr; r += nthr) {
-      const int s = s_lo + r;
-      const double l = ((kff[s] + kfb[s]) + (double)M) - local_logz(d, nc, L, min(s, L - 1));
-      const double n = fabs(l) < 1e9 ? rint(l) : 0.0;
-      tl.li[r] = (int)n;
-      tl.lf[r] = (float)(l - n);
-      tl.fs[r] = ex2((float)l);
-    }
-    __syncthreads();
+    const float* const fsb = tl.fs + fb * RT;
+    const int* const lib = tl.li + fb * RT;
+    const float* const lfb = tl.lf + fb * RT;
+    // staged slot of segment-end row s_lo + h (h < R)
+    const int off = roll ? (s_lo - t0) % R : 0;
+    auto slot = [&](int h) {
+      const int q = off + h;
+      return q >= R ? q - R : q;
+    };
     // ------------------------------------------------------------ stage the tile rows
     // start / end marginals and St - E; transition operands; start sides X
     for (int i = tid; i < nr * Cp; i += nthr) {
@@ -393,7 +450,7 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
         continue;
       }
       const size_t row = (size_t)(s_lo + r);
-      const float f = tl.fs[r];
+      const float f = fsb[r];
       const float tp = pfr[row * 2 * C + c], ta = pfr[row * 2 * C + C + c];
       const float bp = pbr[row * 2 * C + c], ba = pbr[row * 2 * C + C + c];
       const float St = ta * bp * f, E = ba * tp * f;
@@ -405,8 +462,8 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
       tl.pa[i] = tp * f;
       tl.pbt[i] = bp;
       const float pdv = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
-      const int ib = (int)(kfb[row] - kb0) + (si[row * C + c] - si[(size_t)s_lo * C + c]);
-      split_store((sfp[row * C + c] - pdv) - (lg2_sub(ta) + tl.lf[r]), ib - tl.li[r], tl.xi + o,
+      const int ib = (int)(kfb[row] - kbase) + (si[row * C + c] - sib[c]);
+      split_store((sfp[row * C + c] - pdv) - (lg2_sub(ta) + lfb[r]), ib - lib[r], tl.xi + o,
                   tl.xf + o);
     }
     // ------------------------------------------------------------ segment ends, by chunk
@@ -416,11 +473,12 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
       const int base = kc - 1;
       const int nst = max(0, min(base + nr + KH, nh) - base);
       if (kc > 1) __syncthreads();  // the previous chunk's reads are done
-      for (int i = tid; i < nst * C; i += nthr) {
-        const int r = i / C, c = i - r * C;
-        const size_t row = (size_t)(s_lo + base + r);
-        const int ib = (int)(kfb[row] - kb0) + (si[row * C + c] - si[(size_t)s_lo * C + c]);
-        split_store(sfp[row * C + c] + lg2_sub(pbr[row * 2 * C + C + c]), ib, tl.yi + i, tl.yf + i);
+      // rolling: the first tile stages all its rows, later ones the RT below
+      // the previous tile; chunks: all of the chunk's rows, slot = offset
+      const int nnew = roll ? (first ? nst : min(nst, nr)) : nst;
+      for (int i = tid; i < nnew * C; i += nthr) {
+        const int h = i / C, c = i - h * C;
+        stage_y((size_t)(s_lo + base + h), c, slot(h));
       }
       __syncthreads();
       // -------------------------------------------------------- segment marginals
@@ -433,7 +491,7 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
           const int k = idx / C + 1, c = idx - (k - 1) * C;
           if (r + k > Lr) continue;
           if (!SEMICRF_INB(ws.status, r + k - base < nst, SITE_POST_ITEM)) continue;
-          const int o = r * C + c, ok = (r + k - base) * C + c;
+          const int o = r * C + c, ok = slot(r + k - base) * C + c;
           const float z = (tl.yi[ok] - tl.xi[o]) +
                           ((tl.yf[ok] - tl.xf[o]) + (M + __ldg(dur + idx) * l2e()));
           seg_marg[((size_t)b * d.T + s_lo + r) * nd + idx] = ex2(z);
@@ -459,13 +517,13 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
           return;
         const float* yi = tl.yi + c;
         const float* yf = tl.yf + c;
-        float w0i = yi[h0 * C], w0f = yf[h0 * C];
-        float w1i = yi[(h0 + 1) * C], w1f = yf[(h0 + 1) * C];
-        float w2i = yi[(h0 + 2) * C], w2f = yf[(h0 + 2) * C];
+        float w0i = yi[slot(h0) * C], w0f = yf[slot(h0) * C];
+        float w1i = yi[slot(h0 + 1) * C], w1f = yf[slot(h0 + 1) * C];
+        float w2i = yi[slot(h0 + 2) * C], w2f = yf[slot(h0 + 2) * C];
         int r = 0;
 #pragma unroll 4
         for (; r < r_all; ++r) {
-          const int h3 = (h0 + r + 3) * C;
+          const int h3 = slot(h0 + r + 3) * C;
           const float w3i = yi[h3], w3f = yf[h3];
           const float oi = tl.xi[r * C + c], of = tl.xf[r * C + c];
           a[0] += ex2((w0i - oi) + ((w0f - of) + dk[0]));
@@ -482,7 +540,7 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             if (r + k0 + u > Lr) break;
-            const int h = (h0 + r + u) * C;
+            const int h = slot(h0 + r + u) * C;
             a[u] += ex2((yi[h] - oi) + ((yf[h] - of) + dk[u]));
           }
         }
@@ -556,6 +614,12 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
         lacc += tl.dif[r * C + tid];
       }
     }
+    // the next tile's f_s into the other slot (nobody reads it now)
+    if (s_hi - RT > t0) {
+      const int nlo = max(t0, s_hi - 2 * RT);
+      stage_f(nlo, s_lo - nlo, fb ^ 1);
+    }
+    fb ^= 1;
     __syncthreads();  // the next tile overwrites the staged rows
   }
   // register items: the segment's partials

@@ -408,12 +408,6 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
       tl.fs[fb * RT + r] = ex2((float)l);
     }
   };
-  // the end side Y of row `row`, label c, into staged slot p
-  auto stage_y = [&](size_t row, int c, int p) {
-    const int ib = (int)(kfb[row] - kbase) + (si[row * C + c] - sib[c]);
-    split_store(sfp[row * C + c] + lg2_sub(pbr[row * 2 * C + C + c]), ib, tl.yi + (size_t)p * C + c,
-                tl.yf + (size_t)p * C + c);
-  };
   // All segment ends staged at once (KH = K): the staged rows roll.  Row t
   // sits in slot (t - t0) mod R; a tile needs rows [s_lo, s_lo + nr + K), so
   // the next tile down (s_lo - RT) stages only its RT new rows, whose slots
@@ -441,30 +435,55 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
       return q >= R ? q - R : q;
     };
     // ------------------------------------------------------------ stage the tile rows
-    // start / end marginals and St - E; transition operands; start sides X
-    for (int i = tid; i < nr * Cp; i += nthr) {
-      const int r = i / Cp, c = i - r * Cp;
-      if (c >= C) {
-        tl.pa[i] = 0.f;
-        tl.pbt[i] = 0.f;
-        continue;
+    // start / end marginals and St - E; transition operands; start sides X.
+    // SU items per thread at a time, every load of a batch issued before its
+    // first store (the marginal stores could alias the kept rows as far as
+    // the compiler can tell, which would hold each load behind them)
+    constexpr int SU = NQ > 1 ? 4 : 2;  // (the two-CTA variant has half the registers)
+    for (int i0 = tid; i0 < nr * Cp; i0 += SU * nthr) {
+      float tp[SU], ta[SU], bp[SU], ba[SU], pdv[SU], sfv[SU];
+      int siv[SU];
+      double kfv[SU];
+#pragma unroll
+      for (int u = 0; u < SU; ++u) {
+        const int i = i0 + u * nthr;
+        const int r = i / Cp, c = i - r * Cp;
+        const bool ok = i < nr * Cp && c < C;
+        const size_t row = (size_t)(s_lo + (ok ? r : 0));
+        const int cc = ok ? c : 0;
+        tp[u] = ok ? pfr[row * 2 * C + cc] : 0.f;
+        ta[u] = ok ? pfr[row * 2 * C + C + cc] : 0.f;
+        bp[u] = ok ? pbr[row * 2 * C + cc] : 0.f;
+        ba[u] = ok ? pbr[row * 2 * C + C + cc] : 0.f;
+        pdv[u] = (ok && pj) ? ws.pd[((size_t)b * d.Tstride + row) * C + cc] : 0.f;
+        sfv[u] = ok ? sfp[row * C + cc] : 0.f;
+        siv[u] = ok ? si[row * C + cc] - sib[cc] : 0;
+        kfv[u] = ok ? kfb[row] : kbase;
       }
-      const size_t row = (size_t)(s_lo + r);
-      const float f = fsb[r];
-      const float tp = pfr[row * 2 * C + c], ta = pfr[row * 2 * C + C + c];
-      const float bp = pbr[row * 2 * C + c], ba = pbr[row * 2 * C + C + c];
-      const float St = ta * bp * f, E = ba * tp * f;
-      const size_t ob = ((size_t)b * (d.T + 1) + row) * C + c;
-      if (start_marg) start_marg[ob] = St;
-      if (end_marg) end_marg[ob] = E;
-      const int o = r * C + c;
-      tl.dif[o] = (double)St - (double)E;
-      tl.pa[i] = tp * f;
-      tl.pbt[i] = bp;
-      const float pdv = pj ? ws.pd[((size_t)b * d.Tstride + row) * C + c] : 0.f;
-      const int ib = (int)(kfb[row] - kbase) + (si[row * C + c] - sib[c]);
-      split_store((sfp[row * C + c] - pdv) - (lg2_sub(ta) + lfb[r]), ib - lib[r], tl.xi + o,
-                  tl.xf + o);
+#pragma unroll
+      for (int u = 0; u < SU; ++u) {
+        const int i = i0 + u * nthr;
+        if (i >= nr * Cp) break;
+        const int r = i / Cp, c = i - r * Cp;
+        if (c >= C) {
+          tl.pa[i] = 0.f;
+          tl.pbt[i] = 0.f;
+          continue;
+        }
+        const size_t row = (size_t)(s_lo + r);
+        const float f = fsb[r];
+        const float St = ta[u] * bp[u] * f, E = ba[u] * tp[u] * f;
+        const size_t ob = ((size_t)b * (d.T + 1) + row) * C + c;
+        if (start_marg) start_marg[ob] = St;
+        if (end_marg) end_marg[ob] = E;
+        const int o = r * C + c;
+        tl.dif[o] = (double)St - (double)E;
+        tl.pa[i] = tp[u] * f;
+        tl.pbt[i] = bp[u];
+        const int ib = (int)(kfv[u] - kbase) + siv[u];
+        split_store((sfv[u] - pdv[u]) - (lg2_sub(ta[u]) + lfb[r]), ib - lib[r], tl.xi + o,
+                    tl.xf + o);
+      }
     }
     // ------------------------------------------------------------ segment ends, by chunk
     // chunk kc: durations [kc, kc + KH), staged rows at offsets [kc - 1, kc - 1 + nr + KH)
@@ -476,9 +495,28 @@ __global__ void __launch_bounds__(512, NQ > 1 ? 1 : 2)
       // rolling: the first tile stages all its rows, later ones the RT below
       // the previous tile; chunks: all of the chunk's rows, slot = offset
       const int nnew = roll ? (first ? nst : min(nst, nr)) : nst;
-      for (int i = tid; i < nnew * C; i += nthr) {
-        const int h = i / C, c = i - h * C;
-        stage_y((size_t)(s_lo + base + h), c, slot(h));
+      for (int i0 = tid; i0 < nnew * C; i0 += SU * nthr) {
+        float sv[SU], bv[SU];
+        int iv[SU];
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {  // loads first (as above)
+          const int i = i0 + u * nthr;
+          const bool ok = i < nnew * C;
+          const int h = ok ? i / C : 0, c = ok ? i - h * C : 0;
+          const size_t row = (size_t)(s_lo + base + h);
+          iv[u] = (int)(kfb[row] - kbase) + (si[row * C + c] - sib[c]);
+          sv[u] = sfp[row * C + c];
+          bv[u] = pbr[row * 2 * C + C + c];
+        }
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int i = i0 + u * nthr;
+          if (i >= nnew * C) break;
+          const int h = i / C, c = i - h * C;
+          const int p = slot(h);
+          split_store(sv[u] + lg2_sub(bv[u]), iv[u], tl.yi + (size_t)p * C + c,
+                      tl.yf + (size_t)p * C + c);
+        }
       }
       __syncthreads();
       // -------------------------------------------------------- segment marginals

@@ -15,7 +15,7 @@ namespace semicrf {
 
 namespace {
 
-constexpr int FIN_ROWS_HOST = 32;  // must match FIN_ROWS in finalize.cu
+constexpr int FIN_ROWS_HOST = 64;  // must match FIN_ROWS in finalize.cu
 
 int pow2floor(int x) {
   int p = 1;
@@ -186,11 +186,11 @@ int make_dims(int B, int T, int C, int K, Dims& d) {
   if (d.delta < 1) d.delta = 1;
   d.nck = T > 0 ? (T + d.delta - 1) / d.delta : 1;
   d.Tstride = ((T + 1 + TS - 1) / TS) * TS;
-  // Cut-normaliser grid: every 128 positions, sparser for long durations (a
+  // Cut-normaliser grid: every 256 positions, sparser for long durations (a
   // grid point costs K(K+1)/2 C terms; the two rings' rounding drifts by about
   // 1e-7 per position, so linear interpolation over 2048 positions still
   // keeps the marginals' error far below 1e-4)
-  d.GS = 128;
+  d.GS = 256;
   while (d.GS < 2048 && d.GS * 4 < K) d.GS *= 2;
   d.ngrid = T > 0 ? (T - 1) / d.GS + 2 : 1;  // positions 0, GS, 2GS, ... and L - 1
   d.npch = std::max(1, (T + PATH_ROWS - 1) / PATH_ROWS);

@@ -21,7 +21,7 @@
 
 namespace semicrf {
 
-constexpr int FIN_ROWS = 32;
+constexpr int FIN_ROWS = 64;
 
 __global__ void __launch_bounds__(256)
     finalize_positions_kernel(Dims d, WsPtrs ws, const int32_t* __restrict__ lengths,
@@ -59,17 +59,33 @@ __global__ void __launch_bounds__(256)
     mean[c] = center ? msum / (double)L : 0.0;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < (u1 - u0) * C; idx += blockDim.x) {
-    const int u = u0 + idx / C, c = idx % C;
-    const size_t o = ((size_t)b * T + u) * C + c;
-    if (u < L) {
-      const int j = u / delta;
-      const double mu = pinc[(j - j_lo) * C + c] - (double)grad_em[o];
-      grad_em[o] = (float)(gb * (mu - mean[c]));
-      if (pos_marg) pos_marg[o] = (float)mu;
-    } else {
-      grad_em[o] = 0.f;
-      if (pos_marg) pos_marg[o] = 0.f;
+  // FU entries per thread at a time, their loads issued before the stores
+  // (grad_em is read and written here: otherwise each load would wait for
+  // the store before it)
+  constexpr int FU = 4;
+  const int n = (u1 - u0) * C;
+  const size_t ob = ((size_t)b * T + u0) * C;
+  for (int i0 = threadIdx.x; i0 < n; i0 += FU * blockDim.x) {
+    float v[FU];
+#pragma unroll
+    for (int q = 0; q < FU; ++q) {
+      const int idx = i0 + q * blockDim.x;
+      v[q] = (idx < n && u0 + idx / C < L) ? grad_em[ob + idx] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < FU; ++q) {
+      const int idx = i0 + q * blockDim.x;
+      if (idx >= n) break;
+      const int u = u0 + idx / C, c = idx % C;
+      if (u < L) {
+        const int j = u / delta;
+        const double mu = pinc[(j - j_lo) * C + c] - (double)v[q];
+        grad_em[ob + idx] = (float)(gb * (mu - mean[c]));
+        if (pos_marg) pos_marg[ob + idx] = (float)mu;
+      } else {
+        grad_em[ob + idx] = 0.f;
+        if (pos_marg) pos_marg[ob + idx] = 0.f;
+      }
     }
   }
   // boundary rows t in [u0, u1) (and t = T for the last block) past the length

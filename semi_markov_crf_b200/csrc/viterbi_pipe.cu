@@ -604,42 +604,52 @@ __global__ void __launch_bounds__(256)
     w2[q] = (q < C && pg < png) ? __ldg(trans + (size_t)q * C + pc) * l2e() : NEG_INF;
   __syncthreads();
   if (pg >= png) return;
-  // two rows at a time (eight independent chains); per element an add, a
+  // VR rows at a time (4 VR independent chains); per element an add, a
   // compare-select of the index and a max of the value, so a chain's value
   // update does not wait on its compare
-  for (int s = s0 + pg; s <= s1; s += 2 * png) {
-    const int sB = min(s + png, s1);  // the second row (the first again past s1)
-    const float4* va = reinterpret_cast<const float4*>(vsh + (size_t)(s - s0) * VS);
-    const float4* vb = reinterpret_cast<const float4*>(vsh + (size_t)(sB - s0) * VS);
-    float bA[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF}, bB[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
-    int qA[4] = {0, 1, 2, 3}, qB[4] = {0, 1, 2, 3};
+  constexpr int VR = 4;
+  for (int s = s0 + pg; s <= s1; s += VR * png) {
+    const float4* vr[VR];
+#pragma unroll
+    for (int w = 0; w < VR; ++w)  // rows past s1 repeat s1 (not stored)
+      vr[w] = reinterpret_cast<const float4*>(vsh + (size_t)(min(s + w * png, s1) - s0) * VS);
+    float bv[VR][4];
+    int qv[VR][4];
+#pragma unroll
+    for (int w = 0; w < VR; ++w)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        bv[w][u] = NEG_INF;
+        qv[w][u] = u;
+      }
 #pragma unroll
     for (int q4 = 0; q4 < NW / 4; ++q4) {
       if (4 * q4 < VS) {
-        const float4 x = va[q4], y = vb[q4];
-        const float ex[4] = {x.x, x.y, x.z, x.w}, ey[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float e = ex[u] + w2[4 * q4 + u], f = ey[u] + w2[4 * q4 + u];
-          qA[u] = (e > bA[u]) ? 4 * q4 + u : qA[u];
-          bA[u] = fmaxf(bA[u], e);
-          qB[u] = (f > bB[u]) ? 4 * q4 + u : qB[u];
-          bB[u] = fmaxf(bB[u], f);
+        for (int w = 0; w < VR; ++w) {
+          const float4 x = vr[w][q4];
+          const float ex[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float e = ex[u] + w2[4 * q4 + u];
+            qv[w][u] = (e > bv[w][u]) ? 4 * q4 + u : qv[w][u];
+            bv[w][u] = fmaxf(bv[w][u], e);
+          }
         }
       }
     }
     // merge the chains by value, then index: the smallest c' among equal
     // maxima (a chain that never improved on -inf keeps its first index, so
     // an all -inf row yields label 0)
-    auto merge = [](float (&bv)[4], int (&qv)[4]) {
-      if (bv[1] > bv[0] || (bv[1] == bv[0] && qv[1] < qv[0])) { bv[0] = bv[1]; qv[0] = qv[1]; }
-      if (bv[3] > bv[2] || (bv[3] == bv[2] && qv[3] < qv[2])) { bv[2] = bv[3]; qv[2] = qv[3]; }
-      if (bv[2] > bv[0] || (bv[2] == bv[0] && qv[2] < qv[0])) { bv[0] = bv[2]; qv[0] = qv[2]; }
-      return qv[0];
-    };
-    arg[(size_t)s * VS + pc] = merge(bA, qA);
-    const int qb = merge(bB, qB);
-    if (s + png <= s1) arg[(size_t)sB * VS + pc] = qb;
+#pragma unroll
+    for (int w = 0; w < VR; ++w) {
+      float* b = bv[w];
+      int* q = qv[w];
+      if (b[1] > b[0] || (b[1] == b[0] && q[1] < q[0])) { b[0] = b[1]; q[0] = q[1]; }
+      if (b[3] > b[2] || (b[3] == b[2] && q[3] < q[2])) { b[2] = b[3]; q[2] = q[3]; }
+      if (b[2] > b[0] || (b[2] == b[0] && q[2] < q[0])) { b[0] = b[2]; q[0] = q[2]; }
+      if (s + w * png <= s1) arg[(size_t)(s + w * png) * VS + pc] = q[0];
+    }
   }
 }
 

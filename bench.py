@@ -141,14 +141,9 @@ def hbm_bytes_per_position(kernel: str, C: int):
 
 def csrc_digest() -> str:
     """sha256 over the kernel sources, to tie a stored ncu traffic figure to
-    the build it was measured on."""
-    import hashlib
-    h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
-    return h.hexdigest()
+    the build it was measured on (the digest the library compiles in)."""
+    from semi_markov_crf_b200.build import source_digest
+    return source_digest()
 
 
 def stored_traffic(kernel: str, workload: str):

@@ -342,6 +342,14 @@ SEMICRF_API int semicrf_ring_domains(const void *ws, size_t ws_bytes, int B, int
 SEMICRF_API const char *semicrf_strerror(int code);
 
 /*
+ * The sha256 (64 hex digits) of the kernel sources this library was built
+ * from (csrc/*.cu and *.cuh: name, NUL, contents, in name order), or
+ * "unknown" when the build did not define it.  Static string, never NULL.
+ * Lets a caller check that the library it loaded matches the sources.
+ */
+SEMICRF_API const char *semicrf_source_digest(void);
+
+/*
  * Diagnostic: runs the library's bounded shared-memory-barrier wait on a
  * barrier nothing will ever complete, with a limit of `spins` polls, and
  * records the outcome in the workspace status word (SEMICRF_ERR_DEVICE_TIMEOUT

@@ -10,7 +10,9 @@ The binding loads it when SEMICRF_LIBRARY=check.
 Compiles every ``csrc/*.cu`` for ``-gencode arch=compute_100a,code=sm_100a``
 (with -lineinfo) and links a shared library with the CUDA runtime linked
 statically, so the library needs only the driver at run time.  Rebuilds when
-any source or header is newer than the library.
+any source or header is newer than the library.  The sha256 of the kernel
+sources (``source_digest()``) is compiled in: ``semicrf_source_digest()``
+returns it, so a caller can tell a library built from other sources.
 """
 
 from __future__ import annotations
@@ -49,6 +51,18 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def source_digest() -> str:
+    """sha256 over the kernel sources (csrc/*.cu, *.cuh: name, NUL, bytes, in
+    name order)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
 def _stale(lib: str = LIB) -> bool:
     if not os.path.exists(lib):
         return True
@@ -65,6 +79,7 @@ def build(force: bool = False, verbose: bool = False, bounds_check: bool = False
     bdir = BUILD_DIR + ("_check" if bounds_check else "")
     os.makedirs(bdir, exist_ok=True)
     extra = ["-DSEMICRF_BOUNDS_CHECK"] if bounds_check else []
+    extra.append(f'-DSEMICRF_SOURCE_DIGEST="{source_digest()}"')
     from concurrent.futures import ThreadPoolExecutor
 
     def compile_one(src):

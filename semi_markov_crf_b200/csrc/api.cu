@@ -945,6 +945,11 @@ extern "C" int semicrf_ring_domains(const void* ws, size_t ws_bytes, int B, int 
   return SEMICRF_OK;
 }
 
+#ifndef SEMICRF_SOURCE_DIGEST
+#define SEMICRF_SOURCE_DIGEST "unknown"
+#endif
+extern "C" const char* semicrf_source_digest(void) { return SEMICRF_SOURCE_DIGEST; }
+
 extern "C" const char* semicrf_strerror(int code) {
   switch (code) {
     case SEMICRF_OK: return "ok";

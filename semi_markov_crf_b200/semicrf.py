@@ -72,6 +72,8 @@ lib.semicrf_path_score_proj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, 
 lib.semicrf_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i)]
 lib.semicrf_strerror.argtypes = [_i]
 lib.semicrf_strerror.restype = ctypes.c_char_p
+lib.semicrf_source_digest.argtypes = []
+lib.semicrf_source_digest.restype = ctypes.c_char_p
 lib.semicrf_selftest_bounded_wait.argtypes = [_vp, _sz, _i, _vp]
 lib.semicrf_selftest_bounds.argtypes = [_vp, _sz, _vp]
 lib.semicrf_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp, _vp]
@@ -94,6 +96,11 @@ class SemiCRFError(RuntimeError):
 
 def strerror(code: int) -> str:
     return lib.semicrf_strerror(int(code)).decode()
+
+
+def source_digest() -> str:
+    """sha256 of the kernel sources the loaded library was built from."""
+    return lib.semicrf_source_digest().decode()
 
 
 def _check(rc: int, where: str):

@@ -35,7 +35,8 @@ def cases():
 
 def main():
     assert semicrf.library_path.endswith("libsemicrf_b200_check.so"), semicrf.library_path
-    out = {"library": os.path.basename(semicrf.library_path), "cases": {}}
+    out = {"library": os.path.basename(semicrf.library_path), "digest": semicrf.source_digest(),
+           "cases": {}}
     ws0 = semicrf.Workspace(1, 8, 2, 2, 0, "cuda")
     out["selftest_status"] = semicrf.selftest_bounds(ws0)
     for name, c in cases().items():

@@ -36,6 +36,14 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_loaded_library_is_built_from_the_current_sources():
+    from semi_markov_crf_b200 import semicrf
+    from semi_markov_crf_b200.build import source_digest
+    got = semicrf.source_digest()
+    assert len(got) == 64 and got == source_digest(), (
+        "the loaded library was built from other kernel sources: rebuild it")
+
+
 def _ws_bytes(lib, B, T, C, K, flags=0):
     n = ctypes.c_size_t(0)
     rc = lib.semicrf_workspace_bytes(B, T, C, K, ctypes.c_uint(flags), ctypes.byref(n))

@@ -34,6 +34,9 @@ def test_bounds_checked_build_runs_clean():
     out = json.loads(res.stdout.strip().splitlines()[-1])
     print(json.dumps(out))
     assert out["library"] == "libsemicrf_b200_check.so"
+    # the debug build is of the current sources (a stale one would test old code)
+    from semi_markov_crf_b200.build import source_digest
+    assert out["digest"] == source_digest(), "libsemicrf_b200_check.so is stale: rebuild it"
     st = out["selftest_status"]
     assert st & 0xff == 7 and st >> 8 == 13, st   # SEMICRF_ERR_BOUNDS at the self-test's site
     for name, rec in out["cases"].items():

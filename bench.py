@@ -574,7 +574,7 @@ def run_ours(args):
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     name = args.workload
-    base = synth.CONFIGS[name]
+    base = synth.WORKLOADS[name]
     wl = Workload(name, shard_seed(base.seed, rank), dev)
     head, graph = measure(wl, args.steps, args.warmup, flush, world, local, not args.no_graph,
                           peaks, sm_count)
@@ -650,7 +650,7 @@ def run_ours(args):
     extras = {}
     if world == 1:
         for ex in [x for x in args.extras.split(",") if x and x != "none" and x != name]:
-            wx = Workload(ex, synth.CONFIGS[ex].seed, dev)
+            wx = Workload(ex, synth.WORKLOADS[ex].seed, dev)
             rx, gx = measure(wx, min(args.steps, args.extra_steps), min(args.warmup, 3), flush, 1,
                              local, not args.no_graph, peaks, sm_count)
             del gx

@@ -37,7 +37,7 @@ import math
 
 import numpy as np
 
-__all__ = ["Workload", "CONFIGS", "make", "make_custom", "checkpoint_interval"]
+__all__ = ["Workload", "WORKLOADS", "make", "make_custom", "checkpoint_interval"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,7 +56,7 @@ class Workload:
     mode: str = "segments"  # "segments" (onehot + noise) or "noise" (pure N(0,1))
 
 
-CONFIGS = {
+WORKLOADS = {
     "tiny": Workload("tiny", 1, 64, 8, 4, 0, 64, None, 1.0, 0.0, 0.1, mode="noise"),
     "speech": Workload("speech", 32, 800, 30, 39, 1, 300, None, 8.0, 1.5, 0.1),
     "genomic": Workload("genomic", 4, 100_000, 200, 6, 2, 100_000,
@@ -128,7 +128,7 @@ def make(name: str, pad_value=None, B: int | None = None, T: int | None = None,
     padding) and ``gold_start`` [B,T] uint8 (1 where a drawn segment starts;
     two adjacent drawn segments may share a label).
     """
-    w = CONFIGS[name]
+    w = WORKLOADS[name]
     B_ = w.B if B is None else int(B)
     T_ = w.T if T is None else int(T)
     if T is not None and w.len_lo < w.T:

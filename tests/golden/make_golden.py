@@ -131,7 +131,7 @@ def make(name: str):
     # wide label sets: the state-change rows of the first and last sequence
     targeted = {0, B - 1} if C > 64 else set(range(B))
     n_random = 100 if C > 64 else 300
-    seed = 43 if name == "long_k" else synth.CONFIGS[name].seed
+    seed = 43 if name == "long_k" else synth.WORKLOADS[name].seed
     if name == "long_k":  # every position
         rb, ru = np.nonzero(np.arange(T)[None, :] < w["lengths"][:, None])
         bb, bu = np.nonzero(np.arange(T + 1)[None, :] <= w["lengths"][:, None])

@@ -29,7 +29,7 @@ def _worker(rank, world, port, out):
     from semi_markov_crf_b200 import synth
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        seed = bench.shard_seed(synth.CONFIGS["speech"].seed, rank)
+        seed = bench.shard_seed(synth.WORKLOADS["speech"].seed, rank)
         w = synth.make("speech", B=2, T=50, seed=seed)
         t = bench.reduce_max(float(rank + 1) * 1.5)
         g1 = torch.full((3, 3), float(rank + 1))
